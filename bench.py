@@ -1,0 +1,486 @@
+#!/usr/bin/env python
+"""Benchmark: sparse-attention prefill at 64K tokens (+ decode, NSA, fixed graph).
+
+One step = one pass of the DSA prefill hot path over a 65536-token sequence:
+indexer scores -> exact causal top-2048 -> gathered sparse attention (16 query
+heads sharing one KV head, d=128).  `value` is the attention's algorithmic
+FLOPs (4 * d * Hq * sum_t |S_t| = 1.0823e12 per sequence) divided by the time
+of the whole step, summed over ranks (each rank runs its own sequence: weak
+scaling, no data-path collective).
+
+Extra measurements on the same JSON line: the 128K-context decode step with
+IndexCache (F S S S and all-F) in tokens/s, the NSA three-branch forward at
+64K in TFLOP/s, and the fixed-graph workload (16384 tokens) in GB/s.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Under torchrun every rank runs; rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "sparse-attn prefill TFLOP/s @64K + decode tokens/s, % of roofline"
+L2_BYTES = 126 * 1024 * 1024
+FLUSH_BYTES = 2 * L2_BYTES
+
+
+# ----------------------------------------------------------- pure helpers --
+def attn_flops(T: int, topk: int, window: int, Hq: int, d: int) -> float:
+    """4 * d * Hq * sum_t |S_t| with |S_t| = min(t + 1, topk + window)."""
+    K = topk + window
+    n_full = max(0, T - K)
+    s = (min(T, K) * (min(T, K) + 1)) // 2 + n_full * K
+    return 4.0 * d * Hq * s
+
+
+def aggregate(times_ms, units_per_rank):
+    """Whole-job throughput: all ranks' units over the slowest rank's time."""
+    t = max(times_ms)
+    return sum(units_per_rank) / (t / 1e3), t
+
+
+def parse_clocks(csv_text: str):
+    """Summarise `nvidia-smi --query-gpu=... -lms` samples taken while timing."""
+    sm, mx, reasons = [], 0.0, set()
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    for line in csv_text.splitlines():
+        parts = [p.strip() for p in line.split(",")]
+        if len(parts) < 9 or not parts[1].split()[0].replace(".", "").isdigit():
+            continue
+        try:
+            clk = float(parts[1].split()[0])
+            mx = max(mx, float(parts[2].split()[0]))
+        except ValueError:
+            continue
+        sm.append(clk)
+        for n, v in zip(names, parts[5:9]):
+            if v.lower() == "active":
+                reasons.add(n)
+    if not sm:
+        return None
+    loaded = [c for c in sm if c >= 0.5 * max(sm)] or sm
+    return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": sorted(reasons),
+            "samples": len(sm)}
+
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.text = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.text, _ = self.proc.communicate(timeout=10)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.text, _ = self.proc.communicate()
+        return False
+
+    def summary(self):
+        return parse_clocks(getattr(self, "text", "") or "")
+
+
+# ---------------------------------------------------------------- timing --
+def timed_steps(step, steps, warmup, flush, dev, torch):
+    """W untimed warm-ups, then K steps each bracketed by CUDA events on the
+    current stream; L2 is flushed between steps outside the events."""
+    for _ in range(warmup):
+        flush()
+        step()
+    torch.cuda.synchronize(dev)
+    evs = []
+    for _ in range(steps):
+        flush()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        step()
+        b.record()
+        evs.append((a, b))
+    torch.cuda.synchronize(dev)
+    return [a.elapsed_time(b) for a, b in evs]
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-extra", action="store_true", help="skip decode/NSA/fixed-graph lines")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline leg")
+    ap.add_argument("--cpu-sample-rows", type=int, default=0,
+                    help="oracle rows for the CPU baseline (0 = auto, ~10-30 s)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(reference_arm(args, world)))
+        return 0
+
+    import torch
+    import torch.distributed as dist
+
+    from fixed_pattern_sparse_sa_b200 import _lib, api, inputs
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", rank=rank, world_size=world,
+                                timeout=timedelta(seconds=120), device_id=dev)
+
+    lib = _lib.load()
+    w = inputs.WORKLOADS["dsa_prefill64k"]
+    g = inputs.gen_dsa(w.B, w.T, w.Hq, w.Hkv, w.d, w.Hi, w.di, seed=rank)
+    gd = {k: v.to(dev) for k, v in g.items()}
+    flush_buf = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def flush():
+        flush_buf.fill_(1.0)
+
+    K = w.topk + w.window
+    idx = torch.empty((w.B, w.T, K), dtype=torch.int32, device=dev)
+    cnt = torch.empty((w.B, w.T), dtype=torch.int32, device=dev)
+    out = torch.empty((w.B, w.T, w.Hq, w.d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.B, w.T, w.Hq), dtype=torch.float32, device=dev)
+    ws_bytes = lib.sa_indexer_topk_workspace_size(w.B, w.T, w.T, w.Hi, w.di, w.topk, w.window)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+
+    # per-kernel-group timing inside the step (events on the launching stream)
+    ev_idx = []
+    ev_att = []
+
+    def step(record=False):
+        e0 = torch.cuda.Event(enable_timing=True) if record else None
+        e1 = torch.cuda.Event(enable_timing=True) if record else None
+        e2 = torch.cuda.Event(enable_timing=True) if record else None
+        if record:
+            e0.record()
+        api.indexer_topk(gd["q_idx"], gd["k_idx"], gd["w"], w.topk, w.window, out_idx=idx,
+                         out_count=cnt, workspace=ws)
+        if record:
+            e1.record()
+        api.sparse_attn_fwd(gd["q"], gd["k"], gd["v"], idx, out=out, lse=lse)
+        if record:
+            e2.record()
+            ev_idx.append((e0, e1))
+            ev_att.append((e1, e2))
+
+    flops = attn_flops(w.T, w.topk, w.window, w.Hq, w.d)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    n0 = lib.sa_launch_counter()
+    with ClockSampler(local) as clk:
+        times = timed_steps(lambda: step(True), args.steps, args.warmup, flush, dev, torch)
+    launches = (lib.sa_launch_counter() - n0) // (args.steps + args.warmup) * args.steps
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    total_ms = sum(times)
+    t_all = torch.tensor([total_ms], device=dev)
+    if world > 1:
+        dist.all_reduce(t_all, op=dist.ReduceOp.MAX)
+    tmax_ms = float(t_all.item())
+    value = world * flops * args.steps / (tmax_ms / 1e3) / 1e12
+    ms_per_step = tmax_ms / args.steps
+    api.check_device_status()
+    idx_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_idx[-args.steps:])
+    att_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_att[-args.steps:])
+
+    # end to end through the public API with host buffers (pinned)
+    host = {k: v.pin_memory() for k, v in g.items()}
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    lse_h = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = out_h.numel() * out_h.element_size() + lse_h.numel() * lse_h.element_size()
+
+    def e2e_step():
+        for k2, v2 in host.items():
+            gd[k2].copy_(v2, non_blocking=True)
+        step(False)
+        out_h.copy_(out, non_blocking=True)
+        lse_h.copy_(lse, non_blocking=True)
+
+    e2e_value = None
+    if not args.no_e2e:
+        e2e_times = timed_steps(e2e_step, max(2, args.steps // 2), args.warmup, flush, dev, torch)
+        e2e_t = torch.tensor([sum(e2e_times)], device=dev)
+        if world > 1:
+            dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
+        e2e_value = world * flops * len(e2e_times) / (float(e2e_t.item()) / 1e3) / 1e12
+
+    peaks = _peaks()
+    att_tflops = flops / (att_ms / 1e3) / 1e12
+    result = {
+        "metric": METRIC,
+        "value": round(value, 3),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded; q/k/v N(0,1) bf16, indexer int8 U[-8,8], weights U{0..4})",
+        "config": {"workload": "dsa_prefill64k: indexer top-2048 + sparse attention, "
+                               "1 x 65536 tokens, 16 q heads / 1 kv head, d=128",
+                   "global_batch": world, "seq_len": w.T, "topk": w.topk,
+                   "attn_flops_per_seq": flops, "l2": "flushed between steps (252 MB write)",
+                   "parallelism": f"replicas x{world} (one sequence per GPU)"},
+        "breakdown_ms": {"indexer_topk": round(idx_ms, 4), "sparse_attn": round(att_ms, 4)},
+        "roofline": {
+            "kernel": "gather_attn_kernel (sparse attention, D=128)",
+            "bound": "tensor",
+            "achieved": round(att_tflops, 2),
+            "peak": peaks["bf16_tflops"],
+            "unit": "TFLOP/s",
+            "frac": round(att_tflops / peaks["bf16_tflops"], 4),
+            "peak_source": peaks["source"] + " bf16 burst",
+            "traffic": None,
+        },
+        "e2e": None if e2e_value is None else
+               {"value": round(e2e_value, 3), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+        "gpu_launches": int(launches),
+    }
+    clocks = clk.summary()
+    if clocks:
+        result["clocks"] = clocks
+
+    if not args.no_extra:
+        extra = extra_measurements(args, dev, torch, api, lib, inputs, flush, world, peaks)
+        result.update(extra)
+
+    if rank == 0 and world == 1 and not args.no_cpu:
+        result["cpu_baseline"] = cpu_baseline(args)
+    if rank == 0:
+        print(json.dumps(result))
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "of measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "of fallback"}
+
+
+def extra_measurements(args, dev, torch, api, lib, inputs, flush, world, peaks):
+    """Decode (IndexCache), NSA and fixed-graph numbers for the same line."""
+    res = {}
+    steps = max(3, args.steps // 2)
+    # --- decode 32 x 131072, 4 layers ---
+    w = inputs.WORKLOADS["dsa_decode128k"]
+    lays = [inputs.gen_decode_layer(w.B, w.T, w.Hq, w.Hkv, w.d, w.Hi, w.di, layer=i, seed=0,
+                                    device=dev) for i in range(w.layers)]
+    n_split = 16
+    outs = [torch.empty((w.B, 1, w.Hq, w.d), dtype=torch.bfloat16, device=dev) for _ in lays]
+    lses = [torch.empty((w.B, 1, w.Hq), dtype=torch.float32, device=dev) for _ in lays]
+    cache = torch.empty((w.B, 1, w.topk), dtype=torch.int32, device=dev)
+    wsb = api.dsa_decode_workspace_bytes(w.B, 1, w.T, w.Hq, w.d, w.Hi, w.di, w.topk, 0, n_split)
+    wsd = torch.empty(wsb, dtype=torch.uint8, device=dev)
+    dec = {}
+    for pattern in ("FSSS", "FFFF"):
+        def dstep(pattern=pattern):
+            api.dsa_decode_layers(pattern, lays, topk=w.topk, n_split=n_split, outs=outs,
+                                  lses=lses, idx_cache=cache, workspace=wsd)
+        # capture the 4-layer step in a CUDA graph (launch-bound at this size)
+        s = torch.cuda.Stream(dev)
+        s.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(s):
+            dstep()
+        torch.cuda.current_stream(dev).wait_stream(s)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            dstep()
+        times = timed_steps(graph.replay, steps, args.warmup, flush, dev, torch)
+        ms = sum(times) / len(times)
+        n_f = pattern.count("F")
+        bytes_step = n_f * (w.B * w.T * w.di) + w.layers * (w.B * w.topk * 2 * w.d * 2 +
+                                                            w.B * w.Hq * w.d * 2 * 2)
+        dec[pattern] = {"ms_per_step": round(ms, 4),
+                        "tokens_per_s": round(world * w.B / (ms / 1e3), 1),
+                        "algorithmic_bytes": int(bytes_step),
+                        "hbm_frac": round(bytes_step / (ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4)}
+        del graph
+    dec["fsss_over_ffff"] = round(dec["FSSS"]["tokens_per_s"] / dec["FFFF"]["tokens_per_s"], 3)
+    res["decode128k"] = dec
+    del lays, wsd
+    torch.cuda.empty_cache()
+    # --- NSA 64K ---
+    w = inputs.WORKLOADS["nsa64k"]
+    g = inputs.gen_nsa(w.B, w.T, w.Hq, w.Hkv, w.d, seed=0)
+    gd = {k: v.to(dev) for k, v in g.items()}
+    o = torch.empty((w.B, w.T, w.Hq, w.d), dtype=torch.bfloat16, device=dev)
+    cfg = dict(cmp_len=w.cmp_len, cmp_stride=w.cmp_stride, sel_block=w.sel_block,
+               sel_topk=w.sel_topk, window=w.window)
+    sel_holder = {}
+
+    def nstep():
+        _, _, sel = api.nsa_fwd(gd["q"], gd["k"], gd["v"], gd["gates"], out=o, **cfg)
+        sel_holder["sel"] = sel
+    times = timed_steps(nstep, max(2, steps // 2), args.warmup, flush, dev, torch)
+    ms = sum(times) / len(times)
+    nsa_fl = nsa_flops(w, sel_holder["sel"], torch)
+    res["nsa64k"] = {"ms_per_step": round(ms, 3), "tflops": round(nsa_fl / (ms / 1e3) / 1e12, 2),
+                     "algorithmic_flops": nsa_fl,
+                     "tensor_frac": round(nsa_fl / (ms / 1e3) / 1e12 / peaks["bf16_tflops"], 4)}
+    del gd, g, o
+    torch.cuda.empty_cache()
+    # --- fixed graph 16K with coordinate bias ---
+    w = inputs.WORKLOADS["spatial16k"]
+    g = inputs.gen_spatial(w.B, w.T, w.Hq, w.d, beta=w.beta, seed=0)
+    gd = {k: v.to(dev) for k, v in g.items()}
+    o = torch.empty((w.B, w.T, w.Hq, w.d), dtype=torch.bfloat16, device=dev)
+    ls = torch.empty((w.B, w.T, w.Hq), dtype=torch.float32, device=dev)
+
+    def sstep():
+        api.sparse_attn_fwd(gd["q"], gd["k"], gd["v"], pattern=(w.window, w.dilated), cq=gd["cq"],
+                            ck=gd["ck"], beta=gd["beta"], out=o, lse=ls)
+    times = timed_steps(sstep, steps, args.warmup, flush, dev, torch)
+    ms = sum(times) / len(times)
+    byts = sum(gd[k].numel() * gd[k].element_size() for k in ("q", "k", "v", "cq", "ck")) + \
+        o.numel() * 2 + ls.numel() * 4
+    res["spatial16k"] = {"ms_per_step": round(ms, 4), "gbs": round(byts / (ms / 1e3) / 1e9, 1),
+                         "algorithmic_bytes": int(byts),
+                         "hbm_frac": round(byts / (ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4)}
+    return res
+
+
+def nsa_flops(w, sel, torch):
+    """Algorithmic FLOPs of the three NSA branches (4*d per query-head-key)."""
+    T, Hq, d = w.T, w.Hq, w.d
+    t = torch.arange(T, dtype=torch.float64)
+    n_cmp = torch.clamp(torch.div(t - (w.cmp_len - 1), w.cmp_stride, rounding_mode="floor") + 1, min=0)
+    n_win = torch.clamp(t + 1, max=w.window)
+    s = sel.to(torch.int64)                                   # [1,T,Hkv,k]
+    start = s * w.sel_block
+    tt = torch.arange(T, device=s.device).view(1, T, 1, 1)
+    n_sel = torch.where(s >= 0, torch.clamp(torch.minimum(tt - start + 1,
+                                                          torch.full_like(start, w.sel_block)), min=0), 0)
+    n_sel = n_sel.sum(dim=-1).to(torch.float64).sum().item() * (Hq // w.Hkv)
+    return 4.0 * d * (Hq * (n_cmp.sum().item() + n_win.sum().item()) + n_sel)
+
+
+# ------------------------------------------------------------- CPU oracle --
+def cpu_baseline(args, max_seconds=25.0):
+    """Time the CPU oracle (as it stands) on a bounded sample of the prefill
+    workload: the full path (indexer top-k + fp64 attention) for a set of
+    query rows spread over the sequence."""
+    import numpy as np
+
+    import oracle
+    from fixed_pattern_sparse_sa_b200 import inputs
+    w = inputs.WORKLOADS["dsa_prefill64k"]
+    g = inputs.gen_dsa(w.B, w.T, w.Hq, w.Hkv, w.d, w.Hi, w.di, seed=0)
+    n = args.cpu_sample_rows or 64
+    while True:
+        rows = np.linspace(0, w.T - 1, n).astype(np.int64)
+        t0 = time.perf_counter()
+        idx, _ = oracle.indexer_topk(g["q_idx"], g["k_idx"], g["w"], w.topk, w.window, rows=rows)
+        full = np.full((w.B, w.T, w.topk + w.window), -1, dtype=np.int32)
+        full[0, rows] = idx
+        oracle.sparse_attn(g["q"], g["k"], g["v"], full, rows=rows)
+        dt = time.perf_counter() - t0
+        if args.cpu_sample_rows or dt >= 8.0 or n >= 4096:
+            break
+        n = min(4096, int(n * max(2.0, 10.0 / max(dt, 1e-3))))
+    counts = np.minimum(rows + 1, w.topk + w.window)
+    fl = 4.0 * w.d * w.Hq * float(counts.sum())
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n} query rows evenly spaced over the 65536-token prefill "
+                      f"(indexer top-2048 + fp64 attention), {dt:.1f} s"}
+
+
+def reference_arm(args, world):
+    """The reference arm for this build is the CPU oracle (there is no
+    runnable upstream implementation): timed on the host cores, each step a
+    bounded sample of the same workload."""
+    import numpy as np
+
+    import oracle
+    from fixed_pattern_sparse_sa_b200 import inputs
+    w = inputs.WORKLOADS["dsa_prefill64k"]
+    g = inputs.gen_dsa(w.B, w.T, w.Hq, w.Hkv, w.d, w.Hi, w.di, seed=0)
+    n = args.cpu_sample_rows or 48
+    rows = np.linspace(0, w.T - 1, n).astype(np.int64)
+    counts = np.minimum(rows + 1, w.topk + w.window)
+    fl = 4.0 * w.d * w.Hq * float(counts.sum())
+    times = []
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        idx, _ = oracle.indexer_topk(g["q_idx"], g["k_idx"], g["w"], w.topk, w.window, rows=rows)
+        full = np.full((w.B, w.T, w.topk + w.window), -1, dtype=np.int32)
+        full[0, rows] = idx
+        oracle.sparse_attn(g["q"], g["k"], g["v"], full, rows=rows)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = fl * len(times) / total / 1e12
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    sample = f"{n} query rows evenly spaced over the 65536-token prefill per step"
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * total / len(times), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "dsa_prefill64k: indexer top-2048 + sparse attention, "
+                                   "1 x 65536 tokens, 16 q heads / 1 kv head, d=128 (row sample)",
+                       "seq_len": w.T, "topk": w.topk},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,269 @@
+"""Thin torch binding over libsa.so.
+
+Argument marshalling only: every function checks dtypes, devices and
+contiguity, allocates outputs and workspace with torch, and calls the C entry
+point of the same name on the current CUDA stream.  All computation happens in
+the library's kernels; there is no CPU path.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+from typing import Optional, Sequence
+
+import torch
+
+from . import _lib
+from ._lib import SAError, check, sa_dsa_layer, sa_pattern
+
+__all__ = ["indexer_topk", "sparse_attn_fwd", "lse_combine", "nsa_fwd",
+           "dsa_decode_layers", "check_device_status", "SAError"]
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _need(t: Optional[torch.Tensor], name: str, dtype, dev=None, ndim=None):
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (there is no CPU path)")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if dev is not None and t.device != dev:
+        raise ValueError(f"{name} is on {t.device}, expected {dev}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def _workspace(nbytes: int, device) -> Optional[torch.Tensor]:
+    if nbytes == 0:
+        return None
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def check_device_status(device=None):
+    """Wait for the current stream and raise if a kernel found a bad index."""
+    lib = _lib.load()
+    with torch.cuda.device(device if device is not None else torch.cuda.current_device()):
+        check(lib.sa_check_device_status(_stream(None)), "sa_check_device_status")
+
+
+# ------------------------------------------------------------------ indexer --
+def indexer_topk(q_idx, k_idx, w, topk: int, window: int = 0,
+                 q_pos0: Optional[int] = None, out_idx=None, out_count=None, workspace=None):
+    """Exact causal top-k of the lightweight indexer (sa_indexer_topk).
+
+    q_idx int8 [B,Tq,Hi,di], k_idx int8 [B,L,di], w int32 [B,Tq,Hi].
+    q_pos0 defaults to L - Tq (the queries are the last Tq positions).
+    Returns (idx int32 [B,Tq,topk+window], count int32 [B,Tq]).
+    """
+    lib = _lib.load()
+    dev = q_idx.device
+    _need(q_idx, "q_idx", torch.int8, dev, 4)
+    _need(k_idx, "k_idx", torch.int8, dev, 3)
+    _need(w, "w", torch.int32, dev, 3)
+    B, Tq, Hi, di = q_idx.shape
+    L = k_idx.shape[1]
+    if k_idx.shape != (B, L, di) or w.shape != (B, Tq, Hi):
+        raise ValueError("indexer_topk: shape mismatch")
+    pos0 = L - Tq if q_pos0 is None else int(q_pos0)
+    K = topk + window
+    if out_idx is None:
+        out_idx = torch.empty((B, Tq, K), dtype=torch.int32, device=dev)
+    if out_count is None:
+        out_count = torch.empty((B, Tq), dtype=torch.int32, device=dev)
+    nbytes = lib.sa_indexer_topk_workspace_size(B, Tq, L, Hi, di, topk, window)
+    ws = workspace if (workspace is not None and workspace.numel() >= nbytes) \
+        else _workspace(nbytes, dev)
+    with torch.cuda.device(dev):
+        check(lib.sa_indexer_topk(_ptr(q_idx), _ptr(k_idx), _ptr(w), B, Tq, L, Hi, di, pos0,
+                                  topk, window, _ptr(out_idx), _ptr(out_count), _ptr(ws),
+                                  nbytes, _stream(dev)), "sa_indexer_topk")
+    return out_idx, out_count
+
+
+# ---------------------------------------------------------------- attention --
+def sparse_attn_fwd(q, k, v, idx=None, pattern: Optional[Sequence[int]] = None,
+                    cq=None, ck=None, beta=None, scale: Optional[float] = None,
+                    n_split: int = 1, q_pos0: Optional[int] = None,
+                    return_partials: bool = False, out=None, lse=None):
+    """Gathered-KV sparse attention (sa_sparse_attn_fwd).
+
+    q bf16 [B,Tq,Hq,d], k/v bf16 [B,L,Hkv,d]; idx int32 [B,Tq,K] or
+    [B,Tq,idx_heads,K] (-1 padded), or pattern = (window, dilated).
+    Optional coordinate bias cq fp32 [B,Tq,Hq,3], ck fp32 [B,L,Hkv,3],
+    beta fp32 [Hq].  Returns (out bf16 [B,Tq,Hq,d], lse fp32 [B,Tq,Hq]) and,
+    with return_partials (n_split > 1), also (part_o, part_lse).
+    """
+    lib = _lib.load()
+    dev = q.device
+    _need(q, "q", torch.bfloat16, dev, 4)
+    _need(k, "k", torch.bfloat16, dev, 4)
+    _need(v, "v", torch.bfloat16, dev, 4)
+    B, Tq, Hq, d = q.shape
+    L, Hkv = k.shape[1], k.shape[2]
+    if k.shape != (B, L, Hkv, d) or v.shape != k.shape:
+        raise ValueError("sparse_attn_fwd: k/v shape mismatch")
+    pos0 = L - Tq if q_pos0 is None else int(q_pos0)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    pat = None
+    idx_heads, K = 1, 0
+    if idx is not None:
+        _need(idx, "idx", torch.int32, dev)
+        if idx.dim() == 3:
+            idx_heads, K = 1, idx.shape[2]
+        elif idx.dim() == 4:
+            idx_heads, K = idx.shape[2], idx.shape[3]
+        else:
+            raise ValueError("idx must be [B,Tq,K] or [B,Tq,idx_heads,K]")
+        if idx.shape[:2] != (B, Tq):
+            raise ValueError("idx shape mismatch")
+    elif pattern is not None:
+        pat = sa_pattern(int(pattern[0]), int(bool(pattern[1])))
+    else:
+        raise ValueError("need idx or pattern")
+    if cq is not None or ck is not None or beta is not None:
+        _need(cq, "cq", torch.float32, dev, 4)
+        _need(ck, "ck", torch.float32, dev, 4)
+        _need(beta, "beta", torch.float32, dev, 1)
+    if out is None:
+        out = torch.empty((B, Tq, Hq, d), dtype=torch.bfloat16, device=dev)
+    if lse is None:
+        lse = torch.empty((B, Tq, Hq), dtype=torch.float32, device=dev)
+    po = pl = None
+    if n_split > 1:
+        po = torch.empty((n_split, B, Tq, Hq, d), dtype=torch.float32, device=dev)
+        pl = torch.empty((n_split, B, Tq, Hq), dtype=torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        check(lib.sa_sparse_attn_fwd(
+            _ptr(q), _ptr(k), _ptr(v), B, Tq, L, Hq, Hkv, d, pos0,
+            _ptr(idx), idx_heads, K, ctypes.byref(pat) if pat is not None else None,
+            _ptr(cq), _ptr(ck), _ptr(beta), float(scale), int(n_split),
+            _ptr(out), _ptr(lse), _ptr(po), _ptr(pl), None, 0, _stream(dev)),
+            "sa_sparse_attn_fwd")
+    if return_partials:
+        return out, lse, po, pl
+    return out, lse
+
+
+def lse_combine(part_o, part_lse, out=None, lse=None):
+    """Log-sum-exp merge of split partials (sa_lse_combine).
+
+    part_o fp32 [S, ..., d], part_lse fp32 [S, ...] -> (out bf16 [..., d], lse fp32 [...]).
+    """
+    lib = _lib.load()
+    dev = part_o.device
+    _need(part_o, "part_o", torch.float32, dev)
+    _need(part_lse, "part_lse", torch.float32, dev)
+    S, d = part_o.shape[0], part_o.shape[-1]
+    lead = tuple(part_o.shape[1:-1])
+    if tuple(part_lse.shape) != (S, *lead):
+        raise ValueError("lse_combine: shape mismatch")
+    rows = math.prod(lead)
+    if out is None:
+        out = torch.empty((*lead, d), dtype=torch.bfloat16, device=dev)
+    if lse is None:
+        lse = torch.empty(lead, dtype=torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        check(lib.sa_lse_combine(_ptr(part_o), _ptr(part_lse), S, rows, d, _ptr(out), _ptr(lse),
+                                 _stream(dev)), "sa_lse_combine")
+    return out, lse
+
+
+# ---------------------------------------------------------------------- NSA --
+def nsa_fwd(q, k, v, gates, cmp_len: int, cmp_stride: int, sel_block: int, sel_topk: int,
+            window: int, scale: Optional[float] = None, out=None):
+    """NSA forward (sa_nsa_fwd): compressed, selected and window branches.
+
+    Returns (out bf16 [B,T,Hq,d], lse_branches fp32 [B,T,Hq,3],
+    sel_idx int32 [B,T,Hkv,sel_topk]).
+    """
+    lib = _lib.load()
+    dev = q.device
+    _need(q, "q", torch.bfloat16, dev, 4)
+    _need(k, "k", torch.bfloat16, dev, 4)
+    _need(v, "v", torch.bfloat16, dev, 4)
+    _need(gates, "gates", torch.float32, dev, 4)
+    B, T, Hq, d = q.shape
+    Hkv = k.shape[2]
+    if k.shape != (B, T, Hkv, d) or v.shape != k.shape or gates.shape != (B, T, Hq, 3):
+        raise ValueError("nsa_fwd: shape mismatch")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((B, T, Hq, d), dtype=torch.bfloat16, device=dev)
+    lse3 = torch.empty((B, T, Hq, 3), dtype=torch.float32, device=dev)
+    sel = torch.empty((B, T, Hkv, sel_topk), dtype=torch.int32, device=dev)
+    nbytes = lib.sa_nsa_workspace_size(B, T, Hq, Hkv, d, cmp_len, cmp_stride, sel_block, sel_topk)
+    ws = _workspace(nbytes, dev)
+    with torch.cuda.device(dev):
+        check(lib.sa_nsa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(gates), B, T, Hq, Hkv, d, cmp_len,
+                             cmp_stride, sel_block, sel_topk, window, float(scale), _ptr(out),
+                             _ptr(lse3), _ptr(sel), _ptr(ws), nbytes, _stream(dev)), "sa_nsa_fwd")
+    return out, lse3, sel
+
+
+# --------------------------------------------------------------- IndexCache --
+def dsa_decode_layers(pattern: str, layers, topk: int, window: int = 0, n_split: int = 1,
+                      q_pos0: Optional[int] = None, scale: Optional[float] = None,
+                      outs=None, lses=None, idx_cache=None, workspace=None):
+    """IndexCache layer loop (sa_dsa_decode_layers).
+
+    layers: list of dicts with q, k, v, q_idx, k_idx, w (same shapes for every
+    layer).  F layers run the indexer, S layers reuse the cached indices.
+    Returns (outs, lses, idx_cache).
+    """
+    lib = _lib.load()
+    n = len(layers)
+    if len(pattern) < n:
+        raise ValueError("pattern shorter than the layer list")
+    l0 = layers[0]
+    dev = l0["q"].device
+    B, Tq, Hq, d = l0["q"].shape
+    L, Hkv = l0["k"].shape[1], l0["k"].shape[2]
+    Hi, di = l0["q_idx"].shape[2], l0["q_idx"].shape[3]
+    for ly in layers:
+        _need(ly["q"], "q", torch.bfloat16, dev, 4)
+        _need(ly["k"], "k", torch.bfloat16, dev, 4)
+        _need(ly["v"], "v", torch.bfloat16, dev, 4)
+        _need(ly["q_idx"], "q_idx", torch.int8, dev, 4)
+        _need(ly["k_idx"], "k_idx", torch.int8, dev, 3)
+        _need(ly["w"], "w", torch.int32, dev, 3)
+    pos0 = L - Tq if q_pos0 is None else int(q_pos0)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if outs is None:
+        outs = [torch.empty((B, Tq, Hq, d), dtype=torch.bfloat16, device=dev) for _ in range(n)]
+    if lses is None:
+        lses = [torch.empty((B, Tq, Hq), dtype=torch.float32, device=dev) for _ in range(n)]
+    if idx_cache is None:
+        idx_cache = torch.empty((B, Tq, topk + window), dtype=torch.int32, device=dev)
+    arr = (sa_dsa_layer * n)()
+    for i, ly in enumerate(layers):
+        arr[i] = sa_dsa_layer(ly["q"].data_ptr(), ly["k"].data_ptr(), ly["v"].data_ptr(),
+                              ly["q_idx"].data_ptr(), ly["k_idx"].data_ptr(), ly["w"].data_ptr(),
+                              outs[i].data_ptr(), lses[i].data_ptr())
+    nbytes = lib.sa_dsa_decode_layers_workspace_size(B, Tq, L, Hq, d, Hi, di, topk, window, n_split)
+    if workspace is None or workspace.numel() < nbytes:
+        workspace = _workspace(nbytes, dev)
+    with torch.cuda.device(dev):
+        check(lib.sa_dsa_decode_layers(pattern.encode(), n, arr, B, Tq, L, Hq, Hkv, d, Hi, di,
+                                       pos0, topk, window, float(scale), int(n_split),
+                                       _ptr(idx_cache), _ptr(workspace), nbytes, _stream(dev)),
+              "sa_dsa_decode_layers")
+    return outs, lses, idx_cache
+
+
+def dsa_decode_workspace_bytes(B, Tq, L, Hq, d, Hi, di, topk, window=0, n_split=1) -> int:
+    return int(_lib.load().sa_dsa_decode_layers_workspace_size(B, Tq, L, Hq, d, Hi, di, topk,
+                                                               window, n_split))

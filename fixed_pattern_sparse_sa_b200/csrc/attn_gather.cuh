@@ -1,0 +1,373 @@
+// attn_gather.cuh -- gathered-KV sparse attention, one warp per
+// (query, KV head, 16-head chunk, split) work item.
+//
+// Operation (every page reduces to it once a query's index set is known):
+//   z_j = scale * q.k_j + bias_j over j in S,  o = softmax(z) V,  lse = log sum exp z.
+// The 16 query heads that share one KV head form the 16 rows of an m16
+// tensor-core tile, so every gathered K/V row feeds 16 heads ("shared KV
+// fetch" of the NSA page, section "Analisis Profundo").  Keys are streamed in
+// chunks of 32 rows through a per-warp multi-stage cp.async pipeline into
+// XOR-swizzled shared memory, scored with mma.sync m16n8k16 (bf16 -> fp32),
+// folded into an online softmax and multiplied into V with a second mma.
+#pragma once
+
+#include "sa_common.cuh"
+
+namespace sa {
+
+enum KeySource : int {
+    KS_IDX = 0,      // explicit index list idx[b, t, ih, e]
+    KS_PATTERN = 1,  // fixed window + dilated powers of two
+    KS_BLOCKS = 2,   // NSA selected blocks: idx holds block ids
+    KS_RANGE = 3,    // recent window: j = p - window + 1 + e
+    KS_CMP = 4,      // NSA compressed tokens: i = e, visible iff i*stride+len-1 <= p
+};
+
+struct GatherParams {
+    const __nv_bfloat16 *q;   // [B, Tq, Hq, D]
+    const __nv_bfloat16 *k;   // [B, Lk, Hkv, D]
+    const __nv_bfloat16 *v;   // [B, Lk, Hkv, D]
+    const __nv_bfloat16 *klo; // optional low half of k (k ~ k + klo), same layout
+    int B, Tq, Lk, Hq, Hkv, G;
+    long long q_pos0;
+    const int32_t *idx;       // KS_IDX: [B,Tq,idx_heads,K]; KS_BLOCKS: [B,Tq,Hkv,K] block ids
+    int idx_heads, K;
+    int window, dilated;      // KS_PATTERN / KS_RANGE
+    int block;                // KS_BLOCKS block length; KS_CMP stride
+    int cmp_len;              // KS_CMP window length
+    int entries;              // virtual list length per item
+    int per_split;            // entries handled by one split piece
+    int n_split, n_hchunk;
+    const float *cq, *ck, *beta;   // optional coordinate bias
+    float scale_log2;         // scale * log2(e)
+    __nv_bfloat16 *out;       // [B,Tq,Hq,D] (n_split == 1)
+    float *lse;               // [B,Tq,Hq]   (nullable)
+    float *part_o;            // [n_split,B,Tq,Hq,D] (n_split > 1)
+    float *part_lse;          // [n_split,B,Tq,Hq]
+    float *out_f32;           // optional fp32 output [B,Tq,Hq,D] instead of bf16
+    unsigned *err;
+};
+
+// Key position for virtual entry e of the item, or -1 if the entry is empty
+// or masked.  Raises the error word for an explicit index that is out of
+// range or in the future.
+template <int SRC>
+__device__ __forceinline__ int key_at(const GatherParams &p, int b, int t, int g, long long pos,
+                                      int e, int e_end) {
+    if (e >= e_end) return -1;
+    if constexpr (SRC == KS_IDX) {
+        const int32_t *list =
+            p.idx + ((long long)(b * p.Tq + t) * p.idx_heads + (p.idx_heads == 1 ? 0 : g)) * p.K;
+        int j = __ldg(list + e);
+        if (j == -1) return -1;
+        if (j < 0 || j >= p.Lk || (long long)j > pos) {
+            raise_error(p.err, ERR_BAD_INDEX);
+            return -1;
+        }
+        return j;
+    } else if constexpr (SRC == KS_PATTERN) {
+        long long nw = pos + 1 < p.window ? pos + 1 : p.window;
+        if (e < nw) return (int)(pos - e);
+        if (!p.dilated) return -1;
+        // dilated distances 2^i with 2^i >= window (the rest are in the window)
+        int i0 = 0;
+        while ((1LL << i0) < p.window) ++i0;
+        int m = e - (int)nw;
+        if (i0 + m >= 62) return -1;
+        long long o = 1LL << (i0 + m);
+        if (o >= pos) return -1;
+        return (int)(pos - o);
+    } else if constexpr (SRC == KS_BLOCKS) {
+        const int32_t *list = p.idx + ((long long)(b * p.Tq + t) * p.Hkv + g) * p.K;
+        int blk = __ldg(list + e / p.block);
+        if (blk == -1) return -1;
+        long long j = (long long)blk * p.block + e % p.block;
+        if (blk < 0 || (long long)blk * p.block >= p.Lk) {
+            raise_error(p.err, ERR_BAD_BLOCK);
+            return -1;
+        }
+        if (j > pos || j >= p.Lk) return -1;   // causal mask inside the block
+        return (int)j;
+    } else if constexpr (SRC == KS_RANGE) {
+        long long j = pos - p.window + 1 + e;
+        return j < 0 ? -1 : (int)j;
+    } else {  // KS_CMP
+        long long end = (long long)e * p.block + p.cmp_len - 1;
+        return (end <= pos && e < p.Lk) ? e : -1;
+    }
+}
+
+// KLO: keys are held as a bf16 pair (hi, lo) whose sum carries ~16 mantissa
+// bits; q.k is taken on both halves (used for the NSA compressed keys, which
+// are means and do not fit bf16 exactly).
+template <int D, int STAGES, int SRC, bool BIAS, bool KLO = false>
+__global__ void __launch_bounds__(128) gather_attn_kernel(const GatherParams p) {
+    constexpr int NK = 32;                 // keys per chunk
+    constexpr int ROWB = D * 2;            // bytes of one K/V row
+    constexpr int UNITS = ROWB / 16;       // 16-byte units per row
+    constexpr int CH = NK * ROWB;          // bytes of one K (or V) chunk
+    constexpr int KS_D = D / 16;           // k-steps of q.k
+    constexpr int NT_D = D / 8;            // n-tiles of P.V
+    constexpr int CP_ITERS = NK * UNITS / 32;
+    constexpr int SB = (KLO ? 3 : 2) * CH;   // one stage: K | V | (K lo)
+
+    extern __shared__ __align__(1024) unsigned char smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    unsigned char *wsm = smem + warp * (STAGES * (SB + NK * 4));
+    int *keys_s = reinterpret_cast<int *>(wsm + STAGES * SB);
+
+    const long long n_items = (long long)p.B * p.Tq * p.Hkv * p.n_hchunk * p.n_split;
+    const long long item = (long long)blockIdx.x * 4 + warp;
+    if (item >= n_items) return;   // warps are independent: no block barrier below
+
+    long long rem = item;
+    const int s = (int)(rem % p.n_split); rem /= p.n_split;
+    const int hc = (int)(rem % p.n_hchunk); rem /= p.n_hchunk;
+    const int g = (int)(rem % p.Hkv); rem /= p.Hkv;
+    const int t = (int)(rem % p.Tq); rem /= p.Tq;
+    const int b = (int)rem;
+    const long long pos = p.q_pos0 + t;
+
+    const int gr = lane >> 2, qc = lane & 3;
+    const int hr0 = hc * 16 + gr, hr1 = hr0 + 8;          // head index within the group
+    const bool v0 = hr0 < p.G, v1 = hr1 < p.G;
+    const int h0 = g * p.G + hr0, h1 = g * p.G + hr1;
+    const long long qrow0 = ((long long)(b * p.Tq + t) * p.Hq + h0) * D;
+    const long long qrow1 = ((long long)(b * p.Tq + t) * p.Hq + h1) * D;
+
+    // Q fragments (A operand, 16 rows x D), straight from global memory.
+    unsigned qf[KS_D][4];
+    {
+        const unsigned *q0 = reinterpret_cast<const unsigned *>(p.q + qrow0);
+        const unsigned *q1 = reinterpret_cast<const unsigned *>(p.q + qrow1);
+#pragma unroll
+        for (int ks = 0; ks < KS_D; ++ks) {
+            qf[ks][0] = v0 ? __ldg(q0 + ks * 8 + qc) : 0u;
+            qf[ks][1] = v1 ? __ldg(q1 + ks * 8 + qc) : 0u;
+            qf[ks][2] = v0 ? __ldg(q0 + ks * 8 + qc + 4) : 0u;
+            qf[ks][3] = v1 ? __ldg(q1 + ks * 8 + qc + 4) : 0u;
+        }
+    }
+    float cq0[3] = {0.f, 0.f, 0.f}, cq1[3] = {0.f, 0.f, 0.f}, be0 = 0.f, be1 = 0.f;
+    if constexpr (BIAS) {
+        if (v0) {
+            const float *c = p.cq + ((long long)(b * p.Tq + t) * p.Hq + h0) * 3;
+            cq0[0] = c[0]; cq0[1] = c[1]; cq0[2] = c[2];
+            be0 = p.beta[h0] * kLog2e;
+        }
+        if (v1) {
+            const float *c = p.cq + ((long long)(b * p.Tq + t) * p.Hq + h1) * 3;
+            cq1[0] = c[0]; cq1[1] = c[1]; cq1[2] = c[2];
+            be1 = p.beta[h1] * kLog2e;
+        }
+    }
+
+    const int e_beg = s * p.per_split;
+    int e_end = min(p.entries, e_beg + p.per_split);
+    if constexpr (SRC == KS_CMP) {
+        // only the compressed tokens already complete at this position
+        const long long nv = pos >= p.cmp_len - 1 ? (pos - p.cmp_len + 1) / p.block + 1 : 0;
+        e_end = (int)min((long long)e_end, nv);
+    }
+    const int n_chunks = e_end > e_beg ? (e_end - e_beg + NK - 1) / NK : 0;
+
+    const __nv_bfloat16 *kb = p.k + ((long long)b * p.Lk * p.Hkv + g) * D;
+    const __nv_bfloat16 *vb = p.v + ((long long)b * p.Lk * p.Hkv + g) * D;
+    const __nv_bfloat16 *lb = KLO ? p.klo + ((long long)b * p.Lk * p.Hkv + g) * D : nullptr;
+    const long long rstride = (long long)p.Hkv * D;
+
+    auto issue = [&](int ci) {
+        const int st = ci % STAGES;
+        unsigned char *ks_ = wsm + st * SB;
+        unsigned char *vs_ = ks_ + CH;
+        int j = -1;
+        if (ci < n_chunks) j = key_at<SRC>(p, b, t, g, pos, e_beg + ci * NK + lane, e_end);
+        keys_s[st * NK + lane] = j;
+        if (ci < n_chunks) {
+#pragma unroll
+            for (int it = 0; it < CP_ITERS; ++it) {
+                const int lin = it * 32 + lane;
+                const int rr = lin / UNITS, u = lin % UNITS;
+                const int jr = __shfl_sync(0xffffffffu, j, rr);
+                const long long off = jr >= 0 ? (long long)jr * rstride + u * 8 : 0;
+                const int nb = jr >= 0 ? 16 : 0;
+                const int sw = (u ^ (rr & 7)) * 16;
+                cp_async16(ks_ + rr * ROWB + sw, kb + off, nb);
+                cp_async16(vs_ + rr * ROWB + sw, vb + off, nb);
+                if constexpr (KLO) cp_async16(vs_ + CH + rr * ROWB + sw, lb + off, nb);
+            }
+        }
+        cp_async_commit();
+    };
+
+    float o[NT_D][4];
+#pragma unroll
+    for (int i = 0; i < NT_D; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+
+#pragma unroll
+    for (int ci = 0; ci < STAGES - 1; ++ci) issue(ci);
+
+    for (int ci = 0; ci < n_chunks; ++ci) {
+        issue(ci + STAGES - 1);
+        cp_async_wait<STAGES - 1>();
+        __syncwarp();
+        const int st = ci % STAGES;
+        const unsigned char *ks_ = wsm + st * SB;
+        const unsigned char *vs_ = ks_ + CH;
+        const int jl = keys_s[st * NK + lane];
+        const unsigned vmask = __ballot_sync(0xffffffffu, jl >= 0);
+        if (vmask != 0u) {
+            float sc[NK / 8][4];
+#pragma unroll
+            for (int i = 0; i < NK / 8; ++i) sc[i][0] = sc[i][1] = sc[i][2] = sc[i][3] = 0.f;
+#pragma unroll
+            for (int ks = 0; ks < KS_D; ++ks) {
+#pragma unroll
+                for (int np = 0; np < NK / 16; ++np) {
+                    const int mi = lane >> 3, ri = lane & 7;
+                    const int key = np * 16 + (mi >> 1) * 8 + ri;
+                    const int unit = ks * 2 + (mi & 1);
+                    unsigned b0, b1, b2, b3;
+                    ldsm_x4(b0, b1, b2, b3, ks_ + key * ROWB + ((unit ^ (key & 7)) * 16));
+                    mma_bf16_16816(sc[2 * np], qf[ks], b0, b1);
+                    mma_bf16_16816(sc[2 * np + 1], qf[ks], b2, b3);
+                    if constexpr (KLO) {
+                        ldsm_x4(b0, b1, b2, b3, vs_ + CH + key * ROWB + ((unit ^ (key & 7)) * 16));
+                        mma_bf16_16816(sc[2 * np], qf[ks], b0, b1);
+                        mma_bf16_16816(sc[2 * np + 1], qf[ks], b2, b3);
+                    }
+                }
+            }
+            // scale, bias, mask; running max
+            float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+            for (int nt = 0; nt < NK / 8; ++nt) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int kk = nt * 8 + 2 * qc + (e & 1);
+                    float x = sc[nt][e] * p.scale_log2;
+                    if constexpr (BIAS) {
+                        const int jk = __shfl_sync(0xffffffffu, jl, kk);
+                        if (jk >= 0) {
+                            const float *c = p.ck + ((long long)(b * p.Lk + jk) * p.Hkv + g) * 3;
+                            const float *a = (e >> 1) ? cq1 : cq0;
+                            const float dx = a[0] - __ldg(c), dy = a[1] - __ldg(c + 1),
+                                        dz = a[2] - __ldg(c + 2);
+                            x -= ((e >> 1) ? be1 : be0) * (dx * dx + dy * dy + dz * dz);
+                        }
+                    }
+                    x = ((vmask >> kk) & 1u) ? x : -INFINITY;
+                    sc[nt][e] = x;
+                }
+                mx0 = fmaxf(mx0, fmaxf(sc[nt][0], sc[nt][1]));
+                mx1 = fmaxf(mx1, fmaxf(sc[nt][2], sc[nt][3]));
+            }
+            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+            const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+            const float mu0 = mn0 == -INFINITY ? 0.f : mn0;
+            const float mu1 = mn1 == -INFINITY ? 0.f : mn1;
+            const float al0 = exp2f(m0 - mu0), al1 = exp2f(m1 - mu1);
+            m0 = mn0; m1 = mn1;
+            float rs0 = 0.f, rs1 = 0.f;
+#pragma unroll
+            for (int nt = 0; nt < NK / 8; ++nt) {
+                sc[nt][0] = exp2f(sc[nt][0] - mu0);
+                sc[nt][1] = exp2f(sc[nt][1] - mu0);
+                sc[nt][2] = exp2f(sc[nt][2] - mu1);
+                sc[nt][3] = exp2f(sc[nt][3] - mu1);
+                rs0 += sc[nt][0] + sc[nt][1];
+                rs1 += sc[nt][2] + sc[nt][3];
+            }
+            l0 = l0 * al0 + rs0;
+            l1 = l1 * al1 + rs1;
+#pragma unroll
+            for (int i = 0; i < NT_D; ++i) {
+                o[i][0] *= al0; o[i][1] *= al0;
+                o[i][2] *= al1; o[i][3] *= al1;
+            }
+            // P (bf16) * V
+#pragma unroll
+            for (int kp = 0; kp < NK / 16; ++kp) {
+                unsigned pa[4];
+                pa[0] = pack_bf16(sc[2 * kp][0], sc[2 * kp][1]);
+                pa[1] = pack_bf16(sc[2 * kp][2], sc[2 * kp][3]);
+                pa[2] = pack_bf16(sc[2 * kp + 1][0], sc[2 * kp + 1][1]);
+                pa[3] = pack_bf16(sc[2 * kp + 1][2], sc[2 * kp + 1][3]);
+#pragma unroll
+                for (int dp = 0; dp < NT_D / 2; ++dp) {
+                    const int mi = lane >> 3, ri = lane & 7;
+                    const int key = kp * 16 + (mi & 1) * 8 + ri;
+                    const int unit = dp * 2 + (mi >> 1);
+                    unsigned b0, b1, b2, b3;
+                    ldsm_x4_t(b0, b1, b2, b3, vs_ + key * ROWB + ((unit ^ (key & 7)) * 16));
+                    mma_bf16_16816(o[2 * dp], pa, b0, b1);
+                    mma_bf16_16816(o[2 * dp + 1], pa, b2, b3);
+                }
+            }
+        }
+        __syncwarp();
+    }
+    cp_async_wait<0>();
+
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+    const float inv0 = l0 > 0.f ? 1.f / l0 : 0.f, inv1 = l1 > 0.f ? 1.f / l1 : 0.f;
+    const float lse0 = l0 > 0.f ? (m0 + log2f(l0)) * kLn2 : -INFINITY;
+    const float lse1 = l1 > 0.f ? (m1 + log2f(l1)) * kLn2 : -INFINITY;
+
+    const long long orow0 = (long long)(b * p.Tq + t) * p.Hq + h0;
+    const long long orow1 = (long long)(b * p.Tq + t) * p.Hq + h1;
+    if (p.n_split == 1) {
+        if (p.out_f32) {
+#pragma unroll
+            for (int nt = 0; nt < NT_D; ++nt) {
+                const int dcol = nt * 8 + 2 * qc;
+                if (v0) *reinterpret_cast<float2 *>(p.out_f32 + orow0 * D + dcol) =
+                    make_float2(o[nt][0] * inv0, o[nt][1] * inv0);
+                if (v1) *reinterpret_cast<float2 *>(p.out_f32 + orow1 * D + dcol) =
+                    make_float2(o[nt][2] * inv1, o[nt][3] * inv1);
+            }
+        } else {
+#pragma unroll
+            for (int nt = 0; nt < NT_D; ++nt) {
+                const int dcol = nt * 8 + 2 * qc;
+                if (v0) *reinterpret_cast<unsigned *>(p.out + orow0 * D + dcol) =
+                    pack_bf16(o[nt][0] * inv0, o[nt][1] * inv0);
+                if (v1) *reinterpret_cast<unsigned *>(p.out + orow1 * D + dcol) =
+                    pack_bf16(o[nt][2] * inv1, o[nt][3] * inv1);
+            }
+        }
+        if (p.lse && qc == 0) {
+            if (v0) p.lse[orow0] = lse0;
+            if (v1) p.lse[orow1] = lse1;
+        }
+    } else {
+        const long long rows = (long long)p.B * p.Tq * p.Hq;
+        float *po = p.part_o + (long long)s * rows * D;
+#pragma unroll
+        for (int nt = 0; nt < NT_D; ++nt) {
+            const int dcol = nt * 8 + 2 * qc;
+            if (v0) *reinterpret_cast<float2 *>(po + orow0 * D + dcol) =
+                make_float2(o[nt][0] * inv0, o[nt][1] * inv0);
+            if (v1) *reinterpret_cast<float2 *>(po + orow1 * D + dcol) =
+                make_float2(o[nt][2] * inv1, o[nt][3] * inv1);
+        }
+        if (qc == 0) {
+            if (v0) p.part_lse[s * rows + orow0] = lse0;
+            if (v1) p.part_lse[s * rows + orow1] = lse1;
+        }
+    }
+}
+
+template <int D, int STAGES, bool KLO = false>
+constexpr int gather_smem_bytes() {
+    return 4 * STAGES * ((KLO ? 3 : 2) * 32 * D * 2 + 32 * 4);
+}
+
+}  // namespace sa

@@ -1,0 +1,600 @@
+// sa_api.cu -- C ABI entry points of libsa.so (declared in include/sa.h).
+//
+// Host code only validates, sizes workspace and launches; every step of the
+// computation runs in the kernels of attn_gather.cuh, indexer.cuh and
+// nsa_misc.cuh.  There is no CPU fallback.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/sa.h"
+#include "attn_gather.cuh"
+#include "indexer.cuh"
+#include "nsa_misc.cuh"
+
+using namespace sa;
+
+// ------------------------------------------------------------- error state --
+static thread_local std::string g_last_error;
+
+static int fail(int code, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return code;
+}
+
+// Kernels enqueued by this process (all devices), for launch accounting.
+static std::atomic<unsigned long long> g_launches{0};
+
+#define SA_CHECK_LAUNCH(what)                                                              \
+    do {                                                                                   \
+        cudaError_t e_ = cudaGetLastError();                                               \
+        if (e_ != cudaSuccess) return fail(SA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e_)); \
+        g_launches.fetch_add(1, std::memory_order_relaxed);                                \
+    } while (0)
+
+// Device error word: one per device, set with atomicOr by kernels that find a
+// bad index; read and cleared by sa_check_device_status().
+__device__ unsigned g_sa_device_error;
+
+static constexpr int kMaxDevices = 64;
+static unsigned *g_err_ptr[kMaxDevices];
+static std::mutex g_err_mu;
+
+static int device_error_word(unsigned **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(SA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (dev < 0 || dev >= kMaxDevices) return fail(SA_ERR_UNSUPPORTED, "device id %d", dev);
+    std::lock_guard<std::mutex> lk(g_err_mu);
+    if (!g_err_ptr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_sa_device_error);
+        if (e != cudaSuccess)
+            return fail(SA_ERR_CUDA, "cudaGetSymbolAddress: %s", cudaGetErrorString(e));
+        g_err_ptr[dev] = static_cast<unsigned *>(p);
+    }
+    *out = g_err_ptr[dev];
+    return SA_OK;
+}
+
+static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+static bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+static cudaStream_t as_stream(void *s) { return static_cast<cudaStream_t>(s); }
+static size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+template <typename K>
+static int set_smem(K kernel, int bytes) {
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return fail(SA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    return SA_OK;
+}
+
+// -------------------------------------------------------- gather launches --
+template <int D, int SRC, bool BIAS, bool KLO = false>
+static int launch_gather_t(const GatherParams &p, cudaStream_t st) {
+    constexpr int STAGES = D == 128 ? (KLO ? 2 : 3) : 4;
+    constexpr int smem = gather_smem_bytes<D, STAGES, KLO>();
+    auto kern = gather_attn_kernel<D, STAGES, SRC, BIAS, KLO>;
+    int rc = set_smem(kern, smem);
+    if (rc) return rc;
+    const long long items = (long long)p.B * p.Tq * p.Hkv * p.n_hchunk * p.n_split;
+    if (items == 0) return SA_OK;
+    const long long blocks = (items + 3) / 4;
+    kern<<<(unsigned)blocks, 128, smem, st>>>(p);
+    SA_CHECK_LAUNCH("gather_attn_kernel");
+    return SA_OK;
+}
+
+template <int D>
+static int launch_gather_d(const GatherParams &p, int src, bool bias, cudaStream_t st) {
+    switch (src) {
+        case KS_IDX: return bias ? launch_gather_t<D, KS_IDX, true>(p, st) : launch_gather_t<D, KS_IDX, false>(p, st);
+        case KS_PATTERN:
+            return bias ? launch_gather_t<D, KS_PATTERN, true>(p, st) : launch_gather_t<D, KS_PATTERN, false>(p, st);
+        case KS_BLOCKS: return launch_gather_t<D, KS_BLOCKS, false>(p, st);
+        case KS_RANGE: return launch_gather_t<D, KS_RANGE, false>(p, st);
+        case KS_CMP: return launch_gather_t<D, KS_CMP, false, true>(p, st);
+    }
+    return fail(SA_ERR_UNSUPPORTED, "key source %d", src);
+}
+
+static int launch_gather(const GatherParams &p, int d, int src, bool bias, cudaStream_t st) {
+    if (d == 64) return launch_gather_d<64>(p, src, bias, st);
+    if (d == 128) return launch_gather_d<128>(p, src, bias, st);
+    return fail(SA_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
+}
+
+static int launch_combine(const float *po, const float *pl, int n_split, long long rows, int d,
+                          void *out, float *lse, cudaStream_t st) {
+    if (rows == 0) return SA_OK;
+    const unsigned blocks = (unsigned)((rows + 7) / 8);
+    if (d == 64)
+        lse_combine_kernel<64><<<blocks, 256, 0, st>>>(po, pl, n_split, rows, (__nv_bfloat16 *)out, lse);
+    else if (d == 128)
+        lse_combine_kernel<128><<<blocks, 256, 0, st>>>(po, pl, n_split, rows, (__nv_bfloat16 *)out, lse);
+    else
+        return fail(SA_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
+    SA_CHECK_LAUNCH("lse_combine_kernel");
+    return SA_OK;
+}
+
+// Public entry points: C linkage comes from the declarations in sa.h.
+
+int sa_version(void) { return 100; }
+
+uint64_t sa_launch_counter(void) { return g_launches.load(std::memory_order_relaxed); }
+
+const char *sa_last_error_string(void) { return g_last_error.c_str(); }
+
+const char *sa_status_string(int s) {
+    switch (s) {
+        case SA_OK: return "SA_OK";
+        case SA_ERR_INVALID_ARG: return "SA_ERR_INVALID_ARG";
+        case SA_ERR_UNSUPPORTED: return "SA_ERR_UNSUPPORTED";
+        case SA_ERR_WORKSPACE: return "SA_ERR_WORKSPACE";
+        case SA_ERR_CUDA: return "SA_ERR_CUDA";
+        case SA_ERR_DEVICE_ASSERT: return "SA_ERR_DEVICE_ASSERT";
+    }
+    return "SA_ERR_UNKNOWN";
+}
+
+int sa_check_device_status(void *stream) {
+    unsigned *ew = nullptr;
+    int rc = device_error_word(&ew);
+    if (rc) return rc;
+    cudaError_t e = cudaStreamSynchronize(as_stream(stream));
+    if (e != cudaSuccess) return fail(SA_ERR_CUDA, "cudaStreamSynchronize: %s", cudaGetErrorString(e));
+    unsigned word = 0;
+    e = cudaMemcpy(&word, ew, sizeof word, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return fail(SA_ERR_CUDA, "read error word: %s", cudaGetErrorString(e));
+    if (word) {
+        const unsigned zero = 0;
+        e = cudaMemcpy(ew, &zero, sizeof zero, cudaMemcpyHostToDevice);
+        if (e != cudaSuccess) return fail(SA_ERR_CUDA, "clear error word: %s", cudaGetErrorString(e));
+        return fail(SA_ERR_DEVICE_ASSERT, "device error word 0x%x:%s%s", word,
+                    (word & ERR_BAD_INDEX) ? " index out of range or after the query position;" : "",
+                    (word & ERR_BAD_BLOCK) ? " NSA block id outside the sequence;" : "");
+    }
+    return SA_OK;
+}
+
+// ------------------------------------------------------ sparse attention --
+size_t sa_sparse_attn_workspace_size(int B, int Tq, int Hq, int d, int n_split) {
+    if (n_split <= 1 || B <= 0 || Tq <= 0 || Hq <= 0 || d <= 0) return 0;
+    const size_t rows = (size_t)B * Tq * Hq;
+    return round_up((size_t)n_split * rows * d * 4, 256) + round_up((size_t)n_split * rows * 4, 256);
+}
+
+int sa_sparse_attn_fwd(const void *q, const void *k, const void *v, int B, int Tq, int L, int Hq,
+                       int Hkv, int d, int64_t q_pos0, const int32_t *idx, int idx_heads, int K,
+                       const sa_pattern *pattern, const float *cq, const float *ck,
+                       const float *beta, float scale, int n_split, void *out, float *lse,
+                       float *part_o, float *part_lse, void *workspace, size_t workspace_bytes,
+                       void *stream) {
+    if (B <= 0 || Tq < 0 || L <= 0 || Hq <= 0 || Hkv <= 0 || n_split < 1)
+        return fail(SA_ERR_INVALID_ARG, "sparse_attn: bad sizes B=%d Tq=%d L=%d Hq=%d Hkv=%d n_split=%d",
+                    B, Tq, L, Hq, Hkv, n_split);
+    if (Hq % Hkv) return fail(SA_ERR_INVALID_ARG, "sparse_attn: Hq %% Hkv != 0");
+    if (d != 64 && d != 128) return fail(SA_ERR_UNSUPPORTED, "sparse_attn: head dim %d", d);
+    if (q_pos0 < 0 || q_pos0 + Tq > L)
+        return fail(SA_ERR_INVALID_ARG, "sparse_attn: query positions [%lld, %lld) outside [0, L=%d)",
+                    (long long)q_pos0, (long long)q_pos0 + Tq, L);
+    if (!q || !k || !v || !aligned16(q) || !aligned16(k) || !aligned16(v))
+        return fail(SA_ERR_INVALID_ARG, "sparse_attn: q/k/v must be non-null and 16-byte aligned");
+    if (!idx && !pattern) return fail(SA_ERR_INVALID_ARG, "sparse_attn: need idx or pattern");
+    if (idx && (K < 0 || !(idx_heads == 1 || idx_heads == Hkv) || !aligned4(idx)))
+        return fail(SA_ERR_INVALID_ARG, "sparse_attn: idx_heads must be 1 or Hkv, K >= 0");
+    if (!idx && (pattern->window < 1))
+        return fail(SA_ERR_INVALID_ARG, "sparse_attn: pattern window must be >= 1");
+    const bool bias = cq || ck || beta;
+    if (bias && !(cq && ck && beta))
+        return fail(SA_ERR_INVALID_ARG, "sparse_attn: cq, ck and beta go together");
+    if (bias && (!aligned4(cq) || !aligned4(ck) || !aligned4(beta)))
+        return fail(SA_ERR_INVALID_ARG, "sparse_attn: coordinate pointers must be 4-byte aligned");
+    if (n_split == 1 && !out) return fail(SA_ERR_INVALID_ARG, "sparse_attn: out is NULL");
+    if (out && !aligned16(out)) return fail(SA_ERR_INVALID_ARG, "sparse_attn: out must be 16-byte aligned");
+    if (!std::isfinite(scale)) return fail(SA_ERR_INVALID_ARG, "sparse_attn: scale");
+    if (Tq == 0) return SA_OK;
+
+    unsigned *ew = nullptr;
+    int rc = device_error_word(&ew);
+    if (rc) return rc;
+
+    const long long rows = (long long)B * Tq * Hq;
+    float *po = part_o, *pl = part_lse;
+    if (n_split > 1 && (!po || !pl)) {
+        const size_t need = sa_sparse_attn_workspace_size(B, Tq, Hq, d, n_split);
+        if (!workspace || workspace_bytes < need)
+            return fail(SA_ERR_WORKSPACE, "sparse_attn: workspace %zu < %zu", workspace_bytes, need);
+        if (!aligned16(workspace)) return fail(SA_ERR_INVALID_ARG, "sparse_attn: workspace alignment");
+        po = static_cast<float *>(workspace);
+        pl = reinterpret_cast<float *>(static_cast<char *>(workspace) +
+                                       round_up((size_t)n_split * rows * d * 4, 256));
+    }
+    if (n_split > 1 && (!aligned16(po) || !aligned4(pl)))
+        return fail(SA_ERR_INVALID_ARG, "sparse_attn: partial buffers alignment");
+
+    GatherParams p{};
+    p.q = static_cast<const __nv_bfloat16 *>(q);
+    p.k = static_cast<const __nv_bfloat16 *>(k);
+    p.v = static_cast<const __nv_bfloat16 *>(v);
+    p.B = B; p.Tq = Tq; p.Lk = L; p.Hq = Hq; p.Hkv = Hkv; p.G = Hq / Hkv;
+    p.q_pos0 = q_pos0;
+    p.idx = idx; p.idx_heads = idx_heads; p.K = K;
+    int src;
+    if (idx) {
+        src = KS_IDX;
+        p.entries = K;
+    } else {
+        src = KS_PATTERN;
+        p.window = pattern->window;
+        p.dilated = pattern->dilated ? 1 : 0;
+        p.entries = pattern->window + (p.dilated ? 32 : 0);
+    }
+    p.n_split = n_split;
+    p.per_split = n_split > 1 ? (p.entries + n_split - 1) / n_split : p.entries;
+    p.n_hchunk = (p.G + 15) / 16;
+    p.cq = cq; p.ck = ck; p.beta = beta;
+    p.scale_log2 = scale * kLog2e;
+    p.out = static_cast<__nv_bfloat16 *>(out);
+    p.lse = lse;
+    p.part_o = po; p.part_lse = pl;
+    p.err = ew;
+    cudaStream_t st = as_stream(stream);
+    rc = launch_gather(p, d, src, bias, st);
+    if (rc) return rc;
+    if (n_split > 1 && out) return launch_combine(po, pl, n_split, rows, d, out, lse, st);
+    return SA_OK;
+}
+
+int sa_lse_combine(const float *part_o, const float *part_lse, int n_split, int64_t rows, int d,
+                   void *out, float *lse, void *stream) {
+    if (n_split < 1 || rows < 0) return fail(SA_ERR_INVALID_ARG, "lse_combine: n_split=%d rows=%lld", n_split, (long long)rows);
+    if (d != 64 && d != 128) return fail(SA_ERR_UNSUPPORTED, "lse_combine: head dim %d", d);
+    if (!part_o || !part_lse || !out || !aligned16(part_o) || !aligned4(part_lse) || !aligned16(out))
+        return fail(SA_ERR_INVALID_ARG, "lse_combine: null or misaligned pointer");
+    if (lse && !aligned4(lse)) return fail(SA_ERR_INVALID_ARG, "lse_combine: lse alignment");
+    return launch_combine(part_o, part_lse, n_split, rows, d, out, lse, as_stream(stream));
+}
+
+// ------------------------------------------------------------- indexer --
+// Query rows per score chunk: the chunk's int32 scores stay within ~64 MiB so
+// that the select pass re-reads them from L2.
+static int indexer_chunk_rows(int B, int Tq, size_t ld, int Hi) {
+    const size_t budget = (size_t)64 << 20;
+    const int qt = 128 / Hi;
+    size_t rows = budget / ((size_t)B * ld * 4);
+    if (rows < 1) rows = 1;
+    if (rows >= (size_t)qt) rows = rows / qt * qt;
+    if (rows > (size_t)Tq) rows = Tq;
+    if (rows > 65535) rows = 65535;   // grid.y limit of the select launch
+    return (int)rows;
+}
+
+static size_t indexer_ld(int Tq, int L, int64_t q_pos0, int window) {
+    long long pmax = q_pos0 + Tq - 1;
+    long long n = window > 0 ? pmax - window + 1 : pmax + 1;
+    if (n < 1) n = 1;
+    if (n > L) n = L;
+    return round_up((size_t)n, 4);
+}
+
+static bool indexer_shape_ok(int Hi, int di) {
+    return (Hi == 1 || Hi == 2 || Hi == 4 || Hi == 8 || Hi == 16) && (di == 32 || di == 64 || di == 128);
+}
+
+size_t sa_indexer_topk_workspace_size(int B, int Tq, int L, int Hi, int di, int topk, int window) {
+    (void)di; (void)topk;
+    if (B <= 0 || Tq <= 0 || L <= 0 || !(Hi == 1 || Hi == 2 || Hi == 4 || Hi == 8 || Hi == 16)) return 0;
+    // the worst case over q_pos0 is q_pos0 = L - Tq
+    const size_t ld = indexer_ld(Tq, L, L - Tq, window);
+    const int rt = indexer_chunk_rows(B, Tq, ld, Hi);
+    return round_up((size_t)B * rt * ld * 4, 256);
+}
+
+template <int HI, int DI>
+static int launch_score_t(const IdxScoreParams &p, int ncand_max, cudaStream_t st) {
+    constexpr int QT = 128 / HI;
+    const int smem = QT * 128 * 4 + QT * HI * 4;
+    auto kern = idx_score_kernel<HI, DI>;
+    int rc = set_smem(kern, smem);
+    if (rc) return rc;
+    dim3 grid((unsigned)((ncand_max + 127) / 128), (unsigned)((p.Rt + QT - 1) / QT), (unsigned)p.B);
+    kern<<<grid, 128, smem, st>>>(p);
+    SA_CHECK_LAUNCH("idx_score_kernel");
+    return SA_OK;
+}
+
+template <int HI>
+static int launch_score_hi(const IdxScoreParams &p, int di, int ncand_max, cudaStream_t st) {
+    if (di == 32) return launch_score_t<HI, 32>(p, ncand_max, st);
+    if (di == 64) return launch_score_t<HI, 64>(p, ncand_max, st);
+    return launch_score_t<HI, 128>(p, ncand_max, st);
+}
+
+static int launch_score(const IdxScoreParams &p, int Hi, int di, int ncand_max, cudaStream_t st) {
+    switch (Hi) {
+        case 1: return launch_score_hi<1>(p, di, ncand_max, st);
+        case 2: return launch_score_hi<2>(p, di, ncand_max, st);
+        case 4: return launch_score_hi<4>(p, di, ncand_max, st);
+        case 8: return launch_score_hi<8>(p, di, ncand_max, st);
+        case 16: return launch_score_hi<16>(p, di, ncand_max, st);
+    }
+    return fail(SA_ERR_UNSUPPORTED, "indexer heads %d", Hi);
+}
+
+static int launch_select(const SelectParams &p, int cluster, cudaStream_t st) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)cluster, (unsigned)p.Rt, (unsigned)p.B);
+    cfg.blockDim = dim3(SEL_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)cluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, topk_select_kernel, p);
+    if (e != cudaSuccess) return fail(SA_ERR_CUDA, "topk_select_kernel: %s", cudaGetErrorString(e));
+    SA_CHECK_LAUNCH("topk_select_kernel");
+    return SA_OK;
+}
+
+int sa_indexer_topk(const int8_t *q_idx, const int8_t *k_idx, const int32_t *w, int B, int Tq, int L,
+                    int Hi, int di, int64_t q_pos0, int topk, int window, int32_t *out_idx,
+                    int32_t *out_count, void *workspace, size_t workspace_bytes, void *stream) {
+    if (B <= 0 || Tq < 0 || L <= 0 || topk < 0 || window < 0 || topk + window < 1)
+        return fail(SA_ERR_INVALID_ARG, "indexer_topk: bad sizes B=%d Tq=%d L=%d topk=%d window=%d", B, Tq,
+                    L, topk, window);
+    if (!indexer_shape_ok(Hi, di))
+        return fail(SA_ERR_UNSUPPORTED, "indexer_topk: Hi=%d di=%d (Hi in 1,2,4,8,16; di in 32,64,128)", Hi, di);
+    if (q_pos0 < 0 || q_pos0 + Tq > L)
+        return fail(SA_ERR_INVALID_ARG, "indexer_topk: query positions [%lld, %lld) outside [0, L=%d)",
+                    (long long)q_pos0, (long long)q_pos0 + Tq, L);
+    if (!q_idx || !k_idx || !w || !out_idx || !aligned16(q_idx) || !aligned16(k_idx) || !aligned4(w) ||
+        !aligned4(out_idx) || (out_count && !aligned4(out_count)))
+        return fail(SA_ERR_INVALID_ARG, "indexer_topk: null or misaligned pointer");
+    if (Tq == 0) return SA_OK;
+    // chunking is fixed by the worst case (q_pos0 = L - Tq), as in the size query
+    const size_t ld = indexer_ld(Tq, L, q_pos0, window);
+    const int rt = indexer_chunk_rows(B, Tq, indexer_ld(Tq, L, L - Tq, window), Hi);
+    const size_t need = round_up((size_t)B * rt * ld * 4, 256);
+    if (!workspace || workspace_bytes < need)
+        return fail(SA_ERR_WORKSPACE, "indexer_topk: workspace %zu < %zu", workspace_bytes, need);
+    if (!aligned16(workspace)) return fail(SA_ERR_INVALID_ARG, "indexer_topk: workspace alignment");
+    cudaStream_t st = as_stream(stream);
+    int32_t *scores = static_cast<int32_t *>(workspace);
+    const int Kout = topk + window;
+    for (int t0 = 0; t0 < Tq; t0 += rt) {
+        const int rows = std::min(rt, Tq - t0);
+        long long pmax = q_pos0 + t0 + rows - 1;
+        long long ncand = window > 0 ? pmax - window + 1 : pmax + 1;
+        if (ncand > 0) {
+            IdxScoreParams sp{};
+            sp.q = q_idx; sp.k = k_idx; sp.w = w;
+            sp.B = B; sp.Tq = Tq; sp.L = L; sp.q_pos0 = q_pos0; sp.window = window;
+            sp.t0 = t0; sp.Rt = rows; sp.ld = (long long)ld; sp.scores = scores;
+            int rc = launch_score(sp, Hi, di, (int)ncand, st);
+            if (rc) return rc;
+        }
+        SelectParams se{};
+        se.scores = scores; se.ld = (long long)ld;
+        se.B = B; se.Tq = Tq; se.t0 = t0; se.Rt = rows; se.q_pos0 = q_pos0;
+        se.topk = topk; se.window = window; se.Kout = Kout;
+        se.out_idx = out_idx; se.out_count = out_count;
+        // enough CTAs to fill the GPU: split short row lists across a cluster
+        const long long nrow = (long long)B * rows;
+        int cluster = 1;
+        while (cluster < 8 && nrow * cluster < 296 && (long long)ncand / (cluster * 2) >= 4096) cluster *= 2;
+        int rc = launch_select(se, cluster, st);
+        if (rc) return rc;
+    }
+    return SA_OK;
+}
+
+// ----------------------------------------------------------------- NSA --
+struct NsaLayout {
+    int nc, n_blocks;
+    size_t kc_off, klo_off, vc_off, o3_off, l3_off, sel_off, total;
+};
+
+static NsaLayout nsa_layout(int B, int T, int Hq, int Hkv, int d, int cmp_len, int cmp_stride,
+                            int sel_block, int sel_topk) {
+    NsaLayout lay{};
+    lay.nc = T >= cmp_len ? (T - cmp_len) / cmp_stride + 1 : 0;
+    lay.n_blocks = (T + sel_block - 1) / sel_block;
+    const size_t rows = (size_t)B * T * Hq;
+    size_t off = 0;
+    lay.kc_off = off; off += round_up((size_t)B * std::max(lay.nc, 1) * Hkv * d * 2, 256);
+    lay.klo_off = off; off += round_up((size_t)B * std::max(lay.nc, 1) * Hkv * d * 2, 256);
+    lay.vc_off = off; off += round_up((size_t)B * std::max(lay.nc, 1) * Hkv * d * 2, 256);
+    lay.o3_off = off; off += round_up(3 * rows * d * 4, 256);
+    lay.l3_off = off; off += round_up(3 * rows * 4, 256);
+    lay.sel_off = off; off += round_up((size_t)B * T * Hkv * sel_topk * 4, 256);
+    lay.total = off;
+    return lay;
+}
+
+size_t sa_nsa_workspace_size(int B, int T, int Hq, int Hkv, int d, int cmp_len, int cmp_stride,
+                             int sel_block, int sel_topk) {
+    if (B <= 0 || T <= 0 || Hq <= 0 || Hkv <= 0 || d <= 0 || cmp_len <= 0 || cmp_stride <= 0 ||
+        sel_block <= 0 || sel_topk <= 0)
+        return 0;
+    return nsa_layout(B, T, Hq, Hkv, d, cmp_len, cmp_stride, sel_block, sel_topk).total;
+}
+
+template <int D>
+static int launch_nsa_select(const NsaSelectParams &p, cudaStream_t st) {
+    const int wbytes = 2 * 2 * 32 * D * 2 + 32 * 4 + p.n_blocks * 4;
+    const int smem = 4 * ((wbytes + 127) / 128 * 128);
+    if (smem > 227 * 1024) return fail(SA_ERR_UNSUPPORTED, "nsa: %d selection blocks exceed shared memory", p.n_blocks);
+    auto kern = nsa_select_kernel<D>;
+    int rc = set_smem(kern, smem);
+    if (rc) return rc;
+    const long long items = (long long)p.B * p.T * p.Hkv;
+    kern<<<(unsigned)((items + 3) / 4), 128, smem, st>>>(p);
+    SA_CHECK_LAUNCH("nsa_select_kernel");
+    return SA_OK;
+}
+
+int sa_nsa_fwd(const void *q, const void *k, const void *v, const float *gates, int B, int T, int Hq,
+               int Hkv, int d, int cmp_len, int cmp_stride, int sel_block, int sel_topk, int window,
+               float scale, void *out, float *lse_branches, int32_t *sel_idx_out, void *workspace,
+               size_t workspace_bytes, void *stream) {
+    if (B <= 0 || T < 0 || Hq <= 0 || Hkv <= 0 || cmp_len <= 0 || cmp_stride <= 0 || sel_block <= 0 ||
+        sel_topk <= 0 || window <= 0)
+        return fail(SA_ERR_INVALID_ARG, "nsa: bad sizes");
+    if (Hq % Hkv) return fail(SA_ERR_INVALID_ARG, "nsa: Hq %% Hkv != 0");
+    if (Hq / Hkv > 16) return fail(SA_ERR_UNSUPPORTED, "nsa: more than 16 query heads per KV head");
+    if (d != 64 && d != 128) return fail(SA_ERR_UNSUPPORTED, "nsa: head dim %d", d);
+    if (sel_block % cmp_stride || sel_topk > 32)
+        return fail(SA_ERR_UNSUPPORTED, "nsa: need cmp_stride | sel_block and sel_topk <= 32");
+    if (!q || !k || !v || !gates || !out || !aligned16(q) || !aligned16(k) || !aligned16(v) ||
+        !aligned4(gates) || !aligned16(out))
+        return fail(SA_ERR_INVALID_ARG, "nsa: null or misaligned pointer");
+    if (!std::isfinite(scale)) return fail(SA_ERR_INVALID_ARG, "nsa: scale");
+    if (T == 0) return SA_OK;
+    const NsaLayout lay = nsa_layout(B, T, Hq, Hkv, d, cmp_len, cmp_stride, sel_block, sel_topk);
+    if (!workspace || workspace_bytes < lay.total)
+        return fail(SA_ERR_WORKSPACE, "nsa: workspace %zu < %zu", workspace_bytes, lay.total);
+    if (!aligned16(workspace)) return fail(SA_ERR_INVALID_ARG, "nsa: workspace alignment");
+    unsigned *ew = nullptr;
+    int rc = device_error_word(&ew);
+    if (rc) return rc;
+    cudaStream_t st = as_stream(stream);
+    char *ws = static_cast<char *>(workspace);
+    __nv_bfloat16 *kc = reinterpret_cast<__nv_bfloat16 *>(ws + lay.kc_off);
+    __nv_bfloat16 *vc = reinterpret_cast<__nv_bfloat16 *>(ws + lay.vc_off);
+    __nv_bfloat16 *klo = reinterpret_cast<__nv_bfloat16 *>(ws + lay.klo_off);
+    float *o3 = reinterpret_cast<float *>(ws + lay.o3_off);
+    float *l3 = reinterpret_cast<float *>(ws + lay.l3_off);
+    int32_t *sel = sel_idx_out ? sel_idx_out : reinterpret_cast<int32_t *>(ws + lay.sel_off);
+    const long long rows = (long long)B * T * Hq;
+    const int G = Hq / Hkv;
+
+    // 1. compression
+    if (lay.nc > 0) {
+        const long long n2 = (long long)B * lay.nc * Hkv * (d / 2);
+        nsa_compress_kernel<<<(unsigned)((n2 + 255) / 256), 256, 0, st>>>(
+            (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, B, T, Hkv, d, lay.nc, cmp_len, cmp_stride,
+            kc, klo, vc);
+        SA_CHECK_LAUNCH("nsa_compress_kernel");
+    }
+    GatherParams base{};
+    base.q = static_cast<const __nv_bfloat16 *>(q);
+    base.B = B; base.Tq = T; base.Hq = Hq; base.Hkv = Hkv; base.G = G;
+    base.q_pos0 = 0; base.n_split = 1; base.n_hchunk = 1;
+    base.scale_log2 = scale * kLog2e;
+    base.err = ew;
+    // 2. compressed branch -> o3[0], l3[0]
+    {
+        GatherParams p = base;
+        p.k = kc; p.klo = klo; p.v = vc; p.Lk = std::max(lay.nc, 1);
+        p.block = cmp_stride; p.cmp_len = cmp_len;
+        p.entries = lay.nc; p.per_split = lay.nc;
+        p.out_f32 = o3; p.lse = l3;
+        rc = launch_gather(p, d, KS_CMP, false, st);   // nc == 0: zero rows, lse = -inf
+        if (rc) return rc;
+    }
+    // 3. importance + block top-k
+    {
+        NsaSelectParams sp{};
+        sp.q = base.q; sp.kc = kc; sp.klo = klo; sp.lse_cmp = l3;
+        sp.B = B; sp.T = T; sp.Hq = Hq; sp.Hkv = Hkv; sp.G = G; sp.nc = lay.nc;
+        sp.cmp_len = cmp_len; sp.cmp_stride = cmp_stride; sp.sel_block = sel_block;
+        sp.sel_topk = sel_topk; sp.n_blocks = lay.n_blocks;
+        sp.scale_log2 = base.scale_log2;
+        sp.sel_idx = sel; sp.imp_out = nullptr;
+        rc = d == 64 ? launch_nsa_select<64>(sp, st) : launch_nsa_select<128>(sp, st);
+        if (rc) return rc;
+    }
+    // 4. selected branch -> o3[1], l3[1]
+    {
+        GatherParams p = base;
+        p.k = static_cast<const __nv_bfloat16 *>(k); p.v = static_cast<const __nv_bfloat16 *>(v);
+        p.Lk = T; p.idx = sel; p.K = sel_topk; p.block = sel_block;
+        p.entries = sel_topk * sel_block; p.per_split = p.entries;
+        p.out_f32 = o3 + rows * d; p.lse = l3 + rows;
+        rc = launch_gather(p, d, KS_BLOCKS, false, st);
+        if (rc) return rc;
+    }
+    // 5. window branch -> o3[2], l3[2]
+    {
+        GatherParams p = base;
+        p.k = static_cast<const __nv_bfloat16 *>(k); p.v = static_cast<const __nv_bfloat16 *>(v);
+        p.Lk = T; p.window = window; p.entries = window; p.per_split = window;
+        p.out_f32 = o3 + 2 * rows * d; p.lse = l3 + 2 * rows;
+        rc = launch_gather(p, d, KS_RANGE, false, st);
+        if (rc) return rc;
+    }
+    // 6. gated sum
+    {
+        const long long n2 = rows * (d / 2);
+        nsa_gate_kernel<<<(unsigned)((n2 + 255) / 256), 256, 0, st>>>(o3, rows * d, gates, rows, d,
+                                                                       (__nv_bfloat16 *)out);
+        SA_CHECK_LAUNCH("nsa_gate_kernel");
+        if (lse_branches) {
+            nsa_lse_pack_kernel<<<(unsigned)((rows + 255) / 256), 256, 0, st>>>(l3, rows, lse_branches);
+            SA_CHECK_LAUNCH("nsa_lse_pack_kernel");
+        }
+    }
+    return SA_OK;
+}
+
+// ------------------------------------------------------ IndexCache driver --
+size_t sa_dsa_decode_layers_workspace_size(int B, int Tq, int L, int Hq, int d, int Hi, int di,
+                                           int topk, int window, int n_split) {
+    const size_t a = sa_indexer_topk_workspace_size(B, Tq, L, Hi, di, topk, window);
+    const size_t b = sa_sparse_attn_workspace_size(B, Tq, Hq, d, n_split);
+    const size_t idx = round_up((size_t)B * Tq * (topk + window) * 4, 256);
+    return round_up(std::max(a, b), 256) + idx;
+}
+
+int sa_dsa_decode_layers(const char *pattern, int n_layers, const sa_dsa_layer *layers, int B, int Tq,
+                         int L, int Hq, int Hkv, int d, int Hi, int di, int64_t q_pos0, int topk,
+                         int window, float scale, int n_split, int32_t *idx_cache, void *workspace,
+                         size_t workspace_bytes, void *stream) {
+    if (!pattern || !layers || n_layers <= 0 || (int)strlen(pattern) < n_layers)
+        return fail(SA_ERR_INVALID_ARG, "dsa_layers: pattern/layers");
+    if (pattern[0] != 'F') return fail(SA_ERR_INVALID_ARG, "dsa_layers: the first layer must be 'F'");
+    for (int i = 0; i < n_layers; ++i)
+        if (pattern[i] != 'F' && pattern[i] != 'S')
+            return fail(SA_ERR_INVALID_ARG, "dsa_layers: pattern char %d is '%c'", i, pattern[i]);
+    const size_t need = sa_dsa_decode_layers_workspace_size(B, Tq, L, Hq, d, Hi, di, topk, window, n_split);
+    if (!workspace || workspace_bytes < need)
+        return fail(SA_ERR_WORKSPACE, "dsa_layers: workspace %zu < %zu", workspace_bytes, need);
+    if (!aligned16(workspace)) return fail(SA_ERR_INVALID_ARG, "dsa_layers: workspace alignment");
+    const size_t a = sa_indexer_topk_workspace_size(B, Tq, L, Hi, di, topk, window);
+    const size_t b = sa_sparse_attn_workspace_size(B, Tq, Hq, d, n_split);
+    const size_t scratch = round_up(std::max(a, b), 256);
+    int32_t *cache = idx_cache ? idx_cache : reinterpret_cast<int32_t *>(static_cast<char *>(workspace) + scratch);
+    const int K = topk + window;
+    for (int i = 0; i < n_layers; ++i) {
+        const sa_dsa_layer &ly = layers[i];
+        if (pattern[i] == 'F') {
+            int rc = sa_indexer_topk(ly.q_idx, ly.k_idx, ly.w, B, Tq, L, Hi, di, q_pos0, topk, window, cache,
+                                     nullptr, workspace, scratch, stream);
+            if (rc) return rc;
+        }
+        int rc = sa_sparse_attn_fwd(ly.q, ly.k, ly.v, B, Tq, L, Hq, Hkv, d, q_pos0, cache, 1, K, nullptr,
+                                    nullptr, nullptr, nullptr, scale, n_split, ly.out, ly.lse, nullptr, nullptr,
+                                    workspace, scratch, stream);
+        if (rc) return rc;
+    }
+    return SA_OK;
+}
+

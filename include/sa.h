@@ -1,0 +1,222 @@
+/*
+ * sa.h -- C ABI of the B200 (sm_100a) causal sparse-attention library
+ * (libsa.so).
+ *
+ * Every query attends to its own set of earlier positions.  The set is chosen
+ * by a lightweight indexer's top-k (DeepSeek-style sparse attention, with
+ * IndexCache reuse across layers), fixed in advance (a recent window plus
+ * dilated distances 1, 2, 4, 8, ...), or built from NSA's compressed,
+ * selected and window branches.  Partial results merge by a log-sum-exp
+ * softmax combine.
+ *
+ * Conventions shared by every call
+ *  - Tensor pointers are DEVICE pointers owned by the caller; the library
+ *    never allocates or frees memory.  Scratch memory is the caller's
+ *    `workspace`, sized by the matching *_workspace_size() query.
+ *  - Tensors are dense and row-major in the layouts written beside each
+ *    argument (last dimension contiguous).  bf16 is IEEE bfloat16.
+ *    Pointers to bf16/fp32 tensors must be 16-byte aligned.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Calls are asynchronous: they enqueue kernels and return.
+ *  - Query head h reads KV head h / (Hq / Hkv).  Softmax scale `scale`
+ *    multiplies q.k before any bias; pass 1/sqrt(d) for the usual scaling.
+ *  - LSE outputs are natural-log log-sum-exp of the scaled (and biased)
+ *    logits, fp32; an empty set gives lse = -inf and a zero output row.
+ *  - Return value: SA_OK or an sa_status code.  Host-side checks (null or
+ *    misaligned pointers, sizes, unsupported shapes, small workspace) fail
+ *    before anything is enqueued.  Device-side problems found while running
+ *    (an index past the query position or outside [0, L)) skip the offending
+ *    entry and raise a bit in the library's device error word, reported by
+ *    sa_check_device_status().
+ *  - Supported on this build: head dim d in {64, 128}; Hq/Hkv in
+ *    {1, 2, 4, 8, 16}; indexer heads Hi in {1, 2, 4, 8, 16} with indexer
+ *    dim di in {32, 64, 128}; sm_100a only.  Anything else returns
+ *    SA_ERR_UNSUPPORTED; there is no CPU fallback.
+ */
+#ifndef SA_H_
+#define SA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum sa_status {
+    SA_OK = 0,
+    SA_ERR_INVALID_ARG = 1,    /* null/misaligned pointer, inconsistent sizes */
+    SA_ERR_UNSUPPORTED = 2,    /* shape or option outside what is built */
+    SA_ERR_WORKSPACE = 3,      /* workspace smaller than *_workspace_size() */
+    SA_ERR_CUDA = 4,           /* CUDA launch/runtime error (see sa_last_error_string) */
+    SA_ERR_DEVICE_ASSERT = 5   /* device error word was set (bad index found on device) */
+};
+
+/* Fixed index set, generated inside the kernel (no index tensor).
+ * SpatialLM page ("SpatialLM-Mini acelero el entrenamiento ...", section "Como
+ * eligen los tokens a quien escuchar"): the token itself, its nearest
+ * predecessors and the positions at distances 1, 2, 4, 8, ...; never a future
+ * position.  For query position p:
+ *   S_p = { p - o : 0 <= o < window, p - o >= 0 }
+ *       u { p - 2^i : 2^i < p }            (only when dilated != 0)
+ * `window` counts the token itself (self + 64 predecessors = 65). */
+typedef struct sa_pattern {
+    int32_t window;
+    int32_t dilated;
+} sa_pattern;
+
+/* --------------------------------------------------------------------------
+ * Indexer scores and causal top-k.
+ * IndexCache page ("IndexCache: inferencia 82% mas rapida ...", body): a
+ * lightweight indexer scores every earlier token and the query keeps a small
+ * top-scoring subset.  HySparse2 page ("Xiaomi presenta HySparse2 ...",
+ * section "Mas precision con menos memoria"): the most recent tokens are
+ * forced into the set.  Score of query t (position p = q_pos0 + t) for key j:
+ *   I(t, j) = sum_h w[t,h] * max(0, sum_c q_idx[t,h,c] * k_idx[j,c])
+ * computed exactly in int32 (the caller keeps |I| < 2^31).
+ * Forced window W = {max(0, p-window+1) .. p} (empty when window == 0); the
+ * other candidates {0 .. p} \ W are ranked by (I desc, j asc) and the first
+ * min(topk, count) are kept.
+ *   q_idx  int8  [B, Tq, Hi, di]       k_idx int8 [B, L, di]
+ *   w      int32 [B, Tq, Hi]
+ *   out_idx   int32 [B, Tq, topk+window]  ascending positions, -1 padded
+ *   out_count int32 [B, Tq] (nullable)    number of valid entries
+ * Requires 0 <= q_pos0 and q_pos0 + Tq - 1 < L (every query has its key).
+ * Selected positions are bit-exact: the selected set is unique under the
+ * tie rule and is written in ascending order.
+ * ------------------------------------------------------------------------ */
+size_t sa_indexer_topk_workspace_size(int B, int Tq, int L, int Hi, int di,
+                                      int topk, int window);
+int sa_indexer_topk(const int8_t *q_idx, const int8_t *k_idx, const int32_t *w,
+                    int B, int Tq, int L, int Hi, int di, int64_t q_pos0,
+                    int topk, int window,
+                    int32_t *out_idx, int32_t *out_count,
+                    void *workspace, size_t workspace_bytes, void *stream);
+
+/* --------------------------------------------------------------------------
+ * Gathered-KV sparse attention forward.
+ * For each query t (position p = q_pos0 + t) and head h over its index set S:
+ *   z_j = scale * (q[t,h] . k[j,g]) + bias(t, j, h),  j in S
+ *   out[t,h] = sum_j softmax(z)_j v[j,g],   lse[t,h] = log sum_j exp z_j
+ * The set comes from `idx` or, when idx == NULL, from `pattern`.
+ *   q   bf16 [B, Tq, Hq, d]          k, v  bf16 [B, L, Hkv, d]
+ *   idx int32 [B, Tq, idx_heads, K]  -1 = padding; entries must lie in
+ *       [0, min(p, L-1)]; idx_heads is 1 (one list shared by every head) or
+ *       Hkv (one list per KV head).  Any order; a repeated entry counts twice.
+ *   Optional coordinate bias (SpatialLM page, same section: learnable 3-D
+ *   query/key coordinates, a smaller distance giving a larger weight):
+ *       bias = -beta[h] * ||cq[t,h,:] - ck[j,g,:]||^2,
+ *   cq fp32 [B, Tq, Hq, 3], ck fp32 [B, L, Hkv, 3], beta fp32 [Hq]; all three
+ *   NULL for no bias.
+ * n_split = 1: out bf16 [B,Tq,Hq,d] and lse fp32 [B,Tq,Hq] (nullable).
+ * n_split > 1 (split-KV; idx mode only): the K entries are cut into n_split
+ *   contiguous pieces of ceil(K/n_split); piece s writes part_o fp32
+ *   [n_split,B,Tq,Hq,d] and part_lse fp32 [n_split,B,Tq,Hq]; when `out` is
+ *   non-NULL the pieces are then merged by sa_lse_combine into out/lse.
+ *   part_o/part_lse may be NULL, in which case they live in `workspace`.
+ * Star Attention page ("NVIDIA AI Research presenta Star Attention ...",
+ * body) merges per-block results by a distributed softmax: that is the
+ * split-KV mode.
+ * ------------------------------------------------------------------------ */
+size_t sa_sparse_attn_workspace_size(int B, int Tq, int Hq, int d, int n_split);
+int sa_sparse_attn_fwd(const void *q, const void *k, const void *v,
+                       int B, int Tq, int L, int Hq, int Hkv, int d, int64_t q_pos0,
+                       const int32_t *idx, int idx_heads, int K,
+                       const sa_pattern *pattern,
+                       const float *cq, const float *ck, const float *beta,
+                       float scale, int n_split,
+                       void *out, float *lse,
+                       float *part_o, float *part_lse,
+                       void *workspace, size_t workspace_bytes, void *stream);
+
+/* --------------------------------------------------------------------------
+ * Log-sum-exp combine (Star Attention page, body: distributed softmax).
+ *   lse = log sum_s exp(part_lse[s]),  out = sum_s exp(part_lse[s] - lse) part_o[s]
+ * A piece with part_lse = -inf contributes nothing; all empty -> out = 0,
+ * lse = -inf.
+ *   part_o fp32 [n_split, rows, d], part_lse fp32 [n_split, rows]
+ *   out bf16 [rows, d], lse fp32 [rows] (nullable)
+ * ------------------------------------------------------------------------ */
+int sa_lse_combine(const float *part_o, const float *part_lse, int n_split,
+                   int64_t rows, int d, void *out, float *lse, void *stream);
+
+/* --------------------------------------------------------------------------
+ * NSA forward (Native Sparse Attention page, "Puntos Clave" and "Analisis
+ * Profundo"): coarse compression, fine blockwise selection, sliding window.
+ *  1. Kc[i] = mean(k[i*cmp_stride .. i*cmp_stride + cmp_len - 1]) per KV
+ *     head (likewise Vc), i = 0 .. (T - cmp_len) / cmp_stride.
+ *  2. Compressed branch: query t attends to Kc[i] with i*cmp_stride +
+ *     cmp_len - 1 <= t.
+ *  3. Importance of selection block b for KV group g: the compressed-branch
+ *     probabilities of tokens i with i*cmp_stride in [b*sel_block,
+ *     (b+1)*sel_block), summed over those i and over the heads of the group.
+ *  4. Per (t, g): the sel_topk blocks with b*sel_block <= t of largest
+ *     importance (ties -> lower b; fewer candidates -> all).
+ *  5. Selected branch: keys of those blocks, masked to j <= t.
+ *  6. Window branch: keys max(0, t-window+1) .. t.
+ *  7. out = gates[...,0]*o_cmp + gates[...,1]*o_slc + gates[...,2]*o_win.
+ *   q bf16 [B,T,Hq,d], k/v bf16 [B,T,Hkv,d], gates fp32 [B,T,Hq,3]
+ *   out bf16 [B,T,Hq,d]; lse_branches fp32 [B,T,Hq,3] (nullable);
+ *   sel_idx_out int32 [B,T,Hkv,sel_topk] ascending, -1 padded (nullable).
+ * Requires cmp_stride divides sel_block, cmp_len a multiple of cmp_stride,
+ * Hq/Hkv == 16, and sel_topk <= 32.
+ * ------------------------------------------------------------------------ */
+size_t sa_nsa_workspace_size(int B, int T, int Hq, int Hkv, int d, int cmp_len,
+                             int cmp_stride, int sel_block, int sel_topk);
+int sa_nsa_fwd(const void *q, const void *k, const void *v, const float *gates,
+               int B, int T, int Hq, int Hkv, int d,
+               int cmp_len, int cmp_stride, int sel_block, int sel_topk, int window,
+               float scale, void *out, float *lse_branches, int32_t *sel_idx_out,
+               void *workspace, size_t workspace_bytes, void *stream);
+
+/* --------------------------------------------------------------------------
+ * IndexCache layer driver (IndexCache page, body): layers marked 'F' run the
+ * indexer and top-k and overwrite the cached index buffer; layers marked 'S'
+ * skip the indexer and reuse the buffer of the nearest preceding F layer.
+ * pattern[0] must be 'F'.  Every layer then runs sa_sparse_attn_fwd with the
+ * cached indices (split-KV with n_split pieces when n_split > 1).  Works for
+ * decode (Tq = 1, q_pos0 = L - 1) and prefill alike.
+ * ------------------------------------------------------------------------ */
+typedef struct sa_dsa_layer {
+    const void *q;          /* bf16 [B, Tq, Hq, d] */
+    const void *k;          /* bf16 [B, L, Hkv, d] */
+    const void *v;          /* bf16 [B, L, Hkv, d] */
+    const int8_t *q_idx;    /* int8 [B, Tq, Hi, di]  (read on F layers) */
+    const int8_t *k_idx;    /* int8 [B, L, di]       (read on F layers) */
+    const int32_t *w;       /* int32 [B, Tq, Hi]     (read on F layers) */
+    void *out;              /* bf16 [B, Tq, Hq, d] */
+    float *lse;             /* fp32 [B, Tq, Hq] or NULL */
+} sa_dsa_layer;
+
+size_t sa_dsa_decode_layers_workspace_size(int B, int Tq, int L, int Hq, int d,
+                                           int Hi, int di, int topk, int window,
+                                           int n_split);
+int sa_dsa_decode_layers(const char *pattern, int n_layers, const sa_dsa_layer *layers,
+                         int B, int Tq, int L, int Hq, int Hkv, int d, int Hi, int di,
+                         int64_t q_pos0, int topk, int window, float scale, int n_split,
+                         int32_t *idx_cache, void *workspace, size_t workspace_bytes,
+                         void *stream);
+
+/* --------------------------------------------------------------------------
+ * Status helpers.
+ * sa_check_device_status: waits for `stream`, reads and clears the device
+ *   error word of the current device; returns SA_ERR_DEVICE_ASSERT if any
+ *   kernel since the last check found a bad index, else SA_OK (or SA_ERR_CUDA).
+ * sa_last_error_string: message of the last failing call on this host thread.
+ * sa_status_string: fixed name of a status code.
+ * sa_version: library ABI version (major*100 + minor).
+ * sa_launch_counter: number of kernels this process has enqueued through the
+ *   library so far (all devices, all threads); differences around a region
+ *   count the library's launches inside it.
+ * ------------------------------------------------------------------------ */
+int sa_check_device_status(void *stream);
+const char *sa_last_error_string(void);
+const char *sa_status_string(int status);
+int sa_version(void);
+uint64_t sa_launch_counter(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SA_H_ */

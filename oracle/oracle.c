@@ -445,14 +445,15 @@ int oracle_nsa_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v,
     int status = OR_OK;
 #pragma omp parallel
     {
-        int64_t nmax = (nc > T ? nc : T);
-        if (sel_topk * sel_block > nmax) nmax = sel_topk * sel_block;
-        nmax += 1;
+        /* key buffers: the selected branch holds at most sel_topk*sel_block
+           rows, the window branch at most `window`, the compressed branch nc */
+        int64_t nbuf = sel_topk * sel_block > window ? sel_topk * sel_block : window;
+        int64_t nmax = (nc > nbuf ? nc : nbuf) + 1;
         double *z = (double *)malloc(sizeof(double) * (size_t)nmax);
         const double **kr = (const double **)malloc(sizeof(double *) * (size_t)nmax);
         const double **vr = (const double **)malloc(sizeof(double *) * (size_t)nmax);
-        double *kbuf = (double *)malloc(sizeof(double) * (size_t)(nmax * d));
-        double *vbuf = (double *)malloc(sizeof(double) * (size_t)(nmax * d));
+        double *kbuf = (double *)malloc(sizeof(double) * (size_t)((nbuf + 1) * d));
+        double *vbuf = (double *)malloc(sizeof(double) * (size_t)((nbuf + 1) * d));
         double *qv = (double *)malloc(sizeof(double) * (size_t)d);
         double *ob = (double *)malloc(sizeof(double) * (size_t)(3 * Hq * d));
         double *lb = (double *)malloc(sizeof(double) * (size_t)(3 * Hq));

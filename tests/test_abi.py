@@ -1,0 +1,89 @@
+"""CPU checks of the C-ABI boundary: libsa.so loads, exports every symbol
+declared in include/sa.h, and rejects bad arguments on the host before any
+device work (no compute call is made here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from fixed_pattern_sparse_sa_b200 import _lib, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _lib.load()
+
+
+def _header_functions():
+    src = open(os.path.join(ROOT, "include", "sa.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(sa_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_and_binding_agree():
+    assert _header_functions() == sorted(_lib.EXPORTS)
+
+
+def test_every_header_symbol_is_exported(lib):
+    for name in _header_functions():
+        assert hasattr(lib, name), name
+
+
+def test_version_and_status_strings(lib):
+    assert lib.sa_version() == 100
+    assert lib.sa_status_string(0) == b"SA_OK"
+    assert lib.sa_status_string(5) == b"SA_ERR_DEVICE_ASSERT"
+    assert lib.sa_status_string(99) == b"SA_ERR_UNKNOWN"
+
+
+def test_workspace_queries(lib):
+    # indexer scratch: B * rows-per-chunk * row-length int32 scores, rounded
+    n = lib.sa_indexer_topk_workspace_size(1, 512, 512, 2, 32, 64, 32)
+    assert n > 0 and n % 256 == 0
+    assert lib.sa_sparse_attn_workspace_size(2, 3, 4, 64, 1) == 0
+    assert lib.sa_sparse_attn_workspace_size(2, 3, 4, 64, 4) == 4 * 24 * 64 * 4 + 512   # partials + lse (384 B rounded to 256)
+    assert lib.sa_nsa_workspace_size(1, 1024, 16, 1, 64, 32, 16, 64, 16) > 0
+    assert lib.sa_indexer_topk_workspace_size(0, 1, 1, 2, 32, 1, 0) == 0
+
+
+def test_host_validation_rejects_bad_arguments(lib):
+    fake = ctypes.c_void_p(1 << 20)          # never dereferenced: rejected first
+    # n_split < 1
+    assert lib.sa_lse_combine(fake, fake, 0, 4, 64, fake, None, None) == 1
+    # unsupported head dim
+    assert lib.sa_lse_combine(fake, fake, 2, 4, 96, fake, None, None) == 2
+    assert b"head dim" in lib.sa_last_error_string()
+    # misaligned pointer
+    assert lib.sa_lse_combine(ctypes.c_void_p((1 << 20) + 4), fake, 2, 4, 64, fake, None, None) == 1
+    # unsupported indexer head count
+    assert lib.sa_indexer_topk(fake, fake, fake, 1, 8, 8, 3, 32, 0, 4, 0, fake, None,
+                               fake, 1 << 20, None) == 2
+    # query positions beyond the keys
+    assert lib.sa_indexer_topk(fake, fake, fake, 1, 8, 8, 2, 32, 1, 4, 0, fake, None,
+                               fake, 1 << 20, None) == 1
+    # workspace too small
+    assert lib.sa_indexer_topk(fake, fake, fake, 1, 8, 8, 2, 32, 0, 4, 0, fake, None,
+                               fake, 16, None) == 3
+    # pattern must start with F
+    arr = (_lib.sa_dsa_layer * 1)()
+    assert lib.sa_dsa_decode_layers(b"S", 1, arr, 1, 1, 8, 16, 1, 128, 8, 64, 7, 4, 0,
+                                    0.1, 1, None, fake, 1 << 30, None) == 1
+    assert b"first layer" in lib.sa_last_error_string()
+    # NSA: sel_topk too large
+    assert lib.sa_nsa_fwd(fake, fake, fake, fake, 1, 64, 16, 1, 64, 32, 16, 64, 33, 512,
+                          0.1, fake, None, None, fake, 1 << 30, None) == 2
+    # attention: Hq not a multiple of Hkv
+    assert lib.sa_sparse_attn_fwd(fake, fake, fake, 1, 4, 4, 3, 2, 64, 0, fake, 1, 4, None,
+                                  None, None, None, 0.1, 1, fake, None, None, None, None, 0,
+                                  None) == 1
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "absent.so"))
+    monkeypatch.setattr(_lib, "_lib", None)
+    with pytest.raises(ImportError):
+        _lib.load()

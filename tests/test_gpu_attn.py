@@ -1,0 +1,181 @@
+"""GPU parity: gathered-KV sparse attention, split-KV partials, LSE combine,
+fixed pattern with coordinate bias, device error word."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from fixed_pattern_sparse_sa_b200 import api, inputs
+from fixed_pattern_sparse_sa_b200._lib import SAError
+from _parity import assert_lse_close, assert_out_close, sample_rows, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def _random_lists(B, T, heads, K, seed, L=None, q_pos0=0, fill=0.8):
+    """Random unsorted index lists inside the causal range, -1 padded."""
+    rng = np.random.default_rng(seed)
+    L = T if L is None else L
+    idx = np.full((B, T, heads, K), -1, dtype=np.int32)
+    for b in range(B):
+        for t in range(T):
+            p = q_pos0 + t
+            for h in range(heads):
+                n = min(p + 1, int(K * fill) if K > 1 else 1)
+                idx[b, t, h, :n] = rng.choice(p + 1, size=n, replace=False)
+                rng.shuffle(idx[b, t, h])
+    return torch.from_numpy(idx)
+
+
+def test_tiny_dsa_end_to_end(cuda_ok):
+    w = inputs.WORKLOADS["tiny_dsa"]
+    g = inputs.gen_dsa(w.B, w.T, w.Hq, w.Hkv, w.d, w.Hi, w.di, seed=0)
+    gd = to_dev(g)
+    idx, _ = api.indexer_topk(gd["q_idx"], gd["k_idx"], gd["w"], w.topk, w.window)
+    out, lse = api.sparse_attn_fwd(gd["q"], gd["k"], gd["v"], idx)
+    ref_idx, _ = oracle.indexer_topk(g["q_idx"], g["k_idx"], g["w"], w.topk, w.window)
+    ro, rl = oracle.sparse_attn(g["q"], g["k"], g["v"], ref_idx.reshape(1, w.T, -1))
+    assert_out_close(out, ro)
+    assert_lse_close(lse, rl)
+    api.check_device_status()
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("Hq,Hkv", [(16, 1), (4, 1), (8, 8), (8, 2), (32, 1)])
+def test_random_lists(cuda_ok, d, Hq, Hkv):
+    B, T, K = 2, 77, 70
+    g = inputs.gen_dsa(B, T, Hq, Hkv, d, 1, 32, seed=Hq * 7 + d)
+    idx = _random_lists(B, T, 1, K, seed=d + Hq)
+    out, lse = api.sparse_attn_fwd(g["q"].cuda(), g["k"].cuda(), g["v"].cuda(), idx.cuda())
+    ro, rl = oracle.sparse_attn(g["q"], g["k"], g["v"], idx)
+    assert_out_close(out, ro)
+    assert_lse_close(lse, rl)
+
+
+def test_per_kv_head_lists_and_empty_rows(cuda_ok):
+    B, T, Hq, Hkv, d, K = 1, 50, 8, 2, 64, 33
+    g = inputs.gen_dsa(B, T, Hq, Hkv, d, 1, 32, seed=3)
+    idx = _random_lists(B, T, Hkv, K, seed=4, fill=0.5)
+    idx[0, 10:13] = -1                    # empty sets -> zero output, lse = -inf
+    out, lse = api.sparse_attn_fwd(g["q"].cuda(), g["k"].cuda(), g["v"].cuda(), idx.cuda())
+    ro, rl = oracle.sparse_attn(g["q"], g["k"], g["v"], idx)
+    assert_out_close(out, ro)
+    assert_lse_close(lse, rl)
+    assert torch.all(out[0, 10:13] == 0)
+
+
+def test_queries_at_the_end_of_a_longer_cache(cuda_ok):
+    B, Tq, L, Hq, d, K = 3, 5, 900, 16, 128, 300
+    g = inputs.gen_dsa(B, Tq, Hq, 1, d, 1, 32, seed=8, L=L)
+    idx = _random_lists(B, Tq, 1, K, seed=9, L=L, q_pos0=L - Tq, fill=1.0)
+    out, lse = api.sparse_attn_fwd(g["q"].cuda(), g["k"].cuda(), g["v"].cuda(), idx.cuda())
+    ro, rl = oracle.sparse_attn(g["q"], g["k"], g["v"], idx, q_pos0=L - Tq)
+    assert_out_close(out, ro)
+    assert_lse_close(lse, rl)
+
+
+@pytest.mark.parametrize("n_split", [2, 4, 7, 16])
+def test_split_kv_partials_and_combine(cuda_ok, n_split):
+    B, Tq, L, Hq, d, K = 4, 1, 3000, 16, 128, 2048
+    g = inputs.gen_dsa(B, Tq, Hq, 1, d, 1, 32, seed=10, L=L)
+    idx = _random_lists(B, Tq, 1, K, seed=11, L=L, q_pos0=L - 1, fill=1.0)
+    out, lse, po, pl = api.sparse_attn_fwd(g["q"].cuda(), g["k"].cuda(), g["v"].cuda(),
+                                           idx.cuda(), n_split=n_split, return_partials=True)
+    ro, rl = oracle.sparse_attn(g["q"], g["k"], g["v"], idx, q_pos0=L - 1)
+    assert_out_close(out, ro)
+    assert_lse_close(lse, rl)
+    # every piece against the oracle on that piece alone
+    c = -(-K // n_split)
+    for s in range(n_split):
+        part = torch.full_like(idx, -1)
+        part[..., s * c:(s + 1) * c] = idx[..., s * c:(s + 1) * c]
+        so, sl = oracle.sparse_attn(g["q"], g["k"], g["v"], part, q_pos0=L - 1)
+        np.testing.assert_allclose(po[s].cpu().numpy().reshape(so.shape), so, atol=2e-3)
+        assert_lse_close(pl[s], sl)
+    # the standalone combine call on the same partials
+    o2, l2 = api.lse_combine(po, pl)
+    assert_out_close(o2, ro)
+    assert_lse_close(l2, rl)
+
+
+def test_lse_combine_with_empty_pieces(cuda_ok):
+    S, R, d = 5, 37, 64
+    rng = np.random.default_rng(12)
+    po = rng.standard_normal((S, R, d)).astype(np.float32)
+    pl = rng.standard_normal((S, R)).astype(np.float32) * 3
+    pl[1] = -np.inf
+    pl[:, 3] = -np.inf                    # a row with nothing at all
+    out, lse = api.lse_combine(torch.from_numpy(po).cuda(), torch.from_numpy(pl).cuda())
+    ro, rl = oracle.lse_combine(po, pl)
+    assert_out_close(out, ro)
+    assert_lse_close(lse, rl)
+
+
+@pytest.mark.parametrize("T,H,Hkv,d", [(700, 2, 2, 64), (300, 16, 1, 128), (1000, 4, 2, 64)])
+def test_fixed_pattern_with_bias(cuda_ok, T, H, Hkv, d):
+    g = inputs.gen_spatial(1, T, H, d, beta=0.5, seed=T, Hkv=Hkv)
+    gd = to_dev(g)
+    out, lse = api.sparse_attn_fwd(gd["q"], gd["k"], gd["v"], pattern=(65, True),
+                                   cq=gd["cq"], ck=gd["ck"], beta=gd["beta"])
+    idx, _ = oracle.fixed_graph(T, 65, True, cap=100)
+    ro, rl = oracle.sparse_attn(g["q"], g["k"], g["v"], idx.reshape(1, T, -1),
+                                cq=g["cq"], ck=g["ck"], beta=g["beta"])
+    assert_out_close(out, ro)
+    assert_lse_close(lse, rl)
+    # pattern without bias, window only
+    out2, lse2 = api.sparse_attn_fwd(gd["q"], gd["k"], gd["v"], pattern=(9, False))
+    idx2, _ = oracle.fixed_graph(T, 9, False, cap=9)
+    ro2, rl2 = oracle.sparse_attn(g["q"], g["k"], g["v"], idx2.reshape(1, T, -1))
+    assert_out_close(out2, ro2)
+    assert_lse_close(lse2, rl2)
+
+
+def test_spatial16k_full_parity(cuda_ok):
+    w = inputs.WORKLOADS["spatial16k"]
+    g = inputs.gen_spatial(w.B, w.T, w.Hq, w.d, beta=w.beta, seed=0)
+    gd = to_dev(g)
+    out, lse = api.sparse_attn_fwd(gd["q"], gd["k"], gd["v"], pattern=(w.window, w.dilated),
+                                   cq=gd["cq"], ck=gd["ck"], beta=gd["beta"])
+    idx, cnt = oracle.fixed_graph(w.T, w.window, w.dilated, cap=80)
+    assert int(cnt.sum()) == 1161305
+    ro, rl = oracle.sparse_attn(g["q"], g["k"], g["v"], idx.reshape(1, w.T, -1),
+                                cq=g["cq"], ck=g["ck"], beta=g["beta"])
+    assert_out_close(out, ro)
+    assert_lse_close(lse, rl)
+
+
+def test_prefill64k_attention_sampled_rows(cuda_ok):
+    # full-size run in the launch configuration the benchmark times
+    w = inputs.WORKLOADS["dsa_prefill64k"]
+    g = inputs.gen_dsa(w.B, w.T, w.Hq, w.Hkv, w.d, w.Hi, w.di, seed=0)
+    gd = to_dev(g)
+    idx, _ = api.indexer_topk(gd["q_idx"], gd["k_idx"], gd["w"], w.topk, w.window)
+    out, lse = api.sparse_attn_fwd(gd["q"], gd["k"], gd["v"], idx)
+    rows = sample_rows(w.T, 192, seed=2)
+    ref_idx, _ = oracle.indexer_topk(g["q_idx"], g["k_idx"], g["w"], w.topk, w.window, rows=rows)
+    np.testing.assert_array_equal(idx[0].cpu().numpy()[rows], ref_idx)
+    ro, rl = oracle.sparse_attn(g["q"], g["k"], g["v"], idx.cpu(), rows=rows)
+    assert_out_close(out[0][rows], ro)
+    assert_lse_close(lse[0][rows], rl)
+    assert torch.isfinite(out.float()).all()
+    api.check_device_status()
+
+
+def test_bad_index_sets_device_error_word(cuda_ok):
+    B, T, Hq, d = 1, 8, 16, 64
+    g = inputs.gen_dsa(B, T, Hq, 1, d, 1, 32, seed=13)
+    idx = torch.full((B, T, 4), -1, dtype=torch.int32)
+    for t in range(T):
+        idx[0, t, 0] = t
+    idx[0, 2, 1] = 5                       # a future position for query 2
+    out, _ = api.sparse_attn_fwd(g["q"].cuda(), g["k"].cuda(), g["v"].cuda(), idx.cuda())
+    with pytest.raises(SAError) as ei:
+        api.check_device_status()
+    assert ei.value.status == 5
+    api.check_device_status()              # the word was cleared
+    # the offending entry was skipped: row 2 equals attention over {2} alone
+    idx2 = idx.clone(); idx2[0, 2, 1] = -1
+    ro, _ = oracle.sparse_attn(g["q"], g["k"], g["v"], idx2)
+    assert_out_close(out, ro)

@@ -1,0 +1,94 @@
+"""GPU parity: indexer scores + exact causal top-k (bit-exact indices)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from fixed_pattern_sparse_sa_b200 import api, inputs
+from _parity import sample_rows, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def _check_rows(got_idx, got_cnt, ref_idx, ref_cnt, rows=None):
+    gi = got_idx.cpu().numpy().reshape(-1, got_idx.shape[-1])
+    gc = got_cnt.cpu().numpy().reshape(-1)
+    if rows is not None:
+        gi, gc = gi[rows], gc[rows]
+    np.testing.assert_array_equal(gc, ref_cnt)
+    np.testing.assert_array_equal(gi, ref_idx)
+
+
+def test_tiny_dsa_topk_bit_exact(cuda_ok):
+    w = inputs.WORKLOADS["tiny_dsa"]
+    g = inputs.gen_dsa(w.B, w.T, w.Hq, w.Hkv, w.d, w.Hi, w.di, seed=0)
+    gd = to_dev(g)
+    idx, cnt = api.indexer_topk(gd["q_idx"], gd["k_idx"], gd["w"], w.topk, w.window)
+    ref_idx, ref_cnt = oracle.indexer_topk(g["q_idx"], g["k_idx"], g["w"], w.topk, w.window)
+    _check_rows(idx, cnt, ref_idx, ref_cnt)
+    api.check_device_status()
+
+
+@pytest.mark.parametrize("T", [1, 2, 17, 63, 64, 65, 127, 128, 129, 300])
+@pytest.mark.parametrize("Hi,di", [(2, 32), (8, 64), (1, 128), (4, 32), (16, 64)])
+def test_ragged_shapes_bit_exact(cuda_ok, T, Hi, di):
+    g = inputs.gen_dsa(2, T, 1, 1, 64, Hi, di, seed=T * 31 + Hi)
+    gd = to_dev(g)
+    for topk, window in [(16, 0), (5, 4), (T, 0), (40, 8)]:
+        idx, cnt = api.indexer_topk(gd["q_idx"], gd["k_idx"], gd["w"], topk, window)
+        ref_idx, ref_cnt = oracle.indexer_topk(g["q_idx"], g["k_idx"], g["w"], topk, window)
+        _check_rows(idx, cnt, ref_idx, ref_cnt)
+
+
+def test_heavy_ties_bit_exact(cuda_ok):
+    # tiny value range and mostly-zero weights: huge tie groups at the threshold
+    gen = torch.Generator().manual_seed(5)
+    B, T, Hi, di = 1, 700, 8, 32
+    q = torch.randint(-1, 2, (B, T, Hi, di), generator=gen).to(torch.int8)
+    k = torch.randint(-1, 2, (B, T, di), generator=gen).to(torch.int8)
+    w = (torch.rand((B, T, Hi), generator=gen) < 0.2).to(torch.int32)
+    idx, cnt = api.indexer_topk(q.cuda(), k.cuda(), w.cuda(), 64, 16)
+    ref_idx, ref_cnt = oracle.indexer_topk(q, k, w, 64, 16)
+    _check_rows(idx, cnt, ref_idx, ref_cnt)
+
+
+def test_wide_value_range_and_negative_weights(cuda_ok):
+    # large int8 magnitudes and signed weights: scores span > 2^24, forcing
+    # three radix digit passes and negative keys
+    gen = torch.Generator().manual_seed(6)
+    B, T, Hi, di = 1, 400, 4, 128
+    q = torch.randint(-128, 128, (B, T, Hi, di), generator=gen).to(torch.int8)
+    k = torch.randint(-128, 128, (B, T, di), generator=gen).to(torch.int8)
+    w = torch.randint(-300, 301, (B, T, Hi), generator=gen).to(torch.int32)
+    idx, cnt = api.indexer_topk(q.cuda(), k.cuda(), w.cuda(), 50, 0)
+    ref_idx, ref_cnt = oracle.indexer_topk(q, k, w, 50, 0)
+    _check_rows(idx, cnt, ref_idx, ref_cnt)
+
+
+def test_decode_rows_multi_cta_clusters(cuda_ok):
+    # one query per sequence at the last position: the select uses clusters
+    nseq, L = 4, 40000
+    g = inputs.gen_decode_layer(nseq, L, 16, 1, 128, 8, 64, layer=0, seed=7)
+    gd = to_dev(g)
+    idx, cnt = api.indexer_topk(gd["q_idx"], gd["k_idx"], gd["w"], 2048, 0)
+    ref_idx, ref_cnt = oracle.indexer_topk(g["q_idx"], g["k_idx"], g["w"], 2048, 0, q_pos0=L - 1)
+    _check_rows(idx, cnt, ref_idx, ref_cnt)
+
+
+def test_prefill64k_sampled_rows_bit_exact(cuda_ok):
+    w = inputs.WORKLOADS["dsa_prefill64k"]
+    g = inputs.gen_dsa(w.B, w.T, w.Hq, w.Hkv, w.d, w.Hi, w.di, seed=0)
+    gd = to_dev(g)
+    idx, cnt = api.indexer_topk(gd["q_idx"], gd["k_idx"], gd["w"], w.topk, w.window)
+    rows = sample_rows(w.T, 192, seed=1)
+    ref_idx, ref_cnt = oracle.indexer_topk(g["q_idx"], g["k_idx"], g["w"], w.topk, w.window,
+                                           rows=rows)
+    _check_rows(idx, cnt, ref_idx, ref_cnt, rows=rows)
+    # properties that hold for every row
+    c = cnt.cpu().numpy()[0]
+    np.testing.assert_array_equal(c, np.minimum(np.arange(w.T) + 1, w.topk))
+    ii = idx[0].cpu().numpy()
+    valid = ii >= 0
+    assert np.all(ii[valid] <= np.repeat(np.arange(w.T)[:, None], ii.shape[1], 1)[valid])
+    d = np.diff(np.where(valid, ii, np.iinfo(np.int32).max).astype(np.int64), axis=1)
+    assert np.all(d[valid[:, 1:]] > 0), "rows must be strictly ascending"

@@ -1,0 +1,110 @@
+"""GPU parity: NSA three-branch forward and the IndexCache decode driver."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from fixed_pattern_sparse_sa_b200 import api, inputs
+from _parity import assert_lse_close, assert_out_close, sample_rows, to_dev
+
+pytestmark = pytest.mark.gpu
+
+NSA_CFG = dict(cmp_len=32, cmp_stride=16, sel_block=64, sel_topk=16, window=512)
+
+
+def _nsa_check(g, out, lse3, sel, rows, cfg):
+    """Selection parity with the near-tie rule, then outputs against the oracle
+    re-run with the GPU's selection."""
+    ref = oracle.nsa_fwd(g["q"], g["k"], g["v"], g["gates"], rows=rows, **cfg)
+    gsel = sel.cpu().numpy().reshape(-1, sel.shape[2], sel.shape[3])[rows]
+    n_diff = 0
+    for i in range(len(rows)):
+        for gg in range(gsel.shape[1]):
+            a = set(x for x in gsel[i, gg] if x >= 0)
+            b = set(x for x in ref["sel_idx"][i, gg] if x >= 0)
+            if a == b:
+                continue
+            n_diff += 1
+            imp = ref["imp"][i, gg]
+            kth = np.sort(imp[[x for x in b]])[0]           # smallest chosen importance
+            tol = 1e-5 * imp.max()
+            for blk in a ^ b:
+                assert abs(imp[blk] - kth) <= tol, f"row {rows[i]} group {gg}: block {blk} not a near-tie"
+    assert n_diff <= max(2, len(rows) // 100), f"{n_diff} near-tie rows"
+    ref2 = oracle.nsa_fwd(g["q"], g["k"], g["v"], g["gates"], rows=rows, sel_override=gsel, **cfg)
+    B, T, Hq, d = g["q"].shape
+    assert_out_close(out.reshape(-1, Hq, d)[rows], ref2["out"], "nsa out")
+    assert_lse_close(lse3.reshape(-1, Hq, 3)[rows], ref2["lse_branch"], "nsa lse")
+    return n_diff
+
+
+@pytest.mark.parametrize("T", [40, 300, 1100])
+def test_nsa_small_full_parity(cuda_ok, T):
+    g = inputs.gen_nsa(1, T, 32, 2, 64, seed=T)
+    gd = to_dev(g)
+    out, lse3, sel = api.nsa_fwd(gd["q"], gd["k"], gd["v"], gd["gates"], **NSA_CFG)
+    _nsa_check(g, out, lse3, sel, np.arange(T), NSA_CFG)
+
+
+def test_nsa_branches_isolated_by_gates(cuda_ok):
+    T = 700
+    g = inputs.gen_nsa(1, T, 16, 1, 128, seed=3)
+    gd = to_dev(g)
+    ref = oracle.nsa_fwd(g["q"], g["k"], g["v"], g["gates"], **NSA_CFG)
+    for br in range(3):
+        oh = torch.zeros_like(gd["gates"])
+        oh[..., br] = 1.0
+        out, _, sel = api.nsa_fwd(gd["q"], gd["k"], gd["v"], oh, **NSA_CFG)
+        r2 = oracle.nsa_fwd(g["q"], g["k"], g["v"], oh.cpu(),
+                            sel_override=sel.cpu().numpy().reshape(T, 1, -1), **NSA_CFG)
+        assert_out_close(out[0], r2["o_branch"][br], f"branch {br}")
+    assert ref["out"].shape == (T, 16, 128)
+
+
+def test_nsa64k_sampled_rows(cuda_ok):
+    w = inputs.WORKLOADS["nsa64k"]
+    g = inputs.gen_nsa(w.B, w.T, w.Hq, w.Hkv, w.d, seed=0)
+    gd = to_dev(g)
+    cfg = dict(cmp_len=w.cmp_len, cmp_stride=w.cmp_stride, sel_block=w.sel_block,
+               sel_topk=w.sel_topk, window=w.window)
+    out, lse3, sel = api.nsa_fwd(gd["q"], gd["k"], gd["v"], gd["gates"], **cfg)
+    rows = sample_rows(w.T, 48, seed=4, edge=8)
+    _nsa_check(g, out, lse3, sel, rows, cfg)
+    api.check_device_status()
+
+
+def _decode_layers(nseq, L, n_layers, seed, device="cpu"):
+    return [inputs.gen_decode_layer(nseq, L, 16, 1, 128, 8, 64, layer=i, seed=seed, device=device)
+            for i in range(n_layers)]
+
+
+@pytest.mark.parametrize("pattern", ["FSSS", "FFFF", "FSFS"])
+def test_indexcache_decode_small(cuda_ok, pattern):
+    nseq, L = 3, 5000
+    lays = _decode_layers(nseq, L, 4, seed=20)
+    dl = [to_dev(x) for x in lays]
+    outs, lses, cache = api.dsa_decode_layers(pattern, dl, topk=2048, n_split=8)
+    ref = oracle.dsa_layers(pattern, lays, topk=2048)
+    for i in range(4):
+        assert_out_close(outs[i], ref[i][1], f"layer {i}")
+        assert_lse_close(lses[i], ref[i][2], f"layer {i}")
+    np.testing.assert_array_equal(cache.cpu().numpy().reshape(ref[-1][0].shape), ref[-1][0])
+
+
+def test_decode128k_full_size(cuda_ok):
+    # 32 sequences x 131072 cached tokens, 4 layers; caches drawn on the GPU.
+    w = inputs.WORKLOADS["dsa_decode128k"]
+    lays = _decode_layers(w.B, w.T, 4, seed=0, device="cuda")
+    for pattern in ("FSSS", "FFFF"):
+        outs, lses, cache = api.dsa_decode_layers(pattern, lays, topk=w.topk, n_split=16)
+        torch.cuda.synchronize()
+        # oracle on a few sequences of every layer (host copies of those rows)
+        seqs = [0, 17, 31]
+        sub = [{k: v[seqs].cpu() for k, v in lay.items()} for lay in lays]
+        ref = oracle.dsa_layers(pattern, sub, topk=w.topk)
+        for i in range(4):
+            assert_out_close(outs[i][seqs], ref[i][1], f"{pattern} layer {i}")
+            assert_lse_close(lses[i][seqs], ref[i][2], f"{pattern} layer {i}")
+        np.testing.assert_array_equal(cache[seqs].cpu().numpy().reshape(ref[-1][0].shape),
+                                      ref[-1][0])
+    api.check_device_status()
