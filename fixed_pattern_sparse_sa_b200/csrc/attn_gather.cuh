@@ -11,6 +11,8 @@
 // folded into an online softmax and multiplied into V with a second mma.
 #pragma once
 
+#include <climits>
+
 #include "sa_common.cuh"
 
 namespace sa {
@@ -48,23 +50,25 @@ struct GatherParams {
     unsigned *err;
 };
 
-// Key position for virtual entry e of the item, or -1 if the entry is empty
-// or masked.  Raises the error word for an explicit index that is out of
-// range or in the future.
+// Keys are produced in two stages so that the list loads can be issued well
+// before they are needed.  key_raw: the raw list value of virtual entry e (a
+// global load for explicit lists; computed sources give the final key, -1 when
+// masked).  key_finish: validation and translation to a key position, or -1
+// for an empty/masked entry; an explicit index that is out of range or in the
+// future raises the error word and is skipped.
+constexpr int KEY_NONE = INT_MIN;
+
 template <int SRC>
-__device__ __forceinline__ int key_at(const GatherParams &p, int b, int t, int g, long long pos,
-                                      int e, int e_end) {
-    if (e >= e_end) return -1;
+__device__ __forceinline__ int key_raw(const GatherParams &p, int b, int t, int g, long long pos,
+                                       int e, int e_end) {
+    if (e >= e_end) return KEY_NONE;
     if constexpr (SRC == KS_IDX) {
         const int32_t *list =
             p.idx + ((long long)(b * p.Tq + t) * p.idx_heads + (p.idx_heads == 1 ? 0 : g)) * p.K;
-        int j = __ldg(list + e);
-        if (j == -1) return -1;
-        if (j < 0 || j >= p.Lk || (long long)j > pos) {
-            raise_error(p.err, ERR_BAD_INDEX);
-            return -1;
-        }
-        return j;
+        return __ldg(list + e);
+    } else if constexpr (SRC == KS_BLOCKS) {
+        const int32_t *list = p.idx + ((long long)(b * p.Tq + t) * p.Hkv + g) * p.K;
+        return __ldg(list + e / p.block);
     } else if constexpr (SRC == KS_PATTERN) {
         long long nw = pos + 1 < p.window ? pos + 1 : p.window;
         if (e < nw) return (int)(pos - e);
@@ -77,17 +81,6 @@ __device__ __forceinline__ int key_at(const GatherParams &p, int b, int t, int g
         long long o = 1LL << (i0 + m);
         if (o >= pos) return -1;
         return (int)(pos - o);
-    } else if constexpr (SRC == KS_BLOCKS) {
-        const int32_t *list = p.idx + ((long long)(b * p.Tq + t) * p.Hkv + g) * p.K;
-        int blk = __ldg(list + e / p.block);
-        if (blk == -1) return -1;
-        long long j = (long long)blk * p.block + e % p.block;
-        if (blk < 0 || (long long)blk * p.block >= p.Lk) {
-            raise_error(p.err, ERR_BAD_BLOCK);
-            return -1;
-        }
-        if (j > pos || j >= p.Lk) return -1;   // causal mask inside the block
-        return (int)j;
     } else if constexpr (SRC == KS_RANGE) {
         long long j = pos - p.window + 1 + e;
         return j < 0 ? -1 : (int)j;
@@ -97,12 +90,37 @@ __device__ __forceinline__ int key_at(const GatherParams &p, int b, int t, int g
     }
 }
 
+template <int SRC>
+__device__ __forceinline__ int key_finish(const GatherParams &p, long long pos, int raw, int e) {
+    if (raw == KEY_NONE) return -1;
+    if constexpr (SRC == KS_IDX) {
+        if (raw == -1) return -1;
+        if (raw < 0 || raw >= p.Lk || (long long)raw > pos) {
+            raise_error(p.err, ERR_BAD_INDEX);
+            return -1;
+        }
+        return raw;
+    } else if constexpr (SRC == KS_BLOCKS) {
+        const int blk = raw;
+        if (blk == -1) return -1;
+        if (blk < 0 || (long long)blk * p.block >= p.Lk) {
+            raise_error(p.err, ERR_BAD_BLOCK);
+            return -1;
+        }
+        const long long j = (long long)blk * p.block + e % p.block;
+        if (j > pos || j >= p.Lk) return -1;   // causal mask inside the block
+        return (int)j;
+    } else {
+        return raw;
+    }
+}
+
 // KLO: keys are held as a bf16 pair (hi, lo) whose sum carries ~16 mantissa
 // bits; q.k is taken on both halves (used for the NSA compressed keys, which
 // are means and do not fit bf16 exactly).
-template <int D, int STAGES, int SRC, bool BIAS, bool KLO = false>
-__global__ void __launch_bounds__(128) gather_attn_kernel(const GatherParams p) {
-    constexpr int NK = 32;                 // keys per chunk
+template <int D, int STAGES, int SRC, bool BIAS, bool KLO = false, int NK = 32, int NW = 4>
+__global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams p) {
+    // NK keys per chunk, NW independent warps per CTA
     constexpr int ROWB = D * 2;            // bytes of one K/V row
     constexpr int UNITS = ROWB / 16;       // 16-byte units per row
     constexpr int CH = NK * ROWB;          // bytes of one K (or V) chunk
@@ -117,7 +135,7 @@ __global__ void __launch_bounds__(128) gather_attn_kernel(const GatherParams p) 
     int *keys_s = reinterpret_cast<int *>(wsm + STAGES * SB);
 
     const long long n_items = (long long)p.B * p.Tq * p.Hkv * p.n_hchunk * p.n_split;
-    const long long item = (long long)blockIdx.x * 4 + warp;
+    const long long item = (long long)blockIdx.x * NW + warp;
     if (item >= n_items) return;   // warps are independent: no block barrier below
 
     long long rem = item;
@@ -176,13 +194,17 @@ __global__ void __launch_bounds__(128) gather_attn_kernel(const GatherParams p) 
     const __nv_bfloat16 *lb = KLO ? p.klo + ((long long)b * p.Lk * p.Hkv + g) * D : nullptr;
     const long long rstride = (long long)p.Hkv * D;
 
-    auto issue = [&](int ci) {
+    // raw list value of chunk ci for this lane (lane i < NK owns key i)
+    auto raw_of = [&](int ci) -> int {
+        return (ci < n_chunks && lane < NK) ? key_raw<SRC>(p, b, t, g, pos, e_beg + ci * NK + lane, e_end)
+                                            : KEY_NONE;
+    };
+    auto issue = [&](int ci, int raw) {
         const int st = ci % STAGES;
         unsigned char *ks_ = wsm + st * SB;
         unsigned char *vs_ = ks_ + CH;
-        int j = -1;
-        if (ci < n_chunks) j = key_at<SRC>(p, b, t, g, pos, e_beg + ci * NK + lane, e_end);
-        keys_s[st * NK + lane] = j;
+        const int j = key_finish<SRC>(p, pos, raw, e_beg + ci * NK + lane);
+        if (lane < NK) keys_s[st * NK + lane] = j;
         if (ci < n_chunks) {
 #pragma unroll
             for (int it = 0; it < CP_ITERS; ++it) {
@@ -206,16 +228,21 @@ __global__ void __launch_bounds__(128) gather_attn_kernel(const GatherParams p) 
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
 
 #pragma unroll
-    for (int ci = 0; ci < STAGES - 1; ++ci) issue(ci);
+    for (int ci = 0; ci < STAGES - 1; ++ci) issue(ci, raw_of(ci));
+    // list values are loaded two chunks ahead of the K/V copies that use them
+    int raw_a = raw_of(STAGES - 1), raw_b = raw_of(STAGES);
 
     for (int ci = 0; ci < n_chunks; ++ci) {
-        issue(ci + STAGES - 1);
+        const int raw = raw_a;
+        raw_a = raw_b;
+        raw_b = raw_of(ci + STAGES + 1);
+        issue(ci + STAGES - 1, raw);
         cp_async_wait<STAGES - 1>();
         __syncwarp();
         const int st = ci % STAGES;
         const unsigned char *ks_ = wsm + st * SB;
         const unsigned char *vs_ = ks_ + CH;
-        const int jl = keys_s[st * NK + lane];
+        const int jl = lane < NK ? keys_s[st * NK + lane] : -1;
         const unsigned vmask = __ballot_sync(0xffffffffu, jl >= 0);
         if (vmask != 0u) {
             float sc[NK / 8][4];
@@ -271,6 +298,8 @@ __global__ void __launch_bounds__(128) gather_attn_kernel(const GatherParams p) 
             const float mu0 = mn0 == -INFINITY ? 0.f : mn0;
             const float mu1 = mn1 == -INFINITY ? 0.f : mn1;
             const float al0 = exp2f(m0 - mu0), al1 = exp2f(m1 - mu1);
+            // the accumulators need rescaling only when some row's max grew
+            const bool grew = __any_sync(0xffffffffu, mn0 > m0 || mn1 > m1);
             m0 = mn0; m1 = mn1;
             float rs0 = 0.f, rs1 = 0.f;
 #pragma unroll
@@ -284,10 +313,12 @@ __global__ void __launch_bounds__(128) gather_attn_kernel(const GatherParams p) 
             }
             l0 = l0 * al0 + rs0;
             l1 = l1 * al1 + rs1;
+            if (grew) {
 #pragma unroll
-            for (int i = 0; i < NT_D; ++i) {
-                o[i][0] *= al0; o[i][1] *= al0;
-                o[i][2] *= al1; o[i][3] *= al1;
+                for (int i = 0; i < NT_D; ++i) {
+                    o[i][0] *= al0; o[i][1] *= al0;
+                    o[i][2] *= al1; o[i][3] *= al1;
+                }
             }
             // P (bf16) * V
 #pragma unroll
@@ -365,9 +396,9 @@ __global__ void __launch_bounds__(128) gather_attn_kernel(const GatherParams p) 
     }
 }
 
-template <int D, int STAGES, bool KLO = false>
+template <int D, int STAGES, bool KLO = false, int NK = 32, int NW = 4>
 constexpr int gather_smem_bytes() {
-    return 4 * STAGES * ((KLO ? 3 : 2) * 32 * D * 2 + 32 * 4);
+    return NW * STAGES * ((KLO ? 3 : 2) * NK * D * 2 + NK * 4);
 }
 
 }  // namespace sa

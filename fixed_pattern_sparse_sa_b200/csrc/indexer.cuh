@@ -26,6 +26,7 @@
 #include <cooperative_groups.h>
 
 #include "sa_common.cuh"
+#include "tc_common.cuh"
 
 namespace sa {
 
@@ -41,6 +42,7 @@ struct IdxScoreParams {
     int t0, Rt;            // chunk: query rows t0 .. t0+Rt-1 of every batch element
     long long ld;          // row stride of the score buffer (elements)
     int32_t *scores;       // [B, Rt, ld]
+    unsigned *err;         // device error word
 };
 
 // Number of selectable (non-window) candidates of a query at position p.
@@ -49,137 +51,295 @@ __device__ __forceinline__ long long n_candidates(long long p, int window) {
     return n > 0 ? n : 0;
 }
 
-// Tile: 128 keys (4 warps x 2 m-tiles of 16) x 128 (query, head) columns.
+// CTA tile: SC_KEYS keys (8 warps x SC_MT m-tiles of 16) x 128 (query, head)
+// columns (QT = 128 / HI queries).  Each lane keeps the B fragments of all 128
+// columns in registers; each warp walks its keys one m-tile at a time.
+constexpr int SC_WARPS = 8;
+constexpr int SC_MT = 8;                                   // m-tiles per warp
+constexpr int SC_KEYS = SC_WARPS * SC_MT * 16;             // 1024 keys per CTA
+
 template <int HI, int DI>
-__global__ void __launch_bounds__(128) idx_score_kernel(const IdxScoreParams p) {
-    constexpr int KT = 128;                  // keys per CTA
+__global__ void __launch_bounds__(SC_WARPS * 32) idx_score_kernel(const IdxScoreParams p) {
     constexpr int COLS = 128;                // (query, head) columns per CTA
     constexpr int QT = COLS / HI;            // queries per CTA
     constexpr int NT = COLS / 8;             // n-tiles
     constexpr int REG = DI / 16;             // u32 registers per lane per row
     constexpr int KSTEPS = DI / 32;
-    constexpr int NG = 4;                    // n-tiles per accumulator group
     static_assert(HI == 1 || HI == 2 || HI == 4 || HI == 8 || HI == 16, "HI");
     static_assert(DI == 32 || DI == 64 || DI == 128, "DI");
 
-    extern __shared__ __align__(1024) unsigned char smem[];
-    int *tile = reinterpret_cast<int *>(smem);           // [QT][KT]
-    int *ws = tile + QT * KT;                             // [QT*HI]
+    __shared__ int ws[COLS];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gr = lane >> 2, qc = lane & 3;
     const int b = blockIdx.z;
     const int tq0 = p.t0 + blockIdx.y * QT;               // first query of the tile
-    const int j0 = blockIdx.x * KT;
     const int t_last = min(p.t0 + p.Rt, p.Tq) - 1;
     const int tq_last = min(tq0 + QT - 1, t_last);
     if (tq0 > t_last) return;
-    if ((long long)j0 >= n_candidates(p.q_pos0 + tq_last, p.window)) return;   // above the diagonal
+    const long long ncand_last = n_candidates(p.q_pos0 + tq_last, p.window);
+    const int j_cta = blockIdx.x * SC_KEYS;
+    if ((long long)j_cta >= ncand_last) return;           // above the diagonal
 
-    for (int i = threadIdx.x; i < QT * HI; i += blockDim.x) {
+    for (int i = threadIdx.x; i < COLS; i += blockDim.x) {
         const int tq = tq0 + i / HI;
         ws[i] = tq <= tq_last ? __ldg(p.w + ((long long)b * p.Tq + tq) * HI + i % HI) : 0;
     }
-
-    // A fragments: this warp's 32 keys (2 m-tiles), rows gr and gr+8.
-    unsigned a[2][2][REG];
+    // B fragments (query side), all n-tiles, kept in registers
+    unsigned bq[NT][REG];
 #pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
+    for (int nt = 0; nt < NT; ++nt) {
+        const int col = nt * 8 + gr;
+        const int tq = tq0 + col / HI, h = col % HI;
+        const unsigned *src = reinterpret_cast<const unsigned *>(
+            p.q + (((long long)b * p.Tq + tq) * HI + h) * DI + qc * (DI / 4));
+#pragma unroll
+        for (int r = 0; r < REG; ++r) bq[nt][r] = tq <= tq_last ? __ldg(src + r) : 0u;
+    }
+    __syncthreads();
+
+    const int j_warp = j_cta + warp * SC_MT * 16;
+    // A fragments of the next m-tile are fetched one step ahead
+    unsigned a_nx[2][REG];
+    auto load_a = [&](int mt, unsigned (&a)[2][REG]) {
 #pragma unroll
         for (int hr = 0; hr < 2; ++hr) {
-            const int j = j0 + warp * 32 + mt * 16 + gr + hr * 8;
+            const int j = j_warp + mt * 16 + gr + hr * 8;
             const unsigned *src = reinterpret_cast<const unsigned *>(
                 p.k + ((long long)b * p.L + j) * DI + qc * (DI / 4));
 #pragma unroll
-            for (int r = 0; r < REG; ++r) a[mt][hr][r] = j < p.L ? __ldg(src + r) : 0u;
+            for (int r = 0; r < REG; ++r) a[hr][r] = j < p.L ? __ldg(src + r) : 0u;
         }
-    __syncthreads();
+    };
+    if ((long long)j_warp < ncand_last) load_a(0, a_nx);
 
 #pragma unroll 1
-    for (int ng = 0; ng < NT / NG; ++ng) {
-        int acc[2][NG][4];
+    for (int mt = 0; mt < SC_MT; ++mt) {
+        const int jm = j_warp + mt * 16;
+        if ((long long)jm >= ncand_last) break;           // the rest is above the diagonal
+        unsigned a[2][REG];
 #pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
+        for (int hr = 0; hr < 2; ++hr)
 #pragma unroll
-            for (int n = 0; n < NG; ++n) acc[mt][n][0] = acc[mt][n][1] = acc[mt][n][2] = acc[mt][n][3] = 0;
+            for (int r = 0; r < REG; ++r) a[hr][r] = a_nx[hr][r];
+        if (mt + 1 < SC_MT && (long long)(jm + 16) < ncand_last) load_a(mt + 1, a_nx);
+
 #pragma unroll
-        for (int n = 0; n < NG; ++n) {
-            const int nt = ng * NG + n;
-            const int col = nt * 8 + gr;                      // B column held by this lane
-            const int tq = tq0 + col / HI, h = col % HI;
-            unsigned bq[REG];
-            const unsigned *src = reinterpret_cast<const unsigned *>(
-                p.q + (((long long)b * p.Tq + tq) * HI + h) * DI + qc * (DI / 4));
+        for (int ng = 0; ng < NT / 4; ++ng) {
+            int acc[4][4];
 #pragma unroll
-            for (int r = 0; r < REG; ++r) bq[r] = tq <= tq_last ? __ldg(src + r) : 0u;
-#pragma unroll
-            for (int mt = 0; mt < 2; ++mt)
+            for (int n = 0; n < 4; ++n) {
+                acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0;
 #pragma unroll
                 for (int ks = 0; ks < KSTEPS; ++ks)
-                    mma_s8_16832(acc[mt][n], a[mt][0][2 * ks], a[mt][1][2 * ks], a[mt][0][2 * ks + 1],
-                                 a[mt][1][2 * ks + 1], bq[2 * ks], bq[2 * ks + 1]);
-        }
-        // epilogue: w * relu, sum over the heads of each query, stage to smem
+                    mma_s8_16832(acc[n], a[0][2 * ks], a[1][2 * ks], a[0][2 * ks + 1], a[1][2 * ks + 1],
+                                 bq[ng * 4 + n][2 * ks], bq[ng * 4 + n][2 * ks + 1]);
+            }
+            // epilogue: w * relu, sum over the heads of each query, store
+            int pr0 = 0, pr1 = 0;                             // HI == 16: even n-tile's half
 #pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-            for (int n = 0; n < NG; ++n) {
-                const int nt = ng * NG + n;
-                const int c0 = nt * 8 + 2 * qc, c1 = c0 + 1;  // columns of this thread
-                const int w0 = ws[c0], w1 = ws[c1];
-                const int r0a = w0 * max(acc[mt][n][0], 0), r0b = w1 * max(acc[mt][n][1], 0);
-                const int r1a = w0 * max(acc[mt][n][2], 0), r1b = w1 * max(acc[mt][n][3], 0);
-                const int kr0 = warp * 32 + mt * 16 + gr, kr1 = kr0 + 8;
+            for (int n = 0; n < 4; ++n) {
+                const int nt = ng * 4 + n;
+                const int c0 = nt * 8 + 2 * qc;               // columns c0, c0+1 of this thread
+                const int w0 = ws[c0], w1 = ws[c0 + 1];
+                const int s0 = w0 * max(acc[n][0], 0), s1 = w1 * max(acc[n][1], 0);   // key gr
+                const int s2 = w0 * max(acc[n][2], 0), s3 = w1 * max(acc[n][3], 0);   // key gr+8
                 if constexpr (HI == 1) {
-                    tile[(c0)*KT + kr0] = r0a; tile[(c1)*KT + kr0] = r0b;
-                    tile[(c0)*KT + kr1] = r1a; tile[(c1)*KT + kr1] = r1b;
+                    // every column is its own query
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int qi = c0 + (e & 1);
+                        const int key = jm + gr + (e >> 1) * 8;
+                        const int tq = tq0 + qi;
+                        const int v = e == 0 ? s0 : e == 1 ? s1 : e == 2 ? s2 : s3;
+                        if (tq <= tq_last && key < n_candidates(p.q_pos0 + tq, p.window))
+                            p.scores[((long long)b * p.Rt + (tq - p.t0)) * p.ld + key] = v;
+                    }
                 } else {
-                    int s0 = r0a + r0b, s1 = r1a + r1b;
+                    int r0 = s0 + s1, r1 = s2 + s3;
                     if constexpr (HI >= 4) {
-                        s0 += __shfl_xor_sync(0xffffffffu, s0, 1);
-                        s1 += __shfl_xor_sync(0xffffffffu, s1, 1);
+                        r0 += __shfl_xor_sync(0xffffffffu, r0, 1);
+                        r1 += __shfl_xor_sync(0xffffffffu, r1, 1);
                     }
                     if constexpr (HI >= 8) {
-                        s0 += __shfl_xor_sync(0xffffffffu, s0, 2);
-                        s1 += __shfl_xor_sync(0xffffffffu, s1, 2);
+                        r0 += __shfl_xor_sync(0xffffffffu, r0, 2);
+                        r1 += __shfl_xor_sync(0xffffffffu, r1, 2);
                     }
-                    const int qi = c0 / HI;                   // query of this column pair
+                    bool ready = true;
+                    if constexpr (HI == 16) {                  // n-tiles 2m, 2m+1 = one query
+                        if ((n & 1) == 0) { pr0 = r0; pr1 = r1; ready = false; }
+                        else { r0 += pr0; r1 += pr1; }
+                    }
                     constexpr int LEAD = HI >= 8 ? 4 : (HI == 4 ? 2 : 1);
-                    if ((qc % LEAD) == 0) {
-                        if constexpr (HI == 16) {
-                            // a query spans two n-tiles: accumulate both halves
-                            if ((nt & 1) == 0) {
-                                tile[qi * KT + kr0] = s0; tile[qi * KT + kr1] = s1;
-                            } else {
-                                tile[qi * KT + kr0] += s0; tile[qi * KT + kr1] += s1;
-                            }
-                        } else {
-                            tile[qi * KT + kr0] = s0; tile[qi * KT + kr1] = s1;
-                        }
+                    const int tq = tq0 + c0 / HI;
+                    if (ready && (qc % LEAD) == 0 && tq <= tq_last) {
+                        const long long nc = n_candidates(p.q_pos0 + tq, p.window);
+                        int32_t *dst = p.scores + ((long long)b * p.Rt + (tq - p.t0)) * p.ld;
+                        if (jm + gr < nc) dst[jm + gr] = r0;
+                        if (jm + gr + 8 < nc) dst[jm + gr + 8] = r1;
                     }
                 }
             }
-        __syncwarp();
-    }
-    __syncthreads();
-
-    // coalesced write-out of the [QT][KT] tile
-    const bool vec = (p.ld % 4) == 0;
-    for (int i = threadIdx.x; i < QT * (KT / 4); i += blockDim.x) {
-        const int qi = i / (KT / 4), k4 = (i % (KT / 4)) * 4;
-        const int tq = tq0 + qi;
-        if (tq > tq_last) continue;
-        const long long ncand = n_candidates(p.q_pos0 + tq, p.window);
-        const int j = j0 + k4;
-        if (j >= ncand) continue;
-        int32_t *dst = p.scores + ((long long)b * p.Rt + (tq - p.t0)) * p.ld + j;
-        const int *src = tile + qi * KT + k4;
-        if (vec && j + 3 < ncand) {
-            *reinterpret_cast<int4 *>(dst) = *reinterpret_cast<const int4 *>(src);
-        } else {
-            for (int u = 0; u < 4 && j + u < ncand; ++u) dst[u] = src[u];
         }
     }
+}
+
+// ------------------------------------------------- tcgen05 score kernel --
+// Tensor-core (tcgen05, kind::i8) version of the score GEMM.  CTA tile:
+// M = 128 keys (TMEM lanes) x N = 256 (query, head) columns (256/HI queries)
+// x K = DI; the accumulator lives in 256 TMEM columns.  Operands are staged
+// with cp.async in the K-major no-swizzle core-matrix layout: 8-row group r8
+// at r8 * 8*DI bytes, inside it the DI/16 core matrices (8 rows x 16 B)
+// back to back, so LBO = 128 B (next core along K) and SBO = 8*DI (next
+// 8-row group).  Thread i of warp w owns key row 32w+i: it reads that TMEM
+// lane and forms sum_h w*relu(s_h) for every query of the tile.
+constexpr int TC_KT = 8;                 // 128-key tiles per CTA
+constexpr int TC_SMEM = 80 * 1024;       // > 227/3 KB: at most 2 CTAs (2 x 256 TMEM columns) per SM
+constexpr long long TC_WAIT_CYCLES = 4000000000LL;   // ~2 s: bounded wait on the MMA barrier
+
+__device__ __forceinline__ int tc_core_off(int row, int chunk, int di) {
+    return (row >> 3) * (8 * di) + chunk * 128 + (row & 7) * 16;
+}
+
+template <int HI, int DI>
+__global__ void __launch_bounds__(128) idx_score_tc_kernel(const IdxScoreParams p) {
+    constexpr int NCOL = 256;                // N: (query, head) columns
+    constexpr int NQ = NCOL / HI;            // queries per CTA
+    constexpr int CH = DI / 16;              // 16-byte chunks per row
+    constexpr int A_BYTES = 128 * DI;
+    constexpr int B_BYTES = NCOL * DI;
+    static_assert(2 * A_BYTES + B_BYTES + NCOL * 4 + 64 <= TC_SMEM, "smem");
+    constexpr uint32_t IDESC = tc::make_idesc(2 /*s32*/, 1 /*s8*/, 128, NCOL);
+
+    extern __shared__ __align__(1024) unsigned char smem[];
+    unsigned char *a_s = smem;                               // 2 x A tile
+    unsigned char *b_s = smem + 2 * A_BYTES;                 // B tile
+    int *w_s = reinterpret_cast<int *>(b_s + B_BYTES);       // [NCOL]
+    uint64_t *bar = reinterpret_cast<uint64_t *>(w_s + NCOL);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + 1);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int b = blockIdx.z;
+    const int tq0 = p.t0 + blockIdx.y * NQ;
+    const int t_last = min(p.t0 + p.Rt, p.Tq) - 1;
+    const int tq_last = min(tq0 + NQ - 1, t_last);
+    if (tq0 > t_last) return;
+    const long long ncand_last = n_candidates(p.q_pos0 + tq_last, p.window);
+    const int j_cta = blockIdx.x * TC_KT * 128;
+    if ((long long)j_cta >= ncand_last) return;              // above the diagonal (uniform)
+    const int n_tiles = (int)min((long long)TC_KT, (ncand_last - j_cta + 127) / 128);
+
+    if (warp == 0) {
+        tc::tmem_alloc(tmem_slot, NCOL);
+        tc::tmem_relinquish();
+    }
+    if (tid == 0) {
+        tc::mbar_init(bar, 1);
+        tc::mbar_fence_init();
+    }
+    // B tile: rows (q, h) of q_idx are contiguous in memory
+    {
+        const int8_t *src = p.q + (((long long)b * p.Tq + tq0) * HI) * DI;
+        const int nrows_valid = (tq_last - tq0 + 1) * HI;
+        for (int i = tid; i < NCOL * CH; i += 128) {
+            const int row = i / CH, c = i % CH;
+            const bool ok = row < nrows_valid;
+            cp_async16(b_s + tc_core_off(row, c, DI), ok ? src + (long long)row * DI + c * 16 : src, ok ? 16 : 0);
+        }
+        for (int i = tid; i < NCOL; i += 128) {
+            const int tq = tq0 + i / HI;
+            w_s[i] = tq <= tq_last ? __ldg(p.w + ((long long)b * p.Tq + tq) * HI + i % HI) : 0;
+        }
+    }
+    auto load_a = [&](int kt) {
+        unsigned char *dst = a_s + (kt & 1) * A_BYTES;
+        const int j0 = j_cta + kt * 128;
+        const int8_t *src = p.k + ((long long)b * p.L) * DI;
+        for (int i = tid; i < 128 * CH; i += 128) {
+            const int row = i / CH, c = i % CH;
+            const int j = j0 + row;
+            const bool ok = j < p.L;
+            cp_async16(dst + tc_core_off(row, c, DI), ok ? src + (long long)j * DI + c * 16 : src, ok ? 16 : 0);
+        }
+        cp_async_commit();
+    };
+    load_a(0);
+    cp_async_wait<0>();
+    tc::fence_proxy_async_smem();
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+
+    bool timed_out = false;
+    uint32_t pending = 0;   // parity of the MMA batch in flight
+    for (int kt = 0; kt < n_tiles; ++kt) {
+        pending = kt & 1;
+        if (tid == 0) {
+            const uint32_t a_addr = tc::smem_u32(a_s + (kt & 1) * A_BYTES);
+            const uint32_t b_addr = tc::smem_u32(b_s);
+#pragma unroll
+            for (int kk = 0; kk < DI / 32; ++kk) {
+                // K = 32 bytes per MMA = two core matrices along K
+                const uint64_t ad = tc::desc_noswizzle(a_addr + kk * 256, 128, 8 * DI);
+                const uint64_t bd = tc::desc_noswizzle(b_addr + kk * 256, 128, 8 * DI);
+                tc::mma_i8(tmem, ad, bd, IDESC, kk > 0 ? 1u : 0u);
+            }
+            tc::mma_commit(bar);
+        }
+        if (kt + 1 < n_tiles) load_a(kt + 1);                  // other buffer: its MMA is done
+        if (!tc::mbar_wait_bounded(bar, kt & 1, TC_WAIT_CYCLES)) {
+            timed_out = true;
+            raise_error(p.err, ERR_TIMEOUT);
+            break;
+        }
+        tc::fence_after_sync();
+
+        // epilogue: this thread's key row, every query of the tile
+        const int j = j_cta + kt * 128 + warp * 32 + lane;
+        const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+#pragma unroll 1
+        for (int c0 = 0; c0 < NCOL; c0 += 16) {
+            uint32_t r[16];
+            tc::tmem_ld16(trow + c0, r);
+            tc::tmem_ld_wait();
+            if constexpr (HI >= 16) {
+                // one query spans HI/16 loads: accumulate into the first
+                int sc = 0;
+#pragma unroll
+                for (int u = 0; u < 16; ++u) sc += w_s[c0 + u] * max((int)r[u], 0);
+                const int q = c0 / HI;
+                const int tq = tq0 + q;
+                // HI == 16: exactly one load per query
+                if (tq <= tq_last && (long long)j < n_candidates(p.q_pos0 + tq, p.window))
+                    p.scores[((long long)b * p.Rt + (tq - p.t0)) * p.ld + j] = sc;
+            } else {
+#pragma unroll
+                for (int qq = 0; qq < 16 / HI; ++qq) {
+                    int sc = 0;
+#pragma unroll
+                    for (int h = 0; h < HI; ++h) sc += w_s[c0 + qq * HI + h] * max((int)r[qq * HI + h], 0);
+                    const int tq = tq0 + (c0 / HI) + qq;
+                    if (tq <= tq_last && (long long)j < n_candidates(p.q_pos0 + tq, p.window))
+                        p.scores[((long long)b * p.Rt + (tq - p.t0)) * p.ld + j] = sc;
+                }
+            }
+        }
+        // the next MMA overwrites the accumulator and reads the other A buffer
+        tc::fence_before_sync();
+        cp_async_wait<0>();
+        tc::fence_proxy_async_smem();
+        __syncthreads();
+        tc::fence_after_sync();
+    }
+    if (timed_out) {
+        cp_async_wait<0>();
+        // give the tensor core a bounded chance to finish before freeing TMEM
+        tc::mbar_wait_bounded(bar, pending, TC_WAIT_CYCLES / 4);
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tmem, NCOL);
 }
 
 // ------------------------------------------------------------- top-k select --
@@ -189,13 +349,15 @@ struct SelectParams {
     int B, Tq, t0, Rt;
     long long q_pos0;
     int topk, window, Kout;
+    int seg_cap;             // ints of the shared-memory segment buffer (multiple of 4)
     int32_t *out_idx;        // [B, Tq, Kout]
     int32_t *out_count;      // [B, Tq] nullable
 };
 
 constexpr int SEL_THREADS = 512;
-constexpr int SEL_BITS = 12;
+constexpr int SEL_BITS = 11;
 constexpr int SEL_BINS = 1 << SEL_BITS;
+constexpr int SEL_SEG_MAX = 40960;       // largest per-CTA segment (160 KB of int32)
 
 // Inclusive block scan (sum) of one int per thread; `tmp` holds 32 ints.
 __device__ __forceinline__ int block_incl_scan(int v, int *tmp) {
@@ -222,16 +384,21 @@ __device__ __forceinline__ int block_incl_scan(int v, int *tmp) {
     return v + add;
 }
 
+// One cluster per query row; CTA `rank` owns candidates [lo, hi) of the row,
+// held in shared memory for every pass.
 __global__ void __launch_bounds__(SEL_THREADS) topk_select_kernel(const SelectParams p) {
     cg::cluster_group cluster = cg::this_cluster();
     const int C = (int)cluster.num_blocks();
     const int rank = (int)cluster.block_rank();
 
+    extern __shared__ __align__(1024) unsigned char smem[];
+    int *seg_s = reinterpret_cast<int *>(smem);       // [seg_cap]
     __shared__ int hist[2][SEL_BINS];
     __shared__ int red[4];            // local min, max, n_gt, n_eq
     __shared__ int wcnt[2][SEL_THREADS / 32];
     __shared__ int scan_tmp[32];
     __shared__ int bcast[4];
+    __shared__ long long base[2];
 
     const int b = blockIdx.z, tr = blockIdx.y, t = p.t0 + tr;
     if (t >= p.Tq || tr >= p.Rt) return;     // uniform for the whole cluster
@@ -251,9 +418,11 @@ __global__ void __launch_bounds__(SEL_THREADS) topk_select_kernel(const SelectPa
         }
         if (tid == 0 && p.out_count) p.out_count[(long long)b * p.Tq + t] = k_eff + wc;
     }
-    const long long seg = (n + C - 1) / C;
+    // segment of this CTA: a multiple of 4 long so 16-byte loads stay aligned
+    const long long seg = ((n + C - 1) / C + 3) / 4 * 4;
     const long long lo = rank * seg < n ? rank * seg : n;
     const long long hi = lo + seg < n ? lo + seg : n;
+    const int cnt = (int)(hi - lo);
 
     if (k_eff == n) {                          // every candidate is kept
         for (long long j = lo + tid; j < hi; j += blockDim.x) orow[j] = (int)j;
@@ -261,12 +430,36 @@ __global__ void __launch_bounds__(SEL_THREADS) topk_select_kernel(const SelectPa
     }
     if (k_eff == 0) return;
 
-    // 1. min / max of the row
+    // 1. load the segment into shared memory (batched 16-byte loads) + min/max
     int vmin = INT_MAX, vmax = INT_MIN;
-    for (long long j = lo + tid; j < hi; j += blockDim.x) {
-        const int v = __ldg(srow + j);
-        vmin = min(vmin, v);
-        vmax = max(vmax, v);
+    {
+        const int n4 = cnt / 4;
+        const int4 *src4 = reinterpret_cast<const int4 *>(srow + lo);
+        int4 *dst4 = reinterpret_cast<int4 *>(seg_s);
+        constexpr int U = 8;
+        for (int base4 = tid; base4 < n4; base4 += SEL_THREADS * U) {
+            int4 v[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int i = base4 + u * SEL_THREADS;
+                if (i < n4) v[u] = __ldg(src4 + i);
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int i = base4 + u * SEL_THREADS;
+                if (i < n4) {
+                    dst4[i] = v[u];
+                    vmin = min(vmin, min(min(v[u].x, v[u].y), min(v[u].z, v[u].w)));
+                    vmax = max(vmax, max(max(v[u].x, v[u].y), max(v[u].z, v[u].w)));
+                }
+            }
+        }
+        for (int i = n4 * 4 + tid; i < cnt; i += SEL_THREADS) {
+            const int v = __ldg(srow + lo + i);
+            seg_s[i] = v;
+            vmin = min(vmin, v);
+            vmax = max(vmax, v);
+        }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -291,9 +484,9 @@ __global__ void __launch_bounds__(SEL_THREADS) topk_select_kernel(const SelectPa
     const unsigned range = (unsigned)((long long)gmax - (long long)gmin);
     const int nbits = range == 0 ? 0 : 32 - __clz(range);
 
-    // 2. radix passes over u = v - gmin, 12-bit digits from the top
+    // 2. radix passes over u = v - gmin, SEL_BITS-bit digits from the top
     unsigned long long prefix = 0;   // determined high bits of the threshold key
-    int known = nbits;               // bits at and above `known` are determined (all zero above nbits)
+    int known = nbits;               // bits at and above `known` are determined
     int k_rem = k_eff;               // how many still to take at/below the current prefix
     int pass = 0;
     while (known > 0) {
@@ -302,21 +495,21 @@ __global__ void __launch_bounds__(SEL_THREADS) topk_select_kernel(const SelectPa
         int *h = hist[pass & 1];
         for (int i = tid; i < SEL_BINS; i += blockDim.x) h[i] = 0;
         __syncthreads();
-        for (long long j = lo + tid; j < hi; j += blockDim.x) {
-            const unsigned long long u = (unsigned long long)((long long)__ldg(srow + j) - gmin);
+        for (int i = tid; i < cnt; i += SEL_THREADS) {
+            const unsigned long long u = (unsigned long long)((long long)seg_s[i] - gmin);
             if ((u >> known) == prefix) atomicAdd(&h[(u >> shift) & ((1u << width) - 1u)], 1);
         }
         cluster.sync();
         // total histogram, then the digit whose suffix count first reaches k_rem
-        const int per = SEL_BINS / SEL_THREADS;   // bins per thread (8), highest bins first
-        int cnt[SEL_BINS / SEL_THREADS];
+        constexpr int per = SEL_BINS / SEL_THREADS;   // bins per thread, highest bins first
+        int cntb[per];
         int local = 0;
 #pragma unroll
         for (int u = 0; u < per; ++u) {
             const int bin = SEL_BINS - 1 - (tid * per + u);
             int c = 0;
             for (int r = 0; r < C; ++r) c += cluster.map_shared_rank(h, r)[bin];
-            cnt[u] = c;
+            cntb[u] = c;
             local += c;
         }
         const int incl = block_incl_scan(local, scan_tmp);
@@ -324,11 +517,11 @@ __global__ void __launch_bounds__(SEL_THREADS) topk_select_kernel(const SelectPa
 #pragma unroll
         for (int u = 0; u < per; ++u) {
             const int bin = SEL_BINS - 1 - (tid * per + u);
-            if (above < k_rem && above + cnt[u] >= k_rem) {
+            if (above < k_rem && above + cntb[u] >= k_rem) {
                 bcast[2] = bin;
                 bcast[3] = above;
             }
-            above += cnt[u];
+            above += cntb[u];
         }
         __syncthreads();
         const int digit = bcast[2];
@@ -342,12 +535,12 @@ __global__ void __launch_bounds__(SEL_THREADS) topk_select_kernel(const SelectPa
 
     // 3. per-warp counts of (> thr) and (== thr) over warp sub-segments
     const int nw = blockDim.x >> 5, warp = tid >> 5, lane = tid & 31;
-    const long long wseg = ((hi - lo) + nw - 1) / nw;
-    const long long wlo = lo + warp * wseg < hi ? lo + warp * wseg : hi;
-    const long long whi = wlo + wseg < hi ? wlo + wseg : hi;
+    const int wseg = (cnt + nw - 1) / nw;
+    const int wlo = min(warp * wseg, cnt);
+    const int whi = min(wlo + wseg, cnt);
     int ngt = 0, neq = 0;
-    for (long long j = wlo + lane; j < whi; j += 32) {
-        const int v = __ldg(srow + j);
+    for (int i = wlo + lane; i < whi; i += 32) {
+        const int v = seg_s[i];
         ngt += v > thr;
         neq += v == thr;
     }
@@ -361,7 +554,6 @@ __global__ void __launch_bounds__(SEL_THREADS) topk_select_kernel(const SelectPa
         red[2] = a; red[3] = e;
     }
     cluster.sync();
-    __shared__ long long base[2];
     if (tid == 0) {
         long long gb = 0, eb = 0;
         for (int r = 0; r < rank; ++r) {
@@ -378,16 +570,16 @@ __global__ void __launch_bounds__(SEL_THREADS) topk_select_kernel(const SelectPa
     // keys, plus the earlier ties that are kept
     long long sel_base = gt_base + (eq_base < k_rem ? eq_base : k_rem);
     const unsigned lt = (1u << lane) - 1u;
-    for (long long j0 = wlo; j0 < whi; j0 += 32) {
-        const long long j = j0 + lane;
-        const int v = j < whi ? __ldg(srow + j) : INT_MIN;
-        const bool isg = j < whi && v > thr, ise = j < whi && v == thr;
+    for (int i0 = wlo; i0 < whi; i0 += 32) {
+        const int i = i0 + lane;
+        const int v = i < whi ? seg_s[i] : INT_MIN;
+        const bool isg = i < whi && v > thr, ise = i < whi && v == thr;
         const unsigned me = __ballot_sync(0xffffffffu, ise);
         const long long erank = eq_base + __popc(me & lt);
         const bool sel = isg || (ise && erank < k_rem);
         const unsigned ms = __ballot_sync(0xffffffffu, sel);
         const long long slot = sel_base + __popc(ms & lt);
-        if (sel && slot < k_eff) orow[slot] = (int)j;   // slot < k_eff by construction
+        if (sel && slot < k_eff) orow[slot] = (int)(lo + i);   // slot < k_eff by construction
         sel_base += __popc(ms);
         eq_base += __popc(me);
     }

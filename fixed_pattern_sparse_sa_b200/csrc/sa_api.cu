@@ -82,17 +82,22 @@ static int set_smem(K kernel, int bytes) {
 }
 
 // -------------------------------------------------------- gather launches --
+// Launch shape: 8 warps per CTA streaming 16-key chunks, 3 stages deep (a
+// 2-stage ring when the lo-key tile is also staged); 192 KB of shared memory,
+// one CTA and 8 gathering warps per SM.
 template <int D, int SRC, bool BIAS, bool KLO = false>
 static int launch_gather_t(const GatherParams &p, cudaStream_t st) {
-    constexpr int STAGES = D == 128 ? (KLO ? 2 : 3) : 4;
-    constexpr int smem = gather_smem_bytes<D, STAGES, KLO>();
-    auto kern = gather_attn_kernel<D, STAGES, SRC, BIAS, KLO>;
+    constexpr int NK = 16, NW = 8;
+    constexpr int STAGES = KLO ? 2 : 3;
+    constexpr int smem = gather_smem_bytes<D, STAGES, KLO, NK, NW>();
+    static_assert(smem <= 227 * 1024, "shared memory");
+    auto kern = gather_attn_kernel<D, STAGES, SRC, BIAS, KLO, NK, NW>;
     int rc = set_smem(kern, smem);
     if (rc) return rc;
     const long long items = (long long)p.B * p.Tq * p.Hkv * p.n_hchunk * p.n_split;
     if (items == 0) return SA_OK;
-    const long long blocks = (items + 3) / 4;
-    kern<<<(unsigned)blocks, 128, smem, st>>>(p);
+    const long long blocks = (items + NW - 1) / NW;
+    kern<<<(unsigned)blocks, NW * 32, smem, st>>>(p);
     SA_CHECK_LAUNCH("gather_attn_kernel");
     return SA_OK;
 }
@@ -163,9 +168,10 @@ int sa_check_device_status(void *stream) {
         const unsigned zero = 0;
         e = cudaMemcpy(ew, &zero, sizeof zero, cudaMemcpyHostToDevice);
         if (e != cudaSuccess) return fail(SA_ERR_CUDA, "clear error word: %s", cudaGetErrorString(e));
-        return fail(SA_ERR_DEVICE_ASSERT, "device error word 0x%x:%s%s", word,
+        return fail(SA_ERR_DEVICE_ASSERT, "device error word 0x%x:%s%s%s", word,
                     (word & ERR_BAD_INDEX) ? " index out of range or after the query position;" : "",
-                    (word & ERR_BAD_BLOCK) ? " NSA block id outside the sequence;" : "");
+                    (word & ERR_BAD_BLOCK) ? " NSA block id outside the sequence;" : "",
+                    (word & ERR_TIMEOUT) ? " a tensor-core barrier wait timed out;" : "");
     }
     return SA_OK;
 }
@@ -306,14 +312,14 @@ size_t sa_indexer_topk_workspace_size(int B, int Tq, int L, int Hi, int di, int 
 
 template <int HI, int DI>
 static int launch_score_t(const IdxScoreParams &p, int ncand_max, cudaStream_t st) {
-    constexpr int QT = 128 / HI;
-    const int smem = QT * 128 * 4 + QT * HI * 4;
-    auto kern = idx_score_kernel<HI, DI>;
-    int rc = set_smem(kern, smem);
+    constexpr int NQ = 256 / HI;
+    auto kern = idx_score_tc_kernel<HI, DI>;
+    int rc = set_smem(kern, TC_SMEM);
     if (rc) return rc;
-    dim3 grid((unsigned)((ncand_max + 127) / 128), (unsigned)((p.Rt + QT - 1) / QT), (unsigned)p.B);
-    kern<<<grid, 128, smem, st>>>(p);
-    SA_CHECK_LAUNCH("idx_score_kernel");
+    dim3 grid((unsigned)((ncand_max + TC_KT * 128 - 1) / (TC_KT * 128)), (unsigned)((p.Rt + NQ - 1) / NQ),
+              (unsigned)p.B);
+    kern<<<grid, 128, TC_SMEM, st>>>(p);
+    SA_CHECK_LAUNCH("idx_score_tc_kernel");
     return SA_OK;
 }
 
@@ -339,7 +345,9 @@ static int launch_select(const SelectParams &p, int cluster, cudaStream_t st) {
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3((unsigned)cluster, (unsigned)p.Rt, (unsigned)p.B);
     cfg.blockDim = dim3(SEL_THREADS, 1, 1);
-    cfg.dynamicSmemBytes = 0;
+    cfg.dynamicSmemBytes = (size_t)p.seg_cap * 4;
+    int rc = set_smem(topk_select_kernel, p.seg_cap * 4);
+    if (rc) return rc;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -376,6 +384,9 @@ int sa_indexer_topk(const int8_t *q_idx, const int8_t *k_idx, const int32_t *w, 
     if (!workspace || workspace_bytes < need)
         return fail(SA_ERR_WORKSPACE, "indexer_topk: workspace %zu < %zu", workspace_bytes, need);
     if (!aligned16(workspace)) return fail(SA_ERR_INVALID_ARG, "indexer_topk: workspace alignment");
+    unsigned *ew = nullptr;
+    int rc0 = device_error_word(&ew);
+    if (rc0) return rc0;
     cudaStream_t st = as_stream(stream);
     int32_t *scores = static_cast<int32_t *>(workspace);
     const int Kout = topk + window;
@@ -387,7 +398,7 @@ int sa_indexer_topk(const int8_t *q_idx, const int8_t *k_idx, const int32_t *w, 
             IdxScoreParams sp{};
             sp.q = q_idx; sp.k = k_idx; sp.w = w;
             sp.B = B; sp.Tq = Tq; sp.L = L; sp.q_pos0 = q_pos0; sp.window = window;
-            sp.t0 = t0; sp.Rt = rows; sp.ld = (long long)ld; sp.scores = scores;
+            sp.t0 = t0; sp.Rt = rows; sp.ld = (long long)ld; sp.scores = scores; sp.err = ew;
             int rc = launch_score(sp, Hi, di, (int)ncand, st);
             if (rc) return rc;
         }
@@ -396,10 +407,17 @@ int sa_indexer_topk(const int8_t *q_idx, const int8_t *k_idx, const int32_t *w, 
         se.B = B; se.Tq = Tq; se.t0 = t0; se.Rt = rows; se.q_pos0 = q_pos0;
         se.topk = topk; se.window = window; se.Kout = Kout;
         se.out_idx = out_idx; se.out_count = out_count;
-        // enough CTAs to fill the GPU: split short row lists across a cluster
+        // cluster size: every CTA's segment must fit in shared memory; split
+        // short row lists further so the launch fills the GPU
         const long long nrow = (long long)B * rows;
+        const long long nc = std::max(ncand, 1LL);
         int cluster = 1;
-        while (cluster < 8 && nrow * cluster < 296 && (long long)ncand / (cluster * 2) >= 4096) cluster *= 2;
+        while (cluster < 8 && (nc + cluster - 1) / cluster > SEL_SEG_MAX) cluster *= 2;
+        if ((nc + cluster - 1) / cluster > SEL_SEG_MAX)
+            return fail(SA_ERR_UNSUPPORTED, "indexer_topk: %lld candidates per query exceed %d",
+                        nc, 8 * SEL_SEG_MAX);
+        while (cluster < 8 && nrow * cluster < 296 && nc / (cluster * 2) >= 4096) cluster *= 2;
+        se.seg_cap = (int)((((nc + cluster - 1) / cluster) + 3) / 4 * 4);
         int rc = launch_select(se, cluster, st);
         if (rc) return rc;
     }

@@ -12,6 +12,7 @@ namespace sa {
 enum : unsigned {
     ERR_BAD_INDEX = 1u,       // index outside [0, L) or after the query position
     ERR_BAD_BLOCK = 2u,       // NSA block id outside the sequence
+    ERR_TIMEOUT = 4u,         // a bounded wait on the tensor-core barrier gave up
 };
 
 constexpr float kLog2e = 1.4426950408889634f;
