@@ -349,15 +349,16 @@ struct SelectParams {
     int B, Tq, t0, Rt;
     long long q_pos0;
     int topk, window, Kout;
-    int seg_cap;             // ints of the shared-memory segment buffer (multiple of 4)
+    int seg_cap;             // bitmap words per row buffer (>= ceil(n/32) for every row)
     int32_t *out_idx;        // [B, Tq, Kout]
     int32_t *out_count;      // [B, Tq] nullable
 };
 
-constexpr int SEL_THREADS = 512;
-constexpr int SEL_BITS = 11;
+constexpr int SEL_THREADS = 256;
+constexpr int SEL_BITS = 12;
 constexpr int SEL_BINS = 1 << SEL_BITS;
-constexpr int SEL_SEG_MAX = 40960;       // largest per-CTA segment (160 KB of int32)
+constexpr int SEL_TIE_CAP = 2048;        // boundary-bin entries resolved from a list
+constexpr int SEL_MAX_N = 1 << 20;       // candidates per row (bitmaps of n/8 bytes each)
 
 // Inclusive block scan (sum) of one int per thread; `tmp` holds 32 ints.
 __device__ __forceinline__ int block_incl_scan(int v, int *tmp) {
@@ -384,136 +385,123 @@ __device__ __forceinline__ int block_incl_scan(int v, int *tmp) {
     return v + add;
 }
 
-// One cluster per query row; CTA `rank` owns candidates [lo, hi) of the row,
-// held in shared memory for every pass.
-__global__ void __launch_bounds__(SEL_THREADS) topk_select_kernel(const SelectParams p) {
-    cg::cluster_group cluster = cg::this_cluster();
-    const int C = (int)cluster.num_blocks();
-    const int rank = (int)cluster.block_rank();
+__device__ __forceinline__ int block_sum(int v, int *tmp) {
+    v = warp_sum_int(v);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    __syncthreads();
+    if (lane == 0) tmp[warp] = v;
+    __syncthreads();
+    int t = 0;
+    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) t += tmp[i];
+    return t;
+}
 
+// Streams the row [0, n) from global memory (L2) with 16-byte loads, U
+// vectors in flight per thread; f(value, index) is called for every element.
+template <typename F>
+__device__ __forceinline__ void stream_row(const int32_t *row, int n, F f) {
+    constexpr int U = 4;
+    const int n4 = n / 4;
+    const int4 *r4 = reinterpret_cast<const int4 *>(row);
+    for (int b4 = threadIdx.x; b4 < n4; b4 += SEL_THREADS * U) {
+        int4 v[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int i = b4 + u * SEL_THREADS;
+            if (i < n4) v[u] = __ldg(r4 + i);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int i = b4 + u * SEL_THREADS;
+            if (i < n4) {
+                f(v[u].x, 4 * i); f(v[u].y, 4 * i + 1); f(v[u].z, 4 * i + 2); f(v[u].w, 4 * i + 3);
+            }
+        }
+    }
+    for (int i = n4 * 4 + (int)threadIdx.x; i < n; i += SEL_THREADS) f(__ldg(row + i), i);
+}
+
+// Exact top-k of one row, one CTA.  Keys are u = score - row_min (32-bit,
+// unsigned order = score order).  The boundary key is found by histogram
+// passes over the row: a 4096-bin histogram of u >> shift; the bin holding
+// the k-th largest key is refined until its width is 1 or it holds at most
+// SEL_TIE_CAP elements, which are then resolved exactly in shared memory.
+// Keys above the threshold go to a "greater" bitmap, keys equal to it to an
+// "equal" bitmap; the output takes every greater key and the lowest-index
+// equal keys, in ascending position order.
+__global__ void __launch_bounds__(SEL_THREADS) topk_select_kernel(const SelectParams p) {
     extern __shared__ __align__(1024) unsigned char smem[];
-    int *seg_s = reinterpret_cast<int *>(smem);       // [seg_cap]
-    __shared__ int hist[2][SEL_BINS];
-    __shared__ int red[4];            // local min, max, n_gt, n_eq
-    __shared__ int wcnt[2][SEL_THREADS / 32];
+    int *hist = reinterpret_cast<int *>(smem);                        // [SEL_BINS]
+    unsigned *tie_key = reinterpret_cast<unsigned *>(hist + SEL_BINS);  // [SEL_TIE_CAP]
+    int *tie_idx = reinterpret_cast<int *>(tie_key + SEL_TIE_CAP);     // [SEL_TIE_CAP]
+    unsigned *gt_bm = reinterpret_cast<unsigned *>(tie_idx + SEL_TIE_CAP);  // [words]
+    const int words_cap = p.seg_cap;                                     // bitmap words
+    unsigned *eq_bm = gt_bm + words_cap;
     __shared__ int scan_tmp[32];
     __shared__ int bcast[4];
-    __shared__ long long base[2];
+    __shared__ int tie_n;
 
     const int b = blockIdx.z, tr = blockIdx.y, t = p.t0 + tr;
-    if (t >= p.Tq || tr >= p.Rt) return;     // uniform for the whole cluster
+    if (t >= p.Tq || tr >= p.Rt) return;
     const long long pos = p.q_pos0 + t;
-    const long long n = n_candidates(pos, p.window);
+    const int n = (int)n_candidates(pos, p.window);
     const int wc = p.window > 0 ? (int)(pos + 1 < p.window ? pos + 1 : p.window) : 0;
-    const int k_eff = (int)(n < p.topk ? n : p.topk);
+    const int k_eff = n < p.topk ? n : p.topk;
     int32_t *orow = p.out_idx + ((long long)b * p.Tq + t) * p.Kout;
     const int32_t *srow = p.scores + ((long long)b * p.Rt + tr) * p.ld;
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
-    // window entries, padding and count (rank 0 only)
-    if (rank == 0) {
-        for (int i = tid; i < p.Kout - k_eff; i += blockDim.x) {
-            const int o = k_eff + i;
-            orow[o] = i < wc ? (int)(pos - wc + 1 + i) : -1;
-        }
-        if (tid == 0 && p.out_count) p.out_count[(long long)b * p.Tq + t] = k_eff + wc;
-    }
-    // segment of this CTA: a multiple of 4 long so 16-byte loads stay aligned
-    const long long seg = ((n + C - 1) / C + 3) / 4 * 4;
-    const long long lo = rank * seg < n ? rank * seg : n;
-    const long long hi = lo + seg < n ? lo + seg : n;
-    const int cnt = (int)(hi - lo);
-
-    if (k_eff == n) {                          // every candidate is kept
-        for (long long j = lo + tid; j < hi; j += blockDim.x) orow[j] = (int)j;
+    // window entries, padding and count
+    for (int i = tid; i < p.Kout - k_eff; i += SEL_THREADS)
+        orow[k_eff + i] = i < wc ? (int)(pos - wc + 1 + i) : -1;
+    if (tid == 0 && p.out_count) p.out_count[(long long)b * p.Tq + t] = k_eff + wc;
+    if (k_eff == n) {                                 // every candidate is kept
+        for (int j = tid; j < n; j += SEL_THREADS) orow[j] = j;
         return;
     }
     if (k_eff == 0) return;
 
-    // 1. load the segment into shared memory (batched 16-byte loads) + min/max
+    // 1. row min / max
     int vmin = INT_MAX, vmax = INT_MIN;
-    {
-        const int n4 = cnt / 4;
-        const int4 *src4 = reinterpret_cast<const int4 *>(srow + lo);
-        int4 *dst4 = reinterpret_cast<int4 *>(seg_s);
-        constexpr int U = 8;
-        for (int base4 = tid; base4 < n4; base4 += SEL_THREADS * U) {
-            int4 v[U];
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int i = base4 + u * SEL_THREADS;
-                if (i < n4) v[u] = __ldg(src4 + i);
-            }
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int i = base4 + u * SEL_THREADS;
-                if (i < n4) {
-                    dst4[i] = v[u];
-                    vmin = min(vmin, min(min(v[u].x, v[u].y), min(v[u].z, v[u].w)));
-                    vmax = max(vmax, max(max(v[u].x, v[u].y), max(v[u].z, v[u].w)));
-                }
-            }
-        }
-        for (int i = n4 * 4 + tid; i < cnt; i += SEL_THREADS) {
-            const int v = __ldg(srow + lo + i);
-            seg_s[i] = v;
-            vmin = min(vmin, v);
-            vmax = max(vmax, v);
-        }
-    }
+    stream_row(srow, n, [&](int v, int) { vmin = min(vmin, v); vmax = max(vmax, v); });
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
         vmin = min(vmin, __shfl_xor_sync(0xffffffffu, vmin, o));
         vmax = max(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
     }
-    if (tid == 0) { red[0] = INT_MAX; red[1] = INT_MIN; }
+    if (tid == 0) { bcast[0] = INT_MAX; bcast[1] = INT_MIN; }
     __syncthreads();
-    if ((tid & 31) == 0) { atomicMin(&red[0], vmin); atomicMax(&red[1], vmax); }
-    cluster.sync();
-    if (tid == 0) {
-        int mn = INT_MAX, mx = INT_MIN;
-        for (int r = 0; r < C; ++r) {
-            const int *rr = cluster.map_shared_rank(red, r);
-            mn = min(mn, rr[0]);
-            mx = max(mx, rr[1]);
-        }
-        bcast[0] = mn; bcast[1] = mx;
-    }
+    if (lane == 0) { atomicMin(&bcast[0], vmin); atomicMax(&bcast[1], vmax); }
     __syncthreads();
-    const int gmin = bcast[0], gmax = bcast[1];
-    const unsigned range = (unsigned)((long long)gmax - (long long)gmin);
+    const int gmin = bcast[0];
+    const unsigned range = (unsigned)bcast[1] - (unsigned)gmin;
     const int nbits = range == 0 ? 0 : 32 - __clz(range);
 
-    // 2. radix passes over u = v - gmin, SEL_BITS-bit digits from the top
-    unsigned long long prefix = 0;   // determined high bits of the threshold key
-    int known = nbits;               // bits at and above `known` are determined
-    int k_rem = k_eff;               // how many still to take at/below the current prefix
-    int pass = 0;
-    while (known > 0) {
-        const int shift = known > SEL_BITS ? known - SEL_BITS : 0;
-        const int width = known - shift;
-        int *h = hist[pass & 1];
-        for (int i = tid; i < SEL_BINS; i += blockDim.x) h[i] = 0;
+    // 2. histogram refinement: [lo_key, lo_key + 2^width) holds the k-th key
+    unsigned lo_key = 0;
+    int width = nbits;                // bits still undetermined
+    int k_rem = k_eff;                // keys to take at or below lo_key's bin
+    int bin_count = n;                // elements inside the current bin
+    while (width > 0 && (width > SEL_BITS || bin_count > SEL_TIE_CAP)) {
+        const int shift = width > SEL_BITS ? width - SEL_BITS : 0;
+        for (int i = tid; i < SEL_BINS; i += SEL_THREADS) hist[i] = 0;
         __syncthreads();
-        for (int i = tid; i < cnt; i += SEL_THREADS) {
-            const unsigned long long u = (unsigned long long)((long long)seg_s[i] - gmin);
-            if ((u >> known) == prefix) atomicAdd(&h[(u >> shift) & ((1u << width) - 1u)], 1);
-        }
-        cluster.sync();
-        // total histogram, then the digit whose suffix count first reaches k_rem
-        constexpr int per = SEL_BINS / SEL_THREADS;   // bins per thread, highest bins first
+        const unsigned hi_key = lo_key + (width >= 32 ? 0xffffffffu : ((1u << width) - 1u));
+        stream_row(srow, n, [&](int v, int) {
+            const unsigned key = (unsigned)v - (unsigned)gmin;
+            if (key >= lo_key && key <= hi_key) atomicAdd(&hist[(key - lo_key) >> shift], 1);
+        });
+        __syncthreads();
+        constexpr int per = SEL_BINS / SEL_THREADS;   // bins per thread, highest first
         int cntb[per];
         int local = 0;
 #pragma unroll
         for (int u = 0; u < per; ++u) {
-            const int bin = SEL_BINS - 1 - (tid * per + u);
-            int c = 0;
-            for (int r = 0; r < C; ++r) c += cluster.map_shared_rank(h, r)[bin];
-            cntb[u] = c;
-            local += c;
+            cntb[u] = hist[SEL_BINS - 1 - (tid * per + u)];
+            local += cntb[u];
         }
         const int incl = block_incl_scan(local, scan_tmp);
-        int above = incl - local;                 // count in strictly higher bins
+        int above = incl - local;
 #pragma unroll
         for (int u = 0; u < per; ++u) {
             const int bin = SEL_BINS - 1 - (tid * per + u);
@@ -524,66 +512,124 @@ __global__ void __launch_bounds__(SEL_THREADS) topk_select_kernel(const SelectPa
             above += cntb[u];
         }
         __syncthreads();
-        const int digit = bcast[2];
+        const int bin = bcast[2];
         k_rem -= bcast[3];
-        prefix = (prefix << width) | (unsigned long long)digit;
-        known = shift;
-        ++pass;
+        bin_count = hist[bin];
+        lo_key += (unsigned)bin << shift;
+        width = shift;
         __syncthreads();
     }
-    const long long thr = (long long)gmin + (long long)prefix;   // exact k-th largest score
 
-    // 3. per-warp counts of (> thr) and (== thr) over warp sub-segments
-    const int nw = blockDim.x >> 5, warp = tid >> 5, lane = tid & 31;
-    const int wseg = (cnt + nw - 1) / nw;
-    const int wlo = min(warp * wseg, cnt);
-    const int whi = min(wlo + wseg, cnt);
-    int ngt = 0, neq = 0;
-    for (int i = wlo + lane; i < whi; i += 32) {
-        const int v = seg_s[i];
-        ngt += v > thr;
-        neq += v == thr;
-    }
-    ngt = warp_sum_int(ngt);
-    neq = warp_sum_int(neq);
-    if (lane == 0) { wcnt[0][warp] = ngt; wcnt[1][warp] = neq; }
+    // 3. filter pass: bitmaps of keys above the bin; the bin's own elements
+    //    go to the equal bitmap (width 0) or to the tie list
+    const int words = (n + 31) / 32;
+    for (int i = tid; i < words; i += SEL_THREADS) { gt_bm[i] = 0u; eq_bm[i] = 0u; }
+    if (tid == 0) tie_n = 0;
     __syncthreads();
-    if (tid == 0) {
-        int a = 0, e = 0;
-        for (int i = 0; i < nw; ++i) { a += wcnt[0][i]; e += wcnt[1][i]; }
-        red[2] = a; red[3] = e;
-    }
-    cluster.sync();
-    if (tid == 0) {
-        long long gb = 0, eb = 0;
-        for (int r = 0; r < rank; ++r) {
-            const int *rr = cluster.map_shared_rank(red, r);
-            gb += rr[2];
-            eb += rr[3];
+    const unsigned bin_hi = lo_key + (width >= 32 ? 0xffffffffu : ((1u << width) - 1u));
+    stream_row(srow, n, [&](int v, int j) {
+        const unsigned key = (unsigned)v - (unsigned)gmin;
+        if (key > bin_hi) {
+            atomicOr(&gt_bm[j >> 5], 1u << (j & 31));
+        } else if (key >= lo_key) {
+            if (width == 0) {
+                atomicOr(&eq_bm[j >> 5], 1u << (j & 31));
+            } else {
+                const int slot = atomicAdd(&tie_n, 1);
+                if (slot < SEL_TIE_CAP) { tie_key[slot] = key - lo_key; tie_idx[slot] = j; }
+            }
         }
-        base[0] = gb; base[1] = eb;
-    }
+    });
     __syncthreads();
-    long long gt_base = base[0], eq_base = base[1];
-    for (int i = 0; i < warp; ++i) { gt_base += wcnt[0][i]; eq_base += wcnt[1][i]; }
-    // output slot of the first selected key of this warp: all earlier > thr
-    // keys, plus the earlier ties that are kept
-    long long sel_base = gt_base + (eq_base < k_rem ? eq_base : k_rem);
-    const unsigned lt = (1u << lane) - 1u;
-    for (int i0 = wlo; i0 < whi; i0 += 32) {
-        const int i = i0 + lane;
-        const int v = i < whi ? seg_s[i] : INT_MIN;
-        const bool isg = i < whi && v > thr, ise = i < whi && v == thr;
-        const unsigned me = __ballot_sync(0xffffffffu, ise);
-        const long long erank = eq_base + __popc(me & lt);
-        const bool sel = isg || (ise && erank < k_rem);
-        const unsigned ms = __ballot_sync(0xffffffffu, sel);
-        const long long slot = sel_base + __popc(ms & lt);
-        if (sel && slot < k_eff) orow[slot] = (int)(lo + i);   // slot < k_eff by construction
-        sel_base += __popc(ms);
-        eq_base += __popc(me);
+    // 4. resolve the tie list: exact threshold inside the bin (width <= 12 bits)
+    if (width > 0) {
+        const int m = min(tie_n, SEL_TIE_CAP);
+        for (int i = tid; i < SEL_BINS; i += SEL_THREADS) hist[i] = 0;
+        __syncthreads();
+        for (int i = tid; i < m; i += SEL_THREADS) atomicAdd(&hist[tie_key[i]], 1);
+        __syncthreads();
+        constexpr int per = SEL_BINS / SEL_THREADS;
+        int cntb[per];
+        int local = 0;
+#pragma unroll
+        for (int u = 0; u < per; ++u) {
+            cntb[u] = hist[SEL_BINS - 1 - (tid * per + u)];
+            local += cntb[u];
+        }
+        const int incl = block_incl_scan(local, scan_tmp);
+        int above = incl - local;
+#pragma unroll
+        for (int u = 0; u < per; ++u) {
+            const int bin = SEL_BINS - 1 - (tid * per + u);
+            if (above < k_rem && above + cntb[u] >= k_rem) {
+                bcast[2] = bin;
+                bcast[3] = above;
+            }
+            above += cntb[u];
+        }
+        __syncthreads();
+        const unsigned thr_off = (unsigned)bcast[2];
+        k_rem -= bcast[3];
+        for (int i = tid; i < m; i += SEL_THREADS) {
+            const int j = tie_idx[i];
+            if (tie_key[i] > thr_off) atomicOr(&gt_bm[j >> 5], 1u << (j & 31));
+            else if (tie_key[i] == thr_off) atomicOr(&eq_bm[j >> 5], 1u << (j & 31));
+        }
+        __syncthreads();
     }
-    cluster.sync();   // keep shared memory alive until every remote read is done
+
+    // 5. ordered output: warps own contiguous word ranges
+    constexpr int NW = SEL_THREADS / 32;
+    const int wpw = (words + NW - 1) / NW;
+    const int w_lo = min(warp * wpw, words), w_hi = min(w_lo + wpw, words);
+    int gcnt = 0, ecnt = 0;
+    for (int i = w_lo + lane; i < w_hi; i += 32) { gcnt += __popc(gt_bm[i]); ecnt += __popc(eq_bm[i]); }
+    gcnt = warp_sum_int(gcnt);
+    ecnt = warp_sum_int(ecnt);
+    __shared__ int wg[NW], we[NW];
+    if (lane == 0) { wg[warp] = gcnt; we[warp] = ecnt; }
+    __syncthreads();
+    int g_before = 0, e_before = 0;
+    for (int i = 0; i < warp; ++i) { g_before += wg[i]; e_before += we[i]; }
+    int out_base = g_before + min(e_before, k_rem);
+    const unsigned lt = (1u << lane) - 1u;
+    for (int i0 = w_lo; i0 < w_hi; i0 += 32) {
+        const int i = i0 + lane;
+        const unsigned gw = i < w_hi ? gt_bm[i] : 0u;
+        const unsigned ew = i < w_hi ? eq_bm[i] : 0u;
+        // equal keys are taken in index order until k_rem are used
+        const int ec = __popc(ew);
+        int e_incl = ec;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int x = __shfl_up_sync(0xffffffffu, e_incl, o);
+            if (lane >= o) e_incl += x;
+        }
+        const int e_pre = e_before + e_incl - ec;           // equal keys before this word
+        int take = k_rem - e_pre;
+        take = take < 0 ? 0 : (take > ec ? ec : take);
+        unsigned em = 0u, rest = ew;
+        for (int c = 0; c < take; ++c) { const unsigned lowbit = rest & (~rest + 1u); em |= lowbit; rest ^= lowbit; }
+        const unsigned sw = gw | em;
+        const int sc = __popc(sw);
+        int s_incl = sc;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int x = __shfl_up_sync(0xffffffffu, s_incl, o);
+            if (lane >= o) s_incl += x;
+        }
+        int slot = out_base + s_incl - sc;
+        unsigned bits = sw;
+        while (bits) {
+            const int bpos = __ffs(bits) - 1;
+            bits &= bits - 1u;
+            if (slot < k_eff) orow[slot] = i * 32 + bpos;   // slot < k_eff by construction
+            ++slot;
+        }
+        out_base += __shfl_sync(0xffffffffu, s_incl, 31);
+        e_before += __shfl_sync(0xffffffffu, e_incl, 31);
+    }
+    (void)lt;
 }
 
 }  // namespace sa

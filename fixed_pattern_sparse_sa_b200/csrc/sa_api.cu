@@ -341,23 +341,12 @@ static int launch_score(const IdxScoreParams &p, int Hi, int di, int ncand_max, 
     return fail(SA_ERR_UNSUPPORTED, "indexer heads %d", Hi);
 }
 
-static int launch_select(const SelectParams &p, int cluster, cudaStream_t st) {
-    cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3((unsigned)cluster, (unsigned)p.Rt, (unsigned)p.B);
-    cfg.blockDim = dim3(SEL_THREADS, 1, 1);
-    cfg.dynamicSmemBytes = (size_t)p.seg_cap * 4;
-    int rc = set_smem(topk_select_kernel, p.seg_cap * 4);
+static int launch_select(const SelectParams &p, cudaStream_t st) {
+    const int smem = (SEL_BINS + 2 * SEL_TIE_CAP + 2 * p.seg_cap) * 4;
+    int rc = set_smem(topk_select_kernel, smem);
     if (rc) return rc;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)cluster;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, topk_select_kernel, p);
-    if (e != cudaSuccess) return fail(SA_ERR_CUDA, "topk_select_kernel: %s", cudaGetErrorString(e));
+    dim3 grid(1u, (unsigned)p.Rt, (unsigned)p.B);
+    topk_select_kernel<<<grid, SEL_THREADS, smem, st>>>(p);
     SA_CHECK_LAUNCH("topk_select_kernel");
     return SA_OK;
 }
@@ -407,18 +396,11 @@ int sa_indexer_topk(const int8_t *q_idx, const int8_t *k_idx, const int32_t *w, 
         se.B = B; se.Tq = Tq; se.t0 = t0; se.Rt = rows; se.q_pos0 = q_pos0;
         se.topk = topk; se.window = window; se.Kout = Kout;
         se.out_idx = out_idx; se.out_count = out_count;
-        // cluster size: every CTA's segment must fit in shared memory; split
-        // short row lists further so the launch fills the GPU
-        const long long nrow = (long long)B * rows;
         const long long nc = std::max(ncand, 1LL);
-        int cluster = 1;
-        while (cluster < 8 && (nc + cluster - 1) / cluster > SEL_SEG_MAX) cluster *= 2;
-        if ((nc + cluster - 1) / cluster > SEL_SEG_MAX)
-            return fail(SA_ERR_UNSUPPORTED, "indexer_topk: %lld candidates per query exceed %d",
-                        nc, 8 * SEL_SEG_MAX);
-        while (cluster < 8 && nrow * cluster < 296 && nc / (cluster * 2) >= 4096) cluster *= 2;
-        se.seg_cap = (int)((((nc + cluster - 1) / cluster) + 3) / 4 * 4);
-        int rc = launch_select(se, cluster, st);
+        if (nc > SEL_MAX_N)
+            return fail(SA_ERR_UNSUPPORTED, "indexer_topk: %lld candidates per query exceed %d", nc, SEL_MAX_N);
+        se.seg_cap = (int)((nc + 31) / 32);
+        int rc = launch_select(se, st);
         if (rc) return rc;
     }
     return SA_OK;
