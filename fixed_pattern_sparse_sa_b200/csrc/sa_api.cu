@@ -276,77 +276,108 @@ int sa_lse_combine(const float *part_o, const float *part_lse, int n_split, int6
 }
 
 // ------------------------------------------------------------- indexer --
-// Query rows per score chunk: the chunk's int32 scores stay within ~64 MiB so
-// that the select pass re-reads them from L2.
-static int indexer_chunk_rows(int B, int Tq, size_t ld, int Hi) {
-    const size_t budget = (size_t)64 << 20;
-    const int qt = 128 / Hi;
-    size_t rows = budget / ((size_t)B * ld * 4);
-    if (rows < 1) rows = 1;
-    if (rows >= (size_t)qt) rows = rows / qt * qt;
-    if (rows > (size_t)Tq) rows = Tq;
-    if (rows > 65535) rows = 65535;   // grid.y limit of the select launch
-    return (int)rows;
-}
-
-static size_t indexer_ld(int Tq, int L, int64_t q_pos0, int window) {
-    long long pmax = q_pos0 + Tq - 1;
-    long long n = window > 0 ? pmax - window + 1 : pmax + 1;
-    if (n < 1) n = 1;
-    if (n > L) n = L;
-    return round_up((size_t)n, 4);
-}
+// Rows per chunk: sample scores, thresholds and candidate lists of a chunk
+// take about kIdxChunkBudget bytes of workspace.
+static constexpr size_t kIdxChunkBudget = (size_t)1 << 30;
 
 static bool indexer_shape_ok(int Hi, int di) {
     return (Hi == 1 || Hi == 2 || Hi == 4 || Hi == 8 || Hi == 16) && (di == 32 || di == 64 || di == 128);
 }
 
-size_t sa_indexer_topk_workspace_size(int B, int Tq, int L, int Hi, int di, int topk, int window) {
-    (void)di; (void)topk;
-    if (B <= 0 || Tq <= 0 || L <= 0 || !(Hi == 1 || Hi == 2 || Hi == 4 || Hi == 8 || Hi == 16)) return 0;
-    // the worst case over q_pos0 is q_pos0 = L - Tq
-    const size_t ld = indexer_ld(Tq, L, L - Tq, window);
-    const int rt = indexer_chunk_rows(B, Tq, ld, Hi);
-    return round_up((size_t)B * rt * ld * 4, 256);
+// Decode-like shapes (one or two queries per sequence) use a 16-column MMA
+// tile instead of 256 columns.
+static int indexer_ncol(int Tq, int Hi) { return (Tq * Hi <= 16 && Hi <= 8) ? 16 : 256; }
+
+static int indexer_m_cap(int nq_block) { return (int)round_up((size_t)(2 * SAMPLE_TARGET + nq_block), 4); }
+
+// Candidate list capacity per row: about k + 4 sigma entries are expected.
+static int indexer_cand_cap(int topk) { return (int)round_up((size_t)std::max(5120, topk * 5 / 2), 64); }
+
+static size_t indexer_row_bytes(int m_cap, int cap) { return (size_t)m_cap * 4 + 8 + (size_t)cap * 8; }
+
+static int indexer_chunk_rows(int B, int Tq, int nq_block, int m_cap, int cap) {
+    size_t rows = kIdxChunkBudget / ((size_t)B * indexer_row_bytes(m_cap, cap));
+    if (rows < 1) rows = 1;
+    if (rows >= (size_t)nq_block) rows = rows / nq_block * nq_block;
+    if (rows > (size_t)Tq) rows = Tq;
+    if (rows > 65535) rows = 65535;   // grid.y limit
+    return (int)rows;
 }
 
-template <int HI, int DI>
-static int launch_score_t(const IdxScoreParams &p, int ncand_max, cudaStream_t st) {
-    constexpr int NQ = 256 / HI;
-    auto kern = idx_score_tc_kernel<HI, DI>;
-    int rc = set_smem(kern, TC_SMEM);
+struct IdxLayout {
+    int ncol, nq, m_cap, cap, rt;
+    size_t sample_off, tau_off, cnt_off, val_off, idx_off, total;
+};
+
+static IdxLayout indexer_layout(int B, int Tq, int Hi, int topk) {
+    IdxLayout l{};
+    l.ncol = indexer_ncol(Tq, Hi);
+    l.nq = l.ncol / Hi;
+    l.m_cap = indexer_m_cap(l.nq);
+    l.cap = indexer_cand_cap(topk);
+    l.rt = indexer_chunk_rows(B, Tq, l.nq, l.m_cap, l.cap);
+    const size_t rows = (size_t)B * l.rt;
+    size_t off = 0;
+    l.sample_off = off; off += round_up(rows * l.m_cap * 4, 256);
+    l.tau_off = off; off += round_up(rows * 4, 256);
+    l.cnt_off = off; off += round_up(rows * 4, 256);
+    l.val_off = off; off += round_up(rows * l.cap * 4, 256);
+    l.idx_off = off; off += round_up(rows * l.cap * 4, 256);
+    l.total = off;
+    return l;
+}
+
+size_t sa_indexer_topk_workspace_size(int B, int Tq, int L, int Hi, int di, int topk, int window) {
+    (void)L; (void)di; (void)window;
+    if (B <= 0 || Tq <= 0 || topk < 0 || !(Hi == 1 || Hi == 2 || Hi == 4 || Hi == 8 || Hi == 16)) return 0;
+    return indexer_layout(B, Tq, Hi, topk).total;
+}
+
+template <int HI, int DI, int NCOL, int MODE>
+static int launch_score_t(const IdxParams &p, long long n_keys_max, cudaStream_t st) {
+    constexpr int NQ = NCOL / HI;
+    constexpr int smem = tc_smem_bytes<DI, NCOL>();
+    auto kern = idx_score_tc_kernel<HI, DI, NCOL, MODE>;
+    int rc = set_smem(kern, smem);
     if (rc) return rc;
-    dim3 grid((unsigned)((ncand_max + TC_KT * 128 - 1) / (TC_KT * 128)), (unsigned)((p.Rt + NQ - 1) / NQ),
+    dim3 grid((unsigned)((n_keys_max + TC_KT * 128 - 1) / (TC_KT * 128)), (unsigned)((p.Rt + NQ - 1) / NQ),
               (unsigned)p.B);
-    kern<<<grid, 128, TC_SMEM, st>>>(p);
+    kern<<<grid, TC_THREADS, smem, st>>>(p);
     SA_CHECK_LAUNCH("idx_score_tc_kernel");
     return SA_OK;
 }
 
-template <int HI>
-static int launch_score_hi(const IdxScoreParams &p, int di, int ncand_max, cudaStream_t st) {
-    if (di == 32) return launch_score_t<HI, 32>(p, ncand_max, st);
-    if (di == 64) return launch_score_t<HI, 64>(p, ncand_max, st);
-    return launch_score_t<HI, 128>(p, ncand_max, st);
-}
-
-static int launch_score(const IdxScoreParams &p, int Hi, int di, int ncand_max, cudaStream_t st) {
-    switch (Hi) {
-        case 1: return launch_score_hi<1>(p, di, ncand_max, st);
-        case 2: return launch_score_hi<2>(p, di, ncand_max, st);
-        case 4: return launch_score_hi<4>(p, di, ncand_max, st);
-        case 8: return launch_score_hi<8>(p, di, ncand_max, st);
-        case 16: return launch_score_hi<16>(p, di, ncand_max, st);
+template <int HI, int DI, int MODE>
+static int launch_score_n(const IdxParams &p, int ncol, long long n_keys_max, cudaStream_t st) {
+    if constexpr (HI <= 8) {
+        if (ncol == 16) return launch_score_t<HI, DI, 16, MODE>(p, n_keys_max, st);
     }
-    return fail(SA_ERR_UNSUPPORTED, "indexer heads %d", Hi);
+    return launch_score_t<HI, DI, 256, MODE>(p, n_keys_max, st);
 }
 
-static int launch_select(const SelectParams &p, cudaStream_t st) {
-    const int smem = (SEL_BINS + 2 * SEL_TIE_CAP + 2 * p.seg_cap) * 4;
-    int rc = set_smem(topk_select_kernel, smem);
+template <int MODE>
+static int launch_score(const IdxParams &p, int ncol, long long n_keys_max, cudaStream_t st) {
+#define SA_SCORE_DI(HI)                                                                 \
+    if (p.di == 32) return launch_score_n<HI, 32, MODE>(p, ncol, n_keys_max, st);      \
+    if (p.di == 64) return launch_score_n<HI, 64, MODE>(p, ncol, n_keys_max, st);      \
+    return launch_score_n<HI, 128, MODE>(p, ncol, n_keys_max, st);
+    switch (p.Hi) {
+        case 1: { SA_SCORE_DI(1) }
+        case 2: { SA_SCORE_DI(2) }
+        case 4: { SA_SCORE_DI(4) }
+        case 8: { SA_SCORE_DI(8) }
+        case 16: { SA_SCORE_DI(16) }
+    }
+#undef SA_SCORE_DI
+    return fail(SA_ERR_UNSUPPORTED, "indexer heads %d", p.Hi);
+}
+
+template <int DI>
+static int launch_select_t(const IdxParams &p, int words, cudaStream_t st) {
+    const int smem = select_smem_bytes<DI>(words);
+    int rc = set_smem(topk_select_kernel<DI>, smem);
     if (rc) return rc;
-    dim3 grid(1u, (unsigned)p.Rt, (unsigned)p.B);
-    topk_select_kernel<<<grid, SEL_THREADS, smem, st>>>(p);
+    topk_select_kernel<DI><<<dim3(1u, (unsigned)p.Rt, (unsigned)p.B), SEL_THREADS, smem, st>>>(p);
     SA_CHECK_LAUNCH("topk_select_kernel");
     return SA_OK;
 }
@@ -366,41 +397,48 @@ int sa_indexer_topk(const int8_t *q_idx, const int8_t *k_idx, const int32_t *w, 
         !aligned4(out_idx) || (out_count && !aligned4(out_count)))
         return fail(SA_ERR_INVALID_ARG, "indexer_topk: null or misaligned pointer");
     if (Tq == 0) return SA_OK;
-    // chunking is fixed by the worst case (q_pos0 = L - Tq), as in the size query
-    const size_t ld = indexer_ld(Tq, L, q_pos0, window);
-    const int rt = indexer_chunk_rows(B, Tq, indexer_ld(Tq, L, L - Tq, window), Hi);
-    const size_t need = round_up((size_t)B * rt * ld * 4, 256);
-    if (!workspace || workspace_bytes < need)
-        return fail(SA_ERR_WORKSPACE, "indexer_topk: workspace %zu < %zu", workspace_bytes, need);
+    const long long n_max_all = std::max(0LL, (long long)(window > 0 ? q_pos0 + Tq - window : q_pos0 + Tq));
+    if (n_max_all > SEL_MAX_N)
+        return fail(SA_ERR_UNSUPPORTED, "indexer_topk: %lld candidates per query exceed %d", n_max_all, SEL_MAX_N);
+    const IdxLayout lay = indexer_layout(B, Tq, Hi, topk);
+    if (!workspace || workspace_bytes < lay.total)
+        return fail(SA_ERR_WORKSPACE, "indexer_topk: workspace %zu < %zu", workspace_bytes, lay.total);
     if (!aligned16(workspace)) return fail(SA_ERR_INVALID_ARG, "indexer_topk: workspace alignment");
     unsigned *ew = nullptr;
-    int rc0 = device_error_word(&ew);
-    if (rc0) return rc0;
+    int rc = device_error_word(&ew);
+    if (rc) return rc;
     cudaStream_t st = as_stream(stream);
-    int32_t *scores = static_cast<int32_t *>(workspace);
-    const int Kout = topk + window;
-    for (int t0 = 0; t0 < Tq; t0 += rt) {
-        const int rows = std::min(rt, Tq - t0);
-        long long pmax = q_pos0 + t0 + rows - 1;
-        long long ncand = window > 0 ? pmax - window + 1 : pmax + 1;
+    char *ws = static_cast<char *>(workspace);
+
+    IdxParams p{};
+    p.q = q_idx; p.k = k_idx; p.w = w;
+    p.B = B; p.Tq = Tq; p.L = L; p.Hi = Hi; p.di = di;
+    p.q_pos0 = q_pos0; p.window = window; p.topk = topk; p.Kout = topk + window;
+    p.nq_block = lay.nq; p.m_cap = lay.m_cap; p.cand_cap = lay.cap;
+    p.sample = reinterpret_cast<int32_t *>(ws + lay.sample_off);
+    p.tau = reinterpret_cast<int32_t *>(ws + lay.tau_off);
+    p.cand_cnt = reinterpret_cast<int32_t *>(ws + lay.cnt_off);
+    p.cand_val = reinterpret_cast<int32_t *>(ws + lay.val_off);
+    p.cand_idx = reinterpret_cast<int32_t *>(ws + lay.idx_off);
+    p.out_idx = out_idx; p.out_count = out_count; p.err = ew;
+    for (int t0 = 0; t0 < Tq; t0 += lay.rt) {
+        const int rows = std::min(lay.rt, Tq - t0);
+        p.t0 = t0; p.Rt = rows;
+        const long long pmax = q_pos0 + t0 + rows - 1;
+        const long long ncand = std::max(0LL, window > 0 ? pmax - window + 1 : pmax + 1);
+        cudaError_t e = cudaMemsetAsync(p.cand_cnt, 0, (size_t)B * rows * 4, st);
+        if (e != cudaSuccess) return fail(SA_ERR_CUDA, "memset: %s", cudaGetErrorString(e));
         if (ncand > 0) {
-            IdxScoreParams sp{};
-            sp.q = q_idx; sp.k = k_idx; sp.w = w;
-            sp.B = B; sp.Tq = Tq; sp.L = L; sp.q_pos0 = q_pos0; sp.window = window;
-            sp.t0 = t0; sp.Rt = rows; sp.ld = (long long)ld; sp.scores = scores; sp.err = ew;
-            int rc = launch_score(sp, Hi, di, (int)ncand, st);
+            rc = launch_score<MODE_SAMPLE>(p, lay.ncol, (long long)lay.m_cap, st);
+            if (rc) return rc;
+            idx_threshold_kernel<<<dim3(1u, (unsigned)rows, (unsigned)B), SEL_THREADS, 0, st>>>(p);
+            SA_CHECK_LAUNCH("idx_threshold_kernel");
+            rc = launch_score<MODE_FILTER>(p, lay.ncol, ncand, st);
             if (rc) return rc;
         }
-        SelectParams se{};
-        se.scores = scores; se.ld = (long long)ld;
-        se.B = B; se.Tq = Tq; se.t0 = t0; se.Rt = rows; se.q_pos0 = q_pos0;
-        se.topk = topk; se.window = window; se.Kout = Kout;
-        se.out_idx = out_idx; se.out_count = out_count;
-        const long long nc = std::max(ncand, 1LL);
-        if (nc > SEL_MAX_N)
-            return fail(SA_ERR_UNSUPPORTED, "indexer_topk: %lld candidates per query exceed %d", nc, SEL_MAX_N);
-        se.seg_cap = (int)((nc + 31) / 32);
-        int rc = launch_select(se, st);
+        const int words = (int)((std::max(ncand, 1LL) + 31) / 32);
+        rc = di == 32 ? launch_select_t<32>(p, words, st)
+                      : di == 64 ? launch_select_t<64>(p, words, st) : launch_select_t<128>(p, words, st);
         if (rc) return rc;
     }
     return SA_OK;
