@@ -210,6 +210,21 @@ __global__ void __launch_bounds__(TC_THREADS) idx_score_tc_kernel(const IdxParam
 
     const int quad = warp & 3;                     // TMEM lane quadrant of this warp
     const int c_begin = (warp >> 2) * HALF;        // this warp's half of the columns
+    // per-query constants of this warp's queries, held in registers: the
+    // number of candidates (keys j < nt_q are scored) and the threshold
+    constexpr int NQH = HALF / HI;                 // queries in this warp's half
+    constexpr int GQ = NQH < 32 ? NQH : 32;        // queries per append group
+    int nt_r[GQ], tau_r[GQ];
+    auto load_query_consts = [&](int g0) {
+#pragma unroll
+        for (int q = 0; q < GQ; ++q) {
+            const int tq = tq0 + c_begin / HI + g0 + q;
+            const long long nt = tq <= tq_last ? n_candidates(p.q_pos0 + tq, p.window) : 0;
+            nt_r[q] = (int)min(nt, (long long)INT_MAX);
+            tau_r[q] = MODE == MODE_FILTER ? tau_s[c_begin / HI + g0 + q] : 0;
+        }
+    };
+    if (NQH == GQ) load_query_consts(0);
     bool timed_out = false;
     uint32_t pending = 0;   // parity of the MMA batch in flight
     for (int kt = 0; kt < n_tiles; ++kt) {
@@ -243,12 +258,11 @@ __global__ void __launch_bounds__(TC_THREADS) idx_score_tc_kernel(const IdxParam
         const int i_key = j_cta + kt * 128 + quad * 32 + lane;       // tile row -> key index
         const long long j = (long long)stride * i_key;
         const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
-        constexpr int NQH = HALF / HI;                   // queries in this warp's half
-        constexpr int GQ = NQH < 32 ? NQH : 32;          // queries per group
         constexpr int QPL = HI >= STEP ? 1 : STEP / HI;  // queries per TMEM load
         constexpr int HPL = HI >= STEP ? STEP : HI;      // heads of a query in a load
 #pragma unroll 1
         for (int g0 = 0; g0 < NQH; g0 += GQ) {
+            if (NQH != GQ) load_query_consts(g0);
             int sc[GQ];
 #pragma unroll
             for (int c = 0; c < GQ * HI; c += STEP) {
@@ -278,40 +292,34 @@ __global__ void __launch_bounds__(TC_THREADS) idx_score_tc_kernel(const IdxParam
                 }
             }
             const int q_first = c_begin / HI + g0;      // query index (within the CTA) of sc[0]
+            const int row0 = b * p.Rt + (tq0 + q_first - p.t0);   // list row of sc[0]
+            const int jj = (int)min(j, (long long)INT_MAX);
             if constexpr (MODE == MODE_SAMPLE) {
 #pragma unroll
-                for (int q = 0; q < GQ; ++q) {
-                    const int tq = tq0 + q_first + q;
-                    const long long nt = tq <= tq_last ? n_candidates(p.q_pos0 + tq, p.window) : 0;
-                    if (j < nt) p.sample[((long long)b * p.Rt + (tq - p.t0)) * p.m_cap + i_key] = sc[q];
-                }
+                for (int q = 0; q < GQ; ++q)
+                    if (jj < nt_r[q]) p.sample[(long long)(row0 + q) * p.m_cap + i_key] = sc[q];
             } else {
                 unsigned ball[GQ];
                 unsigned keepm = 0u;
                 int mycnt = 0;
 #pragma unroll
                 for (int q = 0; q < GQ; ++q) {
-                    const int tq = tq0 + q_first + q;
-                    const long long nt = tq <= tq_last ? n_candidates(p.q_pos0 + tq, p.window) : 0;
-                    const bool keep = j < nt && sc[q] >= tau_s[q_first + q];
+                    const bool keep = (jj < nt_r[q]) & (sc[q] >= tau_r[q]);
                     keepm |= keep ? (1u << q) : 0u;
                     ball[q] = __ballot_sync(0xffffffffu, keep);
-                    if (lane == q) mycnt = __popc(ball[q]);
+                    mycnt = lane == q ? __popc(ball[q]) : mycnt;
                 }
                 int base = 0;
-                if (lane < GQ && mycnt > 0) {
-                    const int tq = tq0 + q_first + lane;
-                    base = atomicAdd(p.cand_cnt + (long long)b * p.Rt + (tq - p.t0), mycnt);
-                }
+                if (mycnt > 0) base = atomicAdd(p.cand_cnt + row0 + lane, mycnt);   // lane q < GQ
+                const unsigned lt = (1u << lane) - 1u;
 #pragma unroll
                 for (int q = 0; q < GQ; ++q) {
                     if (ball[q] == 0u) continue;                           // warp-uniform
-                    const int bq = __shfl_sync(0xffffffffu, base, q);
-                    const int slot = bq + __popc(ball[q] & ((1u << lane) - 1u));
+                    const int slot = __shfl_sync(0xffffffffu, base, q) + __popc(ball[q] & lt);
                     if (((keepm >> q) & 1u) && slot < p.cand_cap) {
-                        const long long row = (long long)b * p.Rt + (tq0 + q_first + q - p.t0);
-                        p.cand_val[row * p.cand_cap + slot] = sc[q];
-                        p.cand_idx[row * p.cand_cap + slot] = (int)j;
+                        const long long off = (long long)(row0 + q) * p.cand_cap + slot;
+                        p.cand_val[off] = sc[q];
+                        p.cand_idx[off] = jj;
                     }
                 }
             }
@@ -334,8 +342,8 @@ __global__ void __launch_bounds__(TC_THREADS) idx_score_tc_kernel(const IdxParam
 }
 
 // ----------------------------------------------------- block helpers --
-constexpr int SEL_THREADS = 512;
-constexpr int SEL_BITS = 12;
+constexpr int SEL_THREADS = 256;
+constexpr int SEL_BITS = 8;
 constexpr int SEL_BINS = 1 << SEL_BITS;
 constexpr int SEL_TIE_CAP = 2048;        // boundary-bin entries resolved from a list
 constexpr int SEL_MAX_N = 768 * 1024;    // candidates per row (two bitmaps of n/8 bytes in shared memory)
@@ -466,7 +474,7 @@ __device__ __forceinline__ void stream_values(const int32_t *vals, int n, F f) {
 // chosen so that r/m of the n candidates (plus four standard deviations of a
 // sampling count) reach it.  A sample that is the whole row gives the exact
 // k-th largest score.  Rows whose every candidate is kept get INT_MIN.
-__global__ void __launch_bounds__(SEL_THREADS, 2) idx_threshold_kernel(const IdxParams p) {
+__global__ void __launch_bounds__(SEL_THREADS, 4) idx_threshold_kernel(const IdxParams p) {
     __shared__ int hist[SEL_BINS];
     __shared__ int scan_tmp[32];
     __shared__ int bcast[4];
@@ -535,7 +543,7 @@ __host__ __device__ constexpr int select_smem_bytes(int words) {
 // "equal" bitmap; the output takes every greater key and the lowest-position
 // equal keys, in ascending position order.
 template <int DI>
-__global__ void __launch_bounds__(SEL_THREADS, 2) topk_select_kernel(const IdxParams p) {
+__global__ void __launch_bounds__(SEL_THREADS, 4) topk_select_kernel(const IdxParams p) {
     extern __shared__ __align__(1024) unsigned char smem[];
     int *hist = reinterpret_cast<int *>(smem);                          // [SEL_BINS]
     unsigned *tie_key = reinterpret_cast<unsigned *>(hist + SEL_BINS);  // [SEL_TIE_CAP]
@@ -634,7 +642,7 @@ __global__ void __launch_bounds__(SEL_THREADS, 2) topk_select_kernel(const IdxPa
     });
     __syncthreads();
     int k_rem = st.k_rem;
-    if (width > 0) {   // resolve the tie list: exact threshold inside the bin (<= 12 bits)
+    if (width > 0) {   // resolve the tie list: exact threshold inside the bin (<= SEL_BITS bits)
         const int m = min(tie_n, SEL_TIE_CAP);
         RadixState ts{0u, width, k_rem, m};
         auto tie_each = [&](auto f) {
