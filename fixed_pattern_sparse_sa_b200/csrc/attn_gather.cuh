@@ -22,7 +22,9 @@ enum KeySource : int {
     KS_PATTERN = 1,  // fixed window + dilated powers of two
     KS_BLOCKS = 2,   // NSA selected blocks: idx holds block ids
     KS_RANGE = 3,    // recent window: j = p - window + 1 + e
-    KS_CMP = 4,      // NSA compressed tokens: i = e, visible iff i*stride+len-1 <= p
+    KS_PROWS = 4,    // fixed graph, rows = 16/G consecutive queries x G heads: the
+                     // union of their sets (window band + one 16/G-key segment per
+                     // dilated distance), masked per (row, key)
 };
 
 struct GatherParams {
@@ -35,11 +37,12 @@ struct GatherParams {
     const int32_t *idx;       // KS_IDX: [B,Tq,idx_heads,K]; KS_BLOCKS: [B,Tq,Hkv,K] block ids
     int idx_heads, K;
     int window, dilated;      // KS_PATTERN / KS_RANGE
-    int block;                // KS_BLOCKS block length; KS_CMP stride
-    int cmp_len;              // KS_CMP window length
+    int block;                // KS_BLOCKS block length
+    int cmp_len;              // unused by the gather kernel
     int entries;              // virtual list length per item
     int per_split;            // entries handled by one split piece
     int n_split, n_hchunk;
+    int q_units;              // query units of the item grid (Tq, or ceil(Tq/(16/G)) for KS_PROWS)
     const float *cq, *ck, *beta;   // optional coordinate bias
     float scale_log2;         // scale * log2(e)
     __nv_bfloat16 *out;       // [B,Tq,Hq,D] (n_split == 1)
@@ -84,10 +87,32 @@ __device__ __forceinline__ int key_raw(const GatherParams &p, int b, int t, int 
     } else if constexpr (SRC == KS_RANGE) {
         long long j = pos - p.window + 1 + e;
         return j < 0 ? -1 : (int)j;
-    } else {  // KS_CMP
-        long long end = (long long)e * p.block + p.cmp_len - 1;
-        return (end <= pos && e < p.Lk) ? e : -1;
+    } else {  // KS_PROWS: `pos` is the first query's position, see key_prows
+        return -1;
     }
+}
+
+// KS_PROWS: entry e of the union for queries at positions [pa, pb]; returns
+// the key (or -1) and, in seg, 0 for the window band or the dilated distance.
+__device__ __forceinline__ int key_prows(const GatherParams &p, long long pa, long long pb, int nqw, int e,
+                                         int e_end, int &seg) {
+    seg = 0;
+    if (e >= e_end) return -1;
+    const long long lo = pa - p.window + 1 > 0 ? pa - p.window + 1 : 0;
+    const long long nb = pb - lo + 1;
+    if (e < nb) return (int)(lo + e);
+    if (!p.dilated) return -1;
+    int i0 = 0;
+    while ((1LL << i0) < p.window) ++i0;
+    const long long e2 = e - nb;
+    const long long m = e2 / nqw, r = e2 % nqw;
+    if (i0 + m >= 62) return -1;
+    const long long o = 1LL << (i0 + m);
+    if (o >= pb) return -1;
+    const long long j = pa - o + r;
+    if (j < 0 || pa + r > pb) return -1;
+    seg = (int)o;
+    return (int)j;
 }
 
 template <int SRC>
@@ -131,10 +156,12 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
 
     extern __shared__ __align__(1024) unsigned char smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    unsigned char *wsm = smem + warp * (STAGES * (SB + NK * 4));
+    constexpr bool PR = SRC == KS_PROWS;
+    unsigned char *wsm = smem + warp * (STAGES * (SB + NK * (PR ? 8 : 4)));
     int *keys_s = reinterpret_cast<int *>(wsm + STAGES * SB);
+    int *segs_s = keys_s + STAGES * NK;                      // KS_PROWS only
 
-    const long long n_items = (long long)p.B * p.Tq * p.Hkv * p.n_hchunk * p.n_split;
+    const long long n_items = (long long)p.B * p.q_units * p.Hkv * p.n_hchunk * p.n_split;
     const long long item = (long long)blockIdx.x * NW + warp;
     if (item >= n_items) return;   // warps are independent: no block barrier below
 
@@ -142,16 +169,22 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
     const int s = (int)(rem % p.n_split); rem /= p.n_split;
     const int hc = (int)(rem % p.n_hchunk); rem /= p.n_hchunk;
     const int g = (int)(rem % p.Hkv); rem /= p.Hkv;
-    const int t = (int)(rem % p.Tq); rem /= p.Tq;
+    const int tu = (int)(rem % p.q_units); rem /= p.q_units;
     const int b = (int)rem;
+    // rows: 16/G queries x G heads (KS_PROWS) or 16 heads of one query
+    const int nqw = PR ? 16 / p.G : 1;
+    const int t = tu * nqw;                                 // first query of the item
+    const int t_end = min(t + nqw, p.Tq) - 1;              // last query of the item
     const long long pos = p.q_pos0 + t;
 
     const int gr = lane >> 2, qc = lane & 3;
-    const int hr0 = hc * 16 + gr, hr1 = hr0 + 8;          // head index within the group
-    const bool v0 = hr0 < p.G, v1 = hr1 < p.G;
+    const int tr0 = PR ? t + gr / p.G : t, tr1 = PR ? t + (gr + 8) / p.G : t;   // query of each row
+    const int hr0 = PR ? gr % p.G : hc * 16 + gr, hr1 = PR ? (gr + 8) % p.G : hc * 16 + gr + 8;
+    const bool v0 = hr0 < p.G && tr0 <= t_end, v1 = hr1 < p.G && tr1 <= t_end;
+    const long long pos_r0 = p.q_pos0 + tr0, pos_r1 = p.q_pos0 + tr1;
     const int h0 = g * p.G + hr0, h1 = g * p.G + hr1;
-    const long long qrow0 = ((long long)(b * p.Tq + t) * p.Hq + h0) * D;
-    const long long qrow1 = ((long long)(b * p.Tq + t) * p.Hq + h1) * D;
+    const long long qrow0 = ((long long)(b * p.Tq + (v0 ? tr0 : t)) * p.Hq + h0) * D;
+    const long long qrow1 = ((long long)(b * p.Tq + (v1 ? tr1 : t)) * p.Hq + h1) * D;
 
     // Q fragments (A operand, 16 rows x D), straight from global memory.
     unsigned qf[KS_D][4];
@@ -169,12 +202,12 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
     float cq0[3] = {0.f, 0.f, 0.f}, cq1[3] = {0.f, 0.f, 0.f}, be0 = 0.f, be1 = 0.f;
     if constexpr (BIAS) {
         if (v0) {
-            const float *c = p.cq + ((long long)(b * p.Tq + t) * p.Hq + h0) * 3;
+            const float *c = p.cq + ((long long)(b * p.Tq + tr0) * p.Hq + h0) * 3;
             cq0[0] = c[0]; cq0[1] = c[1]; cq0[2] = c[2];
             be0 = p.beta[h0] * kLog2e;
         }
         if (v1) {
-            const float *c = p.cq + ((long long)(b * p.Tq + t) * p.Hq + h1) * 3;
+            const float *c = p.cq + ((long long)(b * p.Tq + tr1) * p.Hq + h1) * 3;
             cq1[0] = c[0]; cq1[1] = c[1]; cq1[2] = c[2];
             be1 = p.beta[h1] * kLog2e;
         }
@@ -182,11 +215,6 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
 
     const int e_beg = s * p.per_split;
     int e_end = min(p.entries, e_beg + p.per_split);
-    if constexpr (SRC == KS_CMP) {
-        // only the compressed tokens already complete at this position
-        const long long nv = pos >= p.cmp_len - 1 ? (pos - p.cmp_len + 1) / p.block + 1 : 0;
-        e_end = (int)min((long long)e_end, nv);
-    }
     const int n_chunks = e_end > e_beg ? (e_end - e_beg + NK - 1) / NK : 0;
 
     const __nv_bfloat16 *kb = p.k + ((long long)b * p.Lk * p.Hkv + g) * D;
@@ -203,8 +231,17 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
         const int st = ci % STAGES;
         unsigned char *ks_ = wsm + st * SB;
         unsigned char *vs_ = ks_ + CH;
-        const int j = key_finish<SRC>(p, pos, raw, e_beg + ci * NK + lane);
-        if (lane < NK) keys_s[st * NK + lane] = j;
+        int j, seg = 0;
+        if constexpr (PR) {
+            j = (ci < n_chunks && lane < NK)
+                    ? key_prows(p, pos, p.q_pos0 + t_end, nqw, e_beg + ci * NK + lane, e_end, seg) : -1;
+        } else {
+            j = key_finish<SRC>(p, pos, raw, e_beg + ci * NK + lane);
+        }
+        if (lane < NK) {
+            keys_s[st * NK + lane] = j;
+            if constexpr (PR) segs_s[st * NK + lane] = seg;
+        }
         if (ci < n_chunks) {
 #pragma unroll
             for (int it = 0; it < CP_ITERS; ++it) {
@@ -243,13 +280,18 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
         const unsigned char *ks_ = wsm + st * SB;
         const unsigned char *vs_ = ks_ + CH;
         const int jl = lane < NK ? keys_s[st * NK + lane] : -1;
+        const int sl = PR && lane < NK ? segs_s[st * NK + lane] : 0;
         const unsigned vmask = __ballot_sync(0xffffffffu, jl >= 0);
         if (vmask != 0u) {
-            float sc[NK / 8][4];
+            // q.k over the head dimension; even and odd k-steps accumulate
+            // into separate registers so more MMA chains are independent
+            float sc[NK / 8][4], sc2[NK / 8][4];
 #pragma unroll
-            for (int i = 0; i < NK / 8; ++i) sc[i][0] = sc[i][1] = sc[i][2] = sc[i][3] = 0.f;
+            for (int i = 0; i < NK / 8; ++i)
+                sc[i][0] = sc[i][1] = sc[i][2] = sc[i][3] = sc2[i][0] = sc2[i][1] = sc2[i][2] = sc2[i][3] = 0.f;
 #pragma unroll
             for (int ks = 0; ks < KS_D; ++ks) {
+                float (&acc)[NK / 8][4] = (ks & 1) ? sc2 : sc;
 #pragma unroll
                 for (int np = 0; np < NK / 16; ++np) {
                     const int mi = lane >> 3, ri = lane & 7;
@@ -257,14 +299,19 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
                     const int unit = ks * 2 + (mi & 1);
                     unsigned b0, b1, b2, b3;
                     ldsm_x4(b0, b1, b2, b3, ks_ + key * ROWB + ((unit ^ (key & 7)) * 16));
-                    mma_bf16_16816(sc[2 * np], qf[ks], b0, b1);
-                    mma_bf16_16816(sc[2 * np + 1], qf[ks], b2, b3);
+                    mma_bf16_16816(acc[2 * np], qf[ks], b0, b1);
+                    mma_bf16_16816(acc[2 * np + 1], qf[ks], b2, b3);
                     if constexpr (KLO) {
                         ldsm_x4(b0, b1, b2, b3, vs_ + CH + key * ROWB + ((unit ^ (key & 7)) * 16));
-                        mma_bf16_16816(sc[2 * np], qf[ks], b0, b1);
-                        mma_bf16_16816(sc[2 * np + 1], qf[ks], b2, b3);
+                        mma_bf16_16816(acc[2 * np], qf[ks], b0, b1);
+                        mma_bf16_16816(acc[2 * np + 1], qf[ks], b2, b3);
                     }
                 }
+            }
+#pragma unroll
+            for (int i = 0; i < NK / 8; ++i) {
+                sc[i][0] += sc2[i][0]; sc[i][1] += sc2[i][1];
+                sc[i][2] += sc2[i][2]; sc[i][3] += sc2[i][3];
             }
             // scale, bias, mask; running max
             float mx0 = -INFINITY, mx1 = -INFINITY;
@@ -284,7 +331,15 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
                             x -= ((e >> 1) ? be1 : be0) * (dx * dx + dy * dy + dz * dz);
                         }
                     }
-                    x = ((vmask >> kk) & 1u) ? x : -INFINITY;
+                    bool ok = (vmask >> kk) & 1u;
+                    if constexpr (PR) {
+                        // the entry's segment decides which rows it belongs to
+                        const int jk = __shfl_sync(0xffffffffu, jl, kk);
+                        const int sk = __shfl_sync(0xffffffffu, sl, kk);
+                        const long long d = ((e >> 1) ? pos_r1 : pos_r0) - jk;
+                        ok = ok && (sk == 0 ? (d >= 0 && d < p.window) : (d == sk && sk < d + jk));
+                    }
+                    x = ok ? x : -INFINITY;
                     sc[nt][e] = x;
                 }
                 mx0 = fmaxf(mx0, fmaxf(sc[nt][0], sc[nt][1]));
@@ -352,8 +407,8 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
     const float lse0 = l0 > 0.f ? (m0 + log2f(l0)) * kLn2 : -INFINITY;
     const float lse1 = l1 > 0.f ? (m1 + log2f(l1)) * kLn2 : -INFINITY;
 
-    const long long orow0 = (long long)(b * p.Tq + t) * p.Hq + h0;
-    const long long orow1 = (long long)(b * p.Tq + t) * p.Hq + h1;
+    const long long orow0 = (long long)(b * p.Tq + tr0) * p.Hq + h0;
+    const long long orow1 = (long long)(b * p.Tq + tr1) * p.Hq + h1;
     if (p.n_split == 1) {
         if (p.out_f32) {
 #pragma unroll
@@ -396,9 +451,9 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
     }
 }
 
-template <int D, int STAGES, bool KLO = false, int NK = 32, int NW = 4>
+template <int D, int STAGES, bool KLO = false, int NK = 32, int NW = 4, bool PR = false>
 constexpr int gather_smem_bytes() {
-    return NW * STAGES * ((KLO ? 3 : 2) * NK * D * 2 + NK * 4);
+    return NW * STAGES * ((KLO ? 3 : 2) * NK * D * 2 + NK * (PR ? 8 : 4));
 }
 
 }  // namespace sa

@@ -74,13 +74,15 @@ __device__ __forceinline__ int sample_stride(const IdxParams &p, int tq0) {
 // the K-major no-swizzle core-matrix layout: 8-row group r8 at r8 * 8*DI
 // bytes, inside it the DI/16 core matrices (8 rows x 16 B) back to back, so
 // LBO = 128 B (next core along K) and SBO = 8*DI (next 8-row group).
-// 8 warps: warps w and w+4 read TMEM lane quadrant w (one key row per thread),
-// each over half of the columns.
+// 16 warps (8 when NCOL < 64): warp w reads TMEM lane quadrant w % 4 (one key
+// row per thread) over part w / 4 of the columns.
 // When every head weight of the tile is >= 0 and every w*q fits int8, the
 // weights are folded into the query operand (w*relu(x) = relu(w*x)), so the
 // epilogue is a plain sum of ReLUs; otherwise it multiplies by w itself.
 constexpr int TC_KT = 16;                // 128-key tiles per CTA (amortises the query-tile setup)
-constexpr int TC_THREADS = 256;
+// threads of a score CTA: 4 column parts of 4 warps, or 2 parts when the
+// tile has fewer than 64 columns
+__host__ __device__ constexpr int tc_threads(int ncol) { return ncol >= 64 ? 512 : 256; }
 constexpr long long TC_WAIT_CYCLES = 4000000000LL;   // ~2 s: bounded wait on the MMA barrier
 enum : int { MODE_SAMPLE = 0, MODE_FILTER = 1 };
 
@@ -96,16 +98,19 @@ __host__ __device__ constexpr int tc_smem_bytes() {
 }
 
 template <int HI, int DI, int NCOL, int MODE>
-__global__ void __launch_bounds__(TC_THREADS) idx_score_tc_kernel(const IdxParams p) {
+__global__ void __launch_bounds__(tc_threads(NCOL), NCOL >= 64 ? 2 : 4) idx_score_tc_kernel(const IdxParams p) {
+    constexpr int TC_THREADS = tc_threads(NCOL);
+    constexpr int PARTS = TC_THREADS / 128;  // column parts (4 warps each)
     constexpr int NQ = NCOL / HI;            // queries per CTA
     constexpr int CH = DI / 16;              // 16-byte chunks per row
     constexpr int A_BYTES = 128 * DI;
     constexpr int B_BYTES = NCOL * DI;
     constexpr int TCOLS = NCOL < 32 ? 32 : NCOL;
-    constexpr int HALF = NCOL / 2;           // columns per warp half
+    constexpr int HALF = NCOL / PARTS;       // columns per warp
     constexpr int STEP = HALF < 16 ? HALF : 16;
     static_assert(NCOL % 16 == 0 && NCOL >= 16 && NCOL <= 256 && NCOL % HI == 0, "NCOL");
     static_assert(HI <= STEP, "the heads of a query must lie within one step of one warp");
+    static_assert(HALF >= 16 || PARTS == 2, "16-column tiles use two column parts");
     static_assert(2 * A_BYTES + B_BYTES + NCOL * 8 + 64 <= tc_smem_bytes<DI, NCOL>(), "smem");
     constexpr uint32_t IDESC = tc::make_idesc(2 /*s32*/, 1 /*s8*/, 128, NCOL);
 
@@ -209,7 +214,7 @@ __global__ void __launch_bounds__(TC_THREADS) idx_score_tc_kernel(const IdxParam
     const uint32_t tmem = *tmem_slot;
 
     const int quad = warp & 3;                     // TMEM lane quadrant of this warp
-    const int c_begin = (warp >> 2) * HALF;        // this warp's half of the columns
+    const int c_begin = (warp >> 2) * HALF;        // this warp's part of the columns
     // per-query constants of this warp's queries, held in registers: the
     // number of candidates (keys j < nt_q are scored) and the threshold
     constexpr int NQH = HALF / HI;                 // queries in this warp's half

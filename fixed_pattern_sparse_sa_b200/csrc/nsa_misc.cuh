@@ -106,31 +106,52 @@ struct NsaSelectParams {
     float *imp_out;            // optional [B,T,Hkv,n_blocks] (tests)
 };
 
+// CTA = SEL_TW consecutive queries of one KV group (warp w: query t0 + w,
+// rows = the group's heads); compressed-key chunks (hi and lo halves) are
+// staged once per CTA and read by every warp.
+constexpr int NSA_TW = 8;
+
 template <int D>
-__global__ void __launch_bounds__(128) nsa_select_kernel(const NsaSelectParams p) {
+constexpr int nsa_select_smem(int n_blocks) {
+    return 3 * 2 * 32 * D * 2 + NSA_TW * (32 * 4 + ((n_blocks * 4 + 15) / 16) * 16);
+}
+
+template <int D>
+__global__ void __launch_bounds__(NSA_TW * 32) nsa_select_kernel(const NsaSelectParams p) {
     constexpr int NK = 32, ROWB = D * 2, UNITS = ROWB / 16, CH = NK * ROWB;
-    constexpr int KS_D = D / 16, STAGES = 2, CP_ITERS = NK * UNITS / 32;
+    constexpr int KS_D = D / 16, STAGES = 3;
     constexpr int SB = 2 * CH;                 // one stage: K hi | K lo
+    constexpr int NTHR = NSA_TW * 32;
     extern __shared__ __align__(1024) unsigned char smem[];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int wbytes = STAGES * SB + NK * 4 + p.n_blocks * 4;
-    unsigned char *wsm = smem + warp * ((wbytes + 127) / 128 * 128);
-    float *colsum = reinterpret_cast<float *>(wsm + STAGES * SB);
-    float *imp = colsum + NK;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
+    const int imp_stride = ((p.n_blocks * 4 + 15) / 16) * 16;        // bytes per warp
+    float *colsum = reinterpret_cast<float *>(smem + STAGES * SB) + warp * 32;
+    float *imp = reinterpret_cast<float *>(smem + STAGES * SB + NSA_TW * 32 * 4 + warp * imp_stride);
 
-    const long long item = (long long)blockIdx.x * 4 + warp;
-    if (item >= (long long)p.B * p.T * p.Hkv) return;
-    const int g = (int)(item % p.Hkv);
-    const int t = (int)((item / p.Hkv) % p.T);
-    const int b = (int)(item / ((long long)p.Hkv * p.T));
+    const int nqb = (p.T + NSA_TW - 1) / NSA_TW;
+    long long rem = blockIdx.x;
+    const int qb = (int)(rem % nqb); rem /= nqb;
+    const int g = (int)(rem % p.Hkv);
+    const int b = (int)(rem / p.Hkv);
+    const int t_first = qb * NSA_TW;
+    const int t_last = min(t_first + NSA_TW - 1, p.T - 1);
+    const int t = t_first + warp;
+    const bool q_ok = t <= t_last;
+    auto n_vis_of = [&](int tt) {
+        return tt >= p.cmp_len - 1 ? min(p.nc, (tt - p.cmp_len + 1) / p.cmp_stride + 1) : 0;
+    };
+    const int n_vis_cta = n_vis_of(t_last);
+    const int n_vis = q_ok ? n_vis_of(t) : 0;
+    const int n_chunks = (n_vis_cta + NK - 1) / NK;
+
     const int gr = lane >> 2, qc = lane & 3;
-    const bool v0 = gr < p.G, v1 = gr + 8 < p.G;
+    const bool v0 = q_ok && gr < p.G, v1 = q_ok && gr + 8 < p.G;
     const int h0 = g * p.G + gr, h1 = h0 + 8;
-
+    const int tq = q_ok ? t : 0;
     unsigned qf[KS_D][4];
     {
-        const unsigned *q0 = reinterpret_cast<const unsigned *>(p.q + ((long long)(b * p.T + t) * p.Hq + h0) * D);
-        const unsigned *q1 = reinterpret_cast<const unsigned *>(p.q + ((long long)(b * p.T + t) * p.Hq + h1) * D);
+        const unsigned *q0 = reinterpret_cast<const unsigned *>(p.q + ((long long)(b * p.T + tq) * p.Hq + h0) * D);
+        const unsigned *q1 = reinterpret_cast<const unsigned *>(p.q + ((long long)(b * p.T + tq) * p.Hq + h1) * D);
 #pragma unroll
         for (int ks = 0; ks < KS_D; ++ks) {
             qf[ks][0] = v0 ? __ldg(q0 + ks * 8 + qc) : 0u;
@@ -139,47 +160,46 @@ __global__ void __launch_bounds__(128) nsa_select_kernel(const NsaSelectParams p
             qf[ks][3] = v1 ? __ldg(q1 + ks * 8 + qc + 4) : 0u;
         }
     }
-    const float ls0 = v0 ? p.lse_cmp[(long long)(b * p.T + t) * p.Hq + h0] * kLog2e : INFINITY;
-    const float ls1 = v1 ? p.lse_cmp[(long long)(b * p.T + t) * p.Hq + h1] * kLog2e : INFINITY;
+    const float ls0 = v0 ? p.lse_cmp[(long long)(b * p.T + tq) * p.Hq + h0] * kLog2e : INFINITY;
+    const float ls1 = v1 ? p.lse_cmp[(long long)(b * p.T + tq) * p.Hq + h1] * kLog2e : INFINITY;
 
-    const int nb_t = t / p.sel_block + 1;                   // candidate blocks
+    const int nb_t = q_ok ? t / p.sel_block + 1 : 0;      // candidate blocks of this query
     for (int i = lane; i < nb_t; i += 32) imp[i] = 0.f;
-    const int n_vis = t >= p.cmp_len - 1 ? min(p.nc, (t - p.cmp_len + 1) / p.cmp_stride + 1) : 0;
-    const int n_chunks = (n_vis + NK - 1) / NK;
     const __nv_bfloat16 *kb = p.kc + ((long long)b * p.nc * p.Hkv + g) * D;
     const __nv_bfloat16 *kl = p.klo + ((long long)b * p.nc * p.Hkv + g) * D;
     const long long rstride = (long long)p.Hkv * D;
 
     auto issue = [&](int ci) {
         if (ci < n_chunks) {
-            unsigned char *ks_ = wsm + (ci % STAGES) * SB;
-#pragma unroll
-            for (int it = 0; it < CP_ITERS; ++it) {
-                const int lin = it * 32 + lane;
+            unsigned char *ks_ = smem + (ci % STAGES) * SB;
+            for (int lin = tid; lin < NK * UNITS; lin += NTHR) {
                 const int rr = lin / UNITS, u = lin % UNITS;
                 const int i = ci * NK + rr;
-                const bool ok = i < n_vis;
+                const bool ok = i < n_vis_cta;
                 const long long off = ok ? (long long)i * rstride + u * 8 : 0;
-                cp_async16(ks_ + rr * ROWB + ((u ^ (rr & 7)) * 16), kb + off, ok ? 16 : 0);
-                cp_async16(ks_ + CH + rr * ROWB + ((u ^ (rr & 7)) * 16), kl + off, ok ? 16 : 0);
+                const int sw = (u ^ (rr & 7)) * 16;
+                cp_async16(ks_ + rr * ROWB + sw, kb + off, ok ? 16 : 0);
+                cp_async16(ks_ + CH + rr * ROWB + sw, kl + off, ok ? 16 : 0);
             }
         }
         cp_async_commit();
     };
 #pragma unroll
     for (int ci = 0; ci < STAGES - 1; ++ci) issue(ci);
-    __syncwarp();
 
     for (int ci = 0; ci < n_chunks; ++ci) {
+        cp_async_wait<STAGES - 2>();
+        __syncthreads();
         issue(ci + STAGES - 1);
-        cp_async_wait<STAGES - 1>();
-        __syncwarp();
-        const unsigned char *ks_ = wsm + (ci % STAGES) * SB;
-        float sc[NK / 8][4];
+        if (ci * NK >= n_vis) continue;                     // warp-uniform: nothing visible
+        const unsigned char *ks_ = smem + (ci % STAGES) * SB;
+        float sc[NK / 8][4], sc2[NK / 8][4];
 #pragma unroll
-        for (int i = 0; i < NK / 8; ++i) sc[i][0] = sc[i][1] = sc[i][2] = sc[i][3] = 0.f;
+        for (int i = 0; i < NK / 8; ++i)
+            sc[i][0] = sc[i][1] = sc[i][2] = sc[i][3] = sc2[i][0] = sc2[i][1] = sc2[i][2] = sc2[i][3] = 0.f;
 #pragma unroll
-        for (int ks = 0; ks < KS_D; ++ks)
+        for (int ks = 0; ks < KS_D; ++ks) {
+            float (&acc)[NK / 8][4] = (ks & 1) ? sc2 : sc;
 #pragma unroll
             for (int np = 0; np < NK / 16; ++np) {
                 const int mi = lane >> 3, ri = lane & 7;
@@ -187,12 +207,13 @@ __global__ void __launch_bounds__(128) nsa_select_kernel(const NsaSelectParams p
                 const int unit = ks * 2 + (mi & 1);
                 unsigned b0, b1, b2, b3;
                 ldsm_x4(b0, b1, b2, b3, ks_ + key * ROWB + ((unit ^ (key & 7)) * 16));
-                mma_bf16_16816(sc[2 * np], qf[ks], b0, b1);
-                mma_bf16_16816(sc[2 * np + 1], qf[ks], b2, b3);
+                mma_bf16_16816(acc[2 * np], qf[ks], b0, b1);
+                mma_bf16_16816(acc[2 * np + 1], qf[ks], b2, b3);
                 ldsm_x4(b0, b1, b2, b3, ks_ + CH + key * ROWB + ((unit ^ (key & 7)) * 16));
-                mma_bf16_16816(sc[2 * np], qf[ks], b0, b1);
-                mma_bf16_16816(sc[2 * np + 1], qf[ks], b2, b3);
+                mma_bf16_16816(acc[2 * np], qf[ks], b0, b1);
+                mma_bf16_16816(acc[2 * np + 1], qf[ks], b2, b3);
             }
+        }
         // probabilities, summed over the group's heads (rows) per column
 #pragma unroll
         for (int nt = 0; nt < NK / 8; ++nt) {
@@ -201,8 +222,8 @@ __global__ void __launch_bounds__(128) nsa_select_kernel(const NsaSelectParams p
             for (int e = 0; e < 2; ++e) {
                 const int i = ci * NK + nt * 8 + 2 * qc + e;
                 const bool ok = i < n_vis;
-                const float p0 = (ok && v0) ? exp2f(sc[nt][e] * p.scale_log2 - ls0) : 0.f;
-                const float p1 = (ok && v1) ? exp2f(sc[nt][2 + e] * p.scale_log2 - ls1) : 0.f;
+                const float p0 = (ok && v0) ? exp2f((sc[nt][e] + sc2[nt][e]) * p.scale_log2 - ls0) : 0.f;
+                const float p1 = (ok && v1) ? exp2f((sc[nt][2 + e] + sc2[nt][2 + e]) * p.scale_log2 - ls1) : 0.f;
                 float x = p0 + p1;
                 x += __shfl_xor_sync(0xffffffffu, x, 4);
                 x += __shfl_xor_sync(0xffffffffu, x, 8);
@@ -234,6 +255,7 @@ __global__ void __launch_bounds__(128) nsa_select_kernel(const NsaSelectParams p
     }
     cp_async_wait<0>();
     __syncwarp();
+    if (!q_ok) return;
 
     const long long orow = ((long long)(b * p.T + t) * p.Hkv + g);
     if (p.imp_out) {

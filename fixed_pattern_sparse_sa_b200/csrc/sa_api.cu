@@ -16,6 +16,7 @@
 
 #include "../../include/sa.h"
 #include "attn_gather.cuh"
+#include "attn_tile.cuh"
 #include "indexer.cuh"
 #include "nsa_misc.cuh"
 
@@ -82,19 +83,25 @@ static int set_smem(K kernel, int bytes) {
 }
 
 // -------------------------------------------------------- gather launches --
-// Launch shape: 8 warps per CTA streaming 16-key chunks, 3 stages deep (a
-// 2-stage ring when the lo-key tile is also staged); 192 KB of shared memory,
-// one CTA and 8 gathering warps per SM.
+// Launch shape: 12 warps per CTA streaming 16-key chunks through a 2-stage
+// ring (8 warps when the lo-key tile is also staged); ~198 KB of shared
+// memory, one CTA and 12 gathering warps per SM.
 template <int D, int SRC, bool BIAS, bool KLO = false>
 static int launch_gather_t(const GatherParams &p, cudaStream_t st) {
-    constexpr int NK = 16, NW = 8;
-    constexpr int STAGES = KLO ? 2 : 3;
-    constexpr int smem = gather_smem_bytes<D, STAGES, KLO, NK, NW>();
+#ifndef SA_ATTN_NW
+#define SA_ATTN_NW 12
+#endif
+#ifndef SA_ATTN_STAGES
+#define SA_ATTN_STAGES 2
+#endif
+    constexpr int NK = 16, NW = KLO ? 8 : SA_ATTN_NW;
+    constexpr int STAGES = KLO ? 2 : SA_ATTN_STAGES;
+    constexpr int smem = gather_smem_bytes<D, STAGES, KLO, NK, NW, SRC == KS_PROWS>();
     static_assert(smem <= 227 * 1024, "shared memory");
     auto kern = gather_attn_kernel<D, STAGES, SRC, BIAS, KLO, NK, NW>;
     int rc = set_smem(kern, smem);
     if (rc) return rc;
-    const long long items = (long long)p.B * p.Tq * p.Hkv * p.n_hchunk * p.n_split;
+    const long long items = (long long)p.B * p.q_units * p.Hkv * p.n_hchunk * p.n_split;
     if (items == 0) return SA_OK;
     const long long blocks = (items + NW - 1) / NW;
     kern<<<(unsigned)blocks, NW * 32, smem, st>>>(p);
@@ -110,7 +117,8 @@ static int launch_gather_d(const GatherParams &p, int src, bool bias, cudaStream
             return bias ? launch_gather_t<D, KS_PATTERN, true>(p, st) : launch_gather_t<D, KS_PATTERN, false>(p, st);
         case KS_BLOCKS: return launch_gather_t<D, KS_BLOCKS, false>(p, st);
         case KS_RANGE: return launch_gather_t<D, KS_RANGE, false>(p, st);
-        case KS_CMP: return launch_gather_t<D, KS_CMP, false, true>(p, st);
+        case KS_PROWS:
+            return bias ? launch_gather_t<D, KS_PROWS, true>(p, st) : launch_gather_t<D, KS_PROWS, false>(p, st);
     }
     return fail(SA_ERR_UNSUPPORTED, "key source %d", src);
 }
@@ -244,14 +252,24 @@ int sa_sparse_attn_fwd(const void *q, const void *k, const void *v, int B, int T
         src = KS_IDX;
         p.entries = K;
     } else {
-        src = KS_PATTERN;
         p.window = pattern->window;
         p.dilated = pattern->dilated ? 1 : 0;
-        p.entries = pattern->window + (p.dilated ? 32 : 0);
+        const int G = Hq / Hkv;
+        if (G < 16 && 16 % G == 0) {
+            // rows = 16/G consecutive queries x G heads over the union of their sets
+            src = KS_PROWS;
+            const int nqw = 16 / G;
+            p.entries = pattern->window + nqw - 1 + (p.dilated ? 32 * nqw : 0);
+            p.q_units = (Tq + nqw - 1) / nqw;
+        } else {
+            src = KS_PATTERN;
+            p.entries = pattern->window + (p.dilated ? 32 : 0);
+        }
     }
     p.n_split = n_split;
     p.per_split = n_split > 1 ? (p.entries + n_split - 1) / n_split : p.entries;
-    p.n_hchunk = (p.G + 15) / 16;
+    p.n_hchunk = src == KS_PROWS ? 1 : (p.G + 15) / 16;
+    if (src != KS_PROWS) p.q_units = Tq;
     p.cq = cq; p.ck = ck; p.beta = beta;
     p.scale_log2 = scale * kLog2e;
     p.out = static_cast<__nv_bfloat16 *>(out);
@@ -342,7 +360,7 @@ static int launch_score_t(const IdxParams &p, long long n_keys_max, cudaStream_t
     if (rc) return rc;
     dim3 grid((unsigned)((n_keys_max + TC_KT * 128 - 1) / (TC_KT * 128)), (unsigned)((p.Rt + NQ - 1) / NQ),
               (unsigned)p.B);
-    kern<<<grid, TC_THREADS, smem, st>>>(p);
+    kern<<<grid, tc_threads(NCOL), smem, st>>>(p);
     SA_CHECK_LAUNCH("idx_score_tc_kernel");
     return SA_OK;
 }
@@ -477,16 +495,37 @@ size_t sa_nsa_workspace_size(int B, int T, int Hq, int Hkv, int d, int cmp_len, 
 
 template <int D>
 static int launch_nsa_select(const NsaSelectParams &p, cudaStream_t st) {
-    const int wbytes = 2 * 2 * 32 * D * 2 + 32 * 4 + p.n_blocks * 4;
-    const int smem = 4 * ((wbytes + 127) / 128 * 128);
+    const int smem = nsa_select_smem<D>(p.n_blocks);
     if (smem > 227 * 1024) return fail(SA_ERR_UNSUPPORTED, "nsa: %d selection blocks exceed shared memory", p.n_blocks);
     auto kern = nsa_select_kernel<D>;
     int rc = set_smem(kern, smem);
     if (rc) return rc;
-    const long long items = (long long)p.B * p.T * p.Hkv;
-    kern<<<(unsigned)((items + 3) / 4), 128, smem, st>>>(p);
+    const long long ctas = (long long)p.B * p.Hkv * ((p.T + NSA_TW - 1) / NSA_TW);
+    kern<<<(unsigned)ctas, NSA_TW * 32, smem, st>>>(p);
     SA_CHECK_LAUNCH("nsa_select_kernel");
     return SA_OK;
+}
+
+// Compressed and window branches: 8 consecutive queries of a KV group per CTA
+// share each staged key chunk.
+constexpr int kTileWarps = 8;
+template <int D, int SRC>
+static int launch_tile_t(const TileParams &p, cudaStream_t st) {
+    constexpr int STAGES = 3;
+    constexpr int smem = tile_smem_bytes<D, STAGES, SRC>();
+    auto kern = tile_attn_kernel<D, STAGES, SRC, kTileWarps>;
+    int rc = set_smem(kern, smem);
+    if (rc) return rc;
+    const long long ctas = (long long)p.B * p.Hkv * ((p.T + kTileWarps - 1) / kTileWarps);
+    if (ctas == 0) return SA_OK;
+    kern<<<(unsigned)ctas, kTileWarps * 32, smem, st>>>(p);
+    SA_CHECK_LAUNCH("tile_attn_kernel");
+    return SA_OK;
+}
+
+static int launch_tile(const TileParams &p, int d, int src, cudaStream_t st) {
+    if (d == 64) return src == TS_CMP ? launch_tile_t<64, TS_CMP>(p, st) : launch_tile_t<64, TS_WINDOW>(p, st);
+    return src == TS_CMP ? launch_tile_t<128, TS_CMP>(p, st) : launch_tile_t<128, TS_WINDOW>(p, st);
 }
 
 int sa_nsa_fwd(const void *q, const void *k, const void *v, const float *gates, int B, int T, int Hq,
@@ -535,17 +574,19 @@ int sa_nsa_fwd(const void *q, const void *k, const void *v, const float *gates, 
     GatherParams base{};
     base.q = static_cast<const __nv_bfloat16 *>(q);
     base.B = B; base.Tq = T; base.Hq = Hq; base.Hkv = Hkv; base.G = G;
-    base.q_pos0 = 0; base.n_split = 1; base.n_hchunk = 1;
+    base.q_pos0 = 0; base.n_split = 1; base.n_hchunk = 1; base.q_units = T;
     base.scale_log2 = scale * kLog2e;
     base.err = ew;
     // 2. compressed branch -> o3[0], l3[0]
+    TileParams tp{};
+    tp.q = base.q; tp.B = B; tp.T = T; tp.Hq = Hq; tp.Hkv = Hkv; tp.G = G;
+    tp.scale_log2 = base.scale_log2;
     {
-        GatherParams p = base;
+        TileParams p = tp;
         p.k = kc; p.klo = klo; p.v = vc; p.Lk = std::max(lay.nc, 1);
-        p.block = cmp_stride; p.cmp_len = cmp_len;
-        p.entries = lay.nc; p.per_split = lay.nc;
+        p.cmp_len = cmp_len; p.cmp_stride = cmp_stride;
         p.out_f32 = o3; p.lse = l3;
-        rc = launch_gather(p, d, KS_CMP, false, st);   // nc == 0: zero rows, lse = -inf
+        rc = launch_tile(p, d, TS_CMP, st);   // nc == 0: zero rows, lse = -inf
         if (rc) return rc;
     }
     // 3. importance + block top-k
@@ -572,11 +613,11 @@ int sa_nsa_fwd(const void *q, const void *k, const void *v, const float *gates, 
     }
     // 5. window branch -> o3[2], l3[2]
     {
-        GatherParams p = base;
+        TileParams p = tp;
         p.k = static_cast<const __nv_bfloat16 *>(k); p.v = static_cast<const __nv_bfloat16 *>(v);
-        p.Lk = T; p.window = window; p.entries = window; p.per_split = window;
+        p.Lk = T; p.window = window;
         p.out_f32 = o3 + 2 * rows * d; p.lse = l3 + 2 * rows;
-        rc = launch_gather(p, d, KS_RANGE, false, st);
+        rc = launch_tile(p, d, TS_WINDOW, st);
         if (rc) return rc;
     }
     // 6. gated sum
