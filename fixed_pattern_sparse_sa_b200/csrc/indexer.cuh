@@ -31,7 +31,8 @@
 
 namespace sa {
 
-constexpr int SAMPLE_TARGET = 2048;       // sampled keys per row (stride = n / target)
+constexpr int SAMPLE_TARGET = 4096;       // sampled keys per row (stride = n / target)
+constexpr double SAMPLE_Z = 4.5;          // safety margin of the sampled threshold, in sigmas
 
 struct IdxParams {
     const int8_t *q;       // [B, Tq, Hi, DI]
@@ -90,11 +91,16 @@ __device__ __forceinline__ int tc_core_off(int row, int chunk, int di) {
     return (row >> 3) * (8 * di) + chunk * 128 + (row & 7) * 16;
 }
 
+// Key tiles are staged through a ring of TC_AS buffers (TC_AS - 1 in flight).
+constexpr int TC_AS = 4;
+
 // Shared memory of one score CTA; at least 80 KB for NCOL = 256 so that at
 // most two CTAs (2 x 256 TMEM columns) share an SM.
 template <int DI, int NCOL>
 __host__ __device__ constexpr int tc_smem_bytes() {
-    return NCOL >= 256 ? 80 * 1024 : 2 * 128 * DI + NCOL * DI + NCOL * 8 + 64;
+    return (NCOL >= 256 && TC_AS * 128 * DI + NCOL * DI + NCOL * 8 + 64 < 80 * 1024)
+               ? 80 * 1024
+               : TC_AS * 128 * DI + NCOL * DI + NCOL * 8 + 64;
 }
 
 template <int HI, int DI, int NCOL, int MODE>
@@ -111,12 +117,12 @@ __global__ void __launch_bounds__(tc_threads(NCOL), NCOL >= 64 ? 2 : 4) idx_scor
     static_assert(NCOL % 16 == 0 && NCOL >= 16 && NCOL <= 256 && NCOL % HI == 0, "NCOL");
     static_assert(HI <= STEP, "the heads of a query must lie within one step of one warp");
     static_assert(HALF >= 16 || PARTS == 2, "16-column tiles use two column parts");
-    static_assert(2 * A_BYTES + B_BYTES + NCOL * 8 + 64 <= tc_smem_bytes<DI, NCOL>(), "smem");
+    static_assert(TC_AS * A_BYTES + B_BYTES + NCOL * 8 + 64 <= tc_smem_bytes<DI, NCOL>(), "smem");
     constexpr uint32_t IDESC = tc::make_idesc(2 /*s32*/, 1 /*s8*/, 128, NCOL);
 
     extern __shared__ __align__(1024) unsigned char smem[];
-    unsigned char *a_s = smem;                               // 2 x A tile
-    unsigned char *b_s = smem + 2 * A_BYTES;                 // B tile
+    unsigned char *a_s = smem;                               // TC_AS x A tile
+    unsigned char *b_s = smem + TC_AS * A_BYTES;             // B tile
     int *w_s = reinterpret_cast<int *>(b_s + B_BYTES);       // [NCOL]
     int *tau_s = w_s + NCOL;                                 // [NQ] (filter mode)
     uint64_t *bar = reinterpret_cast<uint64_t *>(tau_s + NCOL);
@@ -193,20 +199,23 @@ __global__ void __launch_bounds__(tc_threads(NCOL), NCOL >= 64 ? 2 : 4) idx_scor
             *reinterpret_cast<int4 *>(b_s + tc_core_off(row, c, DI)) = v;
         }
     }
-    auto load_a = [&](int kt) {
-        unsigned char *dst = a_s + (kt & 1) * A_BYTES;
-        const int i0 = j_cta + kt * 128;
-        const int8_t *src = p.k + ((long long)b * p.L) * DI;
-        for (int i = tid; i < 128 * CH; i += TC_THREADS) {
-            const int row = i / CH, c = i % CH;
-            const long long j = (long long)stride * (i0 + row);
-            const bool ok = j < p.L;
-            cp_async16(dst + tc_core_off(row, c, DI), ok ? src + j * DI + c * 16 : src, ok ? 16 : 0);
+    auto load_a = [&](int kt) {   // always commits a group (empty past the last tile)
+        if (kt < n_tiles) {
+            unsigned char *dst = a_s + (kt % TC_AS) * A_BYTES;
+            const int i0 = j_cta + kt * 128;
+            const int8_t *src = p.k + ((long long)b * p.L) * DI;
+            for (int i = tid; i < 128 * CH; i += TC_THREADS) {
+                const int row = i / CH, c = i % CH;
+                const long long j = (long long)stride * (i0 + row);
+                const bool ok = j < p.L;
+                cp_async16(dst + tc_core_off(row, c, DI), ok ? src + j * DI + c * 16 : src, ok ? 16 : 0);
+            }
         }
         cp_async_commit();
     };
-    load_a(0);
-    cp_async_wait<0>();
+#pragma unroll
+    for (int s = 0; s < TC_AS - 1; ++s) load_a(s);
+    cp_async_wait<TC_AS - 2>();                              // tile 0 has landed
     tc::fence_proxy_async_smem();
     tc::fence_before_sync();
     __syncthreads();
@@ -235,7 +244,7 @@ __global__ void __launch_bounds__(tc_threads(NCOL), NCOL >= 64 ? 2 : 4) idx_scor
     for (int kt = 0; kt < n_tiles; ++kt) {
         pending = kt & 1;
         if (tid == 0) {
-            const uint32_t a_addr = tc::smem_u32(a_s + (kt & 1) * A_BYTES);
+            const uint32_t a_addr = tc::smem_u32(a_s + (kt % TC_AS) * A_BYTES);
             const uint32_t b_addr = tc::smem_u32(b_s);
 #pragma unroll
             for (int kk = 0; kk < DI / 32; ++kk) {
@@ -246,7 +255,7 @@ __global__ void __launch_bounds__(tc_threads(NCOL), NCOL >= 64 ? 2 : 4) idx_scor
             }
             tc::mma_commit(bar);
         }
-        if (kt + 1 < n_tiles) load_a(kt + 1);                  // other buffer: its MMA is done
+        load_a(kt + TC_AS - 1);                                // buffer of tile kt-1: its MMA is done
         // one thread waits (bounded) and the whole CTA follows its verdict
         if (tid == 0) *wait_ok = tc::mbar_wait_bounded(bar, kt & 1, TC_WAIT_CYCLES) ? 1 : 0;
         __syncthreads();
@@ -329,9 +338,9 @@ __global__ void __launch_bounds__(tc_threads(NCOL), NCOL >= 64 ? 2 : 4) idx_scor
                 }
             }
         }
-        // the next MMA overwrites the accumulator and reads the other A buffer
+        // the next MMA overwrites the accumulator and reads tile kt+1's buffer
         tc::fence_before_sync();
-        cp_async_wait<0>();
+        cp_async_wait<TC_AS - 2>();
         tc::fence_proxy_async_smem();
         __syncthreads();
         tc::fence_after_sync();
@@ -344,6 +353,83 @@ __global__ void __launch_bounds__(tc_threads(NCOL), NCOL >= 64 ? 2 : 4) idx_scor
     tc::fence_before_sync();
     __syncthreads();
     if (warp == 0) tc::tmem_dealloc(tmem, TCOLS);
+}
+
+// ----------------------------------------------- decode-shaped scores --
+// With one or two queries per sequence the score pass is a memory-bound
+// matrix-vector product; it runs on CUDA cores (dp4a) so the keys stream at
+// HBM bandwidth.  CTA = (b, query row, DEC_KEYS keys); thread = key.
+constexpr int DEC_THREADS = 256;
+constexpr int DEC_KEYS = 2048;
+
+template <int DI, int MODE>
+__global__ void __launch_bounds__(DEC_THREADS) idx_score_dp4a_kernel(const IdxParams p) {
+    __shared__ __align__(16) int8_t q_s[16 * DI];
+    __shared__ int w_s[16];
+    const int b = blockIdx.z, tr = blockIdx.y, t = p.t0 + tr;
+    if (t >= p.Tq || tr >= p.Rt) return;
+    const long long nt = n_candidates(p.q_pos0 + t, p.window);
+    const int stride = MODE == MODE_SAMPLE ? sample_stride(p, t) : 1;     // query blocks of one
+    const long long n_keys = MODE == MODE_SAMPLE ? (nt + stride - 1) / stride : nt;
+    const long long i0 = (long long)blockIdx.x * DEC_KEYS;
+    if (i0 >= n_keys) return;
+    const int tid = threadIdx.x, lane = tid & 31;
+    const long long row = (long long)b * p.Rt + tr;
+    const int8_t *qsrc = p.q + ((long long)b * p.Tq + t) * p.Hi * DI;
+    for (int i = tid; i < p.Hi * DI / 16; i += DEC_THREADS)
+        reinterpret_cast<int4 *>(q_s)[i] = __ldg(reinterpret_cast<const int4 *>(qsrc) + i);
+    if (tid < p.Hi) w_s[tid] = __ldg(p.w + ((long long)b * p.Tq + t) * p.Hi + tid);
+    const int tau = MODE == MODE_FILTER ? p.tau[row] : 0;
+    __syncthreads();
+    const int8_t *kb = p.k + (long long)b * p.L * DI;
+    constexpr int U = 2;                                    // keys per thread in flight
+    for (long long base = i0 + tid; base < i0 + DEC_KEYS; base += (long long)DEC_THREADS * U) {
+        int4 kv[U][DI / 16];
+        long long jj[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const long long i = base + (long long)u * DEC_THREADS;
+            jj[u] = (long long)stride * i;
+            const bool ok = i < n_keys && i < i0 + DEC_KEYS && jj[u] < p.L;
+#pragma unroll
+            for (int c = 0; c < DI / 16; ++c)
+                kv[u][c] = ok ? __ldg(reinterpret_cast<const int4 *>(kb + jj[u] * DI) + c) : make_int4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const long long i = base + (long long)u * DEC_THREADS;
+            const bool ok = i < n_keys && i < i0 + DEC_KEYS && jj[u] < nt;
+            int total = 0;
+            for (int h = 0; h < p.Hi; ++h) {
+                const int4 *qv = reinterpret_cast<const int4 *>(q_s + h * DI);
+                int dot = 0;
+#pragma unroll
+                for (int c = 0; c < DI / 16; ++c) {
+                    const int4 a = qv[c];
+                    dot = __dp4a(a.x, kv[u][c].x, dot);
+                    dot = __dp4a(a.y, kv[u][c].y, dot);
+                    dot = __dp4a(a.z, kv[u][c].z, dot);
+                    dot = __dp4a(a.w, kv[u][c].w, dot);
+                }
+                total += w_s[h] * max(dot, 0);
+            }
+            if constexpr (MODE == MODE_SAMPLE) {
+                if (ok) p.sample[row * p.m_cap + i] = total;
+            } else {
+                const bool keep = ok && total >= tau;
+                const unsigned ballot = __ballot_sync(0xffffffffu, keep);
+                if (ballot) {
+                    int slot0 = 0;
+                    if (lane == 0) slot0 = atomicAdd(p.cand_cnt + row, __popc(ballot));
+                    const int slot = __shfl_sync(0xffffffffu, slot0, 0) + __popc(ballot & ((1u << lane) - 1u));
+                    if (keep && slot < p.cand_cap) {
+                        p.cand_val[row * p.cand_cap + slot] = total;
+                        p.cand_idx[row * p.cand_cap + slot] = (int)jj[u];
+                    }
+                }
+            }
+        }
+    }
 }
 
 // ----------------------------------------------------- block helpers --
@@ -499,8 +585,14 @@ __global__ void __launch_bounds__(SEL_THREADS, 4) idx_threshold_kernel(const Idx
     if (s == 1) {
         r = k_eff;
     } else {
-        const double expect = (double)k_eff * m / n;         // sample rank of the k-th key
-        r = (int)ceil(expect + 4.0 * sqrt(expect) + 2.0);
+        // The count of candidates at or above the sample's r-th value is about
+        // s*r with a standard deviation of about s*sqrt(r); r = e + z*sqrt(r)
+        // keeps it z sigmas above k (e = k/s, the sample rank of the k-th key).
+        const double e = (double)k_eff * m / n;
+        double rr = e + SAMPLE_Z * sqrt(e) + 2.0;
+        rr = e + SAMPLE_Z * sqrt(rr) + 2.0;
+        rr = e + SAMPLE_Z * sqrt(rr) + 2.0;
+        r = (int)ceil(rr);
         r = min(r, m);
     }
     const int32_t *vals = p.sample + row * p.m_cap;

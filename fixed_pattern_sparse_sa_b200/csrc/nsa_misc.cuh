@@ -236,18 +236,18 @@ __global__ void __launch_bounds__(NSA_TW * 32) nsa_select_kernel(const NsaSelect
             }
         }
         __syncwarp();
-        // one writer per selection block touched by this chunk, fixed order
+        // one writer per selection block touched by this chunk, fixed order:
+        // block blk holds the compressed tokens [blk*cpb, (blk+1)*cpb)
         {
+            const int cpb = p.sel_block / p.cmp_stride;
             const int i_first = ci * NK;
-            const int blk_first = (i_first * p.cmp_stride) / p.sel_block;
             const int i_last = min(ci * NK + NK, n_vis) - 1;
-            const int blk_last = (i_last * p.cmp_stride) / p.sel_block;
+            const int blk_first = i_first / cpb, blk_last = i_last / cpb;
             for (int blk = blk_first + lane; blk <= blk_last; blk += 32) {
+                const int c_lo = max(blk * cpb, i_first) - i_first;
+                const int c_hi = min((blk + 1) * cpb - 1, i_last) - i_first;
                 float acc = 0.f;
-                for (int c = 0; c < NK; ++c) {
-                    const int i = i_first + c;
-                    if (i <= i_last && (i * p.cmp_stride) / p.sel_block == blk) acc += colsum[c];
-                }
+                for (int c = c_lo; c <= c_hi; ++c) acc += colsum[c];
                 imp[blk] += acc;
             }
         }

@@ -302,14 +302,25 @@ static bool indexer_shape_ok(int Hi, int di) {
     return (Hi == 1 || Hi == 2 || Hi == 4 || Hi == 8 || Hi == 16) && (di == 32 || di == 64 || di == 128);
 }
 
-// Decode-like shapes (one or two queries per sequence) use a 16-column MMA
-// tile instead of 256 columns.
-static int indexer_ncol(int Tq, int Hi) { return (Tq * Hi <= 16 && Hi <= 8) ? 16 : 256; }
+// Decode-like shapes (a query or two per sequence) score on CUDA cores
+// (memory-bound matrix-vector products); the rest on tcgen05 with 256-column
+// tiles.  The sample stride is shared by a block of nq queries.
+static bool indexer_decode_path(int Tq, int Hi) { return Tq * Hi <= 16; }
 
 static int indexer_m_cap(int nq_block) { return (int)round_up((size_t)(2 * SAMPLE_TARGET + nq_block), 4); }
 
-// Candidate list capacity per row: about k + 4 sigma entries are expected.
-static int indexer_cand_cap(int topk) { return (int)round_up((size_t)std::max(5120, topk * 5 / 2), 64); }
+// Candidate list capacity per row.  With sample stride s the threshold sits
+// at sample rank r = e + z*sqrt(r) (e = k/s, as in idx_threshold_kernel), so
+// about s*r candidates reach it, with a standard deviation of about s*sqrt(r);
+// the list holds s*r + z standard deviations.
+static int indexer_cand_cap(int topk, int L) {
+    const double s = std::max(1.0, std::floor((double)L / SAMPLE_TARGET));
+    const double e = topk / s;
+    double r = e + SAMPLE_Z * std::sqrt(e) + 2.0;
+    for (int it = 0; it < 3; ++it) r = e + SAMPLE_Z * std::sqrt(r) + 2.0;
+    const double cap = std::max((double)topk, s * r + SAMPLE_Z * s * std::sqrt(r)) + 256.0;
+    return (int)round_up((size_t)cap, 64);
+}
 
 static size_t indexer_row_bytes(int m_cap, int cap) { return (size_t)m_cap * 4 + 8 + (size_t)cap * 8; }
 
@@ -323,16 +334,17 @@ static int indexer_chunk_rows(int B, int Tq, int nq_block, int m_cap, int cap) {
 }
 
 struct IdxLayout {
-    int ncol, nq, m_cap, cap, rt;
+    bool decode;
+    int nq, m_cap, cap, rt;
     size_t sample_off, tau_off, cnt_off, val_off, idx_off, total;
 };
 
-static IdxLayout indexer_layout(int B, int Tq, int Hi, int topk) {
+static IdxLayout indexer_layout(int B, int Tq, int L, int Hi, int topk) {
     IdxLayout l{};
-    l.ncol = indexer_ncol(Tq, Hi);
-    l.nq = l.ncol / Hi;
+    l.decode = indexer_decode_path(Tq, Hi);
+    l.nq = l.decode ? 1 : 256 / Hi;
     l.m_cap = indexer_m_cap(l.nq);
-    l.cap = indexer_cand_cap(topk);
+    l.cap = indexer_cand_cap(topk, L);
     l.rt = indexer_chunk_rows(B, Tq, l.nq, l.m_cap, l.cap);
     const size_t rows = (size_t)B * l.rt;
     size_t off = 0;
@@ -346,9 +358,9 @@ static IdxLayout indexer_layout(int B, int Tq, int Hi, int topk) {
 }
 
 size_t sa_indexer_topk_workspace_size(int B, int Tq, int L, int Hi, int di, int topk, int window) {
-    (void)L; (void)di; (void)window;
-    if (B <= 0 || Tq <= 0 || topk < 0 || !(Hi == 1 || Hi == 2 || Hi == 4 || Hi == 8 || Hi == 16)) return 0;
-    return indexer_layout(B, Tq, Hi, topk).total;
+    (void)di; (void)window;
+    if (B <= 0 || Tq <= 0 || L <= 0 || topk < 0 || !(Hi == 1 || Hi == 2 || Hi == 4 || Hi == 8 || Hi == 16)) return 0;
+    return indexer_layout(B, Tq, L, Hi, topk).total;
 }
 
 template <int HI, int DI, int NCOL, int MODE>
@@ -365,20 +377,26 @@ static int launch_score_t(const IdxParams &p, long long n_keys_max, cudaStream_t
     return SA_OK;
 }
 
+template <int DI, int MODE>
+static int launch_dp4a_t(const IdxParams &p, long long n_keys_max, cudaStream_t st) {
+    dim3 grid((unsigned)((n_keys_max + DEC_KEYS - 1) / DEC_KEYS), (unsigned)p.Rt, (unsigned)p.B);
+    idx_score_dp4a_kernel<DI, MODE><<<grid, DEC_THREADS, 0, st>>>(p);
+    SA_CHECK_LAUNCH("idx_score_dp4a_kernel");
+    return SA_OK;
+}
+
 template <int HI, int DI, int MODE>
-static int launch_score_n(const IdxParams &p, int ncol, long long n_keys_max, cudaStream_t st) {
-    if constexpr (HI <= 8) {
-        if (ncol == 16) return launch_score_t<HI, DI, 16, MODE>(p, n_keys_max, st);
-    }
+static int launch_score_n(const IdxParams &p, bool decode, long long n_keys_max, cudaStream_t st) {
+    if (decode) return launch_dp4a_t<DI, MODE>(p, n_keys_max, st);
     return launch_score_t<HI, DI, 256, MODE>(p, n_keys_max, st);
 }
 
 template <int MODE>
-static int launch_score(const IdxParams &p, int ncol, long long n_keys_max, cudaStream_t st) {
+static int launch_score(const IdxParams &p, bool decode, long long n_keys_max, cudaStream_t st) {
 #define SA_SCORE_DI(HI)                                                                 \
-    if (p.di == 32) return launch_score_n<HI, 32, MODE>(p, ncol, n_keys_max, st);      \
-    if (p.di == 64) return launch_score_n<HI, 64, MODE>(p, ncol, n_keys_max, st);      \
-    return launch_score_n<HI, 128, MODE>(p, ncol, n_keys_max, st);
+    if (p.di == 32) return launch_score_n<HI, 32, MODE>(p, decode, n_keys_max, st);    \
+    if (p.di == 64) return launch_score_n<HI, 64, MODE>(p, decode, n_keys_max, st);    \
+    return launch_score_n<HI, 128, MODE>(p, decode, n_keys_max, st);
     switch (p.Hi) {
         case 1: { SA_SCORE_DI(1) }
         case 2: { SA_SCORE_DI(2) }
@@ -418,7 +436,7 @@ int sa_indexer_topk(const int8_t *q_idx, const int8_t *k_idx, const int32_t *w, 
     const long long n_max_all = std::max(0LL, (long long)(window > 0 ? q_pos0 + Tq - window : q_pos0 + Tq));
     if (n_max_all > SEL_MAX_N)
         return fail(SA_ERR_UNSUPPORTED, "indexer_topk: %lld candidates per query exceed %d", n_max_all, SEL_MAX_N);
-    const IdxLayout lay = indexer_layout(B, Tq, Hi, topk);
+    const IdxLayout lay = indexer_layout(B, Tq, L, Hi, topk);
     if (!workspace || workspace_bytes < lay.total)
         return fail(SA_ERR_WORKSPACE, "indexer_topk: workspace %zu < %zu", workspace_bytes, lay.total);
     if (!aligned16(workspace)) return fail(SA_ERR_INVALID_ARG, "indexer_topk: workspace alignment");
@@ -447,11 +465,11 @@ int sa_indexer_topk(const int8_t *q_idx, const int8_t *k_idx, const int32_t *w, 
         cudaError_t e = cudaMemsetAsync(p.cand_cnt, 0, (size_t)B * rows * 4, st);
         if (e != cudaSuccess) return fail(SA_ERR_CUDA, "memset: %s", cudaGetErrorString(e));
         if (ncand > 0) {
-            rc = launch_score<MODE_SAMPLE>(p, lay.ncol, (long long)lay.m_cap, st);
+            rc = launch_score<MODE_SAMPLE>(p, lay.decode, (long long)lay.m_cap, st);
             if (rc) return rc;
             idx_threshold_kernel<<<dim3(1u, (unsigned)rows, (unsigned)B), SEL_THREADS, 0, st>>>(p);
             SA_CHECK_LAUNCH("idx_threshold_kernel");
-            rc = launch_score<MODE_FILTER>(p, lay.ncol, ncand, st);
+            rc = launch_score<MODE_FILTER>(p, lay.decode, ncand, st);
             if (rc) return rc;
         }
         const int words = (int)((std::max(ncand, 1LL) + 31) / 32);
