@@ -16,7 +16,7 @@ import torch
 from . import _lib
 from ._lib import SAError, check, sa_dsa_layer, sa_pattern
 
-__all__ = ["indexer_topk", "sparse_attn_fwd", "lse_combine", "nsa_fwd",
+__all__ = ["indexer_topk", "sparse_attn_fwd", "sparse_attn_fwd_split_static", "lse_combine", "nsa_fwd",
            "dsa_decode_layers", "check_device_status", "SAError"]
 
 
@@ -153,6 +153,47 @@ def sparse_attn_fwd(q, k, v, idx=None, pattern: Optional[Sequence[int]] = None,
             "sa_sparse_attn_fwd")
     if return_partials:
         return out, lse, po, pl
+    return out, lse
+
+
+def sparse_attn_fwd_split_static(q, k, v, idx, n_split: int, scale: Optional[float] = None,
+                                 q_pos0: Optional[int] = None, out=None, lse=None):
+    """Split-KV sparse attention over index lists that allocates no device
+    memory (sa_sparse_attn_fwd_split_static).
+
+    For callers that cannot allocate at call time; the partial results live in
+    a fixed 8 MiB array inside the library, so n_split*B*Tq*Hq*(d+1)*4 bytes
+    must fit in it, and calls that may overlap on the GPU must be ordered by
+    the caller.  Pass out/lse to allocate nothing here either.
+    """
+    lib = _lib.load()
+    dev = q.device
+    _need(q, "q", torch.bfloat16, dev, 4)
+    _need(k, "k", torch.bfloat16, dev, 4)
+    _need(v, "v", torch.bfloat16, dev, 4)
+    _need(idx, "idx", torch.int32, dev)
+    B, Tq, Hq, d = q.shape
+    L, Hkv = k.shape[1], k.shape[2]
+    if k.shape != (B, L, Hkv, d) or v.shape != k.shape:
+        raise ValueError("sparse_attn_fwd_split_static: k/v shape mismatch")
+    if idx.dim() == 3:
+        idx_heads, K = 1, idx.shape[2]
+    elif idx.dim() == 4:
+        idx_heads, K = idx.shape[2], idx.shape[3]
+    else:
+        raise ValueError("idx must be [B,Tq,K] or [B,Tq,idx_heads,K]")
+    pos0 = L - Tq if q_pos0 is None else int(q_pos0)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((B, Tq, Hq, d), dtype=torch.bfloat16, device=dev)
+    if lse is None:
+        lse = torch.empty((B, Tq, Hq), dtype=torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        check(lib.sa_sparse_attn_fwd_split_static(
+            _ptr(q), _ptr(k), _ptr(v), B, Tq, L, Hq, Hkv, d, pos0, _ptr(idx), idx_heads, K,
+            float(scale), int(n_split), _ptr(out), _ptr(lse), _stream(dev)),
+            "sa_sparse_attn_fwd_split_static")
     return out, lse
 
 

@@ -283,6 +283,65 @@ int sa_sparse_attn_fwd(const void *q, const void *k, const void *v, int B, int T
     return SA_OK;
 }
 
+// --------------------------------------- split-KV without any allocation --
+// Some callers cannot allocate device memory when they call us: a serving
+// runtime whose device memory is all handed out up front, plugin hosts that
+// pass only input/output buffers, or paths where a cudaMalloc would
+// synchronise the device.  For them
+// the split-KV attention keeps its partial results in a fixed array that is
+// part of the library image instead of a caller workspace.  The array is
+// 8 MiB per GPU that loads the library and lives until the process exits.
+static constexpr size_t kStaticSplitBytes = (size_t)8 << 20;
+static __device__ __align__(256) unsigned char g_static_split[kStaticSplitBytes];
+static unsigned char *g_static_split_ptr[kMaxDevices];
+static std::mutex g_static_split_mu;
+
+// Device address of this device's copy of the array.  Host code must not use
+// the symbol itself as a device pointer: the address is looked up once per
+// device, with that device current, on its first call.
+static int static_split_scratch(unsigned char **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(SA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (dev < 0 || dev >= kMaxDevices) return fail(SA_ERR_UNSUPPORTED, "device id %d", dev);
+    std::lock_guard<std::mutex> lk(g_static_split_mu);
+    if (!g_static_split_ptr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_static_split);
+        if (e != cudaSuccess)
+            return fail(SA_ERR_CUDA, "cudaGetSymbolAddress(static split scratch): %s", cudaGetErrorString(e));
+        g_static_split_ptr[dev] = static_cast<unsigned char *>(p);
+    }
+    *out = g_static_split_ptr[dev];
+    return SA_OK;
+}
+
+int sa_sparse_attn_fwd_split_static(const void *q, const void *k, const void *v, int B, int Tq, int L,
+                                    int Hq, int Hkv, int d, int64_t q_pos0, const int32_t *idx,
+                                    int idx_heads, int K, float scale, int n_split, void *out,
+                                    float *lse, void *stream) {
+    if (n_split < 2) return fail(SA_ERR_INVALID_ARG, "split_static: n_split must be >= 2 (got %d)", n_split);
+    if (!idx || !out) return fail(SA_ERR_INVALID_ARG, "split_static: idx and out are required");
+    if (B <= 0 || Tq < 0 || Hq <= 0 || (d != 64 && d != 128))
+        return fail(SA_ERR_INVALID_ARG, "split_static: bad sizes B=%d Tq=%d Hq=%d d=%d", B, Tq, Hq, d);
+    const size_t rows = (size_t)B * Tq * Hq;
+    const size_t o_bytes = round_up((size_t)n_split * rows * d * 4, 256);
+    const size_t need = o_bytes + round_up((size_t)n_split * rows * 4, 256);
+    if (need > kStaticSplitBytes)
+        return fail(SA_ERR_WORKSPACE,
+                    "split_static: partials need %zu bytes but the built-in scratch holds %zu "
+                    "(n_split * B * Tq * Hq * (d + 1) * 4 must fit); use sa_sparse_attn_fwd with a workspace",
+                    need, kStaticSplitBytes);
+    if (Tq == 0) return SA_OK;
+    unsigned char *scratch = nullptr;
+    int rc = static_split_scratch(&scratch);
+    if (rc) return rc;
+    float *po = reinterpret_cast<float *>(scratch);
+    float *pl = reinterpret_cast<float *>(scratch + o_bytes);
+    return sa_sparse_attn_fwd(q, k, v, B, Tq, L, Hq, Hkv, d, q_pos0, idx, idx_heads, K, nullptr, nullptr,
+                              nullptr, nullptr, scale, n_split, out, lse, po, pl, nullptr, 0, stream);
+}
+
 int sa_lse_combine(const float *part_o, const float *part_lse, int n_split, int64_t rows, int d,
                    void *out, float *lse, void *stream) {
     if (n_split < 1 || rows < 0) return fail(SA_ERR_INVALID_ARG, "lse_combine: n_split=%d rows=%lld", n_split, (long long)rows);

@@ -130,6 +130,32 @@ int sa_sparse_attn_fwd(const void *q, const void *k, const void *v,
                        void *workspace, size_t workspace_bytes, void *stream);
 
 /* --------------------------------------------------------------------------
+ * Split-KV sparse attention that allocates nothing.  No page has a
+ * counterpart: this is a convenience entry point of this library.
+ * For callers that cannot allocate device memory at call time: a serving
+ * runtime whose device memory is all handed out up front, a plugin host that
+ * passes only input and output buffers, or a path where an allocation would
+ * synchronise the device.  Same operation and
+ * layouts as sa_sparse_attn_fwd in idx mode with n_split >= 2 and no bias;
+ * the pieces are always merged into out (and lse when non-NULL).
+ * The partial results live in an 8 MiB array inside the library image, one
+ * per GPU that loads the library, held until the process exits:
+ *   round_up(n_split*B*Tq*Hq*d*4, 256) + round_up(n_split*B*Tq*Hq*4, 256)
+ * must not exceed 8388608 bytes, else SA_ERR_WORKSPACE is returned before
+ * anything is enqueued.  The first call on a device looks up the array's
+ * device address with that device current; make that first call before any
+ * stream capture.  Every call reuses the same array: calls that may overlap
+ * on the GPU (other streams, other host threads) race and must be ordered by
+ * the caller.  Nothing needs clearing between calls (every piece writes all
+ * of its partial rows before the merge reads them).
+ * ------------------------------------------------------------------------ */
+int sa_sparse_attn_fwd_split_static(const void *q, const void *k, const void *v,
+                                    int B, int Tq, int L, int Hq, int Hkv, int d, int64_t q_pos0,
+                                    const int32_t *idx, int idx_heads, int K,
+                                    float scale, int n_split,
+                                    void *out, float *lse, void *stream);
+
+/* --------------------------------------------------------------------------
  * Log-sum-exp combine (Star Attention page, body: distributed softmax).
  *   lse = log sum_s exp(part_lse[s]),  out = sum_s exp(part_lse[s] - lse) part_o[s]
  * A piece with part_lse = -inf contributes nothing; all empty -> out = 0,
