@@ -50,6 +50,22 @@ def aggregate(times_ms, units_per_rank):
     return sum(units_per_rank) / (t / 1e3), t
 
 
+def rank_env(environ=None):
+    """(world, rank, local_rank) from the torchrun environment (1, 0, 0 alone)."""
+    env = os.environ if environ is None else environ
+    return (int(env.get("WORLD_SIZE", "1")), int(env.get("RANK", "0")),
+            int(env.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(x: float, device, torch, dist) -> float:
+    """Largest value of x over all ranks (x itself without a process group).
+    Every rank must call it at the same point."""
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def parse_clocks(csv_text: str):
     """Summarise `nvidia-smi --query-gpu=... -lms` samples taken while timing."""
     sm, mx, reasons = [], 0.0, set()
@@ -144,9 +160,7 @@ def main():
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = rank_env()
 
     if args.impl == "reference":
         if rank == 0:
@@ -213,12 +227,8 @@ def main():
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
-    total_ms = sum(times)
-    t_all = torch.tensor([total_ms], device=dev)
-    if world > 1:
-        dist.all_reduce(t_all, op=dist.ReduceOp.MAX)
-    tmax_ms = float(t_all.item())
-    value = world * flops * args.steps / (tmax_ms / 1e3) / 1e12
+    tmax_ms = max_over_ranks(sum(times), dev, torch, dist)
+    value = aggregate([tmax_ms], [flops * args.steps] * world)[0] / 1e12
     ms_per_step = tmax_ms / args.steps
     api.check_device_status()
     idx_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_idx[-args.steps:])
@@ -241,10 +251,8 @@ def main():
     e2e_value = None
     if not args.no_e2e:
         e2e_times = timed_steps(e2e_step, max(2, args.steps // 2), args.warmup, flush, dev, torch)
-        e2e_t = torch.tensor([sum(e2e_times)], device=dev)
-        if world > 1:
-            dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
-        e2e_value = world * flops * len(e2e_times) / (float(e2e_t.item()) / 1e3) / 1e12
+        e2e_ms = max_over_ranks(sum(e2e_times), dev, torch, dist)
+        e2e_value = aggregate([e2e_ms], [flops * len(e2e_times)] * world)[0] / 1e12
 
     peaks = _peaks()
     att_tflops = flops / (att_ms / 1e3) / 1e12
@@ -315,6 +323,7 @@ def _peaks():
 
 def extra_measurements(args, dev, torch, api, lib, inputs, flush, world, peaks):
     """Decode (IndexCache), NSA and fixed-graph numbers for the same line."""
+    import torch.distributed as dist
     res = {}
     steps = max(3, args.steps // 2)
     # --- decode 32 x 131072, 4 layers ---
@@ -342,7 +351,7 @@ def extra_measurements(args, dev, torch, api, lib, inputs, flush, world, peaks):
         with torch.cuda.graph(graph):
             dstep()
         times = timed_steps(graph.replay, steps, args.warmup, flush, dev, torch)
-        ms = sum(times) / len(times)
+        ms = max_over_ranks(sum(times), dev, torch, dist) / len(times)
         n_f = pattern.count("F")
         bytes_step = n_f * (w.B * w.T * w.di) + w.layers * (w.B * w.topk * 2 * w.d * 2 +
                                                             w.B * w.Hq * w.d * 2 * 2)
@@ -368,7 +377,7 @@ def extra_measurements(args, dev, torch, api, lib, inputs, flush, world, peaks):
         _, _, sel = api.nsa_fwd(gd["q"], gd["k"], gd["v"], gd["gates"], out=o, **cfg)
         sel_holder["sel"] = sel
     times = timed_steps(nstep, max(2, steps // 2), args.warmup, flush, dev, torch)
-    ms = sum(times) / len(times)
+    ms = max_over_ranks(sum(times), dev, torch, dist) / len(times)
     nsa_fl = nsa_flops(w, sel_holder["sel"], torch)
     res["nsa64k"] = {"ms_per_step": round(ms, 3), "tflops": round(nsa_fl / (ms / 1e3) / 1e12, 2),
                      "algorithmic_flops": nsa_fl,
@@ -386,7 +395,7 @@ def extra_measurements(args, dev, torch, api, lib, inputs, flush, world, peaks):
         api.sparse_attn_fwd(gd["q"], gd["k"], gd["v"], pattern=(w.window, w.dilated), cq=gd["cq"],
                             ck=gd["ck"], beta=gd["beta"], out=o, lse=ls)
     times = timed_steps(sstep, steps, args.warmup, flush, dev, torch)
-    ms = sum(times) / len(times)
+    ms = max_over_ranks(sum(times), dev, torch, dist) / len(times)
     byts = sum(gd[k].numel() * gd[k].element_size() for k in ("q", "k", "v", "cq", "ck")) + \
         o.numel() * 2 + ls.numel() * 4
     res["spatial16k"] = {"ms_per_step": round(ms, 4), "gbs": round(byts / (ms / 1e3) / 1e9, 1),
