@@ -18,6 +18,7 @@ Under torchrun every rank runs; rank 0 prints one JSON line.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import math
 import os
@@ -154,6 +155,9 @@ def main():
     ap.add_argument("--no-extra", action="store_true", help="skip decode/NSA/fixed-graph lines")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline leg")
+    ap.add_argument("--seq-len", type=int, default=0,
+                    help="prefill length for profiling captures of a smaller case "
+                         "(default: the 65536-token workload); the JSON line names it")
     ap.add_argument("--cpu-sample-rows", type=int, default=0,
                     help="oracle rows for the CPU baseline (0 = auto, ~10-30 s)")
     args = ap.parse_args()
@@ -181,6 +185,8 @@ def main():
 
     lib = _lib.load()
     w = inputs.WORKLOADS["dsa_prefill64k"]
+    if args.seq_len:
+        w = dataclasses.replace(w, T=int(args.seq_len))
     g = inputs.gen_dsa(w.B, w.T, w.Hq, w.Hkv, w.d, w.Hi, w.di, seed=rank)
     gd = {k: v.to(dev) for k, v in g.items()}
     flush_buf = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
@@ -269,8 +275,8 @@ def main():
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded; q/k/v N(0,1) bf16, indexer int8 U[-8,8], weights U{0..4})",
-        "config": {"workload": "dsa_prefill64k: indexer top-2048 + sparse attention, "
-                               "1 x 65536 tokens, 16 q heads / 1 kv head, d=128",
+        "config": {"workload": f"dsa_prefill{w.T // 1024}k: indexer top-2048 + sparse attention, "
+                               f"1 x {w.T} tokens, 16 q heads / 1 kv head, d=128",
                    "global_batch": world, "seq_len": w.T, "topk": w.topk,
                    "attn_flops_per_seq": flops, "l2": "flushed between steps (252 MB write)",
                    "parallelism": f"replicas x{world} (one sequence per GPU)"},

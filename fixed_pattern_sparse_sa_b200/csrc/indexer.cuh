@@ -94,14 +94,36 @@ __device__ __forceinline__ int tc_core_off(int row, int chunk, int di) {
 // Key tiles are staged through a ring of TC_AS buffers (TC_AS - 1 in flight).
 constexpr int TC_AS = 4;
 
+// Filter pass with at most TC_LIST_NQ queries per CTA: the kept (score, key)
+// pairs of a tile go to per-query lists in shared memory (double-buffered,
+// TC_LCAP = 128 entries = one tile's keys, so they cannot overflow) and are
+// copied to the global lists one tile later, with one global atomic per
+// (query, tile) whose latency hides behind the next tile's epilogue.
+constexpr int TC_LIST_NQ = 32;
+constexpr int TC_LCAP = 128;
+template <int HI, int NCOL, int MODE>
+__host__ __device__ constexpr bool tc_lists() {
+    return MODE == 1 && NCOL / HI <= TC_LIST_NQ;
+}
+template <int HI, int NCOL>
+__host__ __device__ constexpr int tc_list_bytes() {
+    return (3 * (NCOL / HI) * 4 + 2 * (NCOL / HI) * TC_LCAP * 5 + 15) / 16 * 16;
+}
+
 // Shared memory of one score CTA; at least 80 KB for NCOL = 256 so that at
 // most two CTAs (2 x 256 TMEM columns) share an SM.
-template <int DI, int NCOL>
+template <int HI, int DI, int NCOL, int MODE>
 __host__ __device__ constexpr int tc_smem_bytes() {
-    return (NCOL >= 256 && TC_AS * 128 * DI + NCOL * DI + NCOL * 8 + 64 < 80 * 1024)
+    return (NCOL >= 256 &&
+            TC_AS * 128 * DI + NCOL * DI + NCOL * 8 + 64 + (tc_lists<HI, NCOL, MODE>() ? tc_list_bytes<HI, NCOL>() : 0) <
+                80 * 1024)
                ? 80 * 1024
-               : TC_AS * 128 * DI + NCOL * DI + NCOL * 8 + 64;
+               : TC_AS * 128 * DI + NCOL * DI + NCOL * 8 + 64 +
+                     (tc_lists<HI, NCOL, MODE>() ? tc_list_bytes<HI, NCOL>() : 0);
 }
+
+// S + max(x, 0) as one add-then-max: max(S + x, S).
+__device__ __forceinline__ int add_relu(int S, int x) { return __viaddmax_s32(S, x, S); }
 
 template <int HI, int DI, int NCOL, int MODE>
 __global__ void __launch_bounds__(tc_threads(NCOL), NCOL >= 64 ? 2 : 4) idx_score_tc_kernel(const IdxParams p) {
@@ -117,7 +139,10 @@ __global__ void __launch_bounds__(tc_threads(NCOL), NCOL >= 64 ? 2 : 4) idx_scor
     static_assert(NCOL % 16 == 0 && NCOL >= 16 && NCOL <= 256 && NCOL % HI == 0, "NCOL");
     static_assert(HI <= STEP, "the heads of a query must lie within one step of one warp");
     static_assert(HALF >= 16 || PARTS == 2, "16-column tiles use two column parts");
-    static_assert(TC_AS * A_BYTES + B_BYTES + NCOL * 8 + 64 <= tc_smem_bytes<DI, NCOL>(), "smem");
+    constexpr bool LISTS = tc_lists<HI, NCOL, MODE>();
+    static_assert(TC_AS * A_BYTES + B_BYTES + NCOL * 8 + 64 + (LISTS ? tc_list_bytes<HI, NCOL>() : 0) <=
+                      tc_smem_bytes<HI, DI, NCOL, MODE>(), "smem");
+    constexpr int NWARPS = TC_THREADS / 32;
     constexpr uint32_t IDESC = tc::make_idesc(2 /*s32*/, 1 /*s8*/, 128, NCOL);
 
     extern __shared__ __align__(1024) unsigned char smem[];
@@ -129,6 +154,12 @@ __global__ void __launch_bounds__(tc_threads(NCOL), NCOL >= 64 ? 2 : 4) idx_scor
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + 1);
     int *fold_bad = reinterpret_cast<int *>(tmem_slot + 1);
     int *wait_ok = fold_bad + 1;
+    // per-query tile lists (filter pass): counts [2][NQ], global bases [NQ],
+    // scores [2][NQ][TC_LCAP], key offsets within the tile [2][NQ][TC_LCAP]
+    int *lcnt_s = reinterpret_cast<int *>(smem + TC_AS * A_BYTES + B_BYTES + NCOL * 8 + 64);
+    int *lbase_s = lcnt_s + 2 * NQ;
+    int *lval_s = lbase_s + NQ;
+    uint8_t *loff_s = reinterpret_cast<uint8_t *>(lval_s + 2 * NQ * TC_LCAP);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int b = blockIdx.z;
@@ -162,6 +193,9 @@ __global__ void __launch_bounds__(tc_threads(NCOL), NCOL >= 64 ? 2 : 4) idx_scor
             const int tq = tq0 + i;
             tau_s[i] = tq <= tq_last ? p.tau[(long long)b * p.Rt + (tq - p.t0)] : INT_MAX;
         }
+    }
+    if constexpr (LISTS) {
+        for (int i = tid; i < 2 * NQ; i += TC_THREADS) lcnt_s[i] = 0;
     }
     __syncthreads();
     // B tile (rows (q, h) of q_idx are contiguous in memory), weights folded in
@@ -239,6 +273,40 @@ __global__ void __launch_bounds__(tc_threads(NCOL), NCOL >= 64 ? 2 : 4) idx_scor
         }
     };
     if (NQH == GQ) load_query_consts(0);
+    // Filter-pass lists: global row of CTA query q, and the copy of tile kt's
+    // shared list (buffer kt & 1) to the global list at the base reserved
+    // for it; each query's list is copied and then cleared by warp q % NWARPS.
+    auto list_row = [&](int q) -> long long { return (long long)b * p.Rt + (tq0 + q - p.t0); };
+    auto copy_lists = [&](int kt_done) {
+        const int buf = kt_done & 1;
+        const int key0 = j_cta + kt_done * 128;
+        for (int q = warp; q < NQ; q += NWARPS) {
+            const int n = lcnt_s[buf * NQ + q];
+            if (n == 0) continue;                              // warp-uniform
+            const int base = lbase_s[q];
+            const long long roff = list_row(q) * p.cand_cap;
+            for (int e = lane; e < n; e += 32) {
+                const int slot = base + e;
+                if (slot < p.cand_cap) {
+                    p.cand_val[roff + slot] = lval_s[(buf * NQ + q) * TC_LCAP + e];
+                    p.cand_idx[roff + slot] = key0 + loff_s[(buf * NQ + q) * TC_LCAP + e];
+                }
+            }
+            __syncwarp();
+            if (lane == 0) lcnt_s[buf * NQ + q] = 0;
+        }
+    };
+    // one global atomic per (query, tile): lane q of warp 0 reserves room for
+    // tile kt_done's list of query q and returns the base
+    auto reserve_lists = [&](int kt_done) -> int {
+        int base = 0;
+        if (lane < NQ) {
+            const int n = lcnt_s[(kt_done & 1) * NQ + lane];
+            if (n > 0) base = atomicAdd(p.cand_cnt + list_row(lane), n);
+        }
+        return base;
+    };
+
     bool timed_out = false;
     uint32_t pending = 0;   // parity of the MMA batch in flight
     for (int kt = 0; kt < n_tiles; ++kt) {
@@ -255,6 +323,8 @@ __global__ void __launch_bounds__(tc_threads(NCOL), NCOL >= 64 ? 2 : 4) idx_scor
             }
             tc::mma_commit(bar);
         }
+        int list_base = 0;                                     // warp 0: bases for tile kt-1
+        if (LISTS && warp == 0 && kt > 0) list_base = reserve_lists(kt - 1);
         load_a(kt + TC_AS - 1);                                // buffer of tile kt-1: its MMA is done
         // one thread waits (bounded) and the whole CTA follows its verdict
         if (tid == 0) *wait_ok = tc::mbar_wait_bounded(bar, kt & 1, TC_WAIT_CYCLES) ? 1 : 0;
@@ -296,7 +366,7 @@ __global__ void __launch_bounds__(tc_threads(NCOL), NCOL >= 64 ? 2 : 4) idx_scor
                     int v = 0;
                     if (fold) {
 #pragma unroll
-                        for (int h = 0; h < HPL; ++h) v += max((int)r[qq * HPL + h], 0);
+                        for (int h = 0; h < HPL; ++h) v = add_relu(v, (int)r[qq * HPL + h]);
                     } else {
                         const int cw = c_begin + g0 * HI + c + qq * HPL;
 #pragma unroll
@@ -312,6 +382,22 @@ __global__ void __launch_bounds__(tc_threads(NCOL), NCOL >= 64 ? 2 : 4) idx_scor
 #pragma unroll
                 for (int q = 0; q < GQ; ++q)
                     if (jj < nt_r[q]) p.sample[(long long)(row0 + q) * p.m_cap + i_key] = sc[q];
+            } else if constexpr (LISTS) {
+                // kept pairs go to this tile's shared list of their query
+                const int buf = kt & 1;
+                // causal test j < n_candidates(position of query q) as dd < q;
+                // queries past the chunk have tau = INT_MAX
+                const long long ddl = j + (p.window > 0 ? p.window : 0) - 1 - (p.q_pos0 + tq0 + q_first);
+                const int dd = (int)max(min(ddl, (long long)GQ), -1LL);
+#pragma unroll
+                for (int q = 0; q < GQ; ++q) {
+                    if ((dd < q) & (sc[q] >= tau_r[q])) {
+                        const int lq = buf * NQ + q_first + q;
+                        const int slot = atomicAdd(lcnt_s + lq, 1);
+                        lval_s[lq * TC_LCAP + slot] = sc[q];
+                        loff_s[lq * TC_LCAP + slot] = (uint8_t)(quad * 32 + lane);
+                    }
+                }
             } else {
                 unsigned ball[GQ];
                 unsigned keepm = 0u;
@@ -338,12 +424,21 @@ __global__ void __launch_bounds__(tc_threads(NCOL), NCOL >= 64 ? 2 : 4) idx_scor
                 }
             }
         }
+        if (LISTS && warp == 0 && kt > 0 && lane < NQ) lbase_s[lane] = list_base;
         // the next MMA overwrites the accumulator and reads tile kt+1's buffer
         tc::fence_before_sync();
         cp_async_wait<TC_AS - 2>();
         tc::fence_proxy_async_smem();
         __syncthreads();
         tc::fence_after_sync();
+        if (LISTS && kt > 0) copy_lists(kt - 1);
+    }
+    if (LISTS && !timed_out) {                                 // the last tile's lists
+        const int base = warp == 0 ? reserve_lists(n_tiles - 1) : 0;
+        __syncthreads();                                       // tile n_tiles-2's copies are done
+        if (warp == 0 && lane < NQ) lbase_s[lane] = base;
+        __syncthreads();
+        copy_lists(n_tiles - 1);
     }
     if (timed_out) {
         cp_async_wait<0>();

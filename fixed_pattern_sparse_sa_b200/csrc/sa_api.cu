@@ -425,7 +425,7 @@ size_t sa_indexer_topk_workspace_size(int B, int Tq, int L, int Hi, int di, int 
 template <int HI, int DI, int NCOL, int MODE>
 static int launch_score_t(const IdxParams &p, long long n_keys_max, cudaStream_t st) {
     constexpr int NQ = NCOL / HI;
-    constexpr int smem = tc_smem_bytes<DI, NCOL>();
+    constexpr int smem = tc_smem_bytes<HI, DI, NCOL, MODE>();
     auto kern = idx_score_tc_kernel<HI, DI, NCOL, MODE>;
     int rc = set_smem(kern, smem);
     if (rc) return rc;
