@@ -527,6 +527,134 @@ __global__ void __launch_bounds__(DEC_THREADS) idx_score_dp4a_kernel(const IdxPa
     }
 }
 
+// ------------------------------------- decode-shaped scores, tensor cores --
+// One query row and 8 indexer heads of width 64: per 16 keys, two
+// mma.sync m16n8k32 (s8 x s8 -> s32) give the 16 x 8 head scores.  The
+// contraction index is permuted identically on both operands (a dot product
+// does not depend on the order of its terms) so that every thread's share of
+// a key row is one contiguous 16-byte load: logical byte s*32 + h*16 + 4c + e
+// (MMA slice s, fragment half h, thread quad c) lives at physical byte
+// 16c + 8s + 4h + e of the 64-byte row.  A warp's loads cover 8 whole rows
+// per instruction.  Kept (score, key) pairs collect in a per-CTA shared list
+// and reach the global list with one atomic per CTA.
+constexpr int DMMA_THREADS = 256;
+constexpr int DMMA_KEYS = 4096;                 // keys per CTA (512 per warp)
+constexpr int DMMA_U = 4;                       // 16-key groups per warp in flight
+
+template <int MODE>
+__global__ void __launch_bounds__(DMMA_THREADS) idx_score_dec_mma_kernel(const IdxParams p) {
+    constexpr int DI = 64, HI = 8;
+    __shared__ int lcnt_s, lbase_s;
+    __shared__ int lval_s[MODE == MODE_FILTER ? DMMA_KEYS : 1];
+    __shared__ int lidx_s[MODE == MODE_FILTER ? DMMA_KEYS : 1];
+    const int b = blockIdx.z, tr = blockIdx.y, t = p.t0 + tr;
+    if (t >= p.Tq || tr >= p.Rt) return;
+    const long long nt = n_candidates(p.q_pos0 + t, p.window);
+    const int stride = MODE == MODE_SAMPLE ? sample_stride(p, t) : 1;
+    const long long n_keys = MODE == MODE_SAMPLE ? (nt + stride - 1) / stride : nt;
+    const long long i0 = (long long)blockIdx.x * DMMA_KEYS;
+    if (i0 >= n_keys) return;                                       // uniform
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g = lane >> 2, c = lane & 3;
+    const long long row = (long long)b * p.Rt + tr;
+    if (MODE == MODE_FILTER && tid == 0) lcnt_s = 0;
+
+    // B operand: head n = g, this thread's 16 permuted bytes of q
+    const int8_t *qrow = p.q + (((long long)b * p.Tq + t) * HI + g) * DI;
+    int4 qv = __ldg(reinterpret_cast<const int4 *>(qrow) + c);
+    const int wn = __ldg(p.w + ((long long)b * p.Tq + t) * HI + g);   // weight of head g
+    // weights of the two heads whose scores this thread holds (2c, 2c+1)
+    const int w0 = __shfl_sync(0xffffffffu, wn, (2 * c) << 2);
+    const int w1 = __shfl_sync(0xffffffffu, wn, (2 * c + 1) << 2);
+    bool fold_ok = wn >= 0;
+    {
+        int words[4] = {qv.x, qv.y, qv.z, qv.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            unsigned packed = 0;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int x = (int)(signed char)((words[u] >> (8 * e)) & 0xff) * wn;
+                fold_ok &= (x >= -128) & (x <= 127);
+                packed |= ((unsigned)x & 0xffu) << (8 * e);
+            }
+            words[u] = (int)packed;
+        }
+        if (__all_sync(0xffffffffu, fold_ok)) qv = make_int4(words[0], words[1], words[2], words[3]);
+        else fold_ok = false;
+    }
+    const bool fold = __all_sync(0xffffffffu, fold_ok);
+    const int tau = MODE == MODE_FILTER ? p.tau[row] : 0;
+    if (MODE == MODE_FILTER) __syncthreads();                       // lcnt_s initialised
+
+    const int8_t *kb = p.k + (long long)b * p.L * DI;
+    const long long wbeg = i0 + (long long)warp * (DMMA_KEYS / 8);
+    const long long wend = min(wbeg + DMMA_KEYS / 8, n_keys);
+    for (long long gb = wbeg; gb < wend; gb += 16 * DMMA_U) {
+        int4 ka[DMMA_U], kc8[DMMA_U];                               // rows g and g + 8 of each group
+#pragma unroll
+        for (int u = 0; u < DMMA_U; ++u) {
+            const long long ia = gb + 16 * u + g, ib = ia + 8;
+            const long long ja = (long long)stride * ia, jb = (long long)stride * ib;
+            ka[u] = (ia < wend && ja < p.L) ? __ldg(reinterpret_cast<const int4 *>(kb + ja * DI) + c) : make_int4(0, 0, 0, 0);
+            kc8[u] = (ib < wend && jb < p.L) ? __ldg(reinterpret_cast<const int4 *>(kb + jb * DI) + c) : make_int4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < DMMA_U; ++u) {
+            int acc[4] = {0, 0, 0, 0};
+            mma_s8_16832(acc, (unsigned)ka[u].x, (unsigned)kc8[u].x, (unsigned)ka[u].y, (unsigned)kc8[u].y,
+                         (unsigned)qv.x, (unsigned)qv.y);
+            mma_s8_16832(acc, (unsigned)ka[u].z, (unsigned)kc8[u].z, (unsigned)ka[u].w, (unsigned)kc8[u].w,
+                         (unsigned)qv.z, (unsigned)qv.w);
+            // acc: (key g, heads 2c, 2c+1), (key g+8, heads 2c, 2c+1)
+            int va, vb;
+            if (fold) {
+                va = max(acc[0], 0) + max(acc[1], 0);
+                vb = max(acc[2], 0) + max(acc[3], 0);
+            } else {
+                va = w0 * max(acc[0], 0) + w1 * max(acc[1], 0);
+                vb = w0 * max(acc[2], 0) + w1 * max(acc[3], 0);
+            }
+            va += __shfl_xor_sync(0xffffffffu, va, 1);
+            va += __shfl_xor_sync(0xffffffffu, va, 2);
+            vb += __shfl_xor_sync(0xffffffffu, vb, 1);
+            vb += __shfl_xor_sync(0xffffffffu, vb, 2);
+            const long long ia = gb + 16 * u + g, ib = ia + 8;
+            if (c == 0) {
+                if constexpr (MODE == MODE_SAMPLE) {
+                    if (ia < wend) p.sample[row * p.m_cap + ia] = va;
+                    if (ib < wend) p.sample[row * p.m_cap + ib] = vb;
+                } else {
+                    if (ia < wend && va >= tau) {
+                        const int sl = atomicAdd(&lcnt_s, 1);
+                        lval_s[sl] = va;
+                        lidx_s[sl] = (int)ia;
+                    }
+                    if (ib < wend && vb >= tau) {
+                        const int sl = atomicAdd(&lcnt_s, 1);
+                        lval_s[sl] = vb;
+                        lidx_s[sl] = (int)ib;
+                    }
+                }
+            }
+        }
+    }
+    if constexpr (MODE == MODE_FILTER) {
+        __syncthreads();
+        const int n = lcnt_s;
+        if (tid == 0) lbase_s = n > 0 ? atomicAdd(p.cand_cnt + row, n) : 0;
+        __syncthreads();
+        const int base = lbase_s;
+        for (int e = tid; e < n; e += DMMA_THREADS) {
+            const int slot = base + e;
+            if (slot < p.cand_cap) {
+                p.cand_val[row * p.cand_cap + slot] = lval_s[e];
+                p.cand_idx[row * p.cand_cap + slot] = lidx_s[e];
+            }
+        }
+    }
+}
+
 // ----------------------------------------------------- block helpers --
 constexpr int SEL_THREADS = 256;
 constexpr int SEL_BITS = 8;

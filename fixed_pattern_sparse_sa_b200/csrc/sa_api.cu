@@ -10,12 +10,14 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <string>
 
 #include "../../include/sa.h"
 #include "attn_gather.cuh"
+#include "attn_tc.cuh"
 #include "attn_tile.cuh"
 #include "indexer.cuh"
 #include "nsa_misc.cuh"
@@ -127,6 +129,98 @@ static int launch_gather(const GatherParams &p, int d, int src, bool bias, cudaS
     if (d == 64) return launch_gather_d<64>(p, src, bias, st);
     if (d == 128) return launch_gather_d<128>(p, src, bias, st);
     return fail(SA_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
+}
+
+// ------------------------------------------- tensor-core gather launches --
+typedef CUresult (*TensorMapEncodeFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                      const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
+                                      CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                      CUtensorMapFloatOOBfill);
+
+// The driver's tensor-map encoder, looked up once through the runtime (no
+// link-time dependency on libcuda).
+static TensorMapEncodeFn tensor_map_encoder() {
+    static TensorMapEncodeFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<TensorMapEncodeFn>(f);
+    });
+    return fn;
+}
+
+// 2-D bf16 map over `rows` rows of `cols` contiguous elements; box = 64
+// columns (128 bytes) x box_rows rows, 128-byte swizzle.
+static int bf16_tensor_map(CUtensorMap *m, const void *base, long long rows, int cols, int box_rows) {
+    TensorMapEncodeFn enc = tensor_map_encoder();
+    if (!enc) return fail(SA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+    cuuint32_t es[2] = {1u, 1u};
+    const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(SA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return SA_OK;
+}
+
+static int sm_count() {
+    static int cached[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+    if (!cached[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
+// SA_ATTN_PATH=tc routes explicit-list attention (head dim 128, <= 16 heads
+// per KV head, no bias) through attn_tc_kernel.  It is opt-in: with 64-KB
+// K/V stages it keeps fewer gathered bytes in flight per SM than the
+// per-warp mma.sync kernel and measured slower (5.4 vs 3.4 ms for the
+// 32K-token prefill attention).
+static bool attn_tc_allowed() {
+    static int v = -1;
+    if (v < 0) {
+        const char *e = std::getenv("SA_ATTN_PATH");
+        v = (e && std::strcmp(e, "tc") == 0) ? 1 : 0;
+    }
+    return v != 0;
+}
+
+static bool attn_tc_applies(const GatherParams &p, int d, int src, bool bias) {
+    return attn_tc_allowed() && (src == KS_IDX || src == KS_BLOCKS) && !bias && d == 128 && p.G <= 16 &&
+           !p.klo && (!p.out_f32 || p.n_split == 1) && (long long)p.B * p.Lk * p.Hkv < INT_MAX &&
+           (long long)p.B * p.Tq * p.Hq + 16 < INT_MAX;
+}
+
+template <int SRC>
+static int launch_attn_tc(const GatherParams &p, cudaStream_t st) {
+    const long long items = (long long)p.B * p.Tq * p.Hkv * p.n_split;
+    if (items == 0) return SA_OK;
+    if (items > INT_MAX) return fail(SA_ERR_UNSUPPORTED, "attn_tc: %lld work items", items);
+    CUtensorMap qm;
+    int rc = bf16_tensor_map(&qm, p.q, (long long)p.B * p.Tq * p.Hq, 128, 16);
+    if (rc) return rc;
+    AtcParams ap{};
+    ap.g = p;
+    ap.n_items = (int)items;
+    constexpr int smem = AtcSmem<128>::ALLOC;
+    static_assert(smem <= 227 * 1024, "shared memory");
+    auto kern = attn_tc_kernel<128, SRC>;
+    rc = set_smem(kern, smem);
+    if (rc) return rc;
+    const int grid = (int)std::min<long long>(items, sm_count());
+    kern<<<grid, ATC_THREADS, smem, st>>>(qm, ap);
+    SA_CHECK_LAUNCH("attn_tc_kernel");
+    return SA_OK;
 }
 
 static int launch_combine(const float *po, const float *pl, int n_split, long long rows, int d,
@@ -277,7 +371,7 @@ int sa_sparse_attn_fwd(const void *q, const void *k, const void *v, int B, int T
     p.part_o = po; p.part_lse = pl;
     p.err = ew;
     cudaStream_t st = as_stream(stream);
-    rc = launch_gather(p, d, src, bias, st);
+    rc = attn_tc_applies(p, d, src, bias) ? launch_attn_tc<KS_IDX>(p, st) : launch_gather(p, d, src, bias, st);
     if (rc) return rc;
     if (n_split > 1 && out) return launch_combine(po, pl, n_split, rows, d, out, lse, st);
     return SA_OK;
@@ -444,9 +538,20 @@ static int launch_dp4a_t(const IdxParams &p, long long n_keys_max, cudaStream_t 
     return SA_OK;
 }
 
+template <int MODE>
+static int launch_dec_mma_t(const IdxParams &p, long long n_keys_max, cudaStream_t st) {
+    dim3 grid((unsigned)((n_keys_max + DMMA_KEYS - 1) / DMMA_KEYS), (unsigned)p.Rt, (unsigned)p.B);
+    idx_score_dec_mma_kernel<MODE><<<grid, DMMA_THREADS, 0, st>>>(p);
+    SA_CHECK_LAUNCH("idx_score_dec_mma_kernel");
+    return SA_OK;
+}
+
 template <int HI, int DI, int MODE>
 static int launch_score_n(const IdxParams &p, bool decode, long long n_keys_max, cudaStream_t st) {
-    if (decode) return launch_dp4a_t<DI, MODE>(p, n_keys_max, st);
+    if (decode) {
+        if constexpr (HI == 8 && DI == 64) return launch_dec_mma_t<MODE>(p, n_keys_max, st);
+        return launch_dp4a_t<DI, MODE>(p, n_keys_max, st);
+    }
     return launch_score_t<HI, DI, 256, MODE>(p, n_keys_max, st);
 }
 
@@ -685,7 +790,8 @@ int sa_nsa_fwd(const void *q, const void *k, const void *v, const float *gates, 
         p.Lk = T; p.idx = sel; p.K = sel_topk; p.block = sel_block;
         p.entries = sel_topk * sel_block; p.per_split = p.entries;
         p.out_f32 = o3 + rows * d; p.lse = l3 + rows;
-        rc = launch_gather(p, d, KS_BLOCKS, false, st);
+        rc = attn_tc_applies(p, d, KS_BLOCKS, false) ? launch_attn_tc<KS_BLOCKS>(p, st)
+                                                     : launch_gather(p, d, KS_BLOCKS, false, st);
         if (rc) return rc;
     }
     // 5. window branch -> o3[2], l3[2]

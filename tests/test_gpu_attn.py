@@ -100,6 +100,58 @@ def test_split_kv_partials_and_combine(cuda_ok, n_split):
     assert_lse_close(l2, rl)
 
 
+@pytest.mark.parametrize("Hq,Hkv,idx_heads", [(16, 1, 1), (8, 2, 2), (12, 1, 1)])
+def test_d128_empty_rows_ragged_lists_and_bad_index(cuda_ok, Hq, Hkv, idx_heads):
+    # head dim 128 with at most 16 heads per KV head (the tensor-core gather
+    # path): several 128-key tiles plus a ragged tail, empty rows, a future
+    # index that must be reported and skipped
+    B, T, d, K = 2, 300, 128, 290
+    g = inputs.gen_dsa(B, T, Hq, Hkv, d, 1, 32, seed=21 + Hq)
+    idx = _random_lists(B, T, idx_heads, K, seed=22 + Hq, fill=0.9)
+    idx[1, 40:43] = -1
+    out, lse = api.sparse_attn_fwd(g["q"].cuda(), g["k"].cuda(), g["v"].cuda(), idx.cuda())
+    api.check_device_status()
+    ro, rl = oracle.sparse_attn(g["q"], g["k"], g["v"], idx)
+    assert_out_close(out, ro)
+    assert_lse_close(lse, rl)
+    assert torch.all(out[1, 40:43] == 0)
+    bad = idx.clone()
+    bad[0, 5, 0, 0] = 7                    # query 5 cannot see position 7
+    out2, _ = api.sparse_attn_fwd(g["q"].cuda(), g["k"].cuda(), g["v"].cuda(), bad.cuda())
+    with pytest.raises(SAError):
+        api.check_device_status()
+    skip = bad.clone(); skip[0, 5, 0, 0] = -1
+    ro2, _ = oracle.sparse_attn(g["q"], g["k"], g["v"], skip)
+    assert_out_close(out2, ro2)
+
+
+@pytest.mark.parametrize("n_split", [1, 3])
+def test_tensor_core_gather_path(cuda_ok, n_split):
+    # the opt-in tcgen05 gather kernel (SA_ATTN_PATH=tc), in a fresh process:
+    # ragged lists, empty rows, G = 12 and 16, split pieces
+    import subprocess, sys, os
+    code = (
+        "import torch, numpy as np, oracle\n"
+        "from fixed_pattern_sparse_sa_b200 import api, inputs\n"
+        "import sys; sys.path.insert(0, 'tests')\n"
+        "from _parity import assert_out_close, assert_lse_close\n"
+        "from test_gpu_attn import _random_lists\n"
+        "for Hq, seed in ((16, 41), (12, 42)):\n"
+        "    g = inputs.gen_dsa(2, 300, Hq, 1, 128, 1, 32, seed=seed)\n"
+        "    idx = _random_lists(2, 300, 1, 290, seed=seed + 1, fill=0.9)\n"
+        "    idx[1, 40:43] = -1\n"
+        f"    out, lse = api.sparse_attn_fwd(g['q'].cuda(), g['k'].cuda(), g['v'].cuda(), idx.cuda(), n_split={n_split})\n"
+        "    api.check_device_status()\n"
+        "    ro, rl = oracle.sparse_attn(g['q'], g['k'], g['v'], idx)\n"
+        "    assert_out_close(out, ro); assert_lse_close(lse, rl)\n"
+        "print('ok')\n")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, SA_ATTN_PATH="tc")
+    r = subprocess.run([sys.executable, "-c", code], cwd=root, env=env, capture_output=True, text=True,
+                       timeout=300)
+    assert r.returncode == 0 and "ok" in r.stdout, r.stderr[-2000:]
+
+
 def test_lse_combine_with_empty_pieces(cuda_ok):
     S, R, d = 5, 37, 64
     rng = np.random.default_rng(12)

@@ -75,6 +75,23 @@ def test_decode_rows_multi_cta_clusters(cuda_ok):
     _check_rows(idx, cnt, ref_idx, ref_cnt)
 
 
+@pytest.mark.parametrize("Tq,wlo,whi", [(1, -300, 301), (2, 0, 40), (1, 0, 5)])
+def test_decode_shaped_calls_fold_and_signed_weights(cuda_ok, Tq, wlo, whi):
+    # 8 indexer heads of width 64 with one or two queries per sequence (the
+    # tensor-core decode scorer): weights that fold into the query operand,
+    # weights whose product with q leaves int8, and negative weights
+    gen = torch.Generator().manual_seed(40 + Tq + whi)
+    B, L, Hi, di = 3, 20000, 8, 64
+    q = torch.randint(-128, 128, (B, Tq, Hi, di), generator=gen).to(torch.int8)
+    k = torch.randint(-128, 128, (B, L, di), generator=gen).to(torch.int8)
+    w = torch.randint(wlo, whi, (B, Tq, Hi), generator=gen).to(torch.int32)
+    for topk, window in [(2048, 0), (300, 64)]:
+        idx, cnt = api.indexer_topk(q.cuda(), k.cuda(), w.cuda(), topk, window, q_pos0=L - Tq)
+        ref_idx, ref_cnt = oracle.indexer_topk(q, k, w, topk, window, q_pos0=L - Tq)
+        _check_rows(idx, cnt, ref_idx, ref_cnt)
+    api.check_device_status()
+
+
 def test_prefill64k_sampled_rows_bit_exact(cuda_ok):
     w = inputs.WORKLOADS["dsa_prefill64k"]
     g = inputs.gen_dsa(w.B, w.T, w.Hq, w.Hkv, w.d, w.Hi, w.di, seed=0)
