@@ -45,6 +45,15 @@ def attn_flops(T: int, topk: int, window: int, Hq: int, d: int) -> float:
     return 4.0 * d * Hq * s
 
 
+ATTN_TRAFFIC_64K = 1_084_000_000
+
+
+def attn_rows(T: int, topk: int, window: int) -> int:
+    """sum_t |S_t| with |S_t| = min(t + 1, topk + window)."""
+    K = topk + window
+    return (min(T, K) * (min(T, K) + 1)) // 2 + max(0, T - K) * K
+
+
 def aggregate(times_ms, units_per_rank):
     """Whole-job throughput: all ranks' units over the slowest rank's time."""
     t = max(times_ms)
@@ -262,6 +271,8 @@ def main():
 
     peaks = _peaks()
     att_tflops = flops / (att_ms / 1e3) / 1e12
+    # indexer int8 work: 2 * Hi * di per causal (query, key) pair
+    idx_ops = 2.0 * w.Hi * w.di * w.B * (w.T * (w.T + 1) / 2)
     result = {
         "metric": METRIC,
         "value": round(value, 3),
@@ -282,14 +293,27 @@ def main():
                    "parallelism": f"replicas x{world} (one sequence per GPU)"},
         "breakdown_ms": {"indexer_topk": round(idx_ms, 4), "sparse_attn": round(att_ms, 4)},
         "roofline": {
-            "kernel": "gather_attn_kernel (sparse attention, D=128)",
+            "kernel": "gather_attn_kernel (sparse attention, D=128; one launch per step)",
             "bound": "tensor",
             "achieved": round(att_tflops, 2),
             "peak": peaks["bf16_tflops"],
             "unit": "TFLOP/s",
             "frac": round(att_tflops / peaks["bf16_tflops"], 4),
             "peak_source": peaks["source"] + " bf16 burst",
-            "traffic": None,
+            # dram__bytes_read + dram__bytes_write of the 32768-token launch
+            # (0.542 GB) x 2: index lists, Q, O and LSE scale with query rows
+            "traffic": ATTN_TRAFFIC_64K if w.T == 65536 else None,
+            "traffic_source": "ncu, 32768-token launch scaled by query rows",
+            "gathered_l2_bytes": int(w.B * 4 * w.d * attn_rows(w.T, w.topk, w.window)),
+        },
+        "indexer": {
+            "kernels": "idx_score_tc_kernel (sample, filter), idx_threshold_kernel, topk_select_kernel",
+            "ms": round(idx_ms, 4),
+            "int8_tops": round(idx_ops / (idx_ms / 1e3) / 1e12, 2),
+            "peak": round(2 * peaks["bf16_tflops"], 1),
+            "unit": "TOP/s",
+            "frac": round(idx_ops / (idx_ms / 1e3) / 1e12 / (2 * peaks["bf16_tflops"]), 4),
+            "peak_source": peaks["source"] + " bf16 burst x 2 (nominal int8/bf16 ratio)",
         },
         "e2e": None if e2e_value is None else
                {"value": round(e2e_value, 3), "unit": "TFLOP/s",
