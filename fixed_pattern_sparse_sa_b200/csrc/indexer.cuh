@@ -538,8 +538,10 @@ __global__ void __launch_bounds__(DEC_THREADS) idx_score_dp4a_kernel(const IdxPa
 // per instruction.  Kept (score, key) pairs collect in a per-CTA shared list
 // and reach the global list with one atomic per CTA.
 constexpr int DMMA_THREADS = 256;
-constexpr int DMMA_KEYS = 4096;                 // keys per CTA (512 per warp)
+constexpr int DMMA_KEYS = 4096;                 // keys per CTA in the filter pass (512 per warp)
+constexpr int DMMA_KEYS_SAMPLE = 512;           // sampled keys per CTA (the sample is short)
 constexpr int DMMA_U = 4;                       // 16-key groups per warp in flight
+__host__ __device__ constexpr int dmma_keys(int mode) { return mode == 0 ? DMMA_KEYS_SAMPLE : DMMA_KEYS; }
 
 template <int MODE>
 __global__ void __launch_bounds__(DMMA_THREADS) idx_score_dec_mma_kernel(const IdxParams p) {
@@ -552,7 +554,8 @@ __global__ void __launch_bounds__(DMMA_THREADS) idx_score_dec_mma_kernel(const I
     const long long nt = n_candidates(p.q_pos0 + t, p.window);
     const int stride = MODE == MODE_SAMPLE ? sample_stride(p, t) : 1;
     const long long n_keys = MODE == MODE_SAMPLE ? (nt + stride - 1) / stride : nt;
-    const long long i0 = (long long)blockIdx.x * DMMA_KEYS;
+    constexpr int KPC = dmma_keys(MODE);
+    const long long i0 = (long long)blockIdx.x * KPC;
     if (i0 >= n_keys) return;                                       // uniform
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, c = lane & 3;
@@ -588,8 +591,8 @@ __global__ void __launch_bounds__(DMMA_THREADS) idx_score_dec_mma_kernel(const I
     if (MODE == MODE_FILTER) __syncthreads();                       // lcnt_s initialised
 
     const int8_t *kb = p.k + (long long)b * p.L * DI;
-    const long long wbeg = i0 + (long long)warp * (DMMA_KEYS / 8);
-    const long long wend = min(wbeg + DMMA_KEYS / 8, n_keys);
+    const long long wbeg = i0 + (long long)warp * (KPC / 8);
+    const long long wend = min(wbeg + KPC / 8, n_keys);
     for (long long gb = wbeg; gb < wend; gb += 16 * DMMA_U) {
         int4 ka[DMMA_U], kc8[DMMA_U];                               // rows g and g + 8 of each group
 #pragma unroll

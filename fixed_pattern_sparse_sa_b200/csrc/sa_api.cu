@@ -84,31 +84,55 @@ static int set_smem(K kernel, int bytes) {
     return SA_OK;
 }
 
+static int sm_count() {
+    static int cached[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+    if (!cached[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
 // -------------------------------------------------------- gather launches --
 // Launch shape: 12 warps per CTA streaming 16-key chunks through a 2-stage
 // ring (8 warps when the lo-key tile is also staged); ~198 KB of shared
-// memory, one CTA and 12 gathering warps per SM.
-template <int D, int SRC, bool BIAS, bool KLO = false>
-static int launch_gather_t(const GatherParams &p, cudaStream_t st) {
-#ifndef SA_ATTN_NW
-#define SA_ATTN_NW 12
-#endif
+// memory, one CTA and 12 gathering warps per SM.  Small launches (fewer
+// items than 12 per SM, e.g. decode with a few hundred split pieces) use
+// 4-warp CTAs so that every SM gets work.
+template <int D, int SRC, bool BIAS, bool KLO, int NW>
+static int launch_gather_nw(const GatherParams &p, long long items, cudaStream_t st) {
 #ifndef SA_ATTN_STAGES
 #define SA_ATTN_STAGES 2
 #endif
-    constexpr int NK = 16, NW = KLO ? 8 : SA_ATTN_NW;
+    constexpr int NK = 16;
     constexpr int STAGES = KLO ? 2 : SA_ATTN_STAGES;
     constexpr int smem = gather_smem_bytes<D, STAGES, KLO, NK, NW, SRC == KS_PROWS>();
     static_assert(smem <= 227 * 1024, "shared memory");
     auto kern = gather_attn_kernel<D, STAGES, SRC, BIAS, KLO, NK, NW>;
     int rc = set_smem(kern, smem);
     if (rc) return rc;
-    const long long items = (long long)p.B * p.q_units * p.Hkv * p.n_hchunk * p.n_split;
-    if (items == 0) return SA_OK;
     const long long blocks = (items + NW - 1) / NW;
     kern<<<(unsigned)blocks, NW * 32, smem, st>>>(p);
     SA_CHECK_LAUNCH("gather_attn_kernel");
     return SA_OK;
+}
+
+template <int D, int SRC, bool BIAS, bool KLO = false>
+static int launch_gather_t(const GatherParams &p, cudaStream_t st) {
+#ifndef SA_ATTN_NW
+#define SA_ATTN_NW 12
+#endif
+    const long long items = (long long)p.B * p.q_units * p.Hkv * p.n_hchunk * p.n_split;
+    if (items == 0) return SA_OK;
+    if constexpr (KLO) {
+        return launch_gather_nw<D, SRC, BIAS, KLO, 8>(p, items, st);
+    } else {
+        if (items < (long long)sm_count() * SA_ATTN_NW) return launch_gather_nw<D, SRC, BIAS, KLO, 4>(p, items, st);
+        return launch_gather_nw<D, SRC, BIAS, KLO, SA_ATTN_NW>(p, items, st);
+    }
 }
 
 template <int D>
@@ -169,17 +193,6 @@ static int bf16_tensor_map(CUtensorMap *m, const void *base, long long rows, int
     return SA_OK;
 }
 
-static int sm_count() {
-    static int cached[kMaxDevices];
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
-    if (!cached[dev]) {
-        int n = 0;
-        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-        cached[dev] = n;
-    }
-    return cached[dev];
-}
 
 // SA_ATTN_PATH=tc routes explicit-list attention (head dim 128, <= 16 heads
 // per KV head, no bias) through attn_tc_kernel.  It is opt-in: with 64-KB
@@ -540,7 +553,8 @@ static int launch_dp4a_t(const IdxParams &p, long long n_keys_max, cudaStream_t 
 
 template <int MODE>
 static int launch_dec_mma_t(const IdxParams &p, long long n_keys_max, cudaStream_t st) {
-    dim3 grid((unsigned)((n_keys_max + DMMA_KEYS - 1) / DMMA_KEYS), (unsigned)p.Rt, (unsigned)p.B);
+    constexpr int kpc = dmma_keys(MODE);
+    dim3 grid((unsigned)((n_keys_max + kpc - 1) / kpc), (unsigned)p.Rt, (unsigned)p.B);
     idx_score_dec_mma_kernel<MODE><<<grid, DMMA_THREADS, 0, st>>>(p);
     SA_CHECK_LAUNCH("idx_score_dec_mma_kernel");
     return SA_OK;

@@ -75,6 +75,23 @@ def test_decode_rows_multi_cta_clusters(cuda_ok):
     _check_rows(idx, cnt, ref_idx, ref_cnt)
 
 
+@pytest.mark.parametrize("Hi,di,wlo,whi", [(8, 64, -300, 301), (8, 64, 0, 40), (4, 32, -3, 4), (1, 64, 0, 200)])
+def test_prefill_rows_signed_and_wide_weights(cuda_ok, Hi, di, wlo, whi):
+    # prefill shapes with weights that cannot be folded into the query (the
+    # filter pass then multiplies per head), over several 128-row blocks and
+    # a ragged last block, with and without a forced window
+    gen = torch.Generator().manual_seed(60 + Hi + whi)
+    B, T = 2, 1000
+    q = torch.randint(-128, 128, (B, T, Hi, di), generator=gen).to(torch.int8)
+    k = torch.randint(-128, 128, (B, T, di), generator=gen).to(torch.int8)
+    w = torch.randint(wlo, whi, (B, T, Hi), generator=gen).to(torch.int32)
+    for topk, window in [(64, 0), (200, 32)]:
+        idx, cnt = api.indexer_topk(q.cuda(), k.cuda(), w.cuda(), topk, window)
+        ref_idx, ref_cnt = oracle.indexer_topk(q, k, w, topk, window)
+        _check_rows(idx, cnt, ref_idx, ref_cnt)
+    api.check_device_status()
+
+
 @pytest.mark.parametrize("Tq,wlo,whi", [(1, -300, 301), (2, 0, 40), (1, 0, 5)])
 def test_decode_shaped_calls_fold_and_signed_weights(cuda_ok, Tq, wlo, whi):
     # 8 indexer heads of width 64 with one or two queries per sequence (the
