@@ -18,6 +18,7 @@
 #include "../../include/sa.h"
 #include "attn_gather.cuh"
 #include "attn_tc.cuh"
+#include "attn_cmp_tc.cuh"
 #include "attn_tile.cuh"
 #include "indexer.cuh"
 #include "nsa_misc.cuh"
@@ -719,6 +720,54 @@ static int launch_tile_t(const TileParams &p, cudaStream_t st) {
     return SA_OK;
 }
 
+// NSA compressed branch on tcgen05 (head dim 128, <= 16 heads per group).
+static int bf16_tensor_map_3d(CUtensorMap *m, const void *base, int d, int hkv, long long rows) {
+    TensorMapEncodeFn enc = tensor_map_encoder();
+    if (!enc) return fail(SA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+    cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)hkv, (cuuint64_t)rows};
+    cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)hkv * d * 2};
+    cuuint32_t box[3] = {64u, 1u, (cuuint32_t)CT_KT};
+    cuuint32_t es[3] = {1u, 1u, 1u};
+    const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(SA_ERR_CUDA, "cuTensorMapEncodeTiled(3d) failed (%d)", (int)r);
+    return SA_OK;
+}
+
+static int launch_cmp_tc(const TileParams &p, unsigned *err, cudaStream_t st) {
+    const long long ctas = (long long)p.B * p.Hkv * ((p.T + CT_Q - 1) / CT_Q);
+    if (ctas == 0) return SA_OK;
+    if (ctas > INT_MAX) return fail(SA_ERR_UNSUPPORTED, "cmp_tc: %lld CTAs", ctas);
+    CUtensorMap qm, khm, klm, vm;
+    int rc = bf16_tensor_map(&qm, p.q, (long long)p.B * p.T * p.Hq, 128, 16);
+    if (rc) return rc;
+    rc = bf16_tensor_map_3d(&khm, p.k, 128, p.Hkv, (long long)p.B * p.Lk);
+    if (rc) return rc;
+    rc = bf16_tensor_map_3d(&klm, p.klo, 128, p.Hkv, (long long)p.B * p.Lk);
+    if (rc) return rc;
+    rc = bf16_tensor_map_3d(&vm, p.v, 128, p.Hkv, (long long)p.B * p.Lk);
+    if (rc) return rc;
+    CmpTcParams cp{p, err};
+    constexpr int smem = CtSmem::ALLOC;
+    static_assert(smem <= 227 * 1024, "shared memory");
+    rc = set_smem(cmp_tc_kernel, smem);
+    if (rc) return rc;
+    cmp_tc_kernel<<<(unsigned)ctas, CT_THREADS, smem, st>>>(qm, khm, klm, vm, cp);
+    SA_CHECK_LAUNCH("cmp_tc_kernel");
+    return SA_OK;
+}
+
+static bool cmp_tc_applies(const TileParams &p, int d) {
+    static int v = -1;
+    if (v < 0) {
+        const char *e = std::getenv("SA_NSA_CMP_PATH");
+        v = (e && std::strcmp(e, "mma") == 0) ? 0 : 1;
+    }
+    return v && d == 128 && p.G <= 16 && (long long)p.B * p.T * p.Hq + 16 < INT_MAX &&
+           (long long)p.B * p.Lk < INT_MAX;
+}
+
 static int launch_tile(const TileParams &p, int d, int src, cudaStream_t st) {
     if (d == 64) return src == TS_CMP ? launch_tile_t<64, TS_CMP>(p, st) : launch_tile_t<64, TS_WINDOW>(p, st);
     return src == TS_CMP ? launch_tile_t<128, TS_CMP>(p, st) : launch_tile_t<128, TS_WINDOW>(p, st);
@@ -782,7 +831,8 @@ int sa_nsa_fwd(const void *q, const void *k, const void *v, const float *gates, 
         p.k = kc; p.klo = klo; p.v = vc; p.Lk = std::max(lay.nc, 1);
         p.cmp_len = cmp_len; p.cmp_stride = cmp_stride;
         p.out_f32 = o3; p.lse = l3;
-        rc = launch_tile(p, d, TS_CMP, st);   // nc == 0: zero rows, lse = -inf
+        // nc == 0: zero rows, lse = -inf
+        rc = cmp_tc_applies(p, d) ? launch_cmp_tc(p, ew, st) : launch_tile(p, d, TS_CMP, st);
         if (rc) return rc;
     }
     // 3. importance + block top-k

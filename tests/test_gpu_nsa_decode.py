@@ -46,6 +46,17 @@ def test_nsa_small_full_parity(cuda_ok, T):
     _nsa_check(g, out, lse3, sel, np.arange(T), NSA_CFG)
 
 
+@pytest.mark.parametrize("T,Hq,Hkv", [(40, 16, 1), (333, 32, 2), (1100, 16, 2), (2000, 48, 4)])
+def test_nsa_d128_full_parity(cuda_ok, T, Hq, Hkv):
+    # head dim 128 (the tensor-core compressed branch): groups of 16 and 8
+    # heads, ragged query blocks, short sequences with no visible block
+    g = inputs.gen_nsa(1, T, Hq, Hkv, 128, seed=T + Hq)
+    gd = to_dev(g)
+    out, lse3, sel = api.nsa_fwd(gd["q"], gd["k"], gd["v"], gd["gates"], **NSA_CFG)
+    api.check_device_status()
+    _nsa_check(g, out, lse3, sel, np.arange(T), NSA_CFG)
+
+
 def test_nsa_branches_isolated_by_gates(cuda_ok):
     T = 700
     g = inputs.gen_nsa(1, T, 16, 1, 128, seed=3)
