@@ -30,9 +30,9 @@
 
 namespace sa {
 
-constexpr int CT_Q = 8;            // queries per CTA (x 16 heads = 128 rows)
+constexpr int CT_Q = 8;            // queries per item (x 16 heads = 128 rows)
 constexpr int CT_KT = 64;          // compressed keys per tile
-constexpr int CT_STAGES = 2;
+constexpr int CT_STAGES = 3;
 constexpr int CT_THREADS = 192;
 
 struct CtSmem {                    // head dim 128
@@ -44,8 +44,9 @@ struct CtSmem {                    // head dim 128
     static constexpr int OFF_KV = OFF_Q + Q_BYTES;
     static constexpr int OFF_P = OFF_KV + CT_STAGES * STAGE;
     static constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
-    // q_full, kv_full[S], kv_empty[S], s_full[2], s_free[2], p_full[2], pv_done[2], o_full, drain
-    static constexpr int N_BAR = 1 + 2 * CT_STAGES + 8 + 2;
+    // q_full, q_empty, kv_full[S], kv_empty[S], s_full[2], s_free[2], p_full[2],
+    // pv_done[2], o_full, o_free, drain
+    static constexpr int N_BAR = 2 + 2 * CT_STAGES + 8 + 3;
     static constexpr int OFF_MISC = OFF_BAR + N_BAR * 8;
     static constexpr int TOTAL = OFF_MISC + 16;
     static constexpr int ALLOC = TOTAL + 1024;
@@ -64,7 +65,19 @@ __device__ __forceinline__ void load_3d(void *dst, const CUtensorMap *map, int x
 struct CmpTcParams {
     TileParams t;          // q, shapes, cmp_len/stride (Lk = compressed tokens per sequence), outputs
     unsigned *err;
+    int n_items;           // B * Hkv * ceil(T / CT_Q)
 };
+
+// Item -> (b, g, query block); items with the latest (heaviest) query blocks
+// come first so the persistent CTAs finish together.
+__device__ __forceinline__ void ct_item(const TileParams &p, int it, int &b, int &g, int &t0) {
+    const int nqb = (p.T + CT_Q - 1) / CT_Q;
+    const int bg = it % (p.B * p.Hkv);
+    const int qb = nqb - 1 - it / (p.B * p.Hkv);
+    b = bg / p.Hkv;
+    g = bg % p.Hkv;
+    t0 = qb * CT_Q;
+}
 
 __global__ void __launch_bounds__(CT_THREADS, 1)
     cmp_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap khimap,
@@ -76,22 +89,11 @@ __global__ void __launch_bounds__(CT_THREADS, 1)
     extern __shared__ unsigned char smem_raw[];
     unsigned char *smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::OFF_BAR);
-    uint64_t *q_full = bars, *kv_full = bars + 1, *kv_empty = kv_full + CT_STAGES;
+    uint64_t *q_full = bars, *q_empty = bars + 1, *kv_full = bars + 2, *kv_empty = kv_full + CT_STAGES;
     uint64_t *s_full = kv_empty + CT_STAGES, *s_free = s_full + 2, *p_full = s_free + 2, *pv_done = p_full + 2;
-    uint64_t *o_full = pv_done + 2, *drain = o_full + 1;
+    uint64_t *o_full = pv_done + 2, *o_free = o_full + 1, *drain = o_free + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::OFF_MISC + 4);
-
-    // CTA -> (b, g, query block)
-    const int nqb = (p.T + CT_Q - 1) / CT_Q;
-    int rem = blockIdx.x;
-    const int qb = rem % nqb; rem /= nqb;
-    const int g = rem % p.Hkv;
-    const int b = rem / p.Hkv;
-    const int t0 = qb * CT_Q;
-    const int t_last = min(t0 + CT_Q - 1, p.T - 1);
-    const int n_keys = (int)tile_key_end<TS_CMP>(p, t_last);
-    const int n_tiles = (n_keys + CT_KT - 1) / CT_KT;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     if (warp == 1) {
@@ -99,13 +101,13 @@ __global__ void __launch_bounds__(CT_THREADS, 1)
         tc::tmem_relinquish();
     }
     if (tid == 0) {
-        tc::mbar_init(q_full, 1);
+        tc::mbar_init(q_full, 1); tc::mbar_init(q_empty, 1);
         for (int i = 0; i < CT_STAGES; ++i) { tc::mbar_init(kv_full + i, 1); tc::mbar_init(kv_empty + i, 1); }
         for (int i = 0; i < 2; ++i) {
             tc::mbar_init(s_full + i, 1); tc::mbar_init(s_free + i, 128);
             tc::mbar_init(p_full + i, 128); tc::mbar_init(pv_done + i, 1);
         }
-        tc::mbar_init(o_full, 1);
+        tc::mbar_init(o_full, 1); tc::mbar_init(o_free, 128);
         tc::mbar_init(drain, 1);
         *abort_flag = 0;
         tc::mbar_fence_init();
@@ -118,49 +120,63 @@ __global__ void __launch_bounds__(CT_THREADS, 1)
         raise_error(cp.err, ERR_TIMEOUT);
         *abort_flag = 1;
     };
+    auto tiles_of = [&](int t0) -> int {
+        const int t_last = min(t0 + CT_Q - 1, p.T - 1);
+        return ((int)tile_key_end<TS_CMP>(p, t_last) + CT_KT - 1) / CT_KT;
+    };
 
     if (warp == 0) {
         // ------------------------------------------------------ TMA producer
-        if (lane == 0 && n_tiles > 0) {
-            atc::expect_tx(q_full, L::Q_BYTES);
-            for (int w = 0; w < CT_Q; ++w) {
-                const int qrow = (b * p.T + min(t0 + w, p.T - 1)) * p.Hq + g * p.G;
-                for (int h = 0; h < 2; ++h)
-                    atc::load_2d(smem + L::OFF_Q + h * (128 * 128) + w * (16 * 128), &qmap, h * 64, qrow, q_full);
-            }
+        if (lane == 0) {
             bool ok = true;
-            for (int kt = 0; kt < n_tiles && ok; ++kt) {
-                const int st = kt % CT_STAGES;
-                if (!atc::wait(kv_empty + st, ((kt / CT_STAGES) & 1) ^ 1, abort_flag)) { ok = false; break; }
-                atc::expect_tx(kv_full + st, L::STAGE);
-                unsigned char *dst = smem + L::OFF_KV + st * L::STAGE;
-                const int z = b * p.Lk + kt * CT_KT;
-                for (int h = 0; h < 2; ++h) {
-                    atc::load_3d(dst + h * (CT_KT * 128), &khimap, h * 64, g, z, kv_full + st);
-                    atc::load_3d(dst + L::KT_BYTES + h * (CT_KT * 128), &klomap, h * 64, g, z, kv_full + st);
-                    atc::load_3d(dst + 2 * L::KT_BYTES + h * (CT_KT * 128), &vmap, h * 64, g, z, kv_full + st);
+            int tile = 0, qn = 0;
+            for (int it = blockIdx.x; it < cp.n_items && ok; it += gridDim.x) {
+                int b, g, t0;
+                ct_item(p, it, b, g, t0);
+                const int nt = tiles_of(t0);
+                if (nt == 0) continue;                     // the epilogue writes zeros without Q or keys
+                if (!atc::wait(q_empty, (qn & 1) ^ 1, abort_flag)) { ok = false; break; }
+                atc::expect_tx(q_full, L::Q_BYTES);
+                for (int w = 0; w < CT_Q; ++w) {
+                    const int qrow = (b * p.T + min(t0 + w, p.T - 1)) * p.Hq + g * p.G;
+                    for (int h = 0; h < 2; ++h)
+                        atc::load_2d(smem + L::OFF_Q + h * (128 * 128) + w * (16 * 128), &qmap, h * 64, qrow, q_full);
+                }
+                ++qn;
+                for (int kt = 0; kt < nt; ++kt, ++tile) {
+                    const int st = tile % CT_STAGES;
+                    if (!atc::wait(kv_empty + st, ((tile / CT_STAGES) & 1) ^ 1, abort_flag)) { ok = false; break; }
+                    atc::expect_tx(kv_full + st, L::STAGE);
+                    unsigned char *dst = smem + L::OFF_KV + st * L::STAGE;
+                    const int z = b * p.Lk + kt * CT_KT;
+                    for (int h = 0; h < 2; ++h) {
+                        atc::load_3d(dst + h * (CT_KT * 128), &khimap, h * 64, g, z, kv_full + st);
+                        atc::load_3d(dst + L::KT_BYTES + h * (CT_KT * 128), &klomap, h * 64, g, z, kv_full + st);
+                        atc::load_3d(dst + 2 * L::KT_BYTES + h * (CT_KT * 128), &vmap, h * 64, g, z, kv_full + st);
+                    }
                 }
             }
             if (!ok) fail();
             // let the copies land before the CTA exits
-            tc::mbar_wait_bounded(q_full, 0, ATC_WAIT);
-            for (int i = 0; i < CT_STAGES && i < n_tiles; ++i) {
-                const int kt = n_tiles - 1 - i;
+            if (qn > 0) tc::mbar_wait_bounded(q_full, (qn - 1) & 1, ATC_WAIT);
+            for (int i = 0; i < CT_STAGES && i < tile; ++i) {
+                const int kt = tile - 1 - i;
                 tc::mbar_wait_bounded(kv_full + kt % CT_STAGES, (kt / CT_STAGES) & 1, ATC_WAIT);
             }
         }
         __syncwarp();
     } else if (warp == 1) {
         // --------------------------------------------------------------- MMA
-        if (lane == 0 && n_tiles > 0) {
+        if (lane == 0) {
             constexpr uint32_t ID_S = tc::make_idesc(1, 1, 128, CT_KT);
             constexpr uint32_t ID_O = tc::make_idesc(1, 1, 128, D) | (1u << 16);   // B (V) MN-major
             const uint32_t qa = tc::smem_u32(smem + L::OFF_Q);
-            bool ok = atc::wait(q_full, 0, abort_flag);
-            auto issue_s = [&](int kt) -> bool {
-                const int st = kt % CT_STAGES, sb = kt & 1;
-                if (!atc::wait(kv_full + st, (kt / CT_STAGES) & 1, abort_flag)) return false;
-                if (!atc::wait(s_free + sb, ((kt >> 1) & 1) ^ 1, abort_flag)) return false;
+            bool ok = true;
+            int tile = 0, qn = 0, on = 0;   // tiles, Q loads, items with an O result
+            auto issue_s = [&](int tl) -> bool {
+                const int st = tl % CT_STAGES, sb = tl & 1;
+                if (!atc::wait(kv_full + st, (tl / CT_STAGES) & 1, abort_flag)) return false;
+                if (!atc::wait(s_free + sb, ((tl >> 1) & 1) ^ 1, abort_flag)) return false;
                 tc::fence_after_sync();
                 const uint32_t ka = tc::smem_u32(smem + L::OFF_KV + st * L::STAGE);
 #pragma unroll
@@ -175,24 +191,36 @@ __global__ void __launch_bounds__(CT_THREADS, 1)
                 tc::mma_commit(s_full + sb);
                 return true;
             };
-            if (ok) ok = issue_s(0);
-            for (int kt = 0; kt < n_tiles && ok; ++kt) {
-                const int st = kt % CT_STAGES, pb = kt & 1;
-                if (kt + 1 < n_tiles && !issue_s(kt + 1)) { ok = false; break; }
-                if (!atc::wait(p_full + pb, (kt >> 1) & 1, abort_flag)) { ok = false; break; }
-                tc::fence_after_sync();
-                const uint32_t va = tc::smem_u32(smem + L::OFF_KV + st * L::STAGE + 2 * L::KT_BYTES);
-                const uint32_t pa = tc::smem_u32(smem + L::OFF_P + pb * L::P_BYTES);
+            for (int it = blockIdx.x; it < cp.n_items && ok; it += gridDim.x) {
+                int b, g, t0;
+                ct_item(p, it, b, g, t0);
+                const int nt = tiles_of(t0);
+                if (nt == 0) continue;
+                if (!atc::wait(q_full, qn & 1, abort_flag)) { ok = false; break; }
+                ++qn;
+                if (!issue_s(tile)) { ok = false; break; }
+                // the previous item's epilogue must have read O before it is overwritten
+                if (on > 0 && !atc::wait(o_free, (on - 1) & 1, abort_flag)) { ok = false; break; }
+                for (int kt = 0; kt < nt; ++kt, ++tile) {
+                    const int st = tile % CT_STAGES, pb = tile & 1;
+                    if (kt + 1 < nt && !issue_s(tile + 1)) { ok = false; break; }
+                    if (kt + 1 == nt) tc::mma_commit(q_empty);   // Q is free once the last S is done
+                    if (!atc::wait(p_full + pb, (tile >> 1) & 1, abort_flag)) { ok = false; break; }
+                    tc::fence_after_sync();
+                    const uint32_t va = tc::smem_u32(smem + L::OFF_KV + st * L::STAGE + 2 * L::KT_BYTES);
+                    const uint32_t pa = tc::smem_u32(smem + L::OFF_P + pb * L::P_BYTES);
 #pragma unroll
-                for (int kk = 0; kk < CT_KT / 16; ++kk) {
-                    const uint64_t ad = atc::desc_sw128(pa + kk * 32, 16, 1024);
-                    // V: MN-major, 64-column atoms 8 KB apart, 8-key groups 1 KB apart
-                    const uint64_t bd = atc::desc_sw128(va + kk * 2048, CT_KT * 128, 1024);
-                    tc::mma_bf16(tmem + 128, ad, bd, ID_O, (kt > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < CT_KT / 16; ++kk) {
+                        const uint64_t ad = atc::desc_sw128(pa + kk * 32, 16, 1024);
+                        // V: MN-major, 64-column atoms 8 KB apart, 8-key groups 1 KB apart
+                        const uint64_t bd = atc::desc_sw128(va + kk * 2048, CT_KT * 128, 1024);
+                        tc::mma_bf16(tmem + 128, ad, bd, ID_O, (kt > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    tc::mma_commit(kv_empty + st);
+                    tc::mma_commit(pv_done + pb);
+                    if (kt + 1 == nt) tc::mma_commit(o_full);
                 }
-                tc::mma_commit(kv_empty + st);
-                tc::mma_commit(pv_done + pb);
-                if (kt + 1 == n_tiles) tc::mma_commit(o_full);
+                ++on;
             }
             if (!ok) fail();
             tc::mma_commit(drain);
@@ -204,118 +232,135 @@ __global__ void __launch_bounds__(CT_THREADS, 1)
         const int quad = warp & 3;
         const int r = quad * 32 + lane;                   // row = query w x 16 + head h
         const int w = r >> 4, h = r & 15;
-        const int t = t0 + w;
-        const bool row_ok = t <= t_last && h < p.G;
-        const int nv = t <= t_last ? (int)tile_key_end<TS_CMP>(p, t) : 0;
         const uint32_t lrow = (uint32_t)(quad * 32) << 16;
-        float m = -INFINITY, l = 0.f;
         bool ok = true;
-        for (int kt = 0; kt < n_tiles; ++kt) {
-            const int sb = kt & 1, pb = kt & 1;
-            if (!__all_sync(0xffffffffu, atc::wait(s_full + sb, (kt >> 1) & 1, abort_flag))) { ok = false; break; }
-            tc::fence_after_sync();
-            uint32_t sr[CT_KT];
-            {
-                uint32_t (&s0)[16] = *reinterpret_cast<uint32_t(*)[16]>(sr);
-                uint32_t (&s1)[16] = *reinterpret_cast<uint32_t(*)[16]>(sr + 16);
-                uint32_t (&s2)[16] = *reinterpret_cast<uint32_t(*)[16]>(sr + 32);
-                uint32_t (&s3)[16] = *reinterpret_cast<uint32_t(*)[16]>(sr + 48);
-                tc::tmem_ld16(tmem + lrow + sb * CT_KT, s0);
-                tc::tmem_ld16(tmem + lrow + sb * CT_KT + 16, s1);
-                tc::tmem_ld16(tmem + lrow + sb * CT_KT + 32, s2);
-                tc::tmem_ld16(tmem + lrow + sb * CT_KT + 48, s3);
-            }
-            tc::tmem_ld_wait();
-            tc::fence_before_sync();
-            atc::arrive(s_free + sb);
-            const int i0 = kt * CT_KT;
-            float x[CT_KT];
-            float mt = -INFINITY;
-#pragma unroll
-            for (int k = 0; k < CT_KT; ++k) {
-                x[k] = (i0 + k < nv) ? __uint_as_float(sr[k]) * p.scale_log2 : -INFINITY;
-                mt = fmaxf(mt, x[k]);
-            }
-            // raise the running max only when the tile exceeds it by more than 2^8
-            const bool raise = mt > m + 8.f;
-            float alpha = 1.f;
-            if (raise) {
-                alpha = m == -INFINITY ? 0.f : exp2f(m - mt);
-                m = mt;
-                l *= alpha;
-            }
-            if (kt > 0 && __any_sync(0xffffffffu, raise)) {
-                // rescale the O rows of this warp once the previous P.V is done
-                const int pt = kt - 1;
-                if (__all_sync(0xffffffffu, atc::wait(pv_done + (pt & 1), (pt >> 1) & 1, abort_flag))) {
-                    tc::fence_after_sync();
-#pragma unroll
-                    for (int c = 0; c < D; c += 16) {
-                        uint32_t o16[16];
-                        tc::tmem_ld16(tmem + lrow + 128 + c, o16);
-                        tc::tmem_ld_wait();
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) o16[e] = __float_as_uint(__uint_as_float(o16[e]) * alpha);
-                        atc::tmem_st16(tmem + lrow + 128 + c, o16);
-                    }
-                    atc::tmem_st_wait();
-                } else {
+        int tile = 0, on = 0;
+        for (int it = blockIdx.x; it < cp.n_items && ok; it += gridDim.x) {
+            int b, g, t0;
+            ct_item(p, it, b, g, t0);
+            const int nt = tiles_of(t0);
+            const int t_last = min(t0 + CT_Q - 1, p.T - 1);
+            const int t = t0 + w;
+            const bool row_ok = t <= t_last && h < p.G;
+            const int nv = t <= t_last ? (int)tile_key_end<TS_CMP>(p, t) : 0;
+            float m = -INFINITY, l = 0.f;
+            for (int kt = 0; kt < nt; ++kt, ++tile) {
+                const int sb = tile & 1, pb = tile & 1;
+                if (!__all_sync(0xffffffffu, atc::wait(s_full + sb, (tile >> 1) & 1, abort_flag))) {
                     ok = false;
                     break;
                 }
-            }
-            const float mu = m == -INFINITY ? 0.f : m;
-            uint32_t pk[CT_KT / 2];
-            float rs = 0.f;
-#pragma unroll
-            for (int k = 0; k < CT_KT; k += 2) {
-                const float p0 = exp2f(x[k] - mu), p1 = exp2f(x[k + 1] - mu);
-                rs += p0 + p1;
-                pk[k / 2] = pack_bf16(p0, p1);
-            }
-            l += rs;
-            // P buffer pb was last read by the P.V of tile kt - 2
-            if (kt >= 2 && !__all_sync(0xffffffffu, atc::wait(pv_done + pb, ((kt >> 1) & 1) ^ 1, abort_flag))) {
-                ok = false;
-                break;
-            }
-            unsigned char *prow = smem + L::OFF_P + pb * L::P_BYTES + r * 128;
-#pragma unroll
-            for (int c = 0; c < CT_KT / 8; ++c)
-                *reinterpret_cast<uint4 *>(prow + ((c ^ (r & 7)) << 4)) =
-                    make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-            tc::fence_proxy_async_smem();
-            tc::fence_before_sync();
-            atc::arrive(p_full + pb);
-        }
-        // ---------------------------------------------------------- epilogue
-        const long long orow = (long long)(b * p.T + t) * p.Hq + g * p.G + h;
-        bool have_o = false;
-        if (ok && n_tiles > 0) {
-            have_o = __all_sync(0xffffffffu, atc::wait(o_full, 0, abort_flag));
-            if (have_o) tc::fence_after_sync();
-            else ok = false;
-        }
-        const float inv = l > 0.f ? 1.f / l : 0.f;
-#pragma unroll
-        for (int c = 0; c < D; c += 16) {
-            uint32_t o16[16];
-            if (have_o) {
-                tc::tmem_ld16(tmem + lrow + 128 + c, o16);
+                tc::fence_after_sync();
+                uint32_t sr[CT_KT];
+                {
+                    uint32_t (&s0)[16] = *reinterpret_cast<uint32_t(*)[16]>(sr);
+                    uint32_t (&s1)[16] = *reinterpret_cast<uint32_t(*)[16]>(sr + 16);
+                    uint32_t (&s2)[16] = *reinterpret_cast<uint32_t(*)[16]>(sr + 32);
+                    uint32_t (&s3)[16] = *reinterpret_cast<uint32_t(*)[16]>(sr + 48);
+                    tc::tmem_ld16(tmem + lrow + sb * CT_KT, s0);
+                    tc::tmem_ld16(tmem + lrow + sb * CT_KT + 16, s1);
+                    tc::tmem_ld16(tmem + lrow + sb * CT_KT + 32, s2);
+                    tc::tmem_ld16(tmem + lrow + sb * CT_KT + 48, s3);
+                }
                 tc::tmem_ld_wait();
-            } else {
+                tc::fence_before_sync();
+                atc::arrive(s_free + sb);
+                const int i0 = kt * CT_KT;
+                float x[CT_KT];
+                float mt = -INFINITY;
 #pragma unroll
-                for (int e = 0; e < 16; ++e) o16[e] = 0u;
-            }
-            if (row_ok) {
-                float4 *dst = reinterpret_cast<float4 *>(p.out_f32 + orow * D + c);
+                for (int k = 0; k < CT_KT; ++k) {
+                    x[k] = (i0 + k < nv) ? __uint_as_float(sr[k]) * p.scale_log2 : -INFINITY;
+                    mt = fmaxf(mt, x[k]);
+                }
+                // raise the running max only when the tile exceeds it by more than 2^8
+                const bool raise = mt > m + 8.f;
+                float alpha = 1.f;
+                if (raise) {
+                    alpha = m == -INFINITY ? 0.f : exp2f(m - mt);
+                    m = mt;
+                    l *= alpha;
+                }
+                if (kt > 0 && __any_sync(0xffffffffu, raise)) {
+                    // rescale the O rows of this warp once the previous P.V is done
+                    const int pt = tile - 1;
+                    if (__all_sync(0xffffffffu, atc::wait(pv_done + (pt & 1), (pt >> 1) & 1, abort_flag))) {
+                        tc::fence_after_sync();
 #pragma unroll
-                for (int e = 0; e < 16; e += 4)
-                    dst[e / 4] = make_float4(__uint_as_float(o16[e]) * inv, __uint_as_float(o16[e + 1]) * inv,
-                                             __uint_as_float(o16[e + 2]) * inv, __uint_as_float(o16[e + 3]) * inv);
+                        for (int c = 0; c < D; c += 16) {
+                            uint32_t o16[16];
+                            tc::tmem_ld16(tmem + lrow + 128 + c, o16);
+                            tc::tmem_ld_wait();
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) o16[e] = __float_as_uint(__uint_as_float(o16[e]) * alpha);
+                            atc::tmem_st16(tmem + lrow + 128 + c, o16);
+                        }
+                        atc::tmem_st_wait();
+                    } else {
+                        ok = false;
+                        break;
+                    }
+                }
+                const float mu = m == -INFINITY ? 0.f : m;
+                uint32_t pk[CT_KT / 2];
+                float rs = 0.f;
+#pragma unroll
+                for (int k = 0; k < CT_KT; k += 2) {
+                    const float p0 = exp2f(x[k] - mu), p1 = exp2f(x[k + 1] - mu);
+                    rs += p0 + p1;
+                    pk[k / 2] = pack_bf16(p0, p1);
+                }
+                l += rs;
+                // P buffer pb was last read by the P.V of tile - 2
+                if (tile >= 2 &&
+                    !__all_sync(0xffffffffu, atc::wait(pv_done + pb, ((tile >> 1) & 1) ^ 1, abort_flag))) {
+                    ok = false;
+                    break;
+                }
+                unsigned char *prow = smem + L::OFF_P + pb * L::P_BYTES + r * 128;
+#pragma unroll
+                for (int c = 0; c < CT_KT / 8; ++c)
+                    *reinterpret_cast<uint4 *>(prow + ((c ^ (r & 7)) << 4)) =
+                        make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+                tc::fence_proxy_async_smem();
+                tc::fence_before_sync();
+                atc::arrive(p_full + pb);
             }
+            if (!ok) break;
+            // ------------------------------------------------------ epilogue
+            const long long orow = (long long)(b * p.T + t) * p.Hq + g * p.G + h;
+            bool have_o = false;
+            if (nt > 0) {
+                have_o = __all_sync(0xffffffffu, atc::wait(o_full, on & 1, abort_flag));
+                if (!have_o) { ok = false; break; }
+                tc::fence_after_sync();
+            }
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+            for (int c = 0; c < D; c += 16) {
+                uint32_t o16[16];
+                if (have_o) {
+                    tc::tmem_ld16(tmem + lrow + 128 + c, o16);
+                    tc::tmem_ld_wait();
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) o16[e] = 0u;
+                }
+                if (row_ok) {
+                    float4 *dst = reinterpret_cast<float4 *>(p.out_f32 + orow * D + c);
+#pragma unroll
+                    for (int e = 0; e < 16; e += 4)
+                        dst[e / 4] = make_float4(__uint_as_float(o16[e]) * inv, __uint_as_float(o16[e + 1]) * inv,
+                                                 __uint_as_float(o16[e + 2]) * inv, __uint_as_float(o16[e + 3]) * inv);
+                }
+            }
+            if (have_o) {
+                tc::fence_before_sync();
+                atc::arrive(o_free);
+                ++on;
+            }
+            if (row_ok && p.lse) p.lse[orow] = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
         }
-        if (row_ok && p.lse) p.lse[orow] = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
         if (!ok) fail();
     }
     tc::fence_before_sync();

@@ -748,12 +748,13 @@ static int launch_cmp_tc(const TileParams &p, unsigned *err, cudaStream_t st) {
     if (rc) return rc;
     rc = bf16_tensor_map_3d(&vm, p.v, 128, p.Hkv, (long long)p.B * p.Lk);
     if (rc) return rc;
-    CmpTcParams cp{p, err};
+    CmpTcParams cp{p, err, (int)ctas};
     constexpr int smem = CtSmem::ALLOC;
     static_assert(smem <= 227 * 1024, "shared memory");
     rc = set_smem(cmp_tc_kernel, smem);
     if (rc) return rc;
-    cmp_tc_kernel<<<(unsigned)ctas, CT_THREADS, smem, st>>>(qm, khm, klm, vm, cp);
+    const int grid = (int)std::min<long long>(ctas, sm_count());   // persistent: one CTA per SM
+    cmp_tc_kernel<<<grid, CT_THREADS, smem, st>>>(qm, khm, klm, vm, cp);
     SA_CHECK_LAUNCH("cmp_tc_kernel");
     return SA_OK;
 }
