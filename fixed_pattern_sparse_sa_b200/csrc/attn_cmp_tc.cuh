@@ -1,4 +1,5 @@
-// attn_cmp_tc.cuh -- NSA compressed-branch attention on the tcgen05 tensor cores.
+// attn_cmp_tc.cuh -- NSA compressed and sliding-window branches on the tcgen05
+// tensor cores.
 //
 // NSA page ("Native Sparse Attention ...", "Puntos Clave": coarse-grained
 // token compression): every query attends to the compressed keys/values of
@@ -9,7 +10,10 @@
 //   O[128 x d]  += P[128 x 64] . Vc
 // with fp32 accumulators in TMEM (tcgen05.mma kind::f16).  The compressed
 // keys are means and do not fit bf16 exactly, so they are held as a bf16
-// hi/lo pair and S accumulates both halves (Q.K_hi + Q.K_lo).
+// hi/lo pair and S accumulates both halves (Q.K_hi + Q.K_lo).  The same
+// kernel (SRC = TS_WINDOW) runs the sliding-window branch (NSA page, "Puntos
+// Clave": local context) over the raw keys t - window < j <= t, whose union
+// over 8 consecutive queries is again one contiguous key range.
 //
 // Q, K_hi, K_lo and V tiles arrive by TMA box loads in the 128B-swizzled
 // canonical layouts (K-major for Q, K and P; MN-major for V as the B operand
@@ -62,6 +66,14 @@ __device__ __forceinline__ void load_3d(void *dst, const CUtensorMap *map, int x
 }
 }  // namespace atc
 
+// 2^x on the special-function unit (flushes results below the normal range
+// to zero, which a softmax weight can ignore).
+__device__ __forceinline__ float ex2_fast(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 struct CmpTcParams {
     TileParams t;          // q, shapes, cmp_len/stride (Lk = compressed tokens per sequence), outputs
     unsigned *err;
@@ -79,11 +91,13 @@ __device__ __forceinline__ void ct_item(const TileParams &p, int it, int &b, int
     t0 = qb * CT_Q;
 }
 
+template <int SRC>
 __global__ void __launch_bounds__(CT_THREADS, 1)
-    cmp_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap khimap,
+    nsa_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap khimap,
                   const __grid_constant__ CUtensorMap klomap, const __grid_constant__ CUtensorMap vmap,
                   const CmpTcParams cp) {
     constexpr int D = 128;
+    constexpr bool LO = SRC == TS_CMP;             // compressed keys carry a lo half
     using L = CtSmem;
     const TileParams &p = cp.t;
     extern __shared__ unsigned char smem_raw[];
@@ -120,9 +134,11 @@ __global__ void __launch_bounds__(CT_THREADS, 1)
         raise_error(cp.err, ERR_TIMEOUT);
         *abort_flag = 1;
     };
+    // first key of an item's range (window: the first query's window start)
+    auto key_lo = [&](int t0) -> int { return SRC == TS_CMP ? 0 : max(0, t0 - p.window + 1); };
     auto tiles_of = [&](int t0) -> int {
         const int t_last = min(t0 + CT_Q - 1, p.T - 1);
-        return ((int)tile_key_end<TS_CMP>(p, t_last) + CT_KT - 1) / CT_KT;
+        return ((int)tile_key_end<SRC>(p, t_last) - key_lo(t0) + CT_KT - 1) / CT_KT;
     };
 
     if (warp == 0) {
@@ -146,12 +162,12 @@ __global__ void __launch_bounds__(CT_THREADS, 1)
                 for (int kt = 0; kt < nt; ++kt, ++tile) {
                     const int st = tile % CT_STAGES;
                     if (!atc::wait(kv_empty + st, ((tile / CT_STAGES) & 1) ^ 1, abort_flag)) { ok = false; break; }
-                    atc::expect_tx(kv_full + st, L::STAGE);
+                    atc::expect_tx(kv_full + st, LO ? L::STAGE : 2 * L::KT_BYTES);
                     unsigned char *dst = smem + L::OFF_KV + st * L::STAGE;
-                    const int z = b * p.Lk + kt * CT_KT;
+                    const int z = b * p.Lk + key_lo(t0) + kt * CT_KT;
                     for (int h = 0; h < 2; ++h) {
                         atc::load_3d(dst + h * (CT_KT * 128), &khimap, h * 64, g, z, kv_full + st);
-                        atc::load_3d(dst + L::KT_BYTES + h * (CT_KT * 128), &klomap, h * 64, g, z, kv_full + st);
+                        if (LO) atc::load_3d(dst + L::KT_BYTES + h * (CT_KT * 128), &klomap, h * 64, g, z, kv_full + st);
                         atc::load_3d(dst + 2 * L::KT_BYTES + h * (CT_KT * 128), &vmap, h * 64, g, z, kv_full + st);
                     }
                 }
@@ -186,7 +202,7 @@ __global__ void __launch_bounds__(CT_THREADS, 1)
                     const uint64_t bh = atc::desc_sw128(ka + h * (CT_KT * 128) + kk * 32, 16, 1024);
                     const uint64_t bl = atc::desc_sw128(ka + L::KT_BYTES + h * (CT_KT * 128) + kk * 32, 16, 1024);
                     tc::mma_bf16(tmem + sb * CT_KT, ad, bh, ID_S, ks > 0 ? 1u : 0u);
-                    tc::mma_bf16(tmem + sb * CT_KT, ad, bl, ID_S, 1u);
+                    if (LO) tc::mma_bf16(tmem + sb * CT_KT, ad, bl, ID_S, 1u);
                 }
                 tc::mma_commit(s_full + sb);
                 return true;
@@ -242,7 +258,10 @@ __global__ void __launch_bounds__(CT_THREADS, 1)
             const int t_last = min(t0 + CT_Q - 1, p.T - 1);
             const int t = t0 + w;
             const bool row_ok = t <= t_last && h < p.G;
-            const int nv = t <= t_last ? (int)tile_key_end<TS_CMP>(p, t) : 0;
+            // visible keys of this row as item-relative indices [vlo, vhi)
+            const int klo = key_lo(t0);
+            const int vhi = t <= t_last ? (int)tile_key_end<SRC>(p, t) - klo : 0;
+            const int vlo = (t <= t_last && SRC == TS_WINDOW) ? max(0, t - p.window + 1) - klo : 0;
             float m = -INFINITY, l = 0.f;
             for (int kt = 0; kt < nt; ++kt, ++tile) {
                 const int sb = tile & 1, pb = tile & 1;
@@ -266,18 +285,26 @@ __global__ void __launch_bounds__(CT_THREADS, 1)
                 tc::fence_before_sync();
                 atc::arrive(s_free + sb);
                 const int i0 = kt * CT_KT;
-                float x[CT_KT];
+                // row max of the raw scores (masked past the row's visible keys)
+                const bool full = i0 >= vlo && i0 + CT_KT <= vhi;
                 float mt = -INFINITY;
+                if (full) {
 #pragma unroll
-                for (int k = 0; k < CT_KT; ++k) {
-                    x[k] = (i0 + k < nv) ? __uint_as_float(sr[k]) * p.scale_log2 : -INFINITY;
-                    mt = fmaxf(mt, x[k]);
+                    for (int k = 0; k < CT_KT; k += 2)
+                        mt = fmaxf(mt, fmaxf(__uint_as_float(sr[k]), __uint_as_float(sr[k + 1])));
+                } else {
+#pragma unroll
+                    for (int k = 0; k < CT_KT; ++k) {
+                        if (i0 + k < vlo || i0 + k >= vhi) sr[k] = __float_as_uint(-INFINITY);
+                        mt = fmaxf(mt, __uint_as_float(sr[k]));
+                    }
                 }
-                // raise the running max only when the tile exceeds it by more than 2^8
-                const bool raise = mt > m + 8.f;
+                // m is kept in raw-score units; raise it only when the tile
+                // exceeds it by more than 2^8 after scaling
+                const bool raise = mt != -INFINITY && (m == -INFINITY || (mt - m) * p.scale_log2 > 8.f);
                 float alpha = 1.f;
                 if (raise) {
-                    alpha = m == -INFINITY ? 0.f : exp2f(m - mt);
+                    alpha = m == -INFINITY ? 0.f : ex2_fast((m - mt) * p.scale_log2);
                     m = mt;
                     l *= alpha;
                 }
@@ -301,16 +328,19 @@ __global__ void __launch_bounds__(CT_THREADS, 1)
                         break;
                     }
                 }
-                const float mu = m == -INFINITY ? 0.f : m;
+                // p = 2^((s - m) * scale_log2): one FFMA and one ex2 per score
+                const float nb = m == -INFINITY ? 0.f : -m * p.scale_log2;
                 uint32_t pk[CT_KT / 2];
-                float rs = 0.f;
+                float rs0 = 0.f, rs1 = 0.f;
 #pragma unroll
                 for (int k = 0; k < CT_KT; k += 2) {
-                    const float p0 = exp2f(x[k] - mu), p1 = exp2f(x[k + 1] - mu);
-                    rs += p0 + p1;
+                    const float p0 = ex2_fast(fmaf(__uint_as_float(sr[k]), p.scale_log2, nb));
+                    const float p1 = ex2_fast(fmaf(__uint_as_float(sr[k + 1]), p.scale_log2, nb));
+                    rs0 += p0;
+                    rs1 += p1;
                     pk[k / 2] = pack_bf16(p0, p1);
                 }
-                l += rs;
+                l += rs0 + rs1;
                 // P buffer pb was last read by the P.V of tile - 2
                 if (tile >= 2 &&
                     !__all_sync(0xffffffffu, atc::wait(pv_done + pb, ((tile >> 1) & 1) ^ 1, abort_flag))) {
@@ -359,7 +389,7 @@ __global__ void __launch_bounds__(CT_THREADS, 1)
                 atc::arrive(o_free);
                 ++on;
             }
-            if (row_ok && p.lse) p.lse[orow] = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
+            if (row_ok && p.lse) p.lse[orow] = l > 0.f ? (m * p.scale_log2 + log2f(l)) * kLn2 : -INFINITY;
         }
         if (!ok) fail();
     }

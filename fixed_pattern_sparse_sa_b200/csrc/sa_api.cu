@@ -735,27 +735,29 @@ static int bf16_tensor_map_3d(CUtensorMap *m, const void *base, int d, int hkv, 
     return SA_OK;
 }
 
-static int launch_cmp_tc(const TileParams &p, unsigned *err, cudaStream_t st) {
-    const long long ctas = (long long)p.B * p.Hkv * ((p.T + CT_Q - 1) / CT_Q);
-    if (ctas == 0) return SA_OK;
-    if (ctas > INT_MAX) return fail(SA_ERR_UNSUPPORTED, "cmp_tc: %lld CTAs", ctas);
+template <int SRC>
+static int launch_nsa_tc(const TileParams &p, unsigned *err, cudaStream_t st) {
+    const long long items = (long long)p.B * p.Hkv * ((p.T + CT_Q - 1) / CT_Q);
+    if (items == 0) return SA_OK;
+    if (items > INT_MAX) return fail(SA_ERR_UNSUPPORTED, "nsa_tc: %lld items", items);
     CUtensorMap qm, khm, klm, vm;
     int rc = bf16_tensor_map(&qm, p.q, (long long)p.B * p.T * p.Hq, 128, 16);
     if (rc) return rc;
     rc = bf16_tensor_map_3d(&khm, p.k, 128, p.Hkv, (long long)p.B * p.Lk);
     if (rc) return rc;
-    rc = bf16_tensor_map_3d(&klm, p.klo, 128, p.Hkv, (long long)p.B * p.Lk);
+    rc = bf16_tensor_map_3d(&klm, SRC == TS_CMP ? p.klo : p.k, 128, p.Hkv, (long long)p.B * p.Lk);
     if (rc) return rc;
     rc = bf16_tensor_map_3d(&vm, p.v, 128, p.Hkv, (long long)p.B * p.Lk);
     if (rc) return rc;
-    CmpTcParams cp{p, err, (int)ctas};
+    CmpTcParams cp{p, err, (int)items};
     constexpr int smem = CtSmem::ALLOC;
     static_assert(smem <= 227 * 1024, "shared memory");
-    rc = set_smem(cmp_tc_kernel, smem);
+    auto kern = nsa_tc_kernel<SRC>;
+    rc = set_smem(kern, smem);
     if (rc) return rc;
-    const int grid = (int)std::min<long long>(ctas, sm_count());   // persistent: one CTA per SM
-    cmp_tc_kernel<<<grid, CT_THREADS, smem, st>>>(qm, khm, klm, vm, cp);
-    SA_CHECK_LAUNCH("cmp_tc_kernel");
+    const int grid = (int)std::min<long long>(items, sm_count());   // persistent: one CTA per SM
+    kern<<<grid, CT_THREADS, smem, st>>>(qm, khm, klm, vm, cp);
+    SA_CHECK_LAUNCH("nsa_tc_kernel");
     return SA_OK;
 }
 
@@ -833,7 +835,7 @@ int sa_nsa_fwd(const void *q, const void *k, const void *v, const float *gates, 
         p.cmp_len = cmp_len; p.cmp_stride = cmp_stride;
         p.out_f32 = o3; p.lse = l3;
         // nc == 0: zero rows, lse = -inf
-        rc = cmp_tc_applies(p, d) ? launch_cmp_tc(p, ew, st) : launch_tile(p, d, TS_CMP, st);
+        rc = cmp_tc_applies(p, d) ? launch_nsa_tc<TS_CMP>(p, ew, st) : launch_tile(p, d, TS_CMP, st);
         if (rc) return rc;
     }
     // 3. importance + block top-k
@@ -865,7 +867,7 @@ int sa_nsa_fwd(const void *q, const void *k, const void *v, const float *gates, 
         p.k = static_cast<const __nv_bfloat16 *>(k); p.v = static_cast<const __nv_bfloat16 *>(v);
         p.Lk = T; p.window = window;
         p.out_f32 = o3 + 2 * rows * d; p.lse = l3 + 2 * rows;
-        rc = launch_tile(p, d, TS_WINDOW, st);
+        rc = cmp_tc_applies(p, d) ? launch_nsa_tc<TS_WINDOW>(p, ew, st) : launch_tile(p, d, TS_WINDOW, st);
         if (rc) return rc;
     }
     // 6. gated sum
