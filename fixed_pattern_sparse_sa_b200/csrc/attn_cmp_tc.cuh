@@ -399,3 +399,287 @@ __global__ void __launch_bounds__(CT_THREADS, 1)
 }
 
 }  // namespace sa
+
+namespace sa {
+
+// ---------------------------------------------------------------------------
+// NSA block importance and top-k selection on tcgen05 (NSA page, "Puntos
+// Clave": the compressed-branch attention scores rank the selection blocks).
+// Persistent CTAs walk the same 8-query items as nsa_tc_kernel over the
+// compressed keys: S = Q.K_hi^T + Q.K_lo^T in TMEM; thread r (one query head)
+// turns its row into probabilities with the compressed branch's LSE and sums
+// them per selection block (sel_block / cmp_stride consecutive compressed
+// tokens); the 16 heads of a query are summed by a transposing butterfly over
+// the 16 lanes that hold them, so lane h ends with block h of the tile.  The
+// importances of an item stay in shared memory; each query then takes its
+// top-k blocks by repeated arg-max (ties to the lower block), written in
+// ascending order.  Blocks past the last tile have no visible compressed
+// token and count as 0.
+constexpr int IT_STAGES = 4;
+constexpr int IT_MAX_BLOCKS = 2048;   // candidate blocks per query held in shared memory
+
+struct ItSmem {                       // head dim 128
+    static constexpr int Q_BYTES = 128 * 256;
+    static constexpr int KT_BYTES = CT_KT * 256;
+    static constexpr int STAGE = 2 * KT_BYTES;                 // K_hi | K_lo
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_KV = OFF_Q + Q_BYTES;
+    static constexpr int OFF_IMP = OFF_KV + IT_STAGES * STAGE; // [CT_Q][n_blocks] float
+    static constexpr int N_BAR = 2 + 2 * IT_STAGES + 4 + 1;    // q_full, q_empty, kv x2, s_full x2, s_free x2, drain
+    __host__ __device__ static int off_bar(int n_blocks) { return OFF_IMP + CT_Q * n_blocks * 4; }
+    __host__ __device__ static int alloc(int n_blocks) { return off_bar(n_blocks) + N_BAR * 8 + 16 + 1024; }
+};
+
+struct ImpTcParams {
+    TileParams t;          // q, shapes (Lk = compressed tokens), cmp_len / cmp_stride, scale
+    const float *lse_cmp;  // [B,T,Hq] natural log
+    int sel_block, sel_topk, n_blocks;
+    int32_t *sel_idx;      // [B,T,Hkv,sel_topk]
+    unsigned *err;
+    int n_items;
+};
+
+__global__ void __launch_bounds__(CT_THREADS, 1)
+    nsa_imp_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap khimap,
+                      const __grid_constant__ CUtensorMap klomap, const ImpTcParams ip) {
+    constexpr int D = 128;
+    using L = ItSmem;
+    const TileParams &p = ip.t;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
+    const int nbk = ip.n_blocks;
+    float *imp_s = reinterpret_cast<float *>(smem + L::OFF_IMP);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::off_bar(nbk));
+    uint64_t *q_full = bars, *q_empty = bars + 1, *kv_full = bars + 2, *kv_empty = kv_full + IT_STAGES;
+    uint64_t *s_full = kv_empty + IT_STAGES, *s_free = s_full + 2, *drain = s_free + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int cpb = ip.sel_block / p.cmp_stride;              // compressed tokens per block (divides CT_KT)
+    const int nbt = CT_KT / cpb;                              // blocks per tile (<= 16)
+
+    if (warp == 1) {
+        tc::tmem_alloc(tmem_slot, 128);   // S x2
+        tc::tmem_relinquish();
+    }
+    if (tid == 0) {
+        tc::mbar_init(q_full, 1); tc::mbar_init(q_empty, 1);
+        for (int i = 0; i < IT_STAGES; ++i) { tc::mbar_init(kv_full + i, 1); tc::mbar_init(kv_empty + i, 1); }
+        for (int i = 0; i < 2; ++i) { tc::mbar_init(s_full + i, 1); tc::mbar_init(s_free + i, 128); }
+        tc::mbar_init(drain, 1);
+        *abort_flag = 0;
+        tc::mbar_fence_init();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    auto fail = [&]() {
+        raise_error(ip.err, ERR_TIMEOUT);
+        *abort_flag = 1;
+    };
+    auto tiles_of = [&](int t0) -> int {
+        const int t_last = min(t0 + CT_Q - 1, p.T - 1);
+        return ((int)tile_key_end<TS_CMP>(p, t_last) + CT_KT - 1) / CT_KT;
+    };
+
+    if (warp == 0) {
+        if (lane == 0) {
+            bool ok = true;
+            int tile = 0, qn = 0;
+            for (int it = blockIdx.x; it < ip.n_items && ok; it += gridDim.x) {
+                int b, g, t0;
+                ct_item(p, it, b, g, t0);
+                const int nt = tiles_of(t0);
+                if (nt == 0) continue;
+                if (!atc::wait(q_empty, (qn & 1) ^ 1, abort_flag)) { ok = false; break; }
+                atc::expect_tx(q_full, L::Q_BYTES);
+                for (int w = 0; w < CT_Q; ++w) {
+                    const int qrow = (b * p.T + min(t0 + w, p.T - 1)) * p.Hq + g * p.G;
+                    for (int h = 0; h < 2; ++h)
+                        atc::load_2d(smem + L::OFF_Q + h * (128 * 128) + w * (16 * 128), &qmap, h * 64, qrow, q_full);
+                }
+                ++qn;
+                for (int kt = 0; kt < nt; ++kt, ++tile) {
+                    const int st = tile % IT_STAGES;
+                    if (!atc::wait(kv_empty + st, ((tile / IT_STAGES) & 1) ^ 1, abort_flag)) { ok = false; break; }
+                    atc::expect_tx(kv_full + st, L::STAGE);
+                    unsigned char *dst = smem + L::OFF_KV + st * L::STAGE;
+                    const int z = b * p.Lk + kt * CT_KT;
+                    for (int h = 0; h < 2; ++h) {
+                        atc::load_3d(dst + h * (CT_KT * 128), &khimap, h * 64, g, z, kv_full + st);
+                        atc::load_3d(dst + L::KT_BYTES + h * (CT_KT * 128), &klomap, h * 64, g, z, kv_full + st);
+                    }
+                }
+            }
+            if (!ok) fail();
+            if (qn > 0) tc::mbar_wait_bounded(q_full, (qn - 1) & 1, ATC_WAIT);
+            for (int i = 0; i < IT_STAGES && i < tile; ++i) {
+                const int kt = tile - 1 - i;
+                tc::mbar_wait_bounded(kv_full + kt % IT_STAGES, (kt / IT_STAGES) & 1, ATC_WAIT);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t ID_S = tc::make_idesc(1, 1, 128, CT_KT);
+            const uint32_t qa = tc::smem_u32(smem + L::OFF_Q);
+            bool ok = true;
+            int tile = 0, qn = 0;
+            for (int it = blockIdx.x; it < ip.n_items && ok; it += gridDim.x) {
+                int b, g, t0;
+                ct_item(p, it, b, g, t0);
+                const int nt = tiles_of(t0);
+                if (nt == 0) continue;
+                if (!atc::wait(q_full, qn & 1, abort_flag)) { ok = false; break; }
+                ++qn;
+                for (int kt = 0; kt < nt; ++kt, ++tile) {
+                    const int st = tile % IT_STAGES, sb = tile & 1;
+                    if (!atc::wait(kv_full + st, (tile / IT_STAGES) & 1, abort_flag)) { ok = false; break; }
+                    if (!atc::wait(s_free + sb, ((tile >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+                    tc::fence_after_sync();
+                    const uint32_t ka = tc::smem_u32(smem + L::OFF_KV + st * L::STAGE);
+#pragma unroll
+                    for (int ks = 0; ks < D / 16; ++ks) {
+                        const int h = ks / 4, kk = ks % 4;
+                        const uint64_t ad = atc::desc_sw128(qa + h * (128 * 128) + kk * 32, 16, 1024);
+                        const uint64_t bh = atc::desc_sw128(ka + h * (CT_KT * 128) + kk * 32, 16, 1024);
+                        const uint64_t bl = atc::desc_sw128(ka + L::KT_BYTES + h * (CT_KT * 128) + kk * 32, 16, 1024);
+                        tc::mma_bf16(tmem + sb * CT_KT, ad, bh, ID_S, ks > 0 ? 1u : 0u);
+                        tc::mma_bf16(tmem + sb * CT_KT, ad, bl, ID_S, 1u);
+                    }
+                    tc::mma_commit(kv_empty + st);
+                    tc::mma_commit(s_full + sb);
+                    if (kt + 1 == nt) tc::mma_commit(q_empty);
+                }
+            }
+            if (!ok) fail();
+            tc::mma_commit(drain);
+            tc::mbar_wait_bounded(drain, 0, ATC_WAIT);
+        }
+        __syncwarp();
+    } else {
+        const int quad = warp & 3;
+        const int r = quad * 32 + lane;                   // row = query w x 16 + head h
+        const int w = r >> 4, h = r & 15;
+        const uint32_t lrow = (uint32_t)(quad * 32) << 16;
+        bool ok = true;
+        int tile = 0;
+        for (int it = blockIdx.x; it < ip.n_items; it += gridDim.x) {
+            int b, g, t0;
+            ct_item(p, it, b, g, t0);
+            const int nt = tiles_of(t0);
+            const int t_last = min(t0 + CT_Q - 1, p.T - 1);
+            const int t = t0 + w;
+            const bool row_ok = t <= t_last && h < p.G;
+            const int nv = t <= t_last ? (int)tile_key_end<TS_CMP>(p, t) : 0;
+            const float ls = row_ok ? ip.lse_cmp[(long long)(b * p.T + t) * p.Hq + g * p.G + h] * kLog2e : 0.f;
+            for (int kt = 0; kt < nt && ok; ++kt, ++tile) {
+                const int sb = tile & 1;
+                if (!__all_sync(0xffffffffu, atc::wait(s_full + sb, (tile >> 1) & 1, abort_flag))) {
+                    ok = false;
+                    break;
+                }
+                tc::fence_after_sync();
+                uint32_t sr[CT_KT];
+                {
+                    uint32_t (&s0)[16] = *reinterpret_cast<uint32_t(*)[16]>(sr);
+                    uint32_t (&s1)[16] = *reinterpret_cast<uint32_t(*)[16]>(sr + 16);
+                    uint32_t (&s2)[16] = *reinterpret_cast<uint32_t(*)[16]>(sr + 32);
+                    uint32_t (&s3)[16] = *reinterpret_cast<uint32_t(*)[16]>(sr + 48);
+                    tc::tmem_ld16(tmem + lrow + sb * CT_KT, s0);
+                    tc::tmem_ld16(tmem + lrow + sb * CT_KT + 16, s1);
+                    tc::tmem_ld16(tmem + lrow + sb * CT_KT + 32, s2);
+                    tc::tmem_ld16(tmem + lrow + sb * CT_KT + 48, s3);
+                }
+                tc::tmem_ld_wait();
+                tc::fence_before_sync();
+                atc::arrive(s_free + sb);
+                // p = 2^(s * scale_log2 - lse_log2): one FFMA and one ex2 per score
+                const int i0 = kt * CT_KT;
+                const bool full = row_ok && i0 + CT_KT <= nv;
+                float pv[CT_KT];
+#pragma unroll
+                for (int k = 0; k < CT_KT; ++k) {
+                    const float e = ex2_fast(fmaf(__uint_as_float(sr[k]), p.scale_log2, -ls));
+                    pv[k] = (full || (row_ok && i0 + k < nv)) ? e : 0.f;
+                }
+                float bs[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) bs[j] = 0.f;
+                if (cpb == 4) {
+#pragma unroll
+                    for (int k = 0; k < CT_KT; ++k) bs[k / 4] += pv[k];
+                } else {
+#pragma unroll
+                    for (int k = 0; k < CT_KT; ++k) {
+                        const int j = k / cpb;                   // < 16 since cpb >= 4
+#pragma unroll
+                        for (int jj = 0; jj < 16; ++jj)
+                            if (jj == j) bs[jj] += pv[k];
+                    }
+                }
+                // sum over the 16 heads of the query (lane bits 0-3): lane h
+                // ends with the sum of block h of the tile
+#pragma unroll
+                for (int o = 8; o >= 1; o >>= 1) {
+                    const bool hi = (lane & o) != 0;
+#pragma unroll
+                    for (int j = 0; j < o; ++j) {
+                        const float mine = hi ? bs[j + o] : bs[j];
+                        const float other = hi ? bs[j] : bs[j + o];
+                        bs[j] = mine + __shfl_xor_sync(0xffffffffu, other, o);
+                    }
+                }
+                const int blk = kt * nbt + h;
+                if (t <= t_last && h < nbt && blk < nbk) imp_s[w * nbk + blk] = bs[0];
+            }
+            // all importances of the item are in shared memory
+            if (!atc::agree(1, 128, ok)) { ok = false; break; }
+            const int covered = min(nt * nbt, nbk);
+            for (int wq = quad; wq < CT_Q; wq += 4) {     // each softmax warp: two queries
+                const int tq = t0 + wq;
+                if (tq > t_last) break;
+                float *imp = imp_s + wq * nbk;
+                const int nb_t = min(tq / ip.sel_block + 1, nbk);
+                const int k = min(ip.sel_topk, nb_t);
+                for (int i = covered + lane; i < nb_t; i += 32) imp[i] = 0.f;   // no visible token
+                __syncwarp();
+                int mine = -1;
+                for (int rr = 0; rr < k; ++rr) {
+                    float bv = -1.f;
+                    int bi = 0x7fffffff;
+                    for (int i = lane; i < nb_t; i += 32) {
+                        const float x = imp[i];
+                        if (x > bv) { bv = x; bi = i; }  // lanes scan ascending i: ties keep the lower i
+                    }
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) {
+                        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+                        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+                        if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+                    }
+                    if (lane == rr) mine = bi < nb_t ? bi : -1;
+                    if (lane == 0 && bi < nb_t) imp[bi] = -1.f;
+                    __syncwarp();
+                }
+                int rank = 0;
+                for (int rr = 0; rr < k; ++rr) {
+                    const int other = __shfl_sync(0xffffffffu, mine, rr);
+                    rank += (lane < k && other < mine) ? 1 : 0;
+                }
+                int32_t *dst = ip.sel_idx + ((long long)(b * p.T + tq) * p.Hkv + g) * ip.sel_topk;
+                if (lane < k) dst[rank] = mine;
+                for (int i = k + lane; i < ip.sel_topk; i += 32) dst[i] = -1;
+            }
+            // the next item's tiles overwrite imp_s
+            if (!atc::agree(1, 128, ok)) { ok = false; break; }
+        }
+        if (!ok) fail();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 1) tc::tmem_dealloc(tmem, 128);
+}
+
+}  // namespace sa

@@ -761,6 +761,39 @@ static int launch_nsa_tc(const TileParams &p, unsigned *err, cudaStream_t st) {
     return SA_OK;
 }
 
+static int launch_imp_tc(const NsaSelectParams &sp, unsigned *err, cudaStream_t st) {
+    TileParams p{};
+    p.q = sp.q; p.k = sp.kc; p.klo = sp.klo;
+    p.B = sp.B; p.T = sp.T; p.Lk = std::max(sp.nc, 1); p.Hq = sp.Hq; p.Hkv = sp.Hkv; p.G = sp.G;
+    p.cmp_len = sp.cmp_len; p.cmp_stride = sp.cmp_stride; p.scale_log2 = sp.scale_log2;
+    const long long items = (long long)p.B * p.Hkv * ((p.T + CT_Q - 1) / CT_Q);
+    if (items == 0) return SA_OK;
+    if (items > INT_MAX) return fail(SA_ERR_UNSUPPORTED, "imp_tc: %lld items", items);
+    CUtensorMap qm, khm, klm;
+    int rc = bf16_tensor_map(&qm, p.q, (long long)p.B * p.T * p.Hq, 128, 16);
+    if (rc) return rc;
+    rc = bf16_tensor_map_3d(&khm, p.k, 128, p.Hkv, (long long)p.B * p.Lk);
+    if (rc) return rc;
+    rc = bf16_tensor_map_3d(&klm, p.klo, 128, p.Hkv, (long long)p.B * p.Lk);
+    if (rc) return rc;
+    ImpTcParams ip{p, sp.lse_cmp, sp.sel_block, sp.sel_topk, sp.n_blocks, sp.sel_idx, err, (int)items};
+    const int smem = ItSmem::alloc(sp.n_blocks);
+    if (smem > 227 * 1024) return fail(SA_ERR_UNSUPPORTED, "imp_tc: %d blocks", sp.n_blocks);
+    rc = set_smem(nsa_imp_tc_kernel, smem);
+    if (rc) return rc;
+    const int grid = (int)std::min<long long>(items, sm_count());
+    nsa_imp_tc_kernel<<<grid, CT_THREADS, smem, st>>>(qm, khm, klm, ip);
+    SA_CHECK_LAUNCH("nsa_imp_tc_kernel");
+    return SA_OK;
+}
+
+static bool imp_tc_applies(const NsaSelectParams &sp, int d) {
+    const int cpb = sp.sel_block / sp.cmp_stride;
+    return d == 128 && sp.G <= 16 && sp.imp_out == nullptr && sp.n_blocks <= IT_MAX_BLOCKS &&
+           (cpb == 4 || cpb == 8 || cpb == 16 || cpb == 32 || cpb == 64) && sp.sel_topk <= 32 &&
+           (long long)sp.B * sp.T * sp.Hq + 16 < INT_MAX && (long long)sp.B * sp.nc < INT_MAX;
+}
+
 static bool cmp_tc_applies(const TileParams &p, int d) {
     static int v = -1;
     if (v < 0) {
@@ -847,7 +880,10 @@ int sa_nsa_fwd(const void *q, const void *k, const void *v, const float *gates, 
         sp.sel_topk = sel_topk; sp.n_blocks = lay.n_blocks;
         sp.scale_log2 = base.scale_log2;
         sp.sel_idx = sel; sp.imp_out = nullptr;
-        rc = d == 64 ? launch_nsa_select<64>(sp, st) : launch_nsa_select<128>(sp, st);
+        if (cmp_tc_applies(tp, d) && imp_tc_applies(sp, d))
+            rc = launch_imp_tc(sp, ew, st);
+        else
+            rc = d == 64 ? launch_nsa_select<64>(sp, st) : launch_nsa_select<128>(sp, st);
         if (rc) return rc;
     }
     // 4. selected branch -> o3[1], l3[1]
