@@ -167,6 +167,8 @@ def main():
     ap.add_argument("--seq-len", type=int, default=0,
                     help="prefill length for profiling captures of a smaller case "
                          "(default: the 65536-token workload); the JSON line names it")
+    ap.add_argument("--nsa-seq-len", type=int, default=0,
+                    help="NSA length for profiling captures of a smaller case (default 65536)")
     ap.add_argument("--cpu-sample-rows", type=int, default=0,
                     help="oracle rows for the CPU baseline (0 = auto, ~10-30 s)")
     args = ap.parse_args()
@@ -396,6 +398,8 @@ def extra_measurements(args, dev, torch, api, lib, inputs, flush, world, peaks):
     torch.cuda.empty_cache()
     # --- NSA 64K ---
     w = inputs.WORKLOADS["nsa64k"]
+    if args.nsa_seq_len:
+        w = dataclasses.replace(w, T=int(args.nsa_seq_len))
     g = inputs.gen_nsa(w.B, w.T, w.Hq, w.Hkv, w.d, seed=0)
     gd = {k: v.to(dev) for k, v in g.items()}
     o = torch.empty((w.B, w.T, w.Hq, w.d), dtype=torch.bfloat16, device=dev)
@@ -409,9 +413,10 @@ def extra_measurements(args, dev, torch, api, lib, inputs, flush, world, peaks):
     times = timed_steps(nstep, max(2, steps // 2), args.warmup, flush, dev, torch)
     ms = max_over_ranks(sum(times), dev, torch, dist) / len(times)
     nsa_fl = nsa_flops(w, sel_holder["sel"], torch)
-    res["nsa64k"] = {"ms_per_step": round(ms, 3), "tflops": round(nsa_fl / (ms / 1e3) / 1e12, 2),
-                     "algorithmic_flops": nsa_fl,
-                     "tensor_frac": round(nsa_fl / (ms / 1e3) / 1e12 / peaks["bf16_tflops"], 4)}
+    res["nsa64k" if w.T == 65536 else f"nsa{w.T // 1024}k"] = {
+        "ms_per_step": round(ms, 3), "tflops": round(nsa_fl / (ms / 1e3) / 1e12, 2),
+        "algorithmic_flops": nsa_fl,
+        "tensor_frac": round(nsa_fl / (ms / 1e3) / 1e12 / peaks["bf16_tflops"], 4)}
     del gd, g, o
     torch.cuda.empty_cache()
     # --- fixed graph 16K with coordinate bias ---
