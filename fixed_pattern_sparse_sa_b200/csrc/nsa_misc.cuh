@@ -12,33 +12,56 @@ namespace sa {
 // One warp per row; each lane owns d/32 consecutive columns.
 template <int D>
 __global__ void __launch_bounds__(256) lse_combine_kernel(const float *__restrict__ part_o,
-                                                          const float *__restrict__ part_lse,
-                                                          int n_split, long long rows,
-                                                          __nv_bfloat16 *__restrict__ out,
-                                                          float *__restrict__ lse) {
+                                                         const float *__restrict__ part_lse,
+                                                         int n_split, long long rows,
+                                                         __nv_bfloat16 *__restrict__ out,
+                                                         float *__restrict__ lse) {
     constexpr int PER = D / 32;
     const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= rows) return;
-    float m = -INFINITY;
-    for (int s = lane; s < n_split; s += 32) m = fmaxf(m, part_lse[s * rows + row]);
-    m = warp_max(m);
     float acc[PER];
 #pragma unroll
     for (int i = 0; i < PER; ++i) acc[i] = 0.f;
-    float den = 0.f;
-    if (m != -INFINITY) {
-        for (int s = 0; s < n_split; ++s) {
-            const float ls = part_lse[s * rows + row];
-            if (ls == -INFINITY) continue;
-            const float f = exp2f((ls - m) * kLog2e);
-            den += f;
-            const float *src = part_o + ((long long)s * rows + row) * D + lane * PER;
+    float den = 0.f, m = -INFINITY;
+    if (n_split <= 32) {
+        // lane s holds piece s's LSE; the pieces' partial rows are then read
+        // with independent (unrolled) loads
+        const float lsl = lane < n_split ? part_lse[lane * rows + row] : -INFINITY;
+        m = warp_max(lsl);
+        if (m != -INFINITY) {
+            const float fl = lsl == -INFINITY ? 0.f : exp2f((lsl - m) * kLog2e);
+#pragma unroll 8
+            for (int s = 0; s < n_split; ++s) {
+                const float f = __shfl_sync(0xffffffffu, fl, s);
+                const float *src = part_o + ((long long)s * rows + row) * D + lane * PER;
+                if (f != 0.f) {
+                    den += f;
 #pragma unroll
-            for (int i = 0; i < PER; i += 2) {
-                const float2 x = *reinterpret_cast<const float2 *>(src + i);
-                acc[i] += f * x.x;
-                acc[i + 1] += f * x.y;
+                    for (int i = 0; i < PER; i += 2) {
+                        const float2 x = *reinterpret_cast<const float2 *>(src + i);
+                        acc[i] += f * x.x;
+                        acc[i + 1] += f * x.y;
+                    }
+                }
+            }
+        }
+    } else {
+        for (int s = lane; s < n_split; s += 32) m = fmaxf(m, part_lse[s * rows + row]);
+        m = warp_max(m);
+        if (m != -INFINITY) {
+            for (int s = 0; s < n_split; ++s) {
+                const float ls = part_lse[s * rows + row];
+                if (ls == -INFINITY) continue;
+                const float f = exp2f((ls - m) * kLog2e);
+                den += f;
+                const float *src = part_o + ((long long)s * rows + row) * D + lane * PER;
+#pragma unroll
+                for (int i = 0; i < PER; i += 2) {
+                    const float2 x = *reinterpret_cast<const float2 *>(src + i);
+                    acc[i] += f * x.x;
+                    acc[i + 1] += f * x.y;
+                }
             }
         }
     }
