@@ -859,6 +859,18 @@ template <int DI>
 __host__ __device__ constexpr int select_smem_bytes(int words) {
     return (SEL_BINS + 2 * SEL_TIE_CAP) * 4 + 16 * DI + 16 * 4 + 2 * words * 4;
 }
+// The candidate list of a row (scores and positions, cap entries each) is
+// staged in shared memory after the bitmaps when it fits: the select passes
+// then re-read shared memory instead of L2.
+constexpr int SEL_STAGE_MAX = 8192;      // list entries staged in shared memory
+template <int DI>
+__host__ __device__ constexpr int select_stage_off(int words) {
+    return (select_smem_bytes<DI>(words) + 15) / 16 * 16;
+}
+template <int DI>
+__host__ __device__ constexpr int select_smem_staged(int words, int cap) {
+    return select_stage_off<DI>(words) + (cap <= SEL_STAGE_MAX ? 2 * cap * 4 : 0);
+}
 
 // Exact top-k of one row from its candidate list (or, when the list is
 // unusable, from scores recomputed on CUDA cores).  Keys above the
@@ -866,7 +878,7 @@ __host__ __device__ constexpr int select_smem_bytes(int words) {
 // "equal" bitmap; the output takes every greater key and the lowest-position
 // equal keys, in ascending position order.
 template <int DI>
-__global__ void __launch_bounds__(SEL_THREADS, 4) topk_select_kernel(const IdxParams p) {
+__global__ void __launch_bounds__(SEL_THREADS, 3) topk_select_kernel(const IdxParams p) {
     extern __shared__ __align__(1024) unsigned char smem[];
     int *hist = reinterpret_cast<int *>(smem);                          // [SEL_BINS]
     unsigned *tie_key = reinterpret_cast<unsigned *>(hist + SEL_BINS);  // [SEL_TIE_CAP]
@@ -915,9 +927,23 @@ __global__ void __launch_bounds__(SEL_THREADS, 4) topk_select_kernel(const IdxPa
         for (int i = tid; i < p.Hi; i += SEL_THREADS) w_s[i] = __ldg(p.w + ((long long)b * p.Tq + t) * p.Hi + i);
         __syncthreads();
     }
+    // stage the list in shared memory (one pass over L2, 16-byte loads)
+    const bool staged = use_list && p.cand_cap <= SEL_STAGE_MAX;
+    int *lv_s = reinterpret_cast<int *>(smem + select_stage_off<DI>(words));
+    int *li_s = lv_s + p.cand_cap;
+    if (staged) {
+        const int n4 = (cnt + 3) / 4;                 // rows are 16-byte aligned (cap % 64 == 0)
+        for (int i = tid; i < n4; i += SEL_THREADS) {
+            reinterpret_cast<int4 *>(lv_s)[i] = __ldg(reinterpret_cast<const int4 *>(cv) + i);
+            reinterpret_cast<int4 *>(li_s)[i] = __ldg(reinterpret_cast<const int4 *>(ci) + i);
+        }
+        __syncthreads();
+    }
     // every element of the row: (score, position)
     auto for_each = [&](auto f) {
-        if (use_list) {
+        if (staged) {
+            for (int i = tid; i < cnt; i += SEL_THREADS) f(lv_s[i], li_s[i]);
+        } else if (use_list) {
             constexpr int U = 4;
             for (int b0 = tid; b0 < cnt; b0 += SEL_THREADS * U) {
                 int v[U], jj[U];

@@ -589,7 +589,7 @@ static int launch_score(const IdxParams &p, bool decode, long long n_keys_max, c
 
 template <int DI>
 static int launch_select_t(const IdxParams &p, int words, cudaStream_t st) {
-    const int smem = select_smem_bytes<DI>(words);
+    const int smem = select_smem_staged<DI>(words, p.cand_cap);
     int rc = set_smem(topk_select_kernel<DI>, smem);
     if (rc) return rc;
     topk_select_kernel<DI><<<dim3(1u, (unsigned)p.Rt, (unsigned)p.B), SEL_THREADS, smem, st>>>(p);
