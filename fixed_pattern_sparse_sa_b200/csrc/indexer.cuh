@@ -701,7 +701,7 @@ struct RadixState {
 // One histogram refinement step over the keys of the current bin.
 // `for_each(f)` calls f(value, position) for every element of the row.
 // Block-uniform result.
-template <typename ForEach>
+template <int NT = SEL_THREADS, typename ForEach>
 __device__ void radix_refine(RadixState &st, int gmin, int *hist, int *scan_tmp, int *bcast, ForEach for_each) {
     const int tid = threadIdx.x;
     const int shift = st.width > SEL_BITS ? st.width - SEL_BITS : 0;
@@ -714,12 +714,12 @@ __device__ void radix_refine(RadixState &st, int gmin, int *hist, int *scan_tmp,
         if (key >= lo && key <= hi) atomicAdd(&hist[(key - lo) >> shift], 1);
     });
     __syncthreads();
-    constexpr int per = SEL_BINS / SEL_THREADS;   // bins per thread, highest first
+    constexpr int per = NT >= SEL_BINS ? 1 : SEL_BINS / NT;   // bins per thread, highest first
     int cntb[per];
     int local = 0;
 #pragma unroll
     for (int u = 0; u < per; ++u) {
-        cntb[u] = hist[SEL_BINS - 1 - (tid * per + u)];
+        cntb[u] = tid * per + u < SEL_BINS ? hist[SEL_BINS - 1 - (tid * per + u)] : 0;
         local += cntb[u];
     }
     const int incl = block_incl_scan(local, scan_tmp);
@@ -727,7 +727,7 @@ __device__ void radix_refine(RadixState &st, int gmin, int *hist, int *scan_tmp,
 #pragma unroll
     for (int u = 0; u < per; ++u) {
         const int bin = SEL_BINS - 1 - (tid * per + u);
-        if (above < st.k_rem && above + cntb[u] >= st.k_rem) {
+        if (tid * per + u < SEL_BINS && above < st.k_rem && above + cntb[u] >= st.k_rem) {
             bcast[2] = bin;
             bcast[3] = above;
         }
@@ -877,8 +877,8 @@ __host__ __device__ constexpr int select_smem_staged(int words, int cap) {
 // threshold go to a "greater" bitmap over positions, keys equal to it to an
 // "equal" bitmap; the output takes every greater key and the lowest-position
 // equal keys, in ascending position order.
-template <int DI>
-__global__ void __launch_bounds__(SEL_THREADS, 3) topk_select_kernel(const IdxParams p) {
+template <int DI, int NT = SEL_THREADS>
+__global__ void __launch_bounds__(NT, NT <= 256 ? 3 : 1) topk_select_kernel(const IdxParams p) {
     extern __shared__ __align__(1024) unsigned char smem[];
     int *hist = reinterpret_cast<int *>(smem);                          // [SEL_BINS]
     unsigned *tie_key = reinterpret_cast<unsigned *>(hist + SEL_BINS);  // [SEL_TIE_CAP]
@@ -889,7 +889,7 @@ __global__ void __launch_bounds__(SEL_THREADS, 3) topk_select_kernel(const IdxPa
     __shared__ int scan_tmp[32];
     __shared__ int bcast[4];
     __shared__ int tie_n;
-    constexpr int NW = SEL_THREADS / 32;
+    constexpr int NW = NT / 32;
     __shared__ int wg[NW], we[NW];
 
     const int b = blockIdx.z, tr = blockIdx.y, t = p.t0 + tr;
@@ -905,11 +905,11 @@ __global__ void __launch_bounds__(SEL_THREADS, 3) topk_select_kernel(const IdxPa
     unsigned *eq_bm = gt_bm + words;
 
     // window entries, padding and count
-    for (int i = tid; i < p.Kout - k_eff; i += SEL_THREADS)
+    for (int i = tid; i < p.Kout - k_eff; i += NT)
         orow[k_eff + i] = i < wc ? (int)(pos - wc + 1 + i) : -1;
     if (tid == 0 && p.out_count) p.out_count[(long long)b * p.Tq + t] = k_eff + wc;
     if (k_eff == n) {                                 // every candidate is kept
-        for (int j = tid; j < n; j += SEL_THREADS) orow[j] = j;
+        for (int j = tid; j < n; j += NT) orow[j] = j;
         return;
     }
     if (k_eff == 0) return;
@@ -922,9 +922,9 @@ __global__ void __launch_bounds__(SEL_THREADS, 3) topk_select_kernel(const IdxPa
     if (!use_list) {
         // exact recompute: stage this query's indexer vectors and weights
         const int8_t *qsrc = p.q + ((long long)b * p.Tq + t) * p.Hi * DI;
-        for (int i = tid; i < p.Hi * DI / 16; i += SEL_THREADS)
+        for (int i = tid; i < p.Hi * DI / 16; i += NT)
             reinterpret_cast<int4 *>(qrow_s)[i] = __ldg(reinterpret_cast<const int4 *>(qsrc) + i);
-        for (int i = tid; i < p.Hi; i += SEL_THREADS) w_s[i] = __ldg(p.w + ((long long)b * p.Tq + t) * p.Hi + i);
+        for (int i = tid; i < p.Hi; i += NT) w_s[i] = __ldg(p.w + ((long long)b * p.Tq + t) * p.Hi + i);
         __syncthreads();
     }
     // stage the list in shared memory (one pass over L2, 16-byte loads)
@@ -933,7 +933,7 @@ __global__ void __launch_bounds__(SEL_THREADS, 3) topk_select_kernel(const IdxPa
     int *li_s = lv_s + p.cand_cap;
     if (staged) {
         const int n4 = (cnt + 3) / 4;                 // rows are 16-byte aligned (cap % 64 == 0)
-        for (int i = tid; i < n4; i += SEL_THREADS) {
+        for (int i = tid; i < n4; i += NT) {
             reinterpret_cast<int4 *>(lv_s)[i] = __ldg(reinterpret_cast<const int4 *>(cv) + i);
             reinterpret_cast<int4 *>(li_s)[i] = __ldg(reinterpret_cast<const int4 *>(ci) + i);
         }
@@ -942,22 +942,22 @@ __global__ void __launch_bounds__(SEL_THREADS, 3) topk_select_kernel(const IdxPa
     // every element of the row: (score, position)
     auto for_each = [&](auto f) {
         if (staged) {
-            for (int i = tid; i < cnt; i += SEL_THREADS) f(lv_s[i], li_s[i]);
+            for (int i = tid; i < cnt; i += NT) f(lv_s[i], li_s[i]);
         } else if (use_list) {
             constexpr int U = 4;
-            for (int b0 = tid; b0 < cnt; b0 += SEL_THREADS * U) {
+            for (int b0 = tid; b0 < cnt; b0 += NT * U) {
                 int v[U], jj[U];
 #pragma unroll
                 for (int u = 0; u < U; ++u) {
-                    const int i = b0 + u * SEL_THREADS;
+                    const int i = b0 + u * NT;
                     if (i < cnt) { v[u] = __ldg(cv + i); jj[u] = __ldg(ci + i); }
                 }
 #pragma unroll
                 for (int u = 0; u < U; ++u)
-                    if (b0 + u * SEL_THREADS < cnt) f(v[u], jj[u]);
+                    if (b0 + u * NT < cnt) f(v[u], jj[u]);
             }
         } else {
-            for (int j = tid; j < n; j += SEL_THREADS) f(exact_score<DI>(qrow_s, w_s, p.Hi, kb + (long long)j * DI), j);
+            for (int j = tid; j < n; j += NT) f(exact_score<DI>(qrow_s, w_s, p.Hi, kb + (long long)j * DI), j);
         }
     };
 
@@ -966,11 +966,11 @@ __global__ void __launch_bounds__(SEL_THREADS, 3) topk_select_kernel(const IdxPa
     const unsigned range = (unsigned)gmax - (unsigned)gmin;
     RadixState st{0u, range == 0 ? 0 : 32 - __clz(range), k_eff, use_list ? cnt : n};
     while (st.width > 0 && (st.width > SEL_BITS || st.bin_count > SEL_TIE_CAP))
-        radix_refine(st, gmin, hist, scan_tmp, bcast, for_each);
+        radix_refine<NT>(st, gmin, hist, scan_tmp, bcast, for_each);
 
     // filter: bitmaps of keys above the bin; the bin's own elements go to the
     // equal bitmap (width 0) or to the tie list
-    for (int i = tid; i < words; i += SEL_THREADS) { gt_bm[i] = 0u; eq_bm[i] = 0u; }
+    for (int i = tid; i < words; i += NT) { gt_bm[i] = 0u; eq_bm[i] = 0u; }
     if (tid == 0) tie_n = 0;
     __syncthreads();
     const unsigned lo_key = st.lo_key;
@@ -995,12 +995,12 @@ __global__ void __launch_bounds__(SEL_THREADS, 3) topk_select_kernel(const IdxPa
         const int m = min(tie_n, SEL_TIE_CAP);
         RadixState ts{0u, width, k_rem, m};
         auto tie_each = [&](auto f) {
-            for (int i = tid; i < m; i += SEL_THREADS) f((int)tie_key[i], tie_idx[i]);
+            for (int i = tid; i < m; i += NT) f((int)tie_key[i], tie_idx[i]);
         };
-        radix_refine(ts, 0, hist, scan_tmp, bcast, tie_each);   // width <= 12: one step is exact
+        radix_refine<NT>(ts, 0, hist, scan_tmp, bcast, tie_each);   // width <= 12: one step is exact
         const unsigned thr_off = ts.lo_key;
         k_rem = ts.k_rem;
-        for (int i = tid; i < m; i += SEL_THREADS) {
+        for (int i = tid; i < m; i += NT) {
             const int j = tie_idx[i];
             if (tie_key[i] > thr_off) atomicOr(&gt_bm[j >> 5], 1u << (j & 31));
             else if (tie_key[i] == thr_off) atomicOr(&eq_bm[j >> 5], 1u << (j & 31));

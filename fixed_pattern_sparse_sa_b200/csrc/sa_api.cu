@@ -587,14 +587,22 @@ static int launch_score(const IdxParams &p, bool decode, long long n_keys_max, c
     return fail(SA_ERR_UNSUPPORTED, "indexer heads %d", p.Hi);
 }
 
-template <int DI>
-static int launch_select_t(const IdxParams &p, int words, cudaStream_t st) {
+// One CTA per row; when there are few rows (decode) a row gets 1024 threads.
+template <int DI, int NT>
+static int launch_select_nt(const IdxParams &p, int words, cudaStream_t st) {
     const int smem = select_smem_staged<DI>(words, p.cand_cap);
-    int rc = set_smem(topk_select_kernel<DI>, smem);
+    auto kern = topk_select_kernel<DI, NT>;
+    int rc = set_smem(kern, smem);
     if (rc) return rc;
-    topk_select_kernel<DI><<<dim3(1u, (unsigned)p.Rt, (unsigned)p.B), SEL_THREADS, smem, st>>>(p);
+    kern<<<dim3(1u, (unsigned)p.Rt, (unsigned)p.B), NT, smem, st>>>(p);
     SA_CHECK_LAUNCH("topk_select_kernel");
     return SA_OK;
+}
+
+template <int DI>
+static int launch_select_t(const IdxParams &p, int words, cudaStream_t st) {
+    if ((long long)p.B * p.Rt <= sm_count()) return launch_select_nt<DI, 1024>(p, words, st);
+    return launch_select_nt<DI, SEL_THREADS>(p, words, st);
 }
 
 int sa_indexer_topk(const int8_t *q_idx, const int8_t *k_idx, const int32_t *w, int B, int Tq, int L,
