@@ -474,9 +474,9 @@ def cpu_baseline(args, max_seconds=25.0):
         full[0, rows] = idx
         oracle.sparse_attn(g["q"], g["k"], g["v"], full, rows=rows)
         dt = time.perf_counter() - t0
-        if args.cpu_sample_rows or dt >= 8.0 or n >= 4096:
+        if args.cpu_sample_rows or dt >= 8.0 or n >= 16384:
             break
-        n = min(4096, int(n * max(2.0, 10.0 / max(dt, 1e-3))))
+        n = min(16384, int(n * max(2.0, 12.0 / max(dt, 1e-3))))
     counts = np.minimum(rows + 1, w.topk + w.window)
     fl = 4.0 * w.d * w.Hq * float(counts.sum())
     cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
