@@ -31,7 +31,7 @@
 
 namespace sa {
 
-constexpr int SAMPLE_TARGET = 4096;       // sampled keys per row (stride = n / target)
+constexpr int SAMPLE_TARGET = 2048;       // sampled keys per row (stride = n / target)
 constexpr double SAMPLE_Z = 4.5;          // safety margin of the sampled threshold, in sigmas
 
 struct IdxParams {
