@@ -35,23 +35,32 @@
 namespace sa {
 
 constexpr int CT_Q = 8;            // queries per item (x 16 heads = 128 rows)
-constexpr int CT_KT = 64;          // compressed keys per tile
-constexpr int CT_STAGES = 3;
-constexpr int CT_THREADS = 192;
+constexpr int CT_KT = 64;          // compressed keys per tile of the importance kernel
+constexpr int CT_THREADS = 192;    // importance kernel: TMA warp, MMA warp, 4 score warps
+
+// nsa_tc_kernel: 128-key tiles (S = Q.K^T at N = 128), two stages, P in
+// tensor memory as the A operand of P.V, 8 softmax warps.
+constexpr int NT_KT = 128;
+constexpr int NT_STAGES = 2;
+constexpr int NT_THREADS = 320;      // TMA warp, MMA warp, 8 softmax warps (two per TMEM lane quadrant)
+constexpr uint32_t NT_TM_S = 0;      // S: 2 buffers x NT_KT fp32 columns
+constexpr uint32_t NT_TM_P = 256;    // P: 2 buffers x NT_KT / 2 columns (bf16 pairs)
+constexpr uint32_t NT_TM_O = 384;    // O: 128 fp32 columns
+constexpr uint32_t NT_TM_COLS = 512;
 
 struct CtSmem {                    // head dim 128
     static constexpr int Q_BYTES = 128 * 256;              // 2 halves x 128 rows x 128 B
-    static constexpr int KT_BYTES = CT_KT * 256;           // one K (or V) tile: 2 halves x 64 rows x 128 B
+    static constexpr int KT_BYTES = NT_KT * 256;           // one K (or V) tile: 2 halves x 128 rows x 128 B
     static constexpr int STAGE = 3 * KT_BYTES;             // K_hi | K_lo | V
-    static constexpr int P_BYTES = 128 * CT_KT * 2;        // 128 rows x 128 B
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_KV = OFF_Q + Q_BYTES;
-    static constexpr int OFF_P = OFF_KV + CT_STAGES * STAGE;
-    static constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
+    static constexpr int OFF_BAR = OFF_KV + NT_STAGES * STAGE;
     // q_full, q_empty, kv_full[S], kv_empty[S], s_full[2], s_free[2], p_full[2],
     // pv_done[2], o_full, o_free, drain
-    static constexpr int N_BAR = 2 + 2 * CT_STAGES + 8 + 3;
-    static constexpr int OFF_MISC = OFF_BAR + N_BAR * 8;
+    static constexpr int N_BAR = 2 + 2 * NT_STAGES + 8 + 3;
+    // [half][row]: partial row maxima of the current tile, then the row sums
+    static constexpr int OFF_XCH = OFF_BAR + N_BAR * 8;
+    static constexpr int OFF_MISC = OFF_XCH + 2 * 128 * 4;
     static constexpr int TOTAL = OFF_MISC + 16;
     static constexpr int ALLOC = TOTAL + 1024;
 };
@@ -92,7 +101,7 @@ __device__ __forceinline__ void ct_item(const TileParams &p, int it, int &b, int
 }
 
 template <int SRC>
-__global__ void __launch_bounds__(CT_THREADS, 1)
+__global__ void __launch_bounds__(NT_THREADS, 1)
     nsa_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap khimap,
                   const __grid_constant__ CUtensorMap klomap, const __grid_constant__ CUtensorMap vmap,
                   const CmpTcParams cp) {
@@ -103,25 +112,26 @@ __global__ void __launch_bounds__(CT_THREADS, 1)
     extern __shared__ unsigned char smem_raw[];
     unsigned char *smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::OFF_BAR);
-    uint64_t *q_full = bars, *q_empty = bars + 1, *kv_full = bars + 2, *kv_empty = kv_full + CT_STAGES;
-    uint64_t *s_full = kv_empty + CT_STAGES, *s_free = s_full + 2, *p_full = s_free + 2, *pv_done = p_full + 2;
+    uint64_t *q_full = bars, *q_empty = bars + 1, *kv_full = bars + 2, *kv_empty = kv_full + NT_STAGES;
+    uint64_t *s_full = kv_empty + NT_STAGES, *s_free = s_full + 2, *p_full = s_free + 2, *pv_done = p_full + 2;
     uint64_t *o_full = pv_done + 2, *o_free = o_full + 1, *drain = o_free + 1;
+    float *xch = reinterpret_cast<float *>(smem + L::OFF_XCH);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::OFF_MISC + 4);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     if (warp == 1) {
-        tc::tmem_alloc(tmem_slot, 256);   // S x2 (cols 0-127), O (cols 128-255)
+        tc::tmem_alloc(tmem_slot, NT_TM_COLS);
         tc::tmem_relinquish();
     }
     if (tid == 0) {
         tc::mbar_init(q_full, 1); tc::mbar_init(q_empty, 1);
-        for (int i = 0; i < CT_STAGES; ++i) { tc::mbar_init(kv_full + i, 1); tc::mbar_init(kv_empty + i, 1); }
+        for (int i = 0; i < NT_STAGES; ++i) { tc::mbar_init(kv_full + i, 1); tc::mbar_init(kv_empty + i, 1); }
         for (int i = 0; i < 2; ++i) {
-            tc::mbar_init(s_full + i, 1); tc::mbar_init(s_free + i, 128);
-            tc::mbar_init(p_full + i, 128); tc::mbar_init(pv_done + i, 1);
+            tc::mbar_init(s_full + i, 1); tc::mbar_init(s_free + i, 256);
+            tc::mbar_init(p_full + i, 256); tc::mbar_init(pv_done + i, 1);
         }
-        tc::mbar_init(o_full, 1); tc::mbar_init(o_free, 128);
+        tc::mbar_init(o_full, 1); tc::mbar_init(o_free, 256);
         tc::mbar_init(drain, 1);
         *abort_flag = 0;
         tc::mbar_fence_init();
@@ -138,7 +148,7 @@ __global__ void __launch_bounds__(CT_THREADS, 1)
     auto key_lo = [&](int t0) -> int { return SRC == TS_CMP ? 0 : max(0, t0 - p.window + 1); };
     auto tiles_of = [&](int t0) -> int {
         const int t_last = min(t0 + CT_Q - 1, p.T - 1);
-        return ((int)tile_key_end<SRC>(p, t_last) - key_lo(t0) + CT_KT - 1) / CT_KT;
+        return ((int)tile_key_end<SRC>(p, t_last) - key_lo(t0) + NT_KT - 1) / NT_KT;
     };
 
     if (warp == 0) {
@@ -160,38 +170,38 @@ __global__ void __launch_bounds__(CT_THREADS, 1)
                 }
                 ++qn;
                 for (int kt = 0; kt < nt; ++kt, ++tile) {
-                    const int st = tile % CT_STAGES;
-                    if (!atc::wait(kv_empty + st, ((tile / CT_STAGES) & 1) ^ 1, abort_flag)) { ok = false; break; }
+                    const int st = tile % NT_STAGES;
+                    if (!atc::wait(kv_empty + st, ((tile / NT_STAGES) & 1) ^ 1, abort_flag)) { ok = false; break; }
                     atc::expect_tx(kv_full + st, LO ? L::STAGE : 2 * L::KT_BYTES);
                     unsigned char *dst = smem + L::OFF_KV + st * L::STAGE;
-                    const int z = b * p.Lk + key_lo(t0) + kt * CT_KT;
+                    const int z = b * p.Lk + key_lo(t0) + kt * NT_KT;
                     for (int h = 0; h < 2; ++h) {
-                        atc::load_3d(dst + h * (CT_KT * 128), &khimap, h * 64, g, z, kv_full + st);
-                        if (LO) atc::load_3d(dst + L::KT_BYTES + h * (CT_KT * 128), &klomap, h * 64, g, z, kv_full + st);
-                        atc::load_3d(dst + 2 * L::KT_BYTES + h * (CT_KT * 128), &vmap, h * 64, g, z, kv_full + st);
+                        atc::load_3d(dst + h * (NT_KT * 128), &khimap, h * 64, g, z, kv_full + st);
+                        if (LO) atc::load_3d(dst + L::KT_BYTES + h * (NT_KT * 128), &klomap, h * 64, g, z, kv_full + st);
+                        atc::load_3d(dst + 2 * L::KT_BYTES + h * (NT_KT * 128), &vmap, h * 64, g, z, kv_full + st);
                     }
                 }
             }
             if (!ok) fail();
             // let the copies land before the CTA exits
             if (qn > 0) tc::mbar_wait_bounded(q_full, (qn - 1) & 1, ATC_WAIT);
-            for (int i = 0; i < CT_STAGES && i < tile; ++i) {
+            for (int i = 0; i < NT_STAGES && i < tile; ++i) {
                 const int kt = tile - 1 - i;
-                tc::mbar_wait_bounded(kv_full + kt % CT_STAGES, (kt / CT_STAGES) & 1, ATC_WAIT);
+                tc::mbar_wait_bounded(kv_full + kt % NT_STAGES, (kt / NT_STAGES) & 1, ATC_WAIT);
             }
         }
         __syncwarp();
     } else if (warp == 1) {
         // --------------------------------------------------------------- MMA
         if (lane == 0) {
-            constexpr uint32_t ID_S = tc::make_idesc(1, 1, 128, CT_KT);
+            constexpr uint32_t ID_S = tc::make_idesc(1, 1, 128, NT_KT);
             constexpr uint32_t ID_O = tc::make_idesc(1, 1, 128, D) | (1u << 16);   // B (V) MN-major
             const uint32_t qa = tc::smem_u32(smem + L::OFF_Q);
             bool ok = true;
             int tile = 0, qn = 0, on = 0;   // tiles, Q loads, items with an O result
             auto issue_s = [&](int tl) -> bool {
-                const int st = tl % CT_STAGES, sb = tl & 1;
-                if (!atc::wait(kv_full + st, (tl / CT_STAGES) & 1, abort_flag)) return false;
+                const int st = tl % NT_STAGES, sb = tl & 1;
+                if (!atc::wait(kv_full + st, (tl / NT_STAGES) & 1, abort_flag)) return false;
                 if (!atc::wait(s_free + sb, ((tl >> 1) & 1) ^ 1, abort_flag)) return false;
                 tc::fence_after_sync();
                 const uint32_t ka = tc::smem_u32(smem + L::OFF_KV + st * L::STAGE);
@@ -199,10 +209,10 @@ __global__ void __launch_bounds__(CT_THREADS, 1)
                 for (int ks = 0; ks < D / 16; ++ks) {
                     const int h = ks / 4, kk = ks % 4;
                     const uint64_t ad = atc::desc_sw128(qa + h * (128 * 128) + kk * 32, 16, 1024);
-                    const uint64_t bh = atc::desc_sw128(ka + h * (CT_KT * 128) + kk * 32, 16, 1024);
-                    const uint64_t bl = atc::desc_sw128(ka + L::KT_BYTES + h * (CT_KT * 128) + kk * 32, 16, 1024);
-                    tc::mma_bf16(tmem + sb * CT_KT, ad, bh, ID_S, ks > 0 ? 1u : 0u);
-                    if (LO) tc::mma_bf16(tmem + sb * CT_KT, ad, bl, ID_S, 1u);
+                    const uint64_t bh = atc::desc_sw128(ka + h * (NT_KT * 128) + kk * 32, 16, 1024);
+                    const uint64_t bl = atc::desc_sw128(ka + L::KT_BYTES + h * (NT_KT * 128) + kk * 32, 16, 1024);
+                    tc::mma_bf16(tmem + NT_TM_S + sb * NT_KT, ad, bh, ID_S, ks > 0 ? 1u : 0u);
+                    if (LO) tc::mma_bf16(tmem + NT_TM_S + sb * NT_KT, ad, bl, ID_S, 1u);
                 }
                 tc::mma_commit(s_full + sb);
                 return true;
@@ -218,19 +228,19 @@ __global__ void __launch_bounds__(CT_THREADS, 1)
                 // the previous item's epilogue must have read O before it is overwritten
                 if (on > 0 && !atc::wait(o_free, (on - 1) & 1, abort_flag)) { ok = false; break; }
                 for (int kt = 0; kt < nt; ++kt, ++tile) {
-                    const int st = tile % CT_STAGES, pb = tile & 1;
+                    const int st = tile % NT_STAGES, pb = tile & 1;
                     if (kt + 1 < nt && !issue_s(tile + 1)) { ok = false; break; }
                     if (kt + 1 == nt) tc::mma_commit(q_empty);   // Q is free once the last S is done
                     if (!atc::wait(p_full + pb, (tile >> 1) & 1, abort_flag)) { ok = false; break; }
                     tc::fence_after_sync();
+                    // O += P.V: P (A) from tensor memory, V (B) from shared memory
                     const uint32_t va = tc::smem_u32(smem + L::OFF_KV + st * L::STAGE + 2 * L::KT_BYTES);
-                    const uint32_t pa = tc::smem_u32(smem + L::OFF_P + pb * L::P_BYTES);
 #pragma unroll
-                    for (int kk = 0; kk < CT_KT / 16; ++kk) {
-                        const uint64_t ad = atc::desc_sw128(pa + kk * 32, 16, 1024);
-                        // V: MN-major, 64-column atoms 8 KB apart, 8-key groups 1 KB apart
-                        const uint64_t bd = atc::desc_sw128(va + kk * 2048, CT_KT * 128, 1024);
-                        tc::mma_bf16(tmem + 128, ad, bd, ID_O, (kt > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < NT_KT / 16; ++kk) {
+                        // V: MN-major, 64-column atoms NT_KT * 128 B apart, 8-key groups 1 KB apart
+                        const uint64_t bd = atc::desc_sw128(va + kk * 2048, NT_KT * 128, 1024);
+                        tc::mma_bf16_ts(tmem + NT_TM_O, tmem + NT_TM_P + pb * (NT_KT / 2) + kk * 8, bd, ID_O,
+                                        (kt > 0 || kk > 0) ? 1u : 0u);
                     }
                     tc::mma_commit(kv_empty + st);
                     tc::mma_commit(pv_done + pb);
@@ -245,7 +255,15 @@ __global__ void __launch_bounds__(CT_THREADS, 1)
         __syncwarp();
     } else {
         // ----------------------------------------------------- softmax rows
-        const int quad = warp & 3;
+        // Two warps per TMEM lane quadrant share its 32 rows: half 0 takes S
+        // and P columns 0-63 and O columns 0-63 of the quadrant's rows, half 1
+        // the rest.  The pair agrees on each wait through a 64-thread named
+        // barrier (ids 1-4) and swaps partial row maxima (per tile) and row
+        // sums (per item) through shared memory; the agreement at the start
+        // of each tile keeps one exchange slot per row safe to reuse.
+        const int quad = warp & 3, half = (warp - 2) >> 2;
+        const int pair = 1 + quad;
+        constexpr int SC = NT_KT / 2, OC = D / 2;          // S and O columns per warp
         const int r = quad * 32 + lane;                   // row = query w x 16 + head h
         const int w = r >> 4, h = r & 15;
         const uint32_t lrow = (uint32_t)(quad * 32) << 16;
@@ -265,42 +283,40 @@ __global__ void __launch_bounds__(CT_THREADS, 1)
             float m = -INFINITY, l = 0.f;
             for (int kt = 0; kt < nt; ++kt, ++tile) {
                 const int sb = tile & 1, pb = tile & 1;
-                if (!__all_sync(0xffffffffu, atc::wait(s_full + sb, (tile >> 1) & 1, abort_flag))) {
-                    ok = false;
-                    break;
-                }
+                // S of this tile; the P.V of tile - 2 (the last reader of P buffer
+                // pb) was issued before it, so that wait costs nothing
+                bool got = atc::wait(s_full + sb, (tile >> 1) & 1, abort_flag);
+                if (got && tile >= 2) got = atc::wait(pv_done + pb, ((tile >> 1) & 1) ^ 1, abort_flag);
+                if (!atc::agree(pair, 64, got)) { ok = false; break; }
                 tc::fence_after_sync();
-                uint32_t sr[CT_KT];
-                {
-                    uint32_t (&s0)[16] = *reinterpret_cast<uint32_t(*)[16]>(sr);
-                    uint32_t (&s1)[16] = *reinterpret_cast<uint32_t(*)[16]>(sr + 16);
-                    uint32_t (&s2)[16] = *reinterpret_cast<uint32_t(*)[16]>(sr + 32);
-                    uint32_t (&s3)[16] = *reinterpret_cast<uint32_t(*)[16]>(sr + 48);
-                    tc::tmem_ld16(tmem + lrow + sb * CT_KT, s0);
-                    tc::tmem_ld16(tmem + lrow + sb * CT_KT + 16, s1);
-                    tc::tmem_ld16(tmem + lrow + sb * CT_KT + 32, s2);
-                    tc::tmem_ld16(tmem + lrow + sb * CT_KT + 48, s3);
-                }
+                uint32_t sr[SC];
+#pragma unroll
+                for (int c = 0; c < SC; c += 16)
+                    tc::tmem_ld16(tmem + lrow + NT_TM_S + sb * NT_KT + half * SC + c,
+                                  *reinterpret_cast<uint32_t(*)[16]>(sr + c));
                 tc::tmem_ld_wait();
                 tc::fence_before_sync();
                 atc::arrive(s_free + sb);
-                const int i0 = kt * CT_KT;
-                // row max of the raw scores (masked past the row's visible keys)
-                const bool full = i0 >= vlo && i0 + CT_KT <= vhi;
-                float mt = -INFINITY;
-                if (full) {
+                const int i0 = kt * NT_KT + half * SC;
+                // partial row max of the raw scores (masked past the row's visible keys)
+                float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                if (i0 >= vlo && i0 + SC <= vhi) {
 #pragma unroll
-                    for (int k = 0; k < CT_KT; k += 2)
-                        mt = fmaxf(mt, fmaxf(__uint_as_float(sr[k]), __uint_as_float(sr[k + 1])));
+                    for (int k = 0; k < SC; ++k) mx[k & 3] = fmaxf(mx[k & 3], __uint_as_float(sr[k]));
                 } else {
 #pragma unroll
-                    for (int k = 0; k < CT_KT; ++k) {
+                    for (int k = 0; k < SC; ++k) {
                         if (i0 + k < vlo || i0 + k >= vhi) sr[k] = __float_as_uint(-INFINITY);
-                        mt = fmaxf(mt, __uint_as_float(sr[k]));
+                        mx[k & 3] = fmaxf(mx[k & 3], __uint_as_float(sr[k]));
                     }
                 }
+                float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+                xch[half * 128 + r] = mt;
+                atc::named_sync(pair, 64);
+                mt = fmaxf(mt, xch[(half ^ 1) * 128 + r]);
                 // m is kept in raw-score units; raise it only when the tile
-                // exceeds it by more than 2^8 after scaling
+                // exceeds it by more than 2^8 after scaling (both warps of the
+                // pair see the same m and mt, so they decide alike)
                 const bool raise = mt != -INFINITY && (m == -INFINITY || (mt - m) * p.scale_log2 > 8.f);
                 float alpha = 1.f;
                 if (raise) {
@@ -309,50 +325,42 @@ __global__ void __launch_bounds__(CT_THREADS, 1)
                     l *= alpha;
                 }
                 if (kt > 0 && __any_sync(0xffffffffu, raise)) {
-                    // rescale the O rows of this warp once the previous P.V is done
+                    // rescale this warp's O columns once the previous P.V is done
                     const int pt = tile - 1;
-                    if (__all_sync(0xffffffffu, atc::wait(pv_done + (pt & 1), (pt >> 1) & 1, abort_flag))) {
-                        tc::fence_after_sync();
-#pragma unroll
-                        for (int c = 0; c < D; c += 16) {
-                            uint32_t o16[16];
-                            tc::tmem_ld16(tmem + lrow + 128 + c, o16);
-                            tc::tmem_ld_wait();
-#pragma unroll
-                            for (int e = 0; e < 16; ++e) o16[e] = __float_as_uint(__uint_as_float(o16[e]) * alpha);
-                            atc::tmem_st16(tmem + lrow + 128 + c, o16);
-                        }
-                        atc::tmem_st_wait();
-                    } else {
+                    if (!atc::agree(pair, 64, atc::wait(pv_done + (pt & 1), (pt >> 1) & 1, abort_flag))) {
                         ok = false;
                         break;
                     }
+                    tc::fence_after_sync();
+#pragma unroll
+                    for (int c = 0; c < OC; c += 16) {
+                        uint32_t o16[16];
+                        tc::tmem_ld16(tmem + lrow + NT_TM_O + half * OC + c, o16);
+                        tc::tmem_ld_wait();
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) o16[e] = __float_as_uint(__uint_as_float(o16[e]) * alpha);
+                        atc::tmem_st16(tmem + lrow + NT_TM_O + half * OC + c, o16);
+                    }
+                    atc::tmem_st_wait();
                 }
                 // p = 2^((s - m) * scale_log2): one FFMA and one ex2 per score
                 const float nb = m == -INFINITY ? 0.f : -m * p.scale_log2;
-                uint32_t pk[CT_KT / 2];
-                float rs0 = 0.f, rs1 = 0.f;
+                uint32_t pk[SC / 2];
+                float rs[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int k = 0; k < CT_KT; k += 2) {
+                for (int k = 0; k < SC; k += 2) {
                     const float p0 = ex2_fast(fmaf(__uint_as_float(sr[k]), p.scale_log2, nb));
                     const float p1 = ex2_fast(fmaf(__uint_as_float(sr[k + 1]), p.scale_log2, nb));
-                    rs0 += p0;
-                    rs1 += p1;
+                    rs[(k >> 1) & 3] += p0 + p1;
                     pk[k / 2] = pack_bf16(p0, p1);
                 }
-                l += rs0 + rs1;
-                // P buffer pb was last read by the P.V of tile - 2
-                if (tile >= 2 &&
-                    !__all_sync(0xffffffffu, atc::wait(pv_done + pb, ((tile >> 1) & 1) ^ 1, abort_flag))) {
-                    ok = false;
-                    break;
-                }
-                unsigned char *prow = smem + L::OFF_P + pb * L::P_BYTES + r * 128;
+                l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
+                // this warp's keys of row r as packed bf16 pairs in P buffer pb
 #pragma unroll
-                for (int c = 0; c < CT_KT / 8; ++c)
-                    *reinterpret_cast<uint4 *>(prow + ((c ^ (r & 7)) << 4)) =
-                        make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-                tc::fence_proxy_async_smem();
+                for (int c = 0; c < SC / 2; c += 16)
+                    atc::tmem_st16(tmem + lrow + NT_TM_P + pb * (NT_KT / 2) + half * (SC / 2) + c,
+                                   *reinterpret_cast<const uint32_t(*)[16]>(pk + c));
+                atc::tmem_st_wait();
                 tc::fence_before_sync();
                 atc::arrive(p_full + pb);
             }
@@ -360,24 +368,28 @@ __global__ void __launch_bounds__(CT_THREADS, 1)
             // ------------------------------------------------------ epilogue
             const long long orow = (long long)(b * p.T + t) * p.Hq + g * p.G + h;
             bool have_o = false;
+            float lr = 0.f;                               // the row sum over both halves
             if (nt > 0) {
-                have_o = __all_sync(0xffffffffu, atc::wait(o_full, on & 1, abort_flag));
+                have_o = atc::agree(pair, 64, atc::wait(o_full, on & 1, abort_flag));
                 if (!have_o) { ok = false; break; }
                 tc::fence_after_sync();
+                xch[half * 128 + r] = l;
+                atc::named_sync(pair, 64);
+                lr = half == 0 ? l + xch[128 + r] : xch[r] + l;
             }
-            const float inv = l > 0.f ? 1.f / l : 0.f;
+            const float inv = lr > 0.f ? 1.f / lr : 0.f;
 #pragma unroll
-            for (int c = 0; c < D; c += 16) {
+            for (int c = 0; c < OC; c += 16) {
                 uint32_t o16[16];
                 if (have_o) {
-                    tc::tmem_ld16(tmem + lrow + 128 + c, o16);
+                    tc::tmem_ld16(tmem + lrow + NT_TM_O + half * OC + c, o16);
                     tc::tmem_ld_wait();
                 } else {
 #pragma unroll
                     for (int e = 0; e < 16; ++e) o16[e] = 0u;
                 }
                 if (row_ok) {
-                    float4 *dst = reinterpret_cast<float4 *>(p.out_f32 + orow * D + c);
+                    float4 *dst = reinterpret_cast<float4 *>(p.out_f32 + orow * D + half * OC + c);
 #pragma unroll
                     for (int e = 0; e < 16; e += 4)
                         dst[e / 4] = make_float4(__uint_as_float(o16[e]) * inv, __uint_as_float(o16[e + 1]) * inv,
@@ -389,13 +401,13 @@ __global__ void __launch_bounds__(CT_THREADS, 1)
                 atc::arrive(o_free);
                 ++on;
             }
-            if (row_ok && p.lse) p.lse[orow] = l > 0.f ? (m * p.scale_log2 + log2f(l)) * kLn2 : -INFINITY;
+            if (row_ok && half == 0 && p.lse) p.lse[orow] = lr > 0.f ? (m * p.scale_log2 + log2f(lr)) * kLn2 : -INFINITY;
         }
         if (!ok) fail();
     }
     tc::fence_before_sync();
     __syncthreads();
-    if (warp == 1) tc::tmem_dealloc(tmem, 256);
+    if (warp == 1) tc::tmem_dealloc(tmem, NT_TM_COLS);
 }
 
 }  // namespace sa

@@ -729,12 +729,12 @@ static int launch_tile_t(const TileParams &p, cudaStream_t st) {
 }
 
 // NSA compressed branch on tcgen05 (head dim 128, <= 16 heads per group).
-static int bf16_tensor_map_3d(CUtensorMap *m, const void *base, int d, int hkv, long long rows) {
+static int bf16_tensor_map_3d(CUtensorMap *m, const void *base, int d, int hkv, long long rows, int box_rows) {
     TensorMapEncodeFn enc = tensor_map_encoder();
     if (!enc) return fail(SA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
     cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)hkv, (cuuint64_t)rows};
     cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)hkv * d * 2};
-    cuuint32_t box[3] = {64u, 1u, (cuuint32_t)CT_KT};
+    cuuint32_t box[3] = {64u, 1u, (cuuint32_t)box_rows};
     cuuint32_t es[3] = {1u, 1u, 1u};
     const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -751,11 +751,11 @@ static int launch_nsa_tc(const TileParams &p, unsigned *err, cudaStream_t st) {
     CUtensorMap qm, khm, klm, vm;
     int rc = bf16_tensor_map(&qm, p.q, (long long)p.B * p.T * p.Hq, 128, 16);
     if (rc) return rc;
-    rc = bf16_tensor_map_3d(&khm, p.k, 128, p.Hkv, (long long)p.B * p.Lk);
+    rc = bf16_tensor_map_3d(&khm, p.k, 128, p.Hkv, (long long)p.B * p.Lk, NT_KT);
     if (rc) return rc;
-    rc = bf16_tensor_map_3d(&klm, SRC == TS_CMP ? p.klo : p.k, 128, p.Hkv, (long long)p.B * p.Lk);
+    rc = bf16_tensor_map_3d(&klm, SRC == TS_CMP ? p.klo : p.k, 128, p.Hkv, (long long)p.B * p.Lk, NT_KT);
     if (rc) return rc;
-    rc = bf16_tensor_map_3d(&vm, p.v, 128, p.Hkv, (long long)p.B * p.Lk);
+    rc = bf16_tensor_map_3d(&vm, p.v, 128, p.Hkv, (long long)p.B * p.Lk, NT_KT);
     if (rc) return rc;
     CmpTcParams cp{p, err, (int)items};
     constexpr int smem = CtSmem::ALLOC;
@@ -764,7 +764,7 @@ static int launch_nsa_tc(const TileParams &p, unsigned *err, cudaStream_t st) {
     rc = set_smem(kern, smem);
     if (rc) return rc;
     const int grid = (int)std::min<long long>(items, sm_count());   // persistent: one CTA per SM
-    kern<<<grid, CT_THREADS, smem, st>>>(qm, khm, klm, vm, cp);
+    kern<<<grid, NT_THREADS, smem, st>>>(qm, khm, klm, vm, cp);
     SA_CHECK_LAUNCH("nsa_tc_kernel");
     return SA_OK;
 }
@@ -780,9 +780,9 @@ static int launch_imp_tc(const NsaSelectParams &sp, unsigned *err, cudaStream_t 
     CUtensorMap qm, khm, klm;
     int rc = bf16_tensor_map(&qm, p.q, (long long)p.B * p.T * p.Hq, 128, 16);
     if (rc) return rc;
-    rc = bf16_tensor_map_3d(&khm, p.k, 128, p.Hkv, (long long)p.B * p.Lk);
+    rc = bf16_tensor_map_3d(&khm, p.k, 128, p.Hkv, (long long)p.B * p.Lk, CT_KT);
     if (rc) return rc;
-    rc = bf16_tensor_map_3d(&klm, p.klo, 128, p.Hkv, (long long)p.B * p.Lk);
+    rc = bf16_tensor_map_3d(&klm, p.klo, 128, p.Hkv, (long long)p.B * p.Lk, CT_KT);
     if (rc) return rc;
     ImpTcParams ip{p, sp.lse_cmp, sp.sel_block, sp.sel_topk, sp.n_blocks, sp.sel_idx, err, (int)items};
     const int smem = ItSmem::alloc(sp.n_blocks);
