@@ -35,8 +35,6 @@
 namespace sa {
 
 constexpr int CT_Q = 8;            // queries per item (x 16 heads = 128 rows)
-constexpr int CT_KT = 64;          // compressed keys per tile of the importance kernel
-constexpr int CT_THREADS = 192;    // importance kernel: TMA warp, MMA warp, 4 score warps
 
 // nsa_tc_kernel: 128-key tiles (S = Q.K^T at N = 128), two stages, P in
 // tensor memory as the A operand of P.V, 8 softmax warps.
@@ -427,12 +425,14 @@ namespace sa {
 // top-k blocks by repeated arg-max (ties to the lower block), written in
 // ascending order.  Blocks past the last tile have no visible compressed
 // token and count as 0.
-constexpr int IT_STAGES = 4;
+constexpr int IT_KT = 128;            // compressed keys per tile
+constexpr int IT_STAGES = 2;
+constexpr int IT_THREADS = 320;       // TMA warp, MMA warp, 8 score warps (two per TMEM lane quadrant)
 constexpr int IT_MAX_BLOCKS = 2048;   // candidate blocks per query held in shared memory
 
 struct ItSmem {                       // head dim 128
     static constexpr int Q_BYTES = 128 * 256;
-    static constexpr int KT_BYTES = CT_KT * 256;
+    static constexpr int KT_BYTES = IT_KT * 256;
     static constexpr int STAGE = 2 * KT_BYTES;                 // K_hi | K_lo
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_KV = OFF_Q + Q_BYTES;
@@ -451,7 +451,7 @@ struct ImpTcParams {
     int n_items;
 };
 
-__global__ void __launch_bounds__(CT_THREADS, 1)
+__global__ void __launch_bounds__(IT_THREADS, 1)
     nsa_imp_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap khimap,
                       const __grid_constant__ CUtensorMap klomap, const ImpTcParams ip) {
     constexpr int D = 128;
@@ -467,17 +467,17 @@ __global__ void __launch_bounds__(CT_THREADS, 1)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int cpb = ip.sel_block / p.cmp_stride;              // compressed tokens per block (divides CT_KT)
-    const int nbt = CT_KT / cpb;                              // blocks per tile (<= 16)
+    const int cpb = ip.sel_block / p.cmp_stride;              // compressed tokens per block (4..64, divides 64)
+    const int nbh = (IT_KT / 2) / cpb;                        // blocks per half tile (<= 16)
 
     if (warp == 1) {
-        tc::tmem_alloc(tmem_slot, 128);   // S x2
+        tc::tmem_alloc(tmem_slot, 2 * IT_KT);   // S x2
         tc::tmem_relinquish();
     }
     if (tid == 0) {
         tc::mbar_init(q_full, 1); tc::mbar_init(q_empty, 1);
         for (int i = 0; i < IT_STAGES; ++i) { tc::mbar_init(kv_full + i, 1); tc::mbar_init(kv_empty + i, 1); }
-        for (int i = 0; i < 2; ++i) { tc::mbar_init(s_full + i, 1); tc::mbar_init(s_free + i, 128); }
+        for (int i = 0; i < 2; ++i) { tc::mbar_init(s_full + i, 1); tc::mbar_init(s_free + i, 256); }
         tc::mbar_init(drain, 1);
         *abort_flag = 0;
         tc::mbar_fence_init();
@@ -492,7 +492,7 @@ __global__ void __launch_bounds__(CT_THREADS, 1)
     };
     auto tiles_of = [&](int t0) -> int {
         const int t_last = min(t0 + CT_Q - 1, p.T - 1);
-        return ((int)tile_key_end<TS_CMP>(p, t_last) + CT_KT - 1) / CT_KT;
+        return ((int)tile_key_end<TS_CMP>(p, t_last) + IT_KT - 1) / IT_KT;
     };
 
     if (warp == 0) {
@@ -517,10 +517,10 @@ __global__ void __launch_bounds__(CT_THREADS, 1)
                     if (!atc::wait(kv_empty + st, ((tile / IT_STAGES) & 1) ^ 1, abort_flag)) { ok = false; break; }
                     atc::expect_tx(kv_full + st, L::STAGE);
                     unsigned char *dst = smem + L::OFF_KV + st * L::STAGE;
-                    const int z = b * p.Lk + kt * CT_KT;
+                    const int z = b * p.Lk + kt * IT_KT;
                     for (int h = 0; h < 2; ++h) {
-                        atc::load_3d(dst + h * (CT_KT * 128), &khimap, h * 64, g, z, kv_full + st);
-                        atc::load_3d(dst + L::KT_BYTES + h * (CT_KT * 128), &klomap, h * 64, g, z, kv_full + st);
+                        atc::load_3d(dst + h * (IT_KT * 128), &khimap, h * 64, g, z, kv_full + st);
+                        atc::load_3d(dst + L::KT_BYTES + h * (IT_KT * 128), &klomap, h * 64, g, z, kv_full + st);
                     }
                 }
             }
@@ -534,7 +534,7 @@ __global__ void __launch_bounds__(CT_THREADS, 1)
         __syncwarp();
     } else if (warp == 1) {
         if (lane == 0) {
-            constexpr uint32_t ID_S = tc::make_idesc(1, 1, 128, CT_KT);
+            constexpr uint32_t ID_S = tc::make_idesc(1, 1, 128, IT_KT);
             const uint32_t qa = tc::smem_u32(smem + L::OFF_Q);
             bool ok = true;
             int tile = 0, qn = 0;
@@ -555,10 +555,10 @@ __global__ void __launch_bounds__(CT_THREADS, 1)
                     for (int ks = 0; ks < D / 16; ++ks) {
                         const int h = ks / 4, kk = ks % 4;
                         const uint64_t ad = atc::desc_sw128(qa + h * (128 * 128) + kk * 32, 16, 1024);
-                        const uint64_t bh = atc::desc_sw128(ka + h * (CT_KT * 128) + kk * 32, 16, 1024);
-                        const uint64_t bl = atc::desc_sw128(ka + L::KT_BYTES + h * (CT_KT * 128) + kk * 32, 16, 1024);
-                        tc::mma_bf16(tmem + sb * CT_KT, ad, bh, ID_S, ks > 0 ? 1u : 0u);
-                        tc::mma_bf16(tmem + sb * CT_KT, ad, bl, ID_S, 1u);
+                        const uint64_t bh = atc::desc_sw128(ka + h * (IT_KT * 128) + kk * 32, 16, 1024);
+                        const uint64_t bl = atc::desc_sw128(ka + L::KT_BYTES + h * (IT_KT * 128) + kk * 32, 16, 1024);
+                        tc::mma_bf16(tmem + sb * IT_KT, ad, bh, ID_S, ks > 0 ? 1u : 0u);
+                        tc::mma_bf16(tmem + sb * IT_KT, ad, bl, ID_S, 1u);
                     }
                     tc::mma_commit(kv_empty + st);
                     tc::mma_commit(s_full + sb);
@@ -571,7 +571,10 @@ __global__ void __launch_bounds__(CT_THREADS, 1)
         }
         __syncwarp();
     } else {
-        const int quad = warp & 3;
+        // two warps per TMEM lane quadrant: half 0 scores keys 0-63 of each
+        // tile, half 1 keys 64-127; a block never straddles the halves
+        const int quad = warp & 3, half = (warp - 2) >> 2;
+        constexpr int SC = IT_KT / 2;
         const int r = quad * 32 + lane;                   // row = query w x 16 + head h
         const int w = r >> 4, h = r & 15;
         const uint32_t lrow = (uint32_t)(quad * 32) << 16;
@@ -593,26 +596,19 @@ __global__ void __launch_bounds__(CT_THREADS, 1)
                     break;
                 }
                 tc::fence_after_sync();
-                uint32_t sr[CT_KT];
-                {
-                    uint32_t (&s0)[16] = *reinterpret_cast<uint32_t(*)[16]>(sr);
-                    uint32_t (&s1)[16] = *reinterpret_cast<uint32_t(*)[16]>(sr + 16);
-                    uint32_t (&s2)[16] = *reinterpret_cast<uint32_t(*)[16]>(sr + 32);
-                    uint32_t (&s3)[16] = *reinterpret_cast<uint32_t(*)[16]>(sr + 48);
-                    tc::tmem_ld16(tmem + lrow + sb * CT_KT, s0);
-                    tc::tmem_ld16(tmem + lrow + sb * CT_KT + 16, s1);
-                    tc::tmem_ld16(tmem + lrow + sb * CT_KT + 32, s2);
-                    tc::tmem_ld16(tmem + lrow + sb * CT_KT + 48, s3);
-                }
+                uint32_t sr[SC];
+#pragma unroll
+                for (int c = 0; c < SC; c += 16)
+                    tc::tmem_ld16(tmem + lrow + sb * IT_KT + half * SC + c, *reinterpret_cast<uint32_t(*)[16]>(sr + c));
                 tc::tmem_ld_wait();
                 tc::fence_before_sync();
                 atc::arrive(s_free + sb);
                 // p = 2^(s * scale_log2 - lse_log2): one FFMA and one ex2 per score
-                const int i0 = kt * CT_KT;
-                const bool full = row_ok && i0 + CT_KT <= nv;
-                float pv[CT_KT];
+                const int i0 = kt * IT_KT + half * SC;
+                const bool full = row_ok && i0 + SC <= nv;
+                float pv[SC];
 #pragma unroll
-                for (int k = 0; k < CT_KT; ++k) {
+                for (int k = 0; k < SC; ++k) {
                     const float e = ex2_fast(fmaf(__uint_as_float(sr[k]), p.scale_log2, -ls));
                     pv[k] = (full || (row_ok && i0 + k < nv)) ? e : 0.f;
                 }
@@ -621,10 +617,10 @@ __global__ void __launch_bounds__(CT_THREADS, 1)
                 for (int j = 0; j < 16; ++j) bs[j] = 0.f;
                 if (cpb == 4) {
 #pragma unroll
-                    for (int k = 0; k < CT_KT; ++k) bs[k / 4] += pv[k];
+                    for (int k = 0; k < SC; ++k) bs[k / 4] += pv[k];
                 } else {
 #pragma unroll
-                    for (int k = 0; k < CT_KT; ++k) {
+                    for (int k = 0; k < SC; ++k) {
                         const int j = k / cpb;                   // < 16 since cpb >= 4
 #pragma unroll
                         for (int jj = 0; jj < 16; ++jj)
@@ -632,7 +628,7 @@ __global__ void __launch_bounds__(CT_THREADS, 1)
                     }
                 }
                 // sum over the 16 heads of the query (lane bits 0-3): lane h
-                // ends with the sum of block h of the tile
+                // ends with the sum of block h of this half tile
 #pragma unroll
                 for (int o = 8; o >= 1; o >>= 1) {
                     const bool hi = (lane & o) != 0;
@@ -643,55 +639,57 @@ __global__ void __launch_bounds__(CT_THREADS, 1)
                         bs[j] = mine + __shfl_xor_sync(0xffffffffu, other, o);
                     }
                 }
-                const int blk = kt * nbt + h;
-                if (t <= t_last && h < nbt && blk < nbk) imp_s[w * nbk + blk] = bs[0];
+                const int blk = (kt * 2 + half) * nbh + h;
+                if (t <= t_last && h < nbh && blk < nbk) imp_s[w * nbk + blk] = bs[0];
             }
             // all importances of the item are in shared memory
-            if (!atc::agree(1, 128, ok)) { ok = false; break; }
-            const int covered = min(nt * nbt, nbk);
-            for (int wq = quad; wq < CT_Q; wq += 4) {     // each softmax warp: two queries
+            if (!atc::agree(1, 256, ok)) { ok = false; break; }
+            const int covered = min(nt * 2 * nbh, nbk);
+            {
+                const int wq = warp - 2;                  // each score warp: one query
                 const int tq = t0 + wq;
-                if (tq > t_last) break;
-                float *imp = imp_s + wq * nbk;
-                const int nb_t = min(tq / ip.sel_block + 1, nbk);
-                const int k = min(ip.sel_topk, nb_t);
-                for (int i = covered + lane; i < nb_t; i += 32) imp[i] = 0.f;   // no visible token
-                __syncwarp();
-                int mine = -1;
-                for (int rr = 0; rr < k; ++rr) {
-                    float bv = -1.f;
-                    int bi = 0x7fffffff;
-                    for (int i = lane; i < nb_t; i += 32) {
-                        const float x = imp[i];
-                        if (x > bv) { bv = x; bi = i; }  // lanes scan ascending i: ties keep the lower i
-                    }
-#pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) {
-                        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-                        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-                        if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
-                    }
-                    if (lane == rr) mine = bi < nb_t ? bi : -1;
-                    if (lane == 0 && bi < nb_t) imp[bi] = -1.f;
+                if (tq <= t_last) {
+                    float *imp = imp_s + wq * nbk;
+                    const int nb_t = min(tq / ip.sel_block + 1, nbk);
+                    const int k = min(ip.sel_topk, nb_t);
+                    for (int i = covered + lane; i < nb_t; i += 32) imp[i] = 0.f;   // no visible token
                     __syncwarp();
+                    int mine = -1;
+                    for (int rr = 0; rr < k; ++rr) {
+                        float bv = -1.f;
+                        int bi = 0x7fffffff;
+                        for (int i = lane; i < nb_t; i += 32) {
+                            const float x = imp[i];
+                            if (x > bv) { bv = x; bi = i; }  // lanes scan ascending i: ties keep the lower i
+                        }
+#pragma unroll
+                        for (int o = 16; o > 0; o >>= 1) {
+                            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+                            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+                            if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+                        }
+                        if (lane == rr) mine = bi < nb_t ? bi : -1;
+                        if (lane == 0 && bi < nb_t) imp[bi] = -1.f;
+                        __syncwarp();
+                    }
+                    int rank = 0;
+                    for (int rr = 0; rr < k; ++rr) {
+                        const int other = __shfl_sync(0xffffffffu, mine, rr);
+                        rank += (lane < k && other < mine) ? 1 : 0;
+                    }
+                    int32_t *dst = ip.sel_idx + ((long long)(b * p.T + tq) * p.Hkv + g) * ip.sel_topk;
+                    if (lane < k) dst[rank] = mine;
+                    for (int i = k + lane; i < ip.sel_topk; i += 32) dst[i] = -1;
                 }
-                int rank = 0;
-                for (int rr = 0; rr < k; ++rr) {
-                    const int other = __shfl_sync(0xffffffffu, mine, rr);
-                    rank += (lane < k && other < mine) ? 1 : 0;
-                }
-                int32_t *dst = ip.sel_idx + ((long long)(b * p.T + tq) * p.Hkv + g) * ip.sel_topk;
-                if (lane < k) dst[rank] = mine;
-                for (int i = k + lane; i < ip.sel_topk; i += 32) dst[i] = -1;
             }
             // the next item's tiles overwrite imp_s
-            if (!atc::agree(1, 128, ok)) { ok = false; break; }
+            if (!atc::agree(1, 256, ok)) { ok = false; break; }
         }
         if (!ok) fail();
     }
     tc::fence_before_sync();
     __syncthreads();
-    if (warp == 1) tc::tmem_dealloc(tmem, 128);
+    if (warp == 1) tc::tmem_dealloc(tmem, 2 * IT_KT);
 }
 
 }  // namespace sa

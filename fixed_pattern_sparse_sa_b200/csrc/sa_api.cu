@@ -780,9 +780,9 @@ static int launch_imp_tc(const NsaSelectParams &sp, unsigned *err, cudaStream_t 
     CUtensorMap qm, khm, klm;
     int rc = bf16_tensor_map(&qm, p.q, (long long)p.B * p.T * p.Hq, 128, 16);
     if (rc) return rc;
-    rc = bf16_tensor_map_3d(&khm, p.k, 128, p.Hkv, (long long)p.B * p.Lk, CT_KT);
+    rc = bf16_tensor_map_3d(&khm, p.k, 128, p.Hkv, (long long)p.B * p.Lk, IT_KT);
     if (rc) return rc;
-    rc = bf16_tensor_map_3d(&klm, p.klo, 128, p.Hkv, (long long)p.B * p.Lk, CT_KT);
+    rc = bf16_tensor_map_3d(&klm, p.klo, 128, p.Hkv, (long long)p.B * p.Lk, IT_KT);
     if (rc) return rc;
     ImpTcParams ip{p, sp.lse_cmp, sp.sel_block, sp.sel_topk, sp.n_blocks, sp.sel_idx, err, (int)items};
     const int smem = ItSmem::alloc(sp.n_blocks);
@@ -790,7 +790,7 @@ static int launch_imp_tc(const NsaSelectParams &sp, unsigned *err, cudaStream_t 
     rc = set_smem(nsa_imp_tc_kernel, smem);
     if (rc) return rc;
     const int grid = (int)std::min<long long>(items, sm_count());
-    nsa_imp_tc_kernel<<<grid, CT_THREADS, smem, st>>>(qm, khm, klm, ip);
+    nsa_imp_tc_kernel<<<grid, IT_THREADS, smem, st>>>(qm, khm, klm, ip);
     SA_CHECK_LAUNCH("nsa_imp_tc_kernel");
     return SA_OK;
 }
