@@ -6,9 +6,9 @@
 // its KV group whose source blocks it can see (compressed token i is visible
 // to query t iff i*stride + len - 1 <= t).  All queries of a block read the
 // same compressed keys, so the product is dense:
-//   S[128 x 64]  = Q[128 rows x d] . Kc^T   (rows = 8 queries x 16 heads)
-//   O[128 x d]  += P[128 x 64] . Vc
-// with fp32 accumulators in TMEM (tcgen05.mma kind::f16).  The compressed
+//   S[128 x 128]  = Q[128 rows x d] . Kc^T   (rows = 8 queries x 16 heads)
+//   O[128 x d]   += P[128 x 128] . Vc
+// with fp32 accumulators in TMEM (tcgen05.mma kind::f16), 128 keys per tile.  The compressed
 // keys are means and do not fit bf16 exactly, so they are held as a bf16
 // hi/lo pair and S accumulates both halves (Q.K_hi + Q.K_lo).  The same
 // kernel (SRC = TS_WINDOW) runs the sliding-window branch (NSA page, "Puntos
@@ -16,15 +16,20 @@
 // over 8 consecutive queries is again one contiguous key range.
 //
 // Q, K_hi, K_lo and V tiles arrive by TMA box loads in the 128B-swizzled
-// canonical layouts (K-major for Q, K and P; MN-major for V as the B operand
-// of the second product).  Softmax: thread r owns row r (one query head) of
-// S and O -- the row max, exponentials and row sum need no cross-thread
-// reduction; the running max is raised (and the O row rescaled in TMEM) only
-// when a tile's max exceeds it by more than 2^8.
+// canonical layouts (K-major for Q and K; MN-major for V as the B operand of
+// the second product); P goes from the softmax warps to tensor memory and is
+// read there as the A operand of P.V.  Softmax: row r (one query head) is
+// split between two warps of the same TMEM lane quadrant, 64 scores each;
+// they swap partial row maxima and the final row sums through shared memory.
+// The running max is raised (and the O row rescaled in TMEM) only when a
+// tile's max exceeds it by more than 2^8.  Larger tiles halve the hand-offs
+// between the MMA thread and the softmax warps per key, which is what bounds
+// this kernel.
 //
 // Warps: 0 TMA producer (one thread), 1 MMA issuer (one thread) and TMEM
-// owner, 2-5 softmax + epilogue (TMEM lane quadrants 2, 3, 0, 1).  Every wait
-// is bounded; a timeout sets ERR_TIMEOUT and the CTA drains and exits.
+// owner, 2-9 softmax + epilogue (TMEM lane quadrants 2, 3, 0, 1, twice).
+// Every wait is bounded; a timeout sets ERR_TIMEOUT and the CTA drains and
+// exits.
 #pragma once
 
 #include <cuda.h>
@@ -416,14 +421,15 @@ namespace sa {
 // NSA block importance and top-k selection on tcgen05 (NSA page, "Puntos
 // Clave": the compressed-branch attention scores rank the selection blocks).
 // Persistent CTAs walk the same 8-query items as nsa_tc_kernel over the
-// compressed keys: S = Q.K_hi^T + Q.K_lo^T in TMEM; thread r (one query head)
-// turns its row into probabilities with the compressed branch's LSE and sums
+// compressed keys in 128-key tiles: S = Q.K_hi^T + Q.K_lo^T in TMEM; two
+// warps per TMEM lane quadrant each take one 64-key half of row r (one query
+// head), turn it into probabilities with the compressed branch's LSE and sum
 // them per selection block (sel_block / cmp_stride consecutive compressed
-// tokens); the 16 heads of a query are summed by a transposing butterfly over
-// the 16 lanes that hold them, so lane h ends with block h of the tile.  The
-// importances of an item stay in shared memory; each query then takes its
-// top-k blocks by repeated arg-max (ties to the lower block), written in
-// ascending order.  Blocks past the last tile have no visible compressed
+// tokens, never straddling the halves); the 16 heads of a query are summed by
+// a transposing butterfly over the 16 lanes that hold them, so lane h ends
+// with block h of the half tile.  The importances of an item stay in shared
+// memory; each of the 8 score warps then takes one query's top-k blocks by
+// repeated arg-max (ties to the lower block), written in ascending order.  Blocks past the last tile have no visible compressed
 // token and count as 0.
 constexpr int IT_KT = 128;            // compressed keys per tile
 constexpr int IT_STAGES = 2;
