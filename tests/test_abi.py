@@ -50,6 +50,21 @@ def test_workspace_queries(lib):
     assert lib.sa_indexer_topk_workspace_size(0, 1, 1, 2, 32, 1, 0) == 0
 
 
+def test_indexer_workspace_is_chunked_under_one_gib(lib):
+    # the prefill indexer processes its query rows in chunks sized so one
+    # chunk's sample, thresholds and candidate lists stay within 1 GiB: the
+    # workspace grows with the rows until that cap and stays under it after
+    # (longer rows mean longer lists, so fewer rows per chunk)
+    cap = (1 << 30) * 1.01
+    sizes = [lib.sa_indexer_topk_workspace_size(1, t, t, 16, 64, 2048, 0)
+             for t in (1024, 4096, 16384, 65536, 131072)]
+    assert all(a < b for a, b in zip(sizes[:3], sizes[1:4]))
+    assert max(sizes) <= cap and min(sizes[3:]) > 0.9 * (1 << 30)
+    assert lib.sa_indexer_topk_workspace_size(2, 65536, 65536, 16, 64, 2048, 0) <= cap
+    # decode-shaped calls (one query row per sequence) need far less
+    assert lib.sa_indexer_topk_workspace_size(32, 1, 131072, 16, 64, 2048, 0) < sizes[-1] // 100
+
+
 def test_host_validation_rejects_bad_arguments(lib):
     fake = ctypes.c_void_p(1 << 20)          # never dereferenced: rejected first
     # n_split < 1
