@@ -57,6 +57,18 @@ def test_nsa_d128_full_parity(cuda_ok, T, Hq, Hkv):
     _nsa_check(g, out, lse3, sel, np.arange(T), NSA_CFG)
 
 
+def test_nsa_d128_two_sequences_wide_blocks(cuda_ok):
+    # two sequences in one call (batch offsets of Q, the compressed keys and
+    # the selection output) and 128-token selection blocks (8 compressed
+    # tokens per block instead of 4), window 256
+    cfg = dict(cmp_len=32, cmp_stride=16, sel_block=128, sel_topk=4, window=256)
+    g = inputs.gen_nsa(2, 1200, 32, 2, 128, seed=11)
+    gd = to_dev(g)
+    out, lse3, sel = api.nsa_fwd(gd["q"], gd["k"], gd["v"], gd["gates"], **cfg)
+    api.check_device_status()
+    _nsa_check(g, out, lse3, sel, np.arange(2 * 1200), cfg)
+
+
 def test_nsa_branches_isolated_by_gates(cuda_ok):
     T = 700
     g = inputs.gen_nsa(1, T, 16, 1, 128, seed=3)
