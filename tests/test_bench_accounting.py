@@ -30,3 +30,28 @@ def test_prefill_64k_flops_constant():
     n = 65536
     closed = 2048 * 2049 // 2 + (n - 2048) * 2048
     assert bench.attn_rows(n, 2048, 0) == closed
+
+
+def test_nsa_flops_match_brute_force_counts():
+    # 4*d per (query head, key) summed over the three branches: compressed
+    # tokens visible to t, the last `window` keys, and the keys <= t of the
+    # blocks the oracle's top-k picked (shared by the heads of a KV group)
+    import dataclasses
+    import torch
+    w = dataclasses.replace(inputs.WORKLOADS["nsa64k"], T=300, Hq=8, Hkv=2, d=64)
+    g = inputs.gen_nsa(1, w.T, w.Hq, w.Hkv, w.d, seed=5)
+    ref = oracle.nsa_fwd(g["q"], g["k"], g["v"], g["gates"], cmp_len=w.cmp_len, cmp_stride=w.cmp_stride,
+                         sel_block=w.sel_block, sel_topk=w.sel_topk, window=w.window)
+    sel = ref["sel_idx"]                                       # [T, Hkv, k]
+    keys = 0
+    for t in range(w.T):
+        n_cmp = sum(1 for i in range(w.T) if i * w.cmp_stride + w.cmp_len - 1 <= t)
+        n_win = min(t + 1, w.window)
+        keys += w.Hq * (n_cmp + n_win)
+        for gg in range(w.Hkv):
+            for blk in sel[t, gg]:
+                if blk >= 0:
+                    keys += (w.Hq // w.Hkv) * sum(1 for j in range(blk * w.sel_block, (blk + 1) * w.sel_block)
+                                                  if j <= t)
+    got = bench.nsa_flops(w, torch.from_numpy(sel.reshape(1, w.T, w.Hkv, -1).copy()), torch)
+    assert got == 4.0 * w.d * keys
