@@ -12,9 +12,12 @@ subset of flat query rows (b * T + t); ``None`` means all rows.
 Pins: every function here is checked in ``tests/test_oracle_pins.py`` against
 something other than itself (torch float64 scaled_dot_product_attention,
 numpy einsum / lexsort, brute force on tiny inputs, closed forms and
-invariants).  Two readings have no outside pin, and are marked
-"parity unpinned" below: the NSA block-importance mapping and the NSA
-candidate-block rule (the NSA page gives no formula for either).
+invariants).  Two readings are this build's own (the NSA page gives no
+formula for either): the NSA block-importance mapping and the NSA
+candidate-block rule.  They are pinned to that reading by the hand-derived
+table ``tests/golden/nsa_importance.txt`` (a case where mapping compressed
+tokens by their end position, or taking b*sel_block < t, gives other
+values), not to a published formula.
 """
 from __future__ import annotations
 
@@ -236,12 +239,13 @@ def nsa_fwd(q, k, v, gates, cmp_len, cmp_stride, sel_block, sel_topk, window,
     Returns dict: out [n,Hq,d], o_branch [3,n,Hq,d], lse_branch [n,Hq,3],
     sel_idx [n,Hkv,sel_topk], imp [n,Hkv,n_blocks].
 
-    parity unpinned: the importance mapping (selection block b sums the
-    compressed-branch probabilities of compressed tokens whose start lies in
+    The importance mapping (selection block b sums the compressed-branch
+    probabilities of compressed tokens whose start lies in
     [b*sel_block, (b+1)*sel_block), over the heads of the KV group) and the
     candidate rule (blocks with b*sel_block <= t, none forced) are readings of
-    a page that gives no formula; they are checked only for internal
-    consistency and on planted inputs.
+    a page that gives no formula.  They are pinned to that reading by a
+    hand-derived table (tests/golden/nsa_importance.txt), not to a published
+    formula.
     """
     lib = _load()
     B, T, Hq, d = q.shape

@@ -466,6 +466,49 @@ def test_nsa_planted_block_is_selected():
         assert 2 in r["sel_idx"][t, 0].tolist()
 
 
+def _read_nsa_importance_golden():
+    rows = []
+    with open(os.path.join(GOLDEN, "nsa_importance.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            ts, imp, sel1, sel3 = [x.strip() for x in line.split("|")]
+            t_lo, t_hi = (int(x) for x in ts.split())
+            fr = []
+            for x in imp.split():
+                a, _, b = x.partition("/")
+                fr.append(float(a) / float(b or 1))
+            rows.append((t_lo, t_hi, fr, [int(x) for x in sel1.split()],
+                         [int(x) for x in sel3.split()]))
+    return rows
+
+
+def test_nsa_importance_and_candidates_hand_derived():
+    """Block importance (start-position mapping, summed over the group's
+    heads) and the candidate rule b*sel_block <= t against the hand-derived
+    table in tests/golden/nsa_importance.txt."""
+    T, d = 48, 16
+    q = torch.zeros(1, T, 2, d, dtype=torch.bfloat16)
+    q[0, :, 1, 0] = 16.0
+    k = torch.zeros(1, T, 1, d, dtype=torch.bfloat16)
+    k[0, 12:20, 0, 0] = 16.0
+    v = inputs.gen_nsa(1, T, 2, 1, d, seed=23)["v"]
+    gates = torch.full((1, T, 2, 3), 0.5)
+    cfg = dict(cmp_len=8, cmp_stride=4, sel_block=16, window=16, scale=1.0)
+    r3 = oracle.nsa_fwd(q, k, v, gates, sel_topk=3, **cfg)
+    r1 = oracle.nsa_fwd(q, k, v, gates, sel_topk=1, **cfg)
+    covered = set()
+    for t_lo, t_hi, imp, sel1, sel3 in _read_nsa_importance_golden():
+        for t in range(t_lo, t_hi + 1):
+            covered.add(t)
+            np.testing.assert_allclose(r3["imp"][t, 0], imp, rtol=0, atol=1e-12,
+                                       err_msg=f"importance at t={t}")
+            assert r1["sel_idx"][t, 0].tolist() == sel1, f"top-1 at t={t}"
+            assert r3["sel_idx"][t, 0].tolist() == sel3, f"top-3 at t={t}"
+    assert covered == set(range(T))
+
+
 def test_nsa_override_with_own_selection_is_identity():
     g, r = _nsa_small()
     r2 = oracle.nsa_fwd(g["q"], g["k"], g["v"], g["gates"], sel_override=r["sel_idx"],
