@@ -325,6 +325,12 @@ def main():
     clocks = clk.summary()
     if clocks:
         result["clocks"] = clocks
+    # the ceiling of the L2 -> shared-memory gather that bounds the attention
+    ceil = gather_ceiling(lib, dev, torch)
+    gbs_att = result["roofline"]["gathered_l2_bytes"] / (att_ms / 1e3) / 1e9
+    ceil["sparse_attn_gather_gbs"] = round(gbs_att, 1)
+    ceil["sparse_attn_frac_of_ceiling"] = round(gbs_att / max(ceil["cp_async_gbs"], ceil["bulk_gbs"]), 4)
+    result["gather_ceiling"] = ceil
 
     if not args.no_extra:
         extra = extra_measurements(args, dev, torch, api, lib, inputs, flush, world, peaks)
@@ -396,6 +402,54 @@ def extra_measurements(args, dev, torch, api, lib, inputs, flush, world, peaks):
     res["decode128k"] = dec
     del lays, wsd
     torch.cuda.empty_cache()
+    # --- IndexCache on the 64K prefill: 4 layers, F S S S vs all-F ---
+    w = inputs.WORKLOADS["dsa_prefill64k"]
+    T = args.seq_len or w.T
+    lays = []
+    for i in range(4):
+        gl = inputs.gen_dsa(w.B, T, w.Hq, w.Hkv, w.d, w.Hi, w.di, seed=100 + i)
+        lays.append({k: v.to(dev) for k, v in gl.items()})
+    outs = [torch.empty((w.B, T, w.Hq, w.d), dtype=torch.bfloat16, device=dev) for _ in lays]
+    lses = [torch.empty((w.B, T, w.Hq), dtype=torch.float32, device=dev) for _ in lays]
+    cache = torch.empty((w.B, T, w.topk), dtype=torch.int32, device=dev)
+    wsb = api.dsa_decode_workspace_bytes(w.B, T, T, w.Hq, w.d, w.Hi, w.di, w.topk, 0, 1)
+    wsd = torch.empty(wsb, dtype=torch.uint8, device=dev)
+    pre = {}
+    fl4 = 4 * attn_flops(T, w.topk, 0, w.Hq, w.d)
+    for pattern in ("FSSS", "FFFF"):
+        def pstep(pattern=pattern):
+            api.dsa_decode_layers(pattern, lays, topk=w.topk, outs=outs, lses=lses, idx_cache=cache,
+                                  workspace=wsd)
+        times = timed_steps(pstep, 3, args.warmup, flush, dev, torch)
+        ms = max_over_ranks(sum(times), dev, torch, dist) / len(times)
+        pre[pattern] = {"ms_per_step": round(ms, 3), "tflops": round(world * fl4 / (ms / 1e3) / 1e12, 2)}
+    pre["fsss_speedup_over_ffff"] = round(pre["FFFF"]["ms_per_step"] / pre["FSSS"]["ms_per_step"], 3)
+    pre["note"] = ("4 layers x (indexer top-2048 on F layers + sparse attention), "
+                   f"1 x {T} tokens each; tflops = attention FLOPs of the 4 layers / step time")
+    res[f"indexcache_prefill{T // 1024}k"] = pre
+    del lays, outs, lses, cache, wsd
+    torch.cuda.empty_cache()
+    # --- HySparse2-shaped selection on the 64K prefill: window 128 + top-1024 ---
+    gh = inputs.gen_dsa(w.B, T, w.Hq, w.Hkv, w.d, w.Hi, w.di, seed=200)
+    ghd = {k: v.to(dev) for k, v in gh.items()}
+    hk, hw = 1024, 128
+    hidx = torch.empty((w.B, T, hk + hw), dtype=torch.int32, device=dev)
+    hout = torch.empty((w.B, T, w.Hq, w.d), dtype=torch.bfloat16, device=dev)
+    hws = torch.empty(lib.sa_indexer_topk_workspace_size(w.B, T, T, w.Hi, w.di, hk, hw),
+                      dtype=torch.uint8, device=dev)
+
+    def hstep():
+        api.indexer_topk(ghd["q_idx"], ghd["k_idx"], ghd["w"], hk, hw, out_idx=hidx, workspace=hws)
+        api.sparse_attn_fwd(ghd["q"], ghd["k"], ghd["v"], hidx, out=hout)
+    times = timed_steps(hstep, 3, args.warmup, flush, dev, torch)
+    ms = max_over_ranks(sum(times), dev, torch, dist) / len(times)
+    hfl = attn_flops(T, hk, hw, w.Hq, w.d)
+    res[f"hysparse2_prefill{T // 1024}k"] = {
+        "ms_per_step": round(ms, 3), "tflops": round(world * hfl / (ms / 1e3) / 1e12, 2),
+        "note": "indexer top-1024 + forced window 128, then sparse attention; "
+                f"1 x {T} tokens, 16 q heads / 1 kv head, d=128"}
+    del gh, ghd, hidx, hout, hws
+    torch.cuda.empty_cache()
     # --- NSA 64K ---
     w = inputs.WORKLOADS["nsa64k"]
     if args.nsa_seq_len:
@@ -437,6 +491,51 @@ def extra_measurements(args, dev, torch, api, lib, inputs, flush, world, peaks):
                          "algorithmic_bytes": int(byts),
                          "hbm_frac": round(byts / (ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4)}
     return res
+
+
+def gather_ceiling(lib, dev, torch):
+    """L2 -> shared-memory row-gather ceiling (sa_probe_gather): random
+    256-byte rows from a 32 MiB buffer (the K and V of a 65536-token
+    sequence, L2-resident), no arithmetic.  Sweeps warps / ring depth / CTAs
+    per SM for 16-byte cp.async copies and for bulk (TMA engine) copies;
+    returns the best rate of each, timed with CUDA events."""
+    import ctypes
+    n_rows = (32 << 20) // 256
+    buf = torch.randn(n_rows * 128, device=dev).to(torch.bfloat16)
+    sink = torch.zeros(1, dtype=torch.int32, device=dev)
+    n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
+    st = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+    configs = [(0, w, s, c) for w, s, c in ((4, 4, 2), (8, 4, 1), (8, 4, 2), (12, 4, 1), (16, 4, 1),
+                                            (8, 8, 1), (12, 2, 1), (16, 2, 1), (6, 8, 1), (4, 8, 2))]
+    configs += [(1, w, s, c) for w, s, c in ((4, 8, 1), (8, 4, 1), (8, 6, 1), (4, 8, 2), (2, 16, 1))]
+    best = {0: (0.0, None), 1: (0.0, None)}
+    for mode, warps, stages, cps in configs:
+        if (warps * stages * 4096 + warps * 128) * cps > 227 * 1024:
+            continue
+        iters = max(8, int(4e9 / (n_sm * cps * warps * 4096)))
+        nbytes = n_sm * cps * warps * iters * 4096
+
+        def launch():
+            rc = lib.sa_probe_gather(ctypes.c_void_p(buf.data_ptr()), n_rows, mode, warps, stages, iters,
+                                     cps, ctypes.c_void_p(sink.data_ptr()), st)
+            if rc:
+                raise RuntimeError(lib.sa_last_error_string().decode())
+        launch()
+        evs = []
+        for _ in range(3):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(); launch(); b.record()
+            evs.append((a, b))
+        torch.cuda.synchronize(dev)
+        ms = min(a.elapsed_time(b) for a, b in evs)
+        gbs = nbytes / (ms / 1e3) / 1e9
+        if gbs > best[mode][0]:
+            best[mode] = (gbs, {"warps": warps, "stages": stages, "ctas_per_sm": cps})
+    del buf
+    return {"cp_async_gbs": round(best[0][0], 1), "cp_async_config": best[0][1],
+            "bulk_gbs": round(best[1][0], 1), "bulk_config": best[1][1],
+            "source": "sa_probe_gather: random 256-B rows of a 32 MiB L2-resident buffer into "
+                      "shared memory, no math; best of a sweep, CUDA events"}
 
 
 def nsa_flops(w, sel, torch):

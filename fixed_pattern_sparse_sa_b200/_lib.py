@@ -18,11 +18,16 @@ EXPORTS = (
     "sa_dsa_decode_layers_workspace_size", "sa_dsa_decode_layers",
     "sa_check_device_status", "sa_last_error_string", "sa_status_string",
     "sa_version", "sa_launch_counter",
+    "sa_debug_set_spin_limit", "sa_debug_inject_stall", "sa_debug_exact_recompute_rows",
+    "sa_probe_gather",
 )
 
 SA_OK = 0
 STATUS = {0: "SA_OK", 1: "SA_ERR_INVALID_ARG", 2: "SA_ERR_UNSUPPORTED",
-          3: "SA_ERR_WORKSPACE", 4: "SA_ERR_CUDA", 5: "SA_ERR_DEVICE_ASSERT"}
+          3: "SA_ERR_WORKSPACE", 4: "SA_ERR_CUDA", 5: "SA_ERR_DEVICE_ASSERT",
+          6: "SA_ERR_TIMEOUT"}
+SA_ERR_DEVICE_ASSERT = 5
+SA_ERR_TIMEOUT = 6
 
 
 class SAError(RuntimeError):
@@ -77,6 +82,10 @@ def load() -> ctypes.CDLL:
             "sa_status_string": (ctypes.c_char_p, [I]),
             "sa_version": (I, []),
             "sa_launch_counter": (ctypes.c_uint64, []),
+            "sa_debug_set_spin_limit": (I, [ctypes.c_long]),
+            "sa_debug_inject_stall": (I, [I]),
+            "sa_debug_exact_recompute_rows": (I64, []),
+            "sa_probe_gather": (I, [P, I64, I, I, I, I, I, P, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(lib, name)

@@ -17,7 +17,8 @@ from . import _lib
 from ._lib import SAError, check, sa_dsa_layer, sa_pattern
 
 __all__ = ["indexer_topk", "sparse_attn_fwd", "sparse_attn_fwd_split_static", "lse_combine", "nsa_fwd",
-           "dsa_decode_layers", "check_device_status", "SAError"]
+           "dsa_decode_layers", "check_device_status", "debug_set_spin_limit", "debug_inject_stall",
+           "debug_exact_recompute_rows", "SAError"]
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -51,10 +52,38 @@ def _workspace(nbytes: int, device) -> Optional[torch.Tensor]:
 
 
 def check_device_status(device=None):
-    """Wait for the current stream and raise if a kernel found a bad index."""
+    """Wait for the current stream and raise if a kernel found a bad index
+    (SA_ERR_DEVICE_ASSERT) or stopped on a bounded wait (SA_ERR_TIMEOUT)."""
     lib = _lib.load()
     with torch.cuda.device(device if device is not None else torch.cuda.current_device()):
         check(lib.sa_check_device_status(_stream(None)), "sa_check_device_status")
+
+
+def debug_set_spin_limit(cycles: int, device=None):
+    """sa_debug_set_spin_limit: SM clocks a kernel's progress wait may spin
+    before it reports SA_ERR_TIMEOUT; cycles <= 0 restores the default."""
+    lib = _lib.load()
+    with torch.cuda.device(device if device is not None else torch.cuda.current_device()):
+        check(lib.sa_debug_set_spin_limit(int(cycles)), "sa_debug_set_spin_limit")
+
+
+def debug_inject_stall(on: bool, device=None):
+    """sa_debug_inject_stall: make the NSA tensor-core branch kernels wait on
+    a barrier that nothing completes (a test of the timeout path)."""
+    lib = _lib.load()
+    with torch.cuda.device(device if device is not None else torch.cuda.current_device()):
+        check(lib.sa_debug_inject_stall(1 if on else 0), "sa_debug_inject_stall")
+
+
+def debug_exact_recompute_rows(device=None) -> int:
+    """sa_debug_exact_recompute_rows: rows whose top-k was taken by exact
+    recompute since the last call (synchronizes the device)."""
+    lib = _lib.load()
+    with torch.cuda.device(device if device is not None else torch.cuda.current_device()):
+        n = int(lib.sa_debug_exact_recompute_rows())
+    if n < 0:
+        check(-n, "sa_debug_exact_recompute_rows")
+    return n
 
 
 # ------------------------------------------------------------------ indexer --

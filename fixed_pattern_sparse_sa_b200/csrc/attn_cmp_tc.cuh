@@ -159,7 +159,9 @@ __global__ void __launch_bounds__(NT_THREADS, 1)
         if (lane == 0) {
             bool ok = true;
             int tile = 0, qn = 0;
-            for (int it = blockIdx.x; it < cp.n_items && ok; it += gridDim.x) {
+            // test hook: issue nothing, so the MMA thread's first wait runs out
+            const int n_items = debug_stall() ? 0 : cp.n_items;
+            for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
                 int b, g, t0;
                 ct_item(p, it, b, g, t0);
                 const int nt = tiles_of(t0);

@@ -6,7 +6,7 @@
 // The 16 query heads that share one KV head form the 16 rows of an m16
 // tensor-core tile, so every gathered K/V row feeds 16 heads ("shared KV
 // fetch" of the NSA page, section "Analisis Profundo").  Keys are streamed in
-// chunks of 32 rows through a per-warp multi-stage cp.async pipeline into
+// chunks of 16 rows through a per-warp multi-stage cp.async pipeline into
 // XOR-swizzled shared memory, scored with mma.sync m16n8k16 (bf16 -> fp32),
 // folded into an online softmax and multiplied into V with a second mma.
 #pragma once

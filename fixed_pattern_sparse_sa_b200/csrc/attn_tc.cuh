@@ -42,7 +42,7 @@ constexpr int ATC_THREADS = 288;
 constexpr int ATC_PRODUCERS = 128;          // producer threads (warps 0-3)
 constexpr int ATC_MMA_WARP = 4;
 constexpr int ATC_KEYS = 128;               // keys per tile
-constexpr long long ATC_WAIT = 2000000000LL;   // ~1 s in SM clocks
+constexpr long long ATC_WAIT = 2000000000LL;   // ~1 s in SM clocks: drain waits
 
 struct AtcParams {
     GatherParams g;                         // shapes, list, outputs, scale, error word
@@ -136,13 +136,15 @@ __device__ __forceinline__ int f2ord(float x) {
 }
 __device__ __forceinline__ float ord2f(int i) { return __int_as_float(i >= 0 ? i : i ^ 0x7fffffff); }
 
-// Bounded wait that also gives up once another role has aborted.
+// Bounded progress wait (spin_limit() clocks) that also gives up once
+// another role has aborted.
 __device__ __forceinline__ bool wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
     if (tc::mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
+    const long long limit = spin_limit();
     for (unsigned n = 1;; ++n) {
         if (tc::mbar_try_wait(bar, parity)) return true;
-        if ((n & 15u) == 0u && (*abort_flag || clock64() - t0 > ATC_WAIT)) return false;
+        if ((n & 15u) == 0u && (*abort_flag || clock64() - t0 > limit)) return false;
     }
 }
 

@@ -84,7 +84,7 @@ constexpr int TC_KT = 16;                // 128-key tiles per CTA (amortises the
 // threads of a score CTA: 4 column parts of 4 warps, or 2 parts when the
 // tile has fewer than 64 columns
 __host__ __device__ constexpr int tc_threads(int ncol) { return ncol >= 64 ? 512 : 256; }
-constexpr long long TC_WAIT_CYCLES = 4000000000LL;   // ~2 s: bounded wait on the MMA barrier
+constexpr long long TC_WAIT_CYCLES = 4000000000LL;   // ~2 s: drain wait for the MMA in flight
 enum : int { MODE_SAMPLE = 0, MODE_FILTER = 1 };
 
 __device__ __forceinline__ int tc_core_off(int row, int chunk, int di) {
@@ -327,7 +327,7 @@ __global__ void __launch_bounds__(tc_threads(NCOL), NCOL >= 64 ? 2 : 4) idx_scor
         if (LISTS && warp == 0 && kt > 0) list_base = reserve_lists(kt - 1);
         load_a(kt + TC_AS - 1);                                // buffer of tile kt-1: its MMA is done
         // one thread waits (bounded) and the whole CTA follows its verdict
-        if (tid == 0) *wait_ok = tc::mbar_wait_bounded(bar, kt & 1, TC_WAIT_CYCLES) ? 1 : 0;
+        if (tid == 0) *wait_ok = tc::mbar_wait_bounded(bar, kt & 1, spin_limit()) ? 1 : 0;
         __syncthreads();
         if (*wait_ok == 0) {
             timed_out = true;
@@ -832,6 +832,11 @@ __global__ void __launch_bounds__(SEL_THREADS, 4) idx_threshold_kernel(const Idx
 }
 
 // ----------------------------------------------------------- final select --
+// Rows whose top-k was taken by the exact-recompute path (the candidate list
+// was short or overflowed), counted per device; read and cleared by
+// sa_debug_exact_recompute_rows().
+__device__ unsigned long long g_sa_recompute_rows = 0ull;
+
 // Exact score of one (query, key) on CUDA cores (fallback path).
 template <int DI>
 __device__ __forceinline__ int exact_score(const int8_t *qrow_s, const int *w_s, int Hi, const int8_t *krow) {
@@ -916,6 +921,7 @@ __global__ void __launch_bounds__(NT, NT <= 256 ? 3 : 1) topk_select_kernel(cons
 
     const int cnt = p.cand_cnt[row];
     const bool use_list = cnt >= k_eff && cnt <= p.cand_cap;
+    if (!use_list && tid == 0) atomicAdd(&g_sa_recompute_rows, 1ull);
     const int32_t *cv = p.cand_val + row * p.cand_cap;
     const int32_t *ci = p.cand_idx + row * p.cand_cap;
     const int8_t *kb = p.k + (long long)b * p.L * DI;

@@ -22,6 +22,7 @@
 #include "attn_tile.cuh"
 #include "indexer.cuh"
 #include "nsa_misc.cuh"
+#include "probe_gather.cuh"
 
 using namespace sa;
 
@@ -267,6 +268,7 @@ const char *sa_status_string(int s) {
         case SA_ERR_WORKSPACE: return "SA_ERR_WORKSPACE";
         case SA_ERR_CUDA: return "SA_ERR_CUDA";
         case SA_ERR_DEVICE_ASSERT: return "SA_ERR_DEVICE_ASSERT";
+        case SA_ERR_TIMEOUT: return "SA_ERR_TIMEOUT";
     }
     return "SA_ERR_UNKNOWN";
 }
@@ -284,12 +286,40 @@ int sa_check_device_status(void *stream) {
         const unsigned zero = 0;
         e = cudaMemcpy(ew, &zero, sizeof zero, cudaMemcpyHostToDevice);
         if (e != cudaSuccess) return fail(SA_ERR_CUDA, "clear error word: %s", cudaGetErrorString(e));
-        return fail(SA_ERR_DEVICE_ASSERT, "device error word 0x%x:%s%s%s", word,
+        // a timeout leaves outputs undefined, so it outranks a skipped index
+        return fail((word & ERR_TIMEOUT) ? SA_ERR_TIMEOUT : SA_ERR_DEVICE_ASSERT, "device error word 0x%x:%s%s%s",
+                    word,
                     (word & ERR_BAD_INDEX) ? " index out of range or after the query position;" : "",
                     (word & ERR_BAD_BLOCK) ? " NSA block id outside the sequence;" : "",
-                    (word & ERR_TIMEOUT) ? " a tensor-core barrier wait timed out;" : "");
+                    (word & ERR_TIMEOUT) ? " a bounded barrier wait ran out of its spin limit;" : "");
     }
     return SA_OK;
+}
+
+// ------------------------------------------------------- debug controls --
+int sa_debug_set_spin_limit(long cycles) {
+    const long long v = cycles > 0 ? (long long)cycles : kDefaultSpinCycles;
+    cudaError_t e = cudaMemcpyToSymbol(g_sa_spin_cycles, &v, sizeof v);
+    if (e != cudaSuccess) return fail(SA_ERR_CUDA, "set spin limit: %s", cudaGetErrorString(e));
+    return SA_OK;
+}
+
+int sa_debug_inject_stall(int on) {
+    const int v = on ? 1 : 0;
+    cudaError_t e = cudaMemcpyToSymbol(g_sa_debug_stall, &v, sizeof v);
+    if (e != cudaSuccess) return fail(SA_ERR_CUDA, "inject stall: %s", cudaGetErrorString(e));
+    return SA_OK;
+}
+
+int64_t sa_debug_exact_recompute_rows(void) {
+    unsigned long long n = 0;
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e == cudaSuccess) e = cudaMemcpyFromSymbol(&n, g_sa_recompute_rows, sizeof n);
+    if (e != cudaSuccess) return -(int64_t)fail(SA_ERR_CUDA, "read recompute counter: %s", cudaGetErrorString(e));
+    const unsigned long long zero = 0;
+    e = cudaMemcpyToSymbol(g_sa_recompute_rows, &zero, sizeof zero);
+    if (e != cudaSuccess) return -(int64_t)fail(SA_ERR_CUDA, "clear recompute counter: %s", cudaGetErrorString(e));
+    return (int64_t)n;
 }
 
 // ------------------------------------------------------ sparse attention --
@@ -432,9 +462,17 @@ int sa_sparse_attn_fwd_split_static(const void *q, const void *k, const void *v,
     if (!idx || !out) return fail(SA_ERR_INVALID_ARG, "split_static: idx and out are required");
     if (B <= 0 || Tq < 0 || Hq <= 0 || (d != 64 && d != 128))
         return fail(SA_ERR_INVALID_ARG, "split_static: bad sizes B=%d Tq=%d Hq=%d d=%d", B, Tq, Hq, d);
-    const size_t rows = (size_t)B * Tq * Hq;
-    const size_t o_bytes = round_up((size_t)n_split * rows * d * 4, 256);
-    const size_t need = o_bytes + round_up((size_t)n_split * rows * 4, 256);
+    // n_split * B * Tq * Hq * (d + 1) * 4 with every product checked: a
+    // wrapped size must not pass the limit
+    size_t rows = 0, parts = 0, o_elems = 0;
+    if (__builtin_mul_overflow((size_t)B, (size_t)Tq, &rows) || __builtin_mul_overflow(rows, (size_t)Hq, &rows) ||
+        __builtin_mul_overflow(rows, (size_t)n_split, &parts) || __builtin_mul_overflow(parts, (size_t)d, &o_elems) ||
+        o_elems > kStaticSplitBytes / 4 || parts > kStaticSplitBytes / 4)
+        return fail(SA_ERR_WORKSPACE,
+                    "split_static: n_split * B * Tq * Hq * (d + 1) * 4 exceeds the built-in %zu-byte scratch; "
+                    "use sa_sparse_attn_fwd with a workspace", kStaticSplitBytes);
+    const size_t o_bytes = round_up(o_elems * 4, 256);
+    const size_t need = o_bytes + round_up(parts * 4, 256);
     if (need > kStaticSplitBytes)
         return fail(SA_ERR_WORKSPACE,
                     "split_static: partials need %zu bytes but the built-in scratch holds %zu "
@@ -971,3 +1009,38 @@ int sa_dsa_decode_layers(const char *pattern, int n_layers, const sa_dsa_layer *
     return SA_OK;
 }
 
+
+// -------------------------------------------------- gather ceiling probe --
+template <int MODE, int STAGES>
+static int launch_probe(const ProbeParams &p, int ctas, int smem, cudaStream_t st) {
+    auto kern = probe_gather_kernel<MODE, STAGES>;
+    int rc = set_smem(kern, smem);
+    if (rc) return rc;
+    kern<<<ctas, p.warps * 32, smem, st>>>(p);
+    SA_CHECK_LAUNCH("probe_gather_kernel");
+    return SA_OK;
+}
+
+int sa_probe_gather(const void *buf, int64_t n_rows, int mode, int warps, int stages, int iters,
+                    int ctas_per_sm, unsigned *sink, void *stream) {
+    if (!buf || !sink || !aligned16(buf) || !aligned4(sink) || n_rows < 1 || n_rows > UINT_MAX)
+        return fail(SA_ERR_INVALID_ARG, "probe_gather: buffer/sink/rows");
+    if (mode != 0 && mode != 1) return fail(SA_ERR_INVALID_ARG, "probe_gather: mode %d", mode);
+    if (warps < 1 || warps > 16 || iters < 1 || ctas_per_sm < 1 || ctas_per_sm > 8)
+        return fail(SA_ERR_INVALID_ARG, "probe_gather: warps %d iters %d ctas/SM %d", warps, iters, ctas_per_sm);
+    if (mode == 0 ? !(stages == 2 || stages == 4 || stages == 8) : (stages < 2 || stages > 16))
+        return fail(SA_ERR_INVALID_ARG, "probe_gather: stages %d", stages);
+    const int smem = probe_smem_bytes(warps, stages);
+    if ((long long)smem * ctas_per_sm > 227LL * 1024)
+        return fail(SA_ERR_INVALID_ARG, "probe_gather: %d bytes of shared memory x %d CTAs per SM", smem, ctas_per_sm);
+    unsigned *ew = nullptr;
+    int rc = device_error_word(&ew);
+    if (rc) return rc;
+    ProbeParams p{static_cast<const unsigned char *>(buf), (unsigned)n_rows, warps, stages, iters, sink, ew};
+    const int ctas = sm_count() * ctas_per_sm;
+    cudaStream_t st = as_stream(stream);
+    if (mode == 1) return launch_probe<1, 2>(p, ctas, smem, st);
+    if (stages == 2) return launch_probe<0, 2>(p, ctas, smem, st);
+    if (stages == 4) return launch_probe<0, 4>(p, ctas, smem, st);
+    return launch_probe<0, 8>(p, ctas, smem, st);
+}

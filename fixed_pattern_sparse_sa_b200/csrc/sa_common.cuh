@@ -12,8 +12,27 @@ namespace sa {
 enum : unsigned {
     ERR_BAD_INDEX = 1u,       // index outside [0, L) or after the query position
     ERR_BAD_BLOCK = 2u,       // NSA block id outside the sequence
-    ERR_TIMEOUT = 4u,         // a bounded wait on the tensor-core barrier gave up
+    ERR_TIMEOUT = 4u,         // a bounded progress wait gave up (see spin_limit)
 };
+
+// Spin limit of the kernels' progress waits (a barrier a role waits on before
+// it can go on), in SM clocks; the default is about one second.  Set per
+// device by sa_debug_set_spin_limit().  Drain waits (letting the kernel's own
+// copies and MMAs finish before it frees tensor memory and exits) never use
+// it: they keep a fixed long limit, so a short debug limit cannot release
+// memory that an operation in flight still writes.
+constexpr long long kDefaultSpinCycles = 2000000000LL;
+__device__ long long g_sa_spin_cycles = kDefaultSpinCycles;
+__device__ __forceinline__ long long spin_limit() {
+    return *reinterpret_cast<volatile long long *>(&g_sa_spin_cycles);
+}
+
+// Test hook set by sa_debug_inject_stall(): while nonzero, the NSA
+// tensor-core branch kernels issue none of their loads, so the first
+// progress wait of each CTA (on a barrier that nothing will complete) runs
+// out after the spin limit and reports ERR_TIMEOUT.
+__device__ int g_sa_debug_stall = 0;
+__device__ __forceinline__ bool debug_stall() { return *reinterpret_cast<volatile int *>(&g_sa_debug_stall) != 0; }
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;

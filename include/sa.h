@@ -27,11 +27,15 @@
  *    before anything is enqueued.  Device-side problems found while running
  *    (an index past the query position or outside [0, L)) skip the offending
  *    entry and raise a bit in the library's device error word, reported by
- *    sa_check_device_status().
- *  - Supported on this build: head dim d in {64, 128}; Hq/Hkv in
- *    {1, 2, 4, 8, 16}; indexer heads Hi in {1, 2, 4, 8, 16} with indexer
- *    dim di in {32, 64, 128}; sm_100a only.  Anything else returns
- *    SA_ERR_UNSUPPORTED; there is no CPU fallback.
+ *    sa_check_device_status().  Every wait of a kernel on another part of
+ *    itself is bounded (about one second, see sa_debug_set_spin_limit); one
+ *    that runs out stops the kernel cleanly and is reported as
+ *    SA_ERR_TIMEOUT, after which the call's outputs are undefined.
+ *  - Supported on this build: head dim d in {64, 128}; any Hq that is a
+ *    multiple of Hkv (sa_nsa_fwd: Hq/Hkv <= 16); indexer
+ *    heads Hi in {1, 2, 4, 8, 16} with indexer dim di in {32, 64, 128};
+ *    sm_100a only.  Anything else returns SA_ERR_UNSUPPORTED; there is no
+ *    CPU fallback.
  */
 #ifndef SA_H_
 #define SA_H_
@@ -49,7 +53,8 @@ enum sa_status {
     SA_ERR_UNSUPPORTED = 2,    /* shape or option outside what is built */
     SA_ERR_WORKSPACE = 3,      /* workspace smaller than *_workspace_size() */
     SA_ERR_CUDA = 4,           /* CUDA launch/runtime error (see sa_last_error_string) */
-    SA_ERR_DEVICE_ASSERT = 5   /* device error word was set (bad index found on device) */
+    SA_ERR_DEVICE_ASSERT = 5,  /* device error word was set (bad index found on device) */
+    SA_ERR_TIMEOUT = 6         /* a kernel's bounded barrier wait ran out; outputs undefined */
 };
 
 /* Fixed index set, generated inside the kernel (no index tensor).
@@ -146,8 +151,11 @@ int sa_sparse_attn_fwd(const void *q, const void *k, const void *v,
  * device address with that device current; make that first call before any
  * stream capture.  Every call reuses the same array: calls that may overlap
  * on the GPU (other streams, other host threads) race and must be ordered by
- * the caller.  Nothing needs clearing between calls (every piece writes all
- * of its partial rows before the merge reads them).
+ * the caller.  Nothing needs clearing between calls: on a run that completes,
+ * every piece writes all of its partial rows before the merge reads them.
+ * After a kernel stops early (sa_check_device_status returns SA_ERR_TIMEOUT)
+ * the array may hold an earlier call's partials and out/lse are undefined;
+ * check the device status before using them.
  * ------------------------------------------------------------------------ */
 int sa_sparse_attn_fwd_split_static(const void *q, const void *k, const void *v,
                                     int B, int Tq, int L, int Hq, int Hkv, int d, int64_t q_pos0,
@@ -185,7 +193,7 @@ int sa_lse_combine(const float *part_o, const float *part_lse, int n_split,
  *   out bf16 [B,T,Hq,d]; lse_branches fp32 [B,T,Hq,3] (nullable);
  *   sel_idx_out int32 [B,T,Hkv,sel_topk] ascending, -1 padded (nullable).
  * Requires cmp_stride divides sel_block, cmp_len a multiple of cmp_stride,
- * Hq/Hkv == 16, and sel_topk <= 32.
+ * Hq/Hkv <= 16, and sel_topk <= 32.
  * ------------------------------------------------------------------------ */
 size_t sa_nsa_workspace_size(int B, int T, int Hq, int Hkv, int d, int cmp_len,
                              int cmp_stride, int sel_block, int sel_topk);
@@ -226,8 +234,10 @@ int sa_dsa_decode_layers(const char *pattern, int n_layers, const sa_dsa_layer *
 /* --------------------------------------------------------------------------
  * Status helpers.
  * sa_check_device_status: waits for `stream`, reads and clears the device
- *   error word of the current device; returns SA_ERR_DEVICE_ASSERT if any
- *   kernel since the last check found a bad index, else SA_OK (or SA_ERR_CUDA).
+ *   error word of the current device; returns SA_ERR_TIMEOUT if a kernel
+ *   since the last check stopped because a bounded wait ran out (outputs of
+ *   that call undefined), else SA_ERR_DEVICE_ASSERT if one found a bad index,
+ *   else SA_OK (or SA_ERR_CUDA).
  * sa_last_error_string: message of the last failing call on this host thread.
  * sa_status_string: fixed name of a status code.
  * sa_version: library ABI version (major*100 + minor).
@@ -236,6 +246,42 @@ int sa_dsa_decode_layers(const char *pattern, int n_layers, const sa_dsa_layer *
  *   count the library's launches inside it.
  * ------------------------------------------------------------------------ */
 int sa_check_device_status(void *stream);
+
+/* --------------------------------------------------------------------------
+ * Debug controls (no page has a counterpart; they exist to test the failure
+ * paths).  Each applies to the current device, takes effect for kernels
+ * launched after it returns, and must not be called while library kernels
+ * run on that device.
+ * sa_debug_set_spin_limit: SM clocks a kernel's progress wait may spin
+ *   before it gives up (ERR_TIMEOUT -> SA_ERR_TIMEOUT); cycles <= 0 restores
+ *   the default (2e9, about one second).  Waits that drain a kernel's own
+ *   copies and MMAs before it frees tensor memory keep a fixed long limit.
+ * sa_debug_inject_stall: while on != 0, the NSA tensor-core branch kernels
+ *   (head dim 128) issue none of their loads, so each CTA's first wait is on
+ *   a barrier that nothing completes; it runs out after the spin limit and
+ *   sa_nsa_fwd's outputs are undefined.  Nothing is left in flight.
+ * sa_debug_exact_recompute_rows: synchronizes the current device and returns
+ *   the number of rows whose top-k sa_indexer_topk took by exact recompute
+ *   (the sampled-threshold candidate list was short or overflowed) since the
+ *   last call, then clears the count; a negative value is -status.
+ * ------------------------------------------------------------------------ */
+/* --------------------------------------------------------------------------
+ * Measurement helper (no page has a counterpart): the ceiling of the L2 ->
+ * shared-memory row gather that bounds gathered-KV attention.  Launches
+ * ctas_per_sm CTAs per SM of `warps` warps; each warp gathers `iters` stages
+ * of 16 rows of 256 bytes, picked by a hash from buf (n_rows x 256 bytes,
+ * device memory, 16-byte aligned), into a ring of `stages` shared-memory
+ * stages, with no arithmetic on the data.  mode 0: 16-byte cp.async copies
+ * (stages 2, 4 or 8); mode 1: one bulk copy (TMA engine) per row, stages
+ * 2..16.  Bytes moved = SMs * ctas_per_sm * warps * iters * 4096; the caller
+ * times the launch on `stream`.  sink: one device word the kernel adds to.
+ * ------------------------------------------------------------------------ */
+int sa_probe_gather(const void *buf, int64_t n_rows, int mode, int warps, int stages, int iters,
+                    int ctas_per_sm, unsigned *sink, void *stream);
+
+int sa_debug_set_spin_limit(long cycles);
+int sa_debug_inject_stall(int on);
+int64_t sa_debug_exact_recompute_rows(void);
 const char *sa_last_error_string(void);
 const char *sa_status_string(int status);
 int sa_version(void);

@@ -37,6 +37,7 @@ def test_version_and_status_strings(lib):
     assert lib.sa_version() == 100
     assert lib.sa_status_string(0) == b"SA_OK"
     assert lib.sa_status_string(5) == b"SA_ERR_DEVICE_ASSERT"
+    assert lib.sa_status_string(6) == b"SA_ERR_TIMEOUT"
     assert lib.sa_status_string(99) == b"SA_ERR_UNKNOWN"
 
 
@@ -95,6 +96,19 @@ def test_host_validation_rejects_bad_arguments(lib):
     assert lib.sa_sparse_attn_fwd(fake, fake, fake, 1, 4, 4, 3, 2, 64, 0, fake, 1, 4, None,
                                   None, None, None, 0.1, 1, fake, None, None, None, None, 0,
                                   None) == 1
+
+
+def test_static_split_rejects_wrapping_sizes(lib):
+    # n_split * B * Tq * Hq * (d + 1) * 4 must not wrap around size_t and
+    # slip under the 8 MiB limit: each product is checked before anything is
+    # enqueued (the pointers are never dereferenced)
+    fake = ctypes.c_void_p(1 << 20)
+    big = (1 << 31) - 1
+    for B, Tq, Hq, n_split in [(big, big, big, big), (1, 1 << 20, 1 << 20, 1 << 24), (4, 4, 16, 2 ** 30)]:
+        rc = lib.sa_sparse_attn_fwd_split_static(fake, fake, fake, B, Tq, 1 << 20, Hq, 1, 128, 0,
+                                                 fake, 1, 8, 0.1, n_split, fake, None, None)
+        assert rc == 3, (B, Tq, Hq, n_split)
+        assert b"built-in" in lib.sa_last_error_string()
 
 
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):

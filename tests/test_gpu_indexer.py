@@ -66,7 +66,8 @@ def test_wide_value_range_and_negative_weights(cuda_ok):
 
 
 def test_decode_rows_multi_cta_clusters(cuda_ok):
-    # one query per sequence at the last position: the select uses clusters
+    # one query per sequence at the last position: decode-shaped score pass
+    # (tensor-core mma.sync) and the 1024-thread select (one CTA per row)
     nseq, L = 4, 40000
     g = inputs.gen_decode_layer(nseq, L, 16, 1, 128, 8, 64, layer=0, seed=7)
     gd = to_dev(g)
@@ -126,3 +127,42 @@ def test_prefill64k_sampled_rows_bit_exact(cuda_ok):
     assert np.all(ii[valid] <= np.repeat(np.arange(w.T)[:, None], ii.shape[1], 1)[valid])
     d = np.diff(np.where(valid, ii, np.iinfo(np.int32).max).astype(np.int64), axis=1)
     assert np.all(d[valid[:, 1:]] > 0), "rows must be strictly ascending"
+
+
+def _recompute_case(kind, Tq, L, topk, window, Hi=8, di=64):
+    """Inputs on which the sampled threshold cannot give a usable candidate
+    list.  "overflow": every weight is 0, so every score ties at 0 and every
+    candidate reaches the threshold.  "short": scores are high only on every
+    18th key, so half of the positions sampled with stride 9 are high, the
+    threshold sits at the high score and only ~1/18 of the row (fewer than
+    topk keys) reaches it."""
+    gen = torch.Generator().manual_seed(90 + Tq + window)
+    if kind == "overflow":
+        q = torch.randint(-8, 9, (1, Tq, Hi, di), generator=gen).to(torch.int8)
+        k = torch.randint(-8, 9, (1, L, di), generator=gen).to(torch.int8)
+        w = torch.zeros((1, Tq, Hi), dtype=torch.int32)
+    else:
+        q = torch.ones((1, Tq, Hi, di), dtype=torch.int8)
+        k = torch.ones((1, L, di), dtype=torch.int8)
+        k[0, ::18] = 2
+        w = torch.ones((1, Tq, Hi), dtype=torch.int32)
+    return q, k, w
+
+
+@pytest.mark.parametrize("kind", ["overflow", "short"])
+@pytest.mark.parametrize("Tq", [64, 1])
+@pytest.mark.parametrize("window", [0, 64])
+def test_exact_recompute_when_sample_fails(cuda_ok, kind, Tq, window):
+    # L = 20000 makes the sample strided (stride 9 for these rows): the exact
+    # answer must not depend on it.  Tq = 64 runs the tcgen05 score passes,
+    # Tq = 1 the decode-shaped ones; both end in the select kernel's exact
+    # recompute, which the device counter confirms.
+    L, topk = 20000, 2048
+    q, k, w = _recompute_case(kind, Tq, L, topk, window)
+    api.debug_exact_recompute_rows()                     # clear the counter
+    idx, cnt = api.indexer_topk(q.cuda(), k.cuda(), w.cuda(), topk, window, q_pos0=L - Tq)
+    n_re = api.debug_exact_recompute_rows()
+    ref_idx, ref_cnt = oracle.indexer_topk(q, k, w, topk, window, q_pos0=L - Tq)
+    _check_rows(idx, cnt, ref_idx, ref_cnt)
+    assert n_re == Tq, f"{n_re} of {Tq} rows took the exact-recompute path"
+    api.check_device_status()

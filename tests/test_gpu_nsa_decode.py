@@ -131,3 +131,46 @@ def test_decode128k_full_size(cuda_ok):
         np.testing.assert_array_equal(cache[seqs].cpu().numpy().reshape(ref[-1][0].shape),
                                       ref[-1][0])
     api.check_device_status()
+
+
+def _prefill_layers(T, n_layers, seed):
+    return [inputs.gen_dsa(1, T, 16, 1, 128, 8, 64, seed=seed + 1000 * i) for i in range(n_layers)]
+
+
+@pytest.mark.parametrize("pattern", ["FSSS", "FSFS"])
+def test_indexcache_prefill_full_parity(cuda_ok, pattern):
+    # IndexCache on a prefill (IndexCache page, body: the prefill speed-up
+    # comes from S layers skipping the indexer): every query of a 4096-token
+    # sequence, 4 layers with independent inputs, top-512.  Indices are
+    # bit-exact; every layer's output and LSE match the oracle's layer loop.
+    T, topk = 4096, 512
+    lays = _prefill_layers(T, 4, seed=30)
+    dl = [to_dev(x) for x in lays]
+    outs, lses, cache = api.dsa_decode_layers(pattern, dl, topk=topk)
+    api.check_device_status()
+    ref = oracle.dsa_layers(pattern, lays, topk=topk)
+    for i in range(4):
+        assert_out_close(outs[i], ref[i][1], f"{pattern} layer {i}")
+        assert_lse_close(lses[i], ref[i][2], f"{pattern} layer {i}")
+    np.testing.assert_array_equal(cache.cpu().numpy().reshape(ref[-1][0].shape), ref[-1][0])
+
+
+def test_hysparse2_window128_top1024(cuda_ok):
+    # HySparse2 page ("Xiaomi presenta HySparse2 ...", sections "Mas precision
+    # con menos memoria" and "Que significa ..."): the 128 most recent tokens
+    # are always kept and up to 1024 score-chosen tokens are added.  Every row
+    # of an 8192-token prefill: indices bit-exact, attention within tolerance.
+    T, topk, window = 8192, 1024, 128
+    g = inputs.gen_dsa(1, T, 16, 1, 128, 8, 64, seed=44)
+    gd = to_dev(g)
+    idx, cnt = api.indexer_topk(gd["q_idx"], gd["k_idx"], gd["w"], topk, window)
+    out, lse = api.sparse_attn_fwd(gd["q"], gd["k"], gd["v"], idx)
+    api.check_device_status()
+    ref_idx, ref_cnt = oracle.indexer_topk(g["q_idx"], g["k_idx"], g["w"], topk, window)
+    np.testing.assert_array_equal(cnt.cpu().numpy().reshape(-1), ref_cnt)
+    np.testing.assert_array_equal(idx.cpu().numpy().reshape(ref_idx.shape), ref_idx)
+    np.testing.assert_array_equal(ref_cnt, np.minimum(np.arange(T) + 1, topk + window))
+    rows = sample_rows(T, 512, seed=3)
+    ro, rl = oracle.sparse_attn(g["q"], g["k"], g["v"], ref_idx.reshape(1, T, -1), rows=rows)
+    assert_out_close(out.reshape(-1, 16, 128)[rows], ro)
+    assert_lse_close(lse.reshape(-1, 16)[rows], rl)

@@ -1,0 +1,43 @@
+"""GPU check of the timeout path: a kernel whose bounded wait runs out stops
+cleanly, reports SA_ERR_TIMEOUT through sa_check_device_status, and leaves
+the context usable.  The wait is made to run out without any fault: the
+library's stall hook stops the NSA tensor-core branch kernels from issuing
+their loads, so their first barrier wait is on a barrier that nothing will
+complete, and the spin limit is set to a few milliseconds.  No TMA or MMA is
+in flight when the kernel gives up."""
+import numpy as np
+import pytest
+
+import oracle
+from fixed_pattern_sparse_sa_b200 import _lib, api, inputs
+from fixed_pattern_sparse_sa_b200._lib import SAError
+from _parity import assert_lse_close, assert_out_close, to_dev
+
+pytestmark = pytest.mark.gpu
+
+CFG = dict(cmp_len=32, cmp_stride=16, sel_block=64, sel_topk=8, window=128)
+
+
+def test_stalled_wait_reports_timeout_then_recovers(cuda_ok):
+    g = inputs.gen_nsa(1, 333, 32, 2, 128, seed=77)
+    gd = to_dev(g)
+    api.check_device_status()                       # start from a clean error word
+    try:
+        api.debug_set_spin_limit(20_000_000)          # ~10 ms at 1.9 GHz
+        api.debug_inject_stall(True)
+        api.nsa_fwd(gd["q"], gd["k"], gd["v"], gd["gates"], **CFG)
+        with pytest.raises(SAError) as ei:
+            api.check_device_status()
+        assert ei.value.status == _lib.SA_ERR_TIMEOUT, str(ei.value)
+        assert "spin limit" in str(ei.value)
+    finally:
+        api.debug_inject_stall(False)
+        api.debug_set_spin_limit(0)
+    # the error word was cleared by the check, and the next call is correct
+    out, lse3, sel = api.nsa_fwd(gd["q"], gd["k"], gd["v"], gd["gates"], **CFG)
+    api.check_device_status()
+    rows = np.arange(333)
+    ref = oracle.nsa_fwd(g["q"], g["k"], g["v"], g["gates"], rows=rows,
+                         sel_override=sel.cpu().numpy().reshape(333, 2, -1), **CFG)
+    assert_out_close(out.reshape(-1, 32, 128), ref["out"], "nsa out after timeout")
+    assert_lse_close(lse3.reshape(-1, 32, 3), ref["lse_branch"], "nsa lse after timeout")

@@ -4,14 +4,21 @@ instead of allocating.  It is compared with sa_sparse_attn_fwd (caller-owned
 partial buffers) on two calls in a row with different inputs, so a result
 left over from the first call in the shared array would show up in the
 second.  The file name sorts last so that it also runs after every other
-GPU test in the same process."""
+GPU test in the same process.  The second call of a pair is also checked
+against the CPU oracle directly, on the default gather kernel and, in a
+fresh process, on the tcgen05 gather kernel (SA_ATTN_PATH=tc), which writes
+its partials into the same array."""
 import ctypes
 import math
+import os
+import subprocess
+import sys
 
 import numpy as np
 import pytest
 import torch
 
+import oracle
 from fixed_pattern_sparse_sa_b200 import _lib, api
 from fixed_pattern_sparse_sa_b200._lib import SAError
 from _parity import assert_lse_close, assert_out_close
@@ -88,3 +95,38 @@ def test_static_split_rejects_single_piece(cuda_ok):
     q, k, v, idx = _case(1, 8, 16, 2, 64, 8, 1)
     with pytest.raises(SAError, match="n_split"):
         api.sparse_attn_fwd_split_static(q, k, v, idx, n_split=1)
+
+
+def _two_calls_against_oracle(d, n_split):
+    """Two calls in a row with different inputs; the second is compared with
+    the fp64 oracle, so a partial left in the shared array by the first call
+    (or a fault shared with the workspace path) would show."""
+    B, T, Hq, Hkv, K = 1, 120, 16, 1, 100
+    for seed in (31, 32):
+        q, k, v, idx = _case(B, T, Hq, Hkv, d, K, seed + d)
+        rc, out, lse = _static_call(q, k, v, idx, n_split)
+        assert rc == _lib.SA_OK, _lib.load().sa_last_error_string().decode()
+    torch.cuda.synchronize()
+    ro, rl = oracle.sparse_attn(q.cpu(), k.cpu(), v.cpu(), idx.cpu())
+    assert_out_close(out, ro)
+    assert_lse_close(lse, rl)
+    api.check_device_status()
+
+
+@pytest.mark.parametrize("d,n_split", [(128, 4), (64, 2)])
+def test_static_split_second_call_matches_oracle(cuda_ok, d, n_split):
+    _two_calls_against_oracle(d, n_split)
+
+
+def test_static_split_on_tensor_core_gather_kernel(cuda_ok):
+    # SA_ATTN_PATH is read once per process: run the same check in a fresh
+    # process with the tcgen05 gather kernel selected
+    code = ("import sys; sys.path.insert(0, 'tests')\n"
+            "from test_zz_no_alloc import _two_calls_against_oracle\n"
+            "_two_calls_against_oracle(128, 4)\n"
+            "print('ok')\n")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, SA_ATTN_PATH="tc")
+    r = subprocess.run([sys.executable, "-c", code], cwd=root, env=env, capture_output=True, text=True,
+                       timeout=300)
+    assert r.returncode == 0 and "ok" in r.stdout, r.stderr[-2000:]
