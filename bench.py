@@ -169,6 +169,11 @@ def main():
                          "(default: the 65536-token workload); the JSON line names it")
     ap.add_argument("--nsa-seq-len", type=int, default=0,
                     help="NSA length for profiling captures of a smaller case (default 65536)")
+    ap.add_argument("--workload", default="all",
+                    choices=["all", "decode128k", "indexcache_prefill", "hysparse2_prefill", "nsa64k",
+                             "spatial16k"],
+                    help="run only one of the extra measurements (for profiling captures of a "
+                         "single workload); prints its numbers alone")
     ap.add_argument("--cpu-sample-rows", type=int, default=0,
                     help="oracle rows for the CPU baseline (0 = auto, ~10-30 s)")
     args = ap.parse_args()
@@ -195,6 +200,16 @@ def main():
                                 timeout=timedelta(seconds=120), device_id=dev)
 
     lib = _lib.load()
+    if args.workload != "all":
+        flush_buf = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+        res = extra_measurements(args, dev, torch, api, lib, inputs, lambda: flush_buf.fill_(1.0), world,
+                                 _peaks(), only=args.workload)
+        if rank == 0:
+            print(json.dumps({"workload": args.workload, **res}))
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return 0
     w = inputs.WORKLOADS["dsa_prefill64k"]
     if args.seq_len:
         w = dataclasses.replace(w, T=int(args.seq_len))
@@ -329,6 +344,7 @@ def main():
     ceil = gather_ceiling(lib, dev, torch)
     gbs_att = result["roofline"]["gathered_l2_bytes"] / (att_ms / 1e3) / 1e9
     ceil["sparse_attn_gather_gbs"] = round(gbs_att, 1)
+    # random 256-byte rows are what the attention gathers
     ceil["sparse_attn_frac_of_ceiling"] = round(gbs_att / max(ceil["cp_async_gbs"], ceil["bulk_gbs"]), 4)
     result["gather_ceiling"] = ceil
 
@@ -359,137 +375,143 @@ def _peaks():
                 "source": "of fallback"}
 
 
-def extra_measurements(args, dev, torch, api, lib, inputs, flush, world, peaks):
-    """Decode (IndexCache), NSA and fixed-graph numbers for the same line."""
+def extra_measurements(args, dev, torch, api, lib, inputs, flush, world, peaks, only=None):
+    """Decode (IndexCache), IndexCache prefill, HySparse2-shaped prefill, NSA
+    and fixed-graph numbers for the same line; `only` runs one of them."""
     import torch.distributed as dist
     res = {}
     steps = max(3, args.steps // 2)
     # --- decode 32 x 131072, 4 layers ---
-    w = inputs.WORKLOADS["dsa_decode128k"]
-    lays = [inputs.gen_decode_layer(w.B, w.T, w.Hq, w.Hkv, w.d, w.Hi, w.di, layer=i, seed=0,
-                                    device=dev) for i in range(w.layers)]
-    n_split = 16
-    outs = [torch.empty((w.B, 1, w.Hq, w.d), dtype=torch.bfloat16, device=dev) for _ in lays]
-    lses = [torch.empty((w.B, 1, w.Hq), dtype=torch.float32, device=dev) for _ in lays]
-    cache = torch.empty((w.B, 1, w.topk), dtype=torch.int32, device=dev)
-    wsb = api.dsa_decode_workspace_bytes(w.B, 1, w.T, w.Hq, w.d, w.Hi, w.di, w.topk, 0, n_split)
-    wsd = torch.empty(wsb, dtype=torch.uint8, device=dev)
-    dec = {}
-    for pattern in ("FSSS", "FFFF"):
-        def dstep(pattern=pattern):
-            api.dsa_decode_layers(pattern, lays, topk=w.topk, n_split=n_split, outs=outs,
-                                  lses=lses, idx_cache=cache, workspace=wsd)
-        # capture the 4-layer step in a CUDA graph (launch-bound at this size)
-        s = torch.cuda.Stream(dev)
-        s.wait_stream(torch.cuda.current_stream(dev))
-        with torch.cuda.stream(s):
-            dstep()
-        torch.cuda.current_stream(dev).wait_stream(s)
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
-            dstep()
-        times = timed_steps(graph.replay, steps, args.warmup, flush, dev, torch)
-        ms = max_over_ranks(sum(times), dev, torch, dist) / len(times)
-        n_f = pattern.count("F")
-        bytes_step = n_f * (w.B * w.T * w.di) + w.layers * (w.B * w.topk * 2 * w.d * 2 +
-                                                            w.B * w.Hq * w.d * 2 * 2)
-        dec[pattern] = {"ms_per_step": round(ms, 4),
-                        "tokens_per_s": round(world * w.B / (ms / 1e3), 1),
-                        "algorithmic_bytes": int(bytes_step),
-                        "hbm_frac": round(bytes_step / (ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4)}
-        del graph
-    dec["fsss_over_ffff"] = round(dec["FSSS"]["tokens_per_s"] / dec["FFFF"]["tokens_per_s"], 3)
-    res["decode128k"] = dec
-    del lays, wsd
-    torch.cuda.empty_cache()
+    if only in (None, "decode128k"):
+        w = inputs.WORKLOADS["dsa_decode128k"]
+        lays = [inputs.gen_decode_layer(w.B, w.T, w.Hq, w.Hkv, w.d, w.Hi, w.di, layer=i, seed=0,
+                                        device=dev) for i in range(w.layers)]
+        n_split = 16
+        outs = [torch.empty((w.B, 1, w.Hq, w.d), dtype=torch.bfloat16, device=dev) for _ in lays]
+        lses = [torch.empty((w.B, 1, w.Hq), dtype=torch.float32, device=dev) for _ in lays]
+        cache = torch.empty((w.B, 1, w.topk), dtype=torch.int32, device=dev)
+        wsb = api.dsa_decode_workspace_bytes(w.B, 1, w.T, w.Hq, w.d, w.Hi, w.di, w.topk, 0, n_split)
+        wsd = torch.empty(wsb, dtype=torch.uint8, device=dev)
+        dec = {}
+        for pattern in ("FSSS", "FFFF"):
+            def dstep(pattern=pattern):
+                api.dsa_decode_layers(pattern, lays, topk=w.topk, n_split=n_split, outs=outs,
+                                      lses=lses, idx_cache=cache, workspace=wsd)
+            # capture the 4-layer step in a CUDA graph (launch-bound at this size)
+            s = torch.cuda.Stream(dev)
+            s.wait_stream(torch.cuda.current_stream(dev))
+            with torch.cuda.stream(s):
+                dstep()
+            torch.cuda.current_stream(dev).wait_stream(s)
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                dstep()
+            times = timed_steps(graph.replay, steps, args.warmup, flush, dev, torch)
+            ms = max_over_ranks(sum(times), dev, torch, dist) / len(times)
+            n_f = pattern.count("F")
+            bytes_step = n_f * (w.B * w.T * w.di) + w.layers * (w.B * w.topk * 2 * w.d * 2 +
+                                                                w.B * w.Hq * w.d * 2 * 2)
+            dec[pattern] = {"ms_per_step": round(ms, 4),
+                            "tokens_per_s": round(world * w.B / (ms / 1e3), 1),
+                            "algorithmic_bytes": int(bytes_step),
+                            "hbm_frac": round(bytes_step / (ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4)}
+            del graph
+        dec["fsss_over_ffff"] = round(dec["FSSS"]["tokens_per_s"] / dec["FFFF"]["tokens_per_s"], 3)
+        res["decode128k"] = dec
+        del lays, wsd
+        torch.cuda.empty_cache()
     # --- IndexCache on the 64K prefill: 4 layers, F S S S vs all-F ---
-    w = inputs.WORKLOADS["dsa_prefill64k"]
-    T = args.seq_len or w.T
-    lays = []
-    for i in range(4):
-        gl = inputs.gen_dsa(w.B, T, w.Hq, w.Hkv, w.d, w.Hi, w.di, seed=100 + i)
-        lays.append({k: v.to(dev) for k, v in gl.items()})
-    outs = [torch.empty((w.B, T, w.Hq, w.d), dtype=torch.bfloat16, device=dev) for _ in lays]
-    lses = [torch.empty((w.B, T, w.Hq), dtype=torch.float32, device=dev) for _ in lays]
-    cache = torch.empty((w.B, T, w.topk), dtype=torch.int32, device=dev)
-    wsb = api.dsa_decode_workspace_bytes(w.B, T, T, w.Hq, w.d, w.Hi, w.di, w.topk, 0, 1)
-    wsd = torch.empty(wsb, dtype=torch.uint8, device=dev)
-    pre = {}
-    fl4 = 4 * attn_flops(T, w.topk, 0, w.Hq, w.d)
-    for pattern in ("FSSS", "FFFF"):
-        def pstep(pattern=pattern):
-            api.dsa_decode_layers(pattern, lays, topk=w.topk, outs=outs, lses=lses, idx_cache=cache,
-                                  workspace=wsd)
-        times = timed_steps(pstep, 3, args.warmup, flush, dev, torch)
-        ms = max_over_ranks(sum(times), dev, torch, dist) / len(times)
-        pre[pattern] = {"ms_per_step": round(ms, 3), "tflops": round(world * fl4 / (ms / 1e3) / 1e12, 2)}
-    pre["fsss_speedup_over_ffff"] = round(pre["FFFF"]["ms_per_step"] / pre["FSSS"]["ms_per_step"], 3)
-    pre["note"] = ("4 layers x (indexer top-2048 on F layers + sparse attention), "
-                   f"1 x {T} tokens each; tflops = attention FLOPs of the 4 layers / step time")
-    res[f"indexcache_prefill{T // 1024}k"] = pre
-    del lays, outs, lses, cache, wsd
-    torch.cuda.empty_cache()
+    if only in (None, "indexcache_prefill"):
+        w = inputs.WORKLOADS["dsa_prefill64k"]
+        T = args.seq_len or w.T
+        lays = []
+        for i in range(4):
+            gl = inputs.gen_dsa(w.B, T, w.Hq, w.Hkv, w.d, w.Hi, w.di, seed=100 + i)
+            lays.append({k: v.to(dev) for k, v in gl.items()})
+        outs = [torch.empty((w.B, T, w.Hq, w.d), dtype=torch.bfloat16, device=dev) for _ in lays]
+        lses = [torch.empty((w.B, T, w.Hq), dtype=torch.float32, device=dev) for _ in lays]
+        cache = torch.empty((w.B, T, w.topk), dtype=torch.int32, device=dev)
+        wsb = api.dsa_decode_workspace_bytes(w.B, T, T, w.Hq, w.d, w.Hi, w.di, w.topk, 0, 1)
+        wsd = torch.empty(wsb, dtype=torch.uint8, device=dev)
+        pre = {}
+        fl4 = 4 * attn_flops(T, w.topk, 0, w.Hq, w.d)
+        for pattern in ("FSSS", "FFFF"):
+            def pstep(pattern=pattern):
+                api.dsa_decode_layers(pattern, lays, topk=w.topk, outs=outs, lses=lses, idx_cache=cache,
+                                      workspace=wsd)
+            times = timed_steps(pstep, 3, args.warmup, flush, dev, torch)
+            ms = max_over_ranks(sum(times), dev, torch, dist) / len(times)
+            pre[pattern] = {"ms_per_step": round(ms, 3), "tflops": round(world * fl4 / (ms / 1e3) / 1e12, 2)}
+        pre["fsss_speedup_over_ffff"] = round(pre["FFFF"]["ms_per_step"] / pre["FSSS"]["ms_per_step"], 3)
+        pre["note"] = ("4 layers x (indexer top-2048 on F layers + sparse attention), "
+                       f"1 x {T} tokens each; tflops = attention FLOPs of the 4 layers / step time")
+        res[f"indexcache_prefill{T // 1024}k"] = pre
+        del lays, outs, lses, cache, wsd
+        torch.cuda.empty_cache()
     # --- HySparse2-shaped selection on the 64K prefill: window 128 + top-1024 ---
-    gh = inputs.gen_dsa(w.B, T, w.Hq, w.Hkv, w.d, w.Hi, w.di, seed=200)
-    ghd = {k: v.to(dev) for k, v in gh.items()}
-    hk, hw = 1024, 128
-    hidx = torch.empty((w.B, T, hk + hw), dtype=torch.int32, device=dev)
-    hout = torch.empty((w.B, T, w.Hq, w.d), dtype=torch.bfloat16, device=dev)
-    hws = torch.empty(lib.sa_indexer_topk_workspace_size(w.B, T, T, w.Hi, w.di, hk, hw),
-                      dtype=torch.uint8, device=dev)
+    if only in (None, "hysparse2_prefill"):
+        gh = inputs.gen_dsa(w.B, T, w.Hq, w.Hkv, w.d, w.Hi, w.di, seed=200)
+        ghd = {k: v.to(dev) for k, v in gh.items()}
+        hk, hw = 1024, 128
+        hidx = torch.empty((w.B, T, hk + hw), dtype=torch.int32, device=dev)
+        hout = torch.empty((w.B, T, w.Hq, w.d), dtype=torch.bfloat16, device=dev)
+        hws = torch.empty(lib.sa_indexer_topk_workspace_size(w.B, T, T, w.Hi, w.di, hk, hw),
+                          dtype=torch.uint8, device=dev)
 
-    def hstep():
-        api.indexer_topk(ghd["q_idx"], ghd["k_idx"], ghd["w"], hk, hw, out_idx=hidx, workspace=hws)
-        api.sparse_attn_fwd(ghd["q"], ghd["k"], ghd["v"], hidx, out=hout)
-    times = timed_steps(hstep, 3, args.warmup, flush, dev, torch)
-    ms = max_over_ranks(sum(times), dev, torch, dist) / len(times)
-    hfl = attn_flops(T, hk, hw, w.Hq, w.d)
-    res[f"hysparse2_prefill{T // 1024}k"] = {
-        "ms_per_step": round(ms, 3), "tflops": round(world * hfl / (ms / 1e3) / 1e12, 2),
-        "note": "indexer top-1024 + forced window 128, then sparse attention; "
-                f"1 x {T} tokens, 16 q heads / 1 kv head, d=128"}
-    del gh, ghd, hidx, hout, hws
-    torch.cuda.empty_cache()
+        def hstep():
+            api.indexer_topk(ghd["q_idx"], ghd["k_idx"], ghd["w"], hk, hw, out_idx=hidx, workspace=hws)
+            api.sparse_attn_fwd(ghd["q"], ghd["k"], ghd["v"], hidx, out=hout)
+        times = timed_steps(hstep, 3, args.warmup, flush, dev, torch)
+        ms = max_over_ranks(sum(times), dev, torch, dist) / len(times)
+        hfl = attn_flops(T, hk, hw, w.Hq, w.d)
+        res[f"hysparse2_prefill{T // 1024}k"] = {
+            "ms_per_step": round(ms, 3), "tflops": round(world * hfl / (ms / 1e3) / 1e12, 2),
+            "note": "indexer top-1024 + forced window 128, then sparse attention; "
+                    f"1 x {T} tokens, 16 q heads / 1 kv head, d=128"}
+        del gh, ghd, hidx, hout, hws
+        torch.cuda.empty_cache()
     # --- NSA 64K ---
-    w = inputs.WORKLOADS["nsa64k"]
-    if args.nsa_seq_len:
-        w = dataclasses.replace(w, T=int(args.nsa_seq_len))
-    g = inputs.gen_nsa(w.B, w.T, w.Hq, w.Hkv, w.d, seed=0)
-    gd = {k: v.to(dev) for k, v in g.items()}
-    o = torch.empty((w.B, w.T, w.Hq, w.d), dtype=torch.bfloat16, device=dev)
-    cfg = dict(cmp_len=w.cmp_len, cmp_stride=w.cmp_stride, sel_block=w.sel_block,
-               sel_topk=w.sel_topk, window=w.window)
-    sel_holder = {}
+    if only in (None, "nsa64k"):
+        w = inputs.WORKLOADS["nsa64k"]
+        if args.nsa_seq_len:
+            w = dataclasses.replace(w, T=int(args.nsa_seq_len))
+        g = inputs.gen_nsa(w.B, w.T, w.Hq, w.Hkv, w.d, seed=0)
+        gd = {k: v.to(dev) for k, v in g.items()}
+        o = torch.empty((w.B, w.T, w.Hq, w.d), dtype=torch.bfloat16, device=dev)
+        cfg = dict(cmp_len=w.cmp_len, cmp_stride=w.cmp_stride, sel_block=w.sel_block,
+                   sel_topk=w.sel_topk, window=w.window)
+        sel_holder = {}
 
-    def nstep():
-        _, _, sel = api.nsa_fwd(gd["q"], gd["k"], gd["v"], gd["gates"], out=o, **cfg)
-        sel_holder["sel"] = sel
-    times = timed_steps(nstep, max(2, steps // 2), args.warmup, flush, dev, torch)
-    ms = max_over_ranks(sum(times), dev, torch, dist) / len(times)
-    nsa_fl = nsa_flops(w, sel_holder["sel"], torch)
-    res["nsa64k" if w.T == 65536 else f"nsa{w.T // 1024}k"] = {
-        "ms_per_step": round(ms, 3), "tflops": round(nsa_fl / (ms / 1e3) / 1e12, 2),
-        "algorithmic_flops": nsa_fl,
-        "tensor_frac": round(nsa_fl / (ms / 1e3) / 1e12 / peaks["bf16_tflops"], 4)}
-    del gd, g, o
-    torch.cuda.empty_cache()
+        def nstep():
+            _, _, sel = api.nsa_fwd(gd["q"], gd["k"], gd["v"], gd["gates"], out=o, **cfg)
+            sel_holder["sel"] = sel
+        times = timed_steps(nstep, max(2, steps // 2), args.warmup, flush, dev, torch)
+        ms = max_over_ranks(sum(times), dev, torch, dist) / len(times)
+        nsa_fl = nsa_flops(w, sel_holder["sel"], torch)
+        res["nsa64k" if w.T == 65536 else f"nsa{w.T // 1024}k"] = {
+            "ms_per_step": round(ms, 3), "tflops": round(nsa_fl / (ms / 1e3) / 1e12, 2),
+            "algorithmic_flops": nsa_fl,
+            "tensor_frac": round(nsa_fl / (ms / 1e3) / 1e12 / peaks["bf16_tflops"], 4)}
+        del gd, g, o
+        torch.cuda.empty_cache()
     # --- fixed graph 16K with coordinate bias ---
-    w = inputs.WORKLOADS["spatial16k"]
-    g = inputs.gen_spatial(w.B, w.T, w.Hq, w.d, beta=w.beta, seed=0)
-    gd = {k: v.to(dev) for k, v in g.items()}
-    o = torch.empty((w.B, w.T, w.Hq, w.d), dtype=torch.bfloat16, device=dev)
-    ls = torch.empty((w.B, w.T, w.Hq), dtype=torch.float32, device=dev)
+    if only in (None, "spatial16k"):
+        w = inputs.WORKLOADS["spatial16k"]
+        g = inputs.gen_spatial(w.B, w.T, w.Hq, w.d, beta=w.beta, seed=0)
+        gd = {k: v.to(dev) for k, v in g.items()}
+        o = torch.empty((w.B, w.T, w.Hq, w.d), dtype=torch.bfloat16, device=dev)
+        ls = torch.empty((w.B, w.T, w.Hq), dtype=torch.float32, device=dev)
 
-    def sstep():
-        api.sparse_attn_fwd(gd["q"], gd["k"], gd["v"], pattern=(w.window, w.dilated), cq=gd["cq"],
-                            ck=gd["ck"], beta=gd["beta"], out=o, lse=ls)
-    times = timed_steps(sstep, steps, args.warmup, flush, dev, torch)
-    ms = max_over_ranks(sum(times), dev, torch, dist) / len(times)
-    byts = sum(gd[k].numel() * gd[k].element_size() for k in ("q", "k", "v", "cq", "ck")) + \
-        o.numel() * 2 + ls.numel() * 4
-    res["spatial16k"] = {"ms_per_step": round(ms, 4), "gbs": round(byts / (ms / 1e3) / 1e9, 1),
-                         "algorithmic_bytes": int(byts),
-                         "hbm_frac": round(byts / (ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4)}
+        def sstep():
+            api.sparse_attn_fwd(gd["q"], gd["k"], gd["v"], pattern=(w.window, w.dilated), cq=gd["cq"],
+                                ck=gd["ck"], beta=gd["beta"], out=o, lse=ls)
+        times = timed_steps(sstep, steps, args.warmup, flush, dev, torch)
+        ms = max_over_ranks(sum(times), dev, torch, dist) / len(times)
+        byts = sum(gd[k].numel() * gd[k].element_size() for k in ("q", "k", "v", "cq", "ck")) + \
+            o.numel() * 2 + ls.numel() * 4
+        res["spatial16k"] = {"ms_per_step": round(ms, 4), "gbs": round(byts / (ms / 1e3) / 1e9, 1),
+                             "algorithmic_bytes": int(byts),
+                             "hbm_frac": round(byts / (ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4)}
     return res
 
 
@@ -508,12 +530,14 @@ def gather_ceiling(lib, dev, torch):
     configs = [(0, w, s, c) for w, s, c in ((4, 4, 2), (8, 4, 1), (8, 4, 2), (12, 4, 1), (16, 4, 1),
                                             (8, 8, 1), (12, 2, 1), (16, 2, 1), (6, 8, 1), (4, 8, 2))]
     configs += [(1, w, s, c) for w, s, c in ((4, 8, 1), (8, 4, 1), (8, 6, 1), (4, 8, 2), (2, 16, 1))]
-    best = {0: (0.0, None), 1: (0.0, None)}
+    configs += [(2, w, s, c) for w, s, c in ((4, 3, 1), (2, 6, 1), (6, 2, 1), (3, 4, 1), (1, 12, 1))]
+    best = {0: (0.0, None), 1: (0.0, None), 2: (0.0, None)}
     for mode, warps, stages, cps in configs:
-        if (warps * stages * 4096 + warps * 128) * cps > 227 * 1024:
+        sbytes = 16384 if mode == 2 else 4096
+        if (warps * stages * sbytes + warps * 128) * cps > 227 * 1024:
             continue
-        iters = max(8, int(4e9 / (n_sm * cps * warps * 4096)))
-        nbytes = n_sm * cps * warps * iters * 4096
+        iters = max(8, int(4e9 / (n_sm * cps * warps * sbytes)))
+        nbytes = n_sm * cps * warps * iters * sbytes
 
         def launch():
             rc = lib.sa_probe_gather(ctypes.c_void_p(buf.data_ptr()), n_rows, mode, warps, stages, iters,
@@ -534,6 +558,7 @@ def gather_ceiling(lib, dev, torch):
     del buf
     return {"cp_async_gbs": round(best[0][0], 1), "cp_async_config": best[0][1],
             "bulk_gbs": round(best[1][0], 1), "bulk_config": best[1][1],
+            "bulk_16k_block_gbs": round(best[2][0], 1), "bulk_16k_block_config": best[2][1],
             "source": "sa_probe_gather: random 256-B rows of a 32 MiB L2-resident buffer into "
                       "shared memory, no math; best of a sweep, CUDA events"}
 

@@ -663,6 +663,7 @@ constexpr int SEL_THREADS = 256;
 constexpr int SEL_BITS = 8;
 constexpr int SEL_BINS = 1 << SEL_BITS;
 constexpr int SEL_TIE_CAP = 2048;        // boundary-bin entries resolved from a list
+constexpr int SEL_FINE_BINS = 2 * SEL_TIE_CAP;   // exact-histogram bins (they reuse the tie arrays)
 constexpr int SEL_MAX_N = 768 * 1024;    // candidates per row (two bitmaps of n/8 bytes in shared memory)
 
 // Inclusive block scan (sum) of one int per thread; `tmp` holds 32 ints.
@@ -971,6 +972,35 @@ __global__ void __launch_bounds__(NT, NT <= 256 ? 3 : 1) topk_select_kernel(cons
     block_minmax(gmin, gmax, bcast, for_each);
     const unsigned range = (unsigned)gmax - (unsigned)gmin;
     RadixState st{0u, range == 0 ? 0 : 32 - __clz(range), k_eff, use_list ? cnt : n};
+    if (use_list && range < (unsigned)SEL_FINE_BINS) {
+        // narrow score range: one exact histogram (bin = score - min) gives
+        // the k-th largest score directly; the tie arrays serve as its bins
+        int *fh = reinterpret_cast<int *>(tie_key);
+        for (int i = tid; i < SEL_FINE_BINS; i += NT) fh[i] = 0;
+        __syncthreads();
+        for_each([&](int v, int) { atomicAdd(&fh[(unsigned)v - (unsigned)gmin], 1); });
+        __syncthreads();
+        constexpr int PER = SEL_FINE_BINS / NT;               // bins per thread, highest first
+        int cb[PER], local = 0;
+#pragma unroll
+        for (int u = 0; u < PER; ++u) { cb[u] = fh[SEL_FINE_BINS - 1 - (tid * PER + u)]; local += cb[u]; }
+        const int incl = block_incl_scan(local, scan_tmp);
+        int above = incl - local;
+#pragma unroll
+        for (int u = 0; u < PER; ++u) {
+            if (above < k_eff && above + cb[u] >= k_eff) {
+                bcast[2] = SEL_FINE_BINS - 1 - (tid * PER + u);
+                bcast[3] = above;
+            }
+            above += cb[u];
+        }
+        __syncthreads();
+        st.lo_key = (unsigned)bcast[2];
+        st.width = 0;
+        st.k_rem = k_eff - bcast[3];
+        st.bin_count = fh[bcast[2]];
+        __syncthreads();
+    }
     while (st.width > 0 && (st.width > SEL_BITS || st.bin_count > SEL_TIE_CAP))
         radix_refine<NT>(st, gmin, hist, scan_tmp, bcast, for_each);
 

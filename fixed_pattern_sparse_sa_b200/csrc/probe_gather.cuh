@@ -12,7 +12,10 @@
 //   mode 0: 16-byte cp.async copies (a warp moves two 256-byte rows per
 //           instruction), commit groups per stage;
 //   mode 1: bulk copies (cp.async.bulk, the TMA engine), one 256-byte row per
-//           copy, completion on one mbarrier per stage.
+//           copy, completion on one mbarrier per stage;
+//   mode 2: bulk copies of whole 16 KB blocks (64 consecutive 256-byte rows,
+//           the K or V tile of one NSA selection block) at random block
+//           offsets, one copy per stage.
 #pragma once
 
 #include "sa_common.cuh"
@@ -22,6 +25,11 @@ namespace sa {
 
 constexpr int PROBE_ROW = 256;            // bytes per gathered row
 constexpr int PROBE_ROWS_PER_STAGE = 16;  // rows per stage (a 16-key K or V chunk)
+constexpr int PROBE_BLOCK = 16384;        // bytes per copy in mode 2
+template <int MODE>
+__host__ __device__ constexpr int probe_stage_bytes() {
+    return MODE == 2 ? PROBE_BLOCK : PROBE_ROWS_PER_STAGE * PROBE_ROW;
+}
 
 struct ProbeParams {
     const unsigned char *buf;   // n_rows x 256 bytes
@@ -44,7 +52,7 @@ __global__ void __launch_bounds__(512) probe_gather_kernel(const ProbeParams p) 
     extern __shared__ __align__(1024) unsigned char smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (warp >= p.warps) return;
-    constexpr int SB = PROBE_ROWS_PER_STAGE * PROBE_ROW;
+    constexpr int SB = probe_stage_bytes<MODE>();
     unsigned char *ring = smem + (size_t)warp * p.stages * SB;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + (size_t)p.warps * p.stages * SB) + warp * 16;
     const unsigned seed = (blockIdx.x * 64u + warp) * 0x9e3779b9u;
@@ -88,12 +96,15 @@ __global__ void __launch_bounds__(512) probe_gather_kernel(const ProbeParams p) 
                 asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(tc::smem_u32(bars + s)),
                              "r"(SB)
                              : "memory");
-                for (int r = 0; r < PROBE_ROWS_PER_STAGE; ++r) {
-                    const unsigned row = row_of(it, r);
+                constexpr int NCOPY = MODE == 2 ? 1 : PROBE_ROWS_PER_STAGE;
+                constexpr int CB = MODE == 2 ? PROBE_BLOCK : PROBE_ROW;
+                const unsigned n_units = MODE == 2 ? p.n_rows / (PROBE_BLOCK / PROBE_ROW) : p.n_rows;
+                for (int r = 0; r < NCOPY; ++r) {
+                    const unsigned unit = probe_hash(seed + (unsigned)it * PROBE_ROWS_PER_STAGE + (unsigned)r) % n_units;
                     asm volatile(
                         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
-                            tc::smem_u32(dst + r * PROBE_ROW)),
-                        "l"(p.buf + (size_t)row * PROBE_ROW), "r"(PROBE_ROW), "r"(tc::smem_u32(bars + s))
+                            tc::smem_u32(dst + r * CB)),
+                        "l"(p.buf + (size_t)unit * CB), "r"(CB), "r"(tc::smem_u32(bars + s))
                         : "memory");
                 }
                 ++issued;
@@ -112,8 +123,8 @@ __global__ void __launch_bounds__(512) probe_gather_kernel(const ProbeParams p) 
     }
 }
 
-__host__ __device__ constexpr int probe_smem_bytes(int warps, int stages) {
-    return warps * stages * PROBE_ROWS_PER_STAGE * PROBE_ROW + warps * 16 * 8;
+__host__ __device__ constexpr int probe_smem_bytes(int warps, int stages, int mode) {
+    return warps * stages * (mode == 2 ? PROBE_BLOCK : PROBE_ROWS_PER_STAGE * PROBE_ROW) + warps * 16 * 8;
 }
 
 }  // namespace sa

@@ -21,6 +21,7 @@
 #include "attn_cmp_tc.cuh"
 #include "attn_tile.cuh"
 #include "indexer.cuh"
+#include "indexer_filter.cuh"
 #include "nsa_misc.cuh"
 #include "probe_gather.cuh"
 
@@ -539,14 +540,27 @@ static int indexer_chunk_rows(int B, int Tq, int nq_block, int m_cap, int cap) {
 }
 
 struct IdxLayout {
-    bool decode;
+    bool decode, filter_tc;
     int nq, m_cap, cap, rt;
-    size_t sample_off, tau_off, cnt_off, val_off, idx_off, total;
+    size_t sample_off, tau_off, cnt_off, val_off, idx_off, qf_off, wf_off, total;
 };
 
-static IdxLayout indexer_layout(int B, int Tq, int L, int Hi, int topk) {
+// The persistent filter kernel (indexer_filter.cuh) serves prefill-shaped
+// calls with 2..16 indexer heads; SA_IDX_FILTER=tiles selects the earlier
+// per-tile kernel instead (kept for comparison).
+static bool filter_tc_allowed() {
+    static int v = -1;
+    if (v < 0) {
+        const char *e = std::getenv("SA_IDX_FILTER");
+        v = (e && std::strcmp(e, "tiles") == 0) ? 0 : 1;
+    }
+    return v != 0;
+}
+
+static IdxLayout indexer_layout(int B, int Tq, int L, int Hi, int di, int topk) {
     IdxLayout l{};
     l.decode = indexer_decode_path(Tq, Hi);
+    l.filter_tc = !l.decode && Hi >= 2 && filter_tc_allowed();
     l.nq = l.decode ? 1 : 256 / Hi;
     l.m_cap = indexer_m_cap(l.nq);
     l.cap = indexer_cand_cap(topk, L);
@@ -558,14 +572,18 @@ static IdxLayout indexer_layout(int B, int Tq, int L, int Hi, int topk) {
     l.cnt_off = off; off += round_up(rows * 4, 256);
     l.val_off = off; off += round_up(rows * l.cap * 4, 256);
     l.idx_off = off; off += round_up(rows * l.cap * 4, 256);
+    // weights folded into the query operand (persistent filter kernel only)
+    l.qf_off = off; off += l.filter_tc ? round_up((size_t)B * Tq * Hi * di, 256) : 0;
+    l.wf_off = off; off += l.filter_tc ? round_up((size_t)B * Tq * Hi * 4, 256) : 0;
     l.total = off;
     return l;
 }
 
 size_t sa_indexer_topk_workspace_size(int B, int Tq, int L, int Hi, int di, int topk, int window) {
-    (void)di; (void)window;
+    (void)window;
     if (B <= 0 || Tq <= 0 || L <= 0 || topk < 0 || !(Hi == 1 || Hi == 2 || Hi == 4 || Hi == 8 || Hi == 16)) return 0;
-    return indexer_layout(B, Tq, L, Hi, topk).total;
+    if (!(di == 32 || di == 64 || di == 128)) return 0;
+    return indexer_layout(B, Tq, L, Hi, di, topk).total;
 }
 
 template <int HI, int DI, int NCOL, int MODE>
@@ -625,6 +643,67 @@ static int launch_score(const IdxParams &p, bool decode, long long n_keys_max, c
     return fail(SA_ERR_UNSUPPORTED, "indexer heads %d", p.Hi);
 }
 
+// int8 2-D tensor map over `rows` rows of `di` bytes; box = one whole row
+// (di bytes, swizzled with the matching 32B/64B/128B pattern) x box_rows rows.
+static int i8_tensor_map(CUtensorMap *m, const void *base, long long rows, int di, int box_rows) {
+    TensorMapEncodeFn enc = tensor_map_encoder();
+    if (!enc) return fail(SA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+    cuuint64_t dims[2] = {(cuuint64_t)di, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)di};
+    cuuint32_t box[2] = {(cuuint32_t)di, (cuuint32_t)box_rows};
+    cuuint32_t es[2] = {1u, 1u};
+    const CUtensorMapSwizzle sw = di == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                  : di == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+    const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, es,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(SA_ERR_CUDA, "cuTensorMapEncodeTiled(int8) failed (%d)", (int)r);
+    return SA_OK;
+}
+
+template <int HI, int DI>
+static int launch_filter_tc_t(const IdxParams &p, const int8_t *qf, const int32_t *wf, cudaStream_t st) {
+    constexpr int NQ = FT_NCOL / HI;
+    const long long n_units = (long long)p.B * ((p.Rt + NQ - 1) / NQ);
+    if (n_units == 0) return SA_OK;
+    CUtensorMap am, bm;
+    int rc = i8_tensor_map(&am, p.k, (long long)p.B * p.L, DI, 128);
+    if (rc) return rc;
+    rc = i8_tensor_map(&bm, qf, (long long)p.B * p.Tq * HI, DI, FT_NCOL);
+    if (rc) return rc;
+    FtParams fp{p, wf, (int)n_units};
+    constexpr int smem = FtSmem<DI>::ALLOC;
+    static_assert(smem <= 227 * 1024, "shared memory");
+    auto kern = idx_filter_tc_kernel<HI, DI>;
+    rc = set_smem(kern, smem);
+    if (rc) return rc;
+    const int grid = (int)std::min<long long>(n_units, sm_count());
+    kern<<<grid, FT_THREADS, smem, st>>>(am, bm, fp);
+    SA_CHECK_LAUNCH("idx_filter_tc_kernel");
+    return SA_OK;
+}
+
+template <int DI>
+static int launch_filter_tc_d(const IdxParams &p, const int8_t *qf, const int32_t *wf, cudaStream_t st) {
+    switch (p.Hi) {
+        case 2: return launch_filter_tc_t<2, DI>(p, qf, wf, st);
+        case 4: return launch_filter_tc_t<4, DI>(p, qf, wf, st);
+        case 8: return launch_filter_tc_t<8, DI>(p, qf, wf, st);
+        case 16: return launch_filter_tc_t<16, DI>(p, qf, wf, st);
+    }
+    return fail(SA_ERR_UNSUPPORTED, "filter: indexer heads %d", p.Hi);
+}
+
+static int launch_fold(const IdxParams &p, int8_t *qf, int32_t *wf, cudaStream_t st) {
+    const long long n = (long long)p.B * p.Tq * p.Hi;
+    const unsigned blocks = (unsigned)((n + 255) / 256);
+    if (p.di == 32) idx_fold_kernel<32><<<blocks, 256, 0, st>>>(p.q, p.w, qf, wf, n);
+    else if (p.di == 64) idx_fold_kernel<64><<<blocks, 256, 0, st>>>(p.q, p.w, qf, wf, n);
+    else idx_fold_kernel<128><<<blocks, 256, 0, st>>>(p.q, p.w, qf, wf, n);
+    SA_CHECK_LAUNCH("idx_fold_kernel");
+    return SA_OK;
+}
+
 // One CTA per row; when there are few rows (decode) a row gets 1024 threads.
 template <int DI, int NT>
 static int launch_select_nt(const IdxParams &p, int words, cudaStream_t st) {
@@ -661,7 +740,7 @@ int sa_indexer_topk(const int8_t *q_idx, const int8_t *k_idx, const int32_t *w, 
     const long long n_max_all = std::max(0LL, (long long)(window > 0 ? q_pos0 + Tq - window : q_pos0 + Tq));
     if (n_max_all > SEL_MAX_N)
         return fail(SA_ERR_UNSUPPORTED, "indexer_topk: %lld candidates per query exceed %d", n_max_all, SEL_MAX_N);
-    const IdxLayout lay = indexer_layout(B, Tq, L, Hi, topk);
+    const IdxLayout lay = indexer_layout(B, Tq, L, Hi, di, topk);
     if (!workspace || workspace_bytes < lay.total)
         return fail(SA_ERR_WORKSPACE, "indexer_topk: workspace %zu < %zu", workspace_bytes, lay.total);
     if (!aligned16(workspace)) return fail(SA_ERR_INVALID_ARG, "indexer_topk: workspace alignment");
@@ -682,6 +761,13 @@ int sa_indexer_topk(const int8_t *q_idx, const int8_t *k_idx, const int32_t *w, 
     p.cand_val = reinterpret_cast<int32_t *>(ws + lay.val_off);
     p.cand_idx = reinterpret_cast<int32_t *>(ws + lay.idx_off);
     p.out_idx = out_idx; p.out_count = out_count; p.err = ew;
+    int8_t *qf = reinterpret_cast<int8_t *>(ws + lay.qf_off);
+    int32_t *wf = reinterpret_cast<int32_t *>(ws + lay.wf_off);
+    const bool filter_tc = lay.filter_tc && (long long)B * L < INT_MAX && (long long)B * Tq * Hi < INT_MAX;
+    if (filter_tc) {
+        rc = launch_fold(p, qf, wf, st);
+        if (rc) return rc;
+    }
     for (int t0 = 0; t0 < Tq; t0 += lay.rt) {
         const int rows = std::min(lay.rt, Tq - t0);
         p.t0 = t0; p.Rt = rows;
@@ -694,7 +780,11 @@ int sa_indexer_topk(const int8_t *q_idx, const int8_t *k_idx, const int32_t *w, 
             if (rc) return rc;
             idx_threshold_kernel<<<dim3(1u, (unsigned)rows, (unsigned)B), SEL_THREADS, 0, st>>>(p);
             SA_CHECK_LAUNCH("idx_threshold_kernel");
-            rc = launch_score<MODE_FILTER>(p, lay.decode, ncand, st);
+            if (filter_tc)
+                rc = di == 32 ? launch_filter_tc_d<32>(p, qf, wf, st)
+                              : di == 64 ? launch_filter_tc_d<64>(p, qf, wf, st) : launch_filter_tc_d<128>(p, qf, wf, st);
+            else
+                rc = launch_score<MODE_FILTER>(p, lay.decode, ncand, st);
             if (rc) return rc;
         }
         const int words = (int)((std::max(ncand, 1LL) + 31) / 32);
@@ -1025,12 +1115,13 @@ int sa_probe_gather(const void *buf, int64_t n_rows, int mode, int warps, int st
                     int ctas_per_sm, unsigned *sink, void *stream) {
     if (!buf || !sink || !aligned16(buf) || !aligned4(sink) || n_rows < 1 || n_rows > UINT_MAX)
         return fail(SA_ERR_INVALID_ARG, "probe_gather: buffer/sink/rows");
-    if (mode != 0 && mode != 1) return fail(SA_ERR_INVALID_ARG, "probe_gather: mode %d", mode);
+    if (mode < 0 || mode > 2) return fail(SA_ERR_INVALID_ARG, "probe_gather: mode %d", mode);
+    if (mode == 2 && n_rows < PROBE_BLOCK / PROBE_ROW) return fail(SA_ERR_INVALID_ARG, "probe_gather: rows < one block");
     if (warps < 1 || warps > 16 || iters < 1 || ctas_per_sm < 1 || ctas_per_sm > 8)
         return fail(SA_ERR_INVALID_ARG, "probe_gather: warps %d iters %d ctas/SM %d", warps, iters, ctas_per_sm);
     if (mode == 0 ? !(stages == 2 || stages == 4 || stages == 8) : (stages < 2 || stages > 16))
         return fail(SA_ERR_INVALID_ARG, "probe_gather: stages %d", stages);
-    const int smem = probe_smem_bytes(warps, stages);
+    const int smem = probe_smem_bytes(warps, stages, mode);
     if ((long long)smem * ctas_per_sm > 227LL * 1024)
         return fail(SA_ERR_INVALID_ARG, "probe_gather: %d bytes of shared memory x %d CTAs per SM", smem, ctas_per_sm);
     unsigned *ew = nullptr;
@@ -1040,6 +1131,7 @@ int sa_probe_gather(const void *buf, int64_t n_rows, int mode, int warps, int st
     const int ctas = sm_count() * ctas_per_sm;
     cudaStream_t st = as_stream(stream);
     if (mode == 1) return launch_probe<1, 2>(p, ctas, smem, st);
+    if (mode == 2) return launch_probe<2, 2>(p, ctas, smem, st);
     if (stages == 2) return launch_probe<0, 2>(p, ctas, smem, st);
     if (stages == 4) return launch_probe<0, 4>(p, ctas, smem, st);
     return launch_probe<0, 8>(p, ctas, smem, st);

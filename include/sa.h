@@ -273,8 +273,11 @@ int sa_check_device_status(void *stream);
  * device memory, 16-byte aligned), into a ring of `stages` shared-memory
  * stages, with no arithmetic on the data.  mode 0: 16-byte cp.async copies
  * (stages 2, 4 or 8); mode 1: one bulk copy (TMA engine) per row, stages
- * 2..16.  Bytes moved = SMs * ctas_per_sm * warps * iters * 4096; the caller
- * times the launch on `stream`.  sink: one device word the kernel adds to.
+ * 2..16; mode 2: stages of one 16 KB bulk copy of 64 consecutive rows at a
+ * random 64-row block (the K or V of one NSA selection block).  Bytes moved =
+ * SMs * ctas_per_sm * warps * iters * S with S = 4096 (modes 0, 1) or 16384
+ * (mode 2); the caller times the launch on `stream`.  sink: one device word
+ * the kernel adds to.
  * ------------------------------------------------------------------------ */
 int sa_probe_gather(const void *buf, int64_t n_rows, int mode, int warps, int stages, int iters,
                     int ctas_per_sm, unsigned *sink, void *stream);

@@ -55,13 +55,17 @@ def test_indexer_workspace_is_chunked_under_one_gib(lib):
     # the prefill indexer processes its query rows in chunks sized so one
     # chunk's sample, thresholds and candidate lists stay within 1 GiB: the
     # workspace grows with the rows until that cap and stays under it after
-    # (longer rows mean longer lists, so fewer rows per chunk)
-    cap = (1 << 30) * 1.01
+    # (longer rows mean longer lists, so fewer rows per chunk).  Beside the
+    # chunk, prefill-shaped calls keep one copy of the query operand with the
+    # weights folded in: B*Tq*Hi*di bytes plus B*Tq*Hi int32 weights.
+    def cap(B, T, Hi=16, di=64):
+        return (1 << 30) * 1.01 + B * T * Hi * (di + 4) + 1024
     sizes = [lib.sa_indexer_topk_workspace_size(1, t, t, 16, 64, 2048, 0)
              for t in (1024, 4096, 16384, 65536, 131072)]
     assert all(a < b for a, b in zip(sizes[:3], sizes[1:4]))
-    assert max(sizes) <= cap and min(sizes[3:]) > 0.9 * (1 << 30)
-    assert lib.sa_indexer_topk_workspace_size(2, 65536, 65536, 16, 64, 2048, 0) <= cap
+    assert all(s <= cap(1, t) for s, t in zip(sizes, (1024, 4096, 16384, 65536, 131072)))
+    assert min(sizes[3:]) > 0.9 * (1 << 30)
+    assert lib.sa_indexer_topk_workspace_size(2, 65536, 65536, 16, 64, 2048, 0) <= cap(2, 65536)
     # decode-shaped calls (one query row per sequence) need far less
     assert lib.sa_indexer_topk_workspace_size(32, 1, 131072, 16, 64, 2048, 0) < sizes[-1] // 100
 
