@@ -63,11 +63,12 @@ def _load():
             lib.oracle_sparse_attn.argtypes = [P, P, P, I, I, I, I, I, I, I, P, I, I,
                                                P, P, P, D, P, I, P, P, P, P]
             lib.oracle_lse_combine.argtypes = [P, P, I, I, I, P, P]
+            lib.oracle_sparse_attn_bwd.argtypes = [P, P, P, P, I, I, I, I, I, I, I, P, I, I, D, P, P, P]
             lib.oracle_nsa_compress.argtypes = [P, P, I, I, I, I, I, I, P, P]
             lib.oracle_nsa_fwd.argtypes = [P, P, P, P, I, I, I, I, I, I, I, I, I, I, D,
                                            P, I, P, P, P, P, P, P]
             for name in ("oracle_indexer_scores", "oracle_indexer_topk",
-                         "oracle_sparse_attn", "oracle_lse_combine",
+                         "oracle_sparse_attn", "oracle_sparse_attn_bwd", "oracle_lse_combine",
                          "oracle_nsa_compress", "oracle_nsa_fwd"):
                 getattr(lib, name).restype = ctypes.c_int
             _lib = lib
@@ -199,6 +200,33 @@ def sparse_attn(q, k, v, idx, scale=None, q_pos0=0, cq=None, ck=None, beta=None,
     if want_stats:
         return out, lse, psum, maxj
     return out, lse
+
+
+def sparse_attn_bwd(q, k, v, dout, idx, scale=None, q_pos0=0):
+    """fp64 backward of attention over explicit index lists (no bias).
+
+    q/dout [B,Tq,Hq,d] bf16, k/v [B,L,Hkv,d] bf16, idx [B,Tq,K] or
+    [B,Tq,idx_heads,K] int32 (-1 padded).  Returns (dq [B,Tq,Hq,d],
+    dk [B,L,Hkv,d], dv [B,L,Hkv,d]) in fp64.
+    """
+    lib = _load()
+    B, Tq, Hq, d = q.shape
+    L, Hkv = k.shape[1], k.shape[2]
+    ii = _np(idx, np.int32)
+    if ii.ndim == 3:
+        ii = ii.reshape(B, Tq, 1, ii.shape[-1])
+    idx_heads, K = ii.shape[2], ii.shape[3]
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    dq = np.empty((B, Tq, Hq, d), dtype=np.float64)
+    dk = np.empty((B, L, Hkv, d), dtype=np.float64)
+    dv = np.empty((B, L, Hkv, d), dtype=np.float64)
+    _check(lib.oracle_sparse_attn_bwd(_ptr(_np(q, np.uint16)), _ptr(_np(k, np.uint16)),
+                                      _ptr(_np(v, np.uint16)), _ptr(_np(dout, np.uint16)),
+                                      B, Tq, L, Hq, Hkv, d, q_pos0, _ptr(ii), idx_heads, K,
+                                      float(scale), _ptr(dq), _ptr(dk), _ptr(dv)),
+           "sparse_attn_bwd")
+    return dq, dk, dv
 
 
 def lse_combine(part_o, part_lse):

@@ -308,6 +308,101 @@ int oracle_sparse_attn(const uint16_t *q, const uint16_t *k, const uint16_t *v,
 }
 
 /*
+ * Backward of attention over explicit index lists (the gradient of the
+ * forward above without a bias; the training results of the SpatialLM page,
+ * "SpatialLM-Mini acelero el entrenamiento ...", and the backward speed-up of
+ * the NSA page, "Puntos Clave", need it).  For each row r and head h with
+ * p_j = exp(z_j - lse), z_j = scale * (q . k_j):
+ *   dP_j = dO . v_j,   D = sum_j p_j dP_j,   dS_j = p_j (dP_j - D),
+ *   dq  = scale * sum_j dS_j k_j,
+ *   dk_j += scale * dS_j q,     dv_j += p_j dO
+ * (a key listed twice contributes twice).  The forward is recomputed here in
+ * fp64; dout is bf16, widened exactly.  Rows run in parallel; dk and dv are
+ * accumulated with atomic adds.  dq [B,Tq,Hq,d], dk/dv [B,L,Hkv,d], all fp64.
+ */
+int oracle_sparse_attn_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                           const uint16_t *dout, int64_t B, int64_t Tq, int64_t L,
+                           int64_t Hq, int64_t Hkv, int64_t d, int64_t q_pos0,
+                           const int32_t *idx, int64_t idx_heads, int64_t K, double scale,
+                           double *dq, double *dk, double *dv)
+{
+    if (B <= 0 || Tq <= 0 || L <= 0 || Hq <= 0 || Hkv <= 0 || d <= 0 || K < 0 ||
+        Hq % Hkv != 0 || q_pos0 < 0 || !(idx_heads == 1 || idx_heads == Hkv))
+        return OR_BAD_ARG;
+    const int64_t G = Hq / Hkv;
+    for (int64_t e = 0; e < B * L * Hkv * d; ++e) { dk[e] = 0.0; dv[e] = 0.0; }
+    int status = OR_OK;
+#pragma omp parallel
+    {
+        double *z = (double *)malloc(sizeof(double) * (size_t)(K > 0 ? K : 1));
+        double *dp = (double *)malloc(sizeof(double) * (size_t)(K > 0 ? K : 1));
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t r = 0; r < B * Tq; ++r) {
+            if (!z || !dp) { status = OR_BAD_ARG; continue; }
+            int64_t b = r / Tq, t = r % Tq, pos = q_pos0 + t;
+            for (int64_t h = 0; h < Hq; ++h) {
+                int64_t g = h / G;
+                const int32_t *list = idx + (r * idx_heads + (idx_heads == 1 ? 0 : g)) * K;
+                const uint16_t *qv = q + (r * Hq + h) * d;
+                const uint16_t *dov = dout + (r * Hq + h) * d;
+                double *dqv = dq + (r * Hq + h) * d;
+                for (int64_t c = 0; c < d; ++c) dqv[c] = 0.0;
+                /* forward: logits and their log-sum-exp */
+                double m = -INFINITY;
+                for (int64_t e = 0; e < K; ++e) {
+                    int64_t j = list[e];
+                    z[e] = -INFINITY;
+                    if (j < 0) continue;
+                    if (j >= L || j > pos) { status = OR_BAD_INDEX; continue; }
+                    const uint16_t *kv = k + ((b * L + j) * Hkv + g) * d;
+                    double dot = 0.0;
+                    for (int64_t c = 0; c < d; ++c) dot += bf16_to_f64(qv[c]) * bf16_to_f64(kv[c]);
+                    z[e] = scale * dot;
+                    if (z[e] > m) m = z[e];
+                }
+                if (m == -INFINITY) continue;              /* empty set: no gradient */
+                double s = 0.0;
+                for (int64_t e = 0; e < K; ++e)
+                    if (z[e] != -INFINITY) s += exp(z[e] - m);
+                const double lse = m + log(s);
+                /* dP_j and D */
+                double D = 0.0;
+                for (int64_t e = 0; e < K; ++e) {
+                    if (z[e] == -INFINITY) continue;
+                    const uint16_t *vv = v + ((b * L + list[e]) * Hkv + g) * d;
+                    double x = 0.0;
+                    for (int64_t c = 0; c < d; ++c) x += bf16_to_f64(dov[c]) * bf16_to_f64(vv[c]);
+                    dp[e] = x;
+                    D += exp(z[e] - lse) * x;
+                }
+                /* dS_j, then dq, dk_j and dv_j */
+                for (int64_t e = 0; e < K; ++e) {
+                    if (z[e] == -INFINITY) continue;
+                    const int64_t j = list[e];
+                    const double p = exp(z[e] - lse);
+                    const double ds = p * (dp[e] - D);
+                    const uint16_t *kv = k + ((b * L + j) * Hkv + g) * d;
+                    double *dkv = dk + ((b * L + j) * Hkv + g) * d;
+                    double *dvv = dv + ((b * L + j) * Hkv + g) * d;
+                    for (int64_t c = 0; c < d; ++c) {
+                        dqv[c] += scale * ds * bf16_to_f64(kv[c]);
+                        const double a = scale * ds * bf16_to_f64(qv[c]);
+                        const double bv = p * bf16_to_f64(dov[c]);
+#pragma omp atomic
+                        dkv[c] += a;
+#pragma omp atomic
+                        dvv[c] += bv;
+                    }
+                }
+            }
+        }
+        free(z);
+        free(dp);
+    }
+    return status;
+}
+
+/*
  * Distributed-softmax merge (Star Attention page, body): partial results
  * (O_s, lse_s) over disjoint pieces of one softmax are combined as
  *   lse = log sum_s exp(lse_s),   O = sum_s exp(lse_s - lse) O_s.

@@ -540,3 +540,103 @@ def test_indexcache_s_layers_reuse_f_indices():
 def test_indexcache_pattern_must_start_with_f():
     with pytest.raises(oracle.OracleError):
         oracle.dsa_layers("SFFF", _decode_layers(4), topk=8)
+
+
+# ------------------------------------------------------- attention backward --
+def _autograd_ref(q, k, v, dout, bias, scale):
+    """dq, dk, dv of softmax(scale q.k + bias) v by torch float64 autograd;
+    bias [B,Hq,T,L] additive (-inf = not in the set).  GQA by repeating the
+    KV heads (autograd sums their gradients)."""
+    qh = _f64(q).transpose(1, 2).clone().requires_grad_(True)
+    kh = _f64(k).transpose(1, 2).clone().requires_grad_(True)
+    vh = _f64(v).transpose(1, 2).clone().requires_grad_(True)
+    G = qh.shape[1] // kh.shape[1]
+    bias = torch.broadcast_to(bias, (qh.shape[0], qh.shape[1], qh.shape[2], kh.shape[2]))
+    # a row with an empty set has no gradient: give it a finite bias and no
+    # incoming gradient, so softmax stays defined and it contributes nothing
+    empty = torch.isneginf(bias).all(dim=-1, keepdim=True)
+    bias = torch.where(empty, torch.zeros_like(bias), bias)
+    z = torch.matmul(qh, kh.repeat_interleave(G, dim=1).transpose(-1, -2)) * scale + bias
+    p = torch.softmax(z, dim=-1)
+    o = torch.matmul(p, vh.repeat_interleave(G, dim=1))
+    o.backward(_f64(dout).transpose(1, 2).masked_fill(empty, 0.0))
+    return (qh.grad.transpose(1, 2).numpy(), kh.grad.transpose(1, 2).numpy(),
+            vh.grad.transpose(1, 2).numpy())
+
+
+def _bias_from_lists(idx, B, Hq, Hkv, T, L):
+    """Additive bias log(multiplicity) from index lists [B,T,ih,K]."""
+    ii = idx if idx.ndim == 4 else idx[:, :, None, :]
+    mult = np.zeros((B, ii.shape[2], T, L))
+    for b in range(B):
+        for t in range(T):
+            for ih in range(ii.shape[2]):
+                for j in ii[b, t, ih]:
+                    if j >= 0:
+                        mult[b, ih, t, j] += 1
+    G = Hq // Hkv
+    per_head = np.repeat(mult, Hq if ii.shape[2] == 1 else G, axis=1)
+    with np.errstate(divide="ignore"):
+        return torch.from_numpy(np.log(per_head))
+
+
+def _bwd_case(B, T, Hq, Hkv, d, seed):
+    g = inputs.gen_dsa(B, T, Hq, Hkv, d, 1, 32, seed=seed)
+    gen = torch.Generator().manual_seed(seed + 7)
+    dout = torch.randn(B, T, Hq, d, generator=gen).to(torch.bfloat16)
+    return g["q"], g["k"], g["v"], dout
+
+
+def test_backward_complete_set_is_dense_causal_autograd():
+    B, T, Hq, Hkv, d = 1, 40, 4, 2, 16
+    q, k, v, dout = _bwd_case(B, T, Hq, Hkv, d, 70)
+    idx = all_pred_idx(B, T)
+    dq, dk, dv = oracle.sparse_attn_bwd(q, k, v, dout, idx)
+    mask = torch.ones(T, T, dtype=torch.bool).tril()
+    bias = torch.zeros(T, T, dtype=torch.float64).masked_fill(~mask, float("-inf"))
+    rq, rk, rv = _autograd_ref(q, k, v, dout, bias, 1 / math.sqrt(d))
+    np.testing.assert_allclose(dq, rq, atol=1e-10)
+    np.testing.assert_allclose(dk, rk, atol=1e-10)
+    np.testing.assert_allclose(dv, rv, atol=1e-10)
+
+
+@pytest.mark.parametrize("idx_heads", [1, 2])
+def test_backward_random_lists_with_duplicates(idx_heads):
+    # random lists (one shared, or one per KV head), an empty row, a repeated
+    # key (a repeat counts twice: bias log 2 in the dense form)
+    B, T, Hq, Hkv, d, K = 2, 30, 4, 2, 16, 9
+    q, k, v, dout = _bwd_case(B, T, Hq, Hkv, d, 71 + idx_heads)
+    rng = np.random.default_rng(5 + idx_heads)
+    idx = np.full((B, T, idx_heads, K), -1, dtype=np.int32)
+    for b in range(B):
+        for t in range(T):
+            for ih in range(idx_heads):
+                n = min(t + 1, K - 1)
+                idx[b, t, ih, :n] = rng.choice(t + 1, size=n, replace=False)
+                idx[b, t, ih, K - 1] = idx[b, t, ih, 0]          # duplicate
+    idx[1, 5] = -1                                               # empty row
+    ii = idx if idx_heads > 1 else idx[:, :, 0, :]
+    dq, dk, dv = oracle.sparse_attn_bwd(q, k, v, dout, ii)
+    bias = _bias_from_lists(idx, B, Hq, Hkv, T, T)
+    rq, rk, rv = _autograd_ref(q, k, v, dout, bias, 1 / math.sqrt(d))
+    np.testing.assert_allclose(dq, rq, atol=1e-10)
+    np.testing.assert_allclose(dk, rk, atol=1e-10)
+    np.testing.assert_allclose(dv, rv, atol=1e-10)
+    assert np.all(dq[1, 5] == 0)
+
+
+def test_backward_column_sum_identities():
+    # sum_j dS_j = 0 per (row, head), so sum_j dk_j = 0; sum_j p_j = 1 per
+    # non-empty (row, head), so sum_j dv_j = sum of dout over the group's heads
+    B, T, Hq, Hkv, d = 1, 64, 8, 2, 32
+    q, k, v, dout = _bwd_case(B, T, Hq, Hkv, d, 73)
+    rng = np.random.default_rng(9)
+    K = 12
+    idx = np.full((B, T, K), -1, dtype=np.int32)
+    for t in range(T):
+        n = min(t + 1, K)
+        idx[0, t, :n] = rng.choice(t + 1, size=n, replace=False)
+    dq, dk, dv = oracle.sparse_attn_bwd(q, k, v, dout, idx)
+    np.testing.assert_allclose(dk.sum(axis=1), 0.0, atol=1e-10)
+    do = _f64(dout).numpy().reshape(B, T, Hkv, Hq // Hkv, d).sum(axis=(1, 3))
+    np.testing.assert_allclose(dv.sum(axis=1), do, atol=1e-10)
