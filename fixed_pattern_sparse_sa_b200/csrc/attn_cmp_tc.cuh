@@ -68,15 +68,6 @@ struct CtSmem {                    // head dim 128
     static constexpr int ALLOC = TOTAL + 1024;
 };
 
-namespace atc {
-__device__ __forceinline__ void load_3d(void *dst, const CUtensorMap *map, int x, int y, int z, uint64_t *bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3, %4}], [%5];\n" ::"r"(tc::smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(tc::smem_u32(bar))
-        : "memory");
-}
-}  // namespace atc
 
 // 2^x on the special-function unit (flushes results below the normal range
 // to zero, which a softmax weight can ignore).

@@ -24,8 +24,10 @@
 //   warps 5-8  softmax + epilogue: thread r owns key row r of S^T (and row r
 //              of O^T = output column d = r); per-head maxima are combined
 //              across the four warps through shared memory.
-// The running maximum is only raised (and O rescaled in TMEM) when a tile's
-// maximum exceeds it by more than 2^8, so most tiles skip the rescale.
+// The running maximum is only raised (and O rescaled in TMEM) when some
+// logit of a tile exceeds it by more than 2^60: one vote of the softmax
+// group per tile, and the exact cross-warp max only on a tile that needs it
+// (in practice an item's first).
 // Every wait is bounded; on a timeout the kernel records ERR_TIMEOUT, stops
 // issuing work, waits (bounded) for its own copies and frees its TMEM.
 #pragma once
@@ -43,6 +45,7 @@ constexpr int ATC_PRODUCERS = 128;          // producer threads (warps 0-3)
 constexpr int ATC_MMA_WARP = 4;
 constexpr int ATC_KEYS = 128;               // keys per tile
 constexpr long long ATC_WAIT = 2000000000LL;   // ~1 s in SM clocks: drain waits
+constexpr float ATC_RAISE = 60.f;           // log2 headroom of the running softmax max
 
 struct AtcParams {
     GatherParams g;                         // shapes, list, outputs, scale, error word
@@ -65,8 +68,8 @@ struct AtcSmem {
     static constexpr int OFF_RED = OFF_KEYS + ATC_STAGES * ATC_KEYS * 4;
     static constexpr int OFF_BAR = OFF_RED + 1024;
     // barriers: kv_full[S], kv_empty[S], q_full[2], q_empty[2], s_full[2],
-    // s_free[2], p_full[2], pv_done[2], o_full, o_free, drain
-    static constexpr int N_BAR = 2 * ATC_STAGES + 12 + 3;
+    // s_free[2], p_full[2], pv_done[2], o_full, o_free, drain, tma_full[S]
+    static constexpr int N_BAR = 3 * ATC_STAGES + 12 + 3;
     static constexpr int OFF_MISC = OFF_BAR + N_BAR * 8;         // tmem slot, abort flag
     static constexpr int TOTAL = OFF_MISC + 16;
     static constexpr int ALLOC = TOTAL + 1024;                   // room to align the base
@@ -95,6 +98,14 @@ __device__ __forceinline__ void load_2d(void *dst, const CUtensorMap *map, int x
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(tc::smem_u32(bar))
         : "memory");
 }
+// box of a 3-D tensor map at (x, y, z)
+__device__ __forceinline__ void load_3d(void *dst, const CUtensorMap *map, int x, int y, int z, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];\n" ::"r"(tc::smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(tc::smem_u32(bar))
+        : "memory");
+}
 // shared-memory descriptor, 128-byte swizzle
 __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
     uint64_t d = 0;
@@ -116,6 +127,16 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
 __device__ __forceinline__ void named_sync(int id, int n) {
     asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(n) : "memory");
+}
+// Named-barrier OR over the n threads of barrier `id` (same verdict for all).
+__device__ __forceinline__ bool vote_any(int id, int n, bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, %2, %3, p;\n selp.u32 %0, 1, 0, q;\n}\n"
+        : "=r"(r)
+        : "r"((uint32_t)v), "r"(id), "r"(n)
+        : "memory");
+    return r != 0;
 }
 // Named-barrier AND over the n threads of barrier `id`: every thread gets the
 // same verdict, so a failed wait never leaves part of the group behind at a
@@ -159,10 +180,15 @@ __device__ __forceinline__ void atc_item(const GatherParams &p, int it, int &b, 
     b = r;
 }
 
+// SRC = KS_IDX gathers key rows with cp.async; SRC = KS_BLOCKS (NSA selected
+// blocks of p.block consecutive keys) loads each block's K and V rows with TMA
+// box loads (kmap / vmap: [B*Lk rows, Hkv, D] bf16, box = one block).
 template <int D, int SRC>
 __global__ void __launch_bounds__(ATC_THREADS, 1)
-    attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const AtcParams ap) {
+    attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
+                   const __grid_constant__ CUtensorMap vmap, const AtcParams ap) {
     static_assert(D == 128, "the tensor-core gather path handles head dim 128");
+    constexpr bool TMA = SRC == KS_BLOCKS;
     using L = AtcSmem<D>;
     const GatherParams &p = ap.g;
     extern __shared__ unsigned char smem_raw[];
@@ -173,6 +199,7 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
     uint64_t *s_full = q_empty + 2, *s_free = s_full + 2;
     uint64_t *p_full = s_free + 2, *pv_done = p_full + 2;
     uint64_t *o_full = pv_done + 2, *o_free = o_full + 1, *drain = o_free + 1;
+    uint64_t *tma_full = drain + 1;                 // KS_BLOCKS: bytes of a stage's TMA block loads
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::OFF_MISC + 4);
     int *keys_s = reinterpret_cast<int *>(smem + L::OFF_KEYS);
@@ -185,8 +212,12 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
     }
     if (tid == 0) {
         for (int i = 0; i < ATC_STAGES; ++i) {
-            tc::mbar_init(kv_full + i, 2 * ATC_PRODUCERS);
+            // keys (and, with cp.async, copies) of a stage: every producer
+            // thread arrives once for its keys_s entry and once more for its
+            // copies; with TMA block loads the bytes complete tma_full instead
+            tc::mbar_init(kv_full + i, (TMA ? 1 : 2) * ATC_PRODUCERS);
             tc::mbar_init(kv_empty + i, 1);
+            tc::mbar_init(tma_full + i, 1);
         }
         for (int i = 0; i < 2; ++i) {
             tc::mbar_init(q_full + i, 1); tc::mbar_init(q_empty + i, 1);
@@ -287,25 +318,54 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
                 keys_s[st * ATC_KEYS + tid] = key;
                 unsigned char *kdst = smem + L::OFF_KV + st * L::STAGE;
                 unsigned char *vdst = kdst + L::KV_BYTES;
-                // this warp's 32 rows, two 256-byte rows per instruction
+                if constexpr (TMA) {
+                    // the tile's ATC_KEYS / block blocks, each one box load per
+                    // 64-column half of K and of V; a slot with no valid block
+                    // loads block 0 so that masked rows hold finite values
+                    if (tid == 0) {
+                        atc::expect_tx(tma_full + st, 2 * L::KV_BYTES);
+                        const int32_t *list = p.idx + ((long long)(b * p.Tq + t) * p.Hkv + g) * p.K;
+                        for (int i = 0; i < ATC_KEYS / p.block; ++i) {
+                            const int e0 = e_beg + k * ATC_KEYS + i * p.block;
+                            int blk = e0 < min(p.entries, e_beg + per) ? __ldg(list + e0 / p.block) : -1;
+                            if (blk < 0 || (long long)blk * p.block >= p.Lk) blk = 0;
+                            const int z = b * p.Lk + blk * p.block;
+                            for (int h = 0; h < 2; ++h) {
+                                const uint32_t off = (uint32_t)h * (ATC_KEYS * 128) + (uint32_t)(i * p.block) * 128;
+                                atc::load_3d(kdst + off, &kmap, h * 64, g, z, tma_full + st);
+                                atc::load_3d(vdst + off, &vmap, h * 64, g, z, tma_full + st);
+                            }
+                        }
+                    }
+                    atc::arrive(kv_full + st);                       // this thread's keys_s entry
+                } else {
+                    // this warp's 32 rows, two 256-byte rows per instruction
 #pragma unroll 4
-                for (int j = 0; j < 16; ++j) {
-                    const int rr = 2 * j + hi;                       // row within the warp's 32
-                    const int kk = __shfl_sync(0xffffffffu, key, rr);
-                    const int r = warp * 32 + rr;                    // row within the tile
-                    const long long grow = row_base + (long long)(kk >= 0 ? kk : 0) * p.Hkv;
-                    const uint32_t off = ch_off + (uint32_t)r * 128 + ((uint32_t)((ch & 7) ^ (r & 7)) << 4);
-                    cp_async16(kdst + off, p.k + grow * D + ch * 8, kk >= 0 ? 16 : 0);
-                    cp_async16(vdst + off, p.v + grow * D + ch * 8, kk >= 0 ? 16 : 0);
+                    for (int j = 0; j < 16; ++j) {
+                        const int rr = 2 * j + hi;                       // row within the warp's 32
+                        const int kk = __shfl_sync(0xffffffffu, key, rr);
+                        const int r = warp * 32 + rr;                    // row within the tile
+                        const long long grow = row_base + (long long)(kk >= 0 ? kk : 0) * p.Hkv;
+                        const uint32_t off = ch_off + (uint32_t)r * 128 + ((uint32_t)((ch & 7) ^ (r & 7)) << 4);
+                        cp_async16(kdst + off, p.k + grow * D + ch * 8, kk >= 0 ? 16 : 0);
+                        cp_async16(vdst + off, p.v + grow * D + ch * 8, kk >= 0 ? 16 : 0);
+                    }
+                    // the stage completes once every producer thread has arrived
+                    // (releasing its keys_s entry) and the copies of every
+                    // producer thread have landed
+                    atc::arrive(kv_full + st);
+                    atc::arrive_on_copies(kv_full + st);
                 }
-                // the stage completes once every producer thread has arrived
-                // (releasing its keys_s entry) and the copies of every
-                // producer thread have landed
-                atc::arrive(kv_full + st);
-                atc::arrive_on_copies(kv_full + st);
             }
         }
         cp_async_wait<0>();                                  // nothing of ours is still in flight
+        if (TMA && tid == 0) {
+            // the block loads of the last stages land before the CTA exits
+            for (int i = 0; i < ATC_STAGES && i < tile; ++i) {
+                const int ti = tile - 1 - i;
+                tc::mbar_wait_bounded(tma_full + ti % ATC_STAGES, (ti / ATC_STAGES) & 1, ATC_WAIT);
+            }
+        }
         if (!ok && lane == 0) fail();
         if (warp == 0 && lane == 0) {
             for (int i = 0; i < 2 && i < qn; ++i) {
@@ -323,7 +383,7 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
             // S^T(tile) = K . Q^T into S buffer tile & 1
             auto issue_s = [&](int tl, int st, int qb) -> bool {
                 const int sb = tl & 1;
-                if (!atc::wait(kv_full + st, (tl / ATC_STAGES) & 1, abort_flag)) return false;
+                if (!atc::wait((TMA ? tma_full : kv_full) + st, (tl / ATC_STAGES) & 1, abort_flag)) return false;
                 if (!atc::wait(s_free + sb, ((tl >> 1) & 1) ^ 1, abort_flag)) return false;
                 tc::fence_after_sync();
                 tc::fence_proxy_async_smem();   // the copied K rows -> tensor-core reads
@@ -412,35 +472,39 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
                 atc::arrive(s_free + sb);
                 const bool valid = keys_s[st * ATC_KEYS + r] >= 0;
                 float x[16];
-                int wm[16];
+                bool need = false;
 #pragma unroll
                 for (int h = 0; h < 16; ++h) {
                     x[h] = valid ? __uint_as_float(sr[h]) * p.scale_log2 : -INFINITY;
-                    wm[h] = __reduce_max_sync(0xffffffffu, atc::f2ord(x[h]));
+                    need |= x[h] > m[h] + ATC_RAISE;
                 }
-                if (lane == 0) {
+                // The running max m is only a reference point (softmax does not
+                // depend on it) and stays put while no logit exceeds it by more
+                // than 2^ATC_RAISE, which fp32 weights and sums absorb.  One vote
+                // of the group per tile; the exact tile max (two exchanges
+                // through shared memory) only when some logit is above that.
+                if (atc::vote_any(1, 128, need)) {
+                    int wm[16];
 #pragma unroll
-                    for (int h = 0; h < 16; h += 4)
-                        *reinterpret_cast<int4 *>(red_s + sw * 16 + h) = make_int4(wm[h], wm[h + 1], wm[h + 2], wm[h + 3]);
-                }
-                atc::named_sync(1, 128);
-                if (sw == 0 && lane < 16) {
-                    const int* ri = reinterpret_cast<const int *>(red_s);
-                    const int v = max(max(ri[lane], ri[16 + lane]), max(ri[32 + lane], ri[48 + lane]));
-                    red_s[64 + lane] = atc::ord2f(v);
-                }
-                atc::named_sync(1, 128);
-                float mt[16];
+                    for (int h = 0; h < 16; ++h) wm[h] = __reduce_max_sync(0xffffffffu, atc::f2ord(x[h]));
+                    if (lane == 0) {
 #pragma unroll
-                for (int h = 0; h < 16; h += 4) {
-                    const float4 v = *reinterpret_cast<const float4 *>(red_s + 64 + h);
-                    mt[h] = v.x; mt[h + 1] = v.y; mt[h + 2] = v.z; mt[h + 3] = v.w;
-                }
-                // raise the running max only when a tile exceeds it by more than 2^8
-                bool raise = false;
+                        for (int h = 0; h < 16; h += 4)
+                            *reinterpret_cast<int4 *>(red_s + sw * 16 + h) = make_int4(wm[h], wm[h + 1], wm[h + 2], wm[h + 3]);
+                    }
+                    atc::named_sync(1, 128);
+                    if (sw == 0 && lane < 16) {
+                        const int* ri = reinterpret_cast<const int *>(red_s);
+                        const int v = max(max(ri[lane], ri[16 + lane]), max(ri[32 + lane], ri[48 + lane]));
+                        red_s[64 + lane] = atc::ord2f(v);
+                    }
+                    atc::named_sync(1, 128);
+                    float mt[16];
 #pragma unroll
-                for (int h = 0; h < 16; ++h) raise |= mt[h] > m[h] + 8.f;
-                if (raise) {
+                    for (int h = 0; h < 16; h += 4) {
+                        const float4 v = *reinterpret_cast<const float4 *>(red_s + 64 + h);
+                        mt[h] = v.x; mt[h + 1] = v.y; mt[h + 2] = v.z; mt[h + 3] = v.w;
+                    }
                     float alpha[16];
 #pragma unroll
                     for (int h = 0; h < 16; ++h) {

@@ -197,6 +197,22 @@ static int bf16_tensor_map(CUtensorMap *m, const void *base, long long rows, int
 }
 
 
+// 3-D bf16 map over [rows, hkv, d] (d contiguous); box = 64 columns (128
+// bytes) x 1 head x box_rows rows, 128-byte swizzle.
+static int bf16_tensor_map_3d(CUtensorMap *m, const void *base, int d, int hkv, long long rows, int box_rows) {
+    TensorMapEncodeFn enc = tensor_map_encoder();
+    if (!enc) return fail(SA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+    cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)hkv, (cuuint64_t)rows};
+    cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)hkv * d * 2};
+    cuuint32_t box[3] = {64u, 1u, (cuuint32_t)box_rows};
+    cuuint32_t es[3] = {1u, 1u, 1u};
+    const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(SA_ERR_CUDA, "cuTensorMapEncodeTiled(3d) failed (%d)", (int)r);
+    return SA_OK;
+}
+
 // SA_ATTN_PATH=tc routes explicit-list attention (head dim 128, <= 16 heads
 // per KV head, no bias) through attn_tc_kernel.  It is opt-in: with 64-KB
 // K/V stages it keeps fewer gathered bytes in flight per SM than the
@@ -212,8 +228,9 @@ static bool attn_tc_allowed() {
 }
 
 static bool attn_tc_applies(const GatherParams &p, int d, int src, bool bias) {
-    return attn_tc_allowed() && (src == KS_IDX || src == KS_BLOCKS) && !bias && d == 128 && p.G <= 16 &&
-           !p.klo && (!p.out_f32 || p.n_split == 1) && (long long)p.B * p.Lk * p.Hkv < INT_MAX &&
+    const bool blocks_ok = src != KS_BLOCKS || (p.block == 32 || p.block == 64 || p.block == 128);
+    return attn_tc_allowed() && (src == KS_IDX || src == KS_BLOCKS) && blocks_ok && !bias && d == 128 &&
+           p.G <= 16 && !p.klo && (!p.out_f32 || p.n_split == 1) && (long long)p.B * p.Lk * p.Hkv < INT_MAX &&
            (long long)p.B * p.Tq * p.Hq + 16 < INT_MAX;
 }
 
@@ -225,6 +242,15 @@ static int launch_attn_tc(const GatherParams &p, cudaStream_t st) {
     CUtensorMap qm;
     int rc = bf16_tensor_map(&qm, p.q, (long long)p.B * p.Tq * p.Hq, 128, 16);
     if (rc) return rc;
+    // K and V maps for the TMA block loads (selected NSA blocks); unused
+    // when rows are gathered one by one
+    CUtensorMap km = qm, vm = qm;
+    if (SRC == KS_BLOCKS) {
+        rc = bf16_tensor_map_3d(&km, p.k, 128, p.Hkv, (long long)p.B * p.Lk, p.block);
+        if (rc) return rc;
+        rc = bf16_tensor_map_3d(&vm, p.v, 128, p.Hkv, (long long)p.B * p.Lk, p.block);
+        if (rc) return rc;
+    }
     AtcParams ap{};
     ap.g = p;
     ap.n_items = (int)items;
@@ -234,7 +260,7 @@ static int launch_attn_tc(const GatherParams &p, cudaStream_t st) {
     rc = set_smem(kern, smem);
     if (rc) return rc;
     const int grid = (int)std::min<long long>(items, sm_count());
-    kern<<<grid, ATC_THREADS, smem, st>>>(qm, ap);
+    kern<<<grid, ATC_THREADS, smem, st>>>(qm, km, vm, ap);
     SA_CHECK_LAUNCH("attn_tc_kernel");
     return SA_OK;
 }
@@ -856,20 +882,6 @@ static int launch_tile_t(const TileParams &p, cudaStream_t st) {
     return SA_OK;
 }
 
-// NSA compressed branch on tcgen05 (head dim 128, <= 16 heads per group).
-static int bf16_tensor_map_3d(CUtensorMap *m, const void *base, int d, int hkv, long long rows, int box_rows) {
-    TensorMapEncodeFn enc = tensor_map_encoder();
-    if (!enc) return fail(SA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
-    cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)hkv, (cuuint64_t)rows};
-    cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)hkv * d * 2};
-    cuuint32_t box[3] = {64u, 1u, (cuuint32_t)box_rows};
-    cuuint32_t es[3] = {1u, 1u, 1u};
-    const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
-                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return fail(SA_ERR_CUDA, "cuTensorMapEncodeTiled(3d) failed (%d)", (int)r);
-    return SA_OK;
-}
 
 template <int SRC>
 static int launch_nsa_tc(const TileParams &p, unsigned *err, cudaStream_t st) {
