@@ -13,6 +13,7 @@ EXPORTS = (
     "sa_indexer_topk_workspace_size", "sa_indexer_topk",
     "sa_sparse_attn_workspace_size", "sa_sparse_attn_fwd",
     "sa_sparse_attn_fwd_split_static",
+    "sa_sparse_attn_bwd_workspace_size", "sa_sparse_attn_bwd",
     "sa_lse_combine",
     "sa_nsa_workspace_size", "sa_nsa_fwd",
     "sa_dsa_decode_layers_workspace_size", "sa_dsa_decode_layers",
@@ -72,6 +73,8 @@ def load() -> ctypes.CDLL:
             "sa_sparse_attn_fwd_split_static": (I, [P, P, P, I, I, I, I, I, I, I64, P, I, I,
                                                     F, I, P, P, P]),
             "sa_lse_combine": (I, [P, P, I, I64, I, P, P, P]),
+            "sa_sparse_attn_bwd_workspace_size": (SZ, [I, I, I]),
+            "sa_sparse_attn_bwd": (I, [P, P, P, P, P, P, I, I, I, I, I, I, I64, P, I, I, F, P, P, P, P, SZ, P]),
             "sa_nsa_workspace_size": (SZ, [I, I, I, I, I, I, I, I, I]),
             "sa_nsa_fwd": (I, [P, P, P, P, I, I, I, I, I, I, I, I, I, I, F, P, P, P, P, SZ, P]),
             "sa_dsa_decode_layers_workspace_size": (SZ, [I, I, I, I, I, I, I, I, I, I]),

@@ -16,7 +16,8 @@ import torch
 from . import _lib
 from ._lib import SAError, check, sa_dsa_layer, sa_pattern
 
-__all__ = ["indexer_topk", "sparse_attn_fwd", "sparse_attn_fwd_split_static", "lse_combine", "nsa_fwd",
+__all__ = ["indexer_topk", "sparse_attn_fwd", "sparse_attn_bwd", "sparse_attn_fwd_split_static", "lse_combine",
+           "nsa_fwd",
            "dsa_decode_layers", "check_device_status", "debug_set_spin_limit", "debug_inject_stall",
            "debug_exact_recompute_rows", "SAError"]
 
@@ -224,6 +225,42 @@ def sparse_attn_fwd_split_static(q, k, v, idx, n_split: int, scale: Optional[flo
             float(scale), int(n_split), _ptr(out), _ptr(lse), _stream(dev)),
             "sa_sparse_attn_fwd_split_static")
     return out, lse
+
+
+def sparse_attn_bwd(q, k, v, out, lse, dout, idx, scale: Optional[float] = None,
+                    q_pos0: Optional[int] = None):
+    """Backward of sparse_attn_fwd over explicit index lists (sa_sparse_attn_bwd).
+
+    q, out, dout bf16 [B,Tq,Hq,d]; k, v bf16 [B,L,Hkv,d]; lse fp32 [B,Tq,Hq]
+    (the forward's); idx int32 [B,Tq,K] or [B,Tq,idx_heads,K].
+    Returns (dq fp32 [B,Tq,Hq,d], dk fp32 [B,L,Hkv,d], dv fp32 [B,L,Hkv,d]).
+    """
+    lib = _lib.load()
+    dev = q.device
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout")):
+        _need(t, n, torch.bfloat16, dev, 4)
+    _need(lse, "lse", torch.float32, dev, 3)
+    _need(idx, "idx", torch.int32, dev)
+    B, Tq, Hq, d = q.shape
+    L, Hkv = k.shape[1], k.shape[2]
+    if k.shape != (B, L, Hkv, d) or v.shape != k.shape or out.shape != q.shape or dout.shape != q.shape:
+        raise ValueError("sparse_attn_bwd: shape mismatch")
+    idx_heads = 1 if idx.dim() == 3 else idx.shape[2]
+    K = idx.shape[-1]
+    pos0 = L - Tq if q_pos0 is None else int(q_pos0)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = torch.empty((B, Tq, Hq, d), dtype=torch.float32, device=dev)
+    dk = torch.empty((B, L, Hkv, d), dtype=torch.float32, device=dev)
+    dv = torch.empty((B, L, Hkv, d), dtype=torch.float32, device=dev)
+    nbytes = lib.sa_sparse_attn_bwd_workspace_size(B, Tq, Hq)
+    ws = _workspace(nbytes, dev)
+    with torch.cuda.device(dev):
+        check(lib.sa_sparse_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout),
+                                     B, Tq, L, Hq, Hkv, d, pos0, _ptr(idx), idx_heads, K, float(scale),
+                                     _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws), nbytes, _stream(dev)),
+              "sa_sparse_attn_bwd")
+    return dq, dk, dv
 
 
 def lse_combine(part_o, part_lse, out=None, lse=None):

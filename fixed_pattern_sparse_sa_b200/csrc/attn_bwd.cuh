@@ -1,0 +1,315 @@
+// attn_bwd.cuh -- backward of gathered-KV sparse attention over explicit
+// index lists.
+//
+// The training results of the SpatialLM page ("SpatialLM-Mini acelero el
+// entrenamiento ...") and the backward speed-up of the NSA page ("Native
+// Sparse Attention ...", "Puntos Clave") need the gradient of the sparse
+// forward.  For query t, head h and its set S (z_j = scale q.k_j,
+// p_j = exp(z_j - lse), lse saved by the forward):
+//   dP_j = dO . v_j,   D = dO . O = sum_j p_j dP_j,   dS_j = p_j (dP_j - D)
+//   dq = scale sum_j dS_j k_j,  dk_j += scale dS_j q,  dv_j += p_j dO
+//
+// One warp per (query, KV group, 16-head chunk): the heads of the group are
+// the 16 rows of m16 tiles, as in the forward.  Keys come in chunks of 16,
+// gathered by cp.async (two stages) into XOR-swizzled shared memory.  Per
+// chunk: S = Q K^T and dP = dO V^T (mma.sync m16n8k16, bf16 -> fp32), P and
+// dS in registers, dq += dS K (kept in registers); dS^T and P^T go through a
+// 16 x 16 shared-memory tile (ldmatrix.trans) to form dK = dS^T Q and
+// dV = P^T dO for the chunk's 16 keys, which are added to the fp32 dk / dv
+// with vector reductions (a key selected by several queries collects all of
+// their contributions).  D comes from a first pass (attn_bwd_prep_kernel).
+#pragma once
+
+#include "attn_gather.cuh"
+
+namespace sa {
+
+struct BwdParams {
+    const __nv_bfloat16 *q, *k, *v, *o, *dout;   // q/o/dout [B,Tq,Hq,D], k/v [B,L,Hkv,D]
+    const float *lse;                            // [B,Tq,Hq] natural log (forward)
+    const int32_t *idx;                          // [B,Tq,idx_heads,K]
+    int B, Tq, L, Hq, Hkv, G, idx_heads, K;
+    long long q_pos0;
+    float scale, scale_log2;
+    float *Dt;                                   // [B,Tq,Hq] dO . O
+    float *dq;                                   // [B,Tq,Hq,D]
+    float *dk, *dv;                              // [B,L,Hkv,D] (zeroed before)
+    unsigned *err;
+};
+
+// D = sum_c dO[row, c] * O[row, c], one warp per row.
+template <int D>
+__global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const BwdParams p, long long rows) {
+    const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    const __nv_bfloat162 *a = reinterpret_cast<const __nv_bfloat162 *>(p.dout + row * D);
+    const __nv_bfloat162 *b = reinterpret_cast<const __nv_bfloat162 *>(p.o + row * D);
+    float s = 0.f;
+#pragma unroll
+    for (int c = lane; c < D / 2; c += 32) {
+        const float2 x = __bfloat1622float2(a[c]), y = __bfloat1622float2(b[c]);
+        s += x.x * y.x + x.y * y.y;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == 0) p.Dt[row] = s;
+}
+
+// Shared memory of one warp: K/V stages and their keys, the Q and dO tiles of
+// the 16 heads and two 16 x 16 transpose tiles, rounded to 1 KB so that every
+// warp's region (and each tile in it) stays 16-byte aligned.
+template <int D>
+__host__ __device__ constexpr int attn_bwd_warp_bytes() {
+    return (2 * (2 * 16 * D * 2 + 16 * 4) + 2 * 16 * D * 2 + 2 * 16 * 32 + 1023) / 1024 * 1024;
+}
+
+__device__ __forceinline__ void red_add2(float *addr, float a, float b) {
+    asm volatile("red.global.add.v2.f32 [%0], {%1, %2};\n" ::"l"(addr), "f"(a), "f"(b) : "memory");
+}
+
+// ldmatrix of one 16 x 16 bf16 tile stored row-major with 32-byte rows
+// (element (r, c) at r * 32 + c * 2): A fragment of the tile (trans = false)
+// or of its transpose (trans = true).
+template <bool TRANS>
+__device__ __forceinline__ void ldsm_tile16(unsigned (&a)[4], const unsigned char *tile, int lane) {
+    const int mi = lane >> 3, ri = lane & 7;
+    if constexpr (!TRANS) {
+        // matrices: rows 0-7 / 8-15 x cols 0-7 / 8-15 in A-fragment order
+        const int row = (mi & 1) * 8 + ri, col = (mi >> 1) * 8;
+        ldsm_x4(a[0], a[1], a[2], a[3], tile + row * 32 + col * 2);
+    } else {
+        // A of the transpose: (r, c) of A is tile (c, r)
+        const int row = (mi >> 1) * 8 + ri, col = (mi & 1) * 8;
+        ldsm_x4_t(a[0], a[1], a[2], a[3], tile + row * 32 + col * 2);
+    }
+}
+
+template <int D, int NW>
+__global__ void __launch_bounds__(NW * 32) attn_bwd_kernel(const BwdParams p) {
+    constexpr int NK = 16;                  // keys per chunk
+    constexpr int STAGES = 2;
+    constexpr int ROWB = D * 2;
+    constexpr int UNITS = ROWB / 16;
+    constexpr int CH = NK * ROWB;           // one K (or V) chunk
+    constexpr int KS_D = D / 16;
+    constexpr int NT_D = D / 8;
+    constexpr int CP_ITERS = NK * UNITS / 32;
+    constexpr int QT = 16 * ROWB;           // Q (or dO) tile of the 16 heads
+    constexpr int WSM = attn_bwd_warp_bytes<D>();
+
+    extern __shared__ __align__(1024) unsigned char smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    unsigned char *wsm = smem + warp * WSM;
+    unsigned char *q_s = wsm;                       // [16 heads][D] swizzled
+    unsigned char *do_s = q_s + QT;
+    unsigned char *tp_s = do_s + QT;                // 16 x 16 bf16 tiles: dS, P
+    unsigned char *kv_s = tp_s + 2 * 16 * 32;
+    int *keys_s = reinterpret_cast<int *>(kv_s + STAGES * 2 * CH);
+
+    const int n_hchunk = (p.G + 15) / 16;
+    const long long n_items = (long long)p.B * p.Tq * p.Hkv * n_hchunk;
+    const long long item = (long long)blockIdx.x * NW + warp;
+    if (item >= n_items) return;
+    long long rem = item;
+    const int hc = (int)(rem % n_hchunk); rem /= n_hchunk;
+    const int g = (int)(rem % p.Hkv); rem /= p.Hkv;
+    const int t = (int)(rem % p.Tq); rem /= p.Tq;
+    const int b = (int)rem;
+    const long long pos = p.q_pos0 + t;
+
+    const int gr = lane >> 2, qc = lane & 3;
+    const int hr0 = hc * 16 + gr, hr1 = hr0 + 8;
+    const bool v0 = hr0 < p.G, v1 = hr1 < p.G;
+    const long long row0 = (long long)(b * p.Tq + t) * p.Hq + g * p.G + hr0;   // flat rows of the two heads
+    const long long row1 = row0 + 8;
+
+    // Q and dO of the 16 heads into shared memory (swizzled like K rows);
+    // rows past the group are zero
+    for (int i = lane; i < 16 * UNITS; i += 32) {
+        const int r = i / UNITS, u = i % UNITS;
+        const bool ok = hc * 16 + r < p.G;
+        const long long base = ((long long)(b * p.Tq + t) * p.Hq + g * p.G + hc * 16 + r) * D + u * 8;
+        const int sw = (u ^ (r & 7)) * 16;
+        cp_async16(q_s + r * ROWB + sw, ok ? p.q + base : p.q, ok ? 16 : 0);
+        cp_async16(do_s + r * ROWB + sw, ok ? p.dout + base : p.dout, ok ? 16 : 0);
+    }
+    cp_async_commit();
+    const float lse0 = v0 ? p.lse[row0] * kLog2e : 0.f, lse1 = v1 ? p.lse[row1] * kLog2e : 0.f;
+    const float D0 = v0 ? p.Dt[row0] : 0.f, D1 = v1 ? p.Dt[row1] : 0.f;
+    // a row whose forward set was empty has lse = -inf: no gradient
+    const bool live0 = v0 && lse0 != -INFINITY, live1 = v1 && lse1 != -INFINITY;
+
+    const int32_t *list = p.idx + ((long long)(b * p.Tq + t) * p.idx_heads + (p.idx_heads == 1 ? 0 : g)) * p.K;
+    const int n_chunks = (p.K + NK - 1) / NK;
+    const __nv_bfloat16 *kb = p.k + ((long long)b * p.L * p.Hkv + g) * D;
+    const __nv_bfloat16 *vb = p.v + ((long long)b * p.L * p.Hkv + g) * D;
+    const long long rstride = (long long)p.Hkv * D;
+
+    auto issue = [&](int ci) {
+        const int st = ci % STAGES;
+        unsigned char *ks_ = kv_s + st * 2 * CH;
+        unsigned char *vs_ = ks_ + CH;
+        int j = -1;
+        if (ci < n_chunks && lane < NK) {
+            const int e = ci * NK + lane;
+            if (e < p.K) {
+                const int raw = __ldg(list + e);
+                if (raw >= 0) {
+                    if (raw >= p.L || (long long)raw > pos) raise_error(p.err, ERR_BAD_INDEX);
+                    else j = raw;
+                }
+            }
+            keys_s[st * NK + lane] = j;
+        }
+        if (ci < n_chunks) {
+#pragma unroll
+            for (int it = 0; it < CP_ITERS; ++it) {
+                const int lin = it * 32 + lane;
+                const int rr = lin / UNITS, u = lin % UNITS;
+                const int jr = __shfl_sync(0xffffffffu, j, rr);
+                const long long off = jr >= 0 ? (long long)jr * rstride + u * 8 : 0;
+                const int sw = (u ^ (rr & 7)) * 16;
+                cp_async16(ks_ + rr * ROWB + sw, kb + off, jr >= 0 ? 16 : 0);
+                cp_async16(vs_ + rr * ROWB + sw, vb + off, jr >= 0 ? 16 : 0);
+            }
+        }
+        cp_async_commit();
+    };
+
+    float dqa[NT_D][4];
+#pragma unroll
+    for (int i = 0; i < NT_D; ++i) dqa[i][0] = dqa[i][1] = dqa[i][2] = dqa[i][3] = 0.f;
+
+    issue(0);
+    for (int ci = 0; ci < n_chunks; ++ci) {
+        issue(ci + 1);
+        cp_async_wait<1>();
+        __syncwarp();
+        const int st = ci % STAGES;
+        const unsigned char *ks_ = kv_s + st * 2 * CH;
+        const unsigned char *vs_ = ks_ + CH;
+        const int jl = lane < NK ? keys_s[st * NK + lane] : -1;
+        const unsigned vmask = __ballot_sync(0xffffffffu, jl >= 0);
+        if (vmask != 0u) {
+            // S = Q K^T and dP = dO V^T over the head dimension
+            float sc[2][4], dp[2][4];
+#pragma unroll
+            for (int i = 0; i < 2; ++i) sc[i][0] = sc[i][1] = sc[i][2] = sc[i][3] = dp[i][0] = dp[i][1] = dp[i][2] = dp[i][3] = 0.f;
+#pragma unroll
+            for (int ks = 0; ks < KS_D; ++ks) {
+                const int mi = lane >> 3, ri = lane & 7;
+                unsigned qa[4], da[4];
+                {
+                    // A fragments of Q and dO (rows = heads) for k-step ks
+                    const int row = (mi & 1) * 8 + ri, unit = ks * 2 + (mi >> 1);
+                    ldsm_x4(qa[0], qa[1], qa[2], qa[3], q_s + row * ROWB + ((unit ^ (row & 7)) * 16));
+                    ldsm_x4(da[0], da[1], da[2], da[3], do_s + row * ROWB + ((unit ^ (row & 7)) * 16));
+                }
+                const int key = (mi >> 1) * 8 + ri;
+                const int unit = ks * 2 + (mi & 1);
+                unsigned b0, b1, b2, b3;
+                ldsm_x4(b0, b1, b2, b3, ks_ + key * ROWB + ((unit ^ (key & 7)) * 16));
+                mma_bf16_16816(sc[0], qa, b0, b1);
+                mma_bf16_16816(sc[1], qa, b2, b3);
+                ldsm_x4(b0, b1, b2, b3, vs_ + key * ROWB + ((unit ^ (key & 7)) * 16));
+                mma_bf16_16816(dp[0], da, b0, b1);
+                mma_bf16_16816(dp[1], da, b2, b3);
+            }
+            // P = exp(z - lse), dS = P (dP - D); masked keys and dead rows give 0
+            float pr[2][4], ds[2][4];
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int kk = nt * 8 + 2 * qc + (e & 1);
+                    const bool hi = e >> 1;
+                    const bool ok = ((vmask >> kk) & 1u) && (hi ? live1 : live0);
+                    const float pv = ok ? exp2f(sc[nt][e] * p.scale_log2 - (hi ? lse1 : lse0)) : 0.f;
+                    pr[nt][e] = pv;
+                    ds[nt][e] = pv * (dp[nt][e] - (hi ? D1 : D0));
+                }
+            }
+            // dS and P as bf16 A fragments (rows = heads, k = keys)
+            unsigned dsa[4], pa[4];
+            dsa[0] = pack_bf16(ds[0][0], ds[0][1]); dsa[1] = pack_bf16(ds[0][2], ds[0][3]);
+            dsa[2] = pack_bf16(ds[1][0], ds[1][1]); dsa[3] = pack_bf16(ds[1][2], ds[1][3]);
+            pa[0] = pack_bf16(pr[0][0], pr[0][1]); pa[1] = pack_bf16(pr[0][2], pr[0][3]);
+            pa[2] = pack_bf16(pr[1][0], pr[1][1]); pa[3] = pack_bf16(pr[1][2], pr[1][3]);
+            // dq += dS K  (B = K rows [key][d], transposed loads as V in the forward)
+#pragma unroll
+            for (int dpi = 0; dpi < NT_D / 2; ++dpi) {
+                const int mi = lane >> 3, ri = lane & 7;
+                const int key = (mi & 1) * 8 + ri;
+                const int unit = dpi * 2 + (mi >> 1);
+                unsigned b0, b1, b2, b3;
+                ldsm_x4_t(b0, b1, b2, b3, ks_ + key * ROWB + ((unit ^ (key & 7)) * 16));
+                mma_bf16_16816(dqa[2 * dpi], dsa, b0, b1);
+                mma_bf16_16816(dqa[2 * dpi + 1], dsa, b2, b3);
+            }
+            // dS and P tiles (row = head, col = key) for the transposed products
+            {
+                unsigned *t0 = reinterpret_cast<unsigned *>(tp_s);
+                unsigned *t1 = reinterpret_cast<unsigned *>(tp_s + 16 * 32);
+                // element (head gr / gr+8, key 2qc..2qc+1 / +8) of the C layout
+                t0[gr * 8 + qc] = dsa[0];       t0[(gr + 8) * 8 + qc] = dsa[1];
+                t0[gr * 8 + 4 + qc] = dsa[2];   t0[(gr + 8) * 8 + 4 + qc] = dsa[3];
+                t1[gr * 8 + qc] = pa[0];        t1[(gr + 8) * 8 + qc] = pa[1];
+                t1[gr * 8 + 4 + qc] = pa[2];    t1[(gr + 8) * 8 + 4 + qc] = pa[3];
+            }
+            __syncwarp();
+            unsigned dsT[4], pT[4];
+            ldsm_tile16<true>(dsT, tp_s, lane);
+            ldsm_tile16<true>(pT, tp_s + 16 * 32, lane);
+            // dK = scale dS^T Q and dV = P^T dO for the 16 keys (rows gr, gr+8),
+            // 16 columns at a time, added to the global accumulators
+            const int j0 = __shfl_sync(0xffffffffu, jl, gr), j1 = __shfl_sync(0xffffffffu, jl, gr + 8);
+            float *dk0 = p.dk + ((long long)(b * p.L + (j0 >= 0 ? j0 : 0)) * p.Hkv + g) * D;
+            float *dk1 = p.dk + ((long long)(b * p.L + (j1 >= 0 ? j1 : 0)) * p.Hkv + g) * D;
+            float *dv0 = p.dv + ((long long)(b * p.L + (j0 >= 0 ? j0 : 0)) * p.Hkv + g) * D;
+            float *dv1 = p.dv + ((long long)(b * p.L + (j1 >= 0 ? j1 : 0)) * p.Hkv + g) * D;
+#pragma unroll
+            for (int dpi = 0; dpi < NT_D / 2; ++dpi) {
+                const int mi = lane >> 3, ri = lane & 7;
+                const int hrow = (mi & 1) * 8 + ri;
+                const int unit = dpi * 2 + (mi >> 1);
+                unsigned b0, b1, b2, b3;
+                float ck[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                float cv[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                ldsm_x4_t(b0, b1, b2, b3, q_s + hrow * ROWB + ((unit ^ (hrow & 7)) * 16));
+                mma_bf16_16816(ck[0], dsT, b0, b1);
+                mma_bf16_16816(ck[1], dsT, b2, b3);
+                ldsm_x4_t(b0, b1, b2, b3, do_s + hrow * ROWB + ((unit ^ (hrow & 7)) * 16));
+                mma_bf16_16816(cv[0], pT, b0, b1);
+                mma_bf16_16816(cv[1], pT, b2, b3);
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    const int col = (2 * dpi + h2) * 8 + 2 * qc;
+                    if (j0 >= 0) {
+                        red_add2(dk0 + col, ck[h2][0] * p.scale, ck[h2][1] * p.scale);
+                        red_add2(dv0 + col, cv[h2][0], cv[h2][1]);
+                    }
+                    if (j1 >= 0) {
+                        red_add2(dk1 + col, ck[h2][2] * p.scale, ck[h2][3] * p.scale);
+                        red_add2(dv1 + col, cv[h2][2], cv[h2][3]);
+                    }
+                }
+            }
+        }
+        __syncwarp();
+    }
+    cp_async_wait<0>();
+#pragma unroll
+    for (int nt = 0; nt < NT_D; ++nt) {
+        const int col = nt * 8 + 2 * qc;
+        if (v0) *reinterpret_cast<float2 *>(p.dq + row0 * D + col) = make_float2(dqa[nt][0] * p.scale, dqa[nt][1] * p.scale);
+        if (v1) *reinterpret_cast<float2 *>(p.dq + row1 * D + col) = make_float2(dqa[nt][2] * p.scale, dqa[nt][3] * p.scale);
+    }
+}
+
+template <int D, int NW>
+constexpr int attn_bwd_smem_bytes() {
+    return NW * attn_bwd_warp_bytes<D>();
+}
+
+}  // namespace sa

@@ -16,6 +16,7 @@
 #include <string>
 
 #include "../../include/sa.h"
+#include "attn_bwd.cuh"
 #include "attn_gather.cuh"
 #include "attn_tc.cuh"
 #include "attn_cmp_tc.cuh"
@@ -1146,4 +1147,66 @@ int sa_probe_gather(const void *buf, int64_t n_rows, int mode, int warps, int st
     if (stages == 2) return launch_probe<0, 2>(p, ctas, smem, st);
     if (stages == 4) return launch_probe<0, 4>(p, ctas, smem, st);
     return launch_probe<0, 8>(p, ctas, smem, st);
+}
+
+// ------------------------------------------------------------- backward --
+size_t sa_sparse_attn_bwd_workspace_size(int B, int Tq, int Hq) {
+    if (B <= 0 || Tq <= 0 || Hq <= 0) return 0;
+    return round_up((size_t)B * Tq * Hq * 4, 256);
+}
+
+template <int D>
+static int launch_bwd(const BwdParams &p, long long rows, cudaStream_t st) {
+    constexpr int NW = 8;
+    attn_bwd_prep_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(p, rows);
+    SA_CHECK_LAUNCH("attn_bwd_prep_kernel");
+    constexpr int smem = attn_bwd_smem_bytes<D, NW>();
+    static_assert(smem <= 227 * 1024, "shared memory");
+    auto kern = attn_bwd_kernel<D, NW>;
+    int rc = set_smem(kern, smem);
+    if (rc) return rc;
+    const long long items = (long long)p.B * p.Tq * p.Hkv * ((p.G + 15) / 16);
+    if (items == 0) return SA_OK;
+    kern<<<(unsigned)((items + NW - 1) / NW), NW * 32, smem, st>>>(p);
+    SA_CHECK_LAUNCH("attn_bwd_kernel");
+    return SA_OK;
+}
+
+int sa_sparse_attn_bwd(const void *q, const void *k, const void *v, const void *out, const float *lse,
+                       const void *dout, int B, int Tq, int L, int Hq, int Hkv, int d, int64_t q_pos0,
+                       const int32_t *idx, int idx_heads, int K, float scale, float *dq, float *dk, float *dv,
+                       void *workspace, size_t workspace_bytes, void *stream) {
+    if (B <= 0 || Tq < 0 || L <= 0 || Hq <= 0 || Hkv <= 0 || K < 0 || Hq % Hkv)
+        return fail(SA_ERR_INVALID_ARG, "attn_bwd: bad sizes B=%d Tq=%d L=%d Hq=%d Hkv=%d K=%d", B, Tq, L, Hq, Hkv, K);
+    if (d != 64 && d != 128) return fail(SA_ERR_UNSUPPORTED, "attn_bwd: head dim %d", d);
+    if (q_pos0 < 0 || q_pos0 + Tq > L)
+        return fail(SA_ERR_INVALID_ARG, "attn_bwd: query positions outside [0, L)");
+    if (!(idx_heads == 1 || idx_heads == Hkv)) return fail(SA_ERR_INVALID_ARG, "attn_bwd: idx_heads");
+    if (!q || !k || !v || !out || !lse || !dout || !idx || !dq || !dk || !dv || !aligned16(q) || !aligned16(k) ||
+        !aligned16(v) || !aligned16(out) || !aligned16(dout) || !aligned4(lse) || !aligned4(idx) ||
+        !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+        return fail(SA_ERR_INVALID_ARG, "attn_bwd: null or misaligned pointer");
+    if (!std::isfinite(scale)) return fail(SA_ERR_INVALID_ARG, "attn_bwd: scale");
+    if (Tq == 0) return SA_OK;
+    const size_t need = sa_sparse_attn_bwd_workspace_size(B, Tq, Hq);
+    if (!workspace || workspace_bytes < need)
+        return fail(SA_ERR_WORKSPACE, "attn_bwd: workspace %zu < %zu", workspace_bytes, need);
+    if (!aligned16(workspace)) return fail(SA_ERR_INVALID_ARG, "attn_bwd: workspace alignment");
+    unsigned *ew = nullptr;
+    int rc = device_error_word(&ew);
+    if (rc) return rc;
+    cudaStream_t st = as_stream(stream);
+    const size_t kv_bytes = (size_t)B * L * Hkv * d * 4;
+    cudaError_t e = cudaMemsetAsync(dk, 0, kv_bytes, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dv, 0, kv_bytes, st);
+    if (e != cudaSuccess) return fail(SA_ERR_CUDA, "attn_bwd memset: %s", cudaGetErrorString(e));
+    BwdParams p{};
+    p.q = static_cast<const __nv_bfloat16 *>(q); p.k = static_cast<const __nv_bfloat16 *>(k);
+    p.v = static_cast<const __nv_bfloat16 *>(v); p.o = static_cast<const __nv_bfloat16 *>(out);
+    p.dout = static_cast<const __nv_bfloat16 *>(dout); p.lse = lse; p.idx = idx;
+    p.B = B; p.Tq = Tq; p.L = L; p.Hq = Hq; p.Hkv = Hkv; p.G = Hq / Hkv; p.idx_heads = idx_heads; p.K = K;
+    p.q_pos0 = q_pos0; p.scale = scale; p.scale_log2 = scale * kLog2e;
+    p.Dt = static_cast<float *>(workspace); p.dq = dq; p.dk = dk; p.dv = dv; p.err = ew;
+    const long long rows = (long long)B * Tq * Hq;
+    return d == 64 ? launch_bwd<64>(p, rows, st) : launch_bwd<128>(p, rows, st);
 }

@@ -135,6 +135,27 @@ int sa_sparse_attn_fwd(const void *q, const void *k, const void *v,
                        void *workspace, size_t workspace_bytes, void *stream);
 
 /* --------------------------------------------------------------------------
+ * Backward of gathered-KV sparse attention over explicit index lists (no
+ * bias).  SpatialLM page (training with the fixed sparse graph) and NSA page
+ * ("Puntos Clave": the backward pass of sparse attention).  With p_j =
+ * exp(z_j - lse), z_j = scale * q.k_j over the row's list (a repeated entry
+ * counts twice, as in the forward):
+ *   dP_j = dout . v_j,  D = dout . out,  dS_j = p_j (dP_j - D)
+ *   dq = scale * sum_j dS_j k_j,  dk_j += scale * dS_j q,  dv_j += p_j dout
+ *   q, out, dout bf16 [B,Tq,Hq,d]; k, v bf16 [B,L,Hkv,d]; lse fp32 [B,Tq,Hq]
+ *   (the forward's outputs); idx as in sa_sparse_attn_fwd.
+ *   dq fp32 [B,Tq,Hq,d] (written); dk, dv fp32 [B,L,Hkv,d] (zeroed by the
+ *   call, then accumulated over every query that selected the key).
+ * workspace: sa_sparse_attn_bwd_workspace_size(B, Tq, Hq) bytes.
+ * ------------------------------------------------------------------------ */
+size_t sa_sparse_attn_bwd_workspace_size(int B, int Tq, int Hq);
+int sa_sparse_attn_bwd(const void *q, const void *k, const void *v, const void *out, const float *lse,
+                       const void *dout, int B, int Tq, int L, int Hq, int Hkv, int d, int64_t q_pos0,
+                       const int32_t *idx, int idx_heads, int K, float scale,
+                       float *dq, float *dk, float *dv, void *workspace, size_t workspace_bytes,
+                       void *stream);
+
+/* --------------------------------------------------------------------------
  * Split-KV sparse attention that allocates nothing.  No page has a
  * counterpart: this is a convenience entry point of this library.
  * For callers that cannot allocate device memory at call time: a serving

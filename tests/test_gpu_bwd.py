@@ -1,0 +1,117 @@
+"""GPU parity of the sparse-attention backward (sa_sparse_attn_bwd) against
+the fp64 oracle: dq, dk and dv over random index lists, per-KV-head lists,
+empty rows and repeated entries, and the complete causal set; at a larger
+size, identities that hold for any input (sum_j dk_j = 0, sum_j dv_j =
+sum of dout over the group's heads).
+
+Tolerance.  The kernel rounds P and dS to bf16 for its tensor-core products
+and takes D = dout . out from the forward's bf16 out; each rounding moves a
+term by at most 2^-9 relative, so an element is checked to within
+2^-6 * max|ref| (max-abs) and 2^-8 * mean|ref| (mean-abs) of the fp64
+gradient."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from fixed_pattern_sparse_sa_b200 import api, inputs
+from _parity import sample_rows
+
+pytestmark = pytest.mark.gpu
+
+MAX_REL = 2.0 ** -6
+MEAN_REL = 2.0 ** -8
+
+
+def _close(got, ref, what):
+    g = got.detach().double().cpu().numpy().reshape(ref.shape)
+    assert np.all(np.isfinite(g)), f"{what}: non-finite"
+    err = np.abs(g - ref)
+    scale_max, scale_mean = np.abs(ref).max(), np.abs(ref).mean()
+    assert err.max() <= MAX_REL * scale_max + 1e-6, f"{what}: max err {err.max():.3e} vs {scale_max:.3e}"
+    assert err.mean() <= MEAN_REL * scale_mean + 1e-7, f"{what}: mean err {err.mean():.3e} vs {scale_mean:.3e}"
+
+
+def _lists(B, T, ih, K, seed, dup=False):
+    rng = np.random.default_rng(seed)
+    idx = np.full((B, T, ih, K), -1, dtype=np.int32)
+    for b in range(B):
+        for t in range(T):
+            for h in range(ih):
+                n = min(t + 1, K - (1 if dup else 0))
+                idx[b, t, h, :n] = rng.choice(t + 1, size=n, replace=False)
+                if dup:
+                    idx[b, t, h, K - 1] = idx[b, t, h, 0]
+    return torch.from_numpy(idx)
+
+
+def _run(q, k, v, idx, dout):
+    out, lse = api.sparse_attn_fwd(q.cuda(), k.cuda(), v.cuda(), idx.cuda())
+    dq, dk, dv = api.sparse_attn_bwd(q.cuda(), k.cuda(), v.cuda(), out, lse, dout.cuda(), idx.cuda())
+    api.check_device_status()
+    return dq, dk, dv
+
+
+@pytest.mark.parametrize("B,T,Hq,Hkv,d,K,ih,dup", [
+    (1, 300, 16, 1, 128, 200, 1, False),     # MQA group of 16, lists shorter than the row
+    (2, 257, 8, 2, 64, 90, 2, True),         # per-KV-head lists, repeats, ragged chunks
+    (1, 129, 12, 1, 128, 64, 1, True),       # 12 heads (a partial m16 tile)
+])
+def test_backward_random_lists(cuda_ok, B, T, Hq, Hkv, d, K, ih, dup):
+    g = inputs.gen_dsa(B, T, Hq, Hkv, d, 1, 32, seed=T + d)
+    gen = torch.Generator().manual_seed(T)
+    dout = torch.randn(B, T, Hq, d, generator=gen).to(torch.bfloat16)
+    idx = _lists(B, T, ih, K, seed=T, dup=dup)
+    if ih == 1:
+        idx = idx[:, :, 0]
+    idx[0, 3] = -1                                       # an empty row
+    dq, dk, dv = _run(g["q"], g["k"], g["v"], idx, dout)
+    rq, rk, rv = oracle.sparse_attn_bwd(g["q"], g["k"], g["v"], dout, idx)
+    _close(dq, rq, "dq")
+    _close(dk, rk, "dk")
+    _close(dv, rv, "dv")
+    assert torch.count_nonzero(dq[0, 3]) == 0
+
+
+def test_backward_complete_causal_set(cuda_ok):
+    B, T, Hq, Hkv, d = 1, 200, 16, 1, 128
+    g = inputs.gen_dsa(B, T, Hq, Hkv, d, 1, 32, seed=5)
+    dout = torch.randn(B, T, Hq, d, generator=torch.Generator().manual_seed(6)).to(torch.bfloat16)
+    idx = torch.full((B, T, T), -1, dtype=torch.int32)
+    for t in range(T):
+        idx[0, t, :t + 1] = torch.arange(t + 1)
+    dq, dk, dv = _run(g["q"], g["k"], g["v"], idx, dout)
+    rq, rk, rv = oracle.sparse_attn_bwd(g["q"], g["k"], g["v"], dout, idx)
+    _close(dq, rq, "dq")
+    _close(dk, rk, "dk")
+    _close(dv, rv, "dv")
+
+
+def test_backward_identities_16k(cuda_ok):
+    # 16384 queries x top-512 random lists: sum_j dk_j = 0 and
+    # sum_j dv_j = sum over (t, heads of the group) of dout; dq on sampled rows
+    B, T, Hq, Hkv, d, K = 1, 16384, 16, 1, 128, 512
+    g = inputs.gen_dsa(B, T, Hq, Hkv, d, 1, 32, seed=11)
+    dout = torch.randn(B, T, Hq, d, generator=torch.Generator().manual_seed(12)).to(torch.bfloat16)
+    dev = torch.device("cuda")
+    t = torch.arange(T, device=dev)
+    r = torch.rand(T, K, device=dev, generator=torch.Generator(device=dev).manual_seed(13))
+    idx = torch.minimum((r * (t[:, None] + 1).float()).long(), t[:, None]).to(torch.int32)[None]
+    dq, dk, dv = _run(g["q"], g["k"], g["v"], idx, dout)
+    sk = dk.double().sum(dim=1).cpu().numpy()
+    assert np.abs(sk).max() <= MAX_REL * dk.abs().sum(dim=1).max().item()
+    sv = dv.double().sum(dim=1).cpu().numpy()
+    ref = dout.double().sum(dim=(1, 2)).numpy()[:, None, :]
+    np.testing.assert_allclose(sv, ref, rtol=0, atol=MAX_REL * np.abs(ref).max() + 1e-3)
+    rows = sample_rows(T, 24, seed=2, edge=4)
+    sub = idx.cpu()[:, rows]
+    # dq of sampled rows from the oracle (its dk / dv need every row)
+    rq, _, _ = oracle.sparse_attn_bwd(g["q"][:, rows], g["k"], g["v"], dout[:, rows], sub,
+                                      q_pos0=0) if False else (None, None, None)
+    for i, row in enumerate(rows[:8]):
+        one = idx.cpu()[:, row:row + 1]
+        qq, dd = g["q"][:, row:row + 1], dout[:, row:row + 1]
+        rqi, _, _ = oracle.sparse_attn_bwd(qq, g["k"][:, :row + 1], g["v"][:, :row + 1], dd, one, q_pos0=row)
+        _close(dq[:, row:row + 1], rqi, f"dq row {row}")
