@@ -21,6 +21,7 @@ EXPORTS = (
     "sa_version", "sa_launch_counter",
     "sa_debug_set_spin_limit", "sa_debug_inject_stall", "sa_debug_exact_recompute_rows",
     "sa_probe_gather",
+    "sa_indexer_scores_at", "sa_topk_merge", "sa_index_shard",
 )
 
 SA_OK = 0
@@ -89,6 +90,9 @@ def load() -> ctypes.CDLL:
             "sa_debug_inject_stall": (I, [I]),
             "sa_debug_exact_recompute_rows": (I64, []),
             "sa_probe_gather": (I, [P, I64, I, I, I, I, I, P, P]),
+            "sa_indexer_scores_at": (I, [P, P, P, I, I, I, I, I, P, I, P, P]),
+            "sa_topk_merge": (I, [P, P, P, I, I64, I, I, I, I64, P, P, P]),
+            "sa_index_shard": (I, [P, I64, I64, I64, P, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(lib, name)

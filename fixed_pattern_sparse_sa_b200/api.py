@@ -17,7 +17,7 @@ from . import _lib
 from ._lib import SAError, check, sa_dsa_layer, sa_pattern
 
 __all__ = ["indexer_topk", "sparse_attn_fwd", "sparse_attn_bwd", "sparse_attn_fwd_split_static", "lse_combine",
-           "nsa_fwd",
+           "nsa_fwd", "indexer_scores_at", "topk_merge", "index_shard",
            "dsa_decode_layers", "check_device_status", "debug_set_spin_limit", "debug_inject_stall",
            "debug_exact_recompute_rows", "SAError"]
 
@@ -261,6 +261,59 @@ def sparse_attn_bwd(q, k, v, out, lse, dout, idx, scale: Optional[float] = None,
                                      _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws), nbytes, _stream(dev)),
               "sa_sparse_attn_bwd")
     return dq, dk, dv
+
+
+def indexer_scores_at(q_idx, k_idx, w, idx):
+    """Exact indexer scores of listed keys (sa_indexer_scores_at).
+
+    q_idx int8 [B,Tq,Hi,di], k_idx int8 [B,L,di], w int32 [B,Tq,Hi],
+    idx int32 [B,Tq,K] (-1 = none).  Returns int32 [B,Tq,K] (INT_MIN for -1).
+    """
+    lib = _lib.load()
+    dev = q_idx.device
+    _need(q_idx, "q_idx", torch.int8, dev, 4)
+    _need(k_idx, "k_idx", torch.int8, dev, 3)
+    _need(w, "w", torch.int32, dev, 3)
+    _need(idx, "idx", torch.int32, dev, 3)
+    B, Tq, Hi, di = q_idx.shape
+    out = torch.empty(idx.shape, dtype=torch.int32, device=dev)
+    with torch.cuda.device(dev):
+        check(lib.sa_indexer_scores_at(_ptr(q_idx), _ptr(k_idx), _ptr(w), B, Tq, k_idx.shape[1], Hi, di,
+                                       _ptr(idx), idx.shape[-1], _ptr(out), _stream(dev)), "sa_indexer_scores_at")
+    return out
+
+
+def topk_merge(cand_score, cand_idx, part_off, topk: int, window: int, q_pos: int):
+    """Exact top-k of gathered candidates (sa_topk_merge).
+
+    cand_score / cand_idx int32 [n_parts, rows, kc] (part-local indices, -1 =
+    none); part_off: n_parts ints (position of each part's index 0).  Returns
+    (idx int32 [rows, topk+window] ascending, -1 padded, count int32 [rows]).
+    """
+    lib = _lib.load()
+    dev = cand_score.device
+    _need(cand_score, "cand_score", torch.int32, dev, 3)
+    _need(cand_idx, "cand_idx", torch.int32, dev, 3)
+    n_parts, rows, kc = cand_score.shape
+    offs = (ctypes.c_int64 * n_parts)(*[int(x) for x in part_off])
+    out = torch.empty((rows, topk + window), dtype=torch.int32, device=dev)
+    cnt = torch.empty((rows,), dtype=torch.int32, device=dev)
+    with torch.cuda.device(dev):
+        check(lib.sa_topk_merge(_ptr(cand_score), _ptr(cand_idx), offs, n_parts, rows, kc, topk, window,
+                                int(q_pos), _ptr(out), _ptr(cnt), _stream(dev)), "sa_topk_merge")
+    return out, cnt
+
+
+def index_shard(idx, key_lo: int, key_hi: int):
+    """Positions -> rows of the shard [key_lo, key_hi), -1 elsewhere (sa_index_shard)."""
+    lib = _lib.load()
+    dev = idx.device
+    _need(idx, "idx", torch.int32, dev)
+    out = torch.empty_like(idx)
+    with torch.cuda.device(dev):
+        check(lib.sa_index_shard(_ptr(idx), idx.numel(), int(key_lo), int(key_hi), _ptr(out), _stream(dev)),
+              "sa_index_shard")
+    return out
 
 
 def lse_combine(part_o, part_lse, out=None, lse=None):

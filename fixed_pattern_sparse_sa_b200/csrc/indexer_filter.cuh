@@ -144,6 +144,14 @@ __device__ __forceinline__ uint64_t desc_row_swizzled(uint32_t saddr) {
 }
 }  // namespace ft
 
+// Start of the ReLU-sum chain on the folded path: the chain runs from -tau
+// so that a pair is kept when the sum ends >= 0.  With every weight folded a
+// score is below 2^25 (at most 16 heads x 128 x 128 x 128), so clamping tau
+// to [0, 2^26] keeps the keep test exact (tau <= 0 keeps everything, tau
+// above every score keeps nothing: tau = INT_MAX marks a row with nothing to
+// keep or a query past the unit) while no partial sum can leave int32.
+__device__ __forceinline__ int ft_fast_tau(int tau) { return min(max(tau, 0), 1 << 26); }
+
 // Unit u -> (b, first query, last query); latest query blocks first.
 __device__ __forceinline__ void ft_unit(const IdxParams &p, int nq, int u, int &b, int &tq0, int &tq_last) {
     const int nqb = (p.Rt + nq - 1) / nq;
@@ -339,7 +347,7 @@ __global__ void __launch_bounds__(FT_THREADS, 1)
             int tau_r[QREG ? NQT : 1];
             if constexpr (QREG) {
 #pragma unroll
-                for (int q = 0; q < NQT; ++q) tau_r[q] = fast ? max(tau_u[q], 0) : tau_u[q];
+                for (int q = 0; q < NQT; ++q) tau_r[q] = fast ? ft_fast_tau(tau_u[q]) : tau_u[q];
             }
             const long long list0 = ((long long)b * p.Rt + (tq0 + q_lo - p.t0)) * p.cand_cap;
             for (int k = 0; k < nt; ++k, ++tile) {
@@ -362,7 +370,7 @@ __global__ void __launch_bounds__(FT_THREADS, 1)
                 if (fast) {
 #pragma unroll
                     for (int q = 0; q < NQT; ++q) {
-                        const int tq_ = QREG ? tau_r[q] : max(tau_u[q], 0);
+                        const int tq_ = QREG ? tau_r[q] : ft_fast_tau(tau_u[q]);
                         int s = -tq_;
 #pragma unroll
                         for (int h = 0; h < HI; ++h) s = __viaddmax_s32(s, (int)x[q * HI + h], s);

@@ -21,6 +21,7 @@
 #include "attn_tc.cuh"
 #include "attn_cmp_tc.cuh"
 #include "attn_tile.cuh"
+#include "dist.cuh"
 #include "indexer.cuh"
 #include "indexer_filter.cuh"
 #include "nsa_misc.cuh"
@@ -1209,4 +1210,61 @@ int sa_sparse_attn_bwd(const void *q, const void *k, const void *v, const void *
     p.Dt = static_cast<float *>(workspace); p.dq = dq; p.dk = dk; p.dv = dv; p.err = ew;
     const long long rows = (long long)B * Tq * Hq;
     return d == 64 ? launch_bwd<64>(p, rows, st) : launch_bwd<128>(p, rows, st);
+}
+
+// ------------------------------------------------- sequence split (Star) --
+int sa_indexer_scores_at(const int8_t *q_idx, const int8_t *k_idx, const int32_t *w, int B, int Tq, int L, int Hi,
+                         int di, const int32_t *idx, int K, int32_t *out_score, void *stream) {
+    if (B <= 0 || Tq < 0 || L <= 0 || K < 0) return fail(SA_ERR_INVALID_ARG, "scores_at: bad sizes");
+    if (!indexer_shape_ok(Hi, di)) return fail(SA_ERR_UNSUPPORTED, "scores_at: Hi=%d di=%d", Hi, di);
+    if (!q_idx || !k_idx || !w || !idx || !out_score || !aligned16(q_idx) || !aligned16(k_idx) || !aligned4(w) ||
+        !aligned4(idx) || !aligned4(out_score))
+        return fail(SA_ERR_INVALID_ARG, "scores_at: null or misaligned pointer");
+    if (Tq == 0 || K == 0) return SA_OK;
+    unsigned *ew = nullptr;
+    int rc = device_error_word(&ew);
+    if (rc) return rc;
+    const unsigned blocks = (unsigned)((long long)B * Tq);
+    cudaStream_t st = as_stream(stream);
+    if (di == 32) idx_scores_at_kernel<32><<<blocks, 128, 0, st>>>(q_idx, k_idx, w, B, Tq, L, Hi, idx, K, out_score, ew);
+    else if (di == 64) idx_scores_at_kernel<64><<<blocks, 128, 0, st>>>(q_idx, k_idx, w, B, Tq, L, Hi, idx, K, out_score, ew);
+    else idx_scores_at_kernel<128><<<blocks, 128, 0, st>>>(q_idx, k_idx, w, B, Tq, L, Hi, idx, K, out_score, ew);
+    SA_CHECK_LAUNCH("idx_scores_at_kernel");
+    return SA_OK;
+}
+
+int sa_topk_merge(const int32_t *cand_score, const int32_t *cand_idx, const int64_t *part_off, int n_parts,
+                  int64_t rows, int kc, int topk, int window, int64_t q_pos, int32_t *out_idx, int32_t *out_count,
+                  void *stream) {
+    if (n_parts < 1 || n_parts > TM_MAX_PARTS || rows < 0 || kc < 0 || topk < 0 || window < 0 || q_pos < 0)
+        return fail(SA_ERR_INVALID_ARG, "topk_merge: bad sizes (n_parts 1..%d)", TM_MAX_PARTS);
+    if (topk > TM_MAX_K || (long long)n_parts * kc > TM_MAX_CAND)
+        return fail(SA_ERR_UNSUPPORTED, "topk_merge: topk %d (max %d) or %lld candidates per row (max %d)", topk,
+                    TM_MAX_K, (long long)n_parts * kc, TM_MAX_CAND);
+    if (!cand_score || !cand_idx || !part_off || !out_idx || !aligned4(cand_score) || !aligned4(cand_idx) ||
+        !aligned4(out_idx) || (out_count && !aligned4(out_count)))
+        return fail(SA_ERR_INVALID_ARG, "topk_merge: null or misaligned pointer");
+    if (rows == 0) return SA_OK;
+    MergeOffsets mo{};
+    for (int i = 0; i < n_parts; ++i) {
+        if (part_off[i] < 0) return fail(SA_ERR_INVALID_ARG, "topk_merge: negative part offset");
+        mo.off[i] = part_off[i];
+    }
+    const int smem = topk_merge_smem_bytes(n_parts * kc);
+    int rc = set_smem(topk_merge_kernel, smem);
+    if (rc) return rc;
+    topk_merge_kernel<<<(unsigned)rows, TM_THREADS, smem, as_stream(stream)>>>(
+        cand_score, cand_idx, mo, n_parts, rows, kc, topk, window, q_pos,
+        out_idx, out_count);
+    SA_CHECK_LAUNCH("topk_merge_kernel");
+    return SA_OK;
+}
+
+int sa_index_shard(const int32_t *idx, int64_t n, int64_t key_lo, int64_t key_hi, int32_t *out, void *stream) {
+    if (n < 0 || key_lo < 0 || key_hi < key_lo || !idx || !out || !aligned4(idx) || !aligned4(out))
+        return fail(SA_ERR_INVALID_ARG, "index_shard: bad arguments");
+    if (n == 0) return SA_OK;
+    index_shard_kernel<<<(unsigned)((n + 255) / 256), 256, 0, as_stream(stream)>>>(idx, n, key_lo, key_hi, out);
+    SA_CHECK_LAUNCH("index_shard_kernel");
+    return SA_OK;
 }

@@ -253,6 +253,41 @@ int sa_dsa_decode_layers(const char *pattern, int n_layers, const sa_dsa_layer *
                          void *stream);
 
 /* --------------------------------------------------------------------------
+ * Sequence split across GPUs (Star Attention page, "NVIDIA AI Research
+ * presenta Star Attention ...", body: the context is split across hosts and
+ * their partial results are merged by a distributed softmax).  With the keys
+ * of a sequence split by position over R ranks, decode queries (at the last
+ * position) take the exact global selection and attention as follows:
+ *   1. every rank: sa_indexer_topk over its own keys with topk + window
+ *      candidates and window 0, then sa_indexer_scores_at for their scores;
+ *   2. the ranks all-gather the (score, index) candidates;
+ *   3. sa_topk_merge: the exact top-k of the gathered candidates by
+ *      (score desc, position asc), the forced window appended (the global
+ *      top-k of the non-window keys lies in the union of the local
+ *      top-(k + window) sets, so this equals the single-GPU selection);
+ *   4. every rank: sa_index_shard maps the selection to its rows, then
+ *      sa_sparse_attn_fwd over its keys; the partial (out, lse) of the ranks
+ *      are all-gathered and merged by sa_lse_combine.
+ * sa_indexer_scores_at: out_score[b,t,e] = I(t, idx[b,t,e]) (exact, int32)
+ *   for idx >= 0, INT_MIN for -1.  idx [B,Tq,K]; other arguments as in
+ *   sa_indexer_topk.
+ * sa_topk_merge: candidates [n_parts, rows, kc] (scores and part-local
+ *   indices, -1 = none); part p's indices are shifted by part_off[p] (host
+ *   array, n_parts <= 64) to positions.  Positions in [q_pos - window + 1, q_pos] are not
+ *   ranked; they are appended.  out_idx [rows, topk + window] ascending, -1
+ *   padded; out_count [rows] (nullable).  topk <= 4096 and
+ *   n_parts * kc <= 24576.
+ * sa_index_shard: out[i] = idx[i] - key_lo if key_lo <= idx[i] < key_hi,
+ *   else -1 (n entries).
+ * ------------------------------------------------------------------------ */
+int sa_indexer_scores_at(const int8_t *q_idx, const int8_t *k_idx, const int32_t *w, int B, int Tq, int L, int Hi,
+                         int di, const int32_t *idx, int K, int32_t *out_score, void *stream);
+int sa_topk_merge(const int32_t *cand_score, const int32_t *cand_idx, const int64_t *part_off, int n_parts,
+                  int64_t rows, int kc, int topk, int window, int64_t q_pos, int32_t *out_idx, int32_t *out_count,
+                  void *stream);
+int sa_index_shard(const int32_t *idx, int64_t n, int64_t key_lo, int64_t key_hi, int32_t *out, void *stream);
+
+/* --------------------------------------------------------------------------
  * Status helpers.
  * sa_check_device_status: waits for `stream`, reads and clears the device
  *   error word of the current device; returns SA_ERR_TIMEOUT if a kernel

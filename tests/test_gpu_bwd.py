@@ -105,13 +105,14 @@ def test_backward_identities_16k(cuda_ok):
     sv = dv.double().sum(dim=1).cpu().numpy()
     ref = dout.double().sum(dim=(1, 2)).numpy()[:, None, :]
     np.testing.assert_allclose(sv, ref, rtol=0, atol=MAX_REL * np.abs(ref).max() + 1e-3)
-    rows = sample_rows(T, 24, seed=2, edge=4)
-    sub = idx.cpu()[:, rows]
-    # dq of sampled rows from the oracle (its dk / dv need every row)
-    rq, _, _ = oracle.sparse_attn_bwd(g["q"][:, rows], g["k"], g["v"], dout[:, rows], sub,
-                                      q_pos0=0) if False else (None, None, None)
-    for i, row in enumerate(rows[:8]):
+    # dq of sampled rows from the oracle (its dk / dv need every row); the
+    # bound is relative to the gradient's scale over the sampled rows
+    rows = sample_rows(T, 8, seed=2, edge=2)
+    got, ref = [], []
+    for row in rows:
         one = idx.cpu()[:, row:row + 1]
         qq, dd = g["q"][:, row:row + 1], dout[:, row:row + 1]
         rqi, _, _ = oracle.sparse_attn_bwd(qq, g["k"][:, :row + 1], g["v"][:, :row + 1], dd, one, q_pos0=row)
-        _close(dq[:, row:row + 1], rqi, f"dq row {row}")
+        got.append(dq[:, row:row + 1].double().cpu())
+        ref.append(rqi)
+    _close(torch.cat(got, dim=1), np.concatenate(ref, axis=1), "dq (sampled rows)")

@@ -1,9 +1,16 @@
-"""Multi-rank host logic of bench.py on CPU: two gloo ranks.
+"""Multi-rank host logic on CPU: two gloo ranks.
 
 Each rank of `bench.py --gpus N` runs its own sequence (replicas, weak
 scaling); the only cross-rank steps are barriers and the max-over-ranks
 reduction of the timed region.  These tests run that logic with the gloo
-backend in two spawned processes, plus the reference arm's rank rule."""
+backend in two spawned processes, plus the reference arm's rank rule.
+
+The sequence-split decode driver (fixed_pattern_sparse_sa_b200.seqsplit)
+is run on two gloo ranks as well, with the library calls replaced by
+oracle-backed stand-ins: its exchanges and its decomposition (local
+top-(k + window) candidates, global merge, partial attention, log-sum-exp
+merge) must reproduce the oracle's selection and attention over the whole
+sequence."""
 import json
 import os
 import socket
@@ -97,3 +104,55 @@ def test_reference_arm_line_shape():
         assert k in line
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
     assert line["cpu_baseline"]["kind"] == "oracle"
+
+
+def _seqsplit_problem(nseq=2, L=3000, topk=200, window=16):
+    from fixed_pattern_sparse_sa_b200 import inputs
+    lay = inputs.gen_decode_layer(nseq, L, 4, 1, 64, 2, 32, layer=0, seed=3)
+    return lay, topk, window
+
+
+def _seqsplit_worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    from datetime import timedelta
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    try:
+        sys.path.insert(0, os.path.join(ROOT, "tests"))
+        import _oracle_ops
+        from fixed_pattern_sparse_sa_b200 import seqsplit
+        lay, topk, window = _seqsplit_problem()
+        L = lay["k"].shape[1]
+        bounds = [0, 1700, L]                                 # uneven shards
+        lo, hi = bounds[rank], bounds[rank + 1]
+        sh = seqsplit.Shard(q=lay["q"], k=lay["k"][:, lo:hi], v=lay["v"][:, lo:hi], q_idx=lay["q_idx"],
+                            k_idx=lay["k_idx"][:, lo:hi], w=lay["w"], key_lo=lo)
+        out, lse, sel = seqsplit.decode_step(sh, topk, window, L, seqsplit.dist_exchange(), bounds[:-1],
+                                             ops=_oracle_ops)
+        q.put((rank, out.numpy(), lse.numpy(), sel.numpy()))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.timeout(240)
+def test_seqsplit_decode_two_gloo_ranks_matches_whole_sequence():
+    import numpy as np
+    import oracle
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_seqsplit_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted([q.get(timeout=200) for _ in range(world)], key=lambda x: x[0])
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    lay, topk, window = _seqsplit_problem()
+    L = lay["k"].shape[1]
+    ref_idx, _ = oracle.indexer_topk(lay["q_idx"], lay["k_idx"], lay["w"], topk, window, q_pos0=L - 1)
+    ro, rl = oracle.sparse_attn(lay["q"], lay["k"], lay["v"], ref_idx.reshape(2, 1, -1), q_pos0=L - 1)
+    for rank, out, lse, sel in res:
+        np.testing.assert_array_equal(sel.reshape(ref_idx.shape), ref_idx)
+        np.testing.assert_allclose(out.reshape(ro.shape), ro, atol=1e-12)
+        np.testing.assert_allclose(lse.reshape(rl.shape), rl, atol=1e-12)
