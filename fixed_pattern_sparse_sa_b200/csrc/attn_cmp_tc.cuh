@@ -385,11 +385,11 @@ __global__ void __launch_bounds__(NT_THREADS, 1)
                     for (int e = 0; e < 16; ++e) o16[e] = 0u;
                 }
                 if (row_ok) {
+                    float4 *dst = reinterpret_cast<float4 *>(p.out_f32 + orow * D + half * OC + c);
 #pragma unroll
                     for (int e = 0; e < 16; e += 4)
-                        gated_store<4>(p.gate, p.out_f32, orow, orow * D + half * OC + c + e,
-                                       {__uint_as_float(o16[e]) * inv, __uint_as_float(o16[e + 1]) * inv,
-                                        __uint_as_float(o16[e + 2]) * inv, __uint_as_float(o16[e + 3]) * inv});
+                        dst[e / 4] = make_float4(__uint_as_float(o16[e]) * inv, __uint_as_float(o16[e + 1]) * inv,
+                                                 __uint_as_float(o16[e + 2]) * inv, __uint_as_float(o16[e + 3]) * inv);
                 }
             }
             if (have_o) {

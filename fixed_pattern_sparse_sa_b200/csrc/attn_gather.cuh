@@ -50,7 +50,6 @@ struct GatherParams {
     float *part_o;            // [n_split,B,Tq,Hq,D] (n_split > 1)
     float *part_lse;          // [n_split,B,Tq,Hq]
     float *out_f32;           // optional fp32 output [B,Tq,Hq,D] instead of bf16
-    GateOut gate;             // with out_f32: NSA gated-sum mode of the fp32 rows
     unsigned *err;
 };
 
@@ -415,8 +414,10 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
 #pragma unroll
             for (int nt = 0; nt < NT_D; ++nt) {
                 const int dcol = nt * 8 + 2 * qc;
-                if (v0) gated_store<2>(p.gate, p.out_f32, orow0, orow0 * D + dcol, {o[nt][0] * inv0, o[nt][1] * inv0});
-                if (v1) gated_store<2>(p.gate, p.out_f32, orow1, orow1 * D + dcol, {o[nt][2] * inv1, o[nt][3] * inv1});
+                if (v0) *reinterpret_cast<float2 *>(p.out_f32 + orow0 * D + dcol) =
+                    make_float2(o[nt][0] * inv0, o[nt][1] * inv0);
+                if (v1) *reinterpret_cast<float2 *>(p.out_f32 + orow1 * D + dcol) =
+                    make_float2(o[nt][2] * inv1, o[nt][3] * inv1);
             }
         } else {
 #pragma unroll

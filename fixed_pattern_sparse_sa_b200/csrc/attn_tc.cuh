@@ -595,7 +595,7 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
                     if (h < p.G) {
                         const float inv = l[h] > 0.f ? 1.f / l[h] : 0.f;
                         const float o = __uint_as_float(orow[h]) * inv;
-                        if (p.out_f32) gated_store<1>(p.gate, p.out_f32, orow0 + h, (orow0 + h) * D + r, {o});
+                        if (p.out_f32) p.out_f32[(orow0 + h) * D + r] = o;
                         else p.out[(orow0 + h) * D + r] = __float2bfloat16_rn(o);
                     }
                 }

@@ -30,7 +30,6 @@ struct TileParams {
     int cmp_len, cmp_stride;   // TS_CMP
     float scale_log2;
     float *out_f32;            // [B, T, Hq, D]
-    GateOut gate;              // NSA gated-sum mode of out_f32
     float *lse;                // [B, T, Hq]
 };
 
@@ -238,8 +237,8 @@ __global__ void __launch_bounds__(TW * 32) tile_attn_kernel(const TileParams p) 
 #pragma unroll
     for (int nt = 0; nt < NT_D; ++nt) {
         const int dcol = nt * 8 + 2 * qc;
-        if (v0) gated_store<2>(p.gate, p.out_f32, orow0, orow0 * D + dcol, {o[nt][0] * inv0, o[nt][1] * inv0});
-        if (v1) gated_store<2>(p.gate, p.out_f32, orow1, orow1 * D + dcol, {o[nt][2] * inv1, o[nt][3] * inv1});
+        if (v0) *reinterpret_cast<float2 *>(p.out_f32 + orow0 * D + dcol) = make_float2(o[nt][0] * inv0, o[nt][1] * inv0);
+        if (v1) *reinterpret_cast<float2 *>(p.out_f32 + orow1 * D + dcol) = make_float2(o[nt][2] * inv1, o[nt][3] * inv1);
     }
     if (p.lse && qc == 0) {
         if (v0) p.lse[orow0] = l0 > 0.f ? (m0 + log2f(l0)) * kLn2 : -INFINITY;

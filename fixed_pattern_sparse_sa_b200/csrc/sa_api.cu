@@ -839,7 +839,7 @@ static NsaLayout nsa_layout(int B, int T, int Hq, int Hkv, int d, int cmp_len, i
     lay.kc_off = off; off += round_up((size_t)B * std::max(lay.nc, 1) * Hkv * d * 2, 256);
     lay.klo_off = off; off += round_up((size_t)B * std::max(lay.nc, 1) * Hkv * d * 2, 256);
     lay.vc_off = off; off += round_up((size_t)B * std::max(lay.nc, 1) * Hkv * d * 2, 256);
-    lay.o3_off = off; off += round_up(rows * d * 4, 256);   // fp32 gated-sum accumulator
+    lay.o3_off = off; off += round_up(3 * rows * d * 4, 256);
     lay.l3_off = off; off += round_up(3 * rows * 4, 256);
     lay.sel_off = off; off += round_up((size_t)B * T * Hkv * sel_topk * 4, 256);
     lay.total = off;
@@ -1008,7 +1008,7 @@ int sa_nsa_fwd(const void *q, const void *k, const void *v, const float *gates, 
     base.q_pos0 = 0; base.n_split = 1; base.n_hchunk = 1; base.q_units = T;
     base.scale_log2 = scale * kLog2e;
     base.err = ew;
-    // 2. compressed branch: acc = g_c o_cmp; lse -> l3[0]
+    // 2. compressed branch -> o3[0], l3[0]
     TileParams tp{};
     tp.q = base.q; tp.B = B; tp.T = T; tp.Hq = Hq; tp.Hkv = Hkv; tp.G = G;
     tp.scale_log2 = base.scale_log2;
@@ -1017,7 +1017,6 @@ int sa_nsa_fwd(const void *q, const void *k, const void *v, const float *gates, 
         p.k = kc; p.klo = klo; p.v = vc; p.Lk = std::max(lay.nc, 1);
         p.cmp_len = cmp_len; p.cmp_stride = cmp_stride;
         p.out_f32 = o3; p.lse = l3;
-        p.gate = GateOut{gates, nullptr, 0, 0};
         // nc == 0: zero rows, lse = -inf
         rc = cmp_tc_applies(p, d) ? launch_nsa_tc<TS_CMP>(p, ew, st) : launch_tile(p, d, TS_CMP, st);
         if (rc) return rc;
@@ -1037,30 +1036,32 @@ int sa_nsa_fwd(const void *q, const void *k, const void *v, const float *gates, 
             rc = d == 64 ? launch_nsa_select<64>(sp, st) : launch_nsa_select<128>(sp, st);
         if (rc) return rc;
     }
-    // 4. selected branch: acc += g_s o_slc; lse -> l3[1]
+    // 4. selected branch -> o3[1], l3[1]
     {
         GatherParams p = base;
         p.k = static_cast<const __nv_bfloat16 *>(k); p.v = static_cast<const __nv_bfloat16 *>(v);
         p.Lk = T; p.idx = sel; p.K = sel_topk; p.block = sel_block;
         p.entries = sel_topk * sel_block; p.per_split = p.entries;
-        p.out_f32 = o3; p.lse = l3 + rows;
-        p.gate = GateOut{gates, nullptr, 1, 1};
+        p.out_f32 = o3 + rows * d; p.lse = l3 + rows;
         rc = attn_tc_applies(p, d, KS_BLOCKS, false) ? launch_attn_tc<KS_BLOCKS>(p, st)
                                                      : launch_gather(p, d, KS_BLOCKS, false, st);
         if (rc) return rc;
     }
-    // 5. window branch: out = bf16(acc + g_w o_win); lse -> l3[2]
+    // 5. window branch -> o3[2], l3[2]
     {
         TileParams p = tp;
         p.k = static_cast<const __nv_bfloat16 *>(k); p.v = static_cast<const __nv_bfloat16 *>(v);
         p.Lk = T; p.window = window;
-        p.out_f32 = o3; p.lse = l3 + 2 * rows;
-        p.gate = GateOut{gates, static_cast<__nv_bfloat16 *>(out), 2, 2};
+        p.out_f32 = o3 + 2 * rows * d; p.lse = l3 + 2 * rows;
         rc = cmp_tc_applies(p, d) ? launch_nsa_tc<TS_WINDOW>(p, ew, st) : launch_tile(p, d, TS_WINDOW, st);
         if (rc) return rc;
     }
-    // 6. per-branch LSEs (the gated sum happened in the branch epilogues)
+    // 6. gated sum
     {
+        const long long n2 = rows * (d / 2);
+        nsa_gate_kernel<<<(unsigned)((n2 + 255) / 256), 256, 0, st>>>(o3, rows * d, gates, rows, d,
+                                                                       (__nv_bfloat16 *)out);
+        SA_CHECK_LAUNCH("nsa_gate_kernel");
         if (lse_branches) {
             nsa_lse_pack_kernel<<<(unsigned)((rows + 255) / 256), 256, 0, st>>>(l3, rows, lse_branches);
             SA_CHECK_LAUNCH("nsa_lse_pack_kernel");

@@ -91,60 +91,6 @@ __device__ __forceinline__ void mma_s8_16832(int (&d)[4], unsigned a0, unsigned 
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// NSA gated sum folded into the branch epilogues (no separate pass over the
-// branch outputs): with gates [rows, 3] (already sigmoid values) the branch
-// `br` stores its normalised rows o as
-//   mode 0: acc = g o,   mode 1: acc += g o,   mode 2: out = bf16(acc + g o).
-// Without gates (gates == nullptr) o goes to acc unchanged.
-struct GateOut {
-    const float *gates;
-    __nv_bfloat16 *out;
-    int br, mode;
-};
-
-template <int N>
-__device__ __forceinline__ void vload(const float *p, float (&a)[N]) {
-    if constexpr (N == 4) { const float4 v = *reinterpret_cast<const float4 *>(p); a[0] = v.x; a[1] = v.y; a[2] = v.z; a[3] = v.w; }
-    else if constexpr (N == 2) { const float2 v = *reinterpret_cast<const float2 *>(p); a[0] = v.x; a[1] = v.y; }
-    else { a[0] = *p; }
-}
-template <int N>
-__device__ __forceinline__ void vstore(float *p, const float (&a)[N]) {
-    if constexpr (N == 4) *reinterpret_cast<float4 *>(p) = make_float4(a[0], a[1], a[2], a[3]);
-    else if constexpr (N == 2) *reinterpret_cast<float2 *>(p) = make_float2(a[0], a[1]);
-    else *p = a[0];
-}
-
-// N consecutive columns of flat output row `row` (element index idx).
-template <int N>
-__device__ __forceinline__ void gated_store(const GateOut &g, float *acc, long long row, long long idx,
-                                            const float (&v)[N]) {
-    if (!g.gates) { vstore<N>(acc + idx, v); return; }
-    const float gt = __ldg(g.gates + row * 3 + g.br);
-    float o[N];
-#pragma unroll
-    for (int i = 0; i < N; ++i) o[i] = v[i] * gt;
-    if (g.mode >= 1) {
-        float a[N];
-        vload<N>(acc + idx, a);
-#pragma unroll
-        for (int i = 0; i < N; ++i) o[i] += a[i];
-    }
-    if (g.mode == 2) {
-        if constexpr (N == 1) {
-            g.out[idx] = __float2bfloat16_rn(o[0]);
-        } else {
-#pragma unroll
-            for (int i = 0; i < N; i += 2) {
-                __nv_bfloat162 h2 = __floats2bfloat162_rn(o[i], o[i + 1]);
-                *reinterpret_cast<__nv_bfloat162 *>(g.out + idx + i) = h2;
-            }
-        }
-    } else {
-        vstore<N>(acc + idx, o);
-    }
-}
-
 __device__ __forceinline__ unsigned pack_bf16(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<unsigned *>(&v);
