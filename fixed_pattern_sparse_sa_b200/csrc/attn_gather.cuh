@@ -49,6 +49,8 @@ struct GatherParams {
     float *lse;               // [B,Tq,Hq]   (nullable)
     float *part_o;            // [n_split,B,Tq,Hq,D] (n_split > 1)
     float *part_lse;          // [n_split,B,Tq,Hq]
+    int *merge_cnt;           // split-KV with out: per (b, t, g, head chunk) arrival tickets (zeroed);
+                              // the last piece of a group merges the pieces into out / lse
     float *out_f32;           // optional fp32 output [B,Tq,Hq,D] instead of bf16
     unsigned *err;
 };
@@ -138,6 +140,41 @@ __device__ __forceinline__ int key_finish(const GatherParams &p, long long pos, 
     } else {
         return raw;
     }
+}
+
+// Log-sum-exp merge of one output row's n_split pieces (Star Attention page,
+// body: distributed softmax), over D/2 columns starting at c0; the pieces
+// were written by other CTAs of the same launch, so they are read through L2.
+template <int D>
+__device__ __forceinline__ void merge_pieces_half(const float *part_o, const float *part_lse, int n_split,
+                                                  long long rows, long long row, int c0, __nv_bfloat16 *out,
+                                                  float *lse) {
+    float m = -INFINITY;
+    for (int s = 0; s < n_split; ++s) m = fmaxf(m, __ldcg(part_lse + s * rows + row));
+    float acc[D / 2];
+#pragma unroll
+    for (int i = 0; i < D / 2; ++i) acc[i] = 0.f;
+    float den = 0.f;
+    if (m != -INFINITY) {
+        for (int s = 0; s < n_split; ++s) {
+            const float ls = __ldcg(part_lse + s * rows + row);
+            if (ls == -INFINITY) continue;
+            const float f = exp2f((ls - m) * kLog2e);
+            den += f;
+            const float4 *src = reinterpret_cast<const float4 *>(part_o + ((long long)s * rows + row) * D + c0);
+#pragma unroll
+            for (int i = 0; i < D / 8; ++i) {
+                const float4 x = __ldcg(src + i);
+                acc[4 * i] += f * x.x; acc[4 * i + 1] += f * x.y;
+                acc[4 * i + 2] += f * x.z; acc[4 * i + 3] += f * x.w;
+            }
+        }
+    }
+    const float inv = den > 0.f ? 1.f / den : 0.f;
+    unsigned *dst = reinterpret_cast<unsigned *>(out + row * D + c0);
+#pragma unroll
+    for (int i = 0; i < D / 4; ++i) dst[i] = pack_bf16(acc[2 * i] * inv, acc[2 * i + 1] * inv);
+    if (lse) lse[row] = den > 0.f ? m + log2f(den) * kLn2 : -INFINITY;
 }
 
 // KLO: keys are held as a bf16 pair (hi, lo) whose sum carries ~16 mantissa
@@ -447,6 +484,29 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
         if (qc == 0) {
             if (v0) p.part_lse[s * rows + orow0] = lse0;
             if (v1) p.part_lse[s * rows + orow1] = lse1;
+        }
+        if (p.merge_cnt) {
+            // the last piece of the group to arrive merges all pieces (the
+            // others only publish their partial rows): ticket after a fence,
+            // fence before reading the other pieces' rows from L2
+            __threadfence();
+            __syncwarp();
+            int last = 0;
+            if (lane == 0) {
+                int *ticket = p.merge_cnt + ((long long)(b * p.Tq + t) * p.Hkv + g) * p.n_hchunk + hc;
+                last = atomicAdd(ticket, 1) == p.n_split - 1;
+                if (last) *ticket = 0;                     // ready for the next call
+            }
+            if (__shfl_sync(0xffffffffu, last, 0)) {
+                __threadfence();
+                // lane l: head row l / 2 of the item, columns (l % 2) * D/2 .. + D/2
+                const int hr = hc * 16 + (lane >> 1);
+                if (hr < p.G) {
+                    const long long row = (long long)(b * p.Tq + t) * p.Hq + g * p.G + hr;
+                    merge_pieces_half<D>(p.part_o, p.part_lse, p.n_split, rows, row, (lane & 1) * (D / 2), p.out,
+                                         (lane & 1) == 0 ? p.lse : nullptr);
+                }
+            }
         }
     }
 }

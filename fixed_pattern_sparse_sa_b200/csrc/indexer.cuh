@@ -762,6 +762,38 @@ __device__ void block_minmax(int &gmin, int &gmax, int *bcast, ForEach for_each)
     __syncthreads();
 }
 
+// Exact k-th largest when every value lies in [gmin, gmin + SEL_FINE_BINS):
+// one histogram with a bin per value (fh: SEL_FINE_BINS ints of shared
+// memory).  Returns, block-uniform, the k-th largest value's offset from
+// gmin and the number of values above it.
+template <int NT, typename ForEach>
+__device__ void fine_kth(int k, int gmin, int *fh, int *scan_tmp, int *bcast, ForEach for_each, int &bin,
+                         int &above_bin) {
+    const int tid = threadIdx.x;
+    for (int i = tid; i < SEL_FINE_BINS; i += NT) fh[i] = 0;
+    __syncthreads();
+    for_each([&](int v, int) { atomicAdd(&fh[(unsigned)v - (unsigned)gmin], 1); });
+    __syncthreads();
+    constexpr int PER = SEL_FINE_BINS / NT;               // bins per thread, highest first
+    int cb[PER], local = 0;
+#pragma unroll
+    for (int u = 0; u < PER; ++u) { cb[u] = fh[SEL_FINE_BINS - 1 - (tid * PER + u)]; local += cb[u]; }
+    const int incl = block_incl_scan(local, scan_tmp);
+    int above = incl - local;
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+        if (above < k && above + cb[u] >= k) {
+            bcast[2] = SEL_FINE_BINS - 1 - (tid * PER + u);
+            bcast[3] = above;
+        }
+        above += cb[u];
+    }
+    __syncthreads();
+    bin = bcast[2];
+    above_bin = bcast[3];
+    __syncthreads();
+}
+
 // Streams int32 values [0, n) from global memory with 16-byte loads, U vectors
 // in flight per thread; f(value, index).  `vals` must be 16-byte aligned.
 template <typename F>
@@ -794,6 +826,7 @@ __device__ __forceinline__ void stream_values(const int32_t *vals, int n, F f) {
 // k-th largest score.  Rows whose every candidate is kept get INT_MIN.
 __global__ void __launch_bounds__(SEL_THREADS, 4) idx_threshold_kernel(const IdxParams p) {
     __shared__ int hist[SEL_BINS];
+    __shared__ int fine[SEL_FINE_BINS];
     __shared__ int scan_tmp[32];
     __shared__ int bcast[4];
     const int b = blockIdx.z, tr = blockIdx.y, t = p.t0 + tr;
@@ -827,6 +860,13 @@ __global__ void __launch_bounds__(SEL_THREADS, 4) idx_threshold_kernel(const Idx
     int gmin, gmax;
     block_minmax(gmin, gmax, bcast, for_each);
     const unsigned range = (unsigned)gmax - (unsigned)gmin;
+    if (range < (unsigned)SEL_FINE_BINS) {
+        // narrow range: the r-th largest sampled value from one exact histogram
+        int bin, above;
+        fine_kth<SEL_THREADS>(r, gmin, fine, scan_tmp, bcast, for_each, bin, above);
+        if (threadIdx.x == 0) p.tau[row] = (int)((unsigned)gmin + (unsigned)bin);
+        return;
+    }
     RadixState st{0u, range == 0 ? 0 : 32 - __clz(range), r, m};
     while (st.width > 0) radix_refine(st, gmin, hist, scan_tmp, bcast, for_each);
     if (threadIdx.x == 0) p.tau[row] = (int)((unsigned)gmin + st.lo_key);
@@ -975,31 +1015,11 @@ __global__ void __launch_bounds__(NT, NT <= 256 ? 3 : 1) topk_select_kernel(cons
     if (use_list && range < (unsigned)SEL_FINE_BINS) {
         // narrow score range: one exact histogram (bin = score - min) gives
         // the k-th largest score directly; the tie arrays serve as its bins
-        int *fh = reinterpret_cast<int *>(tie_key);
-        for (int i = tid; i < SEL_FINE_BINS; i += NT) fh[i] = 0;
-        __syncthreads();
-        for_each([&](int v, int) { atomicAdd(&fh[(unsigned)v - (unsigned)gmin], 1); });
-        __syncthreads();
-        constexpr int PER = SEL_FINE_BINS / NT;               // bins per thread, highest first
-        int cb[PER], local = 0;
-#pragma unroll
-        for (int u = 0; u < PER; ++u) { cb[u] = fh[SEL_FINE_BINS - 1 - (tid * PER + u)]; local += cb[u]; }
-        const int incl = block_incl_scan(local, scan_tmp);
-        int above = incl - local;
-#pragma unroll
-        for (int u = 0; u < PER; ++u) {
-            if (above < k_eff && above + cb[u] >= k_eff) {
-                bcast[2] = SEL_FINE_BINS - 1 - (tid * PER + u);
-                bcast[3] = above;
-            }
-            above += cb[u];
-        }
-        __syncthreads();
-        st.lo_key = (unsigned)bcast[2];
+        int bin, above;
+        fine_kth<NT>(k_eff, gmin, reinterpret_cast<int *>(tie_key), scan_tmp, bcast, for_each, bin, above);
+        st.lo_key = (unsigned)bin;
         st.width = 0;
-        st.k_rem = k_eff - bcast[3];
-        st.bin_count = fh[bcast[2]];
-        __syncthreads();
+        st.k_rem = k_eff - above;
     }
     while (st.width > 0 && (st.width > SEL_BITS || st.bin_count > SEL_TIE_CAP))
         radix_refine<NT>(st, gmin, hist, scan_tmp, bcast, for_each);

@@ -358,45 +358,72 @@ __global__ void __launch_bounds__(FT_THREADS, 1)
                 }
                 if (bad) continue;                         // stop with the others at the unit's end
                 tc::fence_after_sync();
-                uint32_t x[FT_CW];
-                ft::tmem_ld32(tmem + lrow + ab * FT_NCOL + c0, x);
-                ft::tmem_ld32(tmem + lrow + ab * FT_NCOL + c0 + 32, x + 32);
-                tc::tmem_ld_wait();
-                tc::fence_before_sync();
-                __syncwarp();
-                if (lane == 0) atc::arrive(acc_free + ab);
                 const int j = k * 128 + quad * 32 + lane;  // this thread's key
                 const bool full = (k + 1) * 128 <= nc_first;   // every key visible to every query
-                if (fast) {
+                const unsigned lt = (1u << lane) - 1u;
+                // two halves of this warp's 64 columns (32 registers each); the
+                // accumulator is released once the second half is loaded
 #pragma unroll
-                    for (int q = 0; q < NQT; ++q) {
-                        const int tq_ = QREG ? tau_r[q] : ft_fast_tau(tau_u[q]);
-                        int s = -tq_;
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t x[32];
+                    ft::tmem_ld32(tmem + lrow + ab * FT_NCOL + c0 + half * 32, x);
+                    tc::tmem_ld_wait();
+                    if (half == 1) {
+                        tc::fence_before_sync();
+                        __syncwarp();
+                        if (lane == 0) atc::arrive(acc_free + ab);
+                    }
+                    constexpr int NQH = 32 / HI;              // queries in a half
+                    constexpr int NG = NQH < 8 ? NQH : 8;     // queries per group
+                    // per group: the sums first (independent chains), a keep
+                    // mask, then per query one warp ballot and one shared-memory
+                    // atomic by the lowest keeping lane
 #pragma unroll
-                        for (int h = 0; h < HI; ++h) s = __viaddmax_s32(s, (int)x[q * HI + h], s);
-                        const bool keep = (s >= 0) && (full || j < nc_u[q]);
-                        if (keep) {
-                            const int slot = atomicAdd(cnt_u + q, 1);
-                            if (slot < p.cand_cap) {
-                                const long long off = list0 + (long long)q * p.cand_cap + slot;
-                                p.cand_val[off] = s + tq_;
-                                p.cand_idx[off] = j;
+                    for (int g0 = 0; g0 < NQH; g0 += NG) {
+                        const int qb = half * NQH + g0;       // first query of the group (in this warp)
+                        int sc[NG];
+                        unsigned mask = 0u;
+                        if (fast) {
+#pragma unroll
+                            for (int qq = 0; qq < NG; ++qq) {
+                                const int tq_ = QREG ? tau_r[qb + qq] : ft_fast_tau(tau_u[qb + qq]);
+                                int sacc = -tq_;
+#pragma unroll
+                                for (int h = 0; h < HI; ++h)
+                                    sacc = __viaddmax_s32(sacc, (int)x[(g0 + qq) * HI + h], sacc);
+                                sc[qq] = sacc + tq_;
+                                mask |= (sacc >= 0) ? (1u << qq) : 0u;
+                            }
+                        } else {
+#pragma unroll
+                            for (int qq = 0; qq < NG; ++qq) {
+                                int sacc = 0;
+#pragma unroll
+                                for (int h = 0; h < HI; ++h)
+                                    sacc += w_u[(qb + qq) * HI + h] * max((int)x[(g0 + qq) * HI + h], 0);
+                                sc[qq] = sacc;
+                                mask |= (sacc >= (QREG ? tau_r[qb + qq] : tau_u[qb + qq])) ? (1u << qq) : 0u;
                             }
                         }
-                    }
-                } else {
+                        if (!full) {                           // diagonal tiles: causal bound per query
 #pragma unroll
-                    for (int q = 0; q < NQT; ++q) {
-                        int s = 0;
+                            for (int qq = 0; qq < NG; ++qq)
+                                if (j >= nc_u[qb + qq]) mask &= ~(1u << qq);
+                        }
 #pragma unroll
-                        for (int h = 0; h < HI; ++h) s += w_u[q * HI + h] * max((int)x[q * HI + h], 0);
-                        const bool keep = (s >= (QREG ? tau_r[q] : tau_u[q])) && (full || j < nc_u[q]);
-                        if (keep) {
-                            const int slot = atomicAdd(cnt_u + q, 1);
-                            if (slot < p.cand_cap) {
-                                const long long off = list0 + (long long)q * p.cand_cap + slot;
-                                p.cand_val[off] = s;
-                                p.cand_idx[off] = j;
+                        for (int qq = 0; qq < NG; ++qq) {
+                            const unsigned bal = __ballot_sync(0xffffffffu, (mask >> qq) & 1u);
+                            if (bal) {                         // warp-uniform
+                                const int leader = __ffs(bal) - 1;
+                                int base = 0;
+                                if (lane == leader) base = atomicAdd(cnt_u + qb + qq, __popc(bal));
+                                base = __shfl_sync(0xffffffffu, base, leader);
+                                const int slot = base + __popc(bal & lt);
+                                if (((mask >> qq) & 1u) && slot < p.cand_cap) {
+                                    const long long off = list0 + (long long)(qb + qq) * p.cand_cap + slot;
+                                    p.cand_val[off] = sc[qq];
+                                    p.cand_idx[off] = j;
+                                }
                             }
                         }
                     }

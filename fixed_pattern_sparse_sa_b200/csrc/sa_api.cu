@@ -107,13 +107,10 @@ static int sm_count() {
 // memory, one CTA and 12 gathering warps per SM.  Small launches (fewer
 // items than 12 per SM, e.g. decode with a few hundred split pieces) use
 // 4-warp CTAs so that every SM gets work.
-template <int D, int SRC, bool BIAS, bool KLO, int NW>
+template <int D, int SRC, bool BIAS, bool KLO, int NW, int STAGES_ = 2, int NK_ = 16>
 static int launch_gather_nw(const GatherParams &p, long long items, cudaStream_t st) {
-#ifndef SA_ATTN_STAGES
-#define SA_ATTN_STAGES 2
-#endif
-    constexpr int NK = 16;
-    constexpr int STAGES = KLO ? 2 : SA_ATTN_STAGES;
+    constexpr int NK = NK_;
+    constexpr int STAGES = KLO ? 2 : STAGES_;
     constexpr int smem = gather_smem_bytes<D, STAGES, KLO, NK, NW, SRC == KS_PROWS>();
     static_assert(smem <= 227 * 1024, "shared memory");
     auto kern = gather_attn_kernel<D, STAGES, SRC, BIAS, KLO, NK, NW>;
@@ -132,6 +129,21 @@ static int launch_gather_t(const GatherParams &p, cudaStream_t st) {
 #endif
     const long long items = (long long)p.B * p.q_units * p.Hkv * p.n_hchunk * p.n_split;
     if (items == 0) return SA_OK;
+    if constexpr (SRC == KS_IDX && D == 128 && !BIAS && !KLO) {
+        // ring depth / warps per CTA of the explicit-list kernel: SA_ATTN_CFG
+        // = "9x3" (9 warps, 3 stages), "6x4", "4x3w" (32-key chunks);
+        // default 12 warps x 2 stages of 16 keys
+        static int cfg = -1;
+        if (cfg < 0) {
+            const char *e = std::getenv("SA_ATTN_CFG");
+            cfg = !e ? 0 : !std::strcmp(e, "9x3") ? 1 : !std::strcmp(e, "6x4") ? 2 : !std::strcmp(e, "4x3w") ? 3 : 0;
+        }
+        if (items >= (long long)sm_count() * SA_ATTN_NW) {
+            if (cfg == 1) return launch_gather_nw<D, SRC, BIAS, KLO, 9, 3, 16>(p, items, st);
+            if (cfg == 2) return launch_gather_nw<D, SRC, BIAS, KLO, 6, 4, 16>(p, items, st);
+            if (cfg == 3) return launch_gather_nw<D, SRC, BIAS, KLO, 4, 3, 32>(p, items, st);
+        }
+    }
     if constexpr (KLO) {
         return launch_gather_nw<D, SRC, BIAS, KLO, 8>(p, items, st);
     } else {
@@ -352,10 +364,13 @@ int64_t sa_debug_exact_recompute_rows(void) {
 }
 
 // ------------------------------------------------------ sparse attention --
+// Split-KV workspace: partial rows, partial LSEs and one arrival ticket per
+// (b, t, KV group, 16-head chunk) -- at most B * Tq * Hq of them.
 size_t sa_sparse_attn_workspace_size(int B, int Tq, int Hq, int d, int n_split) {
     if (n_split <= 1 || B <= 0 || Tq <= 0 || Hq <= 0 || d <= 0) return 0;
     const size_t rows = (size_t)B * Tq * Hq;
-    return round_up((size_t)n_split * rows * d * 4, 256) + round_up((size_t)n_split * rows * 4, 256);
+    return round_up((size_t)n_split * rows * d * 4, 256) + round_up((size_t)n_split * rows * 4, 256) +
+           round_up(rows * 4, 256);
 }
 
 int sa_sparse_attn_fwd(const void *q, const void *k, const void *v, int B, int Tq, int L, int Hq,
@@ -395,14 +410,17 @@ int sa_sparse_attn_fwd(const void *q, const void *k, const void *v, int B, int T
 
     const long long rows = (long long)B * Tq * Hq;
     float *po = part_o, *pl = part_lse;
+    int *tickets = nullptr;
     if (n_split > 1 && (!po || !pl)) {
         const size_t need = sa_sparse_attn_workspace_size(B, Tq, Hq, d, n_split);
         if (!workspace || workspace_bytes < need)
             return fail(SA_ERR_WORKSPACE, "sparse_attn: workspace %zu < %zu", workspace_bytes, need);
         if (!aligned16(workspace)) return fail(SA_ERR_INVALID_ARG, "sparse_attn: workspace alignment");
+        const size_t o_bytes = round_up((size_t)n_split * rows * d * 4, 256);
         po = static_cast<float *>(workspace);
-        pl = reinterpret_cast<float *>(static_cast<char *>(workspace) +
-                                       round_up((size_t)n_split * rows * d * 4, 256));
+        pl = reinterpret_cast<float *>(static_cast<char *>(workspace) + o_bytes);
+        tickets = reinterpret_cast<int *>(static_cast<char *>(workspace) + o_bytes +
+                                          round_up((size_t)n_split * rows * 4, 256));
     }
     if (n_split > 1 && (!aligned16(po) || !aligned4(pl)))
         return fail(SA_ERR_INVALID_ARG, "sparse_attn: partial buffers alignment");
@@ -444,9 +462,18 @@ int sa_sparse_attn_fwd(const void *q, const void *k, const void *v, int B, int T
     p.part_o = po; p.part_lse = pl;
     p.err = ew;
     cudaStream_t st = as_stream(stream);
-    rc = attn_tc_applies(p, d, src, bias) ? launch_attn_tc<KS_IDX>(p, st) : launch_gather(p, d, src, bias, st);
+    const bool tc = attn_tc_applies(p, d, src, bias);
+    // with a ticket array the gather kernel's last piece of each group does
+    // the merge itself (no separate combine launch)
+    if (!tc && n_split > 1 && out && tickets) {
+        const size_t nt = (size_t)B * Tq * Hkv * p.n_hchunk;
+        cudaError_t e = cudaMemsetAsync(tickets, 0, nt * 4, st);
+        if (e != cudaSuccess) return fail(SA_ERR_CUDA, "sparse_attn tickets: %s", cudaGetErrorString(e));
+        p.merge_cnt = tickets;
+    }
+    rc = tc ? launch_attn_tc<KS_IDX>(p, st) : launch_gather(p, d, src, bias, st);
     if (rc) return rc;
-    if (n_split > 1 && out) return launch_combine(po, pl, n_split, rows, d, out, lse, st);
+    if (n_split > 1 && out && !p.merge_cnt) return launch_combine(po, pl, n_split, rows, d, out, lse, st);
     return SA_OK;
 }
 

@@ -46,7 +46,8 @@ def test_workspace_queries(lib):
     n = lib.sa_indexer_topk_workspace_size(1, 512, 512, 2, 32, 64, 32)
     assert n > 0 and n % 256 == 0
     assert lib.sa_sparse_attn_workspace_size(2, 3, 4, 64, 1) == 0
-    assert lib.sa_sparse_attn_workspace_size(2, 3, 4, 64, 4) == 4 * 24 * 64 * 4 + 512   # partials + lse (384 B rounded to 256)
+    # partials + lse (384 B rounded to 512) + one merge ticket per row (96 B rounded to 256)
+    assert lib.sa_sparse_attn_workspace_size(2, 3, 4, 64, 4) == 4 * 24 * 64 * 4 + 512 + 256
     assert lib.sa_nsa_workspace_size(1, 1024, 16, 1, 64, 32, 16, 64, 16) > 0
     assert lib.sa_indexer_topk_workspace_size(0, 1, 1, 2, 32, 1, 0) == 0
 
