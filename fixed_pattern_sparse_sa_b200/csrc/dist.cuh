@@ -66,7 +66,7 @@ __global__ void __launch_bounds__(TM_THREADS) topk_merge_kernel(const int32_t *c
                                                                  const MergeOffsets part_off, int n_parts, long long rows,
                                                                  int kc, int topk, int window, long long q_pos,
                                                                  int32_t *out_idx, int32_t *out_count) {
-    extern __shared__ __align__(16) unsigned char smem[];
+    extern __shared__ __align__(1024) unsigned char smem[];
     const int n = n_parts * kc;
     int *sv = reinterpret_cast<int *>(smem);                  // [n] scores
     int *sj = sv + n;                                         // [n] global positions (-1: none)
