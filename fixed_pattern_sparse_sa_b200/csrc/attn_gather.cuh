@@ -194,9 +194,11 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
     extern __shared__ __align__(1024) unsigned char smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr bool PR = SRC == KS_PROWS;
-    unsigned char *wsm = smem + warp * (STAGES * (SB + NK * (PR ? 8 : 4)));
+    constexpr int KEYB = NK * ((PR ? 8 : 4) + (BIAS ? 12 : 0));   // per stage: keys (+ segments, + coordinates)
+    unsigned char *wsm = smem + warp * (STAGES * (SB + KEYB));
     int *keys_s = reinterpret_cast<int *>(wsm + STAGES * SB);
     int *segs_s = keys_s + STAGES * NK;                      // KS_PROWS only
+    float *ck_s = reinterpret_cast<float *>(keys_s + STAGES * NK * (PR ? 2 : 1));   // [STAGES][NK][3] (bias only)
 
     const long long n_items = (long long)p.B * p.q_units * p.Hkv * p.n_hchunk * p.n_split;
     const long long item = (long long)blockIdx.x * NW + warp;
@@ -278,6 +280,16 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
         if (lane < NK) {
             keys_s[st * NK + lane] = j;
             if constexpr (PR) segs_s[st * NK + lane] = seg;
+            if constexpr (BIAS) {
+                // the key's coordinates ride with its K/V rows (same commit group)
+                if (j >= 0) {
+                    const float *c = p.ck + ((long long)(b * p.Lk + j) * p.Hkv + g) * 3;
+                    float *dst = ck_s + (st * NK + lane) * 3;
+                    cp_async4(dst, c);
+                    cp_async4(dst + 1, c + 1);
+                    cp_async4(dst + 2, c + 2);
+                }
+            }
         }
         if (ci < n_chunks) {
 #pragma unroll
@@ -361,10 +373,9 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
                     if constexpr (BIAS) {
                         const int jk = __shfl_sync(0xffffffffu, jl, kk);
                         if (jk >= 0) {
-                            const float *c = p.ck + ((long long)(b * p.Lk + jk) * p.Hkv + g) * 3;
+                            const float *c = ck_s + (st * NK + kk) * 3;
                             const float *a = (e >> 1) ? cq1 : cq0;
-                            const float dx = a[0] - __ldg(c), dy = a[1] - __ldg(c + 1),
-                                        dz = a[2] - __ldg(c + 2);
+                            const float dx = a[0] - c[0], dy = a[1] - c[1], dz = a[2] - c[2];
                             x -= ((e >> 1) ? be1 : be0) * (dx * dx + dy * dy + dz * dz);
                         }
                     }
@@ -511,9 +522,9 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
     }
 }
 
-template <int D, int STAGES, bool KLO = false, int NK = 32, int NW = 4, bool PR = false>
+template <int D, int STAGES, bool KLO = false, int NK = 32, int NW = 4, bool PR = false, bool BIAS = false>
 constexpr int gather_smem_bytes() {
-    return NW * STAGES * ((KLO ? 3 : 2) * NK * D * 2 + NK * (PR ? 8 : 4));
+    return NW * STAGES * ((KLO ? 3 : 2) * NK * D * 2 + NK * ((PR ? 8 : 4) + (BIAS ? 12 : 0)));
 }
 
 }  // namespace sa

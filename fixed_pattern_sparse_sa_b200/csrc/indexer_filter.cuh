@@ -410,20 +410,27 @@ __global__ void __launch_bounds__(FT_THREADS, 1)
                             for (int qq = 0; qq < NG; ++qq)
                                 if (j >= nc_u[qb + qq]) mask &= ~(1u << qq);
                         }
+                        // one ballot per query; lane qq reserves the group's
+                        // slots of query qq (one atomic instruction for the
+                        // whole group, distinct addresses), then every lane
+                        // writes its kept pairs
+                        unsigned bal[NG];
+                        int mycnt = 0;
 #pragma unroll
                         for (int qq = 0; qq < NG; ++qq) {
-                            const unsigned bal = __ballot_sync(0xffffffffu, (mask >> qq) & 1u);
-                            if (bal) {                         // warp-uniform
-                                const int leader = __ffs(bal) - 1;
-                                int base = 0;
-                                if (lane == leader) base = atomicAdd(cnt_u + qb + qq, __popc(bal));
-                                base = __shfl_sync(0xffffffffu, base, leader);
-                                const int slot = base + __popc(bal & lt);
-                                if (((mask >> qq) & 1u) && slot < p.cand_cap) {
-                                    const long long off = list0 + (long long)(qb + qq) * p.cand_cap + slot;
-                                    p.cand_val[off] = sc[qq];
-                                    p.cand_idx[off] = j;
-                                }
+                            bal[qq] = __ballot_sync(0xffffffffu, (mask >> qq) & 1u);
+                            mycnt = lane == qq ? __popc(bal[qq]) : mycnt;
+                        }
+                        int mybase = 0;
+                        if (mycnt > 0) mybase = atomicAdd(cnt_u + qb + lane, mycnt);
+#pragma unroll
+                        for (int qq = 0; qq < NG; ++qq) {
+                            if (bal[qq] == 0u) continue;       // warp-uniform
+                            const int slot = __shfl_sync(0xffffffffu, mybase, qq) + __popc(bal[qq] & lt);
+                            if (((mask >> qq) & 1u) && slot < p.cand_cap) {
+                                const long long off = list0 + (long long)(qb + qq) * p.cand_cap + slot;
+                                p.cand_val[off] = sc[qq];
+                                p.cand_idx[off] = j;
                             }
                         }
                     }

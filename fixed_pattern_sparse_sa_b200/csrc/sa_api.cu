@@ -111,7 +111,7 @@ template <int D, int SRC, bool BIAS, bool KLO, int NW, int STAGES_ = 2, int NK_ 
 static int launch_gather_nw(const GatherParams &p, long long items, cudaStream_t st) {
     constexpr int NK = NK_;
     constexpr int STAGES = KLO ? 2 : STAGES_;
-    constexpr int smem = gather_smem_bytes<D, STAGES, KLO, NK, NW, SRC == KS_PROWS>();
+    constexpr int smem = gather_smem_bytes<D, STAGES, KLO, NK, NW, SRC == KS_PROWS, BIAS>();
     static_assert(smem <= 227 * 1024, "shared memory");
     auto kern = gather_attn_kernel<D, STAGES, SRC, BIAS, KLO, NK, NW>;
     int rc = set_smem(kern, smem);
