@@ -174,6 +174,8 @@ def main():
                              "spatial16k"],
                     help="run only one of the extra measurements (for profiling captures of a "
                          "single workload); prints its numbers alone")
+    ap.add_argument("--decode-split", type=int, default=16,
+                    help="split-KV pieces per decode row (the 2048 selected keys are cut into this many)")
     ap.add_argument("--cpu-sample-rows", type=int, default=0,
                     help="oracle rows for the CPU baseline (0 = auto, ~10-30 s)")
     args = ap.parse_args()
@@ -386,7 +388,7 @@ def extra_measurements(args, dev, torch, api, lib, inputs, flush, world, peaks, 
         w = inputs.WORKLOADS["dsa_decode128k"]
         lays = [inputs.gen_decode_layer(w.B, w.T, w.Hq, w.Hkv, w.d, w.Hi, w.di, layer=i, seed=0,
                                         device=dev) for i in range(w.layers)]
-        n_split = 16
+        n_split = args.decode_split
         outs = [torch.empty((w.B, 1, w.Hq, w.d), dtype=torch.bfloat16, device=dev) for _ in lays]
         lses = [torch.empty((w.B, 1, w.Hq), dtype=torch.float32, device=dev) for _ in lays]
         cache = torch.empty((w.B, 1, w.topk), dtype=torch.int32, device=dev)
@@ -417,6 +419,7 @@ def extra_measurements(args, dev, torch, api, lib, inputs, flush, world, peaks, 
                             "hbm_frac": round(bytes_step / (ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4)}
             del graph
         dec["fsss_over_ffff"] = round(dec["FSSS"]["tokens_per_s"] / dec["FFFF"]["tokens_per_s"], 3)
+        dec["n_split"] = n_split
         res["decode128k"] = dec
         del lays, wsd
         torch.cuda.empty_cache()

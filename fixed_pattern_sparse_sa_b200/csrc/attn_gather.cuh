@@ -13,7 +13,10 @@
 
 #include <climits>
 
+#include <cuda.h>
+
 #include "sa_common.cuh"
+#include "tc_common.cuh"
 
 namespace sa {
 
@@ -180,8 +183,14 @@ __device__ __forceinline__ void merge_pieces_half(const float *part_o, const flo
 // KLO: keys are held as a bf16 pair (hi, lo) whose sum carries ~16 mantissa
 // bits; q.k is taken on both halves (used for the NSA compressed keys, which
 // are means and do not fit bf16 exactly).
-template <int D, int STAGES, int SRC, bool BIAS, bool KLO = false, int NK = 32, int NW = 4>
-__global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams p) {
+// TMAB (NSA selected blocks, head dim 128): the chunk's 16 consecutive rows of
+// a block arrive by TMA box loads (kmap / vmap: [B*Lk rows, Hkv, D], box = 64
+// columns x 1 head x 16 rows, 128-byte swizzle) issued by lane 0, completion
+// on a per-warp mbarrier; a K (or V) chunk is then two 64-column halves of
+// 16 rows x 128 B instead of 16 rows x 256 B.
+template <int D, int STAGES, int SRC, bool BIAS, bool KLO = false, int NK = 32, int NW = 4, bool TMAB = false>
+__global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams p, const __grid_constant__ CUtensorMap kmap,
+                                                              const __grid_constant__ CUtensorMap vmap) {
     // NK keys per chunk, NW independent warps per CTA
     constexpr int ROWB = D * 2;            // bytes of one K/V row
     constexpr int UNITS = ROWB / 16;       // 16-byte units per row
@@ -190,15 +199,33 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
     constexpr int NT_D = D / 8;            // n-tiles of P.V
     constexpr int CP_ITERS = NK * UNITS / 32;
     constexpr int SB = (KLO ? 3 : 2) * CH;   // one stage: K | V | (K lo)
+    static_assert(!TMAB || (SRC == KS_BLOCKS && D == 128 && NK == 16 && !KLO && !BIAS), "TMA block chunks");
 
-    extern __shared__ __align__(1024) unsigned char smem[];
+    extern __shared__ __align__(1024) unsigned char smem_dyn[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr bool PR = SRC == KS_PROWS;
     constexpr int KEYB = NK * ((PR ? 8 : 4) + (BIAS ? 12 : 0));   // per stage: keys (+ segments, + coordinates)
-    unsigned char *wsm = smem + warp * (STAGES * (SB + KEYB));
-    int *keys_s = reinterpret_cast<int *>(wsm + STAGES * SB);
+    // TMA layout: every warp's stages first (1024-byte aligned for the 128-byte
+    // swizzle), then the keys, then one mbarrier per stage and warp
+    unsigned char *smem = TMAB ? smem_dyn + ((1024u - (tc::smem_u32(smem_dyn) & 1023u)) & 1023u) : smem_dyn;
+    unsigned char *wsm = TMAB ? smem + warp * (STAGES * SB) : smem + warp * (STAGES * (SB + KEYB));
+    int *keys_s = TMAB ? reinterpret_cast<int *>(smem + NW * STAGES * SB) + warp * STAGES * NK
+                       : reinterpret_cast<int *>(wsm + STAGES * SB);
+    uint64_t *full_s = reinterpret_cast<uint64_t *>(smem + NW * STAGES * (SB + NK * 4)) + warp * STAGES;
     int *segs_s = keys_s + STAGES * NK;                      // KS_PROWS only
     float *ck_s = reinterpret_cast<float *>(keys_s + STAGES * NK * (PR ? 2 : 1));   // [STAGES][NK][3] (bias only)
+    // byte offset of 16-byte unit u of key row `key` in a K / V chunk
+    auto kv_off = [](int key, int unit) -> int {
+        return TMAB ? (unit >> 3) * (NK * 128) + key * 128 + (((unit & 7) ^ (key & 7)) << 4)
+                    : key * ROWB + ((unit ^ (key & 7)) << 4);
+    };
+    if constexpr (TMAB) {
+        if (lane == 0) {
+            for (int i = 0; i < STAGES; ++i) tc::mbar_init(full_s + i, 1);
+            tc::mbar_fence_init();
+        }
+        __syncwarp();
+    }
 
     const long long n_items = (long long)p.B * p.q_units * p.Hkv * p.n_hchunk * p.n_split;
     const long long item = (long long)blockIdx.x * NW + warp;
@@ -291,6 +318,34 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
                 }
             }
         }
+        if constexpr (TMAB) {
+            // the chunk's 16 rows are consecutive rows of one block: four box
+            // loads (K and V, two 64-column halves each); a chunk without a
+            // valid block loads block 0 so masked rows stay finite
+            if (ci < n_chunks && lane == 0) {
+                const int e0 = e_beg + ci * NK;
+                int blk = raw;                                   // lane 0's raw list value: the block id
+                if (blk == KEY_NONE || blk < 0 || (long long)blk * p.block >= p.Lk) blk = 0;
+                const int z = b * p.Lk + blk * p.block + (e0 % p.block);
+                tc::fence_proxy_async_smem();                    // the stage's last readers are done (syncwarp)
+                asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(tc::smem_u32(full_s + st)),
+                             "r"(2 * CH)
+                             : "memory");
+                for (int h = 0; h < 2; ++h) {
+                    asm volatile(
+                        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+                        " [%0], [%1, {%2, %3, %4}], [%5];\n" ::"r"(tc::smem_u32(ks_ + h * (NK * 128))),
+                        "l"(reinterpret_cast<uint64_t>(&kmap)), "r"(h * 64), "r"(g), "r"(z), "r"(tc::smem_u32(full_s + st))
+                        : "memory");
+                    asm volatile(
+                        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+                        " [%0], [%1, {%2, %3, %4}], [%5];\n" ::"r"(tc::smem_u32(vs_ + h * (NK * 128))),
+                        "l"(reinterpret_cast<uint64_t>(&vmap)), "r"(h * 64), "r"(g), "r"(z), "r"(tc::smem_u32(full_s + st))
+                        : "memory");
+                }
+            }
+            return;
+        }
         if (ci < n_chunks) {
 #pragma unroll
             for (int it = 0; it < CP_ITERS; ++it) {
@@ -312,6 +367,7 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
 #pragma unroll
     for (int i = 0; i < NT_D; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+    bool timed_out = false;
 
 #pragma unroll
     for (int ci = 0; ci < STAGES - 1; ++ci) issue(ci, raw_of(ci));
@@ -323,9 +379,19 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
         raw_a = raw_b;
         raw_b = raw_of(ci + STAGES + 1);
         issue(ci + STAGES - 1, raw);
-        cp_async_wait<STAGES - 1>();
-        __syncwarp();
         const int st = ci % STAGES;
+        if constexpr (TMAB) {
+            // every lane waits for the chunk's bytes (bounded); a timeout is
+            // recorded and the data is ignored, the CTA drains before exit
+            const bool got = __all_sync(0xffffffffu, tc::mbar_wait_bounded(full_s + st, (ci / STAGES) & 1, spin_limit()));
+            if (!got && !timed_out) {
+                timed_out = true;
+                if (lane == 0) raise_error(p.err, ERR_TIMEOUT);
+            }
+        } else {
+            cp_async_wait<STAGES - 1>();
+        }
+        __syncwarp();
         const unsigned char *ks_ = wsm + st * SB;
         const unsigned char *vs_ = ks_ + CH;
         const int jl = lane < NK ? keys_s[st * NK + lane] : -1;
@@ -347,11 +413,11 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
                     const int key = np * 16 + (mi >> 1) * 8 + ri;
                     const int unit = ks * 2 + (mi & 1);
                     unsigned b0, b1, b2, b3;
-                    ldsm_x4(b0, b1, b2, b3, ks_ + key * ROWB + ((unit ^ (key & 7)) * 16));
+                    ldsm_x4(b0, b1, b2, b3, ks_ + kv_off(key, unit));
                     mma_bf16_16816(acc[2 * np], qf[ks], b0, b1);
                     mma_bf16_16816(acc[2 * np + 1], qf[ks], b2, b3);
                     if constexpr (KLO) {
-                        ldsm_x4(b0, b1, b2, b3, vs_ + CH + key * ROWB + ((unit ^ (key & 7)) * 16));
+                        ldsm_x4(b0, b1, b2, b3, vs_ + CH + kv_off(key, unit));
                         mma_bf16_16816(acc[2 * np], qf[ks], b0, b1);
                         mma_bf16_16816(acc[2 * np + 1], qf[ks], b2, b3);
                     }
@@ -437,7 +503,7 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
                     const int key = kp * 16 + (mi & 1) * 8 + ri;
                     const int unit = dp * 2 + (mi >> 1);
                     unsigned b0, b1, b2, b3;
-                    ldsm_x4_t(b0, b1, b2, b3, vs_ + key * ROWB + ((unit ^ (key & 7)) * 16));
+                    ldsm_x4_t(b0, b1, b2, b3, vs_ + kv_off(key, unit));
                     mma_bf16_16816(o[2 * dp], pa, b0, b1);
                     mma_bf16_16816(o[2 * dp + 1], pa, b2, b3);
                 }
@@ -446,6 +512,15 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
         __syncwarp();
     }
     cp_async_wait<0>();
+    if constexpr (TMAB) {
+        // after a timeout some loads may still be in flight: let every
+        // stage's latest phase complete (fixed long limit) before exiting
+        if (timed_out && lane == 0) {
+            for (int ci = (n_chunks > STAGES ? n_chunks - STAGES : 0); ci < n_chunks; ++ci)
+                tc::mbar_wait_bounded(full_s + ci % STAGES, (ci / STAGES) & 1, kDefaultSpinCycles);
+        }
+        __syncwarp();
+    }
 
     l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
     l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
@@ -522,9 +597,11 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
     }
 }
 
-template <int D, int STAGES, bool KLO = false, int NK = 32, int NW = 4, bool PR = false, bool BIAS = false>
+template <int D, int STAGES, bool KLO = false, int NK = 32, int NW = 4, bool PR = false, bool BIAS = false,
+          bool TMAB = false>
 constexpr int gather_smem_bytes() {
-    return NW * STAGES * ((KLO ? 3 : 2) * NK * D * 2 + NK * ((PR ? 8 : 4) + (BIAS ? 12 : 0)));
+    return NW * STAGES * ((KLO ? 3 : 2) * NK * D * 2 + NK * ((PR ? 8 : 4) + (BIAS ? 12 : 0))) +
+           (TMAB ? NW * STAGES * 8 + 1024 : 0);
 }
 
 }  // namespace sa

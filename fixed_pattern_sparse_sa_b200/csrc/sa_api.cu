@@ -101,78 +101,7 @@ static int sm_count() {
     return cached[dev];
 }
 
-// -------------------------------------------------------- gather launches --
-// Launch shape: 12 warps per CTA streaming 16-key chunks through a 2-stage
-// ring (8 warps when the lo-key tile is also staged); ~198 KB of shared
-// memory, one CTA and 12 gathering warps per SM.  Small launches (fewer
-// items than 12 per SM, e.g. decode with a few hundred split pieces) use
-// 4-warp CTAs so that every SM gets work.
-template <int D, int SRC, bool BIAS, bool KLO, int NW, int STAGES_ = 2, int NK_ = 16>
-static int launch_gather_nw(const GatherParams &p, long long items, cudaStream_t st) {
-    constexpr int NK = NK_;
-    constexpr int STAGES = KLO ? 2 : STAGES_;
-    constexpr int smem = gather_smem_bytes<D, STAGES, KLO, NK, NW, SRC == KS_PROWS, BIAS>();
-    static_assert(smem <= 227 * 1024, "shared memory");
-    auto kern = gather_attn_kernel<D, STAGES, SRC, BIAS, KLO, NK, NW>;
-    int rc = set_smem(kern, smem);
-    if (rc) return rc;
-    const long long blocks = (items + NW - 1) / NW;
-    kern<<<(unsigned)blocks, NW * 32, smem, st>>>(p);
-    SA_CHECK_LAUNCH("gather_attn_kernel");
-    return SA_OK;
-}
-
-template <int D, int SRC, bool BIAS, bool KLO = false>
-static int launch_gather_t(const GatherParams &p, cudaStream_t st) {
-#ifndef SA_ATTN_NW
-#define SA_ATTN_NW 12
-#endif
-    const long long items = (long long)p.B * p.q_units * p.Hkv * p.n_hchunk * p.n_split;
-    if (items == 0) return SA_OK;
-    if constexpr (SRC == KS_IDX && D == 128 && !BIAS && !KLO) {
-        // ring depth / warps per CTA of the explicit-list kernel: SA_ATTN_CFG
-        // = "9x3" (9 warps, 3 stages), "6x4", "4x3w" (32-key chunks);
-        // default 12 warps x 2 stages of 16 keys
-        static int cfg = -1;
-        if (cfg < 0) {
-            const char *e = std::getenv("SA_ATTN_CFG");
-            cfg = !e ? 0 : !std::strcmp(e, "9x3") ? 1 : !std::strcmp(e, "6x4") ? 2 : !std::strcmp(e, "4x3w") ? 3 : 0;
-        }
-        if (items >= (long long)sm_count() * SA_ATTN_NW) {
-            if (cfg == 1) return launch_gather_nw<D, SRC, BIAS, KLO, 9, 3, 16>(p, items, st);
-            if (cfg == 2) return launch_gather_nw<D, SRC, BIAS, KLO, 6, 4, 16>(p, items, st);
-            if (cfg == 3) return launch_gather_nw<D, SRC, BIAS, KLO, 4, 3, 32>(p, items, st);
-        }
-    }
-    if constexpr (KLO) {
-        return launch_gather_nw<D, SRC, BIAS, KLO, 8>(p, items, st);
-    } else {
-        if (items < (long long)sm_count() * SA_ATTN_NW) return launch_gather_nw<D, SRC, BIAS, KLO, 4>(p, items, st);
-        return launch_gather_nw<D, SRC, BIAS, KLO, SA_ATTN_NW>(p, items, st);
-    }
-}
-
-template <int D>
-static int launch_gather_d(const GatherParams &p, int src, bool bias, cudaStream_t st) {
-    switch (src) {
-        case KS_IDX: return bias ? launch_gather_t<D, KS_IDX, true>(p, st) : launch_gather_t<D, KS_IDX, false>(p, st);
-        case KS_PATTERN:
-            return bias ? launch_gather_t<D, KS_PATTERN, true>(p, st) : launch_gather_t<D, KS_PATTERN, false>(p, st);
-        case KS_BLOCKS: return launch_gather_t<D, KS_BLOCKS, false>(p, st);
-        case KS_RANGE: return launch_gather_t<D, KS_RANGE, false>(p, st);
-        case KS_PROWS:
-            return bias ? launch_gather_t<D, KS_PROWS, true>(p, st) : launch_gather_t<D, KS_PROWS, false>(p, st);
-    }
-    return fail(SA_ERR_UNSUPPORTED, "key source %d", src);
-}
-
-static int launch_gather(const GatherParams &p, int d, int src, bool bias, cudaStream_t st) {
-    if (d == 64) return launch_gather_d<64>(p, src, bias, st);
-    if (d == 128) return launch_gather_d<128>(p, src, bias, st);
-    return fail(SA_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
-}
-
-// ------------------------------------------- tensor-core gather launches --
+// ------------------------------------------------------------ tensor maps --
 typedef CUresult (*TensorMapEncodeFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                       const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
                                       CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
@@ -226,6 +155,104 @@ static int bf16_tensor_map_3d(CUtensorMap *m, const void *base, int d, int hkv, 
     if (r != CUDA_SUCCESS) return fail(SA_ERR_CUDA, "cuTensorMapEncodeTiled(3d) failed (%d)", (int)r);
     return SA_OK;
 }
+
+// SA_GATHER_TMA=0 keeps the NSA selected branch on per-row cp.async copies
+// (for comparison); by default its 16-row block chunks come by TMA.
+static bool gather_tma_allowed() {
+    static int v = -1;
+    if (v < 0) {
+        const char *e = std::getenv("SA_GATHER_TMA");
+        v = (e && std::strcmp(e, "0") == 0) ? 0 : 1;
+    }
+    return v != 0;
+}
+
+// -------------------------------------------------------- gather launches --
+// Launch shape: 12 warps per CTA streaming 16-key chunks through a 2-stage
+// ring (8 warps when the lo-key tile is also staged); ~198 KB of shared
+// memory, one CTA and 12 gathering warps per SM.  Small launches (fewer
+// items than 12 per SM, e.g. decode with a few hundred split pieces) use
+// 4-warp CTAs so that every SM gets work.
+template <int D, int SRC, bool BIAS, bool KLO, int NW, int STAGES_ = 2, int NK_ = 16, bool TMAB = false>
+static int launch_gather_nw(const GatherParams &p, long long items, cudaStream_t st,
+                            const CUtensorMap *km = nullptr, const CUtensorMap *vm = nullptr) {
+    constexpr int NK = NK_;
+    constexpr int STAGES = KLO ? 2 : STAGES_;
+    constexpr int smem = gather_smem_bytes<D, STAGES, KLO, NK, NW, SRC == KS_PROWS, BIAS, TMAB>();
+    static_assert(smem <= 227 * 1024, "shared memory");
+    auto kern = gather_attn_kernel<D, STAGES, SRC, BIAS, KLO, NK, NW, TMAB>;
+    int rc = set_smem(kern, smem);
+    if (rc) return rc;
+    static const CUtensorMap unused{};                   // the row-gather modes take no tensor map
+    const long long blocks = (items + NW - 1) / NW;
+    kern<<<(unsigned)blocks, NW * 32, smem, st>>>(p, km ? *km : unused, vm ? *vm : unused);
+    SA_CHECK_LAUNCH("gather_attn_kernel");
+    return SA_OK;
+}
+
+template <int D, int SRC, bool BIAS, bool KLO = false>
+static int launch_gather_t(const GatherParams &p, cudaStream_t st) {
+#ifndef SA_ATTN_NW
+#define SA_ATTN_NW 12
+#endif
+    const long long items = (long long)p.B * p.q_units * p.Hkv * p.n_hchunk * p.n_split;
+    if (items == 0) return SA_OK;
+    if constexpr (SRC == KS_IDX && D == 128 && !BIAS && !KLO) {
+        // ring depth / warps per CTA of the explicit-list kernel: SA_ATTN_CFG
+        // = "9x3" (9 warps, 3 stages), "6x4", "4x3w" (32-key chunks);
+        // default 12 warps x 2 stages of 16 keys
+        static int cfg = -1;
+        if (cfg < 0) {
+            const char *e = std::getenv("SA_ATTN_CFG");
+            cfg = !e ? 0 : !std::strcmp(e, "9x3") ? 1 : !std::strcmp(e, "6x4") ? 2 : !std::strcmp(e, "4x3w") ? 3 : 0;
+        }
+        if (items >= (long long)sm_count() * SA_ATTN_NW) {
+            if (cfg == 1) return launch_gather_nw<D, SRC, BIAS, KLO, 9, 3, 16>(p, items, st);
+            if (cfg == 2) return launch_gather_nw<D, SRC, BIAS, KLO, 6, 4, 16>(p, items, st);
+            if (cfg == 3) return launch_gather_nw<D, SRC, BIAS, KLO, 4, 3, 32>(p, items, st);
+        }
+    }
+    if constexpr (SRC == KS_BLOCKS && D == 128 && !BIAS && !KLO) {
+        // NSA selected blocks: 16-row chunks of a block by TMA box loads
+        if (p.block % 16 == 0 && (long long)p.B * p.Lk < INT_MAX && items >= (long long)sm_count() * SA_ATTN_NW &&
+            gather_tma_allowed()) {
+            CUtensorMap km, vm;
+            int rc = bf16_tensor_map_3d(&km, p.k, 128, p.Hkv, (long long)p.B * p.Lk, 16);
+            if (rc) return rc;
+            rc = bf16_tensor_map_3d(&vm, p.v, 128, p.Hkv, (long long)p.B * p.Lk, 16);
+            if (rc) return rc;
+            return launch_gather_nw<D, SRC, BIAS, KLO, SA_ATTN_NW, 2, 16, true>(p, items, st, &km, &vm);
+        }
+    }
+    if constexpr (KLO) {
+        return launch_gather_nw<D, SRC, BIAS, KLO, 8>(p, items, st);
+    } else {
+        if (items < (long long)sm_count() * SA_ATTN_NW) return launch_gather_nw<D, SRC, BIAS, KLO, 4>(p, items, st);
+        return launch_gather_nw<D, SRC, BIAS, KLO, SA_ATTN_NW>(p, items, st);
+    }
+}
+
+template <int D>
+static int launch_gather_d(const GatherParams &p, int src, bool bias, cudaStream_t st) {
+    switch (src) {
+        case KS_IDX: return bias ? launch_gather_t<D, KS_IDX, true>(p, st) : launch_gather_t<D, KS_IDX, false>(p, st);
+        case KS_PATTERN:
+            return bias ? launch_gather_t<D, KS_PATTERN, true>(p, st) : launch_gather_t<D, KS_PATTERN, false>(p, st);
+        case KS_BLOCKS: return launch_gather_t<D, KS_BLOCKS, false>(p, st);
+        case KS_RANGE: return launch_gather_t<D, KS_RANGE, false>(p, st);
+        case KS_PROWS:
+            return bias ? launch_gather_t<D, KS_PROWS, true>(p, st) : launch_gather_t<D, KS_PROWS, false>(p, st);
+    }
+    return fail(SA_ERR_UNSUPPORTED, "key source %d", src);
+}
+
+static int launch_gather(const GatherParams &p, int d, int src, bool bias, cudaStream_t st) {
+    if (d == 64) return launch_gather_d<64>(p, src, bias, st);
+    if (d == 128) return launch_gather_d<128>(p, src, bias, st);
+    return fail(SA_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
+}
+
+// ------------------------------------------- tensor-core gather launches --
 
 // SA_ATTN_PATH=tc routes explicit-list attention (head dim 128, <= 16 heads
 // per KV head, no bias) through attn_tc_kernel.  It is opt-in: with 64-KB
