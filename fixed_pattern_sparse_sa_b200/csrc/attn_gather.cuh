@@ -99,18 +99,18 @@ __device__ __forceinline__ int key_raw(const GatherParams &p, int b, int t, int 
 
 // KS_PROWS: entry e of the union for queries at positions [pa, pb]; returns
 // the key (or -1) and, in seg, 0 for the window band or the dilated distance.
-__device__ __forceinline__ int key_prows(const GatherParams &p, long long pa, long long pb, int nqw, int e,
+// i0 = the first dilated exponent (2^i0 >= window), lq = log2(nqw): both
+// per-kernel constants (nqw = 16 / G is a power of two).
+__device__ __forceinline__ int key_prows(const GatherParams &p, long long pa, long long pb, int lq, int i0, int e,
                                          int e_end, int &seg) {
     seg = 0;
     if (e >= e_end) return -1;
     const long long lo = pa - p.window + 1 > 0 ? pa - p.window + 1 : 0;
-    const long long nb = pb - lo + 1;
+    const int nb = (int)(pb - lo + 1);
     if (e < nb) return (int)(lo + e);
     if (!p.dilated) return -1;
-    int i0 = 0;
-    while ((1LL << i0) < p.window) ++i0;
-    const long long e2 = e - nb;
-    const long long m = e2 / nqw, r = e2 % nqw;
+    const int e2 = e - nb;
+    const int m = e2 >> lq, r = e2 & ((1 << lq) - 1);
     if (i0 + m >= 62) return -1;
     const long long o = 1LL << (i0 + m);
     if (o >= pb) return -1;
@@ -145,24 +145,33 @@ __device__ __forceinline__ int key_finish(const GatherParams &p, long long pos, 
     }
 }
 
-// Log-sum-exp merge of one output row's n_split pieces (Star Attention page,
-// body: distributed softmax), over D/2 columns starting at c0; the pieces
-// were written by other CTAs of the same launch, so they are read through L2.
+// Log-sum-exp merge of the output rows of one item group (Star Attention
+// page, body: distributed softmax) by the warp whose piece arrived last: lane
+// l takes head row l / 2 of the group, columns (l % 2) * D/2 .. + D/2.  The
+// pieces were written by other CTAs of the same launch, so they are read
+// through L2; the LSEs of every piece first (up to 32, independent loads),
+// then the partial rows with several pieces' loads in flight.
 template <int D>
 __device__ __forceinline__ void merge_pieces_half(const float *part_o, const float *part_lse, int n_split,
                                                   long long rows, long long row, int c0, __nv_bfloat16 *out,
                                                   float *lse) {
+    constexpr int MAXS = 32;
+    float ls[MAXS];
     float m = -INFINITY;
-    for (int s = 0; s < n_split; ++s) m = fmaxf(m, __ldcg(part_lse + s * rows + row));
+#pragma unroll
+    for (int s = 0; s < MAXS; ++s) {
+        ls[s] = s < n_split ? __ldcg(part_lse + s * rows + row) : -INFINITY;
+        m = fmaxf(m, ls[s]);
+    }
     float acc[D / 2];
 #pragma unroll
     for (int i = 0; i < D / 2; ++i) acc[i] = 0.f;
     float den = 0.f;
     if (m != -INFINITY) {
-        for (int s = 0; s < n_split; ++s) {
-            const float ls = __ldcg(part_lse + s * rows + row);
-            if (ls == -INFINITY) continue;
-            const float f = exp2f((ls - m) * kLog2e);
+#pragma unroll
+        for (int s = 0; s < MAXS; ++s) {
+            if (s >= n_split || ls[s] == -INFINITY) continue;
+            const float f = exp2f((ls[s] - m) * kLog2e);
             den += f;
             const float4 *src = reinterpret_cast<const float4 *>(part_o + ((long long)s * rows + row) * D + c0);
 #pragma unroll
@@ -239,6 +248,11 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
     const int b = (int)rem;
     // rows: 16/G queries x G heads (KS_PROWS) or 16 heads of one query
     const int nqw = PR ? 16 / p.G : 1;
+    const int lq = 31 - __clz(nqw);                          // log2(nqw)
+    int i0 = 0;                                              // first dilated exponent: 2^i0 >= window
+    if constexpr (PR) {
+        while ((1LL << i0) < p.window) ++i0;
+    }
     const int t = tu * nqw;                                 // first query of the item
     const int t_end = min(t + nqw, p.Tq) - 1;              // last query of the item
     const long long pos = p.q_pos0 + t;
@@ -300,7 +314,7 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
         int j, seg = 0;
         if constexpr (PR) {
             j = (ci < n_chunks && lane < NK)
-                    ? key_prows(p, pos, p.q_pos0 + t_end, nqw, e_beg + ci * NK + lane, e_end, seg) : -1;
+                    ? key_prows(p, pos, p.q_pos0 + t_end, lq, i0, e_beg + ci * NK + lane, e_end, seg) : -1;
         } else {
             j = key_finish<SRC>(p, pos, raw, e_beg + ci * NK + lane);
         }

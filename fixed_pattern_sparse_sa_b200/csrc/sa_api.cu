@@ -492,7 +492,12 @@ int sa_sparse_attn_fwd(const void *q, const void *k, const void *v, int B, int T
     const bool tc = attn_tc_applies(p, d, src, bias);
     // with a ticket array the gather kernel's last piece of each group does
     // the merge itself (no separate combine launch)
-    if (!tc && n_split > 1 && out && tickets) {
+    static int fused = -1;                     // SA_SPLIT_MERGE=kernel: separate combine launch
+    if (fused < 0) {
+        const char *e = std::getenv("SA_SPLIT_MERGE");
+        fused = (e && std::strcmp(e, "kernel") == 0) ? 0 : 1;
+    }
+    if (fused && !tc && n_split > 1 && n_split <= 32 && out && tickets) {
         const size_t nt = (size_t)B * Tq * Hkv * p.n_hchunk;
         cudaError_t e = cudaMemsetAsync(tickets, 0, nt * 4, st);
         if (e != cudaSuccess) return fail(SA_ERR_CUDA, "sparse_attn tickets: %s", cudaGetErrorString(e));
