@@ -10,26 +10,28 @@
 // is then taken from the list (topk_select_kernel in indexer.cuh).
 //
 // Design (one persistent CTA per SM):
-//  * Work unit = one block of NQ = 256 / HI consecutive queries of one
+//  * Work unit = one block of NQ = 224 / HI consecutive queries of one
 //    sequence and ALL of their candidate keys, so a row's list is written by
 //    one CTA only: list slots come from shared-memory counters, never from
 //    global atomics.  Units are taken latest (heaviest) block first.
-//  * MMA: D[128 keys x 256 (query, head) columns] = K_tile . Q_block^T
+//  * MMA: D[128 keys x 224 (query, head) columns] = K_tile . Q_block^T
 //    (tcgen05.mma kind::i8, s32 accumulators in TMEM), K = DI.  Two
-//    accumulators (2 x 256 TMEM columns) let the MMA of tile k+1 run while
-//    the epilogue drains tile k.
+//    accumulators (two 224-column regions of TMEM) let the MMA of tile k+1
+//    run while the epilogue drains tile k.
 //  * Operands arrive by TMA box loads into the K-major swizzled layout whose
 //    swizzle width equals the row (DI bytes: 32B, 64B or 128B swizzle): key
 //    tiles of 128 rows through a FT_STAGES-deep ring, the query block's
-//    256 rows double-buffered by unit.
+//    224 rows double-buffered by unit.
 //  * Weights are folded into the query operand beforehand wherever that is
 //    exact (w >= 0 and every w*q fits int8: w*relu(x) = relu(w*x)); a unit
 //    whose weights all fold sums ReLUs with one DPX add-max per head,
 //    starting from -tau so that the keep test is a sign test.
 //  * Warps: 0 TMA producer (lane 0 issues; all lanes write the unit's
-//    per-query constants), 1 MMA issuer and TMEM owner, 2..17 epilogue:
-//    warp w reads TMEM lane quadrant w % 4 (one key row per thread) over
-//    64 of the 256 columns.
+//    per-query constants), 1 MMA issuer and TMEM owner, 2..29 epilogue:
+//    warp w reads TMEM lane quadrant w % 4 (one key row per thread) over 32
+//    of the 224 columns.  224 columns (not 256) let 28 epilogue warps share
+//    them evenly: the epilogue is bound by latency, and 30 warps per SM at
+//    64 registers hide more of it than 18 warps at 96.
 // Every wait is bounded (progress waits by the spin limit, drains by a fixed
 // long limit); a timeout sets ERR_TIMEOUT, the roles stop together and the
 // CTA drains its copies and MMAs before freeing TMEM.
@@ -42,12 +44,13 @@
 
 namespace sa {
 
-constexpr int FT_NCOL = 256;
+constexpr int FT_NCOL = 224;                      // (query, head) columns of a unit: 7 x 32
 constexpr int FT_STAGES = 6;                      // key-tile ring depth
-constexpr int FT_EPI_WARPS = 16;
+constexpr int FT_EPI_WARPS = 28;                  // 7 per TMEM lane quadrant, 32 columns each
 constexpr int FT_THREADS = (2 + FT_EPI_WARPS) * 32;
-constexpr int FT_CW = FT_NCOL / (FT_EPI_WARPS / 4);   // columns per epilogue warp (64)
-constexpr uint32_t FT_TM_COLS = 512;              // two 256-column accumulators
+constexpr int FT_CW = FT_NCOL / (FT_EPI_WARPS / 4);   // columns per epilogue warp (32)
+constexpr int FT_ACC = 256;                       // TMEM column stride of the two accumulators
+constexpr uint32_t FT_TM_COLS = 512;
 
 template <int DI>
 struct FtSmem {
@@ -305,7 +308,7 @@ __global__ void __launch_bounds__(FT_THREADS, 1)
                     const uint32_t a_addr = tc::smem_u32(smem + L::OFF_A + st * L::A_BYTES);
 #pragma unroll
                     for (int kk = 0; kk < DI / 32; ++kk)
-                        tc::mma_i8(tmem + ab * FT_NCOL, ft::desc_row_swizzled<DI>(a_addr + kk * 32),
+                        tc::mma_i8(tmem + ab * FT_ACC, ft::desc_row_swizzled<DI>(a_addr + kk * 32),
                                    ft::desc_row_swizzled<DI>(b_addr + kk * 32), IDESC, kk > 0 ? 1u : 0u);
                     tc::mma_commit(a_empty + st);
                     tc::mma_commit(acc_full + ab);
@@ -361,14 +364,14 @@ __global__ void __launch_bounds__(FT_THREADS, 1)
                 const int j = k * 128 + quad * 32 + lane;  // this thread's key
                 const bool full = (k + 1) * 128 <= nc_first;   // every key visible to every query
                 const unsigned lt = (1u << lane) - 1u;
-                // two halves of this warp's 64 columns (32 registers each); the
-                // accumulator is released once the second half is loaded
+                // this warp's columns, 32 at a time (32 registers); the
+                // accumulator is released once the last part is loaded
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
+                for (int half = 0; half < FT_CW / 32; ++half) {
                     uint32_t x[32];
-                    ft::tmem_ld32(tmem + lrow + ab * FT_NCOL + c0 + half * 32, x);
+                    ft::tmem_ld32(tmem + lrow + ab * FT_ACC + c0 + half * 32, x);
                     tc::tmem_ld_wait();
-                    if (half == 1) {
+                    if (half == FT_CW / 32 - 1) {
                         tc::fence_before_sync();
                         __syncwarp();
                         if (lane == 0) atc::arrive(acc_free + ab);
