@@ -170,8 +170,8 @@ def main():
     ap.add_argument("--nsa-seq-len", type=int, default=0,
                     help="NSA length for profiling captures of a smaller case (default 65536)")
     ap.add_argument("--workload", default="all",
-                    choices=["all", "decode128k", "indexcache_prefill", "hysparse2_prefill", "nsa64k",
-                             "spatial16k"],
+                    choices=["all", "decode128k", "indexcache_prefill", "hysparse2_prefill", "bwd64k",
+                             "nsa64k", "spatial16k"],
                     help="run only one of the extra measurements (for profiling captures of a "
                          "single workload); prints its numbers alone")
     ap.add_argument("--decode-split", type=int, default=16,
@@ -268,25 +268,86 @@ def main():
     idx_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_idx[-args.steps:])
     att_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_att[-args.steps:])
 
-    # end to end through the public API with host buffers (pinned)
+    # end to end through the public API with host buffers (pinned): every step
+    # copies its inputs host -> device, runs the path and copies out and lse
+    # back.  Steps are pipelined the way a serving loop runs them: step i+1's
+    # inputs go up on one copy stream and step i-1's results come back on
+    # another while step i computes; two sets of device inputs and outputs
+    # keep the copies off the buffers in use.  The serial form (copy, compute,
+    # copy on one stream) is reported beside it.
     host = {k: v.pin_memory() for k, v in g.items()}
-    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    lse_h = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    out_h = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
+    lse_h = [torch.empty(lse.shape, dtype=lse.dtype).pin_memory() for _ in range(2)]
     h2d = sum(v.numel() * v.element_size() for v in host.values())
-    d2h = out_h.numel() * out_h.element_size() + lse_h.numel() * lse_h.element_size()
+    d2h = out.numel() * out.element_size() + lse.numel() * lse.element_size()
 
-    def e2e_step():
+    def e2e_serial_step():
         for k2, v2 in host.items():
             gd[k2].copy_(v2, non_blocking=True)
         step(False)
-        out_h.copy_(out, non_blocking=True)
-        lse_h.copy_(lse, non_blocking=True)
+        out_h[0].copy_(out, non_blocking=True)
+        lse_h[0].copy_(lse, non_blocking=True)
 
-    e2e_value = None
+    e2e_value = e2e_serial = None
     if not args.no_e2e:
-        e2e_times = timed_steps(e2e_step, max(2, args.steps // 2), args.warmup, flush, dev, torch)
+        n_e2e = max(2, args.steps // 2)
+        e2e_times = timed_steps(e2e_serial_step, n_e2e, args.warmup, flush, dev, torch)
         e2e_ms = max_over_ranks(sum(e2e_times), dev, torch, dist)
-        e2e_value = aggregate([e2e_ms], [flops * len(e2e_times)] * world)[0] / 1e12
+        e2e_serial = aggregate([e2e_ms], [flops * len(e2e_times)] * world)[0] / 1e12
+
+        sets = [gd, {k: torch.empty_like(v) for k, v in gd.items()}]
+        outs = [(out, lse), (torch.empty_like(out), torch.empty_like(lse))]
+        s_in, s_cmp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
+        in_ready = [torch.cuda.Event() for _ in range(2)]
+        done = [torch.cuda.Event() for _ in range(2)]
+        out_free = [torch.cuda.Event() for _ in range(2)]
+        started = [False, False]
+
+        def pipelined(n):
+            for i in range(n):
+                s = i % 2
+                with torch.cuda.stream(s_in):
+                    if started[s]:
+                        s_in.wait_event(done[s])          # compute of step i-2 read set s
+                    for k2, v2 in host.items():
+                        sets[s][k2].copy_(v2, non_blocking=True)
+                    in_ready[s].record(s_in)
+                with torch.cuda.stream(s_cmp):
+                    s_cmp.wait_event(in_ready[s])
+                    if started[s]:
+                        s_cmp.wait_event(out_free[s])     # step i-2's results are on the host
+                    o, l = outs[s]
+                    api.indexer_topk(sets[s]["q_idx"], sets[s]["k_idx"], sets[s]["w"], w.topk, w.window,
+                                     out_idx=idx, out_count=cnt, workspace=ws)
+                    api.sparse_attn_fwd(sets[s]["q"], sets[s]["k"], sets[s]["v"], idx, out=o, lse=l)
+                    done[s].record(s_cmp)
+                with torch.cuda.stream(s_out):
+                    s_out.wait_event(done[s])
+                    out_h[s].copy_(outs[s][0], non_blocking=True)
+                    lse_h[s].copy_(outs[s][1], non_blocking=True)
+                    out_free[s].record(s_out)
+                started[s] = True
+
+        cur = torch.cuda.current_stream(dev)
+        pipelined(args.warmup)
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(cur)
+        for st_ in (s_in, s_cmp, s_out):
+            st_.wait_stream(cur)
+        pipelined(args.steps)
+        for st_ in (s_in, s_cmp, s_out):
+            cur.wait_stream(st_)
+        b.record(cur)
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        pipe_ms = max_over_ranks(a.elapsed_time(b), dev, torch, dist)
+        e2e_value = aggregate([pipe_ms], [flops * args.steps] * world)[0] / 1e12
+        api.check_device_status()
 
     peaks = _peaks()
     att_tflops = flops / (att_ms / 1e3) / 1e12
@@ -336,7 +397,9 @@ def main():
         },
         "e2e": None if e2e_value is None else
                {"value": round(e2e_value, 3), "unit": "TFLOP/s",
-                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                "overlap": "h2d / compute / d2h on three streams, two buffer sets; inputs larger than L2",
+                "serial_value": round(e2e_serial, 3)},
         "gpu_launches": int(launches),
     }
     clocks = clk.summary()
@@ -472,6 +535,32 @@ def extra_measurements(args, dev, torch, api, lib, inputs, flush, world, peaks, 
             "note": "indexer top-1024 + forced window 128, then sparse attention; "
                     f"1 x {T} tokens, 16 q heads / 1 kv head, d=128"}
         del gh, ghd, hidx, hout, hws
+        torch.cuda.empty_cache()
+    # --- backward of the 64K sparse attention (dq, dk, dv over the selected keys) ---
+    if only in (None, "bwd64k"):
+        w = inputs.WORKLOADS["dsa_prefill64k"]
+        T = args.seq_len or w.T
+        gb = inputs.gen_dsa(w.B, T, w.Hq, w.Hkv, w.d, w.Hi, w.di, seed=300)
+        gbd = {k: v.to(dev) for k, v in gb.items()}
+        bidx, _ = api.indexer_topk(gbd["q_idx"], gbd["k_idx"], gbd["w"], w.topk, w.window)
+        bout, blse = api.sparse_attn_fwd(gbd["q"], gbd["k"], gbd["v"], bidx)
+        dout = (torch.randn(bout.shape, generator=torch.Generator().manual_seed(301)) * 0.1).to(
+            device=dev, dtype=torch.bfloat16)
+
+        def bstep():
+            api.sparse_attn_bwd(gbd["q"], gbd["k"], gbd["v"], bout, blse, dout, bidx)
+        times = timed_steps(bstep, 3, args.warmup, flush, dev, torch)
+        ms = max_over_ranks(sum(times), dev, torch, dist) / len(times)
+        # S = QK^T recomputed, dP = dO V^T, dV += P^T dO, dQ = dS K, dK += dS^T Q: 10 d per
+        # (query, head, key), 2.5 x the forward's 4 d
+        bfl = 2.5 * attn_flops(T, w.topk, w.window, w.Hq, w.d)
+        res[f"bwd{T // 1024}k"] = {
+            "ms_per_step": round(ms, 3), "tflops": round(world * bfl / (ms / 1e3) / 1e12, 2),
+            "algorithmic_flops": bfl,
+            "tensor_frac": round(bfl / (ms / 1e3) / 1e12 / peaks["bf16_tflops"], 4),
+            "note": f"sparse_attn_bwd over the indexer's top-2048 + window 64, 1 x {T} tokens, "
+                    "16 q heads / 1 kv head, d=128; fp32 dq/dk/dv"}
+        del gb, gbd, bidx, bout, blse, dout
         torch.cuda.empty_cache()
     # --- NSA 64K ---
     if only in (None, "nsa64k"):
