@@ -69,13 +69,6 @@ struct CtSmem {                    // head dim 128
 };
 
 
-// 2^x on the special-function unit (flushes results below the normal range
-// to zero, which a softmax weight can ignore).
-__device__ __forceinline__ float ex2_fast(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
 
 struct CmpTcParams {
     TileParams t;          // q, shapes, cmp_len/stride (Lk = compressed tokens per sequence), outputs

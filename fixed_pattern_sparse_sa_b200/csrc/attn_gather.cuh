@@ -216,8 +216,13 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
     constexpr int KEYB = NK * ((PR ? 8 : 4) + (BIAS ? 12 : 0));   // per stage: keys (+ segments, + coordinates)
     // TMA layout: every warp's stages first (1024-byte aligned for the 128-byte
     // swizzle), then the keys, then one mbarrier per stage and warp
-    unsigned char *smem = TMAB ? smem_dyn + ((1024u - (tc::smem_u32(smem_dyn) & 1023u)) & 1023u) : smem_dyn;
-    unsigned char *wsm = TMAB ? smem + warp * (STAGES * SB) : smem + warp * (STAGES * (SB + KEYB));
+    // cp.async layout: per warp its stages then its keys, the warp's region
+    // padded to 256 bytes from a 256-byte aligned base, so that a K/V row
+    // starts on a 256-byte boundary (the copy loop below relies on it)
+    constexpr int WSTRIDE = STAGES * SB + ((STAGES * KEYB + 255) & ~255);
+    unsigned char *smem = TMAB ? smem_dyn + ((1024u - (tc::smem_u32(smem_dyn) & 1023u)) & 1023u)
+                               : smem_dyn + ((256u - (tc::smem_u32(smem_dyn) & 255u)) & 255u);
+    unsigned char *wsm = TMAB ? smem + warp * (STAGES * SB) : smem + warp * WSTRIDE;
     int *keys_s = TMAB ? reinterpret_cast<int *>(smem + NW * STAGES * SB) + warp * STAGES * NK
                        : reinterpret_cast<int *>(wsm + STAGES * SB);
     uint64_t *full_s = reinterpret_cast<uint64_t *>(smem + NW * STAGES * (SB + NK * 4)) + warp * STAGES;
@@ -278,7 +283,16 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
             qf[ks][2] = v0 ? __ldg(q0 + ks * 8 + qc + 4) : 0u;
             qf[ks][3] = v1 ? __ldg(q1 + ks * 8 + qc + 4) : 0u;
         }
+        // a negative scale is folded into Q (sign bits of both bf16 halves),
+        // so every score below is scaled by |scale| and keeps the order of q.k
+        if (p.scale_log2 < 0.f) {
+#pragma unroll
+            for (int ks = 0; ks < KS_D; ++ks)
+#pragma unroll
+                for (int r = 0; r < 4; ++r) qf[ks][r] ^= 0x80008000u;
+        }
     }
+    const float sl2 = fabsf(p.scale_log2);
     float cq0[3] = {0.f, 0.f, 0.f}, cq1[3] = {0.f, 0.f, 0.f}, be0 = 0.f, be1 = 0.f;
     if constexpr (BIAS) {
         if (v0) {
@@ -301,6 +315,11 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
     const __nv_bfloat16 *vb = p.v + ((long long)b * p.Lk * p.Hkv + g) * D;
     const __nv_bfloat16 *lb = KLO ? p.klo + ((long long)b * p.Lk * p.Hkv + g) * D : nullptr;
     const long long rstride = (long long)p.Hkv * D;
+    // copy lanes: lane = lrow * UNITS + u (u: 16-byte unit of a row, lrow: row within an instruction)
+    constexpr int RPI = 32 / UNITS;
+    const int lrow_c = lane / UNITS, u_c = lane % UNITS;
+    const __nv_bfloat16 *kb_u = kb + u_c * 8, *vb_u = vb + u_c * 8;
+    const __nv_bfloat16 *lb_u = KLO ? lb + u_c * 8 : nullptr;
 
     // raw list value of chunk ci for this lane (lane i < NK owns key i)
     auto raw_of = [&](int ci) -> int {
@@ -361,18 +380,23 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
             return;
         }
         if (ci < n_chunks) {
-#pragma unroll
-            for (int it = 0; it < CP_ITERS; ++it) {
-                const int lin = it * 32 + lane;
-                const int rr = lin / UNITS, u = lin % UNITS;
-                const int jr = __shfl_sync(0xffffffffu, j, rr);
-                const long long off = jr >= 0 ? (long long)jr * rstride + u * 8 : 0;
+            // UNITS lanes per key row, RPI = 32 / UNITS rows per instruction,
+            // so every copy instruction covers whole 128-byte lines.  Lane
+            // (lrow, u) copies unit u of rows it * RPI + lrow to the swizzled
+            // unit u ^ (row & 7); with the stage on a 256-byte boundary that
+            // address is (base ^ (((it * RPI) & 7) << 4)) + it * RPI * ROWB,
+            // one XOR per row; the row offsets are immediates.
+            const uint32_t base = tc::smem_u32(ks_) + lrow_c * ROWB + ((u_c ^ lrow_c) << 4);
+            static_for<CP_ITERS>([&](auto ic) {
+                constexpr int it = decltype(ic)::value;
+                const int jr = __shfl_sync(0xffffffffu, j, it * RPI + lrow_c);
+                const long long jo = (long long)max(jr, 0) * rstride;
                 const int nb = jr >= 0 ? 16 : 0;
-                const int sw = (u ^ (rr & 7)) * 16;
-                cp_async16(ks_ + rr * ROWB + sw, kb + off, nb);
-                cp_async16(vs_ + rr * ROWB + sw, vb + off, nb);
-                if constexpr (KLO) cp_async16(vs_ + CH + rr * ROWB + sw, lb + off, nb);
-            }
+                const uint32_t dst = base ^ (uint32_t)(((it * RPI) & 7) << 4);
+                cp_async16_at<it * RPI * ROWB, 0>(dst, kb_u + jo, nb);
+                cp_async16_at<it * RPI * ROWB + CH, 0>(dst, vb_u + jo, nb);
+                if constexpr (KLO) cp_async16_at<it * RPI * ROWB + 2 * CH, 0>(dst, lb_u + jo, nb);
+            });
         }
         cp_async_commit();
     };
@@ -442,55 +466,83 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
                 sc[i][0] += sc2[i][0]; sc[i][1] += sc2[i][1];
                 sc[i][2] += sc2[i][2]; sc[i][3] += sc2[i][3];
             }
-            // scale, bias, mask; running max
+            // running max.  Plain lists keep the raw q.k (the scale, > 0 after
+            // the sign fold, goes into the exponent's FFMA) and mask only a
+            // chunk with empty entries; bias and row masks scale first.
+            constexpr bool RAW = !BIAS && !PR;
             float mx0 = -INFINITY, mx1 = -INFINITY;
+            constexpr unsigned kFull = NK == 32 ? 0xffffffffu : ((1u << NK) - 1u);
+            const bool partial = RAW && vmask != kFull;        // warp-uniform
+            if constexpr (RAW) {
+                if (partial) {
 #pragma unroll
-            for (int nt = 0; nt < NK / 8; ++nt) {
+                    for (int nt = 0; nt < NK / 8; ++nt)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int kk = nt * 8 + 2 * qc + (e & 1);
-                    float x = sc[nt][e] * p.scale_log2;
-                    if constexpr (BIAS) {
-                        const int jk = __shfl_sync(0xffffffffu, jl, kk);
-                        if (jk >= 0) {
-                            const float *c = ck_s + (st * NK + kk) * 3;
-                            const float *a = (e >> 1) ? cq1 : cq0;
-                            const float dx = a[0] - c[0], dy = a[1] - c[1], dz = a[2] - c[2];
-                            x -= ((e >> 1) ? be1 : be0) * (dx * dx + dy * dy + dz * dz);
-                        }
-                    }
-                    bool ok = (vmask >> kk) & 1u;
-                    if constexpr (PR) {
-                        // the entry's segment decides which rows it belongs to
-                        const int jk = __shfl_sync(0xffffffffu, jl, kk);
-                        const int sk = __shfl_sync(0xffffffffu, sl, kk);
-                        const long long d = ((e >> 1) ? pos_r1 : pos_r0) - jk;
-                        ok = ok && (sk == 0 ? (d >= 0 && d < p.window) : (d == sk && sk < d + jk));
-                    }
-                    x = ok ? x : -INFINITY;
-                    sc[nt][e] = x;
+                        for (int e = 0; e < 4; ++e)
+                            if (!((vmask >> (nt * 8 + 2 * qc + (e & 1))) & 1u)) sc[nt][e] = -INFINITY;
                 }
-                mx0 = fmaxf(mx0, fmaxf(sc[nt][0], sc[nt][1]));
-                mx1 = fmaxf(mx1, fmaxf(sc[nt][2], sc[nt][3]));
+#pragma unroll
+                for (int nt = 0; nt < NK / 8; ++nt) {
+                    mx0 = fmaxf(mx0, fmaxf(sc[nt][0], sc[nt][1]));
+                    mx1 = fmaxf(mx1, fmaxf(sc[nt][2], sc[nt][3]));
+                }
+            } else {
+#pragma unroll
+                for (int nt = 0; nt < NK / 8; ++nt) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int kk = nt * 8 + 2 * qc + (e & 1);
+                        float x = sc[nt][e] * sl2;
+                        if constexpr (BIAS) {
+                            const int jk = __shfl_sync(0xffffffffu, jl, kk);
+                            if (jk >= 0) {
+                                const float *c = ck_s + (st * NK + kk) * 3;
+                                const float *a = (e >> 1) ? cq1 : cq0;
+                                const float dx = a[0] - c[0], dy = a[1] - c[1], dz = a[2] - c[2];
+                                x -= ((e >> 1) ? be1 : be0) * (dx * dx + dy * dy + dz * dz);
+                            }
+                        }
+                        bool ok = (vmask >> kk) & 1u;
+                        if constexpr (PR) {
+                            // the entry's segment decides which rows it belongs to
+                            const int jk = __shfl_sync(0xffffffffu, jl, kk);
+                            const int sk = __shfl_sync(0xffffffffu, sl, kk);
+                            const long long d = ((e >> 1) ? pos_r1 : pos_r0) - jk;
+                            ok = ok && (sk == 0 ? (d >= 0 && d < p.window) : (d == sk && sk < d + jk));
+                        }
+                        x = ok ? x : -INFINITY;
+                        sc[nt][e] = x;
+                    }
+                    mx0 = fmaxf(mx0, fmaxf(sc[nt][0], sc[nt][1]));
+                    mx1 = fmaxf(mx1, fmaxf(sc[nt][2], sc[nt][3]));
+                }
             }
             mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
             mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
             mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
             mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-            const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+            // m0 / m1 and everything below are in the scaled log2 domain
+            constexpr float kOne = 1.f;
+            const float xs = RAW ? sl2 : kOne;                 // factor still to apply to sc
+            const float mn0 = fmaxf(m0, RAW ? mx0 * sl2 : mx0), mn1 = fmaxf(m1, RAW ? mx1 * sl2 : mx1);
             const float mu0 = mn0 == -INFINITY ? 0.f : mn0;
             const float mu1 = mn1 == -INFINITY ? 0.f : mn1;
-            const float al0 = exp2f(m0 - mu0), al1 = exp2f(m1 - mu1);
+            const float al0 = ex2_fast(m0 - mu0), al1 = ex2_fast(m1 - mu1);
             // the accumulators need rescaling only when some row's max grew
             const bool grew = __any_sync(0xffffffffu, mn0 > m0 || mn1 > m1);
             m0 = mn0; m1 = mn1;
             float rs0 = 0.f, rs1 = 0.f;
 #pragma unroll
             for (int nt = 0; nt < NK / 8; ++nt) {
-                sc[nt][0] = exp2f(sc[nt][0] - mu0);
-                sc[nt][1] = exp2f(sc[nt][1] - mu0);
-                sc[nt][2] = exp2f(sc[nt][2] - mu1);
-                sc[nt][3] = exp2f(sc[nt][3] - mu1);
+                sc[nt][0] = ex2_fast(fmaf(sc[nt][0], xs, -mu0));
+                sc[nt][1] = ex2_fast(fmaf(sc[nt][1], xs, -mu0));
+                sc[nt][2] = ex2_fast(fmaf(sc[nt][2], xs, -mu1));
+                sc[nt][3] = ex2_fast(fmaf(sc[nt][3], xs, -mu1));
+                if (partial) {                                 // exact zeros for empty entries (any scale)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        if (!((vmask >> (nt * 8 + 2 * qc + (e & 1))) & 1u)) sc[nt][e] = 0.f;
+                }
                 rs0 += sc[nt][0] + sc[nt][1];
                 rs1 += sc[nt][2] + sc[nt][3];
             }
@@ -614,8 +666,10 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
 template <int D, int STAGES, bool KLO = false, int NK = 32, int NW = 4, bool PR = false, bool BIAS = false,
           bool TMAB = false>
 constexpr int gather_smem_bytes() {
-    return NW * STAGES * ((KLO ? 3 : 2) * NK * D * 2 + NK * ((PR ? 8 : 4) + (BIAS ? 12 : 0))) +
-           (TMAB ? NW * STAGES * 8 + 1024 : 0);
+    constexpr int SB = (KLO ? 3 : 2) * NK * D * 2;
+    constexpr int KEYB = NK * ((PR ? 8 : 4) + (BIAS ? 12 : 0));
+    return TMAB ? NW * STAGES * (SB + KEYB) + NW * STAGES * 8 + 1024
+                : NW * (STAGES * SB + ((STAGES * KEYB + 255) & ~255)) + 256;
 }
 
 }  // namespace sa

@@ -363,7 +363,6 @@ __global__ void __launch_bounds__(FT_THREADS, 1)
                 tc::fence_after_sync();
                 const int j = k * 128 + quad * 32 + lane;  // this thread's key
                 const bool full = (k + 1) * 128 <= nc_first;   // every key visible to every query
-                const unsigned lt = (1u << lane) - 1u;
                 // this warp's columns, 32 at a time (32 registers); the
                 // accumulator is released once the last part is loaded
 #pragma unroll
@@ -379,8 +378,7 @@ __global__ void __launch_bounds__(FT_THREADS, 1)
                     constexpr int NQH = 32 / HI;              // queries in a half
                     constexpr int NG = NQH < 8 ? NQH : 8;     // queries per group
                     // per group: the sums first (independent chains), a keep
-                    // mask, then per query one warp ballot and one shared-memory
-                    // atomic by the lowest keeping lane
+                    // mask, then the kept pairs go to their queries' lists
 #pragma unroll
                     for (int g0 = 0; g0 < NQH; g0 += NG) {
                         const int qb = half * NQH + g0;       // first query of the group (in this warp)
@@ -413,27 +411,22 @@ __global__ void __launch_bounds__(FT_THREADS, 1)
                             for (int qq = 0; qq < NG; ++qq)
                                 if (j >= nc_u[qb + qq]) mask &= ~(1u << qq);
                         }
-                        // one ballot per query; lane qq reserves the group's
-                        // slots of query qq (one atomic instruction for the
-                        // whole group, distinct addresses), then every lane
-                        // writes its kept pairs
-                        unsigned bal[NG];
-                        int mycnt = 0;
+                        // per query: skipped by the whole warp when no lane
+                        // keeps it, else every keeping lane takes its slot with
+                        // its own shared-memory atomic (one per kept pair: ~10%
+                        // of the pairs, fewer instructions than reserving a
+                        // warp's slots by ballot, shuffle and popcount)
 #pragma unroll
                         for (int qq = 0; qq < NG; ++qq) {
-                            bal[qq] = __ballot_sync(0xffffffffu, (mask >> qq) & 1u);
-                            mycnt = lane == qq ? __popc(bal[qq]) : mycnt;
-                        }
-                        int mybase = 0;
-                        if (mycnt > 0) mybase = atomicAdd(cnt_u + qb + lane, mycnt);
-#pragma unroll
-                        for (int qq = 0; qq < NG; ++qq) {
-                            if (bal[qq] == 0u) continue;       // warp-uniform
-                            const int slot = __shfl_sync(0xffffffffu, mybase, qq) + __popc(bal[qq] & lt);
-                            if (((mask >> qq) & 1u) && slot < p.cand_cap) {
-                                const long long off = list0 + (long long)(qb + qq) * p.cand_cap + slot;
-                                p.cand_val[off] = sc[qq];
-                                p.cand_idx[off] = j;
+                            const bool keep = (mask >> qq) & 1u;
+                            if (!__any_sync(0xffffffffu, keep)) continue;   // warp-uniform
+                            if (keep) {
+                                const int slot = atomicAdd(cnt_u + qb + qq, 1);
+                                if (slot < p.cand_cap) {
+                                    const long long off = list0 + (long long)(qb + qq) * p.cand_cap + slot;
+                                    p.cand_val[off] = sc[qq];
+                                    p.cand_idx[off] = j;
+                                }
                             }
                         }
                     }

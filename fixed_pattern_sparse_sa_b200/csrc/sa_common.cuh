@@ -1,6 +1,8 @@
 // sa_common.cuh -- device helpers shared by the library's kernels.
 #pragma once
 
+#include <type_traits>
+#include <utility>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -37,6 +39,14 @@ __device__ __forceinline__ bool debug_stall() { return *reinterpret_cast<volatil
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
+// 2^x on the special-function unit (the PTX ex2.approx instruction; results
+// below the normal range flush to zero, which a softmax weight can ignore).
+__device__ __forceinline__ float ex2_fast(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 __device__ __forceinline__ void raise_error(unsigned *err, unsigned bit) {
     if (err) atomicOr(err, bit);
 }
@@ -47,6 +57,25 @@ __device__ __forceinline__ void cp_async16(void *smem, const void *gmem, int src
     unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gmem),
                  "r"(src_bytes));
+}
+// f(integral_constant<int, 0>), ..., f(integral_constant<int, N-1>): a loop
+// whose index is a compile-time constant (for immediate operands).
+template <typename F, int... I>
+__device__ __forceinline__ void static_for_impl(F &&f, std::integer_sequence<int, I...>) {
+    (f(std::integral_constant<int, I>{}), ...);
+}
+template <int N, typename F>
+__device__ __forceinline__ void static_for(F &&f) {
+    static_for_impl(f, std::make_integer_sequence<int, N>{});
+}
+
+// 16-byte copy from gmem + GOFF bytes to shared address s + SOFF (s a 32-bit
+// shared address): the offsets are immediates, so copies from one base share
+// its registers.
+template <int SOFF, int GOFF>
+__device__ __forceinline__ void cp_async16_at(uint32_t s, const void *gmem, int src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0+%3], [%1+%4], 16, %2;\n" ::"r"(s), "l"(gmem), "r"(src_bytes),
+                 "n"(SOFF), "n"(GOFF));
 }
 // 4-byte asynchronous global->shared copy (cached at all levels).
 __device__ __forceinline__ void cp_async4(void *smem, const void *gmem) {
