@@ -521,16 +521,30 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
             mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
             mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
             mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-            // m0 / m1 and everything below are in the scaled log2 domain
-            constexpr float kOne = 1.f;
+            // m0 / m1 and everything below are in the scaled log2 domain.
+            // m0 / m1 are reference maxima, not running maxima: they move
+            // (and the accumulators are rescaled) only when some row's chunk
+            // maximum exceeds its reference by more than kLazy, so weights
+            // 2^(x - m) stay below 2^kLazy (exact in bf16 up to its usual
+            // rounding, no overflow in fp32 sums) and most chunks skip the
+            // rescale.  softmax is the same for any reference value.
+            constexpr float kOne = 1.f, kLazy = 8.f;
             const float xs = RAW ? sl2 : kOne;                 // factor still to apply to sc
-            const float mn0 = fmaxf(m0, RAW ? mx0 * sl2 : mx0), mn1 = fmaxf(m1, RAW ? mx1 * sl2 : mx1);
-            const float mu0 = mn0 == -INFINITY ? 0.f : mn0;
-            const float mu1 = mn1 == -INFINITY ? 0.f : mn1;
-            const float al0 = ex2_fast(m0 - mu0), al1 = ex2_fast(m1 - mu1);
-            // the accumulators need rescaling only when some row's max grew
-            const bool grew = __any_sync(0xffffffffu, mn0 > m0 || mn1 > m1);
-            m0 = mn0; m1 = mn1;
+            const float cm0 = RAW ? mx0 * sl2 : mx0, cm1 = RAW ? mx1 * sl2 : mx1;
+            if (__any_sync(0xffffffffu, cm0 > m0 + kLazy || cm1 > m1 + kLazy)) {   // warp-uniform
+                const float mn0 = fmaxf(m0, cm0), mn1 = fmaxf(m1, cm1);
+                const float al0 = m0 == -INFINITY ? 0.f : ex2_fast(m0 - mn0);
+                const float al1 = m1 == -INFINITY ? 0.f : ex2_fast(m1 - mn1);
+                m0 = mn0; m1 = mn1;
+                l0 *= al0; l1 *= al1;
+#pragma unroll
+                for (int i = 0; i < NT_D; ++i) {
+                    o[i][0] *= al0; o[i][1] *= al0;
+                    o[i][2] *= al1; o[i][3] *= al1;
+                }
+            }
+            const float mu0 = m0 == -INFINITY ? 0.f : m0;
+            const float mu1 = m1 == -INFINITY ? 0.f : m1;
             float rs0 = 0.f, rs1 = 0.f;
 #pragma unroll
             for (int nt = 0; nt < NK / 8; ++nt) {
@@ -546,15 +560,8 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
                 rs0 += sc[nt][0] + sc[nt][1];
                 rs1 += sc[nt][2] + sc[nt][3];
             }
-            l0 = l0 * al0 + rs0;
-            l1 = l1 * al1 + rs1;
-            if (grew) {
-#pragma unroll
-                for (int i = 0; i < NT_D; ++i) {
-                    o[i][0] *= al0; o[i][1] *= al0;
-                    o[i][2] *= al1; o[i][3] *= al1;
-                }
-            }
+            l0 += rs0;
+            l1 += rs1;
             // P (bf16) * V
 #pragma unroll
             for (int kp = 0; kp < NK / 16; ++kp) {

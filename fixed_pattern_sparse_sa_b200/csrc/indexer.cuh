@@ -47,8 +47,7 @@ struct IdxParams {
     int32_t *sample;       // [B, Rt, m_cap]
     int32_t *tau;          // [B, Rt]
     int cand_cap;          // candidate list capacity per row
-    int32_t *cand_val;     // [B, Rt, cand_cap]
-    int32_t *cand_idx;     // [B, Rt, cand_cap]
+    int2 *cand;            // [B, Rt, cand_cap] (score, key position) pairs
     int32_t *cand_cnt;     // [B, Rt]  (zeroed before the filter pass)
     int32_t *out_idx;      // [B, Tq, Kout]
     int32_t *out_count;    // [B, Tq] nullable
@@ -288,8 +287,8 @@ __global__ void __launch_bounds__(tc_threads(NCOL), NCOL >= 64 ? 2 : 4) idx_scor
             for (int e = lane; e < n; e += 32) {
                 const int slot = base + e;
                 if (slot < p.cand_cap) {
-                    p.cand_val[roff + slot] = lval_s[(buf * NQ + q) * TC_LCAP + e];
-                    p.cand_idx[roff + slot] = key0 + loff_s[(buf * NQ + q) * TC_LCAP + e];
+                    p.cand[roff + slot] = make_int2(lval_s[(buf * NQ + q) * TC_LCAP + e],
+                                                    key0 + loff_s[(buf * NQ + q) * TC_LCAP + e]);
                 }
             }
             __syncwarp();
@@ -418,8 +417,7 @@ __global__ void __launch_bounds__(tc_threads(NCOL), NCOL >= 64 ? 2 : 4) idx_scor
                     const int slot = __shfl_sync(0xffffffffu, base, q) + __popc(ball[q] & lt);
                     if (((keepm >> q) & 1u) && slot < p.cand_cap) {
                         const long long off = (long long)(row0 + q) * p.cand_cap + slot;
-                        p.cand_val[off] = sc[q];
-                        p.cand_idx[off] = jj;
+                        p.cand[off] = make_int2(sc[q], jj);
                     }
                 }
             }
@@ -518,8 +516,7 @@ __global__ void __launch_bounds__(DEC_THREADS) idx_score_dp4a_kernel(const IdxPa
                     if (lane == 0) slot0 = atomicAdd(p.cand_cnt + row, __popc(ballot));
                     const int slot = __shfl_sync(0xffffffffu, slot0, 0) + __popc(ballot & ((1u << lane) - 1u));
                     if (keep && slot < p.cand_cap) {
-                        p.cand_val[row * p.cand_cap + slot] = total;
-                        p.cand_idx[row * p.cand_cap + slot] = (int)jj[u];
+                        p.cand[row * p.cand_cap + slot] = make_int2(total, (int)jj[u]);
                     }
                 }
             }
@@ -651,8 +648,7 @@ __global__ void __launch_bounds__(DMMA_THREADS) idx_score_dec_mma_kernel(const I
         for (int e = tid; e < n; e += DMMA_THREADS) {
             const int slot = base + e;
             if (slot < p.cand_cap) {
-                p.cand_val[row * p.cand_cap + slot] = lval_s[e];
-                p.cand_idx[row * p.cand_cap + slot] = lidx_s[e];
+                p.cand[row * p.cand_cap + slot] = make_int2(lval_s[e], lidx_s[e]);
             }
         }
     }
@@ -740,6 +736,22 @@ __device__ void radix_refine(RadixState &st, int gmin, int *hist, int *scan_tmp,
     st.bin_count = hist[bin];
     st.lo_key += (unsigned)bin << shift;
     st.width = shift;
+    __syncthreads();
+}
+
+// Block min/max of per-thread partial minima and maxima.
+__device__ __forceinline__ void block_minmax_reduce(int vmin, int vmax, int &gmin, int &gmax, int *bcast) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        vmin = min(vmin, __shfl_xor_sync(0xffffffffu, vmin, o));
+        vmax = max(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+    }
+    if (threadIdx.x == 0) { bcast[0] = INT_MAX; bcast[1] = INT_MIN; }
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0) { atomicMin(&bcast[0], vmin); atomicMax(&bcast[1], vmax); }
+    __syncthreads();
+    gmin = bcast[0];
+    gmax = bcast[1];
     __syncthreads();
 }
 
@@ -963,8 +975,7 @@ __global__ void __launch_bounds__(NT, NT <= 256 ? 3 : 1) topk_select_kernel(cons
     const int cnt = p.cand_cnt[row];
     const bool use_list = cnt >= k_eff && cnt <= p.cand_cap;
     if (!use_list && tid == 0) atomicAdd(&g_sa_recompute_rows, 1ull);
-    const int32_t *cv = p.cand_val + row * p.cand_cap;
-    const int32_t *ci = p.cand_idx + row * p.cand_cap;
+    const int2 *cl = p.cand + row * p.cand_cap;
     const int8_t *kb = p.k + (long long)b * p.L * DI;
     if (!use_list) {
         // exact recompute: stage this query's indexer vectors and weights
@@ -974,17 +985,35 @@ __global__ void __launch_bounds__(NT, NT <= 256 ? 3 : 1) topk_select_kernel(cons
         for (int i = tid; i < p.Hi; i += NT) w_s[i] = __ldg(p.w + ((long long)b * p.Tq + t) * p.Hi + i);
         __syncthreads();
     }
-    // stage the list in shared memory (one pass over L2, 16-byte loads)
+    // the bitmaps are cleared first, while the list loads below are in flight
+    for (int i = tid; i < words; i += NT) { gt_bm[i] = 0u; eq_bm[i] = 0u; }
+    if (tid == 0) tie_n = 0;
+    // stage the list in shared memory (one pass over L2, 16-byte loads, U in
+    // flight per thread) and take the score range on the way
     const bool staged = use_list && p.cand_cap <= SEL_STAGE_MAX;
     int *lv_s = reinterpret_cast<int *>(smem + select_stage_off<DI>(words));
     int *li_s = lv_s + p.cand_cap;
+    int smin = INT_MAX, smax = INT_MIN;
     if (staged) {
-        const int n4 = (cnt + 3) / 4;                 // rows are 16-byte aligned (cap % 64 == 0)
-        for (int i = tid; i < n4; i += NT) {
-            reinterpret_cast<int4 *>(lv_s)[i] = __ldg(reinterpret_cast<const int4 *>(cv) + i);
-            reinterpret_cast<int4 *>(li_s)[i] = __ldg(reinterpret_cast<const int4 *>(ci) + i);
+        constexpr int U = 4;
+        const int n2 = (cnt + 1) / 2;                 // rows are 16-byte aligned (cap % 64 == 0)
+        for (int b0 = tid; b0 < n2; b0 += NT * U) {
+            int4 e[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+                if (b0 + u * NT < n2) e[u] = __ldg(reinterpret_cast<const int4 *>(cl) + b0 + u * NT);
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int i = b0 + u * NT;             // pairs 2i and 2i + 1
+                if (i < n2) {
+                    reinterpret_cast<int2 *>(lv_s)[i] = make_int2(e[u].x, e[u].z);
+                    reinterpret_cast<int2 *>(li_s)[i] = make_int2(e[u].y, e[u].w);
+                    smin = min(smin, e[u].x);
+                    smax = max(smax, e[u].x);
+                    if (2 * i + 1 < cnt) { smin = min(smin, e[u].z); smax = max(smax, e[u].z); }
+                }
+            }
         }
-        __syncthreads();
     }
     // every element of the row: (score, position)
     auto for_each = [&](auto f) {
@@ -993,15 +1022,15 @@ __global__ void __launch_bounds__(NT, NT <= 256 ? 3 : 1) topk_select_kernel(cons
         } else if (use_list) {
             constexpr int U = 4;
             for (int b0 = tid; b0 < cnt; b0 += NT * U) {
-                int v[U], jj[U];
+                int2 e[U];
 #pragma unroll
                 for (int u = 0; u < U; ++u) {
                     const int i = b0 + u * NT;
-                    if (i < cnt) { v[u] = __ldg(cv + i); jj[u] = __ldg(ci + i); }
+                    if (i < cnt) e[u] = __ldg(cl + i);
                 }
 #pragma unroll
                 for (int u = 0; u < U; ++u)
-                    if (b0 + u * NT < cnt) f(v[u], jj[u]);
+                    if (b0 + u * NT < cnt) f(e[u].x, e[u].y);
             }
         } else {
             for (int j = tid; j < n; j += NT) f(exact_score<DI>(qrow_s, w_s, p.Hi, kb + (long long)j * DI), j);
@@ -1009,7 +1038,8 @@ __global__ void __launch_bounds__(NT, NT <= 256 ? 3 : 1) topk_select_kernel(cons
     };
 
     int gmin, gmax;
-    block_minmax(gmin, gmax, bcast, for_each);
+    if (staged) block_minmax_reduce(smin, smax, gmin, gmax, bcast);   // its barriers publish the staged list
+    else block_minmax(gmin, gmax, bcast, for_each);
     const unsigned range = (unsigned)gmax - (unsigned)gmin;
     RadixState st{0u, range == 0 ? 0 : 32 - __clz(range), k_eff, use_list ? cnt : n};
     if (use_list && range < (unsigned)SEL_FINE_BINS) {
@@ -1026,9 +1056,6 @@ __global__ void __launch_bounds__(NT, NT <= 256 ? 3 : 1) topk_select_kernel(cons
 
     // filter: bitmaps of keys above the bin; the bin's own elements go to the
     // equal bitmap (width 0) or to the tie list
-    for (int i = tid; i < words; i += NT) { gt_bm[i] = 0u; eq_bm[i] = 0u; }
-    if (tid == 0) tie_n = 0;
-    __syncthreads();
     const unsigned lo_key = st.lo_key;
     const unsigned bin_hi = lo_key + (st.width >= 32 ? 0xffffffffu : ((1u << st.width) - 1u));
     const int width = st.width;

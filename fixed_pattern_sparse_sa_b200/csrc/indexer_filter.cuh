@@ -422,11 +422,8 @@ __global__ void __launch_bounds__(FT_THREADS, 1)
                             if (!__any_sync(0xffffffffu, keep)) continue;   // warp-uniform
                             if (keep) {
                                 const int slot = atomicAdd(cnt_u + qb + qq, 1);
-                                if (slot < p.cand_cap) {
-                                    const long long off = list0 + (long long)(qb + qq) * p.cand_cap + slot;
-                                    p.cand_val[off] = sc[qq];
-                                    p.cand_idx[off] = j;
-                                }
+                                if (slot < p.cand_cap)
+                                    p.cand[list0 + (long long)(qb + qq) * p.cand_cap + slot] = make_int2(sc[qq], j);
                             }
                         }
                     }

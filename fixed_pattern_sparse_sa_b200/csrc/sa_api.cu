@@ -633,7 +633,7 @@ static int indexer_chunk_rows(int B, int Tq, int nq_block, int m_cap, int cap) {
 struct IdxLayout {
     bool decode, filter_tc;
     int nq, m_cap, cap, rt;
-    size_t sample_off, tau_off, cnt_off, val_off, idx_off, qf_off, wf_off, total;
+    size_t sample_off, tau_off, cnt_off, cand_off, qf_off, wf_off, total;
 };
 
 // The persistent filter kernel (indexer_filter.cuh) serves prefill-shaped
@@ -661,8 +661,7 @@ static IdxLayout indexer_layout(int B, int Tq, int L, int Hi, int di, int topk) 
     l.sample_off = off; off += round_up(rows * l.m_cap * 4, 256);
     l.tau_off = off; off += round_up(rows * 4, 256);
     l.cnt_off = off; off += round_up(rows * 4, 256);
-    l.val_off = off; off += round_up(rows * l.cap * 4, 256);
-    l.idx_off = off; off += round_up(rows * l.cap * 4, 256);
+    l.cand_off = off; off += round_up(rows * l.cap * 8, 256);
     // weights folded into the query operand (persistent filter kernel only)
     l.qf_off = off; off += l.filter_tc ? round_up((size_t)B * Tq * Hi * di, 256) : 0;
     l.wf_off = off; off += l.filter_tc ? round_up((size_t)B * Tq * Hi * 4, 256) : 0;
@@ -849,8 +848,7 @@ int sa_indexer_topk(const int8_t *q_idx, const int8_t *k_idx, const int32_t *w, 
     p.sample = reinterpret_cast<int32_t *>(ws + lay.sample_off);
     p.tau = reinterpret_cast<int32_t *>(ws + lay.tau_off);
     p.cand_cnt = reinterpret_cast<int32_t *>(ws + lay.cnt_off);
-    p.cand_val = reinterpret_cast<int32_t *>(ws + lay.val_off);
-    p.cand_idx = reinterpret_cast<int32_t *>(ws + lay.idx_off);
+    p.cand = reinterpret_cast<int2 *>(ws + lay.cand_off);
     p.out_idx = out_idx; p.out_count = out_count; p.err = ew;
     int8_t *qf = reinterpret_cast<int8_t *>(ws + lay.qf_off);
     int32_t *wf = reinterpret_cast<int32_t *>(ws + lay.wf_off);

@@ -231,3 +231,32 @@ def test_bad_index_sets_device_error_word(cuda_ok):
     idx2 = idx.clone(); idx2[0, 2, 1] = -1
     ro, _ = oracle.sparse_attn(g["q"], g["k"], g["v"], idx2)
     assert_out_close(out, ro)
+
+
+@pytest.mark.parametrize("scale", [-0.3, 0.0, 0.21])
+@pytest.mark.parametrize("d,Hq", [(128, 16), (64, 4)])
+def test_explicit_scale_signs(cuda_ok, scale, d, Hq):
+    """Any scale, including negative (folded into Q's sign) and zero (uniform
+    weights over each row's keys); ragged lists leave partial chunks whose
+    empty entries must get exactly zero weight."""
+    B, T, K = 1, 90, 45
+    g = inputs.gen_dsa(B, T, Hq, 1, d, 1, 32, seed=int(scale * 100) + d)
+    idx = _random_lists(B, T, 1, K, seed=d + 5, fill=0.7)
+    out, lse = api.sparse_attn_fwd(g["q"].cuda(), g["k"].cuda(), g["v"].cuda(), idx.cuda(), scale=scale)
+    ro, rl = oracle.sparse_attn(g["q"], g["k"], g["v"], idx, scale=scale)
+    assert_out_close(out, ro)
+    assert_lse_close(lse, rl)
+
+
+@pytest.mark.parametrize("scale", [-0.15, 0.0])
+def test_fixed_pattern_bias_with_explicit_scale(cuda_ok, scale):
+    T, H, d = 300, 16, 128
+    g = inputs.gen_spatial(1, T, H, d, beta=0.5, seed=11)
+    gd = to_dev(g)
+    out, lse = api.sparse_attn_fwd(gd["q"], gd["k"], gd["v"], pattern=(65, True), cq=gd["cq"], ck=gd["ck"],
+                                   beta=gd["beta"], scale=scale)
+    idx, _ = oracle.fixed_graph(T, 65, True, cap=100)
+    ro, rl = oracle.sparse_attn(g["q"], g["k"], g["v"], idx.reshape(1, T, -1), cq=g["cq"], ck=g["ck"],
+                                beta=g["beta"], scale=scale)
+    assert_out_close(out, ro)
+    assert_lse_close(lse, rl)
