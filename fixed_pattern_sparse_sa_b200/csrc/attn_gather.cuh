@@ -316,10 +316,10 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
     const __nv_bfloat16 *lb = KLO ? p.klo + ((long long)b * p.Lk * p.Hkv + g) * D : nullptr;
     const long long rstride = (long long)p.Hkv * D;
     // copy lanes: lane = lrow * UNITS + u (u: 16-byte unit of a row, lrow: row within an instruction)
-    constexpr int RPI = 32 / UNITS;
-    const int lrow_c = lane / UNITS, u_c = lane % UNITS;
-    const __nv_bfloat16 *kb_u = kb + u_c * 8, *vb_u = vb + u_c * 8;
-    const __nv_bfloat16 *lb_u = KLO ? lb + u_c * 8 : nullptr;
+    [[maybe_unused]] constexpr int RPI = 32 / UNITS;
+    [[maybe_unused]] const int lrow_c = lane / UNITS, u_c = lane % UNITS;
+    [[maybe_unused]] const __nv_bfloat16 *kb_u = kb + u_c * 8, *vb_u = vb + u_c * 8;
+    [[maybe_unused]] const __nv_bfloat16 *lb_u = KLO ? lb + u_c * 8 : nullptr;
 
     // raw list value of chunk ci for this lane (lane i < NK owns key i)
     auto raw_of = [&](int ci) -> int {
@@ -380,23 +380,40 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
             return;
         }
         if (ci < n_chunks) {
-            // UNITS lanes per key row, RPI = 32 / UNITS rows per instruction,
-            // so every copy instruction covers whole 128-byte lines.  Lane
-            // (lrow, u) copies unit u of rows it * RPI + lrow to the swizzled
-            // unit u ^ (row & 7); with the stage on a 256-byte boundary that
-            // address is (base ^ (((it * RPI) & 7) << 4)) + it * RPI * ROWB,
-            // one XOR per row; the row offsets are immediates.
-            const uint32_t base = tc::smem_u32(ks_) + lrow_c * ROWB + ((u_c ^ lrow_c) << 4);
-            static_for<CP_ITERS>([&](auto ic) {
-                constexpr int it = decltype(ic)::value;
-                const int jr = __shfl_sync(0xffffffffu, j, it * RPI + lrow_c);
-                const long long jo = (long long)max(jr, 0) * rstride;
-                const int nb = jr >= 0 ? 16 : 0;
-                const uint32_t dst = base ^ (uint32_t)(((it * RPI) & 7) << 4);
-                cp_async16_at<it * RPI * ROWB, 0>(dst, kb_u + jo, nb);
-                cp_async16_at<it * RPI * ROWB + CH, 0>(dst, vb_u + jo, nb);
-                if constexpr (KLO) cp_async16_at<it * RPI * ROWB + 2 * CH, 0>(dst, lb_u + jo, nb);
-            });
+            if constexpr (D == 128) {
+                // UNITS lanes per key row, RPI = 32 / UNITS rows per instruction,
+                // so every copy instruction covers whole 128-byte lines.  Lane
+                // (lrow, u) copies unit u of rows it * RPI + lrow to the swizzled
+                // unit u ^ (row & 7); with the stage on a 256-byte boundary that
+                // address is (base ^ (((it * RPI) & 7) << 4)) + it * RPI * ROWB,
+                // one XOR per row; the row offsets are immediates.
+                const uint32_t base = tc::smem_u32(ks_) + lrow_c * ROWB + ((u_c ^ lrow_c) << 4);
+                static_for<CP_ITERS>([&](auto ic) {
+                    constexpr int it = decltype(ic)::value;
+                    const int jr = __shfl_sync(0xffffffffu, j, it * RPI + lrow_c);
+                    const long long jo = (long long)max(jr, 0) * rstride;
+                    const int nb = jr >= 0 ? 16 : 0;
+                    const uint32_t dst = base ^ (uint32_t)(((it * RPI) & 7) << 4);
+                    cp_async16_at<it * RPI * ROWB, 0>(dst, kb_u + jo, nb);
+                    cp_async16_at<it * RPI * ROWB + CH, 0>(dst, vb_u + jo, nb);
+                    if constexpr (KLO) cp_async16_at<it * RPI * ROWB + 2 * CH, 0>(dst, lb_u + jo, nb);
+                });
+            } else {
+                // head dim 64 (measured faster for the fixed-graph rows): the
+                // same lane mapping with addresses formed per copy
+#pragma unroll
+                for (int it = 0; it < CP_ITERS; ++it) {
+                    const int lin = it * 32 + lane;
+                    const int rr = lin / UNITS, u = lin % UNITS;
+                    const int jr = __shfl_sync(0xffffffffu, j, rr);
+                    const long long off = jr >= 0 ? (long long)jr * rstride + u * 8 : 0;
+                    const int nb = jr >= 0 ? 16 : 0;
+                    const int sw = (u ^ (rr & 7)) * 16;
+                    cp_async16(ks_ + rr * ROWB + sw, kb + off, nb);
+                    cp_async16(vs_ + rr * ROWB + sw, vb + off, nb);
+                    if constexpr (KLO) cp_async16(vs_ + CH + rr * ROWB + sw, lb + off, nb);
+                }
+            }
         }
         cp_async_commit();
     };

@@ -120,6 +120,12 @@ __global__ void __launch_bounds__(256) idx_fold_kernel(const int8_t *__restrict_
 }
 
 namespace ft {
+// Shared-memory counter increment that returns the old value.
+__device__ __forceinline__ int atom_add1_shared(uint32_t addr) {
+    int old;
+    asm volatile("atom.shared.add.u32 %0, [%1], 1;\n" : "=r"(old) : "r"(addr));
+    return old;
+}
 // 32 lanes x 32 consecutive 32-bit columns
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t *r) {
     asm volatile(
@@ -353,6 +359,9 @@ __global__ void __launch_bounds__(FT_THREADS, 1)
                 for (int q = 0; q < NQT; ++q) tau_r[q] = fast ? ft_fast_tau(tau_u[q]) : tau_u[q];
             }
             const long long list0 = ((long long)b * p.Rt + (tq0 + q_lo - p.t0)) * p.cand_cap;
+            int2 *const lbase = p.cand + list0;             // this warp's first query's list
+            const int cap = p.cand_cap;
+            const uint32_t cnt_a = tc::smem_u32(cnt_u);
             for (int k = 0; k < nt; ++k, ++tile) {
                 const int ab = tile & 1;
                 if (!bad && !atc::wait(acc_full + ab, (tile >> 1) & 1, abort_flag)) {
@@ -411,19 +420,16 @@ __global__ void __launch_bounds__(FT_THREADS, 1)
                             for (int qq = 0; qq < NG; ++qq)
                                 if (j >= nc_u[qb + qq]) mask &= ~(1u << qq);
                         }
-                        // per query: skipped by the whole warp when no lane
-                        // keeps it, else every keeping lane takes its slot with
-                        // its own shared-memory atomic (one per kept pair: ~10%
-                        // of the pairs, fewer instructions than reserving a
-                        // warp's slots by ballot, shuffle and popcount)
+                        // every keeping lane takes its list slot with its own
+                        // shared-memory atomic (one per kept pair, ~10% of the
+                        // pairs: fewer instructions than reserving a warp's
+                        // slots by ballot, shuffle and popcount) and stores
+                        // the pair; 32-bit offsets from the unit's list base
 #pragma unroll
                         for (int qq = 0; qq < NG; ++qq) {
-                            const bool keep = (mask >> qq) & 1u;
-                            if (!__any_sync(0xffffffffu, keep)) continue;   // warp-uniform
-                            if (keep) {
-                                const int slot = atomicAdd(cnt_u + qb + qq, 1);
-                                if (slot < p.cand_cap)
-                                    p.cand[list0 + (long long)(qb + qq) * p.cand_cap + slot] = make_int2(sc[qq], j);
+                            if ((mask >> qq) & 1u) {
+                                const int slot = ft::atom_add1_shared(cnt_a + 4u * (uint32_t)(qb + qq));
+                                if (slot < cap) lbase[(qb + qq) * cap + slot] = make_int2(sc[qq], j);
                             }
                         }
                     }

@@ -4,6 +4,7 @@
 // computation runs in the kernels of attn_gather.cuh, indexer.cuh and
 // nsa_misc.cuh.  There is no CPU fallback.
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <atomic>
@@ -44,6 +45,29 @@ static int fail(int code, const char *fmt, ...) {
 
 // Kernels enqueued by this process (all devices), for launch accounting.
 static std::atomic<unsigned long long> g_launches{0};
+
+// SA_LOG=1 in the environment prints every kernel launch (name, grid, block,
+// dynamic shared memory) to stderr.
+static bool log_enabled() {
+    static const bool on = [] {
+        const char *e = std::getenv("SA_LOG");
+        return e && *e && std::strcmp(e, "0") != 0;
+    }();
+    return on;
+}
+static void log_launch(const char *name, dim3 g, dim3 b, size_t smem) {
+    if (log_enabled())
+        std::fprintf(stderr, "[sa] %s grid=(%u,%u,%u) block=(%u,%u,%u) smem=%zu\n", name, g.x, g.y, g.z, b.x, b.y,
+                     b.z, smem);
+}
+
+// NVTX range around each C-ABI call (visible to profilers and tracers;
+// a no-op when none is attached).
+struct TraceRange {
+    explicit TraceRange(const char *name) { nvtxRangePushA(name); }
+    ~TraceRange() { nvtxRangePop(); }
+};
+#define SA_TRACE(name) TraceRange sa_trace_range_(name)
 
 #define SA_CHECK_LAUNCH(what)                                                              \
     do {                                                                                   \
@@ -169,7 +193,7 @@ static bool gather_tma_allowed() {
 
 // -------------------------------------------------------- gather launches --
 // Launch shape: 12 warps per CTA streaming 16-key chunks through a 2-stage
-// ring (8 warps when the lo-key tile is also staged); ~198 KB of shared
+// ring (8 warps when the lo-key tile is also staged); ~200 KB of shared
 // memory, one CTA and 12 gathering warps per SM.  Small launches (fewer
 // items than 12 per SM, e.g. decode with a few hundred split pieces) use
 // 4-warp CTAs so that every SM gets work.
@@ -185,7 +209,8 @@ static int launch_gather_nw(const GatherParams &p, long long items, cudaStream_t
     if (rc) return rc;
     static const CUtensorMap unused{};                   // the row-gather modes take no tensor map
     const long long blocks = (items + NW - 1) / NW;
-    kern<<<(unsigned)blocks, NW * 32, smem, st>>>(p, km ? *km : unused, vm ? *vm : unused);
+    log_launch(__PRETTY_FUNCTION__, (unsigned)blocks, NW * 32, smem),
+        kern<<<(unsigned)blocks, NW * 32, smem, st>>>(p, km ? *km : unused, vm ? *vm : unused);
     SA_CHECK_LAUNCH("gather_attn_kernel");
     return SA_OK;
 }
@@ -227,6 +252,8 @@ static int launch_gather_t(const GatherParams &p, cudaStream_t st) {
     if constexpr (KLO) {
         return launch_gather_nw<D, SRC, BIAS, KLO, 8>(p, items, st);
     } else {
+        // small launches (decode pieces): 4-warp CTAs, 2-stage ring (a 6-stage
+        // ring measured slower for the 128K decode)
         if (items < (long long)sm_count() * SA_ATTN_NW) return launch_gather_nw<D, SRC, BIAS, KLO, 4>(p, items, st);
         return launch_gather_nw<D, SRC, BIAS, KLO, SA_ATTN_NW>(p, items, st);
     }
@@ -301,7 +328,7 @@ static int launch_attn_tc(const GatherParams &p, cudaStream_t st) {
     rc = set_smem(kern, smem);
     if (rc) return rc;
     const int grid = (int)std::min<long long>(items, sm_count());
-    kern<<<grid, ATC_THREADS, smem, st>>>(qm, km, vm, ap);
+    log_launch(__PRETTY_FUNCTION__, grid, ATC_THREADS, smem), kern<<<grid, ATC_THREADS, smem, st>>>(qm, km, vm, ap);
     SA_CHECK_LAUNCH("attn_tc_kernel");
     return SA_OK;
 }
@@ -311,9 +338,11 @@ static int launch_combine(const float *po, const float *pl, int n_split, long lo
     if (rows == 0) return SA_OK;
     const unsigned blocks = (unsigned)((rows + 7) / 8);
     if (d == 64)
-        lse_combine_kernel<64><<<blocks, 256, 0, st>>>(po, pl, n_split, rows, (__nv_bfloat16 *)out, lse);
+        log_launch("lse_combine_kernel<64>", blocks, 256, 0),
+            lse_combine_kernel<64><<<blocks, 256, 0, st>>>(po, pl, n_split, rows, (__nv_bfloat16 *)out, lse);
     else if (d == 128)
-        lse_combine_kernel<128><<<blocks, 256, 0, st>>>(po, pl, n_split, rows, (__nv_bfloat16 *)out, lse);
+        log_launch("lse_combine_kernel<128>", blocks, 256, 0),
+            lse_combine_kernel<128><<<blocks, 256, 0, st>>>(po, pl, n_split, rows, (__nv_bfloat16 *)out, lse);
     else
         return fail(SA_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
     SA_CHECK_LAUNCH("lse_combine_kernel");
@@ -342,6 +371,7 @@ const char *sa_status_string(int s) {
 }
 
 int sa_check_device_status(void *stream) {
+    SA_TRACE("sa_check_device_status");
     unsigned *ew = nullptr;
     int rc = device_error_word(&ew);
     if (rc) return rc;
@@ -406,6 +436,7 @@ int sa_sparse_attn_fwd(const void *q, const void *k, const void *v, int B, int T
                        const float *beta, float scale, int n_split, void *out, float *lse,
                        float *part_o, float *part_lse, void *workspace, size_t workspace_bytes,
                        void *stream) {
+    SA_TRACE("sa_sparse_attn_fwd");
     if (B <= 0 || Tq < 0 || L <= 0 || Hq <= 0 || Hkv <= 0 || n_split < 1)
         return fail(SA_ERR_INVALID_ARG, "sparse_attn: bad sizes B=%d Tq=%d L=%d Hq=%d Hkv=%d n_split=%d",
                     B, Tq, L, Hq, Hkv, n_split);
@@ -550,6 +581,7 @@ int sa_sparse_attn_fwd_split_static(const void *q, const void *k, const void *v,
                                     int Hq, int Hkv, int d, int64_t q_pos0, const int32_t *idx,
                                     int idx_heads, int K, float scale, int n_split, void *out,
                                     float *lse, void *stream) {
+    SA_TRACE("sa_sparse_attn_fwd_split_static");
     if (n_split < 2) return fail(SA_ERR_INVALID_ARG, "split_static: n_split must be >= 2 (got %d)", n_split);
     if (!idx || !out) return fail(SA_ERR_INVALID_ARG, "split_static: idx and out are required");
     if (B <= 0 || Tq < 0 || Hq <= 0 || (d != 64 && d != 128))
@@ -582,6 +614,7 @@ int sa_sparse_attn_fwd_split_static(const void *q, const void *k, const void *v,
 
 int sa_lse_combine(const float *part_o, const float *part_lse, int n_split, int64_t rows, int d,
                    void *out, float *lse, void *stream) {
+    SA_TRACE("sa_lse_combine");
     if (n_split < 1 || rows < 0) return fail(SA_ERR_INVALID_ARG, "lse_combine: n_split=%d rows=%lld", n_split, (long long)rows);
     if (d != 64 && d != 128) return fail(SA_ERR_UNSUPPORTED, "lse_combine: head dim %d", d);
     if (!part_o || !part_lse || !out || !aligned16(part_o) || !aligned4(part_lse) || !aligned16(out))
@@ -685,7 +718,7 @@ static int launch_score_t(const IdxParams &p, long long n_keys_max, cudaStream_t
     if (rc) return rc;
     dim3 grid((unsigned)((n_keys_max + TC_KT * 128 - 1) / (TC_KT * 128)), (unsigned)((p.Rt + NQ - 1) / NQ),
               (unsigned)p.B);
-    kern<<<grid, tc_threads(NCOL), smem, st>>>(p);
+    log_launch(__PRETTY_FUNCTION__, grid, tc_threads(NCOL), smem), kern<<<grid, tc_threads(NCOL), smem, st>>>(p);
     SA_CHECK_LAUNCH("idx_score_tc_kernel");
     return SA_OK;
 }
@@ -693,7 +726,8 @@ static int launch_score_t(const IdxParams &p, long long n_keys_max, cudaStream_t
 template <int DI, int MODE>
 static int launch_dp4a_t(const IdxParams &p, long long n_keys_max, cudaStream_t st) {
     dim3 grid((unsigned)((n_keys_max + DEC_KEYS - 1) / DEC_KEYS), (unsigned)p.Rt, (unsigned)p.B);
-    idx_score_dp4a_kernel<DI, MODE><<<grid, DEC_THREADS, 0, st>>>(p);
+    log_launch("idx_score_dp4a_kernel<DI, MODE>", grid, DEC_THREADS, 0),
+        idx_score_dp4a_kernel<DI, MODE><<<grid, DEC_THREADS, 0, st>>>(p);
     SA_CHECK_LAUNCH("idx_score_dp4a_kernel");
     return SA_OK;
 }
@@ -702,7 +736,8 @@ template <int MODE>
 static int launch_dec_mma_t(const IdxParams &p, long long n_keys_max, cudaStream_t st) {
     constexpr int kpc = dmma_keys(MODE);
     dim3 grid((unsigned)((n_keys_max + kpc - 1) / kpc), (unsigned)p.Rt, (unsigned)p.B);
-    idx_score_dec_mma_kernel<MODE><<<grid, DMMA_THREADS, 0, st>>>(p);
+    log_launch("idx_score_dec_mma_kernel<MODE>", grid, DMMA_THREADS, 0),
+        idx_score_dec_mma_kernel<MODE><<<grid, DMMA_THREADS, 0, st>>>(p);
     SA_CHECK_LAUNCH("idx_score_dec_mma_kernel");
     return SA_OK;
 }
@@ -768,7 +803,7 @@ static int launch_filter_tc_t(const IdxParams &p, const int8_t *qf, const int32_
     rc = set_smem(kern, smem);
     if (rc) return rc;
     const int grid = (int)std::min<long long>(n_units, sm_count());
-    kern<<<grid, FT_THREADS, smem, st>>>(am, bm, fp);
+    log_launch(__PRETTY_FUNCTION__, grid, FT_THREADS, smem), kern<<<grid, FT_THREADS, smem, st>>>(am, bm, fp);
     SA_CHECK_LAUNCH("idx_filter_tc_kernel");
     return SA_OK;
 }
@@ -787,9 +822,12 @@ static int launch_filter_tc_d(const IdxParams &p, const int8_t *qf, const int32_
 static int launch_fold(const IdxParams &p, int8_t *qf, int32_t *wf, cudaStream_t st) {
     const long long n = (long long)p.B * p.Tq * p.Hi;
     const unsigned blocks = (unsigned)((n + 255) / 256);
-    if (p.di == 32) idx_fold_kernel<32><<<blocks, 256, 0, st>>>(p.q, p.w, qf, wf, n);
-    else if (p.di == 64) idx_fold_kernel<64><<<blocks, 256, 0, st>>>(p.q, p.w, qf, wf, n);
-    else idx_fold_kernel<128><<<blocks, 256, 0, st>>>(p.q, p.w, qf, wf, n);
+    if (p.di == 32) log_launch("idx_fold_kernel<32>", blocks, 256, 0),
+        idx_fold_kernel<32><<<blocks, 256, 0, st>>>(p.q, p.w, qf, wf, n);
+    else if (p.di == 64) log_launch("idx_fold_kernel<64>", blocks, 256, 0),
+        idx_fold_kernel<64><<<blocks, 256, 0, st>>>(p.q, p.w, qf, wf, n);
+    else log_launch("idx_fold_kernel<128>", blocks, 256, 0),
+        idx_fold_kernel<128><<<blocks, 256, 0, st>>>(p.q, p.w, qf, wf, n);
     SA_CHECK_LAUNCH("idx_fold_kernel");
     return SA_OK;
 }
@@ -801,7 +839,8 @@ static int launch_select_nt(const IdxParams &p, int words, cudaStream_t st) {
     auto kern = topk_select_kernel<DI, NT>;
     int rc = set_smem(kern, smem);
     if (rc) return rc;
-    kern<<<dim3(1u, (unsigned)p.Rt, (unsigned)p.B), NT, smem, st>>>(p);
+    log_launch(__PRETTY_FUNCTION__, dim3(1u, (unsigned)p.Rt, (unsigned)p.B),
+        NT, smem), kern<<<dim3(1u, (unsigned)p.Rt, (unsigned)p.B), NT, smem, st>>>(p);
     SA_CHECK_LAUNCH("topk_select_kernel");
     return SA_OK;
 }
@@ -815,6 +854,7 @@ static int launch_select_t(const IdxParams &p, int words, cudaStream_t st) {
 int sa_indexer_topk(const int8_t *q_idx, const int8_t *k_idx, const int32_t *w, int B, int Tq, int L,
                     int Hi, int di, int64_t q_pos0, int topk, int window, int32_t *out_idx,
                     int32_t *out_count, void *workspace, size_t workspace_bytes, void *stream) {
+    SA_TRACE("sa_indexer_topk");
     if (B <= 0 || Tq < 0 || L <= 0 || topk < 0 || window < 0 || topk + window < 1)
         return fail(SA_ERR_INVALID_ARG, "indexer_topk: bad sizes B=%d Tq=%d L=%d topk=%d window=%d", B, Tq,
                     L, topk, window);
@@ -867,7 +907,8 @@ int sa_indexer_topk(const int8_t *q_idx, const int8_t *k_idx, const int32_t *w, 
         if (ncand > 0) {
             rc = launch_score<MODE_SAMPLE>(p, lay.decode, (long long)lay.m_cap, st);
             if (rc) return rc;
-            idx_threshold_kernel<<<dim3(1u, (unsigned)rows, (unsigned)B), SEL_THREADS, 0, st>>>(p);
+            log_launch("idx_threshold_kernel", dim3(1u, (unsigned)rows, (unsigned)B),
+                SEL_THREADS, 0), idx_threshold_kernel<<<dim3(1u, (unsigned)rows, (unsigned)B), SEL_THREADS, 0, st>>>(p);
             SA_CHECK_LAUNCH("idx_threshold_kernel");
             if (filter_tc)
                 rc = di == 32 ? launch_filter_tc_d<32>(p, qf, wf, st)
@@ -923,7 +964,8 @@ static int launch_nsa_select(const NsaSelectParams &p, cudaStream_t st) {
     int rc = set_smem(kern, smem);
     if (rc) return rc;
     const long long ctas = (long long)p.B * p.Hkv * ((p.T + NSA_TW - 1) / NSA_TW);
-    kern<<<(unsigned)ctas, NSA_TW * 32, smem, st>>>(p);
+    log_launch(__PRETTY_FUNCTION__, (unsigned)ctas, NSA_TW * 32, smem),
+        kern<<<(unsigned)ctas, NSA_TW * 32, smem, st>>>(p);
     SA_CHECK_LAUNCH("nsa_select_kernel");
     return SA_OK;
 }
@@ -940,7 +982,8 @@ static int launch_tile_t(const TileParams &p, cudaStream_t st) {
     if (rc) return rc;
     const long long ctas = (long long)p.B * p.Hkv * ((p.T + kTileWarps - 1) / kTileWarps);
     if (ctas == 0) return SA_OK;
-    kern<<<(unsigned)ctas, kTileWarps * 32, smem, st>>>(p);
+    log_launch(__PRETTY_FUNCTION__, (unsigned)ctas, kTileWarps * 32, smem),
+        kern<<<(unsigned)ctas, kTileWarps * 32, smem, st>>>(p);
     SA_CHECK_LAUNCH("tile_attn_kernel");
     return SA_OK;
 }
@@ -967,7 +1010,8 @@ static int launch_nsa_tc(const TileParams &p, unsigned *err, cudaStream_t st) {
     rc = set_smem(kern, smem);
     if (rc) return rc;
     const int grid = (int)std::min<long long>(items, sm_count());   // persistent: one CTA per SM
-    kern<<<grid, NT_THREADS, smem, st>>>(qm, khm, klm, vm, cp);
+    log_launch(__PRETTY_FUNCTION__, grid, NT_THREADS, smem),
+        kern<<<grid, NT_THREADS, smem, st>>>(qm, khm, klm, vm, cp);
     SA_CHECK_LAUNCH("nsa_tc_kernel");
     return SA_OK;
 }
@@ -993,7 +1037,8 @@ static int launch_imp_tc(const NsaSelectParams &sp, unsigned *err, cudaStream_t 
     rc = set_smem(nsa_imp_tc_kernel, smem);
     if (rc) return rc;
     const int grid = (int)std::min<long long>(items, sm_count());
-    nsa_imp_tc_kernel<<<grid, IT_THREADS, smem, st>>>(qm, khm, klm, ip);
+    log_launch("nsa_imp_tc_kernel", grid, IT_THREADS, smem),
+        nsa_imp_tc_kernel<<<grid, IT_THREADS, smem, st>>>(qm, khm, klm, ip);
     SA_CHECK_LAUNCH("nsa_imp_tc_kernel");
     return SA_OK;
 }
@@ -1024,6 +1069,7 @@ int sa_nsa_fwd(const void *q, const void *k, const void *v, const float *gates, 
                int Hkv, int d, int cmp_len, int cmp_stride, int sel_block, int sel_topk, int window,
                float scale, void *out, float *lse_branches, int32_t *sel_idx_out, void *workspace,
                size_t workspace_bytes, void *stream) {
+    SA_TRACE("sa_nsa_fwd");
     if (B <= 0 || T < 0 || Hq <= 0 || Hkv <= 0 || cmp_len <= 0 || cmp_stride <= 0 || sel_block <= 0 ||
         sel_topk <= 0 || window <= 0)
         return fail(SA_ERR_INVALID_ARG, "nsa: bad sizes");
@@ -1058,7 +1104,8 @@ int sa_nsa_fwd(const void *q, const void *k, const void *v, const float *gates, 
     // 1. compression
     if (lay.nc > 0) {
         const long long n2 = (long long)B * lay.nc * Hkv * (d / 2);
-        nsa_compress_kernel<<<(unsigned)((n2 + 255) / 256), 256, 0, st>>>(
+        log_launch("nsa_compress_kernel", (unsigned)((n2 + 255) / 256),
+            256, 0), nsa_compress_kernel<<<(unsigned)((n2 + 255) / 256), 256, 0, st>>>(
             (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, B, T, Hkv, d, lay.nc, cmp_len, cmp_stride,
             kc, klo, vc);
         SA_CHECK_LAUNCH("nsa_compress_kernel");
@@ -1120,11 +1167,13 @@ int sa_nsa_fwd(const void *q, const void *k, const void *v, const float *gates, 
     // 6. gated sum
     {
         const long long n2 = rows * (d / 2);
-        nsa_gate_kernel<<<(unsigned)((n2 + 255) / 256), 256, 0, st>>>(o3, rows * d, gates, rows, d,
+        log_launch("nsa_gate_kernel", (unsigned)((n2 + 255) / 256),
+            256, 0), nsa_gate_kernel<<<(unsigned)((n2 + 255) / 256), 256, 0, st>>>(o3, rows * d, gates, rows, d,
                                                                        (__nv_bfloat16 *)out);
         SA_CHECK_LAUNCH("nsa_gate_kernel");
         if (lse_branches) {
-            nsa_lse_pack_kernel<<<(unsigned)((rows + 255) / 256), 256, 0, st>>>(l3, rows, lse_branches);
+            log_launch("nsa_lse_pack_kernel", (unsigned)((rows + 255) / 256),
+                256, 0), nsa_lse_pack_kernel<<<(unsigned)((rows + 255) / 256), 256, 0, st>>>(l3, rows, lse_branches);
             SA_CHECK_LAUNCH("nsa_lse_pack_kernel");
         }
     }
@@ -1144,6 +1193,7 @@ int sa_dsa_decode_layers(const char *pattern, int n_layers, const sa_dsa_layer *
                          int L, int Hq, int Hkv, int d, int Hi, int di, int64_t q_pos0, int topk,
                          int window, float scale, int n_split, int32_t *idx_cache, void *workspace,
                          size_t workspace_bytes, void *stream) {
+    SA_TRACE("sa_dsa_decode_layers");
     if (!pattern || !layers || n_layers <= 0 || (int)strlen(pattern) < n_layers)
         return fail(SA_ERR_INVALID_ARG, "dsa_layers: pattern/layers");
     if (pattern[0] != 'F') return fail(SA_ERR_INVALID_ARG, "dsa_layers: the first layer must be 'F'");
@@ -1181,13 +1231,14 @@ static int launch_probe(const ProbeParams &p, int ctas, int smem, cudaStream_t s
     auto kern = probe_gather_kernel<MODE, STAGES>;
     int rc = set_smem(kern, smem);
     if (rc) return rc;
-    kern<<<ctas, p.warps * 32, smem, st>>>(p);
+    log_launch(__PRETTY_FUNCTION__, ctas, p.warps * 32, smem), kern<<<ctas, p.warps * 32, smem, st>>>(p);
     SA_CHECK_LAUNCH("probe_gather_kernel");
     return SA_OK;
 }
 
 int sa_probe_gather(const void *buf, int64_t n_rows, int mode, int warps, int stages, int iters,
                     int ctas_per_sm, unsigned *sink, void *stream) {
+    SA_TRACE("sa_probe_gather");
     if (!buf || !sink || !aligned16(buf) || !aligned4(sink) || n_rows < 1 || n_rows > UINT_MAX)
         return fail(SA_ERR_INVALID_ARG, "probe_gather: buffer/sink/rows");
     if (mode < 0 || mode > 2) return fail(SA_ERR_INVALID_ARG, "probe_gather: mode %d", mode);
@@ -1221,7 +1272,8 @@ size_t sa_sparse_attn_bwd_workspace_size(int B, int Tq, int Hq) {
 template <int D>
 static int launch_bwd(const BwdParams &p, long long rows, cudaStream_t st) {
     constexpr int NW = 8;
-    attn_bwd_prep_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(p, rows);
+    log_launch("attn_bwd_prep_kernel<D>", (unsigned)((rows + 7) / 8),
+        256, 0), attn_bwd_prep_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(p, rows);
     SA_CHECK_LAUNCH("attn_bwd_prep_kernel");
     constexpr int smem = attn_bwd_smem_bytes<D, NW>();
     static_assert(smem <= 227 * 1024, "shared memory");
@@ -1230,7 +1282,8 @@ static int launch_bwd(const BwdParams &p, long long rows, cudaStream_t st) {
     if (rc) return rc;
     const long long items = (long long)p.B * p.Tq * p.Hkv * ((p.G + 15) / 16);
     if (items == 0) return SA_OK;
-    kern<<<(unsigned)((items + NW - 1) / NW), NW * 32, smem, st>>>(p);
+    log_launch(__PRETTY_FUNCTION__, (unsigned)((items + NW - 1) / NW),
+        NW * 32, smem), kern<<<(unsigned)((items + NW - 1) / NW), NW * 32, smem, st>>>(p);
     SA_CHECK_LAUNCH("attn_bwd_kernel");
     return SA_OK;
 }
@@ -1239,6 +1292,7 @@ int sa_sparse_attn_bwd(const void *q, const void *k, const void *v, const void *
                        const void *dout, int B, int Tq, int L, int Hq, int Hkv, int d, int64_t q_pos0,
                        const int32_t *idx, int idx_heads, int K, float scale, float *dq, float *dk, float *dv,
                        void *workspace, size_t workspace_bytes, void *stream) {
+    SA_TRACE("sa_sparse_attn_bwd");
     if (B <= 0 || Tq < 0 || L <= 0 || Hq <= 0 || Hkv <= 0 || K < 0 || Hq % Hkv)
         return fail(SA_ERR_INVALID_ARG, "attn_bwd: bad sizes B=%d Tq=%d L=%d Hq=%d Hkv=%d K=%d", B, Tq, L, Hq, Hkv, K);
     if (d != 64 && d != 128) return fail(SA_ERR_UNSUPPORTED, "attn_bwd: head dim %d", d);
@@ -1277,6 +1331,7 @@ int sa_sparse_attn_bwd(const void *q, const void *k, const void *v, const void *
 // ------------------------------------------------- sequence split (Star) --
 int sa_indexer_scores_at(const int8_t *q_idx, const int8_t *k_idx, const int32_t *w, int B, int Tq, int L, int Hi,
                          int di, const int32_t *idx, int K, int32_t *out_score, void *stream) {
+    SA_TRACE("sa_indexer_scores_at");
     if (B <= 0 || Tq < 0 || L <= 0 || K < 0) return fail(SA_ERR_INVALID_ARG, "scores_at: bad sizes");
     if (!indexer_shape_ok(Hi, di)) return fail(SA_ERR_UNSUPPORTED, "scores_at: Hi=%d di=%d", Hi, di);
     if (!q_idx || !k_idx || !w || !idx || !out_score || !aligned16(q_idx) || !aligned16(k_idx) || !aligned4(w) ||
@@ -1288,9 +1343,12 @@ int sa_indexer_scores_at(const int8_t *q_idx, const int8_t *k_idx, const int32_t
     if (rc) return rc;
     const unsigned blocks = (unsigned)((long long)B * Tq);
     cudaStream_t st = as_stream(stream);
-    if (di == 32) idx_scores_at_kernel<32><<<blocks, 128, 0, st>>>(q_idx, k_idx, w, B, Tq, L, Hi, idx, K, out_score, ew);
-    else if (di == 64) idx_scores_at_kernel<64><<<blocks, 128, 0, st>>>(q_idx, k_idx, w, B, Tq, L, Hi, idx, K, out_score, ew);
-    else idx_scores_at_kernel<128><<<blocks, 128, 0, st>>>(q_idx, k_idx, w, B, Tq, L, Hi, idx, K, out_score, ew);
+    if (di == 32) log_launch("idx_scores_at_kernel<32>", blocks, 128, 0),
+        idx_scores_at_kernel<32><<<blocks, 128, 0, st>>>(q_idx, k_idx, w, B, Tq, L, Hi, idx, K, out_score, ew);
+    else if (di == 64) log_launch("idx_scores_at_kernel<64>", blocks, 128, 0),
+        idx_scores_at_kernel<64><<<blocks, 128, 0, st>>>(q_idx, k_idx, w, B, Tq, L, Hi, idx, K, out_score, ew);
+    else log_launch("idx_scores_at_kernel<128>", blocks, 128, 0),
+        idx_scores_at_kernel<128><<<blocks, 128, 0, st>>>(q_idx, k_idx, w, B, Tq, L, Hi, idx, K, out_score, ew);
     SA_CHECK_LAUNCH("idx_scores_at_kernel");
     return SA_OK;
 }
@@ -1298,6 +1356,7 @@ int sa_indexer_scores_at(const int8_t *q_idx, const int8_t *k_idx, const int32_t
 int sa_topk_merge(const int32_t *cand_score, const int32_t *cand_idx, const int64_t *part_off, int n_parts,
                   int64_t rows, int kc, int topk, int window, int64_t q_pos, int32_t *out_idx, int32_t *out_count,
                   void *stream) {
+    SA_TRACE("sa_topk_merge");
     if (n_parts < 1 || n_parts > TM_MAX_PARTS || rows < 0 || kc < 0 || topk < 0 || window < 0 || q_pos < 0)
         return fail(SA_ERR_INVALID_ARG, "topk_merge: bad sizes (n_parts 1..%d)", TM_MAX_PARTS);
     if (topk > TM_MAX_K || (long long)n_parts * kc > TM_MAX_CAND)
@@ -1315,7 +1374,8 @@ int sa_topk_merge(const int32_t *cand_score, const int32_t *cand_idx, const int6
     const int smem = topk_merge_smem_bytes(n_parts * kc);
     int rc = set_smem(topk_merge_kernel, smem);
     if (rc) return rc;
-    topk_merge_kernel<<<(unsigned)rows, TM_THREADS, smem, as_stream(stream)>>>(
+    log_launch("topk_merge_kernel", (unsigned)rows, TM_THREADS, smem),
+        topk_merge_kernel<<<(unsigned)rows, TM_THREADS, smem, as_stream(stream)>>>(
         cand_score, cand_idx, mo, n_parts, rows, kc, topk, window, q_pos,
         out_idx, out_count);
     SA_CHECK_LAUNCH("topk_merge_kernel");
@@ -1323,10 +1383,13 @@ int sa_topk_merge(const int32_t *cand_score, const int32_t *cand_idx, const int6
 }
 
 int sa_index_shard(const int32_t *idx, int64_t n, int64_t key_lo, int64_t key_hi, int32_t *out, void *stream) {
+    SA_TRACE("sa_index_shard");
     if (n < 0 || key_lo < 0 || key_hi < key_lo || !idx || !out || !aligned4(idx) || !aligned4(out))
         return fail(SA_ERR_INVALID_ARG, "index_shard: bad arguments");
     if (n == 0) return SA_OK;
-    index_shard_kernel<<<(unsigned)((n + 255) / 256), 256, 0, as_stream(stream)>>>(idx, n, key_lo, key_hi, out);
+    const unsigned blocks = (unsigned)((n + 255) / 256);
+    log_launch("index_shard_kernel", blocks, 256, 0),
+        index_shard_kernel<<<blocks, 256, 0, as_stream(stream)>>>(idx, n, key_lo, key_hi, out);
     SA_CHECK_LAUNCH("index_shard_kernel");
     return SA_OK;
 }

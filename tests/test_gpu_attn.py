@@ -260,3 +260,25 @@ def test_fixed_pattern_bias_with_explicit_scale(cuda_ok, scale):
                                 beta=g["beta"], scale=scale)
     assert_out_close(out, ro)
     assert_lse_close(lse, rl)
+
+
+def test_sa_log_prints_launch_configs(cuda_ok):
+    """SA_LOG=1 prints one line per kernel launch with its grid, block and
+    shared memory (checked in a child process so the setting stays local)."""
+    import os
+    import subprocess
+    import sys
+    code = ("import torch\n"
+            "from fixed_pattern_sparse_sa_b200 import api, inputs\n"
+            "g = inputs.gen_dsa(1, 40, 16, 1, 128, 1, 32, seed=1)\n"
+            "idx = torch.randint(0, 40, (1, 40, 8), dtype=torch.int32)\n"
+            "idx = torch.where(idx <= torch.arange(40).view(1, 40, 1), idx, torch.full_like(idx, -1))\n"
+            "api.sparse_attn_fwd(g['q'].cuda(), g['k'].cuda(), g['v'].cuda(), idx.cuda())\n"
+            "torch.cuda.synchronize()\n")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, SA_LOG="1", PYTHONPATH=root)
+    r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stderr.splitlines() if ln.startswith("[sa] ")]
+    assert any("gather_attn" in ln or "launch_gather" in ln for ln in lines), r.stderr[-2000:]
+    assert all("grid=(" in ln and "block=(" in ln and "smem=" in ln for ln in lines)
