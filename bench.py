@@ -174,6 +174,9 @@ def main():
                              "nsa64k", "spatial16k"],
                     help="run only one of the extra measurements (for profiling captures of a "
                          "single workload); prints its numbers alone")
+    ap.add_argument("--decode-seq-len", type=int, default=0,
+                    help="cache length of the decode workload for profiling captures of a smaller "
+                         "case (default 131072); the JSON line names it")
     ap.add_argument("--decode-split", type=int, default=16,
                     help="split-KV pieces per decode row (the 2048 selected keys are cut into this many)")
     ap.add_argument("--cpu-sample-rows", type=int, default=0,
@@ -449,6 +452,8 @@ def extra_measurements(args, dev, torch, api, lib, inputs, flush, world, peaks, 
     # --- decode 32 x 131072, 4 layers ---
     if only in (None, "decode128k"):
         w = inputs.WORKLOADS["dsa_decode128k"]
+        if args.decode_seq_len:
+            w = dataclasses.replace(w, T=int(args.decode_seq_len))
         lays = [inputs.gen_decode_layer(w.B, w.T, w.Hq, w.Hkv, w.d, w.Hi, w.di, layer=i, seed=0,
                                         device=dev) for i in range(w.layers)]
         n_split = args.decode_split
@@ -483,7 +488,7 @@ def extra_measurements(args, dev, torch, api, lib, inputs, flush, world, peaks, 
             del graph
         dec["fsss_over_ffff"] = round(dec["FSSS"]["tokens_per_s"] / dec["FFFF"]["tokens_per_s"], 3)
         dec["n_split"] = n_split
-        res["decode128k"] = dec
+        res["decode128k" if w.T == 131072 else f"decode{w.T // 1024}k"] = dec
         del lays, wsd
         torch.cuda.empty_cache()
     # --- IndexCache on the 64K prefill: 4 layers, F S S S vs all-F ---

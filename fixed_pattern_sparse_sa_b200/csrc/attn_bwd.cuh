@@ -40,6 +40,7 @@ struct BwdParams {
 // D = sum_c dO[row, c] * O[row, c], one warp per row.
 template <int D>
 __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const BwdParams p, long long rows) {
+    grid_dependency_sync();
     const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= rows) return;
@@ -87,6 +88,7 @@ __device__ __forceinline__ void ldsm_tile16(unsigned (&a)[4], const unsigned cha
 
 template <int D, int NW>
 __global__ void __launch_bounds__(NW * 32) attn_bwd_kernel(const BwdParams p) {
+    grid_dependency_sync();
     constexpr int NK = 16;                  // keys per chunk
     constexpr int STAGES = 2;
     constexpr int ROWB = D * 2;

@@ -92,6 +92,7 @@ __global__ void __launch_bounds__(NT_THREADS, 1)
     nsa_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap khimap,
                   const __grid_constant__ CUtensorMap klomap, const __grid_constant__ CUtensorMap vmap,
                   const CmpTcParams cp) {
+    grid_dependency_sync();
     constexpr int D = 128;
     constexpr bool LO = SRC == TS_CMP;             // compressed keys carry a lo half
     using L = CtSmem;
@@ -446,6 +447,7 @@ struct ImpTcParams {
 __global__ void __launch_bounds__(IT_THREADS, 1)
     nsa_imp_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap khimap,
                       const __grid_constant__ CUtensorMap klomap, const ImpTcParams ip) {
+    grid_dependency_sync();
     constexpr int D = 128;
     using L = ItSmem;
     const TileParams &p = ip.t;

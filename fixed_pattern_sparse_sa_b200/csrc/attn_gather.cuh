@@ -200,6 +200,7 @@ __device__ __forceinline__ void merge_pieces_half(const float *part_o, const flo
 template <int D, int STAGES, int SRC, bool BIAS, bool KLO = false, int NK = 32, int NW = 4, bool TMAB = false>
 __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams p, const __grid_constant__ CUtensorMap kmap,
                                                               const __grid_constant__ CUtensorMap vmap) {
+    grid_dependency_sync();
     // NK keys per chunk, NW independent warps per CTA
     constexpr int ROWB = D * 2;            // bytes of one K/V row
     constexpr int UNITS = ROWB / 16;       // 16-byte units per row
@@ -424,10 +425,15 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
     bool timed_out = false;
 
+    // the list values of the first STAGES + 1 chunks are loaded together (one
+    // memory latency, not one per prologue chunk), then the prologue copies
+    // go out; in the loop, list values run two chunks ahead of their copies
+    int raw0[STAGES + 1];
 #pragma unroll
-    for (int ci = 0; ci < STAGES - 1; ++ci) issue(ci, raw_of(ci));
-    // list values are loaded two chunks ahead of the K/V copies that use them
-    int raw_a = raw_of(STAGES - 1), raw_b = raw_of(STAGES);
+    for (int ci = 0; ci <= STAGES; ++ci) raw0[ci] = raw_of(ci);
+#pragma unroll
+    for (int ci = 0; ci < STAGES - 1; ++ci) issue(ci, raw0[ci]);
+    int raw_a = raw0[STAGES - 1], raw_b = raw0[STAGES];
 
     for (int ci = 0; ci < n_chunks; ++ci) {
         const int raw = raw_a;

@@ -187,6 +187,7 @@ template <int D, int SRC>
 __global__ void __launch_bounds__(ATC_THREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                    const __grid_constant__ CUtensorMap vmap, const AtcParams ap) {
+    grid_dependency_sync();
     static_assert(D == 128, "the tensor-core gather path handles head dim 128");
     constexpr bool TMA = SRC == KS_BLOCKS;
     using L = AtcSmem<D>;

@@ -55,6 +55,7 @@ __device__ __forceinline__ long long tile_key_begin(const TileParams &p, long lo
 
 template <int D, int STAGES, int SRC, int TW>
 __global__ void __launch_bounds__(TW * 32) tile_attn_kernel(const TileParams p) {
+    grid_dependency_sync();
     constexpr bool KLO = SRC == TS_CMP;
     constexpr int NK = 32;
     constexpr int ROWB = D * 2;

@@ -27,6 +27,7 @@ template <int DI>
 __global__ void __launch_bounds__(128) idx_scores_at_kernel(const int8_t *q, const int8_t *k, const int32_t *w,
                                                             int B, int Tq, int L, int Hi, const int32_t *idx, int K,
                                                             int32_t *out, unsigned *err) {
+    grid_dependency_sync();
     __shared__ __align__(16) int8_t qrow_s[16 * DI];
     __shared__ int w_s[16];
     const long long row = blockIdx.x;                  // b * Tq + t
@@ -66,6 +67,7 @@ __global__ void __launch_bounds__(TM_THREADS) topk_merge_kernel(const int32_t *c
                                                                  const MergeOffsets part_off, int n_parts, long long rows,
                                                                  int kc, int topk, int window, long long q_pos,
                                                                  int32_t *out_idx, int32_t *out_count) {
+    grid_dependency_sync();
     extern __shared__ __align__(1024) unsigned char smem[];
     const int n = n_parts * kc;
     int *sv = reinterpret_cast<int *>(smem);                  // [n] scores
@@ -161,6 +163,7 @@ __global__ void __launch_bounds__(TM_THREADS) topk_merge_kernel(const int32_t *c
 
 // Global positions -> rows of the shard [key_lo, key_hi) (other entries -1).
 __global__ void index_shard_kernel(const int32_t *idx, long long n, long long key_lo, long long key_hi, int32_t *out) {
+    grid_dependency_sync();
     const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= n) return;
     const int j = idx[i];

@@ -126,6 +126,7 @@ __device__ __forceinline__ int add_relu(int S, int x) { return __viaddmax_s32(S,
 
 template <int HI, int DI, int NCOL, int MODE>
 __global__ void __launch_bounds__(tc_threads(NCOL), NCOL >= 64 ? 2 : 4) idx_score_tc_kernel(const IdxParams p) {
+    grid_dependency_sync();
     constexpr int TC_THREADS = tc_threads(NCOL);
     constexpr int PARTS = TC_THREADS / 128;  // column parts (4 warps each)
     constexpr int NQ = NCOL / HI;            // queries per CTA
@@ -457,6 +458,7 @@ constexpr int DEC_KEYS = 2048;
 
 template <int DI, int MODE>
 __global__ void __launch_bounds__(DEC_THREADS) idx_score_dp4a_kernel(const IdxParams p) {
+    grid_dependency_sync();
     __shared__ __align__(16) int8_t q_s[16 * DI];
     __shared__ int w_s[16];
     const int b = blockIdx.z, tr = blockIdx.y, t = p.t0 + tr;
@@ -542,6 +544,7 @@ __host__ __device__ constexpr int dmma_keys(int mode) { return mode == 0 ? DMMA_
 
 template <int MODE>
 __global__ void __launch_bounds__(DMMA_THREADS) idx_score_dec_mma_kernel(const IdxParams p) {
+    grid_dependency_sync();
     constexpr int DI = 64, HI = 8;
     __shared__ int lcnt_s, lbase_s;
     __shared__ int lval_s[MODE == MODE_FILTER ? DMMA_KEYS : 1];
@@ -837,6 +840,7 @@ __device__ __forceinline__ void stream_values(const int32_t *vals, int n, F f) {
 // sampling count) reach it.  A sample that is the whole row gives the exact
 // k-th largest score.  Rows whose every candidate is kept get INT_MIN.
 __global__ void __launch_bounds__(SEL_THREADS, 4) idx_threshold_kernel(const IdxParams p) {
+    grid_dependency_sync();
     __shared__ int hist[SEL_BINS];
     __shared__ int fine[SEL_FINE_BINS];
     __shared__ int scan_tmp[32];
@@ -844,6 +848,7 @@ __global__ void __launch_bounds__(SEL_THREADS, 4) idx_threshold_kernel(const Idx
     const int b = blockIdx.z, tr = blockIdx.y, t = p.t0 + tr;
     if (t >= p.Tq || tr >= p.Rt) return;
     const long long row = (long long)b * p.Rt + tr;
+    if (threadIdx.x == 0) p.cand_cnt[row] = 0;                // the filter pass appends from zero
     const int n = (int)n_candidates(p.q_pos0 + t, p.window);
     const int k_eff = n < p.topk ? n : p.topk;
     if (k_eff == n || k_eff == 0) {
@@ -937,6 +942,7 @@ __host__ __device__ constexpr int select_smem_staged(int words, int cap) {
 // equal keys, in ascending position order.
 template <int DI, int NT = SEL_THREADS>
 __global__ void __launch_bounds__(NT, NT <= 256 ? 3 : 1) topk_select_kernel(const IdxParams p) {
+    grid_dependency_sync();
     extern __shared__ __align__(1024) unsigned char smem[];
     int *hist = reinterpret_cast<int *>(smem);                          // [SEL_BINS]
     unsigned *tie_key = reinterpret_cast<unsigned *>(hist + SEL_BINS);  // [SEL_TIE_CAP]

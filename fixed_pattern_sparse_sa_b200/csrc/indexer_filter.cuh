@@ -86,6 +86,7 @@ template <int DI>
 __global__ void __launch_bounds__(256) idx_fold_kernel(const int8_t *__restrict__ q, const int32_t *__restrict__ w,
                                                        int8_t *__restrict__ qf, int32_t *__restrict__ wf,
                                                        long long n_heads) {
+    grid_dependency_sync();
     const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= n_heads) return;
     const int wv = __ldg(w + i);
@@ -178,6 +179,7 @@ template <int HI, int DI>
 __global__ void __launch_bounds__(FT_THREADS, 1)
     idx_filter_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap,
                          const FtParams fp) {
+    grid_dependency_sync();
     constexpr int NQ = FT_NCOL / HI;         // queries per unit
     constexpr int NQT = FT_CW / HI;          // queries per epilogue thread
     constexpr bool QREG = NQT <= 8;          // per-query constants held in registers

@@ -9,15 +9,18 @@ namespace sa {
 // Star Attention page ("NVIDIA AI Research presenta Star Attention ...",
 // body): per-piece softmax results merge by a distributed softmax,
 //   lse = log sum_s exp(lse_s),  o = sum_s exp(lse_s - lse) o_s.
-// One warp per row; each lane owns d/32 consecutive columns.
+// One warp per row (two rows per CTA, so that small calls spread over the
+// SMs); each lane owns d/32 consecutive columns.
+constexpr int COMBINE_ROWS = 2;
 template <int D>
-__global__ void __launch_bounds__(256) lse_combine_kernel(const float *__restrict__ part_o,
+__global__ void __launch_bounds__(COMBINE_ROWS * 32) lse_combine_kernel(const float *__restrict__ part_o,
                                                          const float *__restrict__ part_lse,
                                                          int n_split, long long rows,
                                                          __nv_bfloat16 *__restrict__ out,
                                                          float *__restrict__ lse) {
+    grid_dependency_sync();
     constexpr int PER = D / 32;
-    const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const long long row = (long long)blockIdx.x * COMBINE_ROWS + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= rows) return;
     float acc[PER];
@@ -31,18 +34,19 @@ __global__ void __launch_bounds__(256) lse_combine_kernel(const float *__restric
         m = warp_max(lsl);
         if (m != -INFINITY) {
             const float fl = lsl == -INFINITY ? 0.f : exp2f((lsl - m) * kLog2e);
-#pragma unroll 8
+            den = warp_sum(fl);
+            // every piece's partial row is read (the loads carry no branch and
+            // go out together); an empty piece's row counts with weight 0
+            // whatever it holds
+#pragma unroll 16
             for (int s = 0; s < n_split; ++s) {
                 const float f = __shfl_sync(0xffffffffu, fl, s);
                 const float *src = part_o + ((long long)s * rows + row) * D + lane * PER;
-                if (f != 0.f) {
-                    den += f;
 #pragma unroll
-                    for (int i = 0; i < PER; i += 2) {
-                        const float2 x = *reinterpret_cast<const float2 *>(src + i);
-                        acc[i] += f * x.x;
-                        acc[i + 1] += f * x.y;
-                    }
+                for (int i = 0; i < PER; i += 2) {
+                    const float2 x = __ldcg(reinterpret_cast<const float2 *>(src + i));
+                    acc[i] += f != 0.f ? f * x.x : 0.f;
+                    acc[i + 1] += f != 0.f ? f * x.y : 0.f;
                 }
             }
         }
@@ -84,6 +88,7 @@ __global__ void nsa_compress_kernel(const __nv_bfloat16 *__restrict__ k,
                                     int d, int nc, int len, int stride,
                                     __nv_bfloat16 *__restrict__ kc, __nv_bfloat16 *__restrict__ kc_lo,
                                     __nv_bfloat16 *__restrict__ vc) {
+    grid_dependency_sync();
     const long long total = (long long)B * nc * Hkv * (d / 2);
     const long long i2 = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (i2 >= total) return;
@@ -141,6 +146,7 @@ constexpr int nsa_select_smem(int n_blocks) {
 
 template <int D>
 __global__ void __launch_bounds__(NSA_TW * 32) nsa_select_kernel(const NsaSelectParams p) {
+    grid_dependency_sync();
     constexpr int NK = 32, ROWB = D * 2, UNITS = ROWB / 16, CH = NK * ROWB;
     constexpr int KS_D = D / 16, STAGES = 3;
     constexpr int SB = 2 * CH;                 // one stage: K hi | K lo
@@ -321,6 +327,7 @@ __global__ void __launch_bounds__(NSA_TW * 32) nsa_select_kernel(const NsaSelect
 __global__ void nsa_gate_kernel(const float *__restrict__ o3, long long branch_stride,
                                 const float *__restrict__ gates, long long rows, int d,
                                 __nv_bfloat16 *__restrict__ out) {
+    grid_dependency_sync();
     const long long i2 = (long long)blockIdx.x * blockDim.x + threadIdx.x;   // column pair
     if (i2 >= rows * (d / 2)) return;
     const long long row = i2 / (d / 2);
@@ -334,6 +341,7 @@ __global__ void nsa_gate_kernel(const float *__restrict__ o3, long long branch_s
 
 __global__ void nsa_lse_pack_kernel(const float *__restrict__ l3, long long rows,
                                     float *__restrict__ lse_branches) {
+    grid_dependency_sync();
     const long long r = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (r >= rows) return;
     lse_branches[r * 3 + 0] = l3[r];

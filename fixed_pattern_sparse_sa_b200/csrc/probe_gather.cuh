@@ -49,6 +49,7 @@ __device__ __forceinline__ unsigned probe_hash(unsigned x) {
 // STAGES: ring depth of the cp.async mode (the bulk mode takes p.stages).
 template <int MODE, int STAGES>
 __global__ void __launch_bounds__(512) probe_gather_kernel(const ProbeParams p) {
+    grid_dependency_sync();
     extern __shared__ __align__(1024) unsigned char smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (warp >= p.warps) return;

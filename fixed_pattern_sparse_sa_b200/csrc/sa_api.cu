@@ -61,6 +61,35 @@ static void log_launch(const char *name, dim3 g, dim3 b, size_t smem) {
                      b.z, smem);
 }
 
+// Every kernel is launched with programmatic stream serialization allowed
+// (the kernels begin with grid_dependency_sync), so a dependent kernel's
+// blocks are scheduled while the previous grid's last blocks finish; in a
+// CUDA graph this removes most of the gap between back-to-back launches.
+// SA_PDL=0 launches plainly (for comparison).
+static bool pdl_enabled() {
+    static const bool on = [] {
+        const char *e = std::getenv("SA_PDL");
+        return !(e && std::strcmp(e, "0") == 0);
+    }();
+    return on;
+}
+template <typename... P, typename... A>
+static void launch_k(const char *name, void (*kern)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                     A &&...args) {
+    log_launch(name, grid, block, smem);
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl_enabled() ? 1 : 0;
+    (void)cudaLaunchKernelEx(&cfg, kern, std::forward<A>(args)...);   // errors are read by SA_CHECK_LAUNCH
+}
+
 // NVTX range around each C-ABI call (visible to profilers and tracers;
 // a no-op when none is attached).
 struct TraceRange {
@@ -209,8 +238,7 @@ static int launch_gather_nw(const GatherParams &p, long long items, cudaStream_t
     if (rc) return rc;
     static const CUtensorMap unused{};                   // the row-gather modes take no tensor map
     const long long blocks = (items + NW - 1) / NW;
-    log_launch(__PRETTY_FUNCTION__, (unsigned)blocks, NW * 32, smem),
-        kern<<<(unsigned)blocks, NW * 32, smem, st>>>(p, km ? *km : unused, vm ? *vm : unused);
+    launch_k(__PRETTY_FUNCTION__, kern, (unsigned)blocks, NW * 32, smem, st, p, km ? *km : unused, vm ? *vm : unused);
     SA_CHECK_LAUNCH("gather_attn_kernel");
     return SA_OK;
 }
@@ -252,9 +280,27 @@ static int launch_gather_t(const GatherParams &p, cudaStream_t st) {
     if constexpr (KLO) {
         return launch_gather_nw<D, SRC, BIAS, KLO, 8>(p, items, st);
     } else {
-        // small launches (decode pieces): 4-warp CTAs, 2-stage ring (a 6-stage
-        // ring measured slower for the 128K decode)
-        if (items < (long long)sm_count() * SA_ATTN_NW) return launch_gather_nw<D, SRC, BIAS, KLO, 4>(p, items, st);
+        // small launches (decode pieces): 4-warp CTAs; SA_GATHER_SMALL_STAGES
+        // = 4 or 6 deepens their ring (for comparison), default 2
+        if (items < (long long)sm_count() * SA_ATTN_NW) {
+            static const int small_stages = [] {
+                const char *e = std::getenv("SA_GATHER_SMALL_STAGES");
+                return e ? std::atoi(e) : 2;
+            }();
+            if (small_stages == 6) return launch_gather_nw<D, SRC, BIAS, KLO, 4, 6>(p, items, st);
+            if (small_stages == 4) return launch_gather_nw<D, SRC, BIAS, KLO, 4, 4>(p, items, st);
+            return launch_gather_nw<D, SRC, BIAS, KLO, 4>(p, items, st);
+        }
+        // fixed-graph rows (KS_PROWS): SA_PROWS_NW = 16 or 20 warps per CTA
+        // (fewer registers each, more warps per SM; for comparison)
+        if constexpr (SRC == KS_PROWS && D == 64) {
+            static const int prows_nw = [] {
+                const char *e = std::getenv("SA_PROWS_NW");
+                return e ? std::atoi(e) : 12;
+            }();
+            if (prows_nw == 16) return launch_gather_nw<D, SRC, BIAS, KLO, 16>(p, items, st);
+            if (prows_nw == 20) return launch_gather_nw<D, SRC, BIAS, KLO, 20>(p, items, st);
+        }
         return launch_gather_nw<D, SRC, BIAS, KLO, SA_ATTN_NW>(p, items, st);
     }
 }
@@ -328,7 +374,7 @@ static int launch_attn_tc(const GatherParams &p, cudaStream_t st) {
     rc = set_smem(kern, smem);
     if (rc) return rc;
     const int grid = (int)std::min<long long>(items, sm_count());
-    log_launch(__PRETTY_FUNCTION__, grid, ATC_THREADS, smem), kern<<<grid, ATC_THREADS, smem, st>>>(qm, km, vm, ap);
+    launch_k(__PRETTY_FUNCTION__, kern, grid, ATC_THREADS, smem, st, qm, km, vm, ap);
     SA_CHECK_LAUNCH("attn_tc_kernel");
     return SA_OK;
 }
@@ -336,13 +382,14 @@ static int launch_attn_tc(const GatherParams &p, cudaStream_t st) {
 static int launch_combine(const float *po, const float *pl, int n_split, long long rows, int d,
                           void *out, float *lse, cudaStream_t st) {
     if (rows == 0) return SA_OK;
-    const unsigned blocks = (unsigned)((rows + 7) / 8);
+    const unsigned blocks = (unsigned)((rows + COMBINE_ROWS - 1) / COMBINE_ROWS);
+    constexpr int threads = COMBINE_ROWS * 32;
     if (d == 64)
-        log_launch("lse_combine_kernel<64>", blocks, 256, 0),
-            lse_combine_kernel<64><<<blocks, 256, 0, st>>>(po, pl, n_split, rows, (__nv_bfloat16 *)out, lse);
+        launch_k("lse_combine_kernel<64>", lse_combine_kernel<64>, blocks, threads, 0, st, po, pl, n_split, rows,
+            (__nv_bfloat16 *)out, lse);
     else if (d == 128)
-        log_launch("lse_combine_kernel<128>", blocks, 256, 0),
-            lse_combine_kernel<128><<<blocks, 256, 0, st>>>(po, pl, n_split, rows, (__nv_bfloat16 *)out, lse);
+        launch_k("lse_combine_kernel<128>", lse_combine_kernel<128>, blocks, threads, 0, st, po, pl, n_split, rows,
+            (__nv_bfloat16 *)out, lse);
     else
         return fail(SA_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
     SA_CHECK_LAUNCH("lse_combine_kernel");
@@ -718,7 +765,7 @@ static int launch_score_t(const IdxParams &p, long long n_keys_max, cudaStream_t
     if (rc) return rc;
     dim3 grid((unsigned)((n_keys_max + TC_KT * 128 - 1) / (TC_KT * 128)), (unsigned)((p.Rt + NQ - 1) / NQ),
               (unsigned)p.B);
-    log_launch(__PRETTY_FUNCTION__, grid, tc_threads(NCOL), smem), kern<<<grid, tc_threads(NCOL), smem, st>>>(p);
+    launch_k(__PRETTY_FUNCTION__, kern, grid, tc_threads(NCOL), smem, st, p);
     SA_CHECK_LAUNCH("idx_score_tc_kernel");
     return SA_OK;
 }
@@ -726,8 +773,7 @@ static int launch_score_t(const IdxParams &p, long long n_keys_max, cudaStream_t
 template <int DI, int MODE>
 static int launch_dp4a_t(const IdxParams &p, long long n_keys_max, cudaStream_t st) {
     dim3 grid((unsigned)((n_keys_max + DEC_KEYS - 1) / DEC_KEYS), (unsigned)p.Rt, (unsigned)p.B);
-    log_launch("idx_score_dp4a_kernel<DI, MODE>", grid, DEC_THREADS, 0),
-        idx_score_dp4a_kernel<DI, MODE><<<grid, DEC_THREADS, 0, st>>>(p);
+    launch_k("idx_score_dp4a_kernel<DI, MODE>", idx_score_dp4a_kernel<DI, MODE>, grid, DEC_THREADS, 0, st, p);
     SA_CHECK_LAUNCH("idx_score_dp4a_kernel");
     return SA_OK;
 }
@@ -736,8 +782,7 @@ template <int MODE>
 static int launch_dec_mma_t(const IdxParams &p, long long n_keys_max, cudaStream_t st) {
     constexpr int kpc = dmma_keys(MODE);
     dim3 grid((unsigned)((n_keys_max + kpc - 1) / kpc), (unsigned)p.Rt, (unsigned)p.B);
-    log_launch("idx_score_dec_mma_kernel<MODE>", grid, DMMA_THREADS, 0),
-        idx_score_dec_mma_kernel<MODE><<<grid, DMMA_THREADS, 0, st>>>(p);
+    launch_k("idx_score_dec_mma_kernel<MODE>", idx_score_dec_mma_kernel<MODE>, grid, DMMA_THREADS, 0, st, p);
     SA_CHECK_LAUNCH("idx_score_dec_mma_kernel");
     return SA_OK;
 }
@@ -803,7 +848,7 @@ static int launch_filter_tc_t(const IdxParams &p, const int8_t *qf, const int32_
     rc = set_smem(kern, smem);
     if (rc) return rc;
     const int grid = (int)std::min<long long>(n_units, sm_count());
-    log_launch(__PRETTY_FUNCTION__, grid, FT_THREADS, smem), kern<<<grid, FT_THREADS, smem, st>>>(am, bm, fp);
+    launch_k(__PRETTY_FUNCTION__, kern, grid, FT_THREADS, smem, st, am, bm, fp);
     SA_CHECK_LAUNCH("idx_filter_tc_kernel");
     return SA_OK;
 }
@@ -822,12 +867,9 @@ static int launch_filter_tc_d(const IdxParams &p, const int8_t *qf, const int32_
 static int launch_fold(const IdxParams &p, int8_t *qf, int32_t *wf, cudaStream_t st) {
     const long long n = (long long)p.B * p.Tq * p.Hi;
     const unsigned blocks = (unsigned)((n + 255) / 256);
-    if (p.di == 32) log_launch("idx_fold_kernel<32>", blocks, 256, 0),
-        idx_fold_kernel<32><<<blocks, 256, 0, st>>>(p.q, p.w, qf, wf, n);
-    else if (p.di == 64) log_launch("idx_fold_kernel<64>", blocks, 256, 0),
-        idx_fold_kernel<64><<<blocks, 256, 0, st>>>(p.q, p.w, qf, wf, n);
-    else log_launch("idx_fold_kernel<128>", blocks, 256, 0),
-        idx_fold_kernel<128><<<blocks, 256, 0, st>>>(p.q, p.w, qf, wf, n);
+    if (p.di == 32) launch_k("idx_fold_kernel<32>", idx_fold_kernel<32>, blocks, 256, 0, st, p.q, p.w, qf, wf, n);
+    else if (p.di == 64) launch_k("idx_fold_kernel<64>", idx_fold_kernel<64>, blocks, 256, 0, st, p.q, p.w, qf, wf, n);
+    else launch_k("idx_fold_kernel<128>", idx_fold_kernel<128>, blocks, 256, 0, st, p.q, p.w, qf, wf, n);
     SA_CHECK_LAUNCH("idx_fold_kernel");
     return SA_OK;
 }
@@ -839,8 +881,7 @@ static int launch_select_nt(const IdxParams &p, int words, cudaStream_t st) {
     auto kern = topk_select_kernel<DI, NT>;
     int rc = set_smem(kern, smem);
     if (rc) return rc;
-    log_launch(__PRETTY_FUNCTION__, dim3(1u, (unsigned)p.Rt, (unsigned)p.B),
-        NT, smem), kern<<<dim3(1u, (unsigned)p.Rt, (unsigned)p.B), NT, smem, st>>>(p);
+    launch_k(__PRETTY_FUNCTION__, kern, dim3(1u, (unsigned)p.Rt, (unsigned)p.B), NT, smem, st, p);
     SA_CHECK_LAUNCH("topk_select_kernel");
     return SA_OK;
 }
@@ -902,13 +943,13 @@ int sa_indexer_topk(const int8_t *q_idx, const int8_t *k_idx, const int32_t *w, 
         p.t0 = t0; p.Rt = rows;
         const long long pmax = q_pos0 + t0 + rows - 1;
         const long long ncand = std::max(0LL, window > 0 ? pmax - window + 1 : pmax + 1);
-        cudaError_t e = cudaMemsetAsync(p.cand_cnt, 0, (size_t)B * rows * 4, st);
-        if (e != cudaSuccess) return fail(SA_ERR_CUDA, "memset: %s", cudaGetErrorString(e));
+        // the threshold kernel zeroes each row's list length (no rows have
+        // candidates when ncand == 0, and the select then reads none)
         if (ncand > 0) {
             rc = launch_score<MODE_SAMPLE>(p, lay.decode, (long long)lay.m_cap, st);
             if (rc) return rc;
-            log_launch("idx_threshold_kernel", dim3(1u, (unsigned)rows, (unsigned)B),
-                SEL_THREADS, 0), idx_threshold_kernel<<<dim3(1u, (unsigned)rows, (unsigned)B), SEL_THREADS, 0, st>>>(p);
+            launch_k("idx_threshold_kernel", idx_threshold_kernel, dim3(1u, (unsigned)rows, (unsigned)B), SEL_THREADS,
+                0, st, p);
             SA_CHECK_LAUNCH("idx_threshold_kernel");
             if (filter_tc)
                 rc = di == 32 ? launch_filter_tc_d<32>(p, qf, wf, st)
@@ -964,8 +1005,7 @@ static int launch_nsa_select(const NsaSelectParams &p, cudaStream_t st) {
     int rc = set_smem(kern, smem);
     if (rc) return rc;
     const long long ctas = (long long)p.B * p.Hkv * ((p.T + NSA_TW - 1) / NSA_TW);
-    log_launch(__PRETTY_FUNCTION__, (unsigned)ctas, NSA_TW * 32, smem),
-        kern<<<(unsigned)ctas, NSA_TW * 32, smem, st>>>(p);
+    launch_k(__PRETTY_FUNCTION__, kern, (unsigned)ctas, NSA_TW * 32, smem, st, p);
     SA_CHECK_LAUNCH("nsa_select_kernel");
     return SA_OK;
 }
@@ -982,8 +1022,7 @@ static int launch_tile_t(const TileParams &p, cudaStream_t st) {
     if (rc) return rc;
     const long long ctas = (long long)p.B * p.Hkv * ((p.T + kTileWarps - 1) / kTileWarps);
     if (ctas == 0) return SA_OK;
-    log_launch(__PRETTY_FUNCTION__, (unsigned)ctas, kTileWarps * 32, smem),
-        kern<<<(unsigned)ctas, kTileWarps * 32, smem, st>>>(p);
+    launch_k(__PRETTY_FUNCTION__, kern, (unsigned)ctas, kTileWarps * 32, smem, st, p);
     SA_CHECK_LAUNCH("tile_attn_kernel");
     return SA_OK;
 }
@@ -1010,8 +1049,7 @@ static int launch_nsa_tc(const TileParams &p, unsigned *err, cudaStream_t st) {
     rc = set_smem(kern, smem);
     if (rc) return rc;
     const int grid = (int)std::min<long long>(items, sm_count());   // persistent: one CTA per SM
-    log_launch(__PRETTY_FUNCTION__, grid, NT_THREADS, smem),
-        kern<<<grid, NT_THREADS, smem, st>>>(qm, khm, klm, vm, cp);
+    launch_k(__PRETTY_FUNCTION__, kern, grid, NT_THREADS, smem, st, qm, khm, klm, vm, cp);
     SA_CHECK_LAUNCH("nsa_tc_kernel");
     return SA_OK;
 }
@@ -1037,8 +1075,7 @@ static int launch_imp_tc(const NsaSelectParams &sp, unsigned *err, cudaStream_t 
     rc = set_smem(nsa_imp_tc_kernel, smem);
     if (rc) return rc;
     const int grid = (int)std::min<long long>(items, sm_count());
-    log_launch("nsa_imp_tc_kernel", grid, IT_THREADS, smem),
-        nsa_imp_tc_kernel<<<grid, IT_THREADS, smem, st>>>(qm, khm, klm, ip);
+    launch_k("nsa_imp_tc_kernel", nsa_imp_tc_kernel, grid, IT_THREADS, smem, st, qm, khm, klm, ip);
     SA_CHECK_LAUNCH("nsa_imp_tc_kernel");
     return SA_OK;
 }
@@ -1104,10 +1141,9 @@ int sa_nsa_fwd(const void *q, const void *k, const void *v, const float *gates, 
     // 1. compression
     if (lay.nc > 0) {
         const long long n2 = (long long)B * lay.nc * Hkv * (d / 2);
-        log_launch("nsa_compress_kernel", (unsigned)((n2 + 255) / 256),
-            256, 0), nsa_compress_kernel<<<(unsigned)((n2 + 255) / 256), 256, 0, st>>>(
-            (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, B, T, Hkv, d, lay.nc, cmp_len, cmp_stride,
-            kc, klo, vc);
+        launch_k("nsa_compress_kernel", nsa_compress_kernel, (unsigned)((n2 + 255) / 256), 256, 0, st,
+            (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, B, T, Hkv, d, lay.nc, cmp_len, cmp_stride, kc, klo,
+            vc);
         SA_CHECK_LAUNCH("nsa_compress_kernel");
     }
     GatherParams base{};
@@ -1167,13 +1203,12 @@ int sa_nsa_fwd(const void *q, const void *k, const void *v, const float *gates, 
     // 6. gated sum
     {
         const long long n2 = rows * (d / 2);
-        log_launch("nsa_gate_kernel", (unsigned)((n2 + 255) / 256),
-            256, 0), nsa_gate_kernel<<<(unsigned)((n2 + 255) / 256), 256, 0, st>>>(o3, rows * d, gates, rows, d,
-                                                                       (__nv_bfloat16 *)out);
+        launch_k("nsa_gate_kernel", nsa_gate_kernel, (unsigned)((n2 + 255) / 256), 256, 0, st, o3, rows * d, gates,
+            rows, d, (__nv_bfloat16 *)out);
         SA_CHECK_LAUNCH("nsa_gate_kernel");
         if (lse_branches) {
-            log_launch("nsa_lse_pack_kernel", (unsigned)((rows + 255) / 256),
-                256, 0), nsa_lse_pack_kernel<<<(unsigned)((rows + 255) / 256), 256, 0, st>>>(l3, rows, lse_branches);
+            launch_k("nsa_lse_pack_kernel", nsa_lse_pack_kernel, (unsigned)((rows + 255) / 256), 256, 0, st, l3, rows,
+                lse_branches);
             SA_CHECK_LAUNCH("nsa_lse_pack_kernel");
         }
     }
@@ -1231,7 +1266,7 @@ static int launch_probe(const ProbeParams &p, int ctas, int smem, cudaStream_t s
     auto kern = probe_gather_kernel<MODE, STAGES>;
     int rc = set_smem(kern, smem);
     if (rc) return rc;
-    log_launch(__PRETTY_FUNCTION__, ctas, p.warps * 32, smem), kern<<<ctas, p.warps * 32, smem, st>>>(p);
+    launch_k(__PRETTY_FUNCTION__, kern, ctas, p.warps * 32, smem, st, p);
     SA_CHECK_LAUNCH("probe_gather_kernel");
     return SA_OK;
 }
@@ -1272,8 +1307,7 @@ size_t sa_sparse_attn_bwd_workspace_size(int B, int Tq, int Hq) {
 template <int D>
 static int launch_bwd(const BwdParams &p, long long rows, cudaStream_t st) {
     constexpr int NW = 8;
-    log_launch("attn_bwd_prep_kernel<D>", (unsigned)((rows + 7) / 8),
-        256, 0), attn_bwd_prep_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(p, rows);
+    launch_k("attn_bwd_prep_kernel<D>", attn_bwd_prep_kernel<D>, (unsigned)((rows + 7) / 8), 256, 0, st, p, rows);
     SA_CHECK_LAUNCH("attn_bwd_prep_kernel");
     constexpr int smem = attn_bwd_smem_bytes<D, NW>();
     static_assert(smem <= 227 * 1024, "shared memory");
@@ -1282,8 +1316,7 @@ static int launch_bwd(const BwdParams &p, long long rows, cudaStream_t st) {
     if (rc) return rc;
     const long long items = (long long)p.B * p.Tq * p.Hkv * ((p.G + 15) / 16);
     if (items == 0) return SA_OK;
-    log_launch(__PRETTY_FUNCTION__, (unsigned)((items + NW - 1) / NW),
-        NW * 32, smem), kern<<<(unsigned)((items + NW - 1) / NW), NW * 32, smem, st>>>(p);
+    launch_k(__PRETTY_FUNCTION__, kern, (unsigned)((items + NW - 1) / NW), NW * 32, smem, st, p);
     SA_CHECK_LAUNCH("attn_bwd_kernel");
     return SA_OK;
 }
@@ -1343,12 +1376,12 @@ int sa_indexer_scores_at(const int8_t *q_idx, const int8_t *k_idx, const int32_t
     if (rc) return rc;
     const unsigned blocks = (unsigned)((long long)B * Tq);
     cudaStream_t st = as_stream(stream);
-    if (di == 32) log_launch("idx_scores_at_kernel<32>", blocks, 128, 0),
-        idx_scores_at_kernel<32><<<blocks, 128, 0, st>>>(q_idx, k_idx, w, B, Tq, L, Hi, idx, K, out_score, ew);
-    else if (di == 64) log_launch("idx_scores_at_kernel<64>", blocks, 128, 0),
-        idx_scores_at_kernel<64><<<blocks, 128, 0, st>>>(q_idx, k_idx, w, B, Tq, L, Hi, idx, K, out_score, ew);
-    else log_launch("idx_scores_at_kernel<128>", blocks, 128, 0),
-        idx_scores_at_kernel<128><<<blocks, 128, 0, st>>>(q_idx, k_idx, w, B, Tq, L, Hi, idx, K, out_score, ew);
+    if (di == 32) launch_k("idx_scores_at_kernel<32>", idx_scores_at_kernel<32>, blocks, 128, 0, st, q_idx, k_idx, w,
+        B, Tq, L, Hi, idx, K, out_score, ew);
+    else if (di == 64) launch_k("idx_scores_at_kernel<64>", idx_scores_at_kernel<64>, blocks, 128, 0, st, q_idx,
+        k_idx, w, B, Tq, L, Hi, idx, K, out_score, ew);
+    else launch_k("idx_scores_at_kernel<128>", idx_scores_at_kernel<128>, blocks, 128, 0, st, q_idx, k_idx, w, B, Tq,
+        L, Hi, idx, K, out_score, ew);
     SA_CHECK_LAUNCH("idx_scores_at_kernel");
     return SA_OK;
 }
@@ -1374,10 +1407,8 @@ int sa_topk_merge(const int32_t *cand_score, const int32_t *cand_idx, const int6
     const int smem = topk_merge_smem_bytes(n_parts * kc);
     int rc = set_smem(topk_merge_kernel, smem);
     if (rc) return rc;
-    log_launch("topk_merge_kernel", (unsigned)rows, TM_THREADS, smem),
-        topk_merge_kernel<<<(unsigned)rows, TM_THREADS, smem, as_stream(stream)>>>(
-        cand_score, cand_idx, mo, n_parts, rows, kc, topk, window, q_pos,
-        out_idx, out_count);
+    launch_k("topk_merge_kernel", topk_merge_kernel, (unsigned)rows, TM_THREADS, smem, as_stream(stream), cand_score,
+        cand_idx, mo, n_parts, rows, kc, topk, window, q_pos, out_idx, out_count);
     SA_CHECK_LAUNCH("topk_merge_kernel");
     return SA_OK;
 }
@@ -1388,8 +1419,7 @@ int sa_index_shard(const int32_t *idx, int64_t n, int64_t key_lo, int64_t key_hi
         return fail(SA_ERR_INVALID_ARG, "index_shard: bad arguments");
     if (n == 0) return SA_OK;
     const unsigned blocks = (unsigned)((n + 255) / 256);
-    log_launch("index_shard_kernel", blocks, 256, 0),
-        index_shard_kernel<<<blocks, 256, 0, as_stream(stream)>>>(idx, n, key_lo, key_hi, out);
+    launch_k("index_shard_kernel", index_shard_kernel, blocks, 256, 0, as_stream(stream), idx, n, key_lo, key_hi, out);
     SA_CHECK_LAUNCH("index_shard_kernel");
     return SA_OK;
 }

@@ -47,6 +47,17 @@ __device__ __forceinline__ float ex2_fast(float x) {
     return y;
 }
 
+// Programmatic dependent launch: every kernel starts by waiting for the
+// grid launched before it on the stream to complete (its results visible),
+// then lets the next grid begin launching.  With the launch attribute set,
+// the next kernel's blocks are scheduled while this grid's last blocks run
+// and wait here, instead of launching after the stream drains; without it
+// both instructions do nothing.  Nothing is read or written before the wait.
+__device__ __forceinline__ void grid_dependency_sync() {
+    asm volatile("griddepcontrol.wait;\n" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+}
+
 __device__ __forceinline__ void raise_error(unsigned *err, unsigned bit) {
     if (err) atomicOr(err, bit);
 }
@@ -137,6 +148,11 @@ __device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     return v;
 }
 __device__ __forceinline__ int warp_sum_int(int v) {
