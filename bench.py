@@ -177,8 +177,9 @@ def main():
     ap.add_argument("--decode-seq-len", type=int, default=0,
                     help="cache length of the decode workload for profiling captures of a smaller "
                          "case (default 131072); the JSON line names it")
-    ap.add_argument("--decode-split", type=int, default=16,
-                    help="split-KV pieces per decode row (the 2048 selected keys are cut into this many)")
+    ap.add_argument("--decode-split", type=int, default=4,
+                    help="split-KV pieces per decode row (the 2048 selected keys are cut into this many; "
+                         "each piece is one CTA of 8 warps that merge in shared memory)")
     ap.add_argument("--cpu-sample-rows", type=int, default=0,
                     help="oracle rows for the CPU baseline (0 = auto, ~10-30 s)")
     args = ap.parse_args()

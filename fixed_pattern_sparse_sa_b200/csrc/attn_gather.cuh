@@ -120,6 +120,28 @@ __device__ __forceinline__ int key_prows(const GatherParams &p, long long pa, lo
     return (int)j;
 }
 
+// KS_PROWS: the rows (bit r = row r; row r is query r / G of the item, G
+// heads per query, nq_valid queries in the item) that see key j of segment
+// seg, for queries at positions pa + qi: the window band reaches
+// pa + qi - window < j <= pa + qi, a dilated distance o reaches only the
+// query at j + o, and only when o < its position.
+__device__ __forceinline__ unsigned prows_rowmask(int j, int seg, long long pa, int nq_valid, int window, int G) {
+    if (j < 0) return 0u;
+    const long long rel = (long long)j - pa;                 // key position relative to the first query
+    long long qlo, qhi;
+    if (seg == 0) {
+        qlo = rel > 0 ? rel : 0;
+        qhi = rel + window - 1;
+    } else {
+        qlo = qhi = rel + seg;
+        if ((long long)seg >= pa + qlo) return 0u;
+    }
+    if (qhi > nq_valid - 1) qhi = nq_valid - 1;
+    if (qhi < qlo) return 0u;
+    const int rlo = (int)qlo * G, rhi = ((int)qhi + 1) * G;   // rows [rlo, rhi), rhi <= 16
+    return ((rhi >= 32 ? 0xffffffffu : (1u << rhi)) - 1u) & ~((1u << rlo) - 1u);
+}
+
 template <int SRC>
 __device__ __forceinline__ int key_finish(const GatherParams &p, long long pos, int raw, int e) {
     if (raw == KEY_NONE) return -1;
@@ -197,7 +219,8 @@ __device__ __forceinline__ void merge_pieces_half(const float *part_o, const flo
 // columns x 1 head x 16 rows, 128-byte swizzle) issued by lane 0, completion
 // on a per-warp mbarrier; a K (or V) chunk is then two 64-column halves of
 // 16 rows x 128 B instead of 16 rows x 256 B.
-template <int D, int STAGES, int SRC, bool BIAS, bool KLO = false, int NK = 32, int NW = 4, bool TMAB = false>
+template <int D, int STAGES, int SRC, bool BIAS, bool KLO = false, int NK = 32, int NW = 4, bool TMAB = false,
+          bool CTAM = false>
 __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams p, const __grid_constant__ CUtensorMap kmap,
                                                               const __grid_constant__ CUtensorMap vmap) {
     grid_dependency_sync();
@@ -210,6 +233,7 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
     constexpr int CP_ITERS = NK * UNITS / 32;
     constexpr int SB = (KLO ? 3 : 2) * CH;   // one stage: K | V | (K lo)
     static_assert(!TMAB || (SRC == KS_BLOCKS && D == 128 && NK == 16 && !KLO && !BIAS), "TMA block chunks");
+    static_assert(!CTAM || (SRC == KS_IDX && !TMAB && !KLO && !BIAS), "CTA-merged pieces: explicit lists only");
 
     extern __shared__ __align__(1024) unsigned char smem_dyn[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -243,8 +267,11 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
     }
 
     const long long n_items = (long long)p.B * p.q_units * p.Hkv * p.n_hchunk * p.n_split;
-    const long long item = (long long)blockIdx.x * NW + warp;
-    if (item >= n_items) return;   // warps are independent: no block barrier below
+    // CTAM: one item per CTA, its warps take consecutive parts of the item's
+    // entries and merge in shared memory at the end (the only block barrier);
+    // otherwise one item per warp and the warps never wait for each other
+    const long long item = CTAM ? (long long)blockIdx.x : (long long)blockIdx.x * NW + warp;
+    if (item >= n_items) return;   // CTA-uniform under CTAM
 
     long long rem = item;
     const int s = (int)(rem % p.n_split); rem /= p.n_split;
@@ -267,7 +294,6 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
     const int tr0 = PR ? t + gr / p.G : t, tr1 = PR ? t + (gr + 8) / p.G : t;   // query of each row
     const int hr0 = PR ? gr % p.G : hc * 16 + gr, hr1 = PR ? (gr + 8) % p.G : hc * 16 + gr + 8;
     const bool v0 = hr0 < p.G && tr0 <= t_end, v1 = hr1 < p.G && tr1 <= t_end;
-    const long long pos_r0 = p.q_pos0 + tr0, pos_r1 = p.q_pos0 + tr1;
     const int h0 = g * p.G + hr0, h1 = g * p.G + hr1;
     const long long qrow0 = ((long long)(b * p.Tq + (v0 ? tr0 : t)) * p.Hq + h0) * D;
     const long long qrow1 = ((long long)(b * p.Tq + (v1 ? tr1 : t)) * p.Hq + h1) * D;
@@ -308,8 +334,15 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
         }
     }
 
-    const int e_beg = s * p.per_split;
+    int e_beg = s * p.per_split;
     int e_end = min(p.entries, e_beg + p.per_split);
+    if constexpr (CTAM) {
+        // the warp's part of the piece: whole chunks, consecutive
+        const int len = max(e_end - e_beg, 0);
+        const int part = (len + NW * NK - 1) / (NW * NK) * NK;
+        e_beg = min(e_beg + warp * part, e_end);
+        e_end = min(e_end, e_beg + part);
+    }
     const int n_chunks = e_end > e_beg ? (e_end - e_beg + NK - 1) / NK : 0;
 
     const __nv_bfloat16 *kb = p.k + ((long long)b * p.Lk * p.Hkv + g) * D;
@@ -340,7 +373,7 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
         }
         if (lane < NK) {
             keys_s[st * NK + lane] = j;
-            if constexpr (PR) segs_s[st * NK + lane] = seg;
+            if constexpr (PR) segs_s[st * NK + lane] = (int)prows_rowmask(j, seg, pos, t_end - t + 1, p.window, p.G);
             if constexpr (BIAS) {
                 // the key's coordinates ride with its K/V rows (same commit group)
                 if (j >= 0) {
@@ -510,31 +543,33 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
                     mx1 = fmaxf(mx1, fmaxf(sc[nt][2], sc[nt][3]));
                 }
             } else {
+                // per key of this thread (two per n-tile): its row mask (fixed
+                // graph) and coordinates once, then its two rows
 #pragma unroll
                 for (int nt = 0; nt < NK / 8; ++nt) {
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int kk = nt * 8 + 2 * qc + (e & 1);
-                        float x = sc[nt][e] * sl2;
-                        if constexpr (BIAS) {
-                            const int jk = __shfl_sync(0xffffffffu, jl, kk);
-                            if (jk >= 0) {
-                                const float *c = ck_s + (st * NK + kk) * 3;
-                                const float *a = (e >> 1) ? cq1 : cq0;
-                                const float dx = a[0] - c[0], dy = a[1] - c[1], dz = a[2] - c[2];
-                                x -= ((e >> 1) ? be1 : be0) * (dx * dx + dy * dy + dz * dz);
-                            }
-                        }
-                        bool ok = (vmask >> kk) & 1u;
+                    for (int par = 0; par < 2; ++par) {
+                        const int kk = nt * 8 + 2 * qc + par;
+                        const bool kv = (vmask >> kk) & 1u;
+                        bool ok0 = kv, ok1 = kv;
                         if constexpr (PR) {
-                            // the entry's segment decides which rows it belongs to
-                            const int jk = __shfl_sync(0xffffffffu, jl, kk);
-                            const int sk = __shfl_sync(0xffffffffu, sl, kk);
-                            const long long d = ((e >> 1) ? pos_r1 : pos_r0) - jk;
-                            ok = ok && (sk == 0 ? (d >= 0 && d < p.window) : (d == sk && sk < d + jk));
+                            const unsigned km = (unsigned)__shfl_sync(0xffffffffu, sl, kk);   // rows seeing key kk
+                            ok0 = ok0 && ((km >> gr) & 1u);
+                            ok1 = ok1 && ((km >> (gr + 8)) & 1u);
                         }
-                        x = ok ? x : -INFINITY;
-                        sc[nt][e] = x;
+                        float x0 = sc[nt][par] * sl2, x1 = sc[nt][2 + par] * sl2;
+                        if constexpr (BIAS) {
+                            // an empty entry's coordinates are stale: its
+                            // score is replaced by -inf below
+                            const float *c = ck_s + (st * NK + kk) * 3;
+                            const float c0 = c[0], c1 = c[1], c2 = c[2];
+                            float dx = cq0[0] - c0, dy = cq0[1] - c1, dz = cq0[2] - c2;
+                            x0 -= be0 * (dx * dx + dy * dy + dz * dz);
+                            dx = cq1[0] - c0; dy = cq1[1] - c1; dz = cq1[2] - c2;
+                            x1 -= be1 * (dx * dx + dy * dy + dz * dz);
+                        }
+                        sc[nt][par] = ok0 ? x0 : -INFINITY;
+                        sc[nt][2 + par] = ok1 ? x1 : -INFINITY;
                     }
                     mx0 = fmaxf(mx0, fmaxf(sc[nt][0], sc[nt][1]));
                     mx1 = fmaxf(mx1, fmaxf(sc[nt][2], sc[nt][3]));
@@ -622,6 +657,107 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
     l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
     l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
     l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+    if constexpr (CTAM) {
+        // this warp's rows (reference maximum, sum, unnormalised O) go to its
+        // own stage buffers (its copies are complete), then the CTA merges
+        // the NW parts of each of the 16 rows: M = max m_w, L = sum l_w 2^(m_w - M),
+        // O = sum o_w 2^(m_w - M) / L
+        float *ml_s = reinterpret_cast<float *>(wsm);          // [2][16]: m, l
+        float *o_s = ml_s + 32;                                 // [16][D]
+        if (qc == 0) {
+            ml_s[gr] = m0; ml_s[gr + 8] = m1;
+            ml_s[16 + gr] = l0; ml_s[16 + gr + 8] = l1;
+        }
+#pragma unroll
+        for (int nt = 0; nt < NT_D; ++nt) {
+            const int c = nt * 8 + 2 * qc;
+            *reinterpret_cast<float2 *>(o_s + gr * D + c) = make_float2(o[nt][0], o[nt][1]);
+            *reinterpret_cast<float2 *>(o_s + (gr + 8) * D + c) = make_float2(o[nt][2], o[nt][3]);
+        }
+        __syncthreads();
+        for (int job = threadIdx.x; job < 16 * (D / 4); job += NW * 32) {
+            const int r = job / (D / 4), c = (job % (D / 4)) * 4;
+            const int hr = hc * 16 + r;
+            if (hr >= p.G) continue;
+            float M = -INFINITY;
+#pragma unroll
+            for (int w = 0; w < NW; ++w) M = fmaxf(M, reinterpret_cast<const float *>(smem + w * WSTRIDE)[r]);
+            float L = 0.f;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (M != -INFINITY) {
+#pragma unroll
+                for (int w = 0; w < NW; ++w) {
+                    const float *wb = reinterpret_cast<const float *>(smem + w * WSTRIDE);
+                    const float mw = wb[r];
+                    const float f = mw == -INFINITY ? 0.f : ex2_fast(mw - M);
+                    const float4 x = *reinterpret_cast<const float4 *>(wb + 32 + r * D + c);
+                    L += f * wb[16 + r];
+                    acc.x += f * x.x; acc.y += f * x.y; acc.z += f * x.z; acc.w += f * x.w;
+                }
+            }
+            const float inv = L > 0.f ? 1.f / L : 0.f;
+            const float lsev = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
+            const long long orow = (long long)(b * p.Tq + t) * p.Hq + g * p.G + hr;
+            if (p.n_split == 1) {
+                if (p.out_f32) {
+                    *reinterpret_cast<float4 *>(p.out_f32 + orow * D + c) =
+                        make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+                } else {
+                    *reinterpret_cast<uint2 *>(p.out + orow * D + c) =
+                        make_uint2(pack_bf16(acc.x * inv, acc.y * inv), pack_bf16(acc.z * inv, acc.w * inv));
+                }
+                if (p.lse && c == 0) p.lse[orow] = lsev;
+            } else {
+                const long long rows = (long long)p.B * p.Tq * p.Hq;
+                *reinterpret_cast<float4 *>(p.part_o + ((long long)s * rows + orow) * D + c) =
+                    make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+                if (c == 0) p.part_lse[s * rows + orow] = lsev;
+            }
+        }
+        if (p.n_split > 1 && p.merge_cnt) {
+            // the last CTA of the group to arrive merges every piece's rows
+            // (the others only publish theirs): ticket after a fence, fence
+            // before reading the other pieces' rows from L2
+            __shared__ int last_s;
+            __threadfence();
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                int *ticket = p.merge_cnt + ((long long)(b * p.Tq + t) * p.Hkv + g) * p.n_hchunk + hc;
+                const bool last = atomicAdd(ticket, 1) == p.n_split - 1;
+                if (last) *ticket = 0;                      // ready for the next call
+                last_s = last;
+            }
+            __syncthreads();
+            if (last_s) {
+                __threadfence();
+                const long long rows = (long long)p.B * p.Tq * p.Hq;
+                for (int job = threadIdx.x; job < 16 * (D / 4); job += NW * 32) {
+                    const int r = job / (D / 4), c = (job % (D / 4)) * 4;
+                    const int hr = hc * 16 + r;
+                    if (hr >= p.G) continue;
+                    const long long orow = (long long)(b * p.Tq + t) * p.Hq + g * p.G + hr;
+                    float M = -INFINITY;
+                    for (int q = 0; q < p.n_split; ++q) M = fmaxf(M, __ldcg(p.part_lse + q * rows + orow));
+                    float den = 0.f;
+                    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (M != -INFINITY) {
+                        for (int q = 0; q < p.n_split; ++q) {
+                            const float lq = __ldcg(p.part_lse + q * rows + orow);
+                            const float f = lq == -INFINITY ? 0.f : ex2_fast((lq - M) * kLog2e);
+                            const float4 x = __ldcg(reinterpret_cast<const float4 *>(p.part_o + (q * rows + orow) * D + c));
+                            den += f;
+                            acc.x += f * x.x; acc.y += f * x.y; acc.z += f * x.z; acc.w += f * x.w;
+                        }
+                    }
+                    const float inv = den > 0.f ? 1.f / den : 0.f;
+                    *reinterpret_cast<uint2 *>(p.out + orow * D + c) =
+                        make_uint2(pack_bf16(acc.x * inv, acc.y * inv), pack_bf16(acc.z * inv, acc.w * inv));
+                    if (p.lse && c == 0) p.lse[orow] = den > 0.f ? M + log2f(den) * kLn2 : -INFINITY;
+                }
+            }
+        }
+        return;
+    }
     const float inv0 = l0 > 0.f ? 1.f / l0 : 0.f, inv1 = l1 > 0.f ? 1.f / l1 : 0.f;
     const float lse0 = l0 > 0.f ? (m0 + log2f(l0)) * kLn2 : -INFINITY;
     const float lse1 = l1 > 0.f ? (m1 + log2f(l1)) * kLn2 : -INFINITY;

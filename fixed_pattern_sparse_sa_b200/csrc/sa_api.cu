@@ -220,24 +220,37 @@ static bool gather_tma_allowed() {
     return v != 0;
 }
 
+// SA_GATHER_SMALL=warp: small explicit-list launches keep one warp per item
+// instead of the CTA-merged pieces (for comparison).
+static bool gather_small_per_warp() {
+    static const bool v = [] {
+        const char *e = std::getenv("SA_GATHER_SMALL");
+        return e && std::strcmp(e, "warp") == 0;
+    }();
+    return v;
+}
+#ifndef SA_ATTN_NW
+#define SA_ATTN_NW 12
+#endif
 // -------------------------------------------------------- gather launches --
 // Launch shape: 12 warps per CTA streaming 16-key chunks through a 2-stage
 // ring (8 warps when the lo-key tile is also staged); ~200 KB of shared
 // memory, one CTA and 12 gathering warps per SM.  Small launches (fewer
 // items than 12 per SM, e.g. decode with a few hundred split pieces) use
 // 4-warp CTAs so that every SM gets work.
-template <int D, int SRC, bool BIAS, bool KLO, int NW, int STAGES_ = 2, int NK_ = 16, bool TMAB = false>
+template <int D, int SRC, bool BIAS, bool KLO, int NW, int STAGES_ = 2, int NK_ = 16, bool TMAB = false,
+          bool CTAM = false>
 static int launch_gather_nw(const GatherParams &p, long long items, cudaStream_t st,
                             const CUtensorMap *km = nullptr, const CUtensorMap *vm = nullptr) {
     constexpr int NK = NK_;
     constexpr int STAGES = KLO ? 2 : STAGES_;
     constexpr int smem = gather_smem_bytes<D, STAGES, KLO, NK, NW, SRC == KS_PROWS, BIAS, TMAB>();
     static_assert(smem <= 227 * 1024, "shared memory");
-    auto kern = gather_attn_kernel<D, STAGES, SRC, BIAS, KLO, NK, NW, TMAB>;
+    auto kern = gather_attn_kernel<D, STAGES, SRC, BIAS, KLO, NK, NW, TMAB, CTAM>;
     int rc = set_smem(kern, smem);
     if (rc) return rc;
     static const CUtensorMap unused{};                   // the row-gather modes take no tensor map
-    const long long blocks = (items + NW - 1) / NW;
+    const long long blocks = CTAM ? items : (items + NW - 1) / NW;
     launch_k(__PRETTY_FUNCTION__, kern, (unsigned)blocks, NW * 32, smem, st, p, km ? *km : unused, vm ? *vm : unused);
     SA_CHECK_LAUNCH("gather_attn_kernel");
     return SA_OK;
@@ -245,9 +258,6 @@ static int launch_gather_nw(const GatherParams &p, long long items, cudaStream_t
 
 template <int D, int SRC, bool BIAS, bool KLO = false>
 static int launch_gather_t(const GatherParams &p, cudaStream_t st) {
-#ifndef SA_ATTN_NW
-#define SA_ATTN_NW 12
-#endif
     const long long items = (long long)p.B * p.q_units * p.Hkv * p.n_hchunk * p.n_split;
     if (items == 0) return SA_OK;
     if constexpr (SRC == KS_IDX && D == 128 && !BIAS && !KLO) {
@@ -280,15 +290,17 @@ static int launch_gather_t(const GatherParams &p, cudaStream_t st) {
     if constexpr (KLO) {
         return launch_gather_nw<D, SRC, BIAS, KLO, 8>(p, items, st);
     } else {
-        // small launches (decode pieces): 4-warp CTAs; SA_GATHER_SMALL_STAGES
-        // = 4 or 6 deepens their ring (for comparison), default 2
+        // small launches (decode pieces, fewer items than 12 per SM): with
+        // explicit lists, one CTA of 8 warps per item, the warps splitting the
+        // item's entries and merging in shared memory (8x the warps of one
+        // warp per item, same partial rows); otherwise 4-warp CTAs.
+        // SA_GATHER_SMALL=warp selects the 4-warp form for lists too (for
+        // comparison).
         if (items < (long long)sm_count() * SA_ATTN_NW) {
-            static const int small_stages = [] {
-                const char *e = std::getenv("SA_GATHER_SMALL_STAGES");
-                return e ? std::atoi(e) : 2;
-            }();
-            if (small_stages == 6) return launch_gather_nw<D, SRC, BIAS, KLO, 4, 6>(p, items, st);
-            if (small_stages == 4) return launch_gather_nw<D, SRC, BIAS, KLO, 4, 4>(p, items, st);
+            if constexpr (SRC == KS_IDX && !BIAS) {
+                if (!gather_small_per_warp())
+                    return launch_gather_nw<D, SRC, BIAS, KLO, 8, 2, 16, false, true>(p, items, st);
+            }
             return launch_gather_nw<D, SRC, BIAS, KLO, 4>(p, items, st);
         }
         // fixed-graph rows (KS_PROWS): SA_PROWS_NW = 16 or 20 warps per CTA
@@ -570,10 +582,12 @@ int sa_sparse_attn_fwd(const void *q, const void *k, const void *v, int B, int T
     const bool tc = attn_tc_applies(p, d, src, bias);
     // with a ticket array the gather kernel's last piece of each group does
     // the merge itself (no separate combine launch)
-    // SA_SPLIT_MERGE=fused: the last piece of each group merges (one launch
-    // fewer, but the merge runs on one warp after all pieces: measured slower
-    // for the 32 x 128K decode, 0.211 vs 0.156 ms per F S S S step), else the
-    // separate combine launch
+    // The pieces are merged by a separate combine launch, unless
+    // SA_SPLIT_MERGE=fused: then the last piece of each group to arrive
+    // merges them (its warp, or its whole CTA in the CTA-merged form).  One
+    // launch fewer, but the ticket reset and the serial merge after the
+    // last piece measured slower for the 32 x 128K decode (per F S S S step:
+    // 0.211 vs 0.156 ms one warp per piece, 0.156 vs 0.142 ms CTA-merged).
     static int fused = -1;
     if (fused < 0) {
         const char *e = std::getenv("SA_SPLIT_MERGE");
