@@ -45,7 +45,7 @@ def attn_flops(T: int, topk: int, window: int, Hq: int, d: int) -> float:
     return 4.0 * d * Hq * s
 
 
-ATTN_TRAFFIC_64K = 1_084_000_000
+ATTN_TRAFFIC_64K = 1_079_513_088
 
 
 def attn_rows(T: int, topk: int, window: int) -> int:
@@ -385,13 +385,14 @@ def main():
             "frac": round(att_tflops / peaks["bf16_tflops"], 4),
             "peak_source": peaks["source"] + " bf16 burst",
             # dram__bytes_read + dram__bytes_write of the 32768-token launch
-            # (0.542 GB) x 2: index lists, Q, O and LSE scale with query rows
+            # (0.540 GB) x 2: index lists, Q, O and LSE scale with query rows
             "traffic": ATTN_TRAFFIC_64K if w.T == 65536 else None,
             "traffic_source": "ncu, 32768-token launch scaled by query rows",
             "gathered_l2_bytes": int(w.B * 4 * w.d * attn_rows(w.T, w.topk, w.window)),
         },
         "indexer": {
-            "kernels": "idx_score_tc_kernel (sample, filter), idx_threshold_kernel, topk_select_kernel",
+            "kernels": "idx_score_tc_kernel (sample), idx_threshold_kernel, idx_filter_tc_kernel (filter), "
+                       "topk_select_kernel",
             "ms": round(idx_ms, 4),
             "int8_tops": round(idx_ops / (idx_ms / 1e3) / 1e12, 2),
             "peak": round(2 * peaks["bf16_tflops"], 1),

@@ -282,3 +282,24 @@ def test_sa_log_prints_launch_configs(cuda_ok):
     lines = [ln for ln in r.stderr.splitlines() if ln.startswith("[sa] ")]
     assert any("gather_attn" in ln or "launch_gather" in ln for ln in lines), r.stderr[-2000:]
     assert all("grid=(" in ln and "block=(" in ln and "smem=" in ln for ln in lines)
+
+
+@pytest.mark.parametrize("window", [17, 40, 65, 100])
+def test_fixed_pattern_one_head_per_kv_windows(cuda_ok, window):
+    """One query head per KV head, d = 64: windows whose band fills whole
+    16-key chunks take the dilated keys on the CUDA cores, the others on
+    the tensor cores; both must match the oracle, with and without bias."""
+    T, H, d = 900, 4, 64
+    g = inputs.gen_spatial(1, T, H, d, beta=0.5, seed=window, Hkv=H)
+    gd = to_dev(g)
+    idx, _ = oracle.fixed_graph(T, window, True, cap=window + 16)
+    out, lse = api.sparse_attn_fwd(gd["q"], gd["k"], gd["v"], pattern=(window, True), cq=gd["cq"], ck=gd["ck"],
+                                   beta=gd["beta"])
+    ro, rl = oracle.sparse_attn(g["q"], g["k"], g["v"], idx.reshape(1, T, -1), cq=g["cq"], ck=g["ck"],
+                                beta=g["beta"])
+    assert_out_close(out, ro)
+    assert_lse_close(lse, rl)
+    out2, lse2 = api.sparse_attn_fwd(gd["q"], gd["k"], gd["v"], pattern=(window, True))
+    ro2, rl2 = oracle.sparse_attn(g["q"], g["k"], g["v"], idx.reshape(1, T, -1))
+    assert_out_close(out2, ro2)
+    assert_lse_close(lse2, rl2)
