@@ -358,7 +358,7 @@ __global__ void __launch_bounds__(FT_THREADS, 1)
             int tau_r[QREG ? NQT : 1];
             if constexpr (QREG) {
 #pragma unroll
-                for (int q = 0; q < NQT; ++q) tau_r[q] = fast ? ft_fast_tau(tau_u[q]) : tau_u[q];
+                for (int q = 0; q < NQT; ++q) tau_r[q] = fast ? -ft_fast_tau(tau_u[q]) : tau_u[q];   // fast: -tau
             }
             const long long list0 = ((long long)b * p.Rt + (tq0 + q_lo - p.t0)) * p.cand_cap;
             int2 *const lbase = p.cand + list0;             // this warp's first query's list
@@ -394,17 +394,17 @@ __global__ void __launch_bounds__(FT_THREADS, 1)
                     for (int g0 = 0; g0 < NQH; g0 += NG) {
                         const int qb = half * NQH + g0;       // first query of the group (in this warp)
                         int sc[NG];
-                        unsigned mask = 0u;
+                        bool keep[NG];
                         if (fast) {
 #pragma unroll
                             for (int qq = 0; qq < NG; ++qq) {
-                                const int tq_ = QREG ? tau_r[qb + qq] : ft_fast_tau(tau_u[qb + qq]);
-                                int sacc = -tq_;
+                                const int ntau = QREG ? tau_r[qb + qq] : -ft_fast_tau(tau_u[qb + qq]);
+                                int sacc = ntau;
 #pragma unroll
                                 for (int h = 0; h < HI; ++h)
                                     sacc = __viaddmax_s32(sacc, (int)x[(g0 + qq) * HI + h], sacc);
-                                sc[qq] = sacc + tq_;
-                                mask |= (sacc >= 0) ? (1u << qq) : 0u;
+                                sc[qq] = sacc - ntau;
+                                keep[qq] = sacc >= 0;
                             }
                         } else {
 #pragma unroll
@@ -414,13 +414,12 @@ __global__ void __launch_bounds__(FT_THREADS, 1)
                                 for (int h = 0; h < HI; ++h)
                                     sacc += w_u[(qb + qq) * HI + h] * max((int)x[(g0 + qq) * HI + h], 0);
                                 sc[qq] = sacc;
-                                mask |= (sacc >= (QREG ? tau_r[qb + qq] : tau_u[qb + qq])) ? (1u << qq) : 0u;
+                                keep[qq] = sacc >= (QREG ? tau_r[qb + qq] : tau_u[qb + qq]);
                             }
                         }
                         if (!full) {                           // diagonal tiles: causal bound per query
 #pragma unroll
-                            for (int qq = 0; qq < NG; ++qq)
-                                if (j >= nc_u[qb + qq]) mask &= ~(1u << qq);
+                            for (int qq = 0; qq < NG; ++qq) keep[qq] = keep[qq] && j < nc_u[qb + qq];
                         }
                         // every keeping lane takes its list slot with its own
                         // shared-memory atomic (one per kept pair, ~10% of the
@@ -429,7 +428,7 @@ __global__ void __launch_bounds__(FT_THREADS, 1)
                         // the pair; 32-bit offsets from the unit's list base
 #pragma unroll
                         for (int qq = 0; qq < NG; ++qq) {
-                            if ((mask >> qq) & 1u) {
+                            if (keep[qq]) {
                                 const int slot = ft::atom_add1_shared(cnt_a + 4u * (uint32_t)(qb + qq));
                                 if (slot < cap) lbase[(qb + qq) * cap + slot] = make_int2(sc[qq], j);
                             }
