@@ -1097,53 +1097,48 @@ __global__ void __launch_bounds__(NT, NT <= 256 ? 3 : 1) topk_select_kernel(cons
         __syncthreads();
     }
 
-    // ordered output: warps own contiguous word ranges
+    // ordered output: warps own contiguous word ranges, and inside a warp
+    // each lane a contiguous run of words, so one prefix over the lanes
+    // (not one per 32 words) places every lane's keys
     const int wpw = (words + NW - 1) / NW;
     const int w_lo = min(warp * wpw, words), w_hi = min(w_lo + wpw, words);
-    int gcnt = 0, ecnt = 0;
-    for (int i = w_lo + lane; i < w_hi; i += 32) { gcnt += __popc(gt_bm[i]); ecnt += __popc(eq_bm[i]); }
-    gcnt = warp_sum_int(gcnt);
-    ecnt = warp_sum_int(ecnt);
-    if (lane == 0) { wg[warp] = gcnt; we[warp] = ecnt; }
+    const int wpl = (w_hi - w_lo + 31) / 32;                 // words per lane
+    const int l_lo = min(w_lo + lane * wpl, w_hi), l_hi = min(l_lo + wpl, w_hi);
+    int gl = 0, el = 0;
+    for (int i = l_lo; i < l_hi; ++i) { gl += __popc(gt_bm[i]); el += __popc(eq_bm[i]); }
+    int g_incl = gl, e_incl = el;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int xg = __shfl_up_sync(0xffffffffu, g_incl, o);
+        const int xe = __shfl_up_sync(0xffffffffu, e_incl, o);
+        if (lane >= o) { g_incl += xg; e_incl += xe; }
+    }
+    if (lane == 31) { wg[warp] = g_incl; we[warp] = e_incl; }
     __syncthreads();
     int g_before = 0, e_before = 0;
     for (int i = 0; i < warp; ++i) { g_before += wg[i]; e_before += we[i]; }
-    int out_base = g_before + min(e_before, k_rem);
-    for (int i0 = w_lo; i0 < w_hi; i0 += 32) {
-        const int i = i0 + lane;
-        const unsigned gw = i < w_hi ? gt_bm[i] : 0u;
-        const unsigned ew = i < w_hi ? eq_bm[i] : 0u;
-        // equal keys are taken in position order until k_rem are used
-        const int ec = __popc(ew);
-        int e_incl = ec;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int x = __shfl_up_sync(0xffffffffu, e_incl, o);
-            if (lane >= o) e_incl += x;
+    // equal keys are taken in position order until k_rem are used
+    const int e_pre = e_before + e_incl - el;                 // equal keys before this lane's run
+    int take = k_rem - e_pre;
+    take = take < 0 ? 0 : (take > el ? el : take);
+    int slot = g_before + (g_incl - gl) + min(e_pre, k_rem);
+    for (int i = l_lo; i < l_hi; ++i) {
+        const unsigned ew = eq_bm[i];
+        unsigned em = 0u;
+        if (take >= __popc(ew)) {
+            em = ew;
+        } else {
+            unsigned rest = ew;
+            for (int c = 0; c < take; ++c) { const unsigned lowbit = rest & (~rest + 1u); em |= lowbit; rest ^= lowbit; }
         }
-        const int e_pre = e_before + e_incl - ec;
-        int take = k_rem - e_pre;
-        take = take < 0 ? 0 : (take > ec ? ec : take);
-        unsigned em = 0u, rest = ew;
-        for (int c = 0; c < take; ++c) { const unsigned lowbit = rest & (~rest + 1u); em |= lowbit; rest ^= lowbit; }
-        const unsigned sw = gw | em;
-        const int sc = __popc(sw);
-        int s_incl = sc;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int x = __shfl_up_sync(0xffffffffu, s_incl, o);
-            if (lane >= o) s_incl += x;
-        }
-        int slot = out_base + s_incl - sc;
-        unsigned bits = sw;
+        take -= __popc(em);
+        unsigned bits = gt_bm[i] | em;
         while (bits) {
             const int bpos = __ffs(bits) - 1;
             bits &= bits - 1u;
             if (slot < k_eff) orow[slot] = i * 32 + bpos;   // slot < k_eff by construction
             ++slot;
         }
-        out_base += __shfl_sync(0xffffffffu, s_incl, 31);
-        e_before += __shfl_sync(0xffffffffu, e_incl, 31);
     }
 }
 
