@@ -488,6 +488,15 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
         __syncwarp();
         const unsigned char *ks_ = wsm + st * SB;
         const unsigned char *vs_ = ks_ + CH;
+        // ldmatrix addresses (row-gather layout, 256-byte aligned stages): the
+        // lane's row and the XOR of its swizzle are folded into one base, each
+        // 16-column step is then one XOR.  Q.K^T reads key rows (mi >> 1) * 8 + ri
+        // at unit 2s + (mi & 1), P.V rows (mi & 1) * 8 + ri at unit 2s + (mi >> 1)
+        // (mi = lane / 8, ri = lane % 8); the swizzle XORs the unit with ri
+        [[maybe_unused]] const uint32_t ka_s =
+            tc::smem_u32(ks_) + (uint32_t)((((lane >> 4) * 8) + (lane & 7)) * ROWB + ((((lane >> 3) & 1) ^ (lane & 7)) << 4));
+        [[maybe_unused]] const uint32_t va_s =
+            tc::smem_u32(vs_) + (uint32_t)(((((lane >> 3) & 1) * 8) + (lane & 7)) * ROWB + (((lane >> 4) ^ (lane & 7)) << 4));
         const int jl = lane < NK ? keys_s[st * NK + lane] : -1;
         const int sl = PR && lane < NK ? segs_s[st * NK + lane] : 0;
         const unsigned vmask = __ballot_sync(0xffffffffu, jl >= 0);
@@ -503,15 +512,19 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
                 float (&acc)[NK / 8][4] = (ks & 1) ? sc2 : sc;
 #pragma unroll
                 for (int np = 0; np < NK / 16; ++np) {
-                    const int mi = lane >> 3, ri = lane & 7;
-                    const int key = np * 16 + (mi >> 1) * 8 + ri;
-                    const int unit = ks * 2 + (mi & 1);
                     unsigned b0, b1, b2, b3;
-                    ldsm_x4(b0, b1, b2, b3, ks_ + kv_off(key, unit));
+                    if constexpr (TMAB) {
+                        const int mi = lane >> 3, ri = lane & 7;
+                        const int key = np * 16 + (mi >> 1) * 8 + ri;
+                        const int unit = ks * 2 + (mi & 1);
+                        ldsm_x4(b0, b1, b2, b3, ks_ + kv_off(key, unit));
+                    } else {
+                        ldsm_x4_a(b0, b1, b2, b3, (ka_s + np * 16 * ROWB) ^ (uint32_t)(ks << 5));
+                    }
                     mma_bf16_16816(acc[2 * np], qf[ks], b0, b1);
                     mma_bf16_16816(acc[2 * np + 1], qf[ks], b2, b3);
                     if constexpr (KLO) {
-                        ldsm_x4(b0, b1, b2, b3, vs_ + CH + kv_off(key, unit));
+                        ldsm_x4_a(b0, b1, b2, b3, (ka_s + 2 * CH + np * 16 * ROWB) ^ (uint32_t)(ks << 5));
                         mma_bf16_16816(acc[2 * np], qf[ks], b0, b1);
                         mma_bf16_16816(acc[2 * np + 1], qf[ks], b2, b3);
                     }
@@ -630,11 +643,15 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
                 pa[3] = pack_bf16(sc[2 * kp + 1][2], sc[2 * kp + 1][3]);
 #pragma unroll
                 for (int dp = 0; dp < NT_D / 2; ++dp) {
-                    const int mi = lane >> 3, ri = lane & 7;
-                    const int key = kp * 16 + (mi & 1) * 8 + ri;
-                    const int unit = dp * 2 + (mi >> 1);
                     unsigned b0, b1, b2, b3;
-                    ldsm_x4_t(b0, b1, b2, b3, vs_ + kv_off(key, unit));
+                    if constexpr (TMAB) {
+                        const int mi = lane >> 3, ri = lane & 7;
+                        const int key = kp * 16 + (mi & 1) * 8 + ri;
+                        const int unit = dp * 2 + (mi >> 1);
+                        ldsm_x4_t(b0, b1, b2, b3, vs_ + kv_off(key, unit));
+                    } else {
+                        ldsm_x4_ta(b0, b1, b2, b3, (va_s + kp * 16 * ROWB) ^ (uint32_t)(dp << 5));
+                    }
                     mma_bf16_16816(o[2 * dp], pa, b0, b1);
                     mma_bf16_16816(o[2 * dp + 1], pa, b2, b3);
                 }

@@ -889,6 +889,112 @@ __global__ void __launch_bounds__(SEL_THREADS, 4) idx_threshold_kernel(const Idx
     if (threadIdx.x == 0) p.tau[row] = (int)((unsigned)gmin + st.lo_key);
 }
 
+// Warp-per-row form of idx_threshold_kernel (the default): 8 rows per CTA,
+// each warp streams its row's sample from L2 with 16-byte loads, takes the
+// range with shuffles, then the r-th largest value by 8-bit radix digits
+// from the top (a 256-bin histogram per warp in shared memory, the bin found
+// by a suffix scan over the lanes' 8 bins each).  No block barriers, so the
+// rows of a CTA proceed independently.
+constexpr int THW_WARPS = 8;
+__global__ void __launch_bounds__(THW_WARPS * 32) idx_threshold_warp_kernel(const IdxParams p) {
+    grid_dependency_sync();
+    __shared__ int hist_all[THW_WARPS][SEL_BINS];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long row = (long long)blockIdx.x * THW_WARPS + warp;
+    if (row >= (long long)p.B * p.Rt) return;
+    const int tr = (int)(row % p.Rt), t = p.t0 + tr;
+    if (t >= p.Tq) return;
+    int *hist = hist_all[warp];
+    if (lane == 0) p.cand_cnt[row] = 0;                       // the filter pass appends from zero
+    const int n = (int)n_candidates(p.q_pos0 + t, p.window);
+    const int k_eff = n < p.topk ? n : p.topk;
+    if (k_eff == n || k_eff == 0) {
+        if (lane == 0) p.tau[row] = k_eff == 0 ? INT_MAX : INT_MIN;
+        return;
+    }
+    const int tq0 = p.t0 + ((t - p.t0) / p.nq_block) * p.nq_block;
+    const int s = sample_stride(p, tq0);
+    const int m = (n + s - 1) / s;
+    int r;
+    if (s == 1) {
+        r = k_eff;
+    } else {
+        // the same rank rule as idx_threshold_kernel
+        const double e = (double)k_eff * m / n;
+        double rr = e + SAMPLE_Z * sqrt(e) + 2.0;
+        rr = e + SAMPLE_Z * sqrt(rr) + 2.0;
+        rr = e + SAMPLE_Z * sqrt(rr) + 2.0;
+        r = (int)ceil(rr);
+        r = min(r, m);
+    }
+    const int32_t *vals = p.sample + row * p.m_cap;           // 16-byte aligned rows (m_cap % 4 == 0)
+    const int m4 = m / 4;
+    auto for_each = [&](auto f) {
+        const int4 *v4 = reinterpret_cast<const int4 *>(vals);
+        constexpr int U = 4;
+        for (int b0 = lane; b0 < m4; b0 += 32 * U) {
+            int4 x[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+                if (b0 + 32 * u < m4) x[u] = __ldcg(v4 + b0 + 32 * u);
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+                if (b0 + 32 * u < m4) { f(x[u].x); f(x[u].y); f(x[u].z); f(x[u].w); }
+        }
+        for (int i = 4 * m4 + lane; i < m; i += 32) f(__ldcg(vals + i));
+    };
+    int vmin = INT_MAX, vmax = INT_MIN;
+    for_each([&](int v) { vmin = min(vmin, v); vmax = max(vmax, v); });
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        vmin = min(vmin, __shfl_xor_sync(0xffffffffu, vmin, o));
+        vmax = max(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+    }
+    const unsigned range = (unsigned)vmax - (unsigned)vmin;
+    int width = range == 0 ? 0 : 32 - __clz(range);
+    unsigned lo_key = 0u;                                     // digits chosen so far, in place
+    int r_rem = r;
+    while (width > 0) {
+        const int shift = width > SEL_BITS ? width - SEL_BITS : 0;
+        const unsigned hi_mask = ~((width >= 32) ? 0u : ((1u << width) - 1u));   // bits already fixed
+#pragma unroll
+        for (int i = 0; i < SEL_BINS / 32; ++i) hist[lane * (SEL_BINS / 32) + i] = 0;
+        __syncwarp();
+        for_each([&](int v) {
+            const unsigned key = (unsigned)v - (unsigned)vmin;
+            if ((key & hi_mask) == lo_key) atomicAdd(&hist[(key >> shift) & (SEL_BINS - 1)], 1);
+        });
+        __syncwarp();
+        // lane l holds bins 8l .. 8l+7; counts above each bin from the top
+        int cb[SEL_BINS / 32], local = 0;
+#pragma unroll
+        for (int i = 0; i < SEL_BINS / 32; ++i) { cb[i] = hist[lane * (SEL_BINS / 32) + i]; local += cb[i]; }
+        int suf = local;                                      // inclusive suffix over lanes
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int x = __shfl_down_sync(0xffffffffu, suf, o);
+            if (lane + o < 32) suf += x;
+        }
+        int above = suf - local;                              // values in higher lanes' bins
+        int sel_bin = -1, sel_above = 0;
+#pragma unroll
+        for (int i = SEL_BINS / 32 - 1; i >= 0; --i) {
+            if (sel_bin < 0 && above < r_rem && above + cb[i] >= r_rem) { sel_bin = lane * (SEL_BINS / 32) + i; sel_above = above; }
+            above += cb[i];
+        }
+        const unsigned who = __ballot_sync(0xffffffffu, sel_bin >= 0);
+        if (who == 0u) break;                                 // cannot happen (r <= m); keeps the lower bound
+        const int src = __ffs(who) - 1;                       // exactly one lane holds the bin
+        sel_bin = __shfl_sync(0xffffffffu, sel_bin, src);
+        sel_above = __shfl_sync(0xffffffffu, sel_above, src);
+        r_rem -= sel_above;
+        lo_key |= (unsigned)sel_bin << shift;
+        width = shift;
+        __syncwarp();
+    }
+    if (lane == 0) p.tau[row] = (int)((unsigned)vmin + lo_key);
+}
+
 // ----------------------------------------------------------- final select --
 // Rows whose top-k was taken by the exact-recompute path (the candidate list
 // was short or overflowed), counted per device; read and cleared by

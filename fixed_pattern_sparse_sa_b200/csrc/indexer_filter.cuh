@@ -429,8 +429,11 @@ __global__ void __launch_bounds__(FT_THREADS, 1)
 #pragma unroll
                         for (int qq = 0; qq < NG; ++qq) {
                             if (keep[qq]) {
+                                // past the capacity the row's count marks the list
+                                // unusable (the select recomputes the row), so an
+                                // overflowing pair may land on the last slot
                                 const int slot = ft::atom_add1_shared(cnt_a + 4u * (uint32_t)(qb + qq));
-                                if (slot < cap) lbase[(qb + qq) * cap + slot] = make_int2(sc[qq], j);
+                                lbase[(qb + qq) * cap + min(slot, cap - 1)] = make_int2(sc[qq], j);
                             }
                         }
                     }

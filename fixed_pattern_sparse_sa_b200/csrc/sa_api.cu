@@ -232,6 +232,17 @@ static bool gather_small_per_warp() {
 #ifndef SA_ATTN_NW
 #define SA_ATTN_NW 12
 #endif
+// SA_THRESHOLD=block: one CTA per row for the sampled threshold for every
+// call (for comparison); by default one warp per row when there are rows
+// for 8 warps per SM.
+static bool threshold_per_warp() {
+    static const bool v = [] {
+        const char *e = std::getenv("SA_THRESHOLD");
+        return !(e && std::strcmp(e, "block") == 0);
+    }();
+    return v;
+}
+
 // -------------------------------------------------------- gather launches --
 // Launch shape: 12 warps per CTA streaming 16-key chunks through a 2-stage
 // ring (8 warps when the lo-key tile is also staged); ~200 KB of shared
@@ -962,8 +973,15 @@ int sa_indexer_topk(const int8_t *q_idx, const int8_t *k_idx, const int32_t *w, 
         if (ncand > 0) {
             rc = launch_score<MODE_SAMPLE>(p, lay.decode, (long long)lay.m_cap, st);
             if (rc) return rc;
-            launch_k("idx_threshold_kernel", idx_threshold_kernel, dim3(1u, (unsigned)rows, (unsigned)B), SEL_THREADS,
-                0, st, p);
+            // one warp per row when the rows fill the SMs (prefill); one CTA
+            // per row for a few rows (decode), where a row's latency decides
+            if (threshold_per_warp() && (long long)B * rows >= (long long)sm_count() * THW_WARPS) {
+                const unsigned blocks = (unsigned)(((long long)B * rows + THW_WARPS - 1) / THW_WARPS);
+                launch_k("idx_threshold_warp_kernel", idx_threshold_warp_kernel, blocks, THW_WARPS * 32, 0, st, p);
+            } else {
+                launch_k("idx_threshold_kernel", idx_threshold_kernel, dim3(1u, (unsigned)rows, (unsigned)B),
+                         SEL_THREADS, 0, st, p);
+            }
             SA_CHECK_LAUNCH("idx_threshold_kernel");
             if (filter_tc)
                 rc = di == 32 ? launch_filter_tc_d<32>(p, qf, wf, st)

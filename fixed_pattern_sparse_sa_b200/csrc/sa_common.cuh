@@ -107,6 +107,17 @@ __device__ __forceinline__ void ldsm_x4(unsigned &r0, unsigned &r1, unsigned &r2
                  : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
                  : "r"(s));
 }
+// The same two loads from a 32-bit shared-memory address.
+__device__ __forceinline__ void ldsm_x4_a(unsigned &r0, unsigned &r1, unsigned &r2, unsigned &r3, uint32_t s) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(s));
+}
+__device__ __forceinline__ void ldsm_x4_ta(unsigned &r0, unsigned &r1, unsigned &r2, unsigned &r3, uint32_t s) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(s));
+}
 __device__ __forceinline__ void ldsm_x4_t(unsigned &r0, unsigned &r1, unsigned &r2, unsigned &r3,
                                           const void *smem) {
     unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
