@@ -349,6 +349,7 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
     const __nv_bfloat16 *vb = p.v + ((long long)b * p.Lk * p.Hkv + g) * D;
     const __nv_bfloat16 *lb = KLO ? p.klo + ((long long)b * p.Lk * p.Hkv + g) * D : nullptr;
     const long long rstride = (long long)p.Hkv * D;
+    [[maybe_unused]] const uint32_t rs_bytes = (uint32_t)(rstride * 2);    // Hkv * D * 2 < 2^32
     // copy lanes: lane = lrow * UNITS + u (u: 16-byte unit of a row, lrow: row within an instruction)
     [[maybe_unused]] constexpr int RPI = 32 / UNITS;
     [[maybe_unused]] const int lrow_c = lane / UNITS, u_c = lane % UNITS;
@@ -425,12 +426,17 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
                 static_for<CP_ITERS>([&](auto ic) {
                     constexpr int it = decltype(ic)::value;
                     const int jr = __shfl_sync(0xffffffffu, j, it * RPI + lrow_c);
-                    const long long jo = (long long)max(jr, 0) * rstride;
+                    // row offset in bytes: a 32 x 32 -> 64-bit multiply-add per
+                    // pointer (the row stride Hkv * D * 2 fits 32 bits)
+                    const uint32_t jc = (uint32_t)max(jr, 0);
                     const int nb = jr >= 0 ? 16 : 0;
                     const uint32_t dst = base ^ (uint32_t)(((it * RPI) & 7) << 4);
-                    cp_async16_at<it * RPI * ROWB, 0>(dst, kb_u + jo, nb);
-                    cp_async16_at<it * RPI * ROWB + CH, 0>(dst, vb_u + jo, nb);
-                    if constexpr (KLO) cp_async16_at<it * RPI * ROWB + 2 * CH, 0>(dst, lb_u + jo, nb);
+                    cp_async16_at<it * RPI * ROWB, 0>(dst, reinterpret_cast<const char *>(kb_u) + (size_t)jc * rs_bytes, nb);
+                    cp_async16_at<it * RPI * ROWB + CH, 0>(dst, reinterpret_cast<const char *>(vb_u) + (size_t)jc * rs_bytes,
+                                                         nb);
+                    if constexpr (KLO)
+                        cp_async16_at<it * RPI * ROWB + 2 * CH, 0>(
+                            dst, reinterpret_cast<const char *>(lb_u) + (size_t)jc * rs_bytes, nb);
                 });
             } else {
                 // head dim 64 (measured faster for the fixed-graph rows): the

@@ -343,6 +343,8 @@ static int launch_gather_d(const GatherParams &p, int src, bool bias, cudaStream
 }
 
 static int launch_gather(const GatherParams &p, int d, int src, bool bias, cudaStream_t st) {
+    // the kernel forms a key row's offset as a 32-bit row stride (Hkv * d * 2 bytes) times the key
+    if ((long long)p.Hkv * d * 2 >= (1LL << 32)) return fail(SA_ERR_UNSUPPORTED, "gather: Hkv * d too large");
     if (d == 64) return launch_gather_d<64>(p, src, bias, st);
     if (d == 128) return launch_gather_d<128>(p, src, bias, st);
     return fail(SA_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
