@@ -253,11 +253,6 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
     uint64_t *full_s = reinterpret_cast<uint64_t *>(smem + NW * STAGES * (SB + NK * 4)) + warp * STAGES;
     int *segs_s = keys_s + STAGES * NK;                      // KS_PROWS only
     float *ck_s = reinterpret_cast<float *>(keys_s + STAGES * NK * (PR ? 2 : 1));   // [STAGES][NK][3] (bias only)
-    // byte offset of 16-byte unit u of key row `key` in a K / V chunk
-    auto kv_off = [](int key, int unit) -> int {
-        return TMAB ? (unit >> 3) * (NK * 128) + key * 128 + (((unit & 7) ^ (key & 7)) << 4)
-                    : key * ROWB + ((unit ^ (key & 7)) << 4);
-    };
     if constexpr (TMAB) {
         if (lane == 0) {
             for (int i = 0; i < STAGES; ++i) tc::mbar_init(full_s + i, 1);
@@ -446,12 +441,12 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
                     const int lin = it * 32 + lane;
                     const int rr = lin / UNITS, u = lin % UNITS;
                     const int jr = __shfl_sync(0xffffffffu, j, rr);
-                    const long long off = jr >= 0 ? (long long)jr * rstride + u * 8 : 0;
+                    const size_t off = (size_t)(uint32_t)max(jr, 0) * rs_bytes + u * 16;   // bytes
                     const int nb = jr >= 0 ? 16 : 0;
                     const int sw = (u ^ (rr & 7)) * 16;
-                    cp_async16(ks_ + rr * ROWB + sw, kb + off, nb);
-                    cp_async16(vs_ + rr * ROWB + sw, vb + off, nb);
-                    if constexpr (KLO) cp_async16(vs_ + CH + rr * ROWB + sw, lb + off, nb);
+                    cp_async16(ks_ + rr * ROWB + sw, reinterpret_cast<const char *>(kb) + off, nb);
+                    cp_async16(vs_ + rr * ROWB + sw, reinterpret_cast<const char *>(vb) + off, nb);
+                    if constexpr (KLO) cp_async16(vs_ + CH + rr * ROWB + sw, reinterpret_cast<const char *>(lb) + off, nb);
                 }
             }
         }
@@ -494,9 +489,12 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
         __syncwarp();
         const unsigned char *ks_ = wsm + st * SB;
         const unsigned char *vs_ = ks_ + CH;
-        // ldmatrix addresses (row-gather layout, 256-byte aligned stages): the
-        // lane's row and the XOR of its swizzle are folded into one base, each
-        // 16-column step is then one XOR.  Q.K^T reads key rows (mi >> 1) * 8 + ri
+        // ldmatrix addresses.  Row-gather layout: key row r at r * ROWB, its
+        // 16-byte unit u at ((u ^ (r & 7)) << 4), stages 256-byte aligned.  TMA
+        // block layout: 64-column halves NK * 128 bytes apart, rows of 128
+        // bytes, unit u of a half at (((u & 7) ^ (r & 7)) << 4).  For the
+        // row-gather layout at head dim 128 the lane's row and the XOR of its
+        // swizzle are folded into one base, each 16-column step is then one XOR.  Q.K^T reads key rows (mi >> 1) * 8 + ri
         // at unit 2s + (mi & 1), P.V rows (mi & 1) * 8 + ri at unit 2s + (mi >> 1)
         // (mi = lane / 8, ri = lane % 8); the swizzle XORs the unit with ri
         [[maybe_unused]] const uint32_t ka_s =
@@ -519,17 +517,23 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
 #pragma unroll
                 for (int np = 0; np < NK / 16; ++np) {
                     unsigned b0, b1, b2, b3;
-                    if constexpr (TMAB) {
+                    if constexpr (TMAB || D == 64) {
+                        // per-step swizzle arithmetic: the folded form below
+                        // measured no faster for the TMA block layout and
+                        // slower at head dim 64
                         const int mi = lane >> 3, ri = lane & 7;
                         const int key = np * 16 + (mi >> 1) * 8 + ri;
                         const int unit = ks * 2 + (mi & 1);
-                        ldsm_x4(b0, b1, b2, b3, ks_ + kv_off(key, unit));
+                        const int off = TMAB ? (unit >> 3) * (NK * 128) + key * 128 + (((unit & 7) ^ (key & 7)) << 4)
+                                             : key * ROWB + ((unit ^ (key & 7)) << 4);
+                        ldsm_x4(b0, b1, b2, b3, ks_ + off);
                     } else {
                         ldsm_x4_a(b0, b1, b2, b3, (ka_s + np * 16 * ROWB) ^ (uint32_t)(ks << 5));
                     }
                     mma_bf16_16816(acc[2 * np], qf[ks], b0, b1);
                     mma_bf16_16816(acc[2 * np + 1], qf[ks], b2, b3);
                     if constexpr (KLO) {
+                        // the lo half of the keys, 2 * CH bytes after the hi half
                         ldsm_x4_a(b0, b1, b2, b3, (ka_s + 2 * CH + np * 16 * ROWB) ^ (uint32_t)(ks << 5));
                         mma_bf16_16816(acc[2 * np], qf[ks], b0, b1);
                         mma_bf16_16816(acc[2 * np + 1], qf[ks], b2, b3);
@@ -650,11 +654,13 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
 #pragma unroll
                 for (int dp = 0; dp < NT_D / 2; ++dp) {
                     unsigned b0, b1, b2, b3;
-                    if constexpr (TMAB) {
+                    if constexpr (TMAB || D == 64) {
                         const int mi = lane >> 3, ri = lane & 7;
                         const int key = kp * 16 + (mi & 1) * 8 + ri;
                         const int unit = dp * 2 + (mi >> 1);
-                        ldsm_x4_t(b0, b1, b2, b3, vs_ + kv_off(key, unit));
+                        const int off = TMAB ? (unit >> 3) * (NK * 128) + key * 128 + (((unit & 7) ^ (key & 7)) << 4)
+                                             : key * ROWB + ((unit ^ (key & 7)) << 4);
+                        ldsm_x4_t(b0, b1, b2, b3, vs_ + off);
                     } else {
                         ldsm_x4_ta(b0, b1, b2, b3, (va_s + kp * 16 * ROWB) ^ (uint32_t)(dp << 5));
                     }

@@ -309,8 +309,15 @@ static int launch_gather_t(const GatherParams &p, cudaStream_t st) {
         // comparison).
         if (items < (long long)sm_count() * SA_ATTN_NW) {
             if constexpr (SRC == KS_IDX && !BIAS) {
-                if (!gather_small_per_warp())
+                if (!gather_small_per_warp()) {
+                    // SA_CTAM_STAGES=3: a 3-stage ring per warp (for comparison)
+                    static const int ctam_stages = [] {
+                        const char *e = std::getenv("SA_CTAM_STAGES");
+                        return e ? std::atoi(e) : 2;
+                    }();
+                    if (ctam_stages == 3) return launch_gather_nw<D, SRC, BIAS, KLO, 8, 3, 16, false, true>(p, items, st);
                     return launch_gather_nw<D, SRC, BIAS, KLO, 8, 2, 16, false, true>(p, items, st);
+                }
             }
             return launch_gather_nw<D, SRC, BIAS, KLO, 4>(p, items, st);
         }
