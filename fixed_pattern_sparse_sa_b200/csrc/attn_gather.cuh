@@ -41,6 +41,7 @@ struct GatherParams {
     int idx_heads, K;
     int window, dilated;      // KS_PATTERN / KS_RANGE
     int block;                // KS_BLOCKS block length
+    int block_shift;          // log2(block) when block is a power of two, else -1
     int cmp_len;              // unused by the gather kernel
     int entries;              // virtual list length per item
     int per_split;            // entries handled by one split piece
@@ -76,7 +77,7 @@ __device__ __forceinline__ int key_raw(const GatherParams &p, int b, int t, int 
         return __ldg(list + e);
     } else if constexpr (SRC == KS_BLOCKS) {
         const int32_t *list = p.idx + ((long long)(b * p.Tq + t) * p.Hkv + g) * p.K;
-        return __ldg(list + e / p.block);
+        return __ldg(list + (p.block_shift >= 0 ? e >> p.block_shift : e / p.block));
     } else if constexpr (SRC == KS_PATTERN) {
         long long nw = pos + 1 < p.window ? pos + 1 : p.window;
         if (e < nw) return (int)(pos - e);
@@ -159,7 +160,7 @@ __device__ __forceinline__ int key_finish(const GatherParams &p, long long pos, 
             raise_error(p.err, ERR_BAD_BLOCK);
             return -1;
         }
-        const long long j = (long long)blk * p.block + e % p.block;
+        const long long j = (long long)blk * p.block + (p.block_shift >= 0 ? e & (p.block - 1) : e % p.block);
         if (j > pos || j >= p.Lk) return -1;   // causal mask inside the block
         return (int)j;
     } else {

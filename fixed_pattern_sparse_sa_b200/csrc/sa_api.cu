@@ -209,13 +209,16 @@ static int bf16_tensor_map_3d(CUtensorMap *m, const void *base, int d, int hkv, 
     return SA_OK;
 }
 
-// SA_GATHER_TMA=0 keeps the NSA selected branch on per-row cp.async copies
-// (for comparison); by default its 16-row block chunks come by TMA.
+// SA_GATHER_TMA=1 loads the NSA selected branch's 16-row block chunks by TMA
+// box loads (for comparison); by default they take the per-row cp.async
+// copies of the explicit-list path, measured faster (64K NSA step 30.9 vs
+// 33.9 ms) since those copies issue whole 128-byte lines from per-lane
+// addresses with immediate offsets.
 static bool gather_tma_allowed() {
     static int v = -1;
     if (v < 0) {
         const char *e = std::getenv("SA_GATHER_TMA");
-        v = (e && std::strcmp(e, "0") == 0) ? 0 : 1;
+        v = (e && std::strcmp(e, "1") == 0) ? 1 : 0;
     }
     return v != 0;
 }
@@ -309,15 +312,8 @@ static int launch_gather_t(const GatherParams &p, cudaStream_t st) {
         // comparison).
         if (items < (long long)sm_count() * SA_ATTN_NW) {
             if constexpr (SRC == KS_IDX && !BIAS) {
-                if (!gather_small_per_warp()) {
-                    // SA_CTAM_STAGES=3: a 3-stage ring per warp (for comparison)
-                    static const int ctam_stages = [] {
-                        const char *e = std::getenv("SA_CTAM_STAGES");
-                        return e ? std::atoi(e) : 2;
-                    }();
-                    if (ctam_stages == 3) return launch_gather_nw<D, SRC, BIAS, KLO, 8, 3, 16, false, true>(p, items, st);
+                if (!gather_small_per_warp())
                     return launch_gather_nw<D, SRC, BIAS, KLO, 8, 2, 16, false, true>(p, items, st);
-                }
             }
             return launch_gather_nw<D, SRC, BIAS, KLO, 4>(p, items, st);
         }
@@ -1226,6 +1222,7 @@ int sa_nsa_fwd(const void *q, const void *k, const void *v, const float *gates, 
         GatherParams p = base;
         p.k = static_cast<const __nv_bfloat16 *>(k); p.v = static_cast<const __nv_bfloat16 *>(v);
         p.Lk = T; p.idx = sel; p.K = sel_topk; p.block = sel_block;
+        p.block_shift = (sel_block & (sel_block - 1)) == 0 ? __builtin_ctz((unsigned)sel_block) : -1;
         p.entries = sel_topk * sel_block; p.per_split = p.entries;
         p.out_f32 = o3 + rows * d; p.lse = l3 + rows;
         rc = attn_tc_applies(p, d, KS_BLOCKS, false) ? launch_attn_tc<KS_BLOCKS>(p, st)

@@ -114,12 +114,14 @@ def test_indexcache_decode_small(cuda_ok, pattern):
     np.testing.assert_array_equal(cache.cpu().numpy().reshape(ref[-1][0].shape), ref[-1][0])
 
 
-def test_decode128k_full_size(cuda_ok):
+@pytest.mark.parametrize("n_split", [4, 16])
+def test_decode128k_full_size(cuda_ok, n_split):
     # 32 sequences x 131072 cached tokens, 4 layers; caches drawn on the GPU.
+    # 4 pieces per row is the benchmark's launch form (CTA-merged pieces).
     w = inputs.WORKLOADS["dsa_decode128k"]
     lays = _decode_layers(w.B, w.T, 4, seed=0, device="cuda")
     for pattern in ("FSSS", "FFFF"):
-        outs, lses, cache = api.dsa_decode_layers(pattern, lays, topk=w.topk, n_split=16)
+        outs, lses, cache = api.dsa_decode_layers(pattern, lays, topk=w.topk, n_split=n_split)
         torch.cuda.synchronize()
         # oracle on a few sequences of every layer (host copies of those rows)
         seqs = [0, 17, 31]
