@@ -45,7 +45,7 @@ def attn_flops(T: int, topk: int, window: int, Hq: int, d: int) -> float:
     return 4.0 * d * Hq * s
 
 
-ATTN_TRAFFIC_64K = 1_079_513_088
+ATTN_TRAFFIC_64K = 1_079_603_200
 
 
 def attn_rows(T: int, topk: int, window: int) -> int:
