@@ -781,14 +781,10 @@ __device__ void block_minmax(int &gmin, int &gmax, int *bcast, ForEach for_each)
 // one histogram with a bin per value (fh: SEL_FINE_BINS ints of shared
 // memory).  Returns, block-uniform, the k-th largest value's offset from
 // gmin and the number of values above it.
-template <int NT, typename ForEach>
-__device__ void fine_kth(int k, int gmin, int *fh, int *scan_tmp, int *bcast, ForEach for_each, int &bin,
-                         int &above_bin) {
+// Second half of fine_kth: the k-th largest bin of a filled histogram.
+template <int NT>
+__device__ void fine_scan(int k, const int *fh, int *scan_tmp, int *bcast, int &bin, int &above_bin) {
     const int tid = threadIdx.x;
-    for (int i = tid; i < SEL_FINE_BINS; i += NT) fh[i] = 0;
-    __syncthreads();
-    for_each([&](int v, int) { atomicAdd(&fh[(unsigned)v - (unsigned)gmin], 1); });
-    __syncthreads();
     constexpr int PER = SEL_FINE_BINS / NT;               // bins per thread, highest first
     int cb[PER], local = 0;
 #pragma unroll
@@ -807,6 +803,15 @@ __device__ void fine_kth(int k, int gmin, int *fh, int *scan_tmp, int *bcast, Fo
     bin = bcast[2];
     above_bin = bcast[3];
     __syncthreads();
+}
+template <int NT, typename ForEach>
+__device__ void fine_kth(int k, int gmin, int *fh, int *scan_tmp, int *bcast, ForEach for_each, int &bin,
+                         int &above_bin) {
+    for (int i = threadIdx.x; i < SEL_FINE_BINS; i += NT) fh[i] = 0;
+    __syncthreads();
+    for_each([&](int v, int) { atomicAdd(&fh[(unsigned)v - (unsigned)gmin], 1); });
+    __syncthreads();
+    fine_scan<NT>(k, fh, scan_tmp, bcast, bin, above_bin);
 }
 
 // Streams int32 values [0, n) from global memory with 16-byte loads, U vectors
@@ -1106,6 +1111,17 @@ __global__ void __launch_bounds__(NT, NT <= 256 ? 3 : 1) topk_select_kernel(cons
     int *lv_s = reinterpret_cast<int *>(smem + select_stage_off<DI>(words));
     int *li_s = lv_s + p.cand_cap;
     int smin = INT_MAX, smax = INT_MIN;
+    // Every listed score is >= the row's threshold tau (the filter kept
+    // exactly those), so a histogram with bin = score - tau can be filled
+    // while staging; when every score falls within SEL_FINE_BINS of tau it
+    // gives the k-th largest score without another pass.
+    int *fh = reinterpret_cast<int *>(tie_key);               // the tie arrays serve as its bins
+    const int tau_b = staged ? p.tau[row] : 0;
+    bool wide = false;
+    if (staged) {
+        for (int i = tid; i < SEL_FINE_BINS; i += NT) fh[i] = 0;
+        __syncthreads();
+    }
     if (staged) {
         constexpr int U = 4;
         const int n2 = (cnt + 1) / 2;                 // rows are 16-byte aligned (cap % 64 == 0)
@@ -1122,7 +1138,14 @@ __global__ void __launch_bounds__(NT, NT <= 256 ? 3 : 1) topk_select_kernel(cons
                     reinterpret_cast<int2 *>(li_s)[i] = make_int2(e[u].y, e[u].w);
                     smin = min(smin, e[u].x);
                     smax = max(smax, e[u].x);
-                    if (2 * i + 1 < cnt) { smin = min(smin, e[u].z); smax = max(smax, e[u].z); }
+                    unsigned bin = (unsigned)e[u].x - (unsigned)tau_b;
+                    if (bin < (unsigned)SEL_FINE_BINS) atomicAdd(&fh[bin], 1); else wide = true;
+                    if (2 * i + 1 < cnt) {
+                        smin = min(smin, e[u].z);
+                        smax = max(smax, e[u].z);
+                        bin = (unsigned)e[u].z - (unsigned)tau_b;
+                        if (bin < (unsigned)SEL_FINE_BINS) atomicAdd(&fh[bin], 1); else wide = true;
+                    }
                 }
             }
         }
@@ -1149,19 +1172,32 @@ __global__ void __launch_bounds__(NT, NT <= 256 ? 3 : 1) topk_select_kernel(cons
         }
     };
 
+    // the barrier publishes the staged list and its histogram
+    const bool any_wide = staged ? __syncthreads_or(wide) != 0 : true;
     int gmin, gmax;
-    if (staged) block_minmax_reduce(smin, smax, gmin, gmax, bcast);   // its barriers publish the staged list
-    else block_minmax(gmin, gmax, bcast, for_each);
-    const unsigned range = (unsigned)gmax - (unsigned)gmin;
-    RadixState st{0u, range == 0 ? 0 : 32 - __clz(range), k_eff, use_list ? cnt : n};
-    if (use_list && range < (unsigned)SEL_FINE_BINS) {
-        // narrow score range: one exact histogram (bin = score - min) gives
-        // the k-th largest score directly; the tie arrays serve as its bins
+    RadixState st{0u, 0, k_eff, use_list ? cnt : n};
+    if (!any_wide) {
+        // every score within SEL_FINE_BINS of tau: the k-th largest from the
+        // histogram filled while staging (keys below are relative to tau)
         int bin, above;
-        fine_kth<NT>(k_eff, gmin, reinterpret_cast<int *>(tie_key), scan_tmp, bcast, for_each, bin, above);
+        fine_scan<NT>(k_eff, fh, scan_tmp, bcast, bin, above);
+        gmin = tau_b;
         st.lo_key = (unsigned)bin;
-        st.width = 0;
         st.k_rem = k_eff - above;
+    } else {
+        if (staged) block_minmax_reduce(smin, smax, gmin, gmax, bcast);
+        else block_minmax(gmin, gmax, bcast, for_each);
+        const unsigned range = (unsigned)gmax - (unsigned)gmin;
+        st.width = range == 0 ? 0 : 32 - __clz(range);
+        if (use_list && range < (unsigned)SEL_FINE_BINS) {
+            // narrow score range: one exact histogram (bin = score - min) gives
+            // the k-th largest score directly; the tie arrays serve as its bins
+            int bin, above;
+            fine_kth<NT>(k_eff, gmin, fh, scan_tmp, bcast, for_each, bin, above);
+            st.lo_key = (unsigned)bin;
+            st.width = 0;
+            st.k_rem = k_eff - above;
+        }
     }
     while (st.width > 0 && (st.width > SEL_BITS || st.bin_count > SEL_TIE_CAP))
         radix_refine<NT>(st, gmin, hist, scan_tmp, bcast, for_each);
