@@ -1,5 +1,7 @@
 // attn_gather.cuh -- gathered-KV sparse attention, one warp per
-// (query, KV head, 16-head chunk, split) work item.
+// (query, KV head, 16-head chunk, split) work item, or (CTA-merged form, for
+// launches too small to fill the GPU) one CTA of 8 warps per item whose warps
+// split the item's keys and merge in shared memory.
 //
 // Operation (every page reduces to it once a query's index set is known):
 //   z_j = scale * q.k_j + bias_j over j in S,  o = softmax(z) V,  lse = log sum exp z.
@@ -215,11 +217,13 @@ __device__ __forceinline__ void merge_pieces_half(const float *part_o, const flo
 // KLO: keys are held as a bf16 pair (hi, lo) whose sum carries ~16 mantissa
 // bits; q.k is taken on both halves (used for the NSA compressed keys, which
 // are means and do not fit bf16 exactly).
-// TMAB (NSA selected blocks, head dim 128): the chunk's 16 consecutive rows of
-// a block arrive by TMA box loads (kmap / vmap: [B*Lk rows, Hkv, D], box = 64
-// columns x 1 head x 16 rows, 128-byte swizzle) issued by lane 0, completion
-// on a per-warp mbarrier; a K (or V) chunk is then two 64-column halves of
-// 16 rows x 128 B instead of 16 rows x 256 B.
+// TMAB (NSA selected blocks, head dim 128; opt-in, the row gather measured
+// faster): the chunk's 16 consecutive rows of a block arrive by TMA box loads
+// (kmap / vmap: [B*Lk rows, Hkv, D], box = 64 columns x 1 head x 16 rows,
+// 128-byte swizzle) issued by lane 0, completion on a per-warp mbarrier; a K
+// (or V) chunk is then two 64-column halves of 16 rows x 128 B instead of 16
+// rows x 256 B.
+// CTAM: the CTA-merged form above (explicit lists only).
 template <int D, int STAGES, int SRC, bool BIAS, bool KLO = false, int NK = 32, int NW = 4, bool TMAB = false,
           bool CTAM = false>
 __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams p, const __grid_constant__ CUtensorMap kmap,

@@ -290,7 +290,8 @@ static int launch_gather_t(const GatherParams &p, cudaStream_t st) {
         }
     }
     if constexpr (SRC == KS_BLOCKS && D == 128 && !BIAS && !KLO) {
-        // NSA selected blocks: 16-row chunks of a block by TMA box loads
+        // NSA selected blocks: 16-row chunks of a block by TMA box loads (opt-in,
+        // SA_GATHER_TMA=1; by default the row gather below)
         if (p.block % 16 == 0 && (long long)p.B * p.Lk < INT_MAX && items >= (long long)sm_count() * SA_ATTN_NW &&
             gather_tma_allowed()) {
             CUtensorMap km, vm;
