@@ -603,21 +603,25 @@ __global__ void __launch_bounds__(NW * 32) gather_attn_kernel(const GatherParams
                     mx1 = fmaxf(mx1, fmaxf(sc[nt][2], sc[nt][3]));
                 }
             }
-            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
             // m0 / m1 and everything below are in the scaled log2 domain.
             // m0 / m1 are reference maxima, not running maxima: they move
             // (and the accumulators are rescaled) only when some row's chunk
             // maximum exceeds its reference by more than kLazy, so weights
             // 2^(x - m) stay below 2^kLazy (exact in bf16 up to its usual
             // rounding, no overflow in fp32 sums) and most chunks skip the
-            // rescale.  softmax is the same for any reference value.
+            // rescale.  softmax is the same for any reference value.  The
+            // test needs no row maximum: a row's maximum exceeds m + kLazy iff
+            // one of its four lanes' partial maxima does, so the quad
+            // shuffles run only when the reference moves.
             constexpr float kOne = 1.f, kLazy = 8.f;
             const float xs = RAW ? sl2 : kOne;                 // factor still to apply to sc
-            const float cm0 = RAW ? mx0 * sl2 : mx0, cm1 = RAW ? mx1 * sl2 : mx1;
-            if (__any_sync(0xffffffffu, cm0 > m0 + kLazy || cm1 > m1 + kLazy)) {   // warp-uniform
+            if (__any_sync(0xffffffffu, (RAW ? mx0 * sl2 : mx0) > m0 + kLazy ||
+                                            (RAW ? mx1 * sl2 : mx1) > m1 + kLazy)) {   // warp-uniform
+                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+                const float cm0 = RAW ? mx0 * sl2 : mx0, cm1 = RAW ? mx1 * sl2 : mx1;
                 const float mn0 = fmaxf(m0, cm0), mn1 = fmaxf(m1, cm1);
                 const float al0 = m0 == -INFINITY ? 0.f : ex2_fast(m0 - mn0);
                 const float al1 = m1 == -INFINITY ? 0.f : ex2_fast(m1 - mn1);
