@@ -27,7 +27,34 @@ __global__ void __launch_bounds__(COMBINE_ROWS * 32) lse_combine_kernel(const fl
 #pragma unroll
     for (int i = 0; i < PER; ++i) acc[i] = 0.f;
     float den = 0.f, m = -INFINITY;
-    if (n_split <= 32) {
+    constexpr int PRE = 8;                                    // pieces whose rows load with the LSEs
+    if (n_split <= PRE) {
+        // few pieces (decode): every piece's slice of the row is loaded
+        // together with the LSEs, so the merge costs one memory latency
+        float2 x[PRE][PER / 2];
+        const float lsl = lane < n_split ? __ldcg(part_lse + lane * rows + row) : -INFINITY;
+#pragma unroll
+        for (int q = 0; q < PRE; ++q)
+#pragma unroll
+            for (int i = 0; i < PER / 2; ++i)
+                x[q][i] = q < n_split ? __ldcg(reinterpret_cast<const float2 *>(part_o + ((long long)q * rows + row) * D +
+                                                                                 lane * PER) + i)
+                                      : make_float2(0.f, 0.f);
+        m = warp_max(lsl);
+        if (m != -INFINITY) {
+            const float fl = lsl == -INFINITY ? 0.f : exp2f((lsl - m) * kLog2e);
+            den = warp_sum(fl);
+#pragma unroll
+            for (int q = 0; q < PRE; ++q) {
+                const float f = __shfl_sync(0xffffffffu, fl, q);   // 0 for q >= n_split
+#pragma unroll
+                for (int i = 0; i < PER / 2; ++i) {
+                    acc[2 * i] += f != 0.f ? f * x[q][i].x : 0.f;
+                    acc[2 * i + 1] += f != 0.f ? f * x[q][i].y : 0.f;
+                }
+            }
+        }
+    } else if (n_split <= 32) {
         // lane s holds piece s's LSE; the pieces' partial rows are then read
         // with independent (unrolled) loads
         const float lsl = lane < n_split ? part_lse[lane * rows + row] : -INFINITY;
