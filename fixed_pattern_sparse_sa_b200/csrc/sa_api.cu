@@ -919,6 +919,8 @@ static int launch_select_nt(const IdxParams &p, int words, cudaStream_t st) {
 
 template <int DI>
 static int launch_select_t(const IdxParams &p, int words, cudaStream_t st) {
+    // few rows (decode): 1024-thread CTAs (measured faster than 512 or 256
+    // threads for 32 rows of 131072 candidates)
     if ((long long)p.B * p.Rt <= sm_count()) return launch_select_nt<DI, 1024>(p, words, st);
     return launch_select_nt<DI, SEL_THREADS>(p, words, st);
 }
