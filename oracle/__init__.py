@@ -65,11 +65,13 @@ def _load():
             lib.oracle_lse_combine.argtypes = [P, P, I, I, I, P, P]
             lib.oracle_sparse_attn_bwd.argtypes = [P, P, P, P, I, I, I, I, I, I, I, P, I, I, D, P, P, P]
             lib.oracle_nsa_compress.argtypes = [P, P, I, I, I, I, I, I, P, P]
+            lib.oracle_nsa_bwd.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, I, D,
+                                           P, P, P, P]
             lib.oracle_nsa_fwd.argtypes = [P, P, P, P, I, I, I, I, I, I, I, I, I, I, D,
                                            P, I, P, P, P, P, P, P]
             for name in ("oracle_indexer_scores", "oracle_indexer_topk",
                          "oracle_sparse_attn", "oracle_sparse_attn_bwd", "oracle_lse_combine",
-                         "oracle_nsa_compress", "oracle_nsa_fwd"):
+                         "oracle_nsa_compress", "oracle_nsa_fwd", "oracle_nsa_bwd"):
                 getattr(lib, name).restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -294,6 +296,32 @@ def nsa_fwd(q, k, v, gates, cmp_len, cmp_stride, sel_block, sel_topk, window,
                               window, float(scale), _ptr(r), n, _ptr(so), _ptr(out),
                               _ptr(ob), _ptr(lb), _ptr(si), _ptr(imp)), "nsa_fwd")
     return {"out": out, "o_branch": ob, "lse_branch": lb, "sel_idx": si, "imp": imp}
+
+
+def nsa_bwd(q, k, v, gates, dout, sel_idx, cmp_len, cmp_stride, sel_block, sel_topk,
+            window, scale=None):
+    """fp64 NSA backward (Native Sparse Attention page) with the block choice
+    sel_idx [B*T, Hkv, sel_topk] (the forward's) held fixed.
+
+    Returns dict: dq [B,T,Hq,d], dk / dv [B,T,Hkv,d], dgates [B,T,Hq,3]
+    (gradient with respect to the post-sigmoid gate values).
+    """
+    lib = _load()
+    B, T, Hq, d = q.shape
+    Hkv = k.shape[2]
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    si = _np(sel_idx, np.int32).reshape(B * T, Hkv, sel_topk)
+    dq = np.empty((B, T, Hq, d), dtype=np.float64)
+    dk = np.empty((B, T, Hkv, d), dtype=np.float64)
+    dv = np.empty((B, T, Hkv, d), dtype=np.float64)
+    dg = np.empty((B, T, Hq, 3), dtype=np.float64)
+    _check(lib.oracle_nsa_bwd(_ptr(_np(q, np.uint16)), _ptr(_np(k, np.uint16)),
+                              _ptr(_np(v, np.uint16)), _ptr(_np(gates, np.float32)),
+                              _ptr(_np(dout, np.uint16)), _ptr(si), B, T, Hq, Hkv, d,
+                              cmp_len, cmp_stride, sel_block, sel_topk, window, float(scale),
+                              _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg)), "nsa_bwd")
+    return {"dq": dq, "dk": dk, "dv": dv, "dgates": dg}
 
 
 def dsa_layers(pattern, layers, topk, window=0, q_pos0=None, scale=None):

@@ -659,3 +659,174 @@ int oracle_nsa_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v,
     free(vc);
     return status;
 }
+
+/*
+ * Backward of one softmax branch for one query vector (the gradient of
+ * attend_f64's output o for an upstream gradient dob):
+ *   dP_e = dob . v_e,   D = sum_e p_e dP_e,   dS_e = p_e (dP_e - D)
+ *   dq += scale sum_e dS_e k_e,   dk_e += scale dS_e q,   dv_e += p_e dob
+ * p holds the branch's probabilities; dk/dv rows are shared between query
+ * rows, so their updates are atomic.
+ */
+static void attend_bwd_f64(const double *qv, const double *dob, int64_t d, double scale,
+                           const double *const *krows, const double *const *vrows,
+                           const double *p, int64_t n, double *dq,
+                           double *const *dkrows, double *const *dvrows)
+{
+    double D = 0.0;
+    for (int64_t e = 0; e < n; ++e) {
+        double x = 0.0;
+        for (int64_t c = 0; c < d; ++c) x += dob[c] * vrows[e][c];
+        D += p[e] * x;
+    }
+    for (int64_t e = 0; e < n; ++e) {
+        double x = 0.0;
+        for (int64_t c = 0; c < d; ++c) x += dob[c] * vrows[e][c];
+        const double ds = p[e] * (x - D);
+        for (int64_t c = 0; c < d; ++c) {
+            dq[c] += scale * ds * krows[e][c];
+            const double a = scale * ds * qv[c];
+            const double bv = p[e] * dob[c];
+#pragma omp atomic
+            dkrows[e][c] += a;
+#pragma omp atomic
+            dvrows[e][c] += bv;
+        }
+    }
+}
+
+/*
+ * NSA backward (Native Sparse Attention page, "Puntos Clave": the method is
+ * trained natively and its backward pass is accelerated).  The gradient of
+ * oracle_nsa_fwd's out for an upstream gradient dout, with the block choice
+ * sel (the forward's sel_idx, [B*T, Hkv, sel_topk]) held fixed: the choice
+ * is piecewise constant in the inputs, so no gradient flows through the
+ * importance or the top-k.  Per row and head, for branch br with gate g_br
+ * (the post-sigmoid value the forward multiplied by):
+ *   dgates[br] = dout . o_br,   the branch's upstream gradient is g_br dout,
+ * pushed through that branch's softmax (attend_bwd_f64).  The compressed
+ * branch's key gradients land on the compressed rows Kc_i, Vc_i; since
+ * Kc_i is the mean of K[i*stride .. i*stride+len-1], each of those rows
+ * then receives dKc_i / len (likewise V).
+ * Outputs: dq [B*T,Hq,d], dk/dv [B,T,Hkv,d], dgates [B*T,Hq,3], fp64.
+ */
+int oracle_nsa_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                   const float *gates, const uint16_t *dout, const int32_t *sel,
+                   int64_t B, int64_t T, int64_t Hq, int64_t Hkv, int64_t d,
+                   int64_t cmp_len, int64_t cmp_stride, int64_t sel_block,
+                   int64_t sel_topk, int64_t window, double scale,
+                   double *dq, double *dk, double *dv, double *dgates)
+{
+    if (B <= 0 || T <= 0 || Hq <= 0 || Hkv <= 0 || d <= 0 || Hq % Hkv != 0 ||
+        cmp_len <= 0 || cmp_stride <= 0 || sel_block <= 0 || sel_topk <= 0 || window <= 0)
+        return OR_BAD_ARG;
+    const int64_t G = Hq / Hkv;
+    const int64_t nc = nsa_n_cmp(T, cmp_len, cmp_stride);
+    const int64_t nb = (T + sel_block - 1) / sel_block;
+    const int64_t ncs = nc > 0 ? nc : 1;
+    double *kc = (double *)malloc(sizeof(double) * (size_t)(B * ncs * Hkv * d));
+    double *vc = (double *)malloc(sizeof(double) * (size_t)(B * ncs * Hkv * d));
+    double *dkc = (double *)calloc((size_t)(B * ncs * Hkv * d), sizeof(double));
+    double *dvc = (double *)calloc((size_t)(B * ncs * Hkv * d), sizeof(double));
+    double *kraw = (double *)malloc(sizeof(double) * (size_t)(B * T * Hkv * d));
+    double *vraw = (double *)malloc(sizeof(double) * (size_t)(B * T * Hkv * d));
+    if (!kc || !vc || !dkc || !dvc || !kraw || !vraw) {
+        free(kc); free(vc); free(dkc); free(dvc); free(kraw); free(vraw);
+        return OR_BAD_ARG;
+    }
+    if (nc > 0) oracle_nsa_compress(k, v, B, T, Hkv, d, cmp_len, cmp_stride, kc, vc);
+    for (int64_t e = 0; e < B * T * Hkv * d; ++e) {
+        kraw[e] = bf16_to_f64(k[e]);
+        vraw[e] = bf16_to_f64(v[e]);
+        dk[e] = 0.0;
+        dv[e] = 0.0;
+    }
+    int status = OR_OK;
+#pragma omp parallel
+    {
+        int64_t nmax = sel_topk * sel_block;
+        if (window > nmax) nmax = window;
+        if (nc > nmax) nmax = nc;
+        nmax += 1;
+        double *p = (double *)malloc(sizeof(double) * (size_t)nmax);
+        const double **kr = (const double **)malloc(sizeof(double *) * (size_t)nmax);
+        const double **vr = (const double **)malloc(sizeof(double *) * (size_t)nmax);
+        double **dkr = (double **)malloc(sizeof(double *) * (size_t)nmax);
+        double **dvr = (double **)malloc(sizeof(double *) * (size_t)nmax);
+        double *qv = (double *)malloc(sizeof(double) * (size_t)d);
+        double *dov = (double *)malloc(sizeof(double) * (size_t)d);
+        double *dob = (double *)malloc(sizeof(double) * (size_t)d);
+        double *o = (double *)malloc(sizeof(double) * (size_t)d);
+        int ok = p && kr && vr && dkr && dvr && qv && dov && dob && o;
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t r = 0; r < B * T; ++r) {
+            if (!ok) { status = OR_BAD_ARG; continue; }
+            const int64_t b = r / T, t = r % T;
+            int64_t n_vis = 0;
+            while (n_vis < nc && n_vis * cmp_stride + cmp_len - 1 <= t) ++n_vis;
+            for (int64_t h = 0; h < Hq; ++h) {
+                const int64_t g = h / G;
+                for (int64_t c = 0; c < d; ++c) {
+                    qv[c] = bf16_to_f64(q[(r * Hq + h) * d + c]);
+                    dov[c] = bf16_to_f64(dout[(r * Hq + h) * d + c]);
+                }
+                double *dqv = dq + (r * Hq + h) * d;
+                for (int64_t c = 0; c < d; ++c) dqv[c] = 0.0;
+                for (int br = 0; br < 3; ++br) {
+                    /* the branch's key set, as in the forward */
+                    int64_t n = 0;
+                    if (br == 0) {
+                        for (int64_t i = 0; i < n_vis; ++i) {
+                            const int64_t off = ((b * nc + i) * Hkv + g) * d;
+                            kr[n] = kc + off; vr[n] = vc + off;
+                            dkr[n] = dkc + off; dvr[n] = dvc + off; ++n;
+                        }
+                    } else if (br == 1) {
+                        const int32_t *sg = sel + (r * Hkv + g) * sel_topk;
+                        for (int64_t m = 0; m < sel_topk; ++m) {
+                            const int64_t blk = sg[m];
+                            if (blk < 0) continue;
+                            if (blk >= nb) { status = OR_BAD_INDEX; continue; }
+                            for (int64_t j = blk * sel_block; j < (blk + 1) * sel_block && j <= t && j < T; ++j) {
+                                const int64_t off = ((b * T + j) * Hkv + g) * d;
+                                kr[n] = kraw + off; vr[n] = vraw + off;
+                                dkr[n] = dk + off; dvr[n] = dv + off; ++n;
+                            }
+                        }
+                    } else {
+                        const int64_t lo = t - window + 1 > 0 ? t - window + 1 : 0;
+                        for (int64_t j = lo; j <= t; ++j) {
+                            const int64_t off = ((b * T + j) * Hkv + g) * d;
+                            kr[n] = kraw + off; vr[n] = vraw + off;
+                            dkr[n] = dk + off; dvr[n] = dv + off; ++n;
+                        }
+                    }
+                    double lse;
+                    attend_f64(qv, d, scale, kr, vr, n, p, o, &lse);
+                    const double gb = (double)gates[(r * Hq + h) * 3 + br];
+                    double dg = 0.0;
+                    for (int64_t c = 0; c < d; ++c) {
+                        dg += dov[c] * o[c];
+                        dob[c] = gb * dov[c];
+                    }
+                    dgates[(r * Hq + h) * 3 + br] = dg;
+                    if (n > 0) attend_bwd_f64(qv, dob, d, scale, kr, vr, p, n, dqv, dkr, dvr);
+                }
+            }
+        }
+        free(p); free(kr); free(vr); free(dkr); free(dvr); free(qv); free(dov); free(dob); free(o);
+    }
+    /* compressed rows back to the raw rows they average */
+    for (int64_t b = 0; b < B; ++b)
+        for (int64_t i = 0; i < nc; ++i)
+            for (int64_t u = 0; u < cmp_len; ++u) {
+                const int64_t j = i * cmp_stride + u;
+                for (int64_t g = 0; g < Hkv; ++g)
+                    for (int64_t c = 0; c < d; ++c) {
+                        dk[((b * T + j) * Hkv + g) * d + c] += dkc[((b * nc + i) * Hkv + g) * d + c] / (double)cmp_len;
+                        dv[((b * T + j) * Hkv + g) * d + c] += dvc[((b * nc + i) * Hkv + g) * d + c] / (double)cmp_len;
+                    }
+            }
+    free(kc); free(vc); free(dkc); free(dvc); free(kraw); free(vraw);
+    return status;
+}

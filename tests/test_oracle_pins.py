@@ -640,3 +640,105 @@ def test_backward_column_sum_identities():
     np.testing.assert_allclose(dk.sum(axis=1), 0.0, atol=1e-10)
     do = _f64(dout).numpy().reshape(B, T, Hkv, Hq // Hkv, d).sum(axis=(1, 3))
     np.testing.assert_allclose(dv.sum(axis=1), do, atol=1e-10)
+
+
+# ------------------------------------------------------------ NSA backward --
+def _nsa_torch_out(q, k, v, gates, sel, cmp_len, cmp_stride, sel_block, window, scale):
+    """NSA forward as dense masked softmaxes in torch float64, with the block
+    choice sel [B*T, Hkv, topk] fixed; differentiable in q, k, v, gates.
+    Compressed rows come from torch's unfold + mean."""
+    B, T, Hq, d = q.shape
+    Hkv = k.shape[2]
+    G = Hq // Hkv
+    t = torch.arange(T)[:, None]
+    branches = []
+    # compressed branch over mean-pooled rows
+    if T >= cmp_len:
+        kc = k.unfold(1, cmp_len, cmp_stride).mean(-1)
+        vc = v.unfold(1, cmp_len, cmp_stride).mean(-1)
+        i = torch.arange(kc.shape[1])[None, :]
+        m = ((i * cmp_stride + cmp_len - 1) <= t)[None, None].expand(B, Hkv, T, kc.shape[1])
+        branches.append((kc, vc, m))
+    else:
+        branches.append(None)
+    # selected branch: keys of the chosen blocks, j <= t
+    j = torch.arange(T)
+    ms = torch.zeros(B, Hkv, T, T, dtype=torch.bool)
+    s3 = torch.from_numpy(np.asarray(sel)).reshape(B, T, Hkv, -1)
+    for b in range(B):
+        for tt in range(T):
+            for g in range(Hkv):
+                for blk in s3[b, tt, g].tolist():
+                    if blk >= 0:
+                        ms[b, g, tt] |= (j // sel_block == blk) & (j <= tt)
+    branches.append((k, v, ms))
+    mw = ((j[None, :] <= t) & (j[None, :] > t - window))[None, None].expand(B, Hkv, T, T)
+    branches.append((k, v, mw))
+    out = torch.zeros(B, T, Hq, d, dtype=torch.float64)
+    for br, item in enumerate(branches):
+        if item is None:
+            continue
+        kk, vv, m = item
+        qh = q.transpose(1, 2)                                     # [B,Hq,T,d]
+        kh = kk.transpose(1, 2).repeat_interleave(G, dim=1)
+        vh = vv.transpose(1, 2).repeat_interleave(G, dim=1)
+        mh = m.repeat_interleave(G, dim=1)
+        empty = ~mh.any(dim=-1, keepdim=True)
+        z = torch.matmul(qh, kh.transpose(-1, -2)) * scale
+        z = z.masked_fill(~mh & ~empty, float("-inf"))
+        o = torch.matmul(torch.softmax(z, dim=-1), vh).masked_fill(empty, 0.0)
+        out = out + gates[..., br:br + 1] * o.transpose(1, 2)
+    return out
+
+
+def _nsa_bwd_case(T, Hq, Hkv, d, seed, cfg):
+    g = inputs.gen_nsa(1, T, Hq, Hkv, d, seed=seed)
+    gen = torch.Generator().manual_seed(seed + 3)
+    dout = torch.randn(1, T, Hq, d, generator=gen).to(torch.bfloat16)
+    r = oracle.nsa_fwd(g["q"], g["k"], g["v"], g["gates"], **cfg)
+    gr = oracle.nsa_bwd(g["q"], g["k"], g["v"], g["gates"], dout, r["sel_idx"], **cfg)
+    return g, dout, r, gr
+
+
+@pytest.mark.parametrize("T,Hq,Hkv,d,cfg", [
+    (96, 4, 2, 16, NSA_SMALL),
+    (75, 6, 2, 8, dict(cmp_len=8, cmp_stride=4, sel_block=16, sel_topk=2, window=20)),
+    (40, 2, 1, 8, dict(cmp_len=16, cmp_stride=8, sel_block=16, sel_topk=4, window=64)),
+])
+def test_nsa_backward_matches_dense_autograd(T, Hq, Hkv, d, cfg):
+    # the hand-written chain rule (per-branch softmax backward, gate factor,
+    # compressed-row gradients spread back over the rows they average) against
+    # torch autograd of a dense masked formulation of the same forward
+    g, dout, r, gr = _nsa_bwd_case(T, Hq, Hkv, d, 31 + T, cfg)
+    q = _f64(g["q"]).clone().requires_grad_(True)
+    k = _f64(g["k"]).clone().requires_grad_(True)
+    v = _f64(g["v"]).clone().requires_grad_(True)
+    ga = g["gates"].to(torch.float64).clone().requires_grad_(True)
+    out = _nsa_torch_out(q, k, v, ga, r["sel_idx"], cfg["cmp_len"], cfg["cmp_stride"],
+                         cfg["sel_block"], cfg["window"], 1 / math.sqrt(d))
+    np.testing.assert_allclose(out.detach().numpy()[0], r["out"].reshape(T, Hq, d), atol=1e-12)
+    out.backward(_f64(dout))
+    np.testing.assert_allclose(gr["dq"], q.grad.numpy(), atol=1e-10)
+    np.testing.assert_allclose(gr["dk"], k.grad.numpy(), atol=1e-10)
+    np.testing.assert_allclose(gr["dv"], v.grad.numpy(), atol=1e-10)
+    np.testing.assert_allclose(gr["dgates"], ga.grad.numpy(), atol=1e-10)
+
+
+def test_nsa_backward_column_sums():
+    # each branch's dS sums to 0 over its keys, and the compressed rows pass
+    # their gradient back with weights summing to 1, so sum_j dk_j = 0; each
+    # non-empty branch's probabilities sum to 1, so sum_j dv_j is the
+    # gate-weighted dout of the group's heads over the live branches
+    T, Hq, Hkv, d = 96, 4, 2, 16
+    cfg = NSA_SMALL
+    g, dout, r, gr = _nsa_bwd_case(T, Hq, Hkv, d, 41, cfg)
+    np.testing.assert_allclose(gr["dk"].sum(axis=1), 0.0, atol=1e-10)
+    live = np.isfinite(r["lse_branch"])                             # [T,Hq,3]
+    w = (g["gates"].numpy()[0].astype(np.float64) * live).sum(axis=-1)   # [T,Hq]
+    do = _f64(dout).numpy()[0] * w[..., None]
+    expect = do.reshape(T, Hkv, Hq // Hkv, d).sum(axis=(0, 2))
+    np.testing.assert_allclose(gr["dv"].sum(axis=1)[0], expect, atol=1e-10)
+    # the gate gradient is the upstream gradient against each branch output
+    ob = r["o_branch"].reshape(3, T, Hq, d)
+    np.testing.assert_allclose(gr["dgates"][0], np.einsum("thc,bthc->thb", _f64(dout).numpy()[0], ob),
+                               atol=1e-12)
