@@ -171,7 +171,7 @@ def main():
                     help="NSA length for profiling captures of a smaller case (default 65536)")
     ap.add_argument("--workload", default="all",
                     choices=["all", "decode128k", "indexcache_prefill", "hysparse2_prefill", "bwd64k",
-                             "nsa64k", "spatial16k"],
+                             "nsa64k", "nsa_bwd64k", "spatial16k"],
                     help="run only one of the extra measurements (for profiling captures of a "
                          "single workload); prints its numbers alone")
     ap.add_argument("--decode-seq-len", type=int, default=0,
@@ -592,6 +592,33 @@ def extra_measurements(args, dev, torch, api, lib, inputs, flush, world, peaks, 
             "algorithmic_flops": nsa_fl,
             "tensor_frac": round(nsa_fl / (ms / 1e3) / 1e12 / peaks["bf16_tflops"], 4)}
         del gd, g, o
+        torch.cuda.empty_cache()
+    # --- NSA backward 64K (dq, dk, dv, dgates with the forward's block choice) ---
+    if only in (None, "nsa_bwd64k"):
+        w = inputs.WORKLOADS["nsa64k"]
+        if args.nsa_seq_len:
+            w = dataclasses.replace(w, T=int(args.nsa_seq_len))
+        g = inputs.gen_nsa(w.B, w.T, w.Hq, w.Hkv, w.d, seed=0)
+        gd = {k: v.to(dev) for k, v in g.items()}
+        cfg = dict(cmp_len=w.cmp_len, cmp_stride=w.cmp_stride, sel_block=w.sel_block,
+                   sel_topk=w.sel_topk, window=w.window)
+        _, lse3, sel, o3 = api.nsa_fwd_train(gd["q"], gd["k"], gd["v"], gd["gates"], **cfg)
+        dout = (torch.randn((w.B, w.T, w.Hq, w.d), generator=torch.Generator().manual_seed(302))
+                * 0.1).to(device=dev, dtype=torch.bfloat16)
+
+        def nbstep():
+            api.nsa_bwd(gd["q"], gd["k"], gd["v"], gd["gates"], dout, o3, lse3, sel, **cfg)
+        times = timed_steps(nbstep, 2, args.warmup, flush, dev, torch)
+        ms = max_over_ranks(sum(times), dev, torch, dist) / len(times)
+        # 10 d per (query, head, key) over the three branches, 2.5 x the forward's 4 d
+        bfl = 2.5 * nsa_flops(w, sel, torch)
+        res["nsa_bwd64k" if w.T == 65536 else f"nsa_bwd{w.T // 1024}k"] = {
+            "ms_per_step": round(ms, 3), "tflops": round(bfl / (ms / 1e3) / 1e12, 2),
+            "algorithmic_flops": bfl,
+            "tensor_frac": round(bfl / (ms / 1e3) / 1e12 / peaks["bf16_tflops"], 4),
+            "note": f"nsa_bwd, 1 x {w.T} tokens, 64 q heads / 4 kv heads, d=128; "
+                    "fp32 dq/dk/dv/dgates"}
+        del g, gd, lse3, sel, o3, dout
         torch.cuda.empty_cache()
     # --- fixed graph 16K with coordinate bias ---
     if only in (None, "spatial16k"):

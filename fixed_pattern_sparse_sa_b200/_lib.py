@@ -15,7 +15,8 @@ EXPORTS = (
     "sa_sparse_attn_fwd_split_static",
     "sa_sparse_attn_bwd_workspace_size", "sa_sparse_attn_bwd",
     "sa_lse_combine",
-    "sa_nsa_workspace_size", "sa_nsa_fwd",
+    "sa_nsa_workspace_size", "sa_nsa_fwd", "sa_nsa_fwd_train",
+    "sa_nsa_bwd_workspace_size", "sa_nsa_bwd",
     "sa_dsa_decode_layers_workspace_size", "sa_dsa_decode_layers",
     "sa_check_device_status", "sa_last_error_string", "sa_status_string",
     "sa_version", "sa_launch_counter",
@@ -78,6 +79,10 @@ def load() -> ctypes.CDLL:
             "sa_sparse_attn_bwd": (I, [P, P, P, P, P, P, I, I, I, I, I, I, I64, P, I, I, F, P, P, P, P, SZ, P]),
             "sa_nsa_workspace_size": (SZ, [I, I, I, I, I, I, I, I, I]),
             "sa_nsa_fwd": (I, [P, P, P, P, I, I, I, I, I, I, I, I, I, I, F, P, P, P, P, SZ, P]),
+            "sa_nsa_fwd_train": (I, [P, P, P, P, I, I, I, I, I, I, I, I, I, I, F, P, P, P, P, P, SZ, P]),
+            "sa_nsa_bwd_workspace_size": (SZ, [I, I, I, I, I, I, I]),
+            "sa_nsa_bwd": (I, [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, I, F, P, P, P, P,
+                               P, SZ, P]),
             "sa_dsa_decode_layers_workspace_size": (SZ, [I, I, I, I, I, I, I, I, I, I]),
             "sa_dsa_decode_layers": (I, [ctypes.c_char_p, I, P, I, I, I, I, I, I, I, I, I64,
                                          I, I, F, I, P, P, SZ, P]),

@@ -373,6 +373,77 @@ def nsa_fwd(q, k, v, gates, cmp_len: int, cmp_stride: int, sel_block: int, sel_t
     return out, lse3, sel
 
 
+def nsa_fwd_train(q, k, v, gates, cmp_len: int, cmp_stride: int, sel_block: int, sel_topk: int,
+                  window: int, scale: Optional[float] = None):
+    """NSA forward that also returns what the backward needs (sa_nsa_fwd_train).
+
+    Returns (out bf16 [B,T,Hq,d], lse_branches fp32 [B,T,Hq,3],
+    sel_idx int32 [B,T,Hkv,sel_topk], o_branches fp32 [3,B,T,Hq,d]).
+    """
+    lib = _lib.load()
+    dev = q.device
+    _need(q, "q", torch.bfloat16, dev, 4)
+    _need(k, "k", torch.bfloat16, dev, 4)
+    _need(v, "v", torch.bfloat16, dev, 4)
+    _need(gates, "gates", torch.float32, dev, 4)
+    B, T, Hq, d = q.shape
+    Hkv = k.shape[2]
+    if k.shape != (B, T, Hkv, d) or v.shape != k.shape or gates.shape != (B, T, Hq, 3):
+        raise ValueError("nsa_fwd_train: shape mismatch")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    out = torch.empty((B, T, Hq, d), dtype=torch.bfloat16, device=dev)
+    lse3 = torch.empty((B, T, Hq, 3), dtype=torch.float32, device=dev)
+    sel = torch.empty((B, T, Hkv, sel_topk), dtype=torch.int32, device=dev)
+    o3 = torch.empty((3, B, T, Hq, d), dtype=torch.float32, device=dev)
+    nbytes = lib.sa_nsa_workspace_size(B, T, Hq, Hkv, d, cmp_len, cmp_stride, sel_block, sel_topk)
+    ws = _workspace(nbytes, dev)
+    with torch.cuda.device(dev):
+        check(lib.sa_nsa_fwd_train(_ptr(q), _ptr(k), _ptr(v), _ptr(gates), B, T, Hq, Hkv, d, cmp_len,
+                                   cmp_stride, sel_block, sel_topk, window, float(scale), _ptr(out),
+                                   _ptr(lse3), _ptr(sel), _ptr(o3), _ptr(ws), nbytes, _stream(dev)),
+              "sa_nsa_fwd_train")
+    return out, lse3, sel, o3
+
+
+def nsa_bwd(q, k, v, gates, dout, o_branches, lse_branches, sel_idx, cmp_len: int, cmp_stride: int,
+            sel_block: int, sel_topk: int, window: int, scale: Optional[float] = None):
+    """NSA backward (sa_nsa_bwd) with the forward's block choice held fixed.
+
+    o_branches, lse_branches and sel_idx are nsa_fwd_train's.  Returns
+    (dq fp32 [B,T,Hq,d], dk fp32 [B,T,Hkv,d], dv fp32 [B,T,Hkv,d],
+    dgates fp32 [B,T,Hq,3]).
+    """
+    lib = _lib.load()
+    dev = q.device
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (dout, "dout")):
+        _need(t, n, torch.bfloat16, dev, 4)
+    _need(gates, "gates", torch.float32, dev, 4)
+    _need(o_branches, "o_branches", torch.float32, dev, 5)
+    _need(lse_branches, "lse_branches", torch.float32, dev, 4)
+    _need(sel_idx, "sel_idx", torch.int32, dev, 4)
+    B, T, Hq, d = q.shape
+    Hkv = k.shape[2]
+    if (k.shape != (B, T, Hkv, d) or v.shape != k.shape or dout.shape != q.shape
+            or gates.shape != (B, T, Hq, 3) or o_branches.shape != (3, B, T, Hq, d)
+            or lse_branches.shape != (B, T, Hq, 3) or sel_idx.shape != (B, T, Hkv, sel_topk)):
+        raise ValueError("nsa_bwd: shape mismatch")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = torch.empty((B, T, Hq, d), dtype=torch.float32, device=dev)
+    dk = torch.empty((B, T, Hkv, d), dtype=torch.float32, device=dev)
+    dv = torch.empty((B, T, Hkv, d), dtype=torch.float32, device=dev)
+    dg = torch.empty((B, T, Hq, 3), dtype=torch.float32, device=dev)
+    nbytes = lib.sa_nsa_bwd_workspace_size(B, T, Hq, Hkv, d, cmp_len, cmp_stride)
+    ws = _workspace(nbytes, dev)
+    with torch.cuda.device(dev):
+        check(lib.sa_nsa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(gates), _ptr(dout), _ptr(o_branches),
+                             _ptr(lse_branches), _ptr(sel_idx), B, T, Hq, Hkv, d, cmp_len, cmp_stride,
+                             sel_block, sel_topk, window, float(scale), _ptr(dq), _ptr(dk), _ptr(dv),
+                             _ptr(dg), _ptr(ws), nbytes, _stream(dev)), "sa_nsa_bwd")
+    return dq, dk, dv, dg
+
+
 # --------------------------------------------------------------- IndexCache --
 def dsa_decode_layers(pattern: str, layers, topk: int, window: int = 0, n_split: int = 1,
                       q_pos0: Optional[int] = None, scale: Optional[float] = None,

@@ -18,17 +18,35 @@
 // dV = P^T dO for the chunk's 16 keys, which are added to the fp32 dk / dv
 // with vector reductions (a key selected by several queries collects all of
 // their contributions).  D comes from a first pass (attn_bwd_prep_kernel).
+//
+// The same kernel runs the three NSA branches (Native Sparse Attention page,
+// "Puntos Clave": natively trainable, with a faster backward pass).  The key
+// source is a template parameter: explicit lists (BW_LIST), the keys of
+// selected blocks masked to j <= t (BW_BLOCKS), or a contiguous range per
+// query (BW_RANGE: the sliding window, or the compressed rows visible to
+// t).  Compressed keys come as a bf16 hi/lo pair (HILO) as in the forward.
+// A per-row factor (the branch gate) scales the upstream gradient, the LSE
+// is read with a stride (the forward stores the three branches' LSEs side by
+// side), and dq can accumulate over the branches' launches.
 #pragma once
 
 #include "attn_gather.cuh"
 
 namespace sa {
 
+enum { BW_LIST = 0, BW_BLOCKS = 1, BW_RANGE = 2 };
+
 struct BwdParams {
     const __nv_bfloat16 *q, *k, *v, *o, *dout;   // q/o/dout [B,Tq,Hq,D], k/v [B,L,Hkv,D]
-    const float *lse;                            // [B,Tq,Hq] natural log (forward)
-    const int32_t *idx;                          // [B,Tq,idx_heads,K]
+    const __nv_bfloat16 *klo;                    // HILO: low halves of the keys
+    const float *lse;                            // [rows * lse_stride] natural log (forward)
+    const int32_t *idx;                          // [B,Tq,idx_heads,K] keys (BW_LIST) or blocks (BW_BLOCKS)
+    const float *gate;                           // nullable: factor on dO, gate[row * gate_stride]
     int B, Tq, L, Hq, Hkv, G, idx_heads, K;
+    int lse_stride, gate_stride;
+    int block, block_shift;                      // BW_BLOCKS: keys per block, log2 or -1
+    int window, cmp_len, cmp_stride;             // BW_RANGE: window > 0, else compressed rows
+    int dq_accum;                                // add to dq instead of writing it
     long long q_pos0;
     float scale, scale_log2;
     float *Dt;                                   // [B,Tq,Hq] dO . O
@@ -60,9 +78,9 @@ __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const BwdParams p, l
 // Shared memory of one warp: K/V stages and their keys, the Q and dO tiles of
 // the 16 heads and two 16 x 16 transpose tiles, rounded to 1 KB so that every
 // warp's region (and each tile in it) stays 16-byte aligned.
-template <int D>
+template <int D, bool HILO = false>
 __host__ __device__ constexpr int attn_bwd_warp_bytes() {
-    return (2 * (2 * 16 * D * 2 + 16 * 4) + 2 * 16 * D * 2 + 2 * 16 * 32 + 1023) / 1024 * 1024;
+    return (2 * ((HILO ? 3 : 2) * 16 * D * 2 + 16 * 4) + 2 * 16 * D * 2 + 2 * 16 * 32 + 1023) / 1024 * 1024;
 }
 
 __device__ __forceinline__ void red_add2(float *addr, float a, float b) {
@@ -86,11 +104,12 @@ __device__ __forceinline__ void ldsm_tile16(unsigned (&a)[4], const unsigned cha
     }
 }
 
-template <int D, int NW>
+template <int D, int NW, int SRC = BW_LIST, bool HILO = false>
 __global__ void __launch_bounds__(NW * 32) attn_bwd_kernel(const BwdParams p) {
     grid_dependency_sync();
     constexpr int NK = 16;                  // keys per chunk
     constexpr int STAGES = 2;
+    constexpr int NARR = HILO ? 3 : 2;      // K (+ K low half) and V per stage
     constexpr int ROWB = D * 2;
     constexpr int UNITS = ROWB / 16;
     constexpr int CH = NK * ROWB;           // one K (or V) chunk
@@ -98,7 +117,7 @@ __global__ void __launch_bounds__(NW * 32) attn_bwd_kernel(const BwdParams p) {
     constexpr int NT_D = D / 8;
     constexpr int CP_ITERS = NK * UNITS / 32;
     constexpr int QT = 16 * ROWB;           // Q (or dO) tile of the 16 heads
-    constexpr int WSM = attn_bwd_warp_bytes<D>();
+    constexpr int WSM = attn_bwd_warp_bytes<D, HILO>();
 
     extern __shared__ __align__(1024) unsigned char smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -107,7 +126,7 @@ __global__ void __launch_bounds__(NW * 32) attn_bwd_kernel(const BwdParams p) {
     unsigned char *do_s = q_s + QT;
     unsigned char *tp_s = do_s + QT;                // 16 x 16 bf16 tiles: dS, P
     unsigned char *kv_s = tp_s + 2 * 16 * 32;
-    int *keys_s = reinterpret_cast<int *>(kv_s + STAGES * 2 * CH);
+    int *keys_s = reinterpret_cast<int *>(kv_s + STAGES * NARR * CH);
 
     const int n_hchunk = (p.G + 15) / 16;
     const long long n_items = (long long)p.B * p.Tq * p.Hkv * n_hchunk;
@@ -137,29 +156,65 @@ __global__ void __launch_bounds__(NW * 32) attn_bwd_kernel(const BwdParams p) {
         cp_async16(do_s + r * ROWB + sw, ok ? p.dout + base : p.dout, ok ? 16 : 0);
     }
     cp_async_commit();
-    const float lse0 = v0 ? p.lse[row0] * kLog2e : 0.f, lse1 = v1 ? p.lse[row1] * kLog2e : 0.f;
+    const float lse0 = v0 ? p.lse[row0 * p.lse_stride] * kLog2e : 0.f;
+    const float lse1 = v1 ? p.lse[row1 * p.lse_stride] * kLog2e : 0.f;
     const float D0 = v0 ? p.Dt[row0] : 0.f, D1 = v1 ? p.Dt[row1] : 0.f;
+    const float gs0 = (p.gate && v0) ? p.gate[row0 * p.gate_stride] : 1.f;
+    const float gs1 = (p.gate && v1) ? p.gate[row1 * p.gate_stride] : 1.f;
     // a row whose forward set was empty has lse = -inf: no gradient
     const bool live0 = v0 && lse0 != -INFINITY, live1 = v1 && lse1 != -INFINITY;
 
-    const int32_t *list = p.idx + ((long long)(b * p.Tq + t) * p.idx_heads + (p.idx_heads == 1 ? 0 : g)) * p.K;
-    const int n_chunks = (p.K + NK - 1) / NK;
+    // the query's key entries: list entries, block entries (K blocks x
+    // block keys), or a range [lo, lo + n_e)
+    const int32_t *list = SRC == BW_RANGE ? nullptr
+        : p.idx + ((long long)(b * p.Tq + t) * p.idx_heads + (p.idx_heads == 1 ? 0 : g)) * p.K;
+    int n_e = 0;
+    long long lo = 0;
+    if constexpr (SRC == BW_LIST) {
+        n_e = p.K;
+    } else if constexpr (SRC == BW_BLOCKS) {
+        n_e = p.K * p.block;
+    } else {
+        if (p.window > 0) {
+            lo = pos - p.window + 1 > 0 ? pos - p.window + 1 : 0;
+            n_e = (int)(pos + 1 - lo);
+        } else {
+            const long long nv = pos >= p.cmp_len - 1 ? (pos - p.cmp_len + 1) / p.cmp_stride + 1 : 0;
+            n_e = (int)(nv < p.L ? nv : p.L);
+        }
+    }
+    const int n_chunks = (n_e + NK - 1) / NK;
     const __nv_bfloat16 *kb = p.k + ((long long)b * p.L * p.Hkv + g) * D;
+    const __nv_bfloat16 *klb = HILO ? p.klo + ((long long)b * p.L * p.Hkv + g) * D : nullptr;
     const __nv_bfloat16 *vb = p.v + ((long long)b * p.L * p.Hkv + g) * D;
     const long long rstride = (long long)p.Hkv * D;
 
     auto issue = [&](int ci) {
         const int st = ci % STAGES;
-        unsigned char *ks_ = kv_s + st * 2 * CH;
+        unsigned char *ks_ = kv_s + st * NARR * CH;
         unsigned char *vs_ = ks_ + CH;
+        unsigned char *ls_ = vs_ + CH;          // HILO: K low halves
         int j = -1;
         if (ci < n_chunks && lane < NK) {
             const int e = ci * NK + lane;
-            if (e < p.K) {
-                const int raw = __ldg(list + e);
-                if (raw >= 0) {
-                    if (raw >= p.L || (long long)raw > pos) raise_error(p.err, ERR_BAD_INDEX);
-                    else j = raw;
+            if (e < n_e) {
+                if constexpr (SRC == BW_LIST) {
+                    const int raw = __ldg(list + e);
+                    if (raw >= 0) {
+                        if (raw >= p.L || (long long)raw > pos) raise_error(p.err, ERR_BAD_INDEX);
+                        else j = raw;
+                    }
+                } else if constexpr (SRC == BW_BLOCKS) {
+                    const int bi = p.block_shift >= 0 ? e >> p.block_shift : e / p.block;
+                    const int blk = __ldg(list + bi);
+                    if (blk >= 0) {
+                        const long long j0 = (long long)blk * p.block;
+                        const long long jj = j0 + (e - bi * p.block);
+                        if (j0 >= p.L) raise_error(p.err, ERR_BAD_INDEX);
+                        else if (jj <= pos && jj < p.L) j = (int)jj;
+                    }
+                } else {
+                    j = (int)(lo + e);
                 }
             }
             keys_s[st * NK + lane] = j;
@@ -174,6 +229,7 @@ __global__ void __launch_bounds__(NW * 32) attn_bwd_kernel(const BwdParams p) {
                 const int sw = (u ^ (rr & 7)) * 16;
                 cp_async16(ks_ + rr * ROWB + sw, kb + off, jr >= 0 ? 16 : 0);
                 cp_async16(vs_ + rr * ROWB + sw, vb + off, jr >= 0 ? 16 : 0);
+                if constexpr (HILO) cp_async16(ls_ + rr * ROWB + sw, klb + off, jr >= 0 ? 16 : 0);
             }
         }
         cp_async_commit();
@@ -189,8 +245,9 @@ __global__ void __launch_bounds__(NW * 32) attn_bwd_kernel(const BwdParams p) {
         cp_async_wait<1>();
         __syncwarp();
         const int st = ci % STAGES;
-        const unsigned char *ks_ = kv_s + st * 2 * CH;
+        const unsigned char *ks_ = kv_s + st * NARR * CH;
         const unsigned char *vs_ = ks_ + CH;
+        const unsigned char *ls_ = vs_ + CH;
         const int jl = lane < NK ? keys_s[st * NK + lane] : -1;
         const unsigned vmask = __ballot_sync(0xffffffffu, jl >= 0);
         if (vmask != 0u) {
@@ -214,6 +271,11 @@ __global__ void __launch_bounds__(NW * 32) attn_bwd_kernel(const BwdParams p) {
                 ldsm_x4(b0, b1, b2, b3, ks_ + key * ROWB + ((unit ^ (key & 7)) * 16));
                 mma_bf16_16816(sc[0], qa, b0, b1);
                 mma_bf16_16816(sc[1], qa, b2, b3);
+                if constexpr (HILO) {
+                    ldsm_x4(b0, b1, b2, b3, ls_ + key * ROWB + ((unit ^ (key & 7)) * 16));
+                    mma_bf16_16816(sc[0], qa, b0, b1);
+                    mma_bf16_16816(sc[1], qa, b2, b3);
+                }
                 ldsm_x4(b0, b1, b2, b3, vs_ + key * ROWB + ((unit ^ (key & 7)) * 16));
                 mma_bf16_16816(dp[0], da, b0, b1);
                 mma_bf16_16816(dp[1], da, b2, b3);
@@ -228,8 +290,9 @@ __global__ void __launch_bounds__(NW * 32) attn_bwd_kernel(const BwdParams p) {
                     const bool hi = e >> 1;
                     const bool ok = ((vmask >> kk) & 1u) && (hi ? live1 : live0);
                     const float pv = ok ? exp2f(sc[nt][e] * p.scale_log2 - (hi ? lse1 : lse0)) : 0.f;
-                    pr[nt][e] = pv;
-                    ds[nt][e] = pv * (dp[nt][e] - (hi ? D1 : D0));
+                    const float gv = pv * (hi ? gs1 : gs0);
+                    pr[nt][e] = gv;
+                    ds[nt][e] = gv * (dp[nt][e] - (hi ? D1 : D0));
                 }
             }
             // dS and P as bf16 A fragments (rows = heads, k = keys)
@@ -248,6 +311,11 @@ __global__ void __launch_bounds__(NW * 32) attn_bwd_kernel(const BwdParams p) {
                 ldsm_x4_t(b0, b1, b2, b3, ks_ + key * ROWB + ((unit ^ (key & 7)) * 16));
                 mma_bf16_16816(dqa[2 * dpi], dsa, b0, b1);
                 mma_bf16_16816(dqa[2 * dpi + 1], dsa, b2, b3);
+                if constexpr (HILO) {
+                    ldsm_x4_t(b0, b1, b2, b3, ls_ + key * ROWB + ((unit ^ (key & 7)) * 16));
+                    mma_bf16_16816(dqa[2 * dpi], dsa, b0, b1);
+                    mma_bf16_16816(dqa[2 * dpi + 1], dsa, b2, b3);
+                }
             }
             // dS and P tiles (row = head, col = key) for the transposed products
             {
@@ -304,14 +372,93 @@ __global__ void __launch_bounds__(NW * 32) attn_bwd_kernel(const BwdParams p) {
 #pragma unroll
     for (int nt = 0; nt < NT_D; ++nt) {
         const int col = nt * 8 + 2 * qc;
-        if (v0) *reinterpret_cast<float2 *>(p.dq + row0 * D + col) = make_float2(dqa[nt][0] * p.scale, dqa[nt][1] * p.scale);
-        if (v1) *reinterpret_cast<float2 *>(p.dq + row1 * D + col) = make_float2(dqa[nt][2] * p.scale, dqa[nt][3] * p.scale);
+        float2 a0 = make_float2(dqa[nt][0] * p.scale, dqa[nt][1] * p.scale);
+        float2 a1 = make_float2(dqa[nt][2] * p.scale, dqa[nt][3] * p.scale);
+        float2 *q0 = reinterpret_cast<float2 *>(p.dq + row0 * D + col);
+        float2 *q1 = reinterpret_cast<float2 *>(p.dq + row1 * D + col);
+        if (p.dq_accum) {
+            if (v0) { const float2 o = *q0; a0.x += o.x; a0.y += o.y; }
+            if (v1) { const float2 o = *q1; a1.x += o.x; a1.y += o.y; }
+        }
+        if (v0) *q0 = a0;
+        if (v1) *q1 = a1;
     }
 }
 
-template <int D, int NW>
+template <int D, int NW, bool HILO = false>
 constexpr int attn_bwd_smem_bytes() {
-    return NW * attn_bwd_warp_bytes<D>();
+    return NW * attn_bwd_warp_bytes<D, HILO>();
+}
+
+// NSA: per row, r_b = dO . O_b for the three branch outputs (fp32, [3, rows,
+// D]).  r_b is the branch's D term before the gate factor and the gradient
+// of the output with respect to gate b.  One warp per row.
+template <int D>
+__global__ void __launch_bounds__(256) nsa_bwd_prep_kernel(const __nv_bfloat16 *__restrict__ dout,
+                                                           const float *__restrict__ o3, long long rows,
+                                                           float *__restrict__ Dt, float *__restrict__ dgates) {
+    grid_dependency_sync();
+    const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    const __nv_bfloat162 *a = reinterpret_cast<const __nv_bfloat162 *>(dout + row * D);
+    float s[3] = {0.f, 0.f, 0.f};
+#pragma unroll
+    for (int c = lane; c < D / 2; c += 32) {
+        const float2 x = __bfloat1622float2(a[c]);
+#pragma unroll
+        for (int br = 0; br < 3; ++br) {
+            const float2 y = reinterpret_cast<const float2 *>(o3 + (br * rows + row) * D)[c];
+            s[br] += x.x * y.x + x.y * y.y;
+        }
+    }
+#pragma unroll
+    for (int br = 0; br < 3; ++br) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) s[br] += __shfl_xor_sync(0xffffffffu, s[br], o);
+    }
+    if (lane < 3) {
+        const float r = lane == 0 ? s[0] : (lane == 1 ? s[1] : s[2]);
+        Dt[lane * rows + row] = r;
+        dgates[row * 3 + lane] = r;
+    }
+}
+
+// NSA: the compressed row i is the mean of rows i*stride .. i*stride+len-1,
+// so raw row j receives dKc_i / len from every i that covers it (likewise
+// V).  One thread per 4 columns of a (b, j, g) row; added to dk / dv.
+__global__ void __launch_bounds__(256) nsa_pool_bwd_kernel(const float *__restrict__ dkc, const float *__restrict__ dvc,
+                                                           float *__restrict__ dk, float *__restrict__ dv, int B, int T,
+                                                           int Hkv, int d, int nc, int len, int stride) {
+    grid_dependency_sync();
+    const int d4 = d / 4;
+    const long long total = (long long)B * T * Hkv * d4;
+    const long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (e >= total) return;
+    const int c4 = (int)(e % d4);
+    long long r = e / d4;
+    const int g = (int)(r % Hkv); r /= Hkv;
+    const int j = (int)(r % T);
+    const int b = (int)(r / T);
+    int i_hi = j / stride;
+    if (i_hi > nc - 1) i_hi = nc - 1;
+    const int i_lo = j - len + 1 <= 0 ? 0 : (j - len + stride) / stride;
+    float4 sk = make_float4(0.f, 0.f, 0.f, 0.f), sv = sk;
+    for (int i = i_lo; i <= i_hi; ++i) {
+        const long long o = (((long long)b * nc + i) * Hkv + g) * d4 + c4;
+        const float4 x = reinterpret_cast<const float4 *>(dkc)[o];
+        const float4 y = reinterpret_cast<const float4 *>(dvc)[o];
+        sk.x += x.x; sk.y += x.y; sk.z += x.z; sk.w += x.w;
+        sv.x += y.x; sv.y += y.y; sv.z += y.z; sv.w += y.w;
+    }
+    const float inv = 1.f / (float)len;
+    float4 *pk = reinterpret_cast<float4 *>(dk) + e;
+    float4 *pv = reinterpret_cast<float4 *>(dv) + e;
+    float4 a = *pk, c = *pv;
+    a.x += sk.x * inv; a.y += sk.y * inv; a.z += sk.z * inv; a.w += sk.w * inv;
+    c.x += sv.x * inv; c.y += sv.y * inv; c.z += sv.z * inv; c.w += sv.w * inv;
+    *pk = a;
+    *pv = c;
 }
 
 }  // namespace sa

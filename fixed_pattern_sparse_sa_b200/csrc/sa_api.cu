@@ -1142,11 +1142,10 @@ static int launch_tile(const TileParams &p, int d, int src, cudaStream_t st) {
     return src == TS_CMP ? launch_tile_t<128, TS_CMP>(p, st) : launch_tile_t<128, TS_WINDOW>(p, st);
 }
 
-int sa_nsa_fwd(const void *q, const void *k, const void *v, const float *gates, int B, int T, int Hq,
-               int Hkv, int d, int cmp_len, int cmp_stride, int sel_block, int sel_topk, int window,
-               float scale, void *out, float *lse_branches, int32_t *sel_idx_out, void *workspace,
-               size_t workspace_bytes, void *stream) {
-    SA_TRACE("sa_nsa_fwd");
+static int nsa_fwd_impl(const void *q, const void *k, const void *v, const float *gates, int B, int T, int Hq,
+                        int Hkv, int d, int cmp_len, int cmp_stride, int sel_block, int sel_topk, int window,
+                        float scale, void *out, float *lse_branches, int32_t *sel_idx_out, float *o_branches,
+                        void *workspace, size_t workspace_bytes, void *stream) {
     if (B <= 0 || T < 0 || Hq <= 0 || Hkv <= 0 || cmp_len <= 0 || cmp_stride <= 0 || sel_block <= 0 ||
         sel_topk <= 0 || window <= 0)
         return fail(SA_ERR_INVALID_ARG, "nsa: bad sizes");
@@ -1172,7 +1171,7 @@ int sa_nsa_fwd(const void *q, const void *k, const void *v, const float *gates, 
     __nv_bfloat16 *kc = reinterpret_cast<__nv_bfloat16 *>(ws + lay.kc_off);
     __nv_bfloat16 *vc = reinterpret_cast<__nv_bfloat16 *>(ws + lay.vc_off);
     __nv_bfloat16 *klo = reinterpret_cast<__nv_bfloat16 *>(ws + lay.klo_off);
-    float *o3 = reinterpret_cast<float *>(ws + lay.o3_off);
+    float *o3 = o_branches ? o_branches : reinterpret_cast<float *>(ws + lay.o3_off);
     float *l3 = reinterpret_cast<float *>(ws + lay.l3_off);
     int32_t *sel = sel_idx_out ? sel_idx_out : reinterpret_cast<int32_t *>(ws + lay.sel_off);
     const long long rows = (long long)B * T * Hq;
@@ -1252,6 +1251,178 @@ int sa_nsa_fwd(const void *q, const void *k, const void *v, const float *gates, 
                 lse_branches);
             SA_CHECK_LAUNCH("nsa_lse_pack_kernel");
         }
+    }
+    return SA_OK;
+}
+
+int sa_nsa_fwd(const void *q, const void *k, const void *v, const float *gates, int B, int T, int Hq,
+               int Hkv, int d, int cmp_len, int cmp_stride, int sel_block, int sel_topk, int window,
+               float scale, void *out, float *lse_branches, int32_t *sel_idx_out, void *workspace,
+               size_t workspace_bytes, void *stream) {
+    SA_TRACE("sa_nsa_fwd");
+    return nsa_fwd_impl(q, k, v, gates, B, T, Hq, Hkv, d, cmp_len, cmp_stride, sel_block, sel_topk, window, scale,
+                        out, lse_branches, sel_idx_out, nullptr, workspace, workspace_bytes, stream);
+}
+
+int sa_nsa_fwd_train(const void *q, const void *k, const void *v, const float *gates, int B, int T, int Hq,
+                     int Hkv, int d, int cmp_len, int cmp_stride, int sel_block, int sel_topk, int window,
+                     float scale, void *out, float *lse_branches, int32_t *sel_idx_out, float *o_branches,
+                     void *workspace, size_t workspace_bytes, void *stream) {
+    SA_TRACE("sa_nsa_fwd_train");
+    if (!lse_branches || !sel_idx_out || !o_branches || !aligned4(lse_branches) || !aligned4(sel_idx_out) ||
+        !aligned16(o_branches))
+        return fail(SA_ERR_INVALID_ARG, "nsa_fwd_train: null or misaligned saved-tensor pointer");
+    return nsa_fwd_impl(q, k, v, gates, B, T, Hq, Hkv, d, cmp_len, cmp_stride, sel_block, sel_topk, window, scale,
+                        out, lse_branches, sel_idx_out, o_branches, workspace, workspace_bytes, stream);
+}
+
+// ------------------------------------------------------------ NSA backward --
+struct NsaBwdLayout {
+    int nc;
+    size_t kc_off, klo_off, vc_off, dkc_off, dvc_off, dt_off, total;
+};
+
+static NsaBwdLayout nsa_bwd_layout(int B, int T, int Hq, int Hkv, int d, int cmp_len, int cmp_stride) {
+    NsaBwdLayout lay{};
+    lay.nc = T >= cmp_len ? (T - cmp_len) / cmp_stride + 1 : 0;
+    const size_t crow = (size_t)B * std::max(lay.nc, 1) * Hkv * d;
+    size_t off = 0;
+    lay.kc_off = off; off += round_up(crow * 2, 256);
+    lay.klo_off = off; off += round_up(crow * 2, 256);
+    lay.vc_off = off; off += round_up(crow * 2, 256);
+    lay.dkc_off = off; off += round_up(crow * 4, 256);
+    lay.dvc_off = off; off += round_up(crow * 4, 256);
+    lay.dt_off = off; off += round_up((size_t)3 * B * T * Hq * 4, 256);
+    lay.total = off;
+    return lay;
+}
+
+size_t sa_nsa_bwd_workspace_size(int B, int T, int Hq, int Hkv, int d, int cmp_len, int cmp_stride) {
+    if (B <= 0 || T <= 0 || Hq <= 0 || Hkv <= 0 || d <= 0 || cmp_len <= 0 || cmp_stride <= 0) return 0;
+    return nsa_bwd_layout(B, T, Hq, Hkv, d, cmp_len, cmp_stride).total;
+}
+
+template <int D, int SRC, bool HILO>
+static int launch_bwd_branch(const BwdParams &p, cudaStream_t st) {
+    constexpr int NW = (HILO && D == 128) ? 6 : 8;    // shared memory: 3 arrays per stage with HILO
+    constexpr int smem = attn_bwd_smem_bytes<D, NW, HILO>();
+    static_assert(smem <= 227 * 1024, "shared memory");
+    auto kern = attn_bwd_kernel<D, NW, SRC, HILO>;
+    int rc = set_smem(kern, smem);
+    if (rc) return rc;
+    const long long items = (long long)p.B * p.Tq * p.Hkv * ((p.G + 15) / 16);
+    if (items == 0) return SA_OK;
+    launch_k(__PRETTY_FUNCTION__, kern, (unsigned)((items + NW - 1) / NW), NW * 32, smem, st, p);
+    SA_CHECK_LAUNCH("attn_bwd_kernel");
+    return SA_OK;
+}
+
+template <int D>
+static int nsa_bwd_branches(const BwdParams &base, const float *gates, const float *lse3, long long rows,
+                            float *Dt, const NsaBwdLayout &lay, const __nv_bfloat16 *kc, const __nv_bfloat16 *klo,
+                            const __nv_bfloat16 *vc, float *dkc, float *dvc, const int32_t *sel, int sel_block,
+                            int sel_topk, int window, int cmp_len, int cmp_stride, cudaStream_t st) {
+    // compressed branch: keys Kc (hi/lo), gradients into dKc / dVc; writes dq
+    BwdParams p = base;
+    p.k = kc; p.klo = klo; p.v = vc; p.L = std::max(lay.nc, 1);
+    p.lse = lse3; p.gate = gates; p.Dt = Dt;
+    p.window = 0; p.cmp_len = cmp_len; p.cmp_stride = cmp_stride;
+    p.dk = dkc; p.dv = dvc; p.dq_accum = 0;
+    if (lay.nc == 0) p.L = 0;       // no compressed row is visible to any query
+    int rc = launch_bwd_branch<D, BW_RANGE, true>(p, st);
+    if (rc) return rc;
+    // selected branch: keys of the chosen blocks
+    p = base;
+    p.lse = lse3 + 1; p.gate = gates + 1; p.Dt = Dt + rows;
+    p.idx = sel; p.idx_heads = base.Hkv; p.K = sel_topk; p.block = sel_block;
+    p.block_shift = (sel_block & (sel_block - 1)) == 0 ? __builtin_ctz((unsigned)sel_block) : -1;
+    p.dq_accum = 1;
+    rc = launch_bwd_branch<D, BW_BLOCKS, false>(p, st);
+    if (rc) return rc;
+    // window branch
+    p = base;
+    p.lse = lse3 + 2; p.gate = gates + 2; p.Dt = Dt + 2 * rows;
+    p.window = window; p.dq_accum = 1;
+    return launch_bwd_branch<D, BW_RANGE, false>(p, st);
+}
+
+int sa_nsa_bwd(const void *q, const void *k, const void *v, const float *gates, const void *dout,
+               const float *o_branches, const float *lse_branches, const int32_t *sel_idx, int B, int T, int Hq,
+               int Hkv, int d, int cmp_len, int cmp_stride, int sel_block, int sel_topk, int window, float scale,
+               float *dq, float *dk, float *dv, float *dgates, void *workspace, size_t workspace_bytes,
+               void *stream) {
+    SA_TRACE("sa_nsa_bwd");
+    if (B <= 0 || T < 0 || Hq <= 0 || Hkv <= 0 || cmp_len <= 0 || cmp_stride <= 0 || sel_block <= 0 ||
+        sel_topk <= 0 || window <= 0)
+        return fail(SA_ERR_INVALID_ARG, "nsa_bwd: bad sizes");
+    if (Hq % Hkv) return fail(SA_ERR_INVALID_ARG, "nsa_bwd: Hq %% Hkv != 0");
+    if (d != 64 && d != 128) return fail(SA_ERR_UNSUPPORTED, "nsa_bwd: head dim %d", d);
+    if (!q || !k || !v || !gates || !dout || !o_branches || !lse_branches || !sel_idx || !dq || !dk || !dv ||
+        !dgates || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned4(gates) || !aligned16(dout) ||
+        !aligned16(o_branches) || !aligned4(lse_branches) || !aligned4(sel_idx) || !aligned16(dq) ||
+        !aligned16(dk) || !aligned16(dv) || !aligned4(dgates))
+        return fail(SA_ERR_INVALID_ARG, "nsa_bwd: null or misaligned pointer");
+    if (!std::isfinite(scale)) return fail(SA_ERR_INVALID_ARG, "nsa_bwd: scale");
+    if (T == 0) return SA_OK;
+    if ((long long)sel_topk * sel_block > INT_MAX / 2) return fail(SA_ERR_UNSUPPORTED, "nsa_bwd: selection size");
+    const NsaBwdLayout lay = nsa_bwd_layout(B, T, Hq, Hkv, d, cmp_len, cmp_stride);
+    if (!workspace || workspace_bytes < lay.total)
+        return fail(SA_ERR_WORKSPACE, "nsa_bwd: workspace %zu < %zu", workspace_bytes, lay.total);
+    if (!aligned16(workspace)) return fail(SA_ERR_INVALID_ARG, "nsa_bwd: workspace alignment");
+    unsigned *ew = nullptr;
+    int rc = device_error_word(&ew);
+    if (rc) return rc;
+    cudaStream_t st = as_stream(stream);
+    char *ws = static_cast<char *>(workspace);
+    __nv_bfloat16 *kc = reinterpret_cast<__nv_bfloat16 *>(ws + lay.kc_off);
+    __nv_bfloat16 *klo = reinterpret_cast<__nv_bfloat16 *>(ws + lay.klo_off);
+    __nv_bfloat16 *vc = reinterpret_cast<__nv_bfloat16 *>(ws + lay.vc_off);
+    float *dkc = reinterpret_cast<float *>(ws + lay.dkc_off);
+    float *dvc = reinterpret_cast<float *>(ws + lay.dvc_off);
+    float *Dt = reinterpret_cast<float *>(ws + lay.dt_off);
+    const long long rows = (long long)B * T * Hq;
+    const size_t kv_bytes = (size_t)B * T * Hkv * d * 4;
+    const size_t ckv_bytes = (size_t)B * std::max(lay.nc, 1) * Hkv * d * 4;
+    cudaError_t e = cudaMemsetAsync(dk, 0, kv_bytes, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dv, 0, kv_bytes, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dkc, 0, ckv_bytes, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dvc, 0, ckv_bytes, st);
+    if (e != cudaSuccess) return fail(SA_ERR_CUDA, "nsa_bwd memset: %s", cudaGetErrorString(e));
+    // 1. compressed rows, as in the forward
+    if (lay.nc > 0) {
+        const long long n2 = (long long)B * lay.nc * Hkv * (d / 2);
+        launch_k("nsa_compress_kernel", nsa_compress_kernel, (unsigned)((n2 + 255) / 256), 256, 0, st,
+            (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, B, T, Hkv, d, lay.nc, cmp_len, cmp_stride, kc, klo,
+            vc);
+        SA_CHECK_LAUNCH("nsa_compress_kernel");
+    }
+    // 2. r_b = dO . O_b per row and branch (the D terms and the gate gradients)
+    if (d == 64)
+        launch_k("nsa_bwd_prep_kernel<64>", nsa_bwd_prep_kernel<64>, (unsigned)((rows + 7) / 8), 256, 0, st,
+            (const __nv_bfloat16 *)dout, o_branches, rows, Dt, dgates);
+    else
+        launch_k("nsa_bwd_prep_kernel<128>", nsa_bwd_prep_kernel<128>, (unsigned)((rows + 7) / 8), 256, 0, st,
+            (const __nv_bfloat16 *)dout, o_branches, rows, Dt, dgates);
+    SA_CHECK_LAUNCH("nsa_bwd_prep_kernel");
+    // 3. the three branches' backward (dq accumulates over them)
+    BwdParams base{};
+    base.q = static_cast<const __nv_bfloat16 *>(q); base.k = static_cast<const __nv_bfloat16 *>(k);
+    base.v = static_cast<const __nv_bfloat16 *>(v); base.dout = static_cast<const __nv_bfloat16 *>(dout);
+    base.B = B; base.Tq = T; base.L = T; base.Hq = Hq; base.Hkv = Hkv; base.G = Hq / Hkv; base.idx_heads = 1;
+    base.q_pos0 = 0; base.scale = scale; base.scale_log2 = scale * kLog2e;
+    base.lse_stride = 3; base.gate_stride = 3;
+    base.dq = dq; base.dk = dk; base.dv = dv; base.err = ew;
+    rc = d == 64 ? nsa_bwd_branches<64>(base, gates, lse_branches, rows, Dt, lay, kc, klo, vc, dkc, dvc, sel_idx,
+                                        sel_block, sel_topk, window, cmp_len, cmp_stride, st)
+                 : nsa_bwd_branches<128>(base, gates, lse_branches, rows, Dt, lay, kc, klo, vc, dkc, dvc, sel_idx,
+                                         sel_block, sel_topk, window, cmp_len, cmp_stride, st);
+    if (rc) return rc;
+    // 4. compressed-row gradients back to the rows they average
+    if (lay.nc > 0) {
+        const long long n4 = (long long)B * T * Hkv * (d / 4);
+        launch_k("nsa_pool_bwd_kernel", nsa_pool_bwd_kernel, (unsigned)((n4 + 255) / 256), 256, 0, st,
+            (const float *)dkc, (const float *)dvc, dk, dv, B, T, Hkv, d, lay.nc, cmp_len, cmp_stride);
+        SA_CHECK_LAUNCH("nsa_pool_bwd_kernel");
     }
     return SA_OK;
 }
@@ -1397,6 +1568,7 @@ int sa_sparse_attn_bwd(const void *q, const void *k, const void *v, const void *
     p.dout = static_cast<const __nv_bfloat16 *>(dout); p.lse = lse; p.idx = idx;
     p.B = B; p.Tq = Tq; p.L = L; p.Hq = Hq; p.Hkv = Hkv; p.G = Hq / Hkv; p.idx_heads = idx_heads; p.K = K;
     p.q_pos0 = q_pos0; p.scale = scale; p.scale_log2 = scale * kLog2e;
+    p.lse_stride = 1; p.gate = nullptr; p.dq_accum = 0;
     p.Dt = static_cast<float *>(workspace); p.dq = dq; p.dk = dk; p.dv = dv; p.err = ew;
     const long long rows = (long long)B * Tq * Hq;
     return d == 64 ? launch_bwd<64>(p, rows, st) : launch_bwd<128>(p, rows, st);

@@ -225,6 +225,47 @@ int sa_nsa_fwd(const void *q, const void *k, const void *v, const float *gates,
                void *workspace, size_t workspace_bytes, void *stream);
 
 /* --------------------------------------------------------------------------
+ * NSA forward for training: sa_nsa_fwd, plus the tensors sa_nsa_bwd needs.
+ *   o_branches fp32 [3,B,T,Hq,d]: the ungated branch outputs (compressed,
+ *   selected, window), caller-owned; lse_branches and sel_idx_out are
+ *   required here.  Same workspace as sa_nsa_fwd.
+ * ------------------------------------------------------------------------ */
+int sa_nsa_fwd_train(const void *q, const void *k, const void *v, const float *gates,
+                     int B, int T, int Hq, int Hkv, int d,
+                     int cmp_len, int cmp_stride, int sel_block, int sel_topk, int window,
+                     float scale, void *out, float *lse_branches, int32_t *sel_idx_out,
+                     float *o_branches, void *workspace, size_t workspace_bytes, void *stream);
+
+/* --------------------------------------------------------------------------
+ * NSA backward (Native Sparse Attention page, "Puntos Clave": natively
+ * trainable, with a faster backward pass).  The gradient of sa_nsa_fwd's
+ * out for an upstream gradient dout, with the forward's block choice
+ * (sel_idx) held fixed: the choice is piecewise constant in the inputs, so
+ * no gradient flows through the importance or the top-k.  Per row and
+ * head, branch b (gate value g_b, ungated output O_b, saved lse_b):
+ *   dgates_b = dout . O_b;  the branch's upstream gradient is g_b dout;
+ *   dP_j = g_b dout . v_j,  D = g_b dout . O_b,  dS_j = p_j (dP_j - D),
+ *   dq += scale sum_j dS_j k_j,  dk_j += scale dS_j q,  dv_j += p_j g_b dout.
+ * The compressed branch's key rows are Kc_i (mean of K[i*stride ..
+ * i*stride+len-1]); each of those rows receives dKc_i / len (likewise V).
+ *   q, dout bf16 [B,T,Hq,d]; k, v bf16 [B,T,Hkv,d]; gates fp32 [B,T,Hq,3];
+ *   o_branches, lse_branches, sel_idx: sa_nsa_fwd_train's outputs.
+ *   dq fp32 [B,T,Hq,d]; dk, dv fp32 [B,T,Hkv,d]; dgates fp32 [B,T,Hq,3];
+ *   all written (not accumulated).  d = 64 or 128, any Hq/Hkv.
+ * Workspace: sa_nsa_bwd_workspace_size bytes, 16-byte aligned.  A selected
+ * block past the sequence sets the device error word (SA_ERR_DEVICE_ASSERT
+ * from sa_check_device_status).
+ * ------------------------------------------------------------------------ */
+size_t sa_nsa_bwd_workspace_size(int B, int T, int Hq, int Hkv, int d, int cmp_len,
+                                 int cmp_stride);
+int sa_nsa_bwd(const void *q, const void *k, const void *v, const float *gates,
+               const void *dout, const float *o_branches, const float *lse_branches,
+               const int32_t *sel_idx, int B, int T, int Hq, int Hkv, int d,
+               int cmp_len, int cmp_stride, int sel_block, int sel_topk, int window,
+               float scale, float *dq, float *dk, float *dv, float *dgates,
+               void *workspace, size_t workspace_bytes, void *stream);
+
+/* --------------------------------------------------------------------------
  * IndexCache layer driver (IndexCache page, body): layers marked 'F' run the
  * indexer and top-k and overwrite the cached index buffer; layers marked 'S'
  * skip the indexer and reuse the buffer of the nearest preceding F layer.

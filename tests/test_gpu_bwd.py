@@ -116,3 +116,68 @@ def test_backward_identities_16k(cuda_ok):
         got.append(dq[:, row:row + 1].double().cpu())
         ref.append(rqi)
     _close(torch.cat(got, dim=1), np.concatenate(ref, axis=1), "dq (sampled rows)")
+
+
+# ------------------------------------------------------------ NSA backward --
+# Tolerance as above: P and dS are rounded to bf16 for the tensor-core
+# products, the compressed keys are a bf16 hi/lo pair and the compressed
+# values are rounded once to bf16 (as in the forward).  The block choice is
+# the forward's; the oracle makes its own and the test requires the two to
+# agree, so both sides differentiate the same function.
+def _nsa_bwd_gpu(g, dout, cfg):
+    dev = "cuda"
+    q, k, v, gates = (g[n].to(dev) for n in ("q", "k", "v", "gates"))
+    out, lse3, sel, o3 = api.nsa_fwd_train(q, k, v, gates, **cfg)
+    dq, dk, dv, dg = api.nsa_bwd(q, k, v, gates, dout.to(dev), o3, lse3, sel, **cfg)
+    api.check_device_status()
+    return out, sel, dq, dk, dv, dg
+
+
+@pytest.mark.parametrize("T,Hq,Hkv,d,cfg", [
+    # tcgen05 forward path (d = 128, group of 16), real selection
+    (640, 32, 2, 128, dict(cmp_len=32, cmp_stride=16, sel_block=64, sel_topk=4, window=128)),
+    # d = 64, ragged T, selection blocks not a power of two apart from the window
+    (333, 8, 2, 64, dict(cmp_len=16, cmp_stride=8, sel_block=32, sel_topk=3, window=50)),
+    # 12 heads per KV head, every candidate block chosen, window longer than T
+    (200, 12, 1, 128, dict(cmp_len=32, cmp_stride=16, sel_block=64, sel_topk=16, window=512)),
+    # T shorter than one compressed window: the compressed branch is empty
+    (20, 4, 1, 64, dict(cmp_len=32, cmp_stride=16, sel_block=16, sel_topk=2, window=8)),
+])
+def test_nsa_backward_parity(cuda_ok, T, Hq, Hkv, d, cfg):
+    g = inputs.gen_nsa(1, T, Hq, Hkv, d, seed=100 + T)
+    gen = torch.Generator().manual_seed(200 + T)
+    dout = torch.randn(1, T, Hq, d, generator=gen).to(torch.bfloat16)
+    ref_f = oracle.nsa_fwd(g["q"], g["k"], g["v"], g["gates"], **cfg)
+    ref = oracle.nsa_bwd(g["q"], g["k"], g["v"], g["gates"], dout, ref_f["sel_idx"], **cfg)
+    out, sel, dq, dk, dv, dg = _nsa_bwd_gpu(g, dout, cfg)
+    assert np.array_equal(sel.cpu().numpy().reshape(ref_f["sel_idx"].shape), ref_f["sel_idx"])
+    _close(dq, ref["dq"], "dq")
+    _close(dk, ref["dk"], "dk")
+    _close(dv, ref["dv"], "dv")
+    _close(dg, ref["dgates"], "dgates")
+
+
+def test_nsa_backward_identities_8k(cuda_ok):
+    # any input: sum_j dk_j = 0 per KV head; sum_j dv_j = the gate-weighted
+    # dout of the group's heads over the branches that see at least one key
+    T, Hq, Hkv, d = 8192, 64, 4, 128
+    cfg = dict(cmp_len=32, cmp_stride=16, sel_block=64, sel_topk=16, window=512)
+    g = inputs.gen_nsa(1, T, Hq, Hkv, d, seed=7)
+    gen = torch.Generator().manual_seed(8)
+    dout = torch.randn(1, T, Hq, d, generator=gen).to(torch.bfloat16)
+    out, sel, dq, dk, dv, dg = _nsa_bwd_gpu(g, dout, cfg)
+    dk64, dv64 = dk.double().cpu(), dv.double().cpu()
+    live = torch.ones(T, Hq, 3, dtype=torch.float64)
+    live[: cfg["cmp_len"] - 1, :, 0] = 0.0                 # no compressed row visible yet
+    w = (g["gates"][0].double() * live).sum(-1)             # [T, Hq]
+    do = dout[0].double() * w[..., None]
+    expect = do.reshape(T, Hkv, Hq // Hkv, d).sum(dim=(0, 2))
+    scale = dv64.abs().sum(dim=1)[0]                        # [Hkv, d]
+    assert torch.all((dv64.sum(dim=1)[0] - expect).abs() <= 1e-3 * scale + 1e-3)
+    assert torch.all(dk64.sum(dim=1)[0].abs() <= 1e-3 * dk64.abs().sum(dim=1)[0] + 1e-3)
+    # the gate gradient against the oracle's branch outputs on sampled rows
+    rows = np.array([0, 31, 32, 1000, 4097, T - 1])
+    ref_f = oracle.nsa_fwd(g["q"], g["k"], g["v"], g["gates"], **cfg, rows=rows)
+    dgr = np.einsum("rhc,brhc->rhb", dout[0].double().numpy()[rows],
+                    ref_f["o_branch"].reshape(3, len(rows), Hq, d))
+    _close(dg[0].cpu()[rows], dgr, "dgates (sampled rows)")
