@@ -65,13 +65,15 @@ def _load():
             lib.oracle_lse_combine.argtypes = [P, P, I, I, I, P, P]
             lib.oracle_sparse_attn_bwd.argtypes = [P, P, P, P, I, I, I, I, I, I, I, P, I, I, D, P, P, P]
             lib.oracle_nsa_compress.argtypes = [P, P, I, I, I, I, I, I, P, P]
+            lib.oracle_full_attn_topk.argtypes = [P, P, P, I, I, I, I, I, D, I, I, P, I, P, P, P, P]
             lib.oracle_nsa_bwd.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, I, D,
                                            P, P, P, P]
             lib.oracle_nsa_fwd.argtypes = [P, P, P, P, I, I, I, I, I, I, I, I, I, I, D,
                                            P, I, P, P, P, P, P, P]
             for name in ("oracle_indexer_scores", "oracle_indexer_topk",
                          "oracle_sparse_attn", "oracle_sparse_attn_bwd", "oracle_lse_combine",
-                         "oracle_nsa_compress", "oracle_nsa_fwd", "oracle_nsa_bwd"):
+                         "oracle_nsa_compress", "oracle_nsa_fwd", "oracle_nsa_bwd",
+                         "oracle_full_attn_topk"):
                 getattr(lib, name).restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -322,6 +324,34 @@ def nsa_bwd(q, k, v, gates, dout, sel_idx, cmp_len, cmp_stride, sel_block, sel_t
                               cmp_len, cmp_stride, sel_block, sel_topk, window, float(scale),
                               _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg)), "nsa_bwd")
     return {"dq": dq, "dk": dk, "dv": dv, "dgates": dg}
+
+
+def full_attn_topk(q, k, v, topk, window, scale=None, rows=None, want_scores=False):
+    """A full-attention layer as an exact indexer (HySparse2 page), fp64.
+
+    q [B,T,Hq,d], k/v [B,T,Hkv,d] bf16.  Returns (out [n,Hq,d], lse [n,Hq],
+    idx [n, topk+window] int32) and, with want_scores, scores [n, T]: the
+    full layer's attention probability on each key summed over all heads.
+    The set is the forced window plus the top-k of the other keys by
+    (score desc, index asc), ascending and -1 padded.
+    """
+    lib = _load()
+    B, T, Hq, d = q.shape
+    Hkv = k.shape[2]
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    r, n = _rows(rows, B * T)
+    out = np.empty((n, Hq, d), dtype=np.float64)
+    lse = np.empty((n, Hq), dtype=np.float64)
+    idx = np.empty((n, topk + window), dtype=np.int32)
+    sc = np.empty((n, T), dtype=np.float64) if want_scores else None
+    _check(lib.oracle_full_attn_topk(_ptr(_np(q, np.uint16)), _ptr(_np(k, np.uint16)),
+                                     _ptr(_np(v, np.uint16)), B, T, Hq, Hkv, d, float(scale),
+                                     topk, window, _ptr(r), n, _ptr(out), _ptr(lse), _ptr(idx),
+                                     _ptr(sc)), "full_attn_topk")
+    if want_scores:
+        return out, lse, idx, sc
+    return out, lse, idx
 
 
 def dsa_layers(pattern, layers, topk, window=0, q_pos0=None, scale=None):

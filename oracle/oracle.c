@@ -830,3 +830,101 @@ int oracle_nsa_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v,
     free(kc); free(vc); free(dkc); free(dvc); free(kraw); free(vraw);
     return status;
 }
+
+/* ------------------------------------------------------------------------ */
+/* A full-attention layer as an exact indexer (HySparse2 page, "Que         */
+/* significa para la evolucion de la IA": a few full-attention layers       */
+/* compute exact scores and guide the sparse layers' selection).            */
+/* ------------------------------------------------------------------------ */
+
+typedef struct { double score; int64_t j; } dcand_t;
+
+/* Order: larger score first; equal scores -> lower index first. */
+static int dcand_cmp(const void *a, const void *b)
+{
+    const dcand_t *x = (const dcand_t *)a, *y = (const dcand_t *)b;
+    if (x->score != y->score) return x->score > y->score ? -1 : 1;
+    return (x->j > y->j) - (x->j < y->j);
+}
+
+/*
+ * For the requested rows (flat r = b*T + t, position t):
+ *  1. the full layer itself: causal softmax attention of every head over all
+ *     keys j <= t (fp64): out [n_rows,Hq,d], lse [n_rows,Hq];
+ *  2. the exact score of key j for query t: the attention probability that
+ *     the full layer puts on j, summed over all Hq heads:
+ *       score(t, j) = sum_h exp(scale q_{t,h}.k_{j,g(h)} - lse_{t,h});
+ *  3. the index set for the sparse layers: the forced window W_t =
+ *     {max(0, t-window+1) .. t} plus the top-k of the other keys by
+ *     (score desc, j asc), as in oracle_indexer_topk; ascending, -1 padded
+ *     to topk+window.
+ * scores (nullable) [n_rows, T]: score(t, j) for j <= t, 0 after t.
+ */
+int oracle_full_attn_topk(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                          int64_t B, int64_t T, int64_t Hq, int64_t Hkv, int64_t d,
+                          double scale, int64_t topk, int64_t window,
+                          const int64_t *rows, int64_t n_rows,
+                          double *out, double *lse, int32_t *out_idx, double *scores)
+{
+    if (B <= 0 || T <= 0 || Hq <= 0 || Hkv <= 0 || d <= 0 || Hq % Hkv != 0 ||
+        topk < 0 || window < 0 || topk + window <= 0)
+        return OR_BAD_ARG;
+    if (!rows) n_rows = B * T;
+    const int64_t G = Hq / Hkv;
+    const int64_t K = topk + window;
+    int bad = 0;
+#pragma omp parallel
+    {
+        double *z = (double *)malloc(sizeof(double) * (size_t)T);
+        double *sc = (double *)malloc(sizeof(double) * (size_t)T);
+        double *qv = (double *)malloc(sizeof(double) * (size_t)d);
+        dcand_t *cand = (dcand_t *)malloc(sizeof(dcand_t) * (size_t)T);
+        int32_t *sel = (int32_t *)malloc(sizeof(int32_t) * (size_t)K);
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t i = 0; i < n_rows; ++i) {
+            int64_t r = row_at(rows, i);
+            if (r < 0 || r >= B * T || !z || !sc || !qv || !cand || !sel) { bad = 1; continue; }
+            const int64_t b = r / T, t = r % T;
+            for (int64_t j = 0; j <= t; ++j) sc[j] = 0.0;
+            for (int64_t h = 0; h < Hq; ++h) {
+                const int64_t g = h / G;
+                for (int64_t c = 0; c < d; ++c) qv[c] = bf16_to_f64(q[(r * Hq + h) * d + c]);
+                double m = -INFINITY;
+                for (int64_t j = 0; j <= t; ++j) {
+                    const uint16_t *kr = k + ((b * T + j) * Hkv + g) * d;
+                    double dot = 0.0;
+                    for (int64_t c = 0; c < d; ++c) dot += qv[c] * bf16_to_f64(kr[c]);
+                    z[j] = scale * dot;
+                    if (z[j] > m) m = z[j];
+                }
+                double s = 0.0;
+                for (int64_t j = 0; j <= t; ++j) s += exp(z[j] - m);
+                const double l = m + log(s);
+                if (lse) lse[i * Hq + h] = l;
+                double *o = out ? out + (i * Hq + h) * d : NULL;
+                if (o) for (int64_t c = 0; c < d; ++c) o[c] = 0.0;
+                for (int64_t j = 0; j <= t; ++j) {
+                    const double p = exp(z[j] - l);
+                    sc[j] += p;
+                    if (o) {
+                        const uint16_t *vr = v + ((b * T + j) * Hkv + g) * d;
+                        for (int64_t c = 0; c < d; ++c) o[c] += p * bf16_to_f64(vr[c]);
+                    }
+                }
+            }
+            if (scores)
+                for (int64_t j = 0; j < T; ++j) scores[i * T + j] = j <= t ? sc[j] : 0.0;
+            const int64_t w_lo = window > 0 ? (t - window + 1 > 0 ? t - window + 1 : 0) : t + 1;
+            for (int64_t j = 0; j < w_lo; ++j) { cand[j].score = sc[j]; cand[j].j = j; }
+            qsort(cand, (size_t)w_lo, sizeof(dcand_t), dcand_cmp);
+            const int64_t n_take = w_lo < topk ? w_lo : topk;
+            int64_t n_sel = 0;
+            for (int64_t m2 = 0; m2 < n_take; ++m2) sel[n_sel++] = (int32_t)cand[m2].j;
+            for (int64_t j = w_lo; j <= t; ++j) sel[n_sel++] = (int32_t)j;
+            qsort(sel, (size_t)n_sel, sizeof(int32_t), i32_cmp);
+            for (int64_t m2 = 0; m2 < K; ++m2) out_idx[i * K + m2] = m2 < n_sel ? sel[m2] : -1;
+        }
+        free(z); free(sc); free(qv); free(cand); free(sel);
+    }
+    return bad ? OR_BAD_ARG : OR_OK;
+}

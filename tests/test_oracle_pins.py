@@ -742,3 +742,74 @@ def test_nsa_backward_column_sums():
     ob = r["o_branch"].reshape(3, T, Hq, d)
     np.testing.assert_allclose(gr["dgates"][0], np.einsum("thc,bthc->thb", _f64(dout).numpy()[0], ob),
                                atol=1e-12)
+
+
+# ------------------------------------------- full-attention exact indexer --
+def _full_case(T=70, Hq=4, Hkv=2, d=16, seed=61):
+    g = inputs.gen_dsa(1, T, Hq, Hkv, d, 1, 32, seed=seed)
+    return g["q"], g["k"], g["v"]
+
+
+def _select_ref(scores, T, topk, window):
+    """Window + top-k of the rest by (score desc, index asc) with numpy lexsort."""
+    K = topk + window
+    idx = np.full((T, K), -1, dtype=np.int32)
+    for t in range(T):
+        w_lo = max(0, t - window + 1) if window > 0 else t + 1
+        j = np.arange(w_lo)
+        order = np.lexsort((j, -scores[t, :w_lo]))
+        chosen = np.sort(np.concatenate([j[order[:topk]], np.arange(w_lo, t + 1)]))
+        idx[t, :len(chosen)] = chosen
+    return idx
+
+
+def test_full_attn_indexer_layer_is_causal_sdpa():
+    T, Hq, Hkv, d = 70, 4, 2, 16
+    q, k, v = _full_case(T, Hq, Hkv, d)
+    out, lse, idx, sc = oracle.full_attn_topk(q, k, v, topk=8, window=4, want_scores=True)
+    mask = torch.ones(T, T, dtype=torch.bool).tril()
+    np.testing.assert_allclose(out, sdpa_ref(q, k, v, mask=mask, scale=1 / math.sqrt(d))[0], atol=1e-12)
+    np.testing.assert_allclose(lse, lse_ref(q, k, mask, 1 / math.sqrt(d))[0], atol=1e-12)
+
+
+def test_full_attn_indexer_scores_are_head_summed_probabilities():
+    # torch softmax of the masked logits, summed over the heads; every row
+    # sums to Hq (each head's probabilities sum to one)
+    T, Hq, Hkv, d = 70, 4, 2, 16
+    q, k, v = _full_case(T, Hq, Hkv, d)
+    _, _, _, sc = oracle.full_attn_topk(q, k, v, topk=8, window=4, want_scores=True)
+    qh = _f64(q).transpose(1, 2)
+    kh = _f64(k).transpose(1, 2).repeat_interleave(Hq // Hkv, dim=1)
+    z = torch.matmul(qh, kh.transpose(-1, -2)) / math.sqrt(d)
+    z = z.masked_fill(~torch.ones(T, T, dtype=torch.bool).tril(), float("-inf"))
+    ref = torch.softmax(z, dim=-1).sum(dim=1)[0].numpy()
+    np.testing.assert_allclose(sc, ref, atol=1e-12)
+    np.testing.assert_allclose(sc.sum(axis=1), Hq, atol=1e-12)
+
+
+@pytest.mark.parametrize("topk,window", [(8, 4), (5, 0), (30, 40), (1, 1)])
+def test_full_attn_indexer_selection_matches_lexsort(topk, window):
+    T, Hq, Hkv, d = 70, 4, 2, 16
+    q, k, v = _full_case(T, Hq, Hkv, d)
+    k = k.clone()
+    k[0, 20] = k[0, 10]          # duplicated keys: exactly equal scores, lower index first
+    k[0, 33] = k[0, 10]
+    _, _, idx, sc = oracle.full_attn_topk(q, k, v, topk=topk, window=window, want_scores=True)
+    assert np.all(sc[:, 10][34:] == sc[:, 20][34:]) and np.all(sc[:, 20][34:] == sc[:, 33][34:])
+    np.testing.assert_array_equal(idx, _select_ref(sc, T, topk, window))
+
+
+def test_full_attn_indexer_picks_planted_key():
+    # a key that every head's query points at collects most of each row's
+    # probability and is chosen by every later query
+    T, Hq, Hkv, d = 64, 4, 1, 16
+    q, k, v = _full_case(T, Hq, Hkv, d, seed=62)
+    q = q.clone()
+    k = k.clone()
+    direction = torch.zeros(d)
+    direction[3] = 1.0
+    k[0, 7, 0] = (direction * 8).to(torch.bfloat16)
+    q[0, :, :] = (q[0, :, :].float() * 0.1 + direction * 4).to(torch.bfloat16)
+    _, _, idx = oracle.full_attn_topk(q, k, v, topk=2, window=2)
+    for t in range(10, T):
+        assert 7 in idx[t]
