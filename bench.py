@@ -170,7 +170,8 @@ def main():
     ap.add_argument("--nsa-seq-len", type=int, default=0,
                     help="NSA length for profiling captures of a smaller case (default 65536)")
     ap.add_argument("--workload", default="all",
-                    choices=["all", "decode128k", "indexcache_prefill", "hysparse2_prefill", "bwd64k",
+                    choices=["all", "decode128k", "indexcache_prefill", "hysparse2_prefill",
+                             "hysparse2_full_indexer", "bwd64k",
                              "nsa64k", "nsa_bwd64k", "spatial16k"],
                     help="run only one of the extra measurements (for profiling captures of a "
                          "single workload); prints its numbers alone")
@@ -542,6 +543,33 @@ def extra_measurements(args, dev, torch, api, lib, inputs, flush, world, peaks, 
             "note": "indexer top-1024 + forced window 128, then sparse attention; "
                     f"1 x {T} tokens, 16 q heads / 1 kv head, d=128"}
         del gh, ghd, hidx, hout, hws
+        torch.cuda.empty_cache()
+    # --- HySparse2's full-attention layer as the exact indexer (64K prefill) ---
+    if only in (None, "hysparse2_full_indexer"):
+        w = inputs.WORKLOADS["dsa_prefill64k"]
+        T = args.seq_len or w.T
+        gf = inputs.gen_dsa(w.B, T, w.Hq, w.Hkv, w.d, w.Hi, w.di, seed=210)
+        gfd = {k: v.to(dev) for k, v in gf.items() if k in ("q", "k", "v")}
+        fk, fw = 1024, 128
+        fout = torch.empty((w.B, T, w.Hq, w.d), dtype=torch.bfloat16, device=dev)
+        flse = torch.empty((w.B, T, w.Hq), dtype=torch.float32, device=dev)
+        fidx = torch.empty((w.B, T, fk + fw), dtype=torch.int32, device=dev)
+        fws = torch.empty(lib.sa_full_attn_topk_workspace_size(w.B, T, w.Hq, w.Hkv, w.d, fk, fw),
+                          dtype=torch.uint8, device=dev)
+
+        def fstep():
+            api.full_attn_topk(gfd["q"], gfd["k"], gfd["v"], fk, fw, out=fout, lse=flse, out_idx=fidx,
+                               workspace=fws)
+        times = timed_steps(fstep, 2, args.warmup, flush, dev, torch)
+        ms = max_over_ranks(sum(times), dev, torch, dist) / len(times)
+        pairs = T * (T + 1) / 2
+        ffl = (4.0 + 2.0) * w.d * w.Hq * pairs      # the full layer (4 d) + the score pass (2 d)
+        res[f"hysparse2_full_indexer{T // 1024}k"] = {
+            "ms_per_step": round(ms, 3), "tflops": round(world * ffl / (ms / 1e3) / 1e12, 2),
+            "algorithmic_flops": ffl,
+            "note": "full causal attention layer (out, lse) + exact head-summed probability scores + "
+                    f"window 128 / top-1024 selection; 1 x {T} tokens, 16 q heads / 1 kv head, d=128"}
+        del gf, gfd, fout, flse, fidx, fws
         torch.cuda.empty_cache()
     # --- backward of the 64K sparse attention (dq, dk, dv over the selected keys) ---
     if only in (None, "bwd64k"):

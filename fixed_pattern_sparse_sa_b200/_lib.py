@@ -17,6 +17,7 @@ EXPORTS = (
     "sa_lse_combine",
     "sa_nsa_workspace_size", "sa_nsa_fwd", "sa_nsa_fwd_train",
     "sa_nsa_bwd_workspace_size", "sa_nsa_bwd",
+    "sa_full_attn_topk_workspace_size", "sa_full_attn_topk",
     "sa_dsa_decode_layers_workspace_size", "sa_dsa_decode_layers",
     "sa_check_device_status", "sa_last_error_string", "sa_status_string",
     "sa_version", "sa_launch_counter",
@@ -81,6 +82,8 @@ def load() -> ctypes.CDLL:
             "sa_nsa_fwd": (I, [P, P, P, P, I, I, I, I, I, I, I, I, I, I, F, P, P, P, P, SZ, P]),
             "sa_nsa_fwd_train": (I, [P, P, P, P, I, I, I, I, I, I, I, I, I, I, F, P, P, P, P, P, SZ, P]),
             "sa_nsa_bwd_workspace_size": (SZ, [I, I, I, I, I, I, I]),
+            "sa_full_attn_topk_workspace_size": (SZ, [I, I, I, I, I, I, I]),
+            "sa_full_attn_topk": (I, [P, P, P, I, I, I, I, I, F, I, I, P, P, P, P, SZ, P]),
             "sa_nsa_bwd": (I, [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, I, F, P, P, P, P,
                                P, SZ, P]),
             "sa_dsa_decode_layers_workspace_size": (SZ, [I, I, I, I, I, I, I, I, I, I]),

@@ -444,6 +444,41 @@ def nsa_bwd(q, k, v, gates, dout, o_branches, lse_branches, sel_idx, cmp_len: in
     return dq, dk, dv, dg
 
 
+def full_attn_topk(q, k, v, topk: int, window: int, scale: Optional[float] = None,
+                   out=None, lse=None, out_idx=None, workspace=None):
+    """A full-attention layer as an exact indexer (sa_full_attn_topk).
+
+    q bf16 [B,T,Hq,d], k/v bf16 [B,T,Hkv,d].  Returns (out bf16 [B,T,Hq,d],
+    lse fp32 [B,T,Hq], idx int32 [B,T,topk+window]): the full layer's causal
+    attention and, for the sparse layers, the forced window plus the top-k
+    keys by the full layer's head-summed attention probabilities.
+    """
+    lib = _lib.load()
+    dev = q.device
+    _need(q, "q", torch.bfloat16, dev, 4)
+    _need(k, "k", torch.bfloat16, dev, 4)
+    _need(v, "v", torch.bfloat16, dev, 4)
+    B, T, Hq, d = q.shape
+    Hkv = k.shape[2]
+    if k.shape != (B, T, Hkv, d) or v.shape != k.shape:
+        raise ValueError("full_attn_topk: shape mismatch")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((B, T, Hq, d), dtype=torch.bfloat16, device=dev)
+    if lse is None:
+        lse = torch.empty((B, T, Hq), dtype=torch.float32, device=dev)
+    if out_idx is None:
+        out_idx = torch.empty((B, T, topk + window), dtype=torch.int32, device=dev)
+    nbytes = lib.sa_full_attn_topk_workspace_size(B, T, Hq, Hkv, d, topk, window)
+    ws = workspace if workspace is not None else _workspace(nbytes, dev)
+    with torch.cuda.device(dev):
+        check(lib.sa_full_attn_topk(_ptr(q), _ptr(k), _ptr(v), B, T, Hq, Hkv, d, float(scale), topk,
+                                    window, _ptr(out), _ptr(lse), _ptr(out_idx), _ptr(ws),
+                                    ws.numel() * ws.element_size(), _stream(dev)), "sa_full_attn_topk")
+    return out, lse, out_idx
+
+
 # --------------------------------------------------------------- IndexCache --
 def dsa_decode_layers(pattern: str, layers, topk: int, window: int = 0, n_split: int = 1,
                       q_pos0: Optional[int] = None, scale: Optional[float] = None,

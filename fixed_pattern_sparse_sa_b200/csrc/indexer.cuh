@@ -52,6 +52,8 @@ struct IdxParams {
     int32_t *out_idx;      // [B, Tq, Kout]
     int32_t *out_count;    // [B, Tq] nullable
     unsigned *err;         // device error word
+    const int32_t *dense;  // select's dense mode: [B, Rt, dense_stride] scores (non-negative)
+    long long dense_stride;
 };
 
 // Number of selectable (non-window) candidates of a query at position p.
@@ -1051,7 +1053,9 @@ __host__ __device__ constexpr int select_smem_staged(int words, int cap) {
 // threshold go to a "greater" bitmap over positions, keys equal to it to an
 // "equal" bitmap; the output takes every greater key and the lowest-position
 // equal keys, in ascending position order.
-template <int DI, int NT = SEL_THREADS>
+// DENSE: the row's scores are read from p.dense (every candidate j < n),
+// not from a candidate list or recomputed from the indexer vectors.
+template <int DI, int NT = SEL_THREADS, bool DENSE = false>
 __global__ void __launch_bounds__(NT, NT <= 256 ? 3 : 1) topk_select_kernel(const IdxParams p) {
     grid_dependency_sync();
     extern __shared__ __align__(1024) unsigned char smem[];
@@ -1089,12 +1093,12 @@ __global__ void __launch_bounds__(NT, NT <= 256 ? 3 : 1) topk_select_kernel(cons
     }
     if (k_eff == 0) return;
 
-    const int cnt = p.cand_cnt[row];
-    const bool use_list = cnt >= k_eff && cnt <= p.cand_cap;
-    if (!use_list && tid == 0) atomicAdd(&g_sa_recompute_rows, 1ull);
-    const int2 *cl = p.cand + row * p.cand_cap;
-    const int8_t *kb = p.k + (long long)b * p.L * DI;
-    if (!use_list) {
+    const int cnt = DENSE ? 0 : p.cand_cnt[row];
+    const bool use_list = !DENSE && cnt >= k_eff && cnt <= p.cand_cap;
+    if (!DENSE && !use_list && tid == 0) atomicAdd(&g_sa_recompute_rows, 1ull);
+    const int2 *cl = DENSE ? nullptr : p.cand + row * p.cand_cap;
+    const int8_t *kb = DENSE ? nullptr : p.k + (long long)b * p.L * DI;
+    if (!DENSE && !use_list) {
         // exact recompute: stage this query's indexer vectors and weights
         const int8_t *qsrc = p.q + ((long long)b * p.Tq + t) * p.Hi * DI;
         for (int i = tid; i < p.Hi * DI / 16; i += NT)
@@ -1167,6 +1171,9 @@ __global__ void __launch_bounds__(NT, NT <= 256 ? 3 : 1) topk_select_kernel(cons
                 for (int u = 0; u < U; ++u)
                     if (b0 + u * NT < cnt) f(e[u].x, e[u].y);
             }
+        } else if constexpr (DENSE) {
+            const int32_t *dr = p.dense + row * p.dense_stride;
+            for (int j = tid; j < n; j += NT) f(__ldg(dr + j), j);
         } else {
             for (int j = tid; j < n; j += NT) f(exact_score<DI>(qrow_s, w_s, p.Hi, kb + (long long)j * DI), j);
         }

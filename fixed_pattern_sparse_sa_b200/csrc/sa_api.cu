@@ -23,6 +23,7 @@
 #include "attn_cmp_tc.cuh"
 #include "attn_tile.cuh"
 #include "dist.cuh"
+#include "full_score.cuh"
 #include "indexer.cuh"
 #include "indexer_filter.cuh"
 #include "nsa_misc.cuh"
@@ -1423,6 +1424,135 @@ int sa_nsa_bwd(const void *q, const void *k, const void *v, const float *gates, 
         launch_k("nsa_pool_bwd_kernel", nsa_pool_bwd_kernel, (unsigned)((n4 + 255) / 256), 256, 0, st,
             (const float *)dkc, (const float *)dvc, dk, dv, B, T, Hkv, d, lay.nc, cmp_len, cmp_stride);
         SA_CHECK_LAUNCH("nsa_pool_bwd_kernel");
+    }
+    return SA_OK;
+}
+
+// ------------------------------------- full-attention exact indexer --
+// Query rows per score/select chunk: the chunk's dense scores stay under
+// 1 GiB.
+static int full_chunk_rows(int B, int T) {
+    const long long stride = (T + 3) / 4 * 4;
+    const long long r = (1LL << 28) / ((long long)B * stride);
+    return (int)std::max(1LL, std::min<long long>(r, T));
+}
+
+struct FullLayout {
+    int rows_chunk;
+    long long stride;
+    size_t of32_off, lse_off, dense_off, total;
+};
+
+static FullLayout full_layout(int B, int T, int Hq, int d) {
+    FullLayout lay{};
+    lay.rows_chunk = full_chunk_rows(B, T);
+    lay.stride = (T + 3) / 4 * 4;
+    const size_t rows = (size_t)B * T * Hq;
+    size_t off = 0;
+    lay.of32_off = off; off += round_up(rows * d * 4, 256);
+    lay.lse_off = off; off += round_up(rows * 4, 256);
+    lay.dense_off = off; off += round_up((size_t)B * lay.rows_chunk * lay.stride * 4, 256);
+    lay.total = off;
+    return lay;
+}
+
+size_t sa_full_attn_topk_workspace_size(int B, int T, int Hq, int Hkv, int d, int topk, int window) {
+    (void)Hkv; (void)topk; (void)window;
+    if (B <= 0 || T <= 0 || Hq <= 0 || d <= 0) return 0;
+    return full_layout(B, T, Hq, d).total;
+}
+
+template <int D>
+static int launch_full_score(const FullScoreParams &p, cudaStream_t st) {
+    constexpr int smem = full_score_smem<D>();
+    auto kern = full_score_kernel<D>;
+    int rc = set_smem(kern, smem);
+    if (rc) return rc;
+    const long long ctas = (long long)p.B * ((p.Rt + FS_WARPS - 1) / FS_WARPS);
+    if (ctas == 0) return SA_OK;
+    launch_k(__PRETTY_FUNCTION__, kern, (unsigned)ctas, FS_WARPS * 32, smem, st, p);
+    SA_CHECK_LAUNCH("full_score_kernel");
+    return SA_OK;
+}
+
+template <int NT>
+static int launch_select_dense(const IdxParams &p, int words, cudaStream_t st) {
+    const int smem = select_smem_staged<64>(words, 0);
+    auto kern = topk_select_kernel<64, NT, true>;
+    int rc = set_smem(kern, smem);
+    if (rc) return rc;
+    launch_k(__PRETTY_FUNCTION__, kern, dim3(1u, (unsigned)p.Rt, (unsigned)p.B), NT, smem, st, p);
+    SA_CHECK_LAUNCH("topk_select_kernel");
+    return SA_OK;
+}
+
+int sa_full_attn_topk(const void *q, const void *k, const void *v, int B, int T, int Hq, int Hkv, int d,
+                      float scale, int topk, int window, void *out, float *lse, int32_t *out_idx,
+                      void *workspace, size_t workspace_bytes, void *stream) {
+    SA_TRACE("sa_full_attn_topk");
+    if (B <= 0 || T < 0 || Hq <= 0 || Hkv <= 0 || topk < 0 || window < 0 || topk + window < 1)
+        return fail(SA_ERR_INVALID_ARG, "full_attn_topk: bad sizes");
+    if (Hq % Hkv) return fail(SA_ERR_INVALID_ARG, "full_attn_topk: Hq %% Hkv != 0");
+    if (d != 64 && d != 128) return fail(SA_ERR_UNSUPPORTED, "full_attn_topk: head dim %d", d);
+    if (!q || !k || !v || !out_idx || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned4(out_idx) ||
+        (out && !aligned16(out)) || (lse && !aligned4(lse)))
+        return fail(SA_ERR_INVALID_ARG, "full_attn_topk: null or misaligned pointer");
+    if (!std::isfinite(scale)) return fail(SA_ERR_INVALID_ARG, "full_attn_topk: scale");
+    if (T == 0) return SA_OK;
+    const FullLayout lay = full_layout(B, T, Hq, d);
+    if (!workspace || workspace_bytes < lay.total)
+        return fail(SA_ERR_WORKSPACE, "full_attn_topk: workspace %zu < %zu", workspace_bytes, lay.total);
+    if (!aligned16(workspace)) return fail(SA_ERR_INVALID_ARG, "full_attn_topk: workspace alignment");
+    unsigned *ew = nullptr;
+    int rc = device_error_word(&ew);
+    if (rc) return rc;
+    cudaStream_t st = as_stream(stream);
+    char *ws = static_cast<char *>(workspace);
+    float *of32 = reinterpret_cast<float *>(ws + lay.of32_off);
+    float *lse_ = lse ? lse : reinterpret_cast<float *>(ws + lay.lse_off);
+    int32_t *dense = reinterpret_cast<int32_t *>(ws + lay.dense_off);
+    const int G = Hq / Hkv;
+    const long long rows = (long long)B * T * Hq;
+    // 1. the full layer: causal attention over every earlier key (a window
+    //    as long as the sequence)
+    {
+        TileParams p{};
+        p.q = static_cast<const __nv_bfloat16 *>(q); p.k = static_cast<const __nv_bfloat16 *>(k);
+        p.v = static_cast<const __nv_bfloat16 *>(v);
+        p.B = B; p.T = T; p.Lk = T; p.Hq = Hq; p.Hkv = Hkv; p.G = G;
+        p.window = T; p.scale_log2 = scale * kLog2e;
+        p.out_f32 = of32; p.lse = lse_;
+        rc = (G <= 16 && cmp_tc_applies(p, d)) ? launch_nsa_tc<TS_WINDOW>(p, ew, st)
+                                                 : launch_tile(p, d, TS_WINDOW, st);
+        if (rc) return rc;
+        if (out) {
+            const long long n2 = rows * d / 2;
+            launch_k("f32_to_bf16_kernel", f32_to_bf16_kernel, (unsigned)((n2 + 255) / 256), 256, 0, st,
+                (const float *)of32, n2, (__nv_bfloat16 *)out);
+            SA_CHECK_LAUNCH("f32_to_bf16_kernel");
+        }
+    }
+    // 2 + 3. per chunk of query rows: exact scores, then the exact top-k
+    for (int t0 = 0; t0 < T; t0 += lay.rows_chunk) {
+        const int Rt = std::min(lay.rows_chunk, T - t0);
+        FullScoreParams fp{};
+        fp.q = static_cast<const __nv_bfloat16 *>(q); fp.k = static_cast<const __nv_bfloat16 *>(k);
+        fp.lse = lse_;
+        fp.B = B; fp.T = T; fp.Hq = Hq; fp.Hkv = Hkv; fp.G = G;
+        fp.t0 = t0; fp.Rt = Rt; fp.window = window; fp.scale_log2 = scale * kLog2e;
+        fp.dense = dense; fp.stride = lay.stride;
+        rc = d == 64 ? launch_full_score<64>(fp, st) : launch_full_score<128>(fp, st);
+        if (rc) return rc;
+        IdxParams ip{};
+        ip.B = B; ip.Tq = T; ip.L = T; ip.q_pos0 = 0; ip.window = window; ip.topk = topk;
+        ip.Kout = topk + window; ip.t0 = t0; ip.Rt = Rt;
+        ip.out_idx = out_idx; ip.out_count = nullptr; ip.err = ew;
+        ip.dense = dense; ip.dense_stride = lay.stride;
+        const long long ncand = window > 0 ? (long long)t0 + Rt - window : (long long)t0 + Rt;
+        const int words = (int)((std::max(ncand, 1LL) + 31) / 32);
+        rc = ((long long)B * Rt <= sm_count()) ? launch_select_dense<1024>(ip, words, st)
+                                                : launch_select_dense<SEL_THREADS>(ip, words, st);
+        if (rc) return rc;
     }
     return SA_OK;
 }

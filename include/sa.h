@@ -266,6 +266,38 @@ int sa_nsa_bwd(const void *q, const void *k, const void *v, const float *gates,
                void *workspace, size_t workspace_bytes, void *stream);
 
 /* --------------------------------------------------------------------------
+ * A full-attention layer as an exact indexer (HySparse2 page, "Xiaomi
+ * presenta HySparse2 ...", section "Que significa para la evolucion de la
+ * IA": a few full-attention layers compute exact scores and guide the
+ * selection of the sparse layers).
+ *  1. The full layer: causal softmax attention of every head over all keys
+ *     j <= t: out, lse.
+ *  2. Exact score of key j for query t: the probability the full layer puts
+ *     on j, summed over all Hq heads,
+ *       score(t, j) = sum_h exp(scale q_{t,h}.k_{j,g(h)} - lse_{t,h}).
+ *  3. Index set for the sparse layers (HySparse2 page, "Mas precision con
+ *     menos memoria": the most recent tokens are forced in, score-chosen ones
+ *     are added): the window {max(0, t-window+1) .. t} plus the top-k of the
+ *     other keys by (score desc, j asc); ascending, -1 padded to
+ *     topk + window, the layout of sa_indexer_topk (one set per query, shared
+ *     by all heads; feed it to sa_sparse_attn_fwd).
+ * Scores are fp32 on the device: where two keys' exact scores differ by less
+ * than fp32 rounding of the sum, the order between them may differ from the
+ * exact one.
+ *   q bf16 [B,T,Hq,d], k/v bf16 [B,T,Hkv,d]; out bf16 [B,T,Hq,d] (nullable);
+ *   lse fp32 [B,T,Hq] (nullable); out_idx int32 [B,T,topk+window].
+ * d = 64 or 128.  Workspace: sa_full_attn_topk_workspace_size bytes (the
+ * fp32 output, the LSE and the dense scores of a chunk of query rows,
+ * at most 1 GiB), 16-byte aligned.
+ * ------------------------------------------------------------------------ */
+size_t sa_full_attn_topk_workspace_size(int B, int T, int Hq, int Hkv, int d, int topk,
+                                        int window);
+int sa_full_attn_topk(const void *q, const void *k, const void *v, int B, int T, int Hq,
+                      int Hkv, int d, float scale, int topk, int window, void *out,
+                      float *lse, int32_t *out_idx, void *workspace, size_t workspace_bytes,
+                      void *stream);
+
+/* --------------------------------------------------------------------------
  * IndexCache layer driver (IndexCache page, body): layers marked 'F' run the
  * indexer and top-k and overwrite the cached index buffer; layers marked 'S'
  * skip the indexer and reuse the buffer of the nearest preceding F layer.
