@@ -81,7 +81,7 @@ def load() -> ctypes.CDLL:
             "sa_nsa_workspace_size": (SZ, [I, I, I, I, I, I, I, I, I]),
             "sa_nsa_fwd": (I, [P, P, P, P, I, I, I, I, I, I, I, I, I, I, F, P, P, P, P, SZ, P]),
             "sa_nsa_fwd_train": (I, [P, P, P, P, I, I, I, I, I, I, I, I, I, I, F, P, P, P, P, P, SZ, P]),
-            "sa_nsa_bwd_workspace_size": (SZ, [I, I, I, I, I, I, I]),
+            "sa_nsa_bwd_workspace_size": (SZ, [I, I, I, I, I, I, I, I, I]),
             "sa_full_attn_topk_workspace_size": (SZ, [I, I, I, I, I, I, I]),
             "sa_full_attn_topk": (I, [P, P, P, I, I, I, I, I, F, I, I, P, P, P, P, SZ, P]),
             "sa_nsa_bwd": (I, [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, I, F, P, P, P, P,

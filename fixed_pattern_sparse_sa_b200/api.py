@@ -434,7 +434,7 @@ def nsa_bwd(q, k, v, gates, dout, o_branches, lse_branches, sel_idx, cmp_len: in
     dk = torch.empty((B, T, Hkv, d), dtype=torch.float32, device=dev)
     dv = torch.empty((B, T, Hkv, d), dtype=torch.float32, device=dev)
     dg = torch.empty((B, T, Hq, 3), dtype=torch.float32, device=dev)
-    nbytes = lib.sa_nsa_bwd_workspace_size(B, T, Hq, Hkv, d, cmp_len, cmp_stride)
+    nbytes = lib.sa_nsa_bwd_workspace_size(B, T, Hq, Hkv, d, cmp_len, cmp_stride, sel_block, sel_topk)
     ws = _workspace(nbytes, dev)
     with torch.cuda.device(dev):
         check(lib.sa_nsa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(gates), _ptr(dout), _ptr(o_branches),

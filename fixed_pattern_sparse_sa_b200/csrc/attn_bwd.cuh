@@ -104,7 +104,8 @@ __device__ __forceinline__ void ldsm_tile16(unsigned (&a)[4], const unsigned cha
     }
 }
 
-template <int D, int NW, int SRC = BW_LIST, bool HILO = false>
+// DKV = false: dq only (the key-major attn_bwd_kv_kernel gives dk / dv).
+template <int D, int NW, int SRC = BW_LIST, bool HILO = false, bool DKV = true>
 __global__ void __launch_bounds__(NW * 32) attn_bwd_kernel(const BwdParams p) {
     grid_dependency_sync();
     constexpr int NK = 16;                  // keys per chunk
@@ -317,6 +318,7 @@ __global__ void __launch_bounds__(NW * 32) attn_bwd_kernel(const BwdParams p) {
                     mma_bf16_16816(dqa[2 * dpi + 1], dsa, b2, b3);
                 }
             }
+            if constexpr (DKV) {
             // dS and P tiles (row = head, col = key) for the transposed products
             {
                 unsigned *t0 = reinterpret_cast<unsigned *>(tp_s);
@@ -365,6 +367,7 @@ __global__ void __launch_bounds__(NW * 32) attn_bwd_kernel(const BwdParams p) {
                     }
                 }
             }
+            }   // DKV
         }
         __syncwarp();
     }
@@ -383,6 +386,340 @@ __global__ void __launch_bounds__(NW * 32) attn_bwd_kernel(const BwdParams p) {
         if (v0) *q0 = a0;
         if (v1) *q1 = a1;
     }
+}
+
+// Key-major backward of a range branch (the sliding window, or the
+// compressed rows): dK and dV of a block of KB = 16 * KV_NWK keys of one KV
+// group, summed in registers over the queries that see them, so that a key
+// gets one reduction per CTA instead of one per (query, key).  The queries
+// seeing the block are cut into splits of q_split (one CTA each).  The CTA
+// stages the block's K (and K low halves) and V once; per query and 16-head
+// chunk it stages Q_t and dO_t (two stages, cp.async) with the heads' lse,
+// D and gate.  Warp w owns keys 16w .. 16w+15: S^T = K Q_t^T and
+// dP^T = V dO_t^T (rows = keys, columns = heads), P^T and dS^T in registers,
+// dV += P^T dO_t and dK += dS^T Q_t with the C fragments reused as A
+// fragments.  dq of the branch comes from attn_bwd_kernel with DKV = false.
+constexpr int KV_NWK = 4;
+
+// Selected branch: the queries that chose each block, as lists per
+// (b, g, block) (built by the three kernels below), cut into work items of
+// at most q_split queries.
+struct KvLists {
+    const int32_t *qlist;   // queries, grouped by list
+    const int32_t *qoff;    // [n_lists + 1] list starts
+    const int2 *items;      // (list, split) work items
+    const int32_t *n_items; // device count of items
+    int nb;                 // selection blocks per sequence
+    int sel_block;
+    int n_kbpb;             // key blocks of KB keys per selection block
+};
+
+template <int D, bool HILO>
+constexpr int attn_bwd_kv_smem() {
+    return (HILO ? 3 : 2) * 16 * KV_NWK * D * 2 + 2 * ((2 * 16 * D * 2 + 3 * 16 * 4 + 1023) / 1024 * 1024);
+}
+
+// Queries that see at least one key of [j_first, j_last] (range branches).
+__device__ __forceinline__ void kv_query_range(const BwdParams &p, long long j_first, long long j_last,
+                                               long long &q_lo, long long &q_hi) {
+    if (p.window > 0) {
+        q_lo = j_first;
+        q_hi = j_last + p.window < (long long)p.Tq ? j_last + p.window : (long long)p.Tq;
+    } else {
+        q_lo = j_first * p.cmp_stride + p.cmp_len - 1;
+        q_hi = p.Tq;
+    }
+}
+
+template <int D, bool HILO, bool LISTS = false>
+__global__ void __launch_bounds__(KV_NWK * 32) attn_bwd_kv_kernel(const BwdParams p, int n_kb, int n_split,
+                                                                  int q_split, const KvLists kl) {
+    grid_dependency_sync();
+    constexpr int KB = 16 * KV_NWK;
+    constexpr int NT = KV_NWK * 32;
+    constexpr int ROWB = D * 2;
+    constexpr int UNITS = ROWB / 16;
+    constexpr int KS_D = D / 16;
+    constexpr int NT_D = D / 8;
+    constexpr int KCH = KB * ROWB;
+    constexpr int QT = 16 * ROWB;
+    constexpr int QSTAGE = (2 * QT + 3 * 16 * 4 + 1023) / 1024 * 1024;
+    extern __shared__ __align__(1024) unsigned char smem[];
+    unsigned char *k_s = smem;
+    unsigned char *v_s = smem + KCH;
+    unsigned char *l_s = smem + 2 * KCH;                    // HILO: K low halves
+    unsigned char *qst = smem + (HILO ? 3 : 2) * KCH;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int gr = lane >> 2, qc = lane & 3;
+    int b, g;
+    long long j_first, j_end, qa, qe;
+    const int32_t *ql = nullptr;
+    if constexpr (LISTS) {
+        // work item (list, split) x key block of the selection block
+        const int item = blockIdx.x / kl.n_kbpb, kbs = blockIdx.x % kl.n_kbpb;
+        if (item >= *kl.n_items) return;
+        const int2 wi = kl.items[item];
+        const int blk = wi.x % kl.nb;
+        g = (wi.x / kl.nb) % p.Hkv;
+        b = wi.x / kl.nb / p.Hkv;
+        j_first = (long long)blk * kl.sel_block + (long long)kbs * KB;
+        j_end = (long long)blk * kl.sel_block + kl.sel_block;
+        if (j_end > p.L) j_end = p.L;
+        if (j_first >= j_end) return;
+        const long long o0 = kl.qoff[wi.x], o1 = kl.qoff[wi.x + 1];
+        qa = o0 + (long long)wi.y * q_split;
+        qe = qa + q_split < o1 ? qa + q_split : o1;
+        ql = kl.qlist;
+    } else {
+        long long rem = blockIdx.x;
+        const int s = (int)(rem % n_split); rem /= n_split;
+        const int kb = (int)(rem % n_kb); rem /= n_kb;
+        g = (int)(rem % p.Hkv); rem /= p.Hkv;
+        b = (int)rem;
+        j_first = (long long)kb * KB;
+        if (j_first >= p.L) return;
+        j_end = j_first + KB < (long long)p.L ? j_first + KB : (long long)p.L;
+        long long q_lo, q_hi;
+        kv_query_range(p, j_first, j_end - 1, q_lo, q_hi);
+        qa = q_lo + (long long)s * q_split;
+        qe = qa + q_split < q_hi ? qa + q_split : q_hi;
+    }
+    if (qa >= qe) return;                                   // the whole CTA leaves together
+    const int n_hc = (p.G + 15) / 16;
+    const int n_it = (int)(qe - qa) * n_hc;
+
+    // the key block (rows past L are zero)
+    const long long rstride = (long long)p.Hkv * D;
+    const __nv_bfloat16 *kbase = p.k + ((long long)b * p.L * p.Hkv + g) * D;
+    const __nv_bfloat16 *vbase = p.v + ((long long)b * p.L * p.Hkv + g) * D;
+    const __nv_bfloat16 *lbase = HILO ? p.klo + ((long long)b * p.L * p.Hkv + g) * D : nullptr;
+    for (int i = threadIdx.x; i < KB * UNITS; i += NT) {
+        const int r = i / UNITS, u = i % UNITS;
+        const long long j = j_first + r;
+        const bool ok = j < j_end;
+        const long long off = ok ? j * rstride + u * 8 : 0;
+        const int sw = (u ^ (r & 7)) * 16;
+        cp_async16(k_s + r * ROWB + sw, kbase + off, ok ? 16 : 0);
+        cp_async16(v_s + r * ROWB + sw, vbase + off, ok ? 16 : 0);
+        if constexpr (HILO) cp_async16(l_s + r * ROWB + sw, lbase + off, ok ? 16 : 0);
+    }
+
+    // one query stage: Q_t and dO_t of 16 heads, then lse2 / D / gate of the heads
+    auto issue = [&](int it) {
+        if (it < n_it) {
+            const long long t = LISTS ? (long long)__ldg(ql + qa + it / n_hc) : qa + it / n_hc;
+            const int hc = it % n_hc;
+            unsigned char *st = qst + (it & 1) * QSTAGE;
+            float *fs = reinterpret_cast<float *>(st + 2 * QT);
+            const long long row0 = ((long long)b * p.Tq + t) * p.Hq + (long long)g * p.G + hc * 16;
+            for (int i = threadIdx.x; i < 16 * UNITS; i += NT) {
+                const int r = i / UNITS, u = i % UNITS;
+                const bool ok = hc * 16 + r < p.G;
+                const long long src = (row0 + r) * D + u * 8;
+                const int sw = (u ^ (r & 7)) * 16;
+                cp_async16(st + r * ROWB + sw, ok ? p.q + src : p.q, ok ? 16 : 0);
+                cp_async16(st + QT + r * ROWB + sw, ok ? p.dout + src : p.dout, ok ? 16 : 0);
+            }
+            if (threadIdx.x < 16) {
+                const int r = threadIdx.x;
+                const bool ok = hc * 16 + r < p.G;
+                const long long row = row0 + r;
+                const float l = ok ? p.lse[row * p.lse_stride] : -INFINITY;
+                // a head with no key (lse = -inf) or past the group gets P = 0
+                fs[r] = l != -INFINITY ? l * kLog2e : INFINITY;
+                fs[16 + r] = ok ? p.Dt[row] : 0.f;
+                fs[32 + r] = ok ? (p.gate ? p.gate[row * p.gate_stride] : 1.f) : 0.f;
+            }
+        }
+        cp_async_commit();
+    };
+
+    float dka[NT_D][4], dva[NT_D][4];
+#pragma unroll
+    for (int i = 0; i < NT_D; ++i) {
+        dka[i][0] = dka[i][1] = dka[i][2] = dka[i][3] = 0.f;
+        dva[i][0] = dva[i][1] = dva[i][2] = dva[i][3] = 0.f;
+    }
+    const long long jk0 = j_first + warp * 16 + gr, jk1 = jk0 + 8;
+    const unsigned char *kw = k_s + warp * 16 * ROWB;
+    const unsigned char *vw = v_s + warp * 16 * ROWB;
+    const unsigned char *lw = l_s + warp * 16 * ROWB;
+
+    issue(0);
+    for (int it = 0; it < n_it; ++it) {
+        issue(it + 1);
+        cp_async_wait<1>();
+        __syncthreads();
+        const long long t = LISTS ? (long long)__ldg(ql + qa + it / n_hc) : qa + it / n_hc;
+        const unsigned char *q_t = qst + (it & 1) * QSTAGE;
+        const unsigned char *do_t = q_t + QT;
+        const float *fs = reinterpret_cast<const float *>(q_t + 2 * QT);
+        auto visible = [&](long long j) -> bool {
+            if (j >= j_end) return false;
+            if (LISTS) return j <= t;
+            if (p.window > 0) return j <= t && j > t - p.window;
+            return j * p.cmp_stride + p.cmp_len - 1 <= t;
+        };
+        const bool vk0 = visible(jk0), vk1 = visible(jk1);
+        if (__any_sync(0xffffffffu, vk0 || vk1)) {
+            float sc[2][4], dp[2][4];
+#pragma unroll
+            for (int i = 0; i < 2; ++i) sc[i][0] = sc[i][1] = sc[i][2] = sc[i][3] = dp[i][0] = dp[i][1] = dp[i][2] = dp[i][3] = 0.f;
+            const int mi = lane >> 3, ri = lane & 7;
+#pragma unroll
+            for (int ks = 0; ks < KS_D; ++ks) {
+                unsigned ka[4], va[4];
+                {
+                    // A fragments: the warp's 16 keys (rows) for k-step ks
+                    const int row = (mi & 1) * 8 + ri, unit = ks * 2 + (mi >> 1);
+                    ldsm_x4(ka[0], ka[1], ka[2], ka[3], kw + row * ROWB + ((unit ^ (row & 7)) * 16));
+                    ldsm_x4(va[0], va[1], va[2], va[3], vw + row * ROWB + ((unit ^ (row & 7)) * 16));
+                }
+                // B fragments: the 16 heads of Q_t / dO_t (columns)
+                const int hrow = (mi >> 1) * 8 + ri;
+                const int unit = ks * 2 + (mi & 1);
+                unsigned b0, b1, b2, b3;
+                ldsm_x4(b0, b1, b2, b3, q_t + hrow * ROWB + ((unit ^ (hrow & 7)) * 16));
+                mma_bf16_16816(sc[0], ka, b0, b1);
+                mma_bf16_16816(sc[1], ka, b2, b3);
+                if constexpr (HILO) {
+                    unsigned la[4];
+                    const int row = (mi & 1) * 8 + ri, unit2 = ks * 2 + (mi >> 1);
+                    ldsm_x4(la[0], la[1], la[2], la[3], lw + row * ROWB + ((unit2 ^ (row & 7)) * 16));
+                    mma_bf16_16816(sc[0], la, b0, b1);
+                    mma_bf16_16816(sc[1], la, b2, b3);
+                }
+                ldsm_x4(b0, b1, b2, b3, do_t + hrow * ROWB + ((unit ^ (hrow & 7)) * 16));
+                mma_bf16_16816(dp[0], va, b0, b1);
+                mma_bf16_16816(dp[1], va, b2, b3);
+            }
+            // P^T (gate folded in) and dS^T: rows = keys gr / gr+8, columns = heads
+            float pg[2][4], ds[2][4];
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int h = nt * 8 + 2 * qc + (e & 1);
+                    const bool vk = (e >> 1) ? vk1 : vk0;
+                    const float pv = vk ? exp2f(sc[nt][e] * p.scale_log2 - fs[h]) : 0.f;
+                    const float gv = pv * fs[32 + h];
+                    pg[nt][e] = gv;
+                    ds[nt][e] = gv * (dp[nt][e] - fs[16 + h]);
+                }
+            }
+            unsigned pa[4], dsa[4];
+            pa[0] = pack_bf16(pg[0][0], pg[0][1]); pa[1] = pack_bf16(pg[0][2], pg[0][3]);
+            pa[2] = pack_bf16(pg[1][0], pg[1][1]); pa[3] = pack_bf16(pg[1][2], pg[1][3]);
+            dsa[0] = pack_bf16(ds[0][0], ds[0][1]); dsa[1] = pack_bf16(ds[0][2], ds[0][3]);
+            dsa[2] = pack_bf16(ds[1][0], ds[1][1]); dsa[3] = pack_bf16(ds[1][2], ds[1][3]);
+            // dV += P^T dO_t, dK += dS^T Q_t (B = the [head][d] tiles, transposed loads)
+#pragma unroll
+            for (int dpi = 0; dpi < NT_D / 2; ++dpi) {
+                const int hrow = (mi & 1) * 8 + ri;
+                const int unit = dpi * 2 + (mi >> 1);
+                unsigned b0, b1, b2, b3;
+                ldsm_x4_t(b0, b1, b2, b3, do_t + hrow * ROWB + ((unit ^ (hrow & 7)) * 16));
+                mma_bf16_16816(dva[2 * dpi], pa, b0, b1);
+                mma_bf16_16816(dva[2 * dpi + 1], pa, b2, b3);
+                ldsm_x4_t(b0, b1, b2, b3, q_t + hrow * ROWB + ((unit ^ (hrow & 7)) * 16));
+                mma_bf16_16816(dka[2 * dpi], dsa, b0, b1);
+                mma_bf16_16816(dka[2 * dpi + 1], dsa, b2, b3);
+            }
+        }
+        __syncthreads();
+    }
+    cp_async_wait<0>();
+    // one reduction per key and column for this CTA's queries
+    float *dk0 = p.dk + ((long long)(b * (long long)p.L + (jk0 < j_end ? jk0 : 0)) * p.Hkv + g) * D;
+    float *dk1 = p.dk + ((long long)(b * (long long)p.L + (jk1 < j_end ? jk1 : 0)) * p.Hkv + g) * D;
+    float *dv0 = p.dv + ((long long)(b * (long long)p.L + (jk0 < j_end ? jk0 : 0)) * p.Hkv + g) * D;
+    float *dv1 = p.dv + ((long long)(b * (long long)p.L + (jk1 < j_end ? jk1 : 0)) * p.Hkv + g) * D;
+#pragma unroll
+    for (int nt = 0; nt < NT_D; ++nt) {
+        const int col = nt * 8 + 2 * qc;
+        if (jk0 < j_end) {
+            red_add2(dk0 + col, dka[nt][0] * p.scale, dka[nt][1] * p.scale);
+            red_add2(dv0 + col, dva[nt][0], dva[nt][1]);
+        }
+        if (jk1 < j_end) {
+            red_add2(dk1 + col, dka[nt][2] * p.scale, dka[nt][3] * p.scale);
+            red_add2(dv1 + col, dva[nt][2], dva[nt][3]);
+        }
+    }
+}
+
+// Inverse of the block choice: per (b, g, block) the queries that chose it.
+// 1. counts per list
+__global__ void __launch_bounds__(256) bwd_sel_count_kernel(const int32_t *__restrict__ sel, long long n_entries,
+                                                            int T, int Hkv, int K, int nb, int32_t *__restrict__ cnt) {
+    grid_dependency_sync();
+    const long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (e >= n_entries) return;
+    const int blk = sel[e];
+    if (blk < 0 || blk >= nb) return;
+    const long long bt_g = e / K;                  // (b, t, g)
+    const int g = (int)(bt_g % Hkv);
+    const long long b = bt_g / Hkv / T;
+    atomicAdd(cnt + (b * Hkv + g) * nb + blk, 1);
+}
+
+// 2. one CTA: list starts (exclusive scan of the counts), fill cursors, and
+//    the (list, split) work items of at most q_split queries each
+__global__ void __launch_bounds__(1024) bwd_sel_scan_kernel(const int32_t *__restrict__ cnt, int n_lists,
+                                                            int q_split, int32_t *__restrict__ qoff,
+                                                            int32_t *__restrict__ cursor, int2 *__restrict__ items,
+                                                            int32_t *__restrict__ n_items) {
+    grid_dependency_sync();
+    __shared__ int s_off[1024], s_it[1024];
+    __shared__ int carry_off, carry_it;
+    if (threadIdx.x == 0) { carry_off = 0; carry_it = 0; }
+    __syncthreads();
+    for (int base = 0; base < n_lists; base += 1024) {
+        const int l = base + threadIdx.x;
+        const int c = l < n_lists ? cnt[l] : 0;
+        const int ni = (c + q_split - 1) / q_split;
+        s_off[threadIdx.x] = c;
+        s_it[threadIdx.x] = ni;
+        __syncthreads();
+        for (int o = 1; o < 1024; o <<= 1) {          // inclusive scans (Hillis-Steele)
+            const int a = threadIdx.x >= o ? s_off[threadIdx.x - o] : 0;
+            const int bb = threadIdx.x >= o ? s_it[threadIdx.x - o] : 0;
+            __syncthreads();
+            s_off[threadIdx.x] += a;
+            s_it[threadIdx.x] += bb;
+            __syncthreads();
+        }
+        const int off = carry_off + s_off[threadIdx.x] - c;
+        const int it0 = carry_it + s_it[threadIdx.x] - ni;
+        if (l < n_lists) {
+            qoff[l] = off;
+            cursor[l] = off;
+            for (int s = 0; s < ni; ++s) items[it0 + s] = make_int2(l, s);
+        }
+        __syncthreads();
+        if (threadIdx.x == 1023) { carry_off += s_off[1023]; carry_it += s_it[1023]; }
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) { qoff[n_lists] = carry_off; *n_items = carry_it; }
+}
+
+// 3. the queries into their lists (order inside a list is not fixed)
+__global__ void __launch_bounds__(256) bwd_sel_fill_kernel(const int32_t *__restrict__ sel, long long n_entries,
+                                                           int T, int Hkv, int K, int nb,
+                                                           int32_t *__restrict__ cursor, int32_t *__restrict__ qlist) {
+    grid_dependency_sync();
+    const long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (e >= n_entries) return;
+    const int blk = sel[e];
+    if (blk < 0 || blk >= nb) return;
+    const long long bt_g = e / K;
+    const int g = (int)(bt_g % Hkv);
+    const long long bt = bt_g / Hkv;
+    const int t = (int)(bt % T);
+    const long long b = bt / T;
+    const int pos = atomicAdd(cursor + (b * Hkv + g) * nb + blk, 1);
+    qlist[pos] = t;
 }
 
 template <int D, int NW, bool HILO = false>

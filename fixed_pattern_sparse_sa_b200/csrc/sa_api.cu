@@ -1278,14 +1278,23 @@ int sa_nsa_fwd_train(const void *q, const void *k, const void *v, const float *g
 }
 
 // ------------------------------------------------------------ NSA backward --
+constexpr int KV_SEL_SPLIT = 256;     // queries per work item of the selected branch's key-major pass
+
 struct NsaBwdLayout {
-    int nc;
-    size_t kc_off, klo_off, vc_off, dkc_off, dvc_off, dt_off, total;
+    int nc, nb;
+    long long n_lists, n_entries, max_items;
+    size_t kc_off, klo_off, vc_off, dkc_off, dvc_off, dt_off;
+    size_t cnt_off, qoff_off, cur_off, items_off, nitems_off, qlist_off, total;
 };
 
-static NsaBwdLayout nsa_bwd_layout(int B, int T, int Hq, int Hkv, int d, int cmp_len, int cmp_stride) {
+static NsaBwdLayout nsa_bwd_layout(int B, int T, int Hq, int Hkv, int d, int cmp_len, int cmp_stride,
+                                   int sel_block, int sel_topk) {
     NsaBwdLayout lay{};
     lay.nc = T >= cmp_len ? (T - cmp_len) / cmp_stride + 1 : 0;
+    lay.nb = (T + sel_block - 1) / sel_block;
+    lay.n_lists = (long long)B * Hkv * lay.nb;
+    lay.n_entries = (long long)B * T * Hkv * sel_topk;
+    lay.max_items = lay.n_lists + (lay.n_entries + KV_SEL_SPLIT - 1) / KV_SEL_SPLIT;
     const size_t crow = (size_t)B * std::max(lay.nc, 1) * Hkv * d;
     size_t off = 0;
     lay.kc_off = off; off += round_up(crow * 2, 256);
@@ -1294,21 +1303,30 @@ static NsaBwdLayout nsa_bwd_layout(int B, int T, int Hq, int Hkv, int d, int cmp
     lay.dkc_off = off; off += round_up(crow * 4, 256);
     lay.dvc_off = off; off += round_up(crow * 4, 256);
     lay.dt_off = off; off += round_up((size_t)3 * B * T * Hq * 4, 256);
+    lay.cnt_off = off; off += round_up((size_t)lay.n_lists * 4, 256);
+    lay.qoff_off = off; off += round_up((size_t)(lay.n_lists + 1) * 4, 256);
+    lay.cur_off = off; off += round_up((size_t)lay.n_lists * 4, 256);
+    lay.items_off = off; off += round_up((size_t)lay.max_items * 8, 256);
+    lay.nitems_off = off; off += 256;
+    lay.qlist_off = off; off += round_up((size_t)lay.n_entries * 4, 256);
     lay.total = off;
     return lay;
 }
 
-size_t sa_nsa_bwd_workspace_size(int B, int T, int Hq, int Hkv, int d, int cmp_len, int cmp_stride) {
-    if (B <= 0 || T <= 0 || Hq <= 0 || Hkv <= 0 || d <= 0 || cmp_len <= 0 || cmp_stride <= 0) return 0;
-    return nsa_bwd_layout(B, T, Hq, Hkv, d, cmp_len, cmp_stride).total;
+size_t sa_nsa_bwd_workspace_size(int B, int T, int Hq, int Hkv, int d, int cmp_len, int cmp_stride,
+                                 int sel_block, int sel_topk) {
+    if (B <= 0 || T <= 0 || Hq <= 0 || Hkv <= 0 || d <= 0 || cmp_len <= 0 || cmp_stride <= 0 ||
+        sel_block <= 0 || sel_topk <= 0)
+        return 0;
+    return nsa_bwd_layout(B, T, Hq, Hkv, d, cmp_len, cmp_stride, sel_block, sel_topk).total;
 }
 
-template <int D, int SRC, bool HILO>
+template <int D, int SRC, bool HILO, bool DKV = true>
 static int launch_bwd_branch(const BwdParams &p, cudaStream_t st) {
     constexpr int NW = (HILO && D == 128) ? 6 : 8;    // shared memory: 3 arrays per stage with HILO
     constexpr int smem = attn_bwd_smem_bytes<D, NW, HILO>();
     static_assert(smem <= 227 * 1024, "shared memory");
-    auto kern = attn_bwd_kernel<D, NW, SRC, HILO>;
+    auto kern = attn_bwd_kernel<D, NW, SRC, HILO, DKV>;
     int rc = set_smem(kern, smem);
     if (rc) return rc;
     const long long items = (long long)p.B * p.Tq * p.Hkv * ((p.G + 15) / 16);
@@ -1318,11 +1336,71 @@ static int launch_bwd_branch(const BwdParams &p, cudaStream_t st) {
     return SA_OK;
 }
 
+// Key-major dK / dV of a range branch (window, or compressed rows).
+template <int D, bool HILO>
+static int launch_bwd_kv(const BwdParams &p, cudaStream_t st) {
+    if (p.L <= 0) return SA_OK;
+    constexpr int smem = attn_bwd_kv_smem<D, HILO>();
+    static_assert(smem <= 227 * 1024, "shared memory");
+    auto kern = attn_bwd_kv_kernel<D, HILO>;
+    int rc = set_smem(kern, smem);
+    if (rc) return rc;
+    constexpr int KB = 16 * KV_NWK;
+    const int n_kb = (p.L + KB - 1) / KB;
+    // queries per CTA: long ranges (compressed rows) in 512s, the window's in 256s
+    const int q_split = p.window > 0 ? 256 : 512;
+    const long long span = p.window > 0 ? (long long)KB - 1 + p.window : (long long)p.Tq;
+    const int n_split = (int)std::max(1LL, (span + q_split - 1) / q_split);
+    const long long ctas = (long long)p.B * p.Hkv * n_kb * n_split;
+    if (ctas > INT_MAX) return fail(SA_ERR_UNSUPPORTED, "attn_bwd_kv: %lld CTAs", ctas);
+    launch_k(__PRETTY_FUNCTION__, kern, (unsigned)ctas, KV_NWK * 32, smem, st, p, n_kb, n_split, q_split,
+             KvLists{});
+    SA_CHECK_LAUNCH("attn_bwd_kv_kernel");
+    return SA_OK;
+}
+
+// Key-major dK / dV of the selected branch over the inverse block lists.
+template <int D>
+static int launch_bwd_kv_lists(const BwdParams &p, const NsaBwdLayout &lay, char *ws, const int32_t *sel,
+                               int sel_block, int sel_topk, cudaStream_t st) {
+    int32_t *cnt = reinterpret_cast<int32_t *>(ws + lay.cnt_off);
+    int32_t *qoff = reinterpret_cast<int32_t *>(ws + lay.qoff_off);
+    int32_t *cur = reinterpret_cast<int32_t *>(ws + lay.cur_off);
+    int2 *items = reinterpret_cast<int2 *>(ws + lay.items_off);
+    int32_t *n_items = reinterpret_cast<int32_t *>(ws + lay.nitems_off);
+    int32_t *qlist = reinterpret_cast<int32_t *>(ws + lay.qlist_off);
+    if (lay.n_lists > INT_MAX || lay.max_items * 8 > INT_MAX) return fail(SA_ERR_UNSUPPORTED, "nsa_bwd: lists");
+    cudaError_t e = cudaMemsetAsync(cnt, 0, (size_t)lay.n_lists * 4, st);
+    if (e != cudaSuccess) return fail(SA_ERR_CUDA, "nsa_bwd memset: %s", cudaGetErrorString(e));
+    const unsigned eg = (unsigned)((lay.n_entries + 255) / 256);
+    launch_k("bwd_sel_count_kernel", bwd_sel_count_kernel, eg, 256, 0, st, sel, lay.n_entries, p.Tq, p.Hkv, sel_topk,
+             lay.nb, cnt);
+    SA_CHECK_LAUNCH("bwd_sel_count_kernel");
+    launch_k("bwd_sel_scan_kernel", bwd_sel_scan_kernel, 1u, 1024, 0, st, (const int32_t *)cnt, (int)lay.n_lists,
+             KV_SEL_SPLIT, qoff, cur, items, n_items);
+    SA_CHECK_LAUNCH("bwd_sel_scan_kernel");
+    launch_k("bwd_sel_fill_kernel", bwd_sel_fill_kernel, eg, 256, 0, st, sel, lay.n_entries, p.Tq, p.Hkv, sel_topk,
+             lay.nb, cur, qlist);
+    SA_CHECK_LAUNCH("bwd_sel_fill_kernel");
+    constexpr int smem = attn_bwd_kv_smem<D, false>();
+    auto kern = attn_bwd_kv_kernel<D, false, true>;
+    int rc = set_smem(kern, smem);
+    if (rc) return rc;
+    constexpr int KB = 16 * KV_NWK;
+    KvLists kl{qlist, qoff, items, n_items, lay.nb, sel_block, (sel_block + KB - 1) / KB};
+    const long long ctas = lay.max_items * kl.n_kbpb;
+    if (ctas > INT_MAX) return fail(SA_ERR_UNSUPPORTED, "attn_bwd_kv: %lld CTAs", ctas);
+    launch_k(__PRETTY_FUNCTION__, kern, (unsigned)ctas, KV_NWK * 32, smem, st, p, 0, 0, KV_SEL_SPLIT, kl);
+    SA_CHECK_LAUNCH("attn_bwd_kv_kernel");
+    return SA_OK;
+}
+
 template <int D>
 static int nsa_bwd_branches(const BwdParams &base, const float *gates, const float *lse3, long long rows,
-                            float *Dt, const NsaBwdLayout &lay, const __nv_bfloat16 *kc, const __nv_bfloat16 *klo,
-                            const __nv_bfloat16 *vc, float *dkc, float *dvc, const int32_t *sel, int sel_block,
-                            int sel_topk, int window, int cmp_len, int cmp_stride, cudaStream_t st) {
+                            float *Dt, const NsaBwdLayout &lay, char *ws, const __nv_bfloat16 *kc,
+                            const __nv_bfloat16 *klo, const __nv_bfloat16 *vc, float *dkc, float *dvc,
+                            const int32_t *sel, int sel_block, int sel_topk, int window, int cmp_len,
+                            int cmp_stride, cudaStream_t st) {
     // compressed branch: keys Kc (hi/lo), gradients into dKc / dVc; writes dq
     BwdParams p = base;
     p.k = kc; p.klo = klo; p.v = vc; p.L = std::max(lay.nc, 1);
@@ -1330,7 +1408,9 @@ static int nsa_bwd_branches(const BwdParams &base, const float *gates, const flo
     p.window = 0; p.cmp_len = cmp_len; p.cmp_stride = cmp_stride;
     p.dk = dkc; p.dv = dvc; p.dq_accum = 0;
     if (lay.nc == 0) p.L = 0;       // no compressed row is visible to any query
-    int rc = launch_bwd_branch<D, BW_RANGE, true>(p, st);
+    int rc = launch_bwd_branch<D, BW_RANGE, true, false>(p, st);     // dq
+    if (rc) return rc;
+    rc = launch_bwd_kv<D, true>(p, st);                             // dKc, dVc
     if (rc) return rc;
     // selected branch: keys of the chosen blocks
     p = base;
@@ -1338,13 +1418,17 @@ static int nsa_bwd_branches(const BwdParams &base, const float *gates, const flo
     p.idx = sel; p.idx_heads = base.Hkv; p.K = sel_topk; p.block = sel_block;
     p.block_shift = (sel_block & (sel_block - 1)) == 0 ? __builtin_ctz((unsigned)sel_block) : -1;
     p.dq_accum = 1;
-    rc = launch_bwd_branch<D, BW_BLOCKS, false>(p, st);
+    rc = launch_bwd_branch<D, BW_BLOCKS, false, false>(p, st);          // dq
+    if (rc) return rc;
+    rc = launch_bwd_kv_lists<D>(p, lay, ws, sel, sel_block, sel_topk, st);   // dk, dv
     if (rc) return rc;
     // window branch
     p = base;
     p.lse = lse3 + 2; p.gate = gates + 2; p.Dt = Dt + 2 * rows;
     p.window = window; p.dq_accum = 1;
-    return launch_bwd_branch<D, BW_RANGE, false>(p, st);
+    rc = launch_bwd_branch<D, BW_RANGE, false, false>(p, st);           // dq
+    if (rc) return rc;
+    return launch_bwd_kv<D, false>(p, st);                              // dk, dv
 }
 
 int sa_nsa_bwd(const void *q, const void *k, const void *v, const float *gates, const void *dout,
@@ -1366,7 +1450,7 @@ int sa_nsa_bwd(const void *q, const void *k, const void *v, const float *gates, 
     if (!std::isfinite(scale)) return fail(SA_ERR_INVALID_ARG, "nsa_bwd: scale");
     if (T == 0) return SA_OK;
     if ((long long)sel_topk * sel_block > INT_MAX / 2) return fail(SA_ERR_UNSUPPORTED, "nsa_bwd: selection size");
-    const NsaBwdLayout lay = nsa_bwd_layout(B, T, Hq, Hkv, d, cmp_len, cmp_stride);
+    const NsaBwdLayout lay = nsa_bwd_layout(B, T, Hq, Hkv, d, cmp_len, cmp_stride, sel_block, sel_topk);
     if (!workspace || workspace_bytes < lay.total)
         return fail(SA_ERR_WORKSPACE, "nsa_bwd: workspace %zu < %zu", workspace_bytes, lay.total);
     if (!aligned16(workspace)) return fail(SA_ERR_INVALID_ARG, "nsa_bwd: workspace alignment");
@@ -1413,10 +1497,10 @@ int sa_nsa_bwd(const void *q, const void *k, const void *v, const float *gates, 
     base.q_pos0 = 0; base.scale = scale; base.scale_log2 = scale * kLog2e;
     base.lse_stride = 3; base.gate_stride = 3;
     base.dq = dq; base.dk = dk; base.dv = dv; base.err = ew;
-    rc = d == 64 ? nsa_bwd_branches<64>(base, gates, lse_branches, rows, Dt, lay, kc, klo, vc, dkc, dvc, sel_idx,
-                                        sel_block, sel_topk, window, cmp_len, cmp_stride, st)
-                 : nsa_bwd_branches<128>(base, gates, lse_branches, rows, Dt, lay, kc, klo, vc, dkc, dvc, sel_idx,
-                                         sel_block, sel_topk, window, cmp_len, cmp_stride, st);
+    rc = d == 64 ? nsa_bwd_branches<64>(base, gates, lse_branches, rows, Dt, lay, ws, kc, klo, vc, dkc, dvc,
+                                        sel_idx, sel_block, sel_topk, window, cmp_len, cmp_stride, st)
+                 : nsa_bwd_branches<128>(base, gates, lse_branches, rows, Dt, lay, ws, kc, klo, vc, dkc, dvc,
+                                         sel_idx, sel_block, sel_topk, window, cmp_len, cmp_stride, st);
     if (rc) return rc;
     // 4. compressed-row gradients back to the rows they average
     if (lay.nc > 0) {

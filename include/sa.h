@@ -257,7 +257,7 @@ int sa_nsa_fwd_train(const void *q, const void *k, const void *v, const float *g
  * from sa_check_device_status).
  * ------------------------------------------------------------------------ */
 size_t sa_nsa_bwd_workspace_size(int B, int T, int Hq, int Hkv, int d, int cmp_len,
-                                 int cmp_stride);
+                                 int cmp_stride, int sel_block, int sel_topk);
 int sa_nsa_bwd(const void *q, const void *k, const void *v, const float *gates,
                const void *dout, const float *o_branches, const float *lse_branches,
                const int32_t *sel_idx, int B, int T, int Hq, int Hkv, int d,
