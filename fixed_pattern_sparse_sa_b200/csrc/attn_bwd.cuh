@@ -521,15 +521,17 @@ __global__ void __launch_bounds__(KV_NWK * 32) attn_bwd_kv_kernel(const BwdParam
                 cp_async16(st + r * ROWB + sw, ok ? p.q + src : p.q, ok ? 16 : 0);
                 cp_async16(st + QT + r * ROWB + sw, ok ? p.dout + src : p.dout, ok ? 16 : 0);
             }
-            if (threadIdx.x < 16) {
-                const int r = threadIdx.x;
+            if (threadIdx.x < 48) {
+                // lse, D and gate of the 16 heads, copied asynchronously with the
+                // tiles (zero past the group: a zero gate gives P = 0)
+                const int r = threadIdx.x & 15, which = threadIdx.x >> 4;
                 const bool ok = hc * 16 + r < p.G;
                 const long long row = row0 + r;
-                const float l = ok ? p.lse[row * p.lse_stride] : -INFINITY;
-                // a head with no key (lse = -inf) or past the group gets P = 0
-                fs[r] = l != -INFINITY ? l * kLog2e : INFINITY;
-                fs[16 + r] = ok ? p.Dt[row] : 0.f;
-                fs[32 + r] = ok ? (p.gate ? p.gate[row * p.gate_stride] : 1.f) : 0.f;
+                const float *src = which == 0 ? p.lse + row * p.lse_stride
+                                 : which == 1 ? p.Dt + row
+                                 : (p.gate ? p.gate + row * p.gate_stride : p.lse);
+                if (which == 2 && !p.gate && ok) fs[32 + r] = 1.f;
+                else cp_async4_zfill(fs + which * 16 + r, ok ? src : p.lse, ok ? 4 : 0);
             }
         }
         cp_async_commit();
@@ -594,7 +596,8 @@ __global__ void __launch_bounds__(KV_NWK * 32) attn_bwd_kv_kernel(const BwdParam
                 mma_bf16_16816(dp[0], va, b0, b1);
                 mma_bf16_16816(dp[1], va, b2, b3);
             }
-            // P^T (gate folded in) and dS^T: rows = keys gr / gr+8, columns = heads
+            // P^T (gate folded in) and dS^T: rows = keys gr / gr+8, columns = heads;
+            // a head with no key (lse = -inf) gets P = 0
             float pg[2][4], ds[2][4];
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt) {
@@ -602,7 +605,8 @@ __global__ void __launch_bounds__(KV_NWK * 32) attn_bwd_kv_kernel(const BwdParam
                 for (int e = 0; e < 4; ++e) {
                     const int h = nt * 8 + 2 * qc + (e & 1);
                     const bool vk = (e >> 1) ? vk1 : vk0;
-                    const float pv = vk ? exp2f(sc[nt][e] * p.scale_log2 - fs[h]) : 0.f;
+                    const float lh = fs[h];
+                    const float pv = (vk && lh != -INFINITY) ? exp2f(sc[nt][e] * p.scale_log2 - lh * kLog2e) : 0.f;
                     const float gv = pv * fs[32 + h];
                     pg[nt][e] = gv;
                     ds[nt][e] = gv * (dp[nt][e] - fs[16 + h]);
@@ -646,6 +650,198 @@ __global__ void __launch_bounds__(KV_NWK * 32) attn_bwd_kv_kernel(const BwdParam
             red_add2(dk1 + col, dka[nt][2] * p.scale, dka[nt][3] * p.scale);
             red_add2(dv1 + col, dva[nt][2], dva[nt][3]);
         }
+    }
+}
+
+// dq of a range branch (the window, or the compressed rows) with the keys
+// shared: a CTA = 8 consecutive queries of one KV group (one warp each, the
+// group's 16-head chunk hc); chunks of 32 keys of the union of their ranges
+// are staged once per CTA (K, K low halves, V; two stages, cp.async) and
+// every warp runs S = Q K^T, dP = dO V^T, dS = gate P (dP - D) and
+// dq += dS K on its own query (Q and dO A fragments held in registers).
+constexpr int DQ_WARPS = 8;
+constexpr int DQ_NK = 32;
+
+template <int D, bool HILO>
+constexpr int attn_bwd_dq_tile_smem() {
+    return 2 * (HILO ? 3 : 2) * DQ_NK * D * 2;
+}
+
+template <int D, bool HILO>
+__global__ void __launch_bounds__(DQ_WARPS * 32) attn_bwd_dq_tile_kernel(const BwdParams p) {
+    grid_dependency_sync();
+    constexpr int ROWB = D * 2;
+    constexpr int UNITS = ROWB / 16;
+    constexpr int KS_D = D / 16;
+    constexpr int NT_D = D / 8;
+    constexpr int NARR = HILO ? 3 : 2;
+    constexpr int CH = DQ_NK * ROWB;
+    constexpr int CP_ITERS = NARR * DQ_NK * UNITS / (DQ_WARPS * 32);
+    static_assert(CP_ITERS * DQ_WARPS * 32 == NARR * DQ_NK * UNITS, "copy split");
+    extern __shared__ __align__(1024) unsigned char smem[];
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int gr = lane >> 2, qc = lane & 3;
+    const int n_hc = (p.G + 15) / 16;
+    const int nqb = (p.Tq + DQ_WARPS - 1) / DQ_WARPS;
+    long long rem = blockIdx.x;
+    const int qb = (int)(rem % nqb); rem /= nqb;
+    const int hc = (int)(rem % n_hc); rem /= n_hc;
+    const int g = (int)(rem % p.Hkv); rem /= p.Hkv;
+    const int b = (int)rem;
+    const int t = qb * DQ_WARPS + warp;
+    const bool tv = t < p.Tq;
+    const int t_first = qb * DQ_WARPS;
+    const int t_last = min(t_first + DQ_WARPS, p.Tq) - 1;
+    // key range of a query, and the union over the CTA's queries
+    auto range_of = [&](long long tt, long long &lo, long long &hi) {
+        if (p.window > 0) {
+            lo = tt - p.window + 1 > 0 ? tt - p.window + 1 : 0;
+            hi = tt + 1;
+        } else {
+            const long long nv = tt >= p.cmp_len - 1 ? (tt - p.cmp_len + 1) / p.cmp_stride + 1 : 0;
+            lo = 0;
+            hi = nv < p.L ? nv : p.L;
+        }
+    };
+    long long u_lo, u_hi, dummy, w_lo = 0, w_hi = 0;
+    range_of(t_first, u_lo, dummy);
+    range_of(t_last, dummy, u_hi);
+    if (tv) range_of(t, w_lo, w_hi);
+    const int n_chunks = u_hi > u_lo ? (int)((u_hi - u_lo + DQ_NK - 1) / DQ_NK) : 0;
+
+    const int hr0 = hc * 16 + gr, hr1 = hr0 + 8;
+    const bool v0 = tv && hr0 < p.G, v1 = tv && hr1 < p.G;
+    const long long rowb = ((long long)b * p.Tq + (tv ? t : 0)) * p.Hq + (long long)g * p.G + hc * 16;
+    const long long row0 = rowb + gr, row1 = row0 + 8;
+    float lse0 = v0 ? p.lse[row0 * p.lse_stride] : -INFINITY, lse1 = v1 ? p.lse[row1 * p.lse_stride] : -INFINITY;
+    const bool live0 = v0 && lse0 != -INFINITY, live1 = v1 && lse1 != -INFINITY;
+    lse0 *= kLog2e; lse1 *= kLog2e;
+    const float D0 = v0 ? p.Dt[row0] : 0.f, D1 = v1 ? p.Dt[row1] : 0.f;
+    const float gs0 = (p.gate && v0) ? p.gate[row0 * p.gate_stride] : 1.f;
+    const float gs1 = (p.gate && v1) ? p.gate[row1 * p.gate_stride] : 1.f;
+    // Q and dO A fragments of the 16 heads (zero past the group)
+    unsigned qa[KS_D][4], da[KS_D][4];
+#pragma unroll
+    for (int ks = 0; ks < KS_D; ++ks) {
+        const int c0 = ks * 16 + 2 * qc;
+        const unsigned *q0 = reinterpret_cast<const unsigned *>(p.q + row0 * D + c0);
+        const unsigned *q1 = reinterpret_cast<const unsigned *>(p.q + row1 * D + c0);
+        const unsigned *d0 = reinterpret_cast<const unsigned *>(p.dout + row0 * D + c0);
+        const unsigned *d1 = reinterpret_cast<const unsigned *>(p.dout + row1 * D + c0);
+        qa[ks][0] = v0 ? __ldg(q0) : 0u; qa[ks][1] = v1 ? __ldg(q1) : 0u;
+        qa[ks][2] = v0 ? __ldg(q0 + 4) : 0u; qa[ks][3] = v1 ? __ldg(q1 + 4) : 0u;
+        da[ks][0] = v0 ? __ldg(d0) : 0u; da[ks][1] = v1 ? __ldg(d1) : 0u;
+        da[ks][2] = v0 ? __ldg(d0 + 4) : 0u; da[ks][3] = v1 ? __ldg(d1 + 4) : 0u;
+    }
+
+    const long long rstride = (long long)p.Hkv * D;
+    const __nv_bfloat16 *kbase = p.k + ((long long)b * p.L * p.Hkv + g) * D;
+    const __nv_bfloat16 *vbase = p.v + ((long long)b * p.L * p.Hkv + g) * D;
+    const __nv_bfloat16 *lbase = HILO ? p.klo + ((long long)b * p.L * p.Hkv + g) * D : nullptr;
+    auto issue = [&](int ci) {
+        if (ci < n_chunks) {
+            unsigned char *st = smem + (ci & 1) * NARR * CH;
+#pragma unroll
+            for (int it = 0; it < CP_ITERS; ++it) {
+                const int lin = (it * DQ_WARPS + warp) * 32 + lane;
+                const int arr = lin / (DQ_NK * UNITS);
+                const int rr = (lin / UNITS) % DQ_NK, u = lin % UNITS;
+                const long long j = u_lo + (long long)ci * DQ_NK + rr;
+                const bool ok = j < u_hi;
+                const __nv_bfloat16 *src = arr == 0 ? kbase : (arr == 1 ? vbase : lbase);
+                cp_async16(st + arr * CH + rr * ROWB + ((u ^ (rr & 7)) * 16),
+                           ok ? src + j * rstride + u * 8 : kbase, ok ? 16 : 0);
+            }
+        }
+        cp_async_commit();
+    };
+
+    float dqa[NT_D][4];
+#pragma unroll
+    for (int i = 0; i < NT_D; ++i) dqa[i][0] = dqa[i][1] = dqa[i][2] = dqa[i][3] = 0.f;
+    issue(0);
+    for (int ci = 0; ci < n_chunks; ++ci) {
+        issue(ci + 1);
+        cp_async_wait<1>();
+        __syncthreads();
+        const long long j0 = u_lo + (long long)ci * DQ_NK;
+        if (tv && j0 < w_hi && j0 + DQ_NK > w_lo) {
+            const unsigned char *ks_ = smem + (ci & 1) * NARR * CH;
+            const unsigned char *vs_ = ks_ + CH;
+            const unsigned char *ls_ = vs_ + CH;
+            const int mi = lane >> 3, ri = lane & 7;
+#pragma unroll
+            for (int kh = 0; kh < DQ_NK / 16; ++kh) {
+                float sc[2][4], dp[2][4];
+#pragma unroll
+                for (int i = 0; i < 2; ++i) sc[i][0] = sc[i][1] = sc[i][2] = sc[i][3] = dp[i][0] = dp[i][1] = dp[i][2] = dp[i][3] = 0.f;
+                const int key = kh * 16 + (mi >> 1) * 8 + ri;
+#pragma unroll
+                for (int ks = 0; ks < KS_D; ++ks) {
+                    const int unit = ks * 2 + (mi & 1);
+                    unsigned b0, b1, b2, b3;
+                    ldsm_x4(b0, b1, b2, b3, ks_ + key * ROWB + ((unit ^ (key & 7)) * 16));
+                    mma_bf16_16816(sc[0], qa[ks], b0, b1);
+                    mma_bf16_16816(sc[1], qa[ks], b2, b3);
+                    if constexpr (HILO) {
+                        ldsm_x4(b0, b1, b2, b3, ls_ + key * ROWB + ((unit ^ (key & 7)) * 16));
+                        mma_bf16_16816(sc[0], qa[ks], b0, b1);
+                        mma_bf16_16816(sc[1], qa[ks], b2, b3);
+                    }
+                    ldsm_x4(b0, b1, b2, b3, vs_ + key * ROWB + ((unit ^ (key & 7)) * 16));
+                    mma_bf16_16816(dp[0], da[ks], b0, b1);
+                    mma_bf16_16816(dp[1], da[ks], b2, b3);
+                }
+                // dS = gate P (dP - D) over this query's own range
+                float ds[2][4];
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const long long j = j0 + kh * 16 + nt * 8 + 2 * qc + (e & 1);
+                        const bool hi = e >> 1;
+                        const bool ok = j >= w_lo && j < w_hi && (hi ? live1 : live0);
+                        const float pv = ok ? exp2f(sc[nt][e] * p.scale_log2 - (hi ? lse1 : lse0)) : 0.f;
+                        ds[nt][e] = pv * (hi ? gs1 : gs0) * (dp[nt][e] - (hi ? D1 : D0));
+                    }
+                }
+                unsigned dsa[4];
+                dsa[0] = pack_bf16(ds[0][0], ds[0][1]); dsa[1] = pack_bf16(ds[0][2], ds[0][3]);
+                dsa[2] = pack_bf16(ds[1][0], ds[1][1]); dsa[3] = pack_bf16(ds[1][2], ds[1][3]);
+                // dq += dS K (B = K rows [key][d], transposed loads)
+#pragma unroll
+                for (int dpi = 0; dpi < NT_D / 2; ++dpi) {
+                    const int krow = kh * 16 + (mi & 1) * 8 + ri;
+                    const int unit = dpi * 2 + (mi >> 1);
+                    unsigned b0, b1, b2, b3;
+                    ldsm_x4_t(b0, b1, b2, b3, ks_ + krow * ROWB + ((unit ^ (krow & 7)) * 16));
+                    mma_bf16_16816(dqa[2 * dpi], dsa, b0, b1);
+                    mma_bf16_16816(dqa[2 * dpi + 1], dsa, b2, b3);
+                    if constexpr (HILO) {
+                        ldsm_x4_t(b0, b1, b2, b3, ls_ + krow * ROWB + ((unit ^ (krow & 7)) * 16));
+                        mma_bf16_16816(dqa[2 * dpi], dsa, b0, b1);
+                        mma_bf16_16816(dqa[2 * dpi + 1], dsa, b2, b3);
+                    }
+                }
+            }
+        }
+        __syncthreads();
+    }
+    cp_async_wait<0>();
+#pragma unroll
+    for (int nt = 0; nt < NT_D; ++nt) {
+        const int col = nt * 8 + 2 * qc;
+        float2 a0 = make_float2(dqa[nt][0] * p.scale, dqa[nt][1] * p.scale);
+        float2 a1 = make_float2(dqa[nt][2] * p.scale, dqa[nt][3] * p.scale);
+        float2 *q0 = reinterpret_cast<float2 *>(p.dq + row0 * D + col);
+        float2 *q1 = reinterpret_cast<float2 *>(p.dq + row1 * D + col);
+        if (p.dq_accum) {
+            if (v0) { const float2 o = *q0; a0.x += o.x; a0.y += o.y; }
+            if (v1) { const float2 o = *q1; a1.x += o.x; a1.y += o.y; }
+        }
+        if (v0) *q0 = a0;
+        if (v1) *q1 = a1;
     }
 }
 

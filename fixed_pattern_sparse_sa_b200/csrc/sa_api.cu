@@ -1336,6 +1336,21 @@ static int launch_bwd_branch(const BwdParams &p, cudaStream_t st) {
     return SA_OK;
 }
 
+// dq of a range branch with the key chunks shared by 8 consecutive queries.
+template <int D, bool HILO>
+static int launch_bwd_dq_tile(const BwdParams &p, cudaStream_t st) {
+    constexpr int smem = attn_bwd_dq_tile_smem<D, HILO>();
+    auto kern = attn_bwd_dq_tile_kernel<D, HILO>;
+    int rc = set_smem(kern, smem);
+    if (rc) return rc;
+    const long long ctas = (long long)p.B * p.Hkv * ((p.G + 15) / 16) * ((p.Tq + DQ_WARPS - 1) / DQ_WARPS);
+    if (ctas == 0) return SA_OK;
+    if (ctas > INT_MAX) return fail(SA_ERR_UNSUPPORTED, "attn_bwd_dq: %lld CTAs", ctas);
+    launch_k(__PRETTY_FUNCTION__, kern, (unsigned)ctas, DQ_WARPS * 32, smem, st, p);
+    SA_CHECK_LAUNCH("attn_bwd_dq_tile_kernel");
+    return SA_OK;
+}
+
 // Key-major dK / dV of a range branch (window, or compressed rows).
 template <int D, bool HILO>
 static int launch_bwd_kv(const BwdParams &p, cudaStream_t st) {
@@ -1408,7 +1423,7 @@ static int nsa_bwd_branches(const BwdParams &base, const float *gates, const flo
     p.window = 0; p.cmp_len = cmp_len; p.cmp_stride = cmp_stride;
     p.dk = dkc; p.dv = dvc; p.dq_accum = 0;
     if (lay.nc == 0) p.L = 0;       // no compressed row is visible to any query
-    int rc = launch_bwd_branch<D, BW_RANGE, true, false>(p, st);     // dq
+    int rc = launch_bwd_dq_tile<D, true>(p, st);                     // dq
     if (rc) return rc;
     rc = launch_bwd_kv<D, true>(p, st);                             // dKc, dVc
     if (rc) return rc;
@@ -1426,7 +1441,7 @@ static int nsa_bwd_branches(const BwdParams &base, const float *gates, const flo
     p = base;
     p.lse = lse3 + 2; p.gate = gates + 2; p.Dt = Dt + 2 * rows;
     p.window = window; p.dq_accum = 1;
-    rc = launch_bwd_branch<D, BW_RANGE, false, false>(p, st);           // dq
+    rc = launch_bwd_dq_tile<D, false>(p, st);                          // dq
     if (rc) return rc;
     return launch_bwd_kv<D, false>(p, st);                              // dk, dv
 }
