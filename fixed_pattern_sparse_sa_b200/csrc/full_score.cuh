@@ -52,7 +52,7 @@ __device__ __forceinline__ long long fs_candidates(long long t, int window) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(FS_WARPS * 32) full_score_kernel(const FullScoreParams p) {
+__global__ void __launch_bounds__(FS_WARPS * 32, 2) full_score_kernel(const FullScoreParams p) {
     grid_dependency_sync();
     constexpr int ROWB = D * 2;
     constexpr int UNITS = ROWB / 16;
@@ -79,8 +79,26 @@ __global__ void __launch_bounds__(FS_WARPS * 32) full_score_kernel(const FullSco
     const int n_hc = (p.G + 15) / 16;
     int32_t *drow = p.dense + ((long long)b * p.Rt + (valid ? tr : 0)) * p.stride;
 
+    // Q A fragments of a 16-head chunk (rows past the group are zero)
+    auto load_q = [&](int g, int hc, unsigned (&qa)[KS_D][4]) {
+        const int h0 = g * p.G + hc * 16;
+        const bool r0 = hc * 16 + gr < p.G, r1 = hc * 16 + gr + 8 < p.G;
+        const __nv_bfloat16 *qrow = p.q + ((long long)(b * p.T + (valid ? t : 0)) * p.Hq + h0) * D;
+#pragma unroll
+        for (int ks = 0; ks < KS_D; ++ks) {
+            const int c0 = ks * 16 + 2 * qc;
+            qa[ks][0] = r0 ? __ldg(reinterpret_cast<const unsigned *>(qrow + (long long)gr * D + c0)) : 0u;
+            qa[ks][1] = r1 ? __ldg(reinterpret_cast<const unsigned *>(qrow + (long long)(gr + 8) * D + c0)) : 0u;
+            qa[ks][2] = r0 ? __ldg(reinterpret_cast<const unsigned *>(qrow + (long long)gr * D + c0 + 8)) : 0u;
+            qa[ks][3] = r1 ? __ldg(reinterpret_cast<const unsigned *>(qrow + (long long)(gr + 8) * D + c0 + 8)) : 0u;
+        }
+    };
+    unsigned qa[KS_D][4];
+
     for (int g = 0; g < p.Hkv; ++g) {
         const __nv_bfloat16 *kb = p.k + ((long long)b * p.T * p.Hkv + g) * D;
+        // one head chunk (G <= 16): its fragments stay in registers for the whole key loop
+        if (n_hc == 1 && valid) load_q(g, 0, qa);
         const long long rstride = (long long)p.Hkv * D;
         auto issue = [&](int ci) {
             if (ci < n_chunks) {
@@ -111,21 +129,14 @@ __global__ void __launch_bounds__(FS_WARPS * 32) full_score_kernel(const FullSco
                 for (int hc = 0; hc < n_hc; ++hc) {
                     const int h0 = g * p.G + hc * 16;
                     const bool r0 = hc * 16 + gr < p.G, r1 = hc * 16 + gr + 8 < p.G;
-                    const __nv_bfloat16 *qrow = p.q + ((long long)(b * p.T + t) * p.Hq + h0) * D;
                     const float *lrow = p.lse + (long long)(b * p.T + t) * p.Hq + h0;
                     const float l0 = r0 ? lrow[gr] * kLog2e : 0.f, l1 = r1 ? lrow[gr + 8] * kLog2e : 0.f;
+                    if (n_hc > 1) load_q(g, hc, qa);
                     float sc[8][4];
 #pragma unroll
                     for (int nt = 0; nt < 8; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
 #pragma unroll
                     for (int ks = 0; ks < KS_D; ++ks) {
-                        // A fragment of the 16 heads (rows) for k-step ks, from global (L1)
-                        unsigned qa[4];
-                        const int c0 = ks * 16 + 2 * qc;
-                        qa[0] = r0 ? __ldg(reinterpret_cast<const unsigned *>(qrow + (long long)gr * D + c0)) : 0u;
-                        qa[1] = r1 ? __ldg(reinterpret_cast<const unsigned *>(qrow + (long long)(gr + 8) * D + c0)) : 0u;
-                        qa[2] = r0 ? __ldg(reinterpret_cast<const unsigned *>(qrow + (long long)gr * D + c0 + 8)) : 0u;
-                        qa[3] = r1 ? __ldg(reinterpret_cast<const unsigned *>(qrow + (long long)(gr + 8) * D + c0 + 8)) : 0u;
                         const int mi = lane >> 3, ri = lane & 7;
 #pragma unroll
                         for (int kg = 0; kg < 4; ++kg) {
@@ -133,8 +144,8 @@ __global__ void __launch_bounds__(FS_WARPS * 32) full_score_kernel(const FullSco
                             const int unit = ks * 2 + (mi & 1);
                             unsigned b0, b1, b2, b3;
                             ldsm_x4(b0, b1, b2, b3, ks_ + key * ROWB + ((unit ^ (key & 7)) * 16));
-                            mma_bf16_16816(sc[2 * kg], qa, b0, b1);
-                            mma_bf16_16816(sc[2 * kg + 1], qa, b2, b3);
+                            mma_bf16_16816(sc[2 * kg], qa[ks], b0, b1);
+                            mma_bf16_16816(sc[2 * kg + 1], qa[ks], b2, b3);
                         }
                     }
                     // P of the two rows of each column, summed over the 16 heads
