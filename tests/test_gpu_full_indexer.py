@@ -67,6 +67,7 @@ def _check_sets(idx, ref_idx, sc, topk, window, T, rows):
     (2, 257, 8, 2, 64, 40, 8),          # two KV groups summed, d = 64, ragged chunks
     (1, 200, 12, 1, 128, 300, 20),      # k larger than the candidates: all kept
     (1, 130, 4, 4, 64, 16, 0),          # no window
+    (1, 2065, 16, 1, 128, 1024, 128),   # the HySparse2 selection, ragged, several score chunks of keys
 ])
 def test_full_attn_indexer_parity(cuda_ok, B, T, Hq, Hkv, d, topk, window):
     g = inputs.gen_dsa(B, T, Hq, Hkv, d, 1, 32, seed=T + d)
