@@ -279,7 +279,9 @@ def main():
     # inputs go up on one copy stream and step i-1's results come back on
     # another while step i computes; two sets of device inputs and outputs
     # keep the copies off the buffers in use.  The serial form (copy, compute,
-    # copy on one stream) is reported beside it.
+    # copy on one stream) is reported beside it.  The pipelined loop runs at
+    # least 30 steps: its first upload and last readback (~6 + ~5 ms at 64K)
+    # are fill and drain, which a serving loop pays once.
     host = {k: v.pin_memory() for k, v in g.items()}
     out_h = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
     lse_h = [torch.empty(lse.shape, dtype=lse.dtype).pin_memory() for _ in range(2)]
@@ -294,6 +296,7 @@ def main():
         lse_h[0].copy_(lse, non_blocking=True)
 
     e2e_value = e2e_serial = None
+    n_pipe = 0
     if not args.no_e2e:
         n_e2e = max(2, args.steps // 2)
         e2e_times = timed_steps(e2e_serial_step, n_e2e, args.warmup, flush, dev, torch)
@@ -340,10 +343,11 @@ def main():
             dist.barrier()
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
+        n_pipe = max(args.steps, 30)
         a.record(cur)
         for st_ in (s_in, s_cmp, s_out):
             st_.wait_stream(cur)
-        pipelined(args.steps)
+        pipelined(n_pipe)
         for st_ in (s_in, s_cmp, s_out):
             cur.wait_stream(st_)
         b.record(cur)
@@ -351,7 +355,7 @@ def main():
         if world > 1:
             dist.barrier()
         pipe_ms = max_over_ranks(a.elapsed_time(b), dev, torch, dist)
-        e2e_value = aggregate([pipe_ms], [flops * args.steps] * world)[0] / 1e12
+        e2e_value = aggregate([pipe_ms], [flops * n_pipe] * world)[0] / 1e12
         api.check_device_status()
 
     peaks = _peaks()
@@ -405,7 +409,7 @@ def main():
                {"value": round(e2e_value, 3), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                 "overlap": "h2d / compute / d2h on three streams, two buffer sets; inputs larger than L2",
-                "serial_value": round(e2e_serial, 3)},
+                "pipelined_steps": n_pipe, "serial_value": round(e2e_serial, 3)},
         "gpu_launches": int(launches),
     }
     clocks = clk.summary()

@@ -1384,7 +1384,8 @@ static int launch_bwd_kv_lists(const BwdParams &p, const NsaBwdLayout &lay, char
     int2 *items = reinterpret_cast<int2 *>(ws + lay.items_off);
     int32_t *n_items = reinterpret_cast<int32_t *>(ws + lay.nitems_off);
     int32_t *qlist = reinterpret_cast<int32_t *>(ws + lay.qlist_off);
-    if (lay.n_lists > INT_MAX || lay.max_items * 8 > INT_MAX) return fail(SA_ERR_UNSUPPORTED, "nsa_bwd: lists");
+    if (lay.n_lists >= INT_MAX || lay.n_entries > INT_MAX || lay.max_items * 8 > INT_MAX)
+        return fail(SA_ERR_UNSUPPORTED, "nsa_bwd: %lld block choices exceed the int32 lists", lay.n_entries);
     cudaError_t e = cudaMemsetAsync(cnt, 0, (size_t)lay.n_lists * 4, st);
     if (e != cudaSuccess) return fail(SA_ERR_CUDA, "nsa_bwd memset: %s", cudaGetErrorString(e));
     const unsigned eg = (unsigned)((lay.n_entries + 255) / 256);

@@ -50,6 +50,13 @@ def test_workspace_queries(lib):
     assert lib.sa_sparse_attn_workspace_size(2, 3, 4, 64, 4) == 4 * 24 * 64 * 4 + 512 + 256
     assert lib.sa_nsa_workspace_size(1, 1024, 16, 1, 64, 32, 16, 64, 16) > 0
     assert lib.sa_indexer_topk_workspace_size(0, 1, 1, 2, 32, 1, 0) == 0
+    # NSA backward: compressed rows, their fp32 gradients, D terms, block lists
+    assert lib.sa_nsa_bwd_workspace_size(1, 1024, 16, 1, 64, 32, 16, 64, 16) > 0
+    assert lib.sa_nsa_bwd_workspace_size(1, 1024, 16, 1, 64, 32, 16, 0, 16) == 0
+    # exact indexer: fp32 layer output + lse + one chunk of dense scores (<= 1 GiB)
+    full = lib.sa_full_attn_topk_workspace_size(1, 65536, 16, 1, 128, 1024, 128)
+    rows = 65536 * 16
+    assert (1 << 30) < full <= rows * 128 * 4 + rows * 4 + (1 << 30) + 1024
 
 
 def test_indexer_workspace_is_chunked_under_one_gib(lib):
@@ -97,6 +104,25 @@ def test_host_validation_rejects_bad_arguments(lib):
     # NSA: sel_topk too large
     assert lib.sa_nsa_fwd(fake, fake, fake, fake, 1, 64, 16, 1, 64, 32, 16, 64, 33, 512,
                           0.1, fake, None, None, fake, 1 << 30, None) == 2
+    # NSA training forward: the saved branch outputs are required
+    assert lib.sa_nsa_fwd_train(fake, fake, fake, fake, 1, 64, 16, 1, 64, 32, 16, 64, 16, 512,
+                                0.1, fake, fake, fake, None, fake, 1 << 30, None) == 1
+    # NSA backward: head dim, a missing saved tensor, workspace too small
+    assert lib.sa_nsa_bwd(fake, fake, fake, fake, fake, fake, fake, fake, 1, 64, 16, 1, 96, 32, 16,
+                          64, 16, 512, 0.1, fake, fake, fake, fake, fake, 1 << 30, None) == 2
+    assert lib.sa_nsa_bwd(fake, fake, fake, fake, fake, None, fake, fake, 1, 64, 16, 1, 64, 32, 16,
+                          64, 16, 512, 0.1, fake, fake, fake, fake, fake, 1 << 30, None) == 1
+    assert lib.sa_nsa_bwd(fake, fake, fake, fake, fake, fake, fake, fake, 1, 64, 16, 1, 64, 32, 16,
+                          64, 16, 512, 0.1, fake, fake, fake, fake, fake, 64, None) == 3
+    # exact indexer from a full layer: Hq not a multiple of Hkv, head dim, no set size, workspace
+    assert lib.sa_full_attn_topk(fake, fake, fake, 1, 64, 6, 4, 64, 0.1, 8, 4, None, None, fake,
+                                 fake, 1 << 30, None) == 1
+    assert lib.sa_full_attn_topk(fake, fake, fake, 1, 64, 4, 1, 96, 0.1, 8, 4, None, None, fake,
+                                 fake, 1 << 30, None) == 2
+    assert lib.sa_full_attn_topk(fake, fake, fake, 1, 64, 4, 1, 64, 0.1, 0, 0, None, None, fake,
+                                 fake, 1 << 30, None) == 1
+    assert lib.sa_full_attn_topk(fake, fake, fake, 1, 64, 4, 1, 64, 0.1, 8, 4, None, None, fake,
+                                 fake, 64, None) == 3
     # attention: Hq not a multiple of Hkv
     assert lib.sa_sparse_attn_fwd(fake, fake, fake, 1, 4, 4, 3, 2, 64, 0, fake, 1, 4, None,
                                   None, None, None, 0.1, 1, fake, None, None, None, None, 0,

@@ -184,3 +184,22 @@ def test_nsa_backward_identities_8k(cuda_ok):
     dgr = np.einsum("rhc,brhc->rhb", dout[0].double().numpy()[rows],
                     ref_f["o_branch"].reshape(3, len(rows), Hq, d))
     _close(dg[0].cpu()[rows], dgr, "dgates (sampled rows)")
+
+
+def test_nsa_backward_bad_block_sets_error_word(cuda_ok):
+    # a selected block past the sequence is skipped and reported through the
+    # device error word (status 5); the word is cleared by the check
+    from fixed_pattern_sparse_sa_b200._lib import SAError
+    T, Hq, Hkv, d = 128, 4, 1, 64
+    cfg = dict(cmp_len=16, cmp_stride=8, sel_block=16, sel_topk=2, window=16)
+    g = inputs.gen_nsa(1, T, Hq, Hkv, d, seed=5)
+    q, k, v, gates = (g[n].cuda() for n in ("q", "k", "v", "gates"))
+    out, lse3, sel, o3 = api.nsa_fwd_train(q, k, v, gates, **cfg)
+    api.check_device_status()
+    sel[0, 50, 0, 0] = 1000
+    dout = torch.randn(1, T, Hq, d, generator=torch.Generator().manual_seed(6)).to(torch.bfloat16).cuda()
+    api.nsa_bwd(q, k, v, gates, dout, o3, lse3, sel, **cfg)
+    with pytest.raises(SAError) as ei:
+        api.check_device_status()
+    assert ei.value.status == 5
+    api.check_device_status()
