@@ -27,6 +27,7 @@
 #include "indexer.cuh"
 #include "indexer_filter.cuh"
 #include "nsa_misc.cuh"
+#include "nsa_bwd_tc.cuh"
 #include "probe_gather.cuh"
 
 using namespace sa;
@@ -1351,6 +1352,49 @@ static int launch_bwd_dq_tile(const BwdParams &p, cudaStream_t st) {
     return SA_OK;
 }
 
+// dq of a range branch on the tensor cores (head dim 128, at most 16 heads
+// per KV head); SA_NSA_BWD_DQ=mma selects the mma.sync kernel instead.
+static bool dq_tc_allowed(const BwdParams &p, int d) {
+    static int v = -1;
+    if (v < 0) {
+        const char *e = std::getenv("SA_NSA_BWD_DQ");
+        v = (e && std::strcmp(e, "mma") == 0) ? 0 : 1;
+    }
+    return v && d == 128 && p.G <= 16 && (long long)p.B * p.Tq * p.Hq + 16 < INT_MAX &&
+           (long long)p.B * std::max(p.L, 1) < INT_MAX;
+}
+
+template <int SRC>
+static int launch_nsa_dq_tc(const BwdParams &bp, cudaStream_t st) {
+    DqTcParams cp{};
+    TileParams &t = cp.t;
+    t.q = bp.q; t.k = bp.k; t.klo = SRC == TS_CMP ? bp.klo : bp.k; t.v = bp.v;
+    t.B = bp.B; t.T = bp.Tq; t.Lk = std::max(bp.L, 1); t.Hq = bp.Hq; t.Hkv = bp.Hkv; t.G = bp.G;
+    t.window = bp.window; t.cmp_len = bp.cmp_len; t.cmp_stride = bp.cmp_stride; t.scale_log2 = bp.scale_log2;
+    cp.lse = bp.lse; cp.Dt = bp.Dt; cp.gate = bp.gate; cp.lse_stride = bp.lse_stride; cp.gate_stride = bp.gate_stride;
+    cp.dq = bp.dq; cp.dq_accum = bp.dq_accum; cp.scale = bp.scale; cp.err = bp.err;
+    const long long items = (long long)bp.B * bp.Hkv * ((bp.Tq + CT_Q - 1) / CT_Q);
+    if (items == 0) return SA_OK;
+    if (items > INT_MAX) return fail(SA_ERR_UNSUPPORTED, "nsa_dq_tc: %lld items", items);
+    cp.n_items = (int)items;
+    CUtensorMap qm, dm, khm, klm, vm;
+    int rc = bf16_tensor_map(&qm, bp.q, (long long)bp.B * bp.Tq * bp.Hq, 128, 16);
+    if (!rc) rc = bf16_tensor_map(&dm, bp.dout, (long long)bp.B * bp.Tq * bp.Hq, 128, 16);
+    if (!rc) rc = bf16_tensor_map_3d(&khm, t.k, 128, bp.Hkv, (long long)bp.B * t.Lk, DQ_KT);
+    if (!rc) rc = bf16_tensor_map_3d(&klm, t.klo, 128, bp.Hkv, (long long)bp.B * t.Lk, DQ_KT);
+    if (!rc) rc = bf16_tensor_map_3d(&vm, t.v, 128, bp.Hkv, (long long)bp.B * t.Lk, DQ_KT);
+    if (rc) return rc;
+    constexpr int smem = DqSmem::ALLOC;
+    static_assert(smem <= 227 * 1024, "shared memory");
+    auto kern = nsa_dq_tc_kernel<SRC>;
+    rc = set_smem(kern, smem);
+    if (rc) return rc;
+    const int grid = (int)std::min<long long>(items, sm_count());
+    launch_k(__PRETTY_FUNCTION__, kern, grid, DQ_THREADS, smem, st, qm, dm, khm, klm, vm, cp);
+    SA_CHECK_LAUNCH("nsa_dq_tc_kernel");
+    return SA_OK;
+}
+
 // Key-major dK / dV of a range branch (window, or compressed rows).
 template <int D, bool HILO>
 static int launch_bwd_kv(const BwdParams &p, cudaStream_t st) {
@@ -1424,7 +1468,8 @@ static int nsa_bwd_branches(const BwdParams &base, const float *gates, const flo
     p.window = 0; p.cmp_len = cmp_len; p.cmp_stride = cmp_stride;
     p.dk = dkc; p.dv = dvc; p.dq_accum = 0;
     if (lay.nc == 0) p.L = 0;       // no compressed row is visible to any query
-    int rc = launch_bwd_dq_tile<D, true>(p, st);                     // dq
+    int rc = dq_tc_allowed(p, D) ? launch_nsa_dq_tc<TS_CMP>(p, st)   // dq
+                                 : launch_bwd_dq_tile<D, true>(p, st);
     if (rc) return rc;
     rc = launch_bwd_kv<D, true>(p, st);                             // dKc, dVc
     if (rc) return rc;
@@ -1442,7 +1487,8 @@ static int nsa_bwd_branches(const BwdParams &base, const float *gates, const flo
     p = base;
     p.lse = lse3 + 2; p.gate = gates + 2; p.Dt = Dt + 2 * rows;
     p.window = window; p.dq_accum = 1;
-    rc = launch_bwd_dq_tile<D, false>(p, st);                          // dq
+    rc = dq_tc_allowed(p, D) ? launch_nsa_dq_tc<TS_WINDOW>(p, st)       // dq
+                             : launch_bwd_dq_tile<D, false>(p, st);
     if (rc) return rc;
     return launch_bwd_kv<D, false>(p, st);                              // dk, dv
 }

@@ -208,7 +208,9 @@ def test_prefill64k_attention_sampled_rows(cuda_ok):
     rows = sample_rows(w.T, 192, seed=2)
     ref_idx, _ = oracle.indexer_topk(g["q_idx"], g["k_idx"], g["w"], w.topk, w.window, rows=rows)
     np.testing.assert_array_equal(idx[0].cpu().numpy()[rows], ref_idx)
-    ro, rl = oracle.sparse_attn(g["q"], g["k"], g["v"], idx.cpu(), rows=rows)
+    full = np.full((1, w.T, ref_idx.shape[-1]), -1, dtype=np.int32)     # the oracle's own sets
+    full[0, rows] = ref_idx
+    ro, rl = oracle.sparse_attn(g["q"], g["k"], g["v"], full, rows=rows)
     assert_out_close(out[0][rows], ro)
     assert_lse_close(lse[0][rows], rl)
     assert torch.isfinite(out.float()).all()

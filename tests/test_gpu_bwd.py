@@ -96,9 +96,9 @@ def test_backward_identities_16k(cuda_ok):
     g = inputs.gen_dsa(B, T, Hq, Hkv, d, 1, 32, seed=11)
     dout = torch.randn(B, T, Hq, d, generator=torch.Generator().manual_seed(12)).to(torch.bfloat16)
     dev = torch.device("cuda")
-    t = torch.arange(T, device=dev)
-    r = torch.rand(T, K, device=dev, generator=torch.Generator(device=dev).manual_seed(13))
-    idx = torch.minimum((r * (t[:, None] + 1).float()).long(), t[:, None]).to(torch.int32)[None]
+    t = torch.arange(T)
+    r = torch.rand(T, K, generator=torch.Generator().manual_seed(13))    # seeded input lists, drawn on the host
+    idx = torch.minimum((r * (t[:, None] + 1).float()).long(), t[:, None]).to(torch.int32)[None].to(dev)
     dq, dk, dv = _run(g["q"], g["k"], g["v"], idx, dout)
     sk = dk.double().sum(dim=1).cpu().numpy()
     assert np.abs(sk).max() <= MAX_REL * dk.abs().sum(dim=1).max().item()

@@ -13,28 +13,37 @@ NSA_CFG = dict(cmp_len=32, cmp_stride=16, sel_block=64, sel_topk=16, window=512)
 
 
 def _nsa_check(g, out, lse3, sel, rows, cfg):
-    """Selection parity with the near-tie rule, then outputs against the oracle
-    re-run with the GPU's selection."""
+    """Selection parity with the near-tie rule, then the outputs against the
+    oracle's own run: every output and branch LSE on the rows whose block
+    choice equals the oracle's; on a near-tie row (its choice differs by
+    blocks of equal importance up to 1e-5 of the row maximum) the LSEs of the
+    compressed and window branches, which do not depend on the choice."""
     ref = oracle.nsa_fwd(g["q"], g["k"], g["v"], g["gates"], rows=rows, **cfg)
     gsel = sel.cpu().numpy().reshape(-1, sel.shape[2], sel.shape[3])[rows]
-    n_diff = 0
+    same = np.ones(len(rows), dtype=bool)
     for i in range(len(rows)):
         for gg in range(gsel.shape[1]):
             a = set(x for x in gsel[i, gg] if x >= 0)
             b = set(x for x in ref["sel_idx"][i, gg] if x >= 0)
             if a == b:
                 continue
-            n_diff += 1
+            same[i] = False
             imp = ref["imp"][i, gg]
             kth = np.sort(imp[[x for x in b]])[0]           # smallest chosen importance
             tol = 1e-5 * imp.max()
             for blk in a ^ b:
                 assert abs(imp[blk] - kth) <= tol, f"row {rows[i]} group {gg}: block {blk} not a near-tie"
+    n_diff = int((~same).sum())
     assert n_diff <= max(2, len(rows) // 100), f"{n_diff} near-tie rows"
-    ref2 = oracle.nsa_fwd(g["q"], g["k"], g["v"], g["gates"], rows=rows, sel_override=gsel, **cfg)
     B, T, Hq, d = g["q"].shape
-    assert_out_close(out.reshape(-1, Hq, d)[rows], ref2["out"], "nsa out")
-    assert_lse_close(lse3.reshape(-1, Hq, 3)[rows], ref2["lse_branch"], "nsa lse")
+    o = out.reshape(-1, Hq, d)[rows]
+    l3 = lse3.reshape(-1, Hq, 3)[rows]
+    keep = np.nonzero(same)[0]
+    assert_out_close(o[keep], ref["out"][keep], "nsa out")
+    assert_lse_close(l3[keep], ref["lse_branch"][keep], "nsa lse")
+    if n_diff:
+        tie = np.nonzero(~same)[0]
+        assert_lse_close(l3[tie][..., [0, 2]], ref["lse_branch"][tie][..., [0, 2]], "nsa lse (near ties)")
     return n_diff
 
 
@@ -78,9 +87,13 @@ def test_nsa_branches_isolated_by_gates(cuda_ok):
         oh = torch.zeros_like(gd["gates"])
         oh[..., br] = 1.0
         out, _, sel = api.nsa_fwd(gd["q"], gd["k"], gd["v"], oh, **NSA_CFG)
-        r2 = oracle.nsa_fwd(g["q"], g["k"], g["v"], oh.cpu(),
-                            sel_override=sel.cpu().numpy().reshape(T, 1, -1), **NSA_CFG)
-        assert_out_close(out[0], r2["o_branch"][br], f"branch {br}")
+        # the branch outputs do not depend on the gates; the selected branch
+        # is compared on the rows whose block choice equals the oracle's
+        same = np.all(np.sort(sel.cpu().numpy().reshape(T, -1), axis=1)
+                      == np.sort(ref["sel_idx"].reshape(T, -1), axis=1), axis=1)
+        rows = np.arange(T) if br != 1 else np.nonzero(same)[0]
+        assert len(rows) >= T - max(2, T // 100)
+        assert_out_close(out[0][rows], ref["o_branch"][br][rows], f"branch {br}")
     assert ref["out"].shape == (T, 16, 128)
 
 
