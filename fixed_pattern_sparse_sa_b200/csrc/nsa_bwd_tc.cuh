@@ -24,6 +24,7 @@
 // timeout sets ERR_TIMEOUT and the CTA drains and exits.
 #pragma once
 
+#include "attn_bwd.cuh"
 #include "attn_cmp_tc.cuh"
 
 namespace sa {
@@ -342,6 +343,388 @@ __global__ void __launch_bounds__(DQ_THREADS, 1)
     tc::fence_before_sync();
     __syncthreads();
     if (warp == 1) tc::tmem_dealloc(tmem, DQ_TM_COLS);
+}
+
+
+// ------------------------------------------------------------------------
+// dk / dv of the NSA compressed and window branches on the tcgen05 tensor
+// cores, key-major: an item is 128 keys of one KV group (the TMEM lanes) and
+// a run of up to KV_QSPLIT tiles of the queries that see them, each tile 4
+// consecutive queries x 16 heads = 64 columns.  The keys' K_hi (+ K_lo) and
+// V stay in shared memory for the item; per query tile one thread issues
+//   S^T = K Q_t^T (+ K_lo Q_t^T)   and   dP^T = V dO_t^T      (N = 64)
+// into tensor memory; the score warps (one key row per thread) form
+//   P^T = gate * exp2(S^T * scale_log2 - lse2),  dS^T = P^T (dP^T - D)
+// masked to the (key, query) pairs the branch relates, and store both as
+// bf16 pairs in tensor memory over the S^T / dP^T columns they have just
+// read (two buffers, so the next tile's S^T / dP^T overlaps this tile's
+// scores); the MMA thread then adds
+//   dV += P^T dO_t   and   dK += dS^T Q_t        (A from TMEM, B MN-major)
+// into two 128-column accumulators that live for the whole item.  At the end
+// of an item the score warps add dK * scale and dV to the global fp32 rows
+// (one reduction per key and column per item).  The per-row lse / D / gate
+// of a query tile come as one 1 KB bulk copy of a packed array
+// (nsa_kv_scalars_kernel).
+constexpr int KV_QT = 4;                 // queries per tile (x 16 heads = 64 columns)
+constexpr int KV_QSPLIT = 64;            // query tiles per item
+constexpr int KV_THREADS = 320;
+// buffer b (b = 0, 1) at b * 128: S^T in columns 0-63, dP^T in 64-127; P^T
+// and dS^T overwrite them as bf16 pairs (score-warp half h writes the pairs of
+// its 32 columns into the first 16 of them)
+constexpr uint32_t KV_TM_S = 0;
+constexpr uint32_t KV_TM_DP = 64;
+constexpr uint32_t KV_TM_V = 256;        // dV: 128 fp32 columns
+constexpr uint32_t KV_TM_K = 384;        // dK: 128
+constexpr uint32_t KV_TM_COLS = 512;
+
+struct KvSmem {                          // head dim 128
+    static constexpr int KT_BYTES = 128 * 256;           // one K (or V) tile: 2 halves x 128 rows x 128 B
+    static constexpr int QT_BYTES = 64 * 256;            // one Q (or dO) tile: 2 halves x 64 rows x 128 B
+    static constexpr int SC_BYTES = KV_QT * 16 * 16;     // lse, D, gate, pad of the tile's 64 rows
+    static constexpr int QSTAGE = 2 * QT_BYTES + 1024;   // Q | dO | scalars (1 KB slot)
+    static constexpr int OFF_K = 0;                      // K_hi | K_lo | V
+    static constexpr int OFF_Q = OFF_K + 3 * KT_BYTES;
+    static constexpr int OFF_BAR = OFF_Q + 2 * QSTAGE;
+    // kv_full, kv_empty, q_full[2], q_empty[2], s_full[2], pd_full[2], pd_done[2], acc_full, acc_free, drain
+    static constexpr int N_BAR = 2 + 4 + 2 + 4 + 3;
+    static constexpr int OFF_MISC = OFF_BAR + N_BAR * 8;
+    static constexpr int TOTAL = OFF_MISC + 16;
+    static constexpr int ALLOC = TOTAL + 1024;
+};
+
+struct KvTcParams {
+    TileParams t;            // k (K_hi), klo, v, shapes (T queries, Lk keys), window / cmp_len / cmp_stride, scale_log2
+    const float4 *scal;      // [B, Hkv, T, 16] (lse natural, D, gate, 0) of this branch
+    float *dk, *dv;          // [B, Lk, Hkv, 128] fp32, added to
+    float scale;
+    unsigned *err;
+    int n_kt;                // key tiles per sequence
+    int n_split;             // query splits per key tile
+    int n_items;             // B * Hkv * n_kt * n_split
+};
+
+// Queries [q_lo, q_hi) that see at least one key of [j0, j1] (range branches).
+template <int SRC>
+__device__ __forceinline__ void kv_tc_range(const TileParams &p, int j0, int j1, int &q_lo, int &q_hi) {
+    if constexpr (SRC == TS_CMP) {
+        q_lo = j0 * p.cmp_stride + p.cmp_len - 1;
+        q_hi = p.T;
+    } else {
+        q_lo = j0;
+        q_hi = min(p.T, j1 + p.window);
+    }
+}
+
+// Item -> (b, g, key tile, first query tile, number of query tiles); 0 tiles = empty.
+template <int SRC>
+__device__ __forceinline__ int kv_tc_item(const KvTcParams &cp, int it, int &b, int &g, int &kt, int &qt0) {
+    const TileParams &p = cp.t;
+    const int s = it % cp.n_split;
+    int rem = it / cp.n_split;
+    kt = rem % cp.n_kt; rem /= cp.n_kt;
+    g = rem % p.Hkv;
+    b = rem / p.Hkv;
+    const int j0 = kt * 128, j1 = min(j0 + 127, p.Lk - 1);
+    int q_lo, q_hi;
+    kv_tc_range<SRC>(p, j0, j1, q_lo, q_hi);
+    if (q_lo >= q_hi) return 0;
+    const int a0 = q_lo / KV_QT;                               // first query tile (aligned)
+    const int n_all = (q_hi + KV_QT - 1) / KV_QT - a0;
+    qt0 = a0 + s * KV_QSPLIT;
+    const int n = n_all - s * KV_QSPLIT;
+    return n <= 0 ? 0 : min(n, KV_QSPLIT);
+}
+
+template <int SRC>
+__global__ void __launch_bounds__(KV_THREADS, 1)
+    nsa_kv_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap domap,
+                     const __grid_constant__ CUtensorMap khimap, const __grid_constant__ CUtensorMap klomap,
+                     const __grid_constant__ CUtensorMap vmap, const KvTcParams cp) {
+    grid_dependency_sync();
+    constexpr int D = 128;
+    constexpr bool LO = SRC == TS_CMP;
+    using L = KvSmem;
+    const TileParams &p = cp.t;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::OFF_BAR);
+    uint64_t *kv_full = bars, *kv_empty = bars + 1, *q_full = bars + 2, *q_empty = bars + 4;
+    uint64_t *s_full = bars + 6, *pd_full = bars + 8, *pd_done = bars + 10;
+    uint64_t *acc_full = bars + 12, *acc_free = bars + 13, *drain = bars + 14;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::OFF_MISC);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::OFF_MISC + 4);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    if (warp == 1) {
+        tc::tmem_alloc(tmem_slot, KV_TM_COLS);
+        tc::tmem_relinquish();
+    }
+    if (tid == 0) {
+        tc::mbar_init(kv_full, 1); tc::mbar_init(kv_empty, 1);
+        for (int i = 0; i < 2; ++i) {
+            tc::mbar_init(q_full + i, 1); tc::mbar_init(q_empty + i, 1);
+            tc::mbar_init(pd_full + i, 256); tc::mbar_init(pd_done + i, 1);
+            tc::mbar_init(s_full + i, 1);
+        }
+        tc::mbar_init(acc_full, 1); tc::mbar_init(acc_free, 256);
+        tc::mbar_init(drain, 1);
+        *abort_flag = 0;
+        tc::mbar_fence_init();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    auto fail = [&]() {
+        raise_error(cp.err, ERR_TIMEOUT);
+        *abort_flag = 1;
+    };
+
+    if (warp == 0) {
+        // ------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            bool ok = true;
+            int qt = 0, kn = 0;                           // query tiles and key tiles loaded
+            const int n_items = debug_stall() ? 0 : cp.n_items;
+            for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+                int b, g, kt, qt0;
+                const int nq = kv_tc_item<SRC>(cp, it, b, g, kt, qt0);
+                if (nq == 0) continue;
+                // the keys of the item, once the previous item's last MMA is done
+                if (!atc::wait(kv_empty, (kn & 1) ^ 1, abort_flag)) { ok = false; break; }
+                atc::expect_tx(kv_full, LO ? 3 * L::KT_BYTES : 2 * L::KT_BYTES);
+                const int z = b * p.Lk + kt * 128;
+                for (int h = 0; h < 2; ++h) {
+                    atc::load_3d(smem + L::OFF_K + h * (128 * 128), &khimap, h * 64, g, z, kv_full);
+                    if (LO) atc::load_3d(smem + L::OFF_K + L::KT_BYTES + h * (128 * 128), &klomap, h * 64, g, z, kv_full);
+                    atc::load_3d(smem + L::OFF_K + 2 * L::KT_BYTES + h * (128 * 128), &vmap, h * 64, g, z, kv_full);
+                }
+                ++kn;
+                for (int i = 0; i < nq; ++i, ++qt) {
+                    const int qs = qt & 1;
+                    if (!atc::wait(q_empty + qs, ((qt >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+                    unsigned char *dst = smem + L::OFF_Q + qs * L::QSTAGE;
+                    const int t0 = (qt0 + i) * KV_QT;
+                    atc::expect_tx(q_full + qs, 2 * L::QT_BYTES + L::SC_BYTES);
+                    for (int w = 0; w < KV_QT; ++w) {
+                        const int qrow = (b * p.T + min(t0 + w, p.T - 1)) * p.Hq + g * p.G;
+                        for (int h = 0; h < 2; ++h) {
+                            atc::load_2d(dst + h * (64 * 128) + w * (16 * 128), &qmap, h * 64, qrow, q_full + qs);
+                            atc::load_2d(dst + L::QT_BYTES + h * (64 * 128) + w * (16 * 128), &domap, h * 64, qrow,
+                                         q_full + qs);
+                        }
+                    }
+                    // lse / D / gate of the tile's rows: 4 consecutive queries of (b, g), one 1 KB copy
+                    // (rows past the sequence read the last query's, masked later)
+                    const int tc0 = min(t0, p.T - KV_QT);
+                    const float4 *src = cp.scal + ((long long)(b * p.Hkv + g) * p.T + tc0) * 16;
+                    asm volatile(
+                        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+                            tc::smem_u32(dst + 2 * L::QT_BYTES)),
+                        "l"(src), "r"(L::SC_BYTES), "r"(tc::smem_u32(q_full + qs))
+                        : "memory");
+                }
+            }
+            if (!ok) fail();
+            // let the copies land before the CTA exits
+            if (kn > 0) tc::mbar_wait_bounded(kv_full, (kn - 1) & 1, ATC_WAIT);
+            for (int i = 0; i < 2 && i < qt; ++i) {
+                const int q = qt - 1 - i;
+                tc::mbar_wait_bounded(q_full + (q & 1), (q >> 1) & 1, ATC_WAIT);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // --------------------------------------------------------------- MMA
+        if (lane == 0) {
+            constexpr uint32_t ID_S = tc::make_idesc(1, 1, 128, 64);
+            constexpr uint32_t ID_A = tc::make_idesc(1, 1, 128, D) | (1u << 16);   // B (dO, Q) MN-major
+            const uint32_t ka = tc::smem_u32(smem + L::OFF_K);
+            bool ok = true;
+            int qt = 0, kn = 0, an = 0;
+            // S^T and dP^T of query tile q (stage q & 1) into buffer q & 1, once
+            // the dV / dK products of tile q - 2 (which read that buffer) are done
+            auto issue_s = [&](int q) -> bool {
+                const int qs = q & 1, b = q & 1;
+                if (!atc::wait(q_full + qs, (q >> 1) & 1, abort_flag)) return false;
+                if (q >= 2 && !atc::wait(pd_done + b, ((q >> 1) & 1) ^ 1, abort_flag)) return false;
+                tc::fence_after_sync();
+                const uint32_t qa = tc::smem_u32(smem + L::OFF_Q + qs * L::QSTAGE);
+                const uint32_t da = qa + L::QT_BYTES;
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    const int h = ks / 4, kk = ks % 4;
+                    const uint64_t akh = atc::desc_sw128(ka + h * (128 * 128) + kk * 32, 16, 1024);
+                    const uint64_t akl = atc::desc_sw128(ka + L::KT_BYTES + h * (128 * 128) + kk * 32, 16, 1024);
+                    const uint64_t av = atc::desc_sw128(ka + 2 * L::KT_BYTES + h * (128 * 128) + kk * 32, 16, 1024);
+                    const uint64_t bq = atc::desc_sw128(qa + h * (64 * 128) + kk * 32, 16, 1024);
+                    const uint64_t bd = atc::desc_sw128(da + h * (64 * 128) + kk * 32, 16, 1024);
+                    tc::mma_bf16(tmem + b * 128 + KV_TM_S, akh, bq, ID_S, ks > 0 ? 1u : 0u);
+                    if (LO) tc::mma_bf16(tmem + b * 128 + KV_TM_S, akl, bq, ID_S, 1u);
+                    tc::mma_bf16(tmem + b * 128 + KV_TM_DP, av, bd, ID_S, ks > 0 ? 1u : 0u);
+                }
+                tc::mma_commit(s_full + b);
+                return true;
+            };
+            for (int it = blockIdx.x; it < cp.n_items && ok; it += gridDim.x) {
+                int b, g, kt, qt0;
+                const int nq = kv_tc_item<SRC>(cp, it, b, g, kt, qt0);
+                if (nq == 0) continue;
+                if (!atc::wait(kv_full, kn & 1, abort_flag)) { ok = false; break; }
+                ++kn;
+                if (!issue_s(qt)) { ok = false; break; }
+                // the previous item's epilogue must have read dV / dK
+                if (an > 0 && !atc::wait(acc_free, (an - 1) & 1, abort_flag)) { ok = false; break; }
+                for (int i = 0; i < nq; ++i, ++qt) {
+                    const int qs = qt & 1, pb = qt & 1;
+                    if (i + 1 < nq && !issue_s(qt + 1)) { ok = false; break; }
+                    if (!atc::wait(pd_full + pb, (qt >> 1) & 1, abort_flag)) { ok = false; break; }
+                    tc::fence_after_sync();
+                    const uint32_t qa = tc::smem_u32(smem + L::OFF_Q + qs * L::QSTAGE);
+                    const uint32_t da = qa + L::QT_BYTES;
+                    // dV += P^T dO_t, dK += dS^T Q_t: A from tensor memory, B MN-major
+#pragma unroll
+                    for (int kk = 0; kk < 64 / 16; ++kk) {
+                        const uint32_t pc = pb * 128 + (kk < 2 ? kk * 8 : 32 + (kk - 2) * 8);
+                        const uint64_t bdo = atc::desc_sw128(da + kk * 2048, 64 * 128, 1024);
+                        const uint64_t bqq = atc::desc_sw128(qa + kk * 2048, 64 * 128, 1024);
+                        const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
+                        tc::mma_bf16_ts(tmem + KV_TM_V, tmem + pc + KV_TM_S, bdo, ID_A, acc);
+                        tc::mma_bf16_ts(tmem + KV_TM_K, tmem + pc + KV_TM_DP, bqq, ID_A, acc);
+                    }
+                    tc::mma_commit(q_empty + qs);
+                    tc::mma_commit(pd_done + pb);
+                }
+                if (!ok) break;
+                tc::mma_commit(kv_empty);
+                tc::mma_commit(acc_full);
+                ++an;
+            }
+            if (!ok) fail();
+            tc::mma_commit(drain);
+            tc::mbar_wait_bounded(drain, 0, ATC_WAIT);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------ score warps
+        // Thread = one key (TMEM lane); the two warps of a lane quadrant take
+        // the query-tile columns 0-31 / 32-63 and the dV / dK columns 0-63 /
+        // 64-127.  The pair agrees on each wait through a 64-thread named barrier.
+        const int quad = warp & 3, half = (warp - 2) >> 2;
+        const int pair = 1 + quad;
+        constexpr int SC = 32, OC = D / 2;
+        const int kr = quad * 32 + lane;                  // key row of the tile
+        const uint32_t lrow = (uint32_t)(quad * 32) << 16;
+        bool ok = true;
+        int qt = 0, an = 0;
+        for (int it = blockIdx.x; it < cp.n_items && ok; it += gridDim.x) {
+            int b, g, kt, qt0;
+            const int nq = kv_tc_item<SRC>(cp, it, b, g, kt, qt0);
+            if (nq == 0) continue;
+            const int j = kt * 128 + kr;                  // this thread's key
+            for (int i = 0; i < nq; ++i, ++qt) {
+                const int qs = qt & 1, pb = qt & 1;
+                // S^T / dP^T of the tile (its MMA waited for the Q / dO stage, and
+                // with it the scalars' copy; the wait below makes them visible)
+                bool got = atc::wait(s_full + pb, (qt >> 1) & 1, abort_flag);
+                if (got) got = atc::wait(q_full + qs, (qt >> 1) & 1, abort_flag);
+                if (!atc::agree(pair, 64, got)) { ok = false; break; }
+                tc::fence_after_sync();
+                uint32_t sr[SC], dr[SC];
+#pragma unroll
+                for (int c = 0; c < SC; c += 16) {
+                    tc::tmem_ld16(tmem + lrow + pb * 128 + KV_TM_S + half * SC + c,
+                                  *reinterpret_cast<uint32_t(*)[16]>(sr + c));
+                    tc::tmem_ld16(tmem + lrow + pb * 128 + KV_TM_DP + half * SC + c,
+                                  *reinterpret_cast<uint32_t(*)[16]>(dr + c));
+                }
+                tc::tmem_ld_wait();
+                const float4 *sc = reinterpret_cast<const float4 *>(smem + L::OFF_Q + qs * L::QSTAGE + 2 * L::QT_BYTES);
+                const int t0 = (qt0 + i) * KV_QT;
+                const int tc0 = min(t0, p.T - KV_QT);
+                uint32_t pp[SC / 2], dp2[SC / 2];
+#pragma unroll
+                for (int c = 0; c < SC; c += 2) {
+                    float pv[2], dv2[2];
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int col = half * SC + c + e;         // q-row of the tile: query col/16, head col%16
+                        const int t = t0 + (col >> 4);
+                        // rows past the sequence read the last query's slot (masked below)
+                        const float4 s4 = sc[(min(t, p.T - 1) - tc0) * 16 + (col & 15)];
+                        bool vis;
+                        if constexpr (SRC == TS_CMP) vis = j < p.Lk && j * p.cmp_stride + p.cmp_len - 1 <= t;
+                        else vis = j <= t && j > t - p.window;
+                        vis = vis && t < p.T && s4.x != -INFINITY;
+                        const float pr = vis ? s4.z * exp2f(fmaf(__uint_as_float(sr[c + e]), p.scale_log2,
+                                                                  -s4.x * kLog2e)) : 0.f;
+                        pv[e] = pr;
+                        dv2[e] = pr * (__uint_as_float(dr[c + e]) - s4.y);
+                    }
+                    pp[c / 2] = pack_bf16(pv[0], pv[1]);
+                    dp2[c / 2] = pack_bf16(dv2[0], dv2[1]);
+                }
+                // the pairs over the first 16 of the 32 columns this warp has read
+                atc::tmem_st16(tmem + lrow + pb * 128 + KV_TM_S + half * SC, *reinterpret_cast<const uint32_t(*)[16]>(pp));
+                atc::tmem_st16(tmem + lrow + pb * 128 + KV_TM_DP + half * SC, *reinterpret_cast<const uint32_t(*)[16]>(dp2));
+                atc::tmem_st_wait();
+                tc::fence_before_sync();
+                atc::arrive(pd_full + pb);
+            }
+            if (!ok) break;
+            // ------------------------------------------------------ epilogue
+            if (!atc::agree(pair, 64, atc::wait(acc_full, an & 1, abort_flag))) { ok = false; break; }
+            tc::fence_after_sync();
+            const bool kv_ok = j < p.Lk;
+            float *dvr = cp.dv + (((long long)b * p.Lk + (kv_ok ? j : 0)) * p.Hkv + g) * D + half * OC;
+            float *dkr = cp.dk + (((long long)b * p.Lk + (kv_ok ? j : 0)) * p.Hkv + g) * D + half * OC;
+#pragma unroll
+            for (int c = 0; c < OC; c += 16) {
+                uint32_t v16[16], k16[16];
+                tc::tmem_ld16(tmem + lrow + KV_TM_V + half * OC + c, v16);
+                tc::tmem_ld16(tmem + lrow + KV_TM_K + half * OC + c, k16);
+                tc::tmem_ld_wait();
+                if (kv_ok) {
+#pragma unroll
+                    for (int e = 0; e < 16; e += 2) {
+                        red_add2(dvr + c + e, __uint_as_float(v16[e]), __uint_as_float(v16[e + 1]));
+                        red_add2(dkr + c + e, __uint_as_float(k16[e]) * cp.scale, __uint_as_float(k16[e + 1]) * cp.scale);
+                    }
+                }
+            }
+            tc::fence_before_sync();
+            atc::arrive(acc_free);
+            ++an;
+        }
+        if (!ok) fail();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 1) tc::tmem_dealloc(tmem, KV_TM_COLS);
+}
+
+// Packed per-(b, g, query, head) scalars of one branch for nsa_kv_tc_kernel:
+// (lse natural, D, gate, 0); heads past the group get lse = -inf, gate 0.
+__global__ void __launch_bounds__(256) nsa_kv_scalars_kernel(const float *__restrict__ lse, int lse_stride,
+                                                             const float *__restrict__ Dt,
+                                                             const float *__restrict__ gate, int gate_stride,
+                                                             int B, int T, int Hq, int Hkv, int G,
+                                                             float4 *__restrict__ out) {
+    grid_dependency_sync();
+    const long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const long long total = (long long)B * Hkv * T * 16;
+    if (e >= total) return;
+    const int h = (int)(e % 16);
+    long long r = e / 16;
+    const int t = (int)(r % T); r /= T;
+    const int g = (int)(r % Hkv);
+    const int b = (int)(r / Hkv);
+    float4 v = make_float4(-INFINITY, 0.f, 0.f, 0.f);
+    if (h < G) {
+        const long long row = ((long long)b * T + t) * Hq + (long long)g * G + h;
+        v = make_float4(lse[row * lse_stride], Dt[row], gate ? gate[row * gate_stride] : 1.f, 0.f);
+    }
+    out[e] = v;
 }
 
 }  // namespace sa

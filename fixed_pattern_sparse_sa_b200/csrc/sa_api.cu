@@ -1285,7 +1285,7 @@ struct NsaBwdLayout {
     int nc, nb;
     long long n_lists, n_entries, max_items;
     size_t kc_off, klo_off, vc_off, dkc_off, dvc_off, dt_off;
-    size_t cnt_off, qoff_off, cur_off, items_off, nitems_off, qlist_off, total;
+    size_t cnt_off, qoff_off, cur_off, items_off, nitems_off, qlist_off, scal_off, total;
 };
 
 static NsaBwdLayout nsa_bwd_layout(int B, int T, int Hq, int Hkv, int d, int cmp_len, int cmp_stride,
@@ -1310,6 +1310,8 @@ static NsaBwdLayout nsa_bwd_layout(int B, int T, int Hq, int Hkv, int d, int cmp
     lay.items_off = off; off += round_up((size_t)lay.max_items * 8, 256);
     lay.nitems_off = off; off += 256;
     lay.qlist_off = off; off += round_up((size_t)lay.n_entries * 4, 256);
+    // packed lse / D / gate of one branch for the tensor-core key-major pass
+    lay.scal_off = off; off += round_up((size_t)B * Hkv * T * 16 * 16, 256);
     lay.total = off;
     return lay;
 }
@@ -1395,6 +1397,56 @@ static int launch_nsa_dq_tc(const BwdParams &bp, cudaStream_t st) {
     return SA_OK;
 }
 
+// Key-major dK / dV of a range branch on the tensor cores (head dim 128, at
+// most 16 heads per KV head); SA_NSA_BWD_KV=mma selects the mma.sync kernel.
+static bool kv_tc_allowed(const BwdParams &p, int d) {
+    static int v = -1;
+    if (v < 0) {
+        const char *e = std::getenv("SA_NSA_BWD_KV");
+        v = (e && std::strcmp(e, "mma") == 0) ? 0 : 1;
+    }
+    return v && d == 128 && p.G <= 16 && p.Tq >= KV_QT && p.L >= 1 &&
+           (long long)p.B * p.Tq * p.Hq + 16 < INT_MAX && (long long)p.B * p.L + 128 < INT_MAX;
+}
+
+template <int SRC>
+static int launch_nsa_kv_tc(const BwdParams &bp, float4 *scal, cudaStream_t st) {
+    const long long n_sc = (long long)bp.B * bp.Hkv * bp.Tq * 16;
+    launch_k("nsa_kv_scalars_kernel", nsa_kv_scalars_kernel, (unsigned)((n_sc + 255) / 256), 256, 0, st,
+             bp.lse, bp.lse_stride, (const float *)bp.Dt, bp.gate, bp.gate_stride, bp.B, bp.Tq, bp.Hq, bp.Hkv, bp.G,
+             scal);
+    SA_CHECK_LAUNCH("nsa_kv_scalars_kernel");
+    KvTcParams cp{};
+    TileParams &t = cp.t;
+    t.q = bp.q; t.k = bp.k; t.klo = SRC == TS_CMP ? bp.klo : bp.k; t.v = bp.v;
+    t.B = bp.B; t.T = bp.Tq; t.Lk = bp.L; t.Hq = bp.Hq; t.Hkv = bp.Hkv; t.G = bp.G;
+    t.window = bp.window; t.cmp_len = bp.cmp_len; t.cmp_stride = bp.cmp_stride; t.scale_log2 = bp.scale_log2;
+    cp.scal = scal; cp.dk = bp.dk; cp.dv = bp.dv; cp.scale = bp.scale; cp.err = bp.err;
+    cp.n_kt = (bp.L + 127) / 128;
+    const long long max_tiles = SRC == TS_CMP ? bp.Tq / KV_QT + 2 : (128 + (long long)bp.window) / KV_QT + 2;
+    cp.n_split = (int)((max_tiles + KV_QSPLIT - 1) / KV_QSPLIT);
+    const long long items = (long long)bp.B * bp.Hkv * cp.n_kt * cp.n_split;
+    if (items == 0) return SA_OK;
+    if (items > INT_MAX) return fail(SA_ERR_UNSUPPORTED, "nsa_kv_tc: %lld items", items);
+    cp.n_items = (int)items;
+    CUtensorMap qm, dm, khm, klm, vm;
+    int rc = bf16_tensor_map(&qm, bp.q, (long long)bp.B * bp.Tq * bp.Hq, 128, 16);
+    if (!rc) rc = bf16_tensor_map(&dm, bp.dout, (long long)bp.B * bp.Tq * bp.Hq, 128, 16);
+    if (!rc) rc = bf16_tensor_map_3d(&khm, t.k, 128, bp.Hkv, (long long)bp.B * bp.L, 128);
+    if (!rc) rc = bf16_tensor_map_3d(&klm, t.klo, 128, bp.Hkv, (long long)bp.B * bp.L, 128);
+    if (!rc) rc = bf16_tensor_map_3d(&vm, t.v, 128, bp.Hkv, (long long)bp.B * bp.L, 128);
+    if (rc) return rc;
+    constexpr int smem = KvSmem::ALLOC;
+    static_assert(smem <= 227 * 1024, "shared memory");
+    auto kern = nsa_kv_tc_kernel<SRC>;
+    rc = set_smem(kern, smem);
+    if (rc) return rc;
+    const int grid = (int)std::min<long long>(items, sm_count());
+    launch_k(__PRETTY_FUNCTION__, kern, grid, KV_THREADS, smem, st, qm, dm, khm, klm, vm, cp);
+    SA_CHECK_LAUNCH("nsa_kv_tc_kernel");
+    return SA_OK;
+}
+
 // Key-major dK / dV of a range branch (window, or compressed rows).
 template <int D, bool HILO>
 static int launch_bwd_kv(const BwdParams &p, cudaStream_t st) {
@@ -1461,6 +1513,7 @@ static int nsa_bwd_branches(const BwdParams &base, const float *gates, const flo
                             const __nv_bfloat16 *klo, const __nv_bfloat16 *vc, float *dkc, float *dvc,
                             const int32_t *sel, int sel_block, int sel_topk, int window, int cmp_len,
                             int cmp_stride, cudaStream_t st) {
+    float4 *scal = reinterpret_cast<float4 *>(ws + lay.scal_off);
     // compressed branch: keys Kc (hi/lo), gradients into dKc / dVc; writes dq
     BwdParams p = base;
     p.k = kc; p.klo = klo; p.v = vc; p.L = std::max(lay.nc, 1);
@@ -1471,7 +1524,8 @@ static int nsa_bwd_branches(const BwdParams &base, const float *gates, const flo
     int rc = dq_tc_allowed(p, D) ? launch_nsa_dq_tc<TS_CMP>(p, st)   // dq
                                  : launch_bwd_dq_tile<D, true>(p, st);
     if (rc) return rc;
-    rc = launch_bwd_kv<D, true>(p, st);                             // dKc, dVc
+    rc = kv_tc_allowed(p, D) ? launch_nsa_kv_tc<TS_CMP>(p, scal, st)   // dKc, dVc
+                             : launch_bwd_kv<D, true>(p, st);
     if (rc) return rc;
     // selected branch: keys of the chosen blocks
     p = base;
@@ -1490,7 +1544,8 @@ static int nsa_bwd_branches(const BwdParams &base, const float *gates, const flo
     rc = dq_tc_allowed(p, D) ? launch_nsa_dq_tc<TS_WINDOW>(p, st)       // dq
                              : launch_bwd_dq_tile<D, false>(p, st);
     if (rc) return rc;
-    return launch_bwd_kv<D, false>(p, st);                              // dk, dv
+    return kv_tc_allowed(p, D) ? launch_nsa_kv_tc<TS_WINDOW>(p, scal, st)   // dk, dv
+                               : launch_bwd_kv<D, false>(p, st);
 }
 
 int sa_nsa_bwd(const void *q, const void *k, const void *v, const float *gates, const void *dout,
