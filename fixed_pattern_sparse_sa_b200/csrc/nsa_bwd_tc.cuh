@@ -30,7 +30,7 @@
 namespace sa {
 
 constexpr int DQ_KT = 64;               // keys per tile
-constexpr int DQ_STAGES = 2;
+constexpr int DQ_STAGES = 3;
 constexpr int DQ_THREADS = 320;
 constexpr uint32_t DQ_TM_S = 0;         // S: 2 buffers x 64 fp32 columns
 constexpr uint32_t DQ_TM_DP = 128;      // dP: 2 buffers x 64
@@ -364,9 +364,10 @@ __global__ void __launch_bounds__(DQ_THREADS, 1)
 // of an item the score warps add dK * scale and dV to the global fp32 rows
 // (one reduction per key and column per item).  The per-row lse / D / gate
 // of a query tile come as one 1 KB bulk copy of a packed array
-// (nsa_kv_scalars_kernel).
+// (nsa_kv_scalars_kernel); three such stages are in flight.
 constexpr int KV_QT = 4;                 // queries per tile (x 16 heads = 64 columns)
 constexpr int KV_QSPLIT = 64;            // query tiles per item
+constexpr int KV_QSTAGES = 3;            // Q / dO / scalar stages
 constexpr int KV_THREADS = 320;
 // buffer b (b = 0, 1) at b * 128: S^T in columns 0-63, dP^T in 64-127; P^T
 // and dS^T overwrite them as bf16 pairs (score-warp half h writes the pairs of
@@ -384,9 +385,9 @@ struct KvSmem {                          // head dim 128
     static constexpr int QSTAGE = 2 * QT_BYTES + 1024;   // Q | dO | scalars (1 KB slot)
     static constexpr int OFF_K = 0;                      // K_hi | K_lo | V
     static constexpr int OFF_Q = OFF_K + 3 * KT_BYTES;
-    static constexpr int OFF_BAR = OFF_Q + 2 * QSTAGE;
-    // kv_full, kv_empty, q_full[2], q_empty[2], s_full[2], pd_full[2], pd_done[2], acc_full, acc_free, drain
-    static constexpr int N_BAR = 2 + 4 + 2 + 4 + 3;
+    static constexpr int OFF_BAR = OFF_Q + KV_QSTAGES * QSTAGE;
+    // kv_full, kv_empty, q_full[S], q_empty[S], s_full[2], pd_full[2], pd_done[2], acc_full, acc_free, drain
+    static constexpr int N_BAR = 2 + 2 * KV_QSTAGES + 6 + 3;
     static constexpr int OFF_MISC = OFF_BAR + N_BAR * 8;
     static constexpr int TOTAL = OFF_MISC + 16;
     static constexpr int ALLOC = TOTAL + 1024;
@@ -448,9 +449,9 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
     extern __shared__ unsigned char smem_raw[];
     unsigned char *smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::OFF_BAR);
-    uint64_t *kv_full = bars, *kv_empty = bars + 1, *q_full = bars + 2, *q_empty = bars + 4;
-    uint64_t *s_full = bars + 6, *pd_full = bars + 8, *pd_done = bars + 10;
-    uint64_t *acc_full = bars + 12, *acc_free = bars + 13, *drain = bars + 14;
+    uint64_t *kv_full = bars, *kv_empty = bars + 1, *q_full = bars + 2, *q_empty = q_full + KV_QSTAGES;
+    uint64_t *s_full = q_empty + KV_QSTAGES, *pd_full = s_full + 2, *pd_done = pd_full + 2;
+    uint64_t *acc_full = pd_done + 2, *acc_free = acc_full + 1, *drain = acc_free + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::OFF_MISC + 4);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -461,8 +462,8 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
     }
     if (tid == 0) {
         tc::mbar_init(kv_full, 1); tc::mbar_init(kv_empty, 1);
+        for (int i = 0; i < KV_QSTAGES; ++i) { tc::mbar_init(q_full + i, 1); tc::mbar_init(q_empty + i, 1); }
         for (int i = 0; i < 2; ++i) {
-            tc::mbar_init(q_full + i, 1); tc::mbar_init(q_empty + i, 1);
             tc::mbar_init(pd_full + i, 256); tc::mbar_init(pd_done + i, 1);
             tc::mbar_init(s_full + i, 1);
         }
@@ -501,8 +502,8 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
                 }
                 ++kn;
                 for (int i = 0; i < nq; ++i, ++qt) {
-                    const int qs = qt & 1;
-                    if (!atc::wait(q_empty + qs, ((qt >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+                    const int qs = qt % KV_QSTAGES;
+                    if (!atc::wait(q_empty + qs, ((qt / KV_QSTAGES) & 1) ^ 1, abort_flag)) { ok = false; break; }
                     unsigned char *dst = smem + L::OFF_Q + qs * L::QSTAGE;
                     const int t0 = (qt0 + i) * KV_QT;
                     atc::expect_tx(q_full + qs, 2 * L::QT_BYTES + L::SC_BYTES);
@@ -528,9 +529,9 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
             if (!ok) fail();
             // let the copies land before the CTA exits
             if (kn > 0) tc::mbar_wait_bounded(kv_full, (kn - 1) & 1, ATC_WAIT);
-            for (int i = 0; i < 2 && i < qt; ++i) {
+            for (int i = 0; i < KV_QSTAGES && i < qt; ++i) {
                 const int q = qt - 1 - i;
-                tc::mbar_wait_bounded(q_full + (q & 1), (q >> 1) & 1, ATC_WAIT);
+                tc::mbar_wait_bounded(q_full + q % KV_QSTAGES, (q / KV_QSTAGES) & 1, ATC_WAIT);
             }
         }
         __syncwarp();
@@ -545,8 +546,8 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
             // S^T and dP^T of query tile q (stage q & 1) into buffer q & 1, once
             // the dV / dK products of tile q - 2 (which read that buffer) are done
             auto issue_s = [&](int q) -> bool {
-                const int qs = q & 1, b = q & 1;
-                if (!atc::wait(q_full + qs, (q >> 1) & 1, abort_flag)) return false;
+                const int qs = q % KV_QSTAGES, b = q & 1;
+                if (!atc::wait(q_full + qs, (q / KV_QSTAGES) & 1, abort_flag)) return false;
                 if (q >= 2 && !atc::wait(pd_done + b, ((q >> 1) & 1) ^ 1, abort_flag)) return false;
                 tc::fence_after_sync();
                 const uint32_t qa = tc::smem_u32(smem + L::OFF_Q + qs * L::QSTAGE);
@@ -576,7 +577,7 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
                 // the previous item's epilogue must have read dV / dK
                 if (an > 0 && !atc::wait(acc_free, (an - 1) & 1, abort_flag)) { ok = false; break; }
                 for (int i = 0; i < nq; ++i, ++qt) {
-                    const int qs = qt & 1, pb = qt & 1;
+                    const int qs = qt % KV_QSTAGES, pb = qt & 1;
                     if (i + 1 < nq && !issue_s(qt + 1)) { ok = false; break; }
                     if (!atc::wait(pd_full + pb, (qt >> 1) & 1, abort_flag)) { ok = false; break; }
                     tc::fence_after_sync();
@@ -623,11 +624,11 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
             if (nq == 0) continue;
             const int j = kt * 128 + kr;                  // this thread's key
             for (int i = 0; i < nq; ++i, ++qt) {
-                const int qs = qt & 1, pb = qt & 1;
+                const int qs = qt % KV_QSTAGES, pb = qt & 1;
                 // S^T / dP^T of the tile (its MMA waited for the Q / dO stage, and
                 // with it the scalars' copy; the wait below makes them visible)
                 bool got = atc::wait(s_full + pb, (qt >> 1) & 1, abort_flag);
-                if (got) got = atc::wait(q_full + qs, (qt >> 1) & 1, abort_flag);
+                if (got) got = atc::wait(q_full + qs, (qt / KV_QSTAGES) & 1, abort_flag);
                 if (!atc::agree(pair, 64, got)) { ok = false; break; }
                 tc::fence_after_sync();
                 uint32_t sr[SC], dr[SC];
