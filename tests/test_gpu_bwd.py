@@ -160,6 +160,24 @@ def test_nsa_backward_parity(cuda_ok, T, Hq, Hkv, d, cfg):
     _close(dg, ref["dgates"], "dgates")
 
 
+def test_nsa_backward_two_sequences(cuda_ok):
+    # two sequences in one call: batch offsets of every kernel (the tcgen05
+    # dq and key-major passes, the inverse block lists, the pooling backward)
+    B, T, Hq, Hkv, d = 2, 420, 16, 2, 128
+    cfg = dict(cmp_len=32, cmp_stride=16, sel_block=64, sel_topk=3, window=96)
+    g = inputs.gen_nsa(B, T, Hq, Hkv, d, seed=77)
+    gen = torch.Generator().manual_seed(78)
+    dout = torch.randn(B, T, Hq, d, generator=gen).to(torch.bfloat16)
+    ref_f = oracle.nsa_fwd(g["q"], g["k"], g["v"], g["gates"], **cfg)
+    ref = oracle.nsa_bwd(g["q"], g["k"], g["v"], g["gates"], dout, ref_f["sel_idx"], **cfg)
+    out, sel, dq, dk, dv, dg = _nsa_bwd_gpu(g, dout, cfg)
+    assert np.array_equal(sel.cpu().numpy().reshape(ref_f["sel_idx"].shape), ref_f["sel_idx"])
+    _close(dq, ref["dq"], "dq")
+    _close(dk, ref["dk"], "dk")
+    _close(dv, ref["dv"], "dv")
+    _close(dg, ref["dgates"], "dgates")
+
+
 def test_nsa_backward_identities_8k(cuda_ok):
     # any input: sum_j dk_j = 0 per KV head; sum_j dv_j = the gate-weighted
     # dout of the group's heads over the branches that see at least one key
