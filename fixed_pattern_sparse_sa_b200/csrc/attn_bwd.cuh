@@ -19,15 +19,20 @@
 // with vector reductions (a key selected by several queries collects all of
 // their contributions).  D comes from a first pass (attn_bwd_prep_kernel).
 //
-// The same kernel runs the three NSA branches (Native Sparse Attention page,
+// The same kernel serves the NSA backward (Native Sparse Attention page,
 // "Puntos Clave": natively trainable, with a faster backward pass).  The key
 // source is a template parameter: explicit lists (BW_LIST), the keys of
-// selected blocks masked to j <= t (BW_BLOCKS), or a contiguous range per
-// query (BW_RANGE: the sliding window, or the compressed rows visible to
-// t).  Compressed keys come as a bf16 hi/lo pair (HILO) as in the forward.
-// A per-row factor (the branch gate) scales the upstream gradient, the LSE
-// is read with a stride (the forward stores the three branches' LSEs side by
-// side), and dq can accumulate over the branches' launches.
+// selected blocks masked to j <= t (BW_BLOCKS: the selected branch's dq), or
+// a contiguous range per query (BW_RANGE: the sliding window, or the
+// compressed rows visible to t, with the keys as a bf16 hi/lo pair (HILO) as
+// in the forward; the range branches normally take attn_bwd_dq_tile_kernel
+// or the tcgen05 kernels of nsa_bwd_tc.cuh instead).  A per-row factor (the
+// branch gate) scales the upstream gradient, the LSE is read with a stride
+// (the forward stores the three branches' LSEs side by side), and dq can
+// accumulate over the branches' launches.  The key-major
+// attn_bwd_kv_kernel below gives dk / dv without per-(query, key)
+// reductions for the range branches and, over inverse block lists, for the
+// selected blocks.
 #pragma once
 
 #include "attn_gather.cuh"
