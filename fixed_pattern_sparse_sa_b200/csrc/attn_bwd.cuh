@@ -850,6 +850,194 @@ __global__ void __launch_bounds__(DQ_WARPS * 32) attn_bwd_dq_tile_kernel(const B
     }
 }
 
+// dq of the NSA selected branch: one warp per (query, KV group) with at most
+// 16 heads.  The chunks are 16 consecutive keys of one selected block, only
+// those holding keys <= t (a block's chunk count is ceil(valid keys / 16));
+// the chunk -> block mapping is a ballot over the lanes' prefix counts.  K
+// and V chunks are gathered per warp by cp.async into a 3-stage ring; Q and
+// dO A fragments stay in registers; S = Q K^T, dP = dO V^T, dS = gate P
+// (dP - D), dq += dS K.
+constexpr int DQB_WARPS = 8;
+constexpr int DQB_STAGES = 3;
+
+template <int D>
+constexpr int attn_bwd_dq_blocks_smem() {
+    return DQB_WARPS * DQB_STAGES * 2 * 16 * D * 2;
+}
+
+template <int D>
+__global__ void __launch_bounds__(DQB_WARPS * 32) attn_bwd_dq_blocks_kernel(const BwdParams p) {
+    grid_dependency_sync();
+    constexpr int NK = 16;
+    constexpr int ROWB = D * 2;
+    constexpr int UNITS = ROWB / 16;
+    constexpr int KS_D = D / 16;
+    constexpr int NT_D = D / 8;
+    constexpr int CH = NK * ROWB;
+    constexpr int CP_ITERS = NK * UNITS / 32;
+    extern __shared__ __align__(1024) unsigned char smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int gr = lane >> 2, qc = lane & 3;
+    const long long item = (long long)blockIdx.x * DQB_WARPS + warp;
+    if (item >= (long long)p.B * p.Tq * p.Hkv) return;       // no block-wide barrier in this kernel
+    const int g = (int)(item % p.Hkv);
+    const long long bt = item / p.Hkv;
+    const int t = (int)(bt % p.Tq), b = (int)(bt / p.Tq);
+    const long long pos = p.q_pos0 + t;
+    unsigned char *wsm = smem + warp * (DQB_STAGES * 2 * CH);
+
+    const bool v0 = gr < p.G, v1 = gr + 8 < p.G;
+    const long long row0 = (bt * p.Hq + (long long)g * p.G + gr), row1 = row0 + 8;
+    float lse0 = v0 ? p.lse[row0 * p.lse_stride] : -INFINITY, lse1 = v1 ? p.lse[row1 * p.lse_stride] : -INFINITY;
+    const bool live0 = v0 && lse0 != -INFINITY, live1 = v1 && lse1 != -INFINITY;
+    lse0 *= kLog2e; lse1 *= kLog2e;
+    const float D0 = v0 ? p.Dt[row0] : 0.f, D1 = v1 ? p.Dt[row1] : 0.f;
+    const float gs0 = (p.gate && v0) ? p.gate[row0 * p.gate_stride] : 1.f;
+    const float gs1 = (p.gate && v1) ? p.gate[row1 * p.gate_stride] : 1.f;
+    unsigned qa[KS_D][4], da[KS_D][4];
+#pragma unroll
+    for (int ks = 0; ks < KS_D; ++ks) {
+        const int c0 = ks * 16 + 2 * qc;
+        const unsigned *q0 = reinterpret_cast<const unsigned *>(p.q + (v0 ? row0 : 0) * D + c0);
+        const unsigned *q1 = reinterpret_cast<const unsigned *>(p.q + (v1 ? row1 : 0) * D + c0);
+        const unsigned *d0 = reinterpret_cast<const unsigned *>(p.dout + (v0 ? row0 : 0) * D + c0);
+        const unsigned *d1 = reinterpret_cast<const unsigned *>(p.dout + (v1 ? row1 : 0) * D + c0);
+        qa[ks][0] = v0 ? __ldg(q0) : 0u; qa[ks][1] = v1 ? __ldg(q1) : 0u;
+        qa[ks][2] = v0 ? __ldg(q0 + 4) : 0u; qa[ks][3] = v1 ? __ldg(q1 + 4) : 0u;
+        da[ks][0] = v0 ? __ldg(d0) : 0u; da[ks][1] = v1 ? __ldg(d1) : 0u;
+        da[ks][2] = v0 ? __ldg(d0 + 4) : 0u; da[ks][3] = v1 ? __ldg(d1 + 4) : 0u;
+    }
+
+    // lane m < K: block m of the list, its first key, last visible key and chunk count
+    const int32_t *list = p.idx + (bt * p.idx_heads + (p.idx_heads == 1 ? 0 : g)) * p.K;
+    long long jb = 0, je = -1;
+    int nch = 0;
+    if (lane < p.K) {
+        const int blk = __ldg(list + lane);
+        if (blk >= 0) {
+            jb = (long long)blk * p.block;
+            if (jb >= p.L) {
+                raise_error(p.err, ERR_BAD_INDEX);
+            } else {
+                je = jb + p.block - 1;
+                if (je > pos) je = pos;
+                if (je > p.L - 1) je = p.L - 1;
+                if (je >= jb) nch = (int)((je - jb + NK) / NK);
+            }
+        }
+    }
+    int pre = nch;                                    // inclusive prefix of the chunk counts
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int x = __shfl_up_sync(0xffffffffu, pre, o);
+        if (lane >= o) pre += x;
+    }
+    const int n_chunks = __shfl_sync(0xffffffffu, pre, 31);
+    const int pex = pre - nch;                        // exclusive prefix
+    // chunk ci -> (first key, last key of its block)
+    auto chunk_of = [&](int ci, long long &j0, long long &jl) {
+        const unsigned m_mask = __ballot_sync(0xffffffffu, nch > 0 && pex <= ci);
+        const int m = 31 - __clz(m_mask);           // last block starting at or before ci
+        const int off = ci - __shfl_sync(0xffffffffu, pex, m);
+        j0 = __shfl_sync(0xffffffffu, jb, m) + (long long)off * NK;
+        jl = __shfl_sync(0xffffffffu, je, m);
+    };
+    const long long rstride = (long long)p.Hkv * D;
+    const __nv_bfloat16 *kbase = p.k + ((long long)b * p.L * p.Hkv + g) * D;
+    const __nv_bfloat16 *vbase = p.v + ((long long)b * p.L * p.Hkv + g) * D;
+    auto issue = [&](int ci) {
+        if (ci < n_chunks) {
+            long long j0, jl;
+            chunk_of(ci, j0, jl);
+            unsigned char *st = wsm + (ci % DQB_STAGES) * 2 * CH;
+#pragma unroll
+            for (int it = 0; it < CP_ITERS; ++it) {
+                const int lin = it * 32 + lane;
+                const int r = lin / UNITS, u = lin % UNITS;
+                const long long j = j0 + r;
+                const bool ok = j <= jl;
+                const long long off = ok ? j * rstride + u * 8 : 0;
+                const int sw = (u ^ (r & 7)) * 16;
+                cp_async16(st + r * ROWB + sw, kbase + off, ok ? 16 : 0);
+                cp_async16(st + CH + r * ROWB + sw, vbase + off, ok ? 16 : 0);
+            }
+        }
+        cp_async_commit();
+    };
+
+    float dqa[NT_D][4];
+#pragma unroll
+    for (int i = 0; i < NT_D; ++i) dqa[i][0] = dqa[i][1] = dqa[i][2] = dqa[i][3] = 0.f;
+    issue(0);
+    issue(1);
+    const int mi = lane >> 3, ri = lane & 7;
+    for (int ci = 0; ci < n_chunks; ++ci) {
+        issue(ci + 2);
+        cp_async_wait<2>();
+        __syncwarp();
+        long long j0, jl;
+        chunk_of(ci, j0, jl);
+        const int nvalid = (int)min((long long)NK, jl - j0 + 1);
+        const unsigned char *ks_ = wsm + (ci % DQB_STAGES) * 2 * CH;
+        const unsigned char *vs_ = ks_ + CH;
+        float sc[2][4], dp[2][4];
+#pragma unroll
+        for (int i = 0; i < 2; ++i) sc[i][0] = sc[i][1] = sc[i][2] = sc[i][3] = dp[i][0] = dp[i][1] = dp[i][2] = dp[i][3] = 0.f;
+        const int key = (mi >> 1) * 8 + ri;
+#pragma unroll
+        for (int ks = 0; ks < KS_D; ++ks) {
+            const int unit = ks * 2 + (mi & 1);
+            unsigned b0, b1, b2, b3;
+            ldsm_x4(b0, b1, b2, b3, ks_ + key * ROWB + ((unit ^ (key & 7)) * 16));
+            mma_bf16_16816(sc[0], qa[ks], b0, b1);
+            mma_bf16_16816(sc[1], qa[ks], b2, b3);
+            ldsm_x4(b0, b1, b2, b3, vs_ + key * ROWB + ((unit ^ (key & 7)) * 16));
+            mma_bf16_16816(dp[0], da[ks], b0, b1);
+            mma_bf16_16816(dp[1], da[ks], b2, b3);
+        }
+        float ds[2][4];
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int kk = nt * 8 + 2 * qc + (e & 1);
+                const bool hi = e >> 1;
+                const bool ok = kk < nvalid && (hi ? live1 : live0);
+                const float pv = ok ? exp2f(sc[nt][e] * p.scale_log2 - (hi ? lse1 : lse0)) : 0.f;
+                ds[nt][e] = pv * (hi ? gs1 : gs0) * (dp[nt][e] - (hi ? D1 : D0));
+            }
+        }
+        unsigned dsa[4];
+        dsa[0] = pack_bf16(ds[0][0], ds[0][1]); dsa[1] = pack_bf16(ds[0][2], ds[0][3]);
+        dsa[2] = pack_bf16(ds[1][0], ds[1][1]); dsa[3] = pack_bf16(ds[1][2], ds[1][3]);
+#pragma unroll
+        for (int dpi = 0; dpi < NT_D / 2; ++dpi) {
+            const int krow = (mi & 1) * 8 + ri;
+            const int unit = dpi * 2 + (mi >> 1);
+            unsigned b0, b1, b2, b3;
+            ldsm_x4_t(b0, b1, b2, b3, ks_ + krow * ROWB + ((unit ^ (krow & 7)) * 16));
+            mma_bf16_16816(dqa[2 * dpi], dsa, b0, b1);
+            mma_bf16_16816(dqa[2 * dpi + 1], dsa, b2, b3);
+        }
+        __syncwarp();
+    }
+    cp_async_wait<0>();
+#pragma unroll
+    for (int nt = 0; nt < NT_D; ++nt) {
+        const int col = nt * 8 + 2 * qc;
+        float2 a0 = make_float2(dqa[nt][0] * p.scale, dqa[nt][1] * p.scale);
+        float2 a1 = make_float2(dqa[nt][2] * p.scale, dqa[nt][3] * p.scale);
+        float2 *q0 = reinterpret_cast<float2 *>(p.dq + row0 * D + col);
+        float2 *q1 = reinterpret_cast<float2 *>(p.dq + row1 * D + col);
+        if (p.dq_accum) {
+            if (v0) { const float2 o = *q0; a0.x += o.x; a0.y += o.y; }
+            if (v1) { const float2 o = *q1; a1.x += o.x; a1.y += o.y; }
+        }
+        if (v0) *q0 = a0;
+        if (v1) *q1 = a1;
+    }
+}
+
 // Inverse of the block choice: per (b, g, block) the queries that chose it.
 // 1. counts per list
 __global__ void __launch_bounds__(256) bwd_sel_count_kernel(const int32_t *__restrict__ sel, long long n_entries,

@@ -1339,6 +1339,28 @@ static int launch_bwd_branch(const BwdParams &p, cudaStream_t st) {
     return SA_OK;
 }
 
+// dq of the selected branch, one warp per (query, KV group) (at most 16 heads
+// per KV head and 32 blocks); SA_NSA_BWD_SEL=v1 selects the generic kernel.
+template <int D>
+static int launch_bwd_dq_blocks(const BwdParams &p, cudaStream_t st) {
+    static int v = -1;
+    if (v < 0) {
+        const char *e = std::getenv("SA_NSA_BWD_SEL");
+        v = (e && std::strcmp(e, "v1") == 0) ? 0 : 1;
+    }
+    if (!v || p.G > 16 || p.K > 32) return launch_bwd_branch<D, BW_BLOCKS, false, false>(p, st);
+    constexpr int smem = attn_bwd_dq_blocks_smem<D>();
+    static_assert(smem <= 227 * 1024, "shared memory");
+    auto kern = attn_bwd_dq_blocks_kernel<D>;
+    int rc = set_smem(kern, smem);
+    if (rc) return rc;
+    const long long items = (long long)p.B * p.Tq * p.Hkv;
+    if (items == 0) return SA_OK;
+    launch_k(__PRETTY_FUNCTION__, kern, (unsigned)((items + DQB_WARPS - 1) / DQB_WARPS), DQB_WARPS * 32, smem, st, p);
+    SA_CHECK_LAUNCH("attn_bwd_dq_blocks_kernel");
+    return SA_OK;
+}
+
 // dq of a range branch with the key chunks shared by 8 consecutive queries.
 template <int D, bool HILO>
 static int launch_bwd_dq_tile(const BwdParams &p, cudaStream_t st) {
@@ -1533,7 +1555,7 @@ static int nsa_bwd_branches(const BwdParams &base, const float *gates, const flo
     p.idx = sel; p.idx_heads = base.Hkv; p.K = sel_topk; p.block = sel_block;
     p.block_shift = (sel_block & (sel_block - 1)) == 0 ? __builtin_ctz((unsigned)sel_block) : -1;
     p.dq_accum = 1;
-    rc = launch_bwd_branch<D, BW_BLOCKS, false, false>(p, st);          // dq
+    rc = launch_bwd_dq_blocks<D>(p, st);                                // dq
     if (rc) return rc;
     rc = launch_bwd_kv_lists<D>(p, lay, ws, sel, sel_block, sel_topk, st);   // dk, dv
     if (rc) return rc;
