@@ -295,7 +295,7 @@ __global__ void __launch_bounds__(NW * 32) attn_bwd_kernel(const BwdParams p) {
                     const int kk = nt * 8 + 2 * qc + (e & 1);
                     const bool hi = e >> 1;
                     const bool ok = ((vmask >> kk) & 1u) && (hi ? live1 : live0);
-                    const float pv = ok ? exp2f(sc[nt][e] * p.scale_log2 - (hi ? lse1 : lse0)) : 0.f;
+                    const float pv = ok ? ex2_fast(sc[nt][e] * p.scale_log2 - (hi ? lse1 : lse0)) : 0.f;
                     const float gv = pv * (hi ? gs1 : gs0);
                     pr[nt][e] = gv;
                     ds[nt][e] = gv * (dp[nt][e] - (hi ? D1 : D0));
@@ -611,7 +611,7 @@ __global__ void __launch_bounds__(KV_NWK * 32) attn_bwd_kv_kernel(const BwdParam
                     const int h = nt * 8 + 2 * qc + (e & 1);
                     const bool vk = (e >> 1) ? vk1 : vk0;
                     const float lh = fs[h];
-                    const float pv = (vk && lh != -INFINITY) ? exp2f(sc[nt][e] * p.scale_log2 - lh * kLog2e) : 0.f;
+                    const float pv = (vk && lh != -INFINITY) ? ex2_fast(sc[nt][e] * p.scale_log2 - lh * kLog2e) : 0.f;
                     const float gv = pv * fs[32 + h];
                     pg[nt][e] = gv;
                     ds[nt][e] = gv * (dp[nt][e] - fs[16 + h]);
@@ -807,7 +807,7 @@ __global__ void __launch_bounds__(DQ_WARPS * 32) attn_bwd_dq_tile_kernel(const B
                         const long long j = j0 + kh * 16 + nt * 8 + 2 * qc + (e & 1);
                         const bool hi = e >> 1;
                         const bool ok = j >= w_lo && j < w_hi && (hi ? live1 : live0);
-                        const float pv = ok ? exp2f(sc[nt][e] * p.scale_log2 - (hi ? lse1 : lse0)) : 0.f;
+                        const float pv = ok ? ex2_fast(sc[nt][e] * p.scale_log2 - (hi ? lse1 : lse0)) : 0.f;
                         ds[nt][e] = pv * (hi ? gs1 : gs0) * (dp[nt][e] - (hi ? D1 : D0));
                     }
                 }
@@ -1003,7 +1003,7 @@ __global__ void __launch_bounds__(DQB_WARPS * 32) attn_bwd_dq_blocks_kernel(cons
                 const int kk = nt * 8 + 2 * qc + (e & 1);
                 const bool hi = e >> 1;
                 const bool ok = kk < nvalid && (hi ? live1 : live0);
-                const float pv = ok ? exp2f(sc[nt][e] * p.scale_log2 - (hi ? lse1 : lse0)) : 0.f;
+                const float pv = ok ? ex2_fast(sc[nt][e] * p.scale_log2 - (hi ? lse1 : lse0)) : 0.f;
                 ds[nt][e] = pv * (hi ? gs1 : gs0) * (dp[nt][e] - (hi ? D1 : D0));
             }
         }

@@ -288,7 +288,7 @@ __global__ void __launch_bounds__(DQ_THREADS, 1)
                     for (int e = 0; e < 2; ++e) {
                         const int i = i0 + k + e;
                         const bool vis = i >= vlo && i < vhi;
-                        const float pv = vis ? exp2f(fmaf(__uint_as_float(sr[k + e]), p.scale_log2, nb)) : 0.f;
+                        const float pv = vis ? ex2_fast(fmaf(__uint_as_float(sr[k + e]), p.scale_log2, nb)) : 0.f;
                         ds2[e] = pv * gr_ * (__uint_as_float(dr[k + e]) - Dr);
                     }
                     pk[k / 2] = pack_bf16(ds2[0], ds2[1]);
@@ -657,7 +657,7 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
                         if constexpr (SRC == TS_CMP) vis = j < p.Lk && j * p.cmp_stride + p.cmp_len - 1 <= t;
                         else vis = j <= t && j > t - p.window;
                         vis = vis && t < p.T && s4.x != -INFINITY;
-                        const float pr = vis ? s4.z * exp2f(fmaf(__uint_as_float(sr[c + e]), p.scale_log2,
+                        const float pr = vis ? s4.z * ex2_fast(fmaf(__uint_as_float(sr[c + e]), p.scale_log2,
                                                                   -s4.x * kLog2e)) : 0.f;
                         pv[e] = pr;
                         dv2[e] = pr * (__uint_as_float(dr[c + e]) - s4.y);
