@@ -156,8 +156,8 @@ __global__ void __launch_bounds__(FS_WARPS * 32, 2) full_score_kernel(const Full
                             const long long j = j0 + nt * 8 + 2 * qc + c;
                             const bool kj = j < n_w;
                             float s = 0.f;
-                            if (kj && r0) s += exp2f(sc[nt][c] * p.scale_log2 - l0);
-                            if (kj && r1) s += exp2f(sc[nt][2 + c] * p.scale_log2 - l1);
+                            if (kj && r0) s += ex2_fast(sc[nt][c] * p.scale_log2 - l0);
+                            if (kj && r1) s += ex2_fast(sc[nt][2 + c] * p.scale_log2 - l1);
                             s += __shfl_xor_sync(0xffffffffu, s, 4);
                             s += __shfl_xor_sync(0xffffffffu, s, 8);
                             s += __shfl_xor_sync(0xffffffffu, s, 16);
