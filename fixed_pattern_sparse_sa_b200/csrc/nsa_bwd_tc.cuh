@@ -393,6 +393,11 @@ struct KvSmem {                          // head dim 128
     static constexpr int ALLOC = TOTAL + 1024;
 };
 
+// Key source of the key-major pass beside the two range branches: the
+// selected blocks, each a 64-key block (half of the 128 TMEM lanes, the rest
+// masked) walked over the queries of its inverse list.
+constexpr int KV_LISTS = 2;
+
 struct KvTcParams {
     TileParams t;            // k (K_hi), klo, v, shapes (T queries, Lk keys), window / cmp_len / cmp_stride, scale_log2
     const float4 *scal;      // [B, Hkv, T, 16] (lse natural, D, gate, 0) of this branch
@@ -401,7 +406,12 @@ struct KvTcParams {
     unsigned *err;
     int n_kt;                // key tiles per sequence
     int n_split;             // query splits per key tile
-    int n_items;             // B * Hkv * n_kt * n_split
+    int n_items;             // B * Hkv * n_kt * n_split (range branches)
+    // KV_LISTS: the inverse block lists (see bwd_sel_* kernels)
+    const int32_t *qlist, *qoff;
+    const int2 *items;
+    const int32_t *n_items_dev;
+    int nb, sel_block, list_split;
 };
 
 // Queries [q_lo, q_hi) that see at least one key of [j0, j1] (range branches).
@@ -416,24 +426,42 @@ __device__ __forceinline__ void kv_tc_range(const TileParams &p, int j0, int j1,
     }
 }
 
-// Item -> (b, g, key tile, first query tile, number of query tiles); 0 tiles = empty.
+// Item -> (b, g, keys [j0, jend), first query tile or list entry, list end);
+// returns the number of query tiles (0 = empty item).
 template <int SRC>
-__device__ __forceinline__ int kv_tc_item(const KvTcParams &cp, int it, int &b, int &g, int &kt, int &qt0) {
+__device__ __forceinline__ int kv_tc_item(const KvTcParams &cp, int it, int &b, int &g, int &j0, int &jend, int &qt0,
+                                          int &qlim) {
     const TileParams &p = cp.t;
-    const int s = it % cp.n_split;
-    int rem = it / cp.n_split;
-    kt = rem % cp.n_kt; rem /= cp.n_kt;
-    g = rem % p.Hkv;
-    b = rem / p.Hkv;
-    const int j0 = kt * 128, j1 = min(j0 + 127, p.Lk - 1);
-    int q_lo, q_hi;
-    kv_tc_range<SRC>(p, j0, j1, q_lo, q_hi);
-    if (q_lo >= q_hi) return 0;
-    const int a0 = q_lo / KV_QT;                               // first query tile (aligned)
-    const int n_all = (q_hi + KV_QT - 1) / KV_QT - a0;
-    qt0 = a0 + s * KV_QSPLIT;
-    const int n = n_all - s * KV_QSPLIT;
-    return n <= 0 ? 0 : min(n, KV_QSPLIT);
+    if constexpr (SRC == KV_LISTS) {
+        const int2 wi = cp.items[it];
+        const int blk = wi.x % cp.nb;
+        g = (wi.x / cp.nb) % p.Hkv;
+        b = wi.x / cp.nb / p.Hkv;
+        j0 = blk * cp.sel_block;
+        jend = min(j0 + cp.sel_block, p.Lk);
+        if (j0 >= jend) return 0;
+        const int o1 = cp.qoff[wi.x + 1];
+        qt0 = cp.qoff[wi.x] + wi.y * cp.list_split;           // first list entry
+        qlim = min(o1, qt0 + cp.list_split);
+        return qlim > qt0 ? (qlim - qt0 + KV_QT - 1) / KV_QT : 0;
+    } else {
+        const int s = it % cp.n_split;
+        int rem = it / cp.n_split;
+        const int kt = rem % cp.n_kt; rem /= cp.n_kt;
+        g = rem % p.Hkv;
+        b = rem / p.Hkv;
+        j0 = kt * 128;
+        jend = min(j0 + 128, p.Lk);
+        qlim = p.T;
+        int q_lo, q_hi;
+        kv_tc_range<SRC>(p, j0, jend - 1, q_lo, q_hi);
+        if (q_lo >= q_hi) return 0;
+        const int a0 = q_lo / KV_QT;                               // first query tile (aligned)
+        const int n_all = (q_hi + KV_QT - 1) / KV_QT - a0;
+        qt0 = a0 + s * KV_QSPLIT;
+        const int n = n_all - s * KV_QSPLIT;
+        return n <= 0 ? 0 : min(n, KV_QSPLIT);
+    }
 }
 
 template <int SRC>
@@ -444,6 +472,7 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
     grid_dependency_sync();
     constexpr int D = 128;
     constexpr bool LO = SRC == TS_CMP;
+    constexpr bool LS = SRC == KV_LISTS;
     using L = KvSmem;
     const TileParams &p = cp.t;
     extern __shared__ unsigned char smem_raw[];
@@ -480,21 +509,24 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
         raise_error(cp.err, ERR_TIMEOUT);
         *abort_flag = 1;
     };
+    const int n_items_all = LS ? *cp.n_items_dev : cp.n_items;
+    // query of list entry e of an item (entries past its end read its last one, masked later)
+    auto list_t = [&](int e, int qlim) -> int { return __ldg(cp.qlist + min(e, qlim - 1)); };
 
     if (warp == 0) {
         // ------------------------------------------------------ TMA producer
         if (lane == 0) {
             bool ok = true;
             int qt = 0, kn = 0;                           // query tiles and key tiles loaded
-            const int n_items = debug_stall() ? 0 : cp.n_items;
+            const int n_items = debug_stall() ? 0 : n_items_all;
             for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-                int b, g, kt, qt0;
-                const int nq = kv_tc_item<SRC>(cp, it, b, g, kt, qt0);
+                int b, g, j0, jend, qt0, qlim;
+                const int nq = kv_tc_item<SRC>(cp, it, b, g, j0, jend, qt0, qlim);
                 if (nq == 0) continue;
                 // the keys of the item, once the previous item's last MMA is done
                 if (!atc::wait(kv_empty, (kn & 1) ^ 1, abort_flag)) { ok = false; break; }
                 atc::expect_tx(kv_full, LO ? 3 * L::KT_BYTES : 2 * L::KT_BYTES);
-                const int z = b * p.Lk + kt * 128;
+                const int z = b * p.Lk + j0;
                 for (int h = 0; h < 2; ++h) {
                     atc::load_3d(smem + L::OFF_K + h * (128 * 128), &khimap, h * 64, g, z, kv_full);
                     if (LO) atc::load_3d(smem + L::OFF_K + L::KT_BYTES + h * (128 * 128), &klomap, h * 64, g, z, kv_full);
@@ -508,7 +540,8 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
                     const int t0 = (qt0 + i) * KV_QT;
                     atc::expect_tx(q_full + qs, 2 * L::QT_BYTES + L::SC_BYTES);
                     for (int w = 0; w < KV_QT; ++w) {
-                        const int qrow = (b * p.T + min(t0 + w, p.T - 1)) * p.Hq + g * p.G;
+                        const int tw = LS ? list_t(qt0 + i * KV_QT + w, qlim) : min(t0 + w, p.T - 1);
+                        const int qrow = (b * p.T + tw) * p.Hq + g * p.G;
                         for (int h = 0; h < 2; ++h) {
                             atc::load_2d(dst + h * (64 * 128) + w * (16 * 128), &qmap, h * 64, qrow, q_full + qs);
                             atc::load_2d(dst + L::QT_BYTES + h * (64 * 128) + w * (16 * 128), &domap, h * 64, qrow,
@@ -516,14 +549,27 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
                         }
                     }
                     // lse / D / gate of the tile's rows: 4 consecutive queries of (b, g), one 1 KB copy
-                    // (rows past the sequence read the last query's, masked later)
-                    const int tc0 = min(t0, p.T - KV_QT);
-                    const float4 *src = cp.scal + ((long long)(b * p.Hkv + g) * p.T + tc0) * 16;
-                    asm volatile(
-                        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
-                            tc::smem_u32(dst + 2 * L::QT_BYTES)),
-                        "l"(src), "r"(L::SC_BYTES), "r"(tc::smem_u32(q_full + qs))
-                        : "memory");
+                    // (rows past the sequence read the last query's, masked later); list queries one
+                    // 256 B copy each
+                    if constexpr (LS) {
+                        for (int w = 0; w < KV_QT; ++w) {
+                            const int tw = list_t(qt0 + i * KV_QT + w, qlim);
+                            const float4 *src = cp.scal + ((long long)(b * p.Hkv + g) * p.T + tw) * 16;
+                            asm volatile(
+                                "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+                                    tc::smem_u32(dst + 2 * L::QT_BYTES + w * 256)),
+                                "l"(src), "r"(256), "r"(tc::smem_u32(q_full + qs))
+                                : "memory");
+                        }
+                    } else {
+                        const int tc0 = min(t0, p.T - KV_QT);
+                        const float4 *src = cp.scal + ((long long)(b * p.Hkv + g) * p.T + tc0) * 16;
+                        asm volatile(
+                            "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+                                tc::smem_u32(dst + 2 * L::QT_BYTES)),
+                            "l"(src), "r"(L::SC_BYTES), "r"(tc::smem_u32(q_full + qs))
+                            : "memory");
+                    }
                 }
             }
             if (!ok) fail();
@@ -567,9 +613,9 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
                 tc::mma_commit(s_full + b);
                 return true;
             };
-            for (int it = blockIdx.x; it < cp.n_items && ok; it += gridDim.x) {
-                int b, g, kt, qt0;
-                const int nq = kv_tc_item<SRC>(cp, it, b, g, kt, qt0);
+            for (int it = blockIdx.x; it < n_items_all && ok; it += gridDim.x) {
+                int b, g, j0, jend, qt0, qlim;
+                const int nq = kv_tc_item<SRC>(cp, it, b, g, j0, jend, qt0, qlim);
                 if (nq == 0) continue;
                 if (!atc::wait(kv_full, kn & 1, abort_flag)) { ok = false; break; }
                 ++kn;
@@ -618,11 +664,11 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
         const uint32_t lrow = (uint32_t)(quad * 32) << 16;
         bool ok = true;
         int qt = 0, an = 0;
-        for (int it = blockIdx.x; it < cp.n_items && ok; it += gridDim.x) {
-            int b, g, kt, qt0;
-            const int nq = kv_tc_item<SRC>(cp, it, b, g, kt, qt0);
+        for (int it = blockIdx.x; it < n_items_all && ok; it += gridDim.x) {
+            int b, g, j0, jend, qt0, qlim;
+            const int nq = kv_tc_item<SRC>(cp, it, b, g, j0, jend, qt0, qlim);
             if (nq == 0) continue;
-            const int j = kt * 128 + kr;                  // this thread's key
+            const int j = j0 + kr;                        // this thread's key
             for (int i = 0; i < nq; ++i, ++qt) {
                 const int qs = qt % KV_QSTAGES, pb = qt & 1;
                 // S^T / dP^T of the tile (its MMA waited for the Q / dO stage, and
@@ -643,6 +689,17 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
                 const float4 *sc = reinterpret_cast<const float4 *>(smem + L::OFF_Q + qs * L::QSTAGE + 2 * L::QT_BYTES);
                 const int t0 = (qt0 + i) * KV_QT;
                 const int tc0 = min(t0, p.T - KV_QT);
+                // list queries of this warp's two columns groups (w = 2 half, 2 half + 1)
+                int tl[2] = {0, 0};
+                bool vl[2] = {false, false};
+                if constexpr (LS) {
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const int e = qt0 + i * KV_QT + 2 * half + u;
+                        vl[u] = e < qlim;
+                        tl[u] = list_t(e, qlim);
+                    }
+                }
                 uint32_t pp[SC / 2], dp2[SC / 2];
 #pragma unroll
                 for (int c = 0; c < SC; c += 2) {
@@ -650,13 +707,23 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
                         const int col = half * SC + c + e;         // q-row of the tile: query col/16, head col%16
-                        const int t = t0 + (col >> 4);
-                        // rows past the sequence read the last query's slot (masked below)
-                        const float4 s4 = sc[(min(t, p.T - 1) - tc0) * 16 + (col & 15)];
                         bool vis;
-                        if constexpr (SRC == TS_CMP) vis = j < p.Lk && j * p.cmp_stride + p.cmp_len - 1 <= t;
-                        else vis = j <= t && j > t - p.window;
-                        vis = vis && t < p.T && s4.x != -INFINITY;
+                        float4 s4;
+                        if constexpr (LS) {
+                            // the list query of column group col / 16 chose this key's block
+                            const int u = (col >> 4) & 1;
+                            const int t = tl[u];
+                            s4 = sc[col];
+                            vis = vl[u] && j < jend && j <= t;
+                        } else {
+                            const int t = t0 + (col >> 4);
+                            // rows past the sequence read the last query's slot (masked below)
+                            s4 = sc[(min(t, p.T - 1) - tc0) * 16 + (col & 15)];
+                            if constexpr (SRC == TS_CMP) vis = j < p.Lk && j * p.cmp_stride + p.cmp_len - 1 <= t;
+                            else vis = j <= t && j > t - p.window;
+                            vis = vis && t < p.T;
+                        }
+                        vis = vis && s4.x != -INFINITY;
                         const float pr = vis ? s4.z * ex2_fast(fmaf(__uint_as_float(sr[c + e]), p.scale_log2,
                                                                   -s4.x * kLog2e)) : 0.f;
                         pv[e] = pr;
@@ -676,7 +743,7 @@ __global__ void __launch_bounds__(KV_THREADS, 1)
             // ------------------------------------------------------ epilogue
             if (!atc::agree(pair, 64, atc::wait(acc_full, an & 1, abort_flag))) { ok = false; break; }
             tc::fence_after_sync();
-            const bool kv_ok = j < p.Lk;
+            const bool kv_ok = j < jend;
             float *dvr = cp.dv + (((long long)b * p.Lk + (kv_ok ? j : 0)) * p.Hkv + g) * D + half * OC;
             float *dkr = cp.dk + (((long long)b * p.Lk + (kv_ok ? j : 0)) * p.Hkv + g) * D + half * OC;
 #pragma unroll

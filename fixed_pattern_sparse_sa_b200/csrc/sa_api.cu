@@ -1516,6 +1516,36 @@ static int launch_bwd_kv_lists(const BwdParams &p, const NsaBwdLayout &lay, char
     launch_k("bwd_sel_fill_kernel", bwd_sel_fill_kernel, eg, 256, 0, st, sel, lay.n_entries, p.Tq, p.Hkv, sel_topk,
              lay.nb, cur, qlist);
     SA_CHECK_LAUNCH("bwd_sel_fill_kernel");
+    if (D == 128 && kv_tc_allowed(p, D) && sel_block <= 128) {
+        // tcgen05 key-major pass: each block in a 128-key tile, its list's queries in tiles of 4
+        float4 *scal = reinterpret_cast<float4 *>(ws + lay.scal_off);
+        const long long n_sc = (long long)p.B * p.Hkv * p.Tq * 16;
+        launch_k("nsa_kv_scalars_kernel", nsa_kv_scalars_kernel, (unsigned)((n_sc + 255) / 256), 256, 0, st,
+                 p.lse, p.lse_stride, (const float *)p.Dt, p.gate, p.gate_stride, p.B, p.Tq, p.Hq, p.Hkv, p.G, scal);
+        SA_CHECK_LAUNCH("nsa_kv_scalars_kernel");
+        KvTcParams cp{};
+        TileParams &t = cp.t;
+        t.q = p.q; t.k = p.k; t.klo = p.k; t.v = p.v;
+        t.B = p.B; t.T = p.Tq; t.Lk = p.L; t.Hq = p.Hq; t.Hkv = p.Hkv; t.G = p.G; t.scale_log2 = p.scale_log2;
+        cp.scal = scal; cp.dk = p.dk; cp.dv = p.dv; cp.scale = p.scale; cp.err = p.err;
+        cp.qlist = qlist; cp.qoff = qoff; cp.items = items; cp.n_items_dev = n_items;
+        cp.nb = lay.nb; cp.sel_block = sel_block; cp.list_split = KV_SEL_SPLIT;
+        static_assert(KV_SEL_SPLIT == KV_QSPLIT * KV_QT, "list work items are KV_QSPLIT query tiles");
+        CUtensorMap qm, dm, khm, vm;
+        int rc = bf16_tensor_map(&qm, p.q, (long long)p.B * p.Tq * p.Hq, 128, 16);
+        if (!rc) rc = bf16_tensor_map(&dm, p.dout, (long long)p.B * p.Tq * p.Hq, 128, 16);
+        if (!rc) rc = bf16_tensor_map_3d(&khm, p.k, 128, p.Hkv, (long long)p.B * p.L, 128);
+        if (!rc) rc = bf16_tensor_map_3d(&vm, p.v, 128, p.Hkv, (long long)p.B * p.L, 128);
+        if (rc) return rc;
+        constexpr int smem = KvSmem::ALLOC;
+        auto kern = nsa_kv_tc_kernel<KV_LISTS>;
+        rc = set_smem(kern, smem);
+        if (rc) return rc;
+        const int grid = (int)std::min<long long>(lay.max_items, sm_count());
+        launch_k(__PRETTY_FUNCTION__, kern, grid, KV_THREADS, smem, st, qm, dm, khm, khm, vm, cp);
+        SA_CHECK_LAUNCH("nsa_kv_tc_kernel");
+        return SA_OK;
+    }
     constexpr int smem = attn_bwd_kv_smem<D, false>();
     auto kern = attn_bwd_kv_kernel<D, false, true>;
     int rc = set_smem(kern, smem);
