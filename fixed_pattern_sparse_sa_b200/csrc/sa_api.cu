@@ -162,7 +162,7 @@ typedef CUresult (*TensorMapEncodeFn)(CUtensorMap *, CUtensorMapDataType, cuuint
                                       CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
                                       CUtensorMapFloatOOBfill);
 
-// The driver's tensor-map encoder, looked up once through the runtime (no
+// The CUDA driver API's tensor-map encoder, looked up once through the runtime (no
 // link-time dependency on libcuda).
 static TensorMapEncodeFn tensor_map_encoder() {
     static TensorMapEncodeFn fn = nullptr;
