@@ -9,8 +9,11 @@ of the whole step, summed over ranks (each rank runs its own sequence: weak
 scaling, no data-path collective).
 
 Extra measurements on the same JSON line: the 128K-context decode step with
-IndexCache (F S S S and all-F) in tokens/s, the NSA three-branch forward at
-64K in TFLOP/s, and the fixed-graph workload (16384 tokens) in GB/s.
+IndexCache (F S S S and all-F) in tokens/s, the IndexCache prefill (4 x 64K),
+the HySparse2-shaped prefill (window 128 + top-1024) and the HySparse2 full
+layer as the exact indexer, the backward of the sparse attention and of NSA,
+the NSA three-branch forward at 64K in TFLOP/s, the fixed-graph workload
+(16384 tokens) in GB/s, and the L2 gather-ceiling probe.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 Under torchrun every rank runs; rank 0 prints one JSON line.
