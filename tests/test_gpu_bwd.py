@@ -142,6 +142,8 @@ def _nsa_bwd_gpu(g, dout, cfg):
     (200, 12, 1, 128, dict(cmp_len=32, cmp_stride=16, sel_block=64, sel_topk=16, window=512)),
     # T shorter than one compressed window: the compressed branch is empty
     (20, 4, 1, 64, dict(cmp_len=32, cmp_stride=16, sel_block=16, sel_topk=2, window=8)),
+    # the same at head dim 128 (the tcgen05 dq pass writes dq with no key tile)
+    (21, 16, 1, 128, dict(cmp_len=32, cmp_stride=16, sel_block=16, sel_topk=2, window=8)),
     # the 64K workload's branch settings on a ragged 2065-token sequence: several
     # 256 / 512-query splits per key block, block lists longer than one work item
     (2065, 16, 1, 128, dict(cmp_len=32, cmp_stride=16, sel_block=64, sel_topk=16, window=512)),
