@@ -101,3 +101,20 @@ def test_full_attn_indexer_16k_sampled_rows(cuda_ok):
     assert torch.all(valid[:, :-1] | ~valid[:, 1:])             # entries first, then padding
     assert torch.all((ii[:, 1:] > ii[:, :-1]) | ~valid[:, 1:])  # ascending
     assert torch.all(ii.max(dim=1).values.cpu() == t)
+
+
+def test_full_attn_indexer_32k_row_chunks(cuda_ok):
+    # 32768 tokens: the dense scores are taken in four chunks of 8192 query
+    # rows (1 GiB each); sampled rows on both sides of every chunk boundary
+    B, T, Hq, Hkv, d, topk, window = 1, 32768, 16, 1, 128, 1024, 128
+    g = inputs.gen_dsa(B, T, Hq, Hkv, d, 1, 32, seed=12)
+    q, k, v = g["q"], g["k"], g["v"]
+    out, lse, idx = api.full_attn_topk(q.cuda(), k.cuda(), v.cuda(), topk, window)
+    api.check_device_status()
+    rows = np.array([3, 8191, 8192, 8193, 16383, 16384, 24575, 24576, T - 1])
+    ref_out, ref_lse, ref_idx, sc = oracle.full_attn_topk(q, k, v, topk, window, rows=rows,
+                                                          want_scores=True)
+    _check_out(out, lse, ref_out, ref_lse, rows)
+    _check_sets(idx, ref_idx, sc, topk, window, T, rows)
+    cnt = (idx[0] >= 0).sum(dim=1).cpu()
+    assert torch.equal(cnt, torch.clamp(torch.arange(T) + 1, max=topk + window))
