@@ -21,8 +21,18 @@
 // over the heads stay in fp32 (shuffles across the row groups of the
 // fragment).  Groups are the outer loop; a group after the first adds to the
 // scores the same lanes wrote for the previous one.
+//
+// full_score_tc_kernel is the same pass on the tcgen05 tensor cores for head
+// dim 128 and 16 query heads per KV head, key-major: a 128-key tile of K is
+// the M side and the 16 queries x 16 heads of a query block the N side,
+//   S^T[128 keys x 256 (query, head)] = K_tile . Q_blk^T     (kind::f16)
+// into one of two 256-column TMEM buffers.  A score thread owns one key (one
+// TMEM lane) and eight queries, so the sum over the heads is a sum of the 16
+// columns of a query in its own registers: no shuffles; a warp stores 128
+// bytes of a dense row per query.
 #pragma once
 
+#include "attn_tc.cuh"
 #include "sa_common.cuh"
 
 namespace sa {
@@ -186,6 +196,256 @@ __global__ void __launch_bounds__(FS_WARPS * 32, 2) full_score_kernel(const Full
         cp_async_wait<0>();
         __syncthreads();
     }
+}
+
+// ------------------------------------------------- tcgen05 form (d = 128)
+constexpr int FX_QB = 16;                 // queries per block (x 16 heads = 256 columns)
+constexpr int FX_KT = 128;                // keys per tile
+constexpr int FX_KSTAGES = 4;
+constexpr int FX_PIECE = 32;              // key tiles per work item
+constexpr int FX_THREADS = 320;
+constexpr uint32_t FX_TM_COLS = 512;      // two S buffers of 256 columns
+
+struct FxSmem {
+    static constexpr int Q_BYTES = FX_QB * 16 * 256;      // 2 halves x 256 rows x 128 B
+    static constexpr int K_BYTES = FX_KT * 256;           // 2 halves x 128 rows x 128 B
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_K = OFF_Q + Q_BYTES;
+    static constexpr int OFF_LSE = OFF_K + FX_KSTAGES * K_BYTES;   // [16 queries][16 heads] natural lse
+    static constexpr int OFF_BAR = OFF_LSE + FX_QB * 16 * 4;
+    // q_full, q_empty, lse_free, k_full[S], k_empty[S], s_full[2], s_empty[2], drain
+    static constexpr int N_BAR = 3 + 2 * FX_KSTAGES + 4 + 1;
+    static constexpr int OFF_MISC = OFF_BAR + N_BAR * 8;           // tmem slot, abort flag
+    static constexpr int TOTAL = OFF_MISC + 16;
+    static constexpr int ALLOC = TOTAL + 1024;
+};
+
+struct FxParams {
+    FullScoreParams f;
+    int nqb;            // query blocks per batch element (ceil(Rt / 16))
+    int n_items;        // n_piece * B * nqb
+    unsigned *err;
+};
+
+// Item -> (b, query block, first key tile, tile count); 0 = empty item.
+// Pieces are the slow index, so every block's first piece comes first.
+__device__ __forceinline__ int fx_item(const FxParams &cp, int it, int &b, int &qb, int &kt0) {
+    const FullScoreParams &p = cp.f;
+    const int per = p.B * cp.nqb;
+    const int s = it / per, r = it % per;
+    b = r / cp.nqb;
+    qb = r % cp.nqb;
+    const int tr_last = min(qb * FX_QB + FX_QB, p.Rt) - 1;
+    const long long n_max = fs_candidates((long long)p.t0 + tr_last, p.window);
+    const int n_kt = (int)((n_max + FX_KT - 1) / FX_KT);
+    kt0 = s * FX_PIECE;
+    return kt0 < n_kt ? min(FX_PIECE, n_kt - kt0) : 0;
+}
+
+__global__ void __launch_bounds__(FX_THREADS, 1)
+    full_score_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
+                         const FxParams cp) {
+    grid_dependency_sync();
+    using L = FxSmem;
+    const FullScoreParams &p = cp.f;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::OFF_BAR);
+    uint64_t *q_full = bars, *q_empty = bars + 1, *lse_free = bars + 2;
+    uint64_t *k_full = bars + 3, *k_empty = k_full + FX_KSTAGES;
+    uint64_t *s_full = k_empty + FX_KSTAGES, *s_empty = s_full + 2, *drain = s_empty + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::OFF_MISC);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::OFF_MISC + 4);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    if (warp == 1) {
+        tc::tmem_alloc(tmem_slot, FX_TM_COLS);
+        tc::tmem_relinquish();
+    }
+    if (tid == 0) {
+        tc::mbar_init(q_full, 1); tc::mbar_init(q_empty, 1); tc::mbar_init(lse_free, 256);
+        for (int i = 0; i < FX_KSTAGES; ++i) { tc::mbar_init(k_full + i, 1); tc::mbar_init(k_empty + i, 1); }
+        for (int i = 0; i < 2; ++i) { tc::mbar_init(s_full + i, 1); tc::mbar_init(s_empty + i, 256); }
+        tc::mbar_init(drain, 1);
+        *abort_flag = 0;
+        tc::mbar_fence_init();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    auto fail = [&]() {
+        raise_error(cp.err, ERR_TIMEOUT);
+        *abort_flag = 1;
+    };
+
+    if (warp == 0) {
+        // ------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            bool ok = true;
+            int qn = 0, kn = 0;                           // Q blocks and K tiles issued
+            const int n_items = debug_stall() ? 0 : cp.n_items;
+            for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+                int b, qb, kt0;
+                const int nt = fx_item(cp, it, b, qb, kt0);
+                if (nt == 0) continue;
+                const int tb = p.t0 + qb * FX_QB;         // first query of the block
+                for (int g = 0; g < p.Hkv && ok; ++g) {
+                    // the previous block's last MMA and last score reads are done
+                    if (qn > 0 && (!atc::wait(q_empty, (qn - 1) & 1, abort_flag) ||
+                                   !atc::wait(lse_free, (qn - 1) & 1, abort_flag))) { ok = false; break; }
+                    atc::expect_tx(q_full, L::Q_BYTES + FX_QB * 64);
+                    for (int w = 0; w < FX_QB; ++w) {
+                        // queries past the sequence load the last one (masked by the score warps)
+                        const int tw = min(tb + w, p.T - 1);
+                        const int qrow = (b * p.T + tw) * p.Hq + g * 16;
+                        for (int h = 0; h < 2; ++h)
+                            atc::load_2d(smem + L::OFF_Q + h * (FX_QB * 16 * 128) + w * (16 * 128), &qmap, h * 64,
+                                         qrow, q_full);
+                        asm volatile(
+                            "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+                                tc::smem_u32(smem + L::OFF_LSE + w * 64)),
+                            "l"(p.lse + (long long)qrow), "r"(64), "r"(tc::smem_u32(q_full))
+                            : "memory");
+                    }
+                    ++qn;
+                    for (int i = 0; i < nt; ++i) {
+                        const int ks = kn % FX_KSTAGES;
+                        if (!atc::wait(k_empty + ks, ((kn / FX_KSTAGES) & 1) ^ 1, abort_flag)) { ok = false; break; }
+                        atc::expect_tx(k_full + ks, L::K_BYTES);
+                        const int z = b * p.T + (kt0 + i) * FX_KT;
+                        for (int h = 0; h < 2; ++h)
+                            atc::load_3d(smem + L::OFF_K + ks * L::K_BYTES + h * (FX_KT * 128), &kmap, h * 64, g, z,
+                                         k_full + ks);
+                        ++kn;
+                    }
+                }
+            }
+            if (!ok) fail();
+            // let the copies land before the CTA exits
+            if (qn > 0) tc::mbar_wait_bounded(q_full, (qn - 1) & 1, ATC_WAIT);
+            for (int i = 0; i < FX_KSTAGES && i < kn; ++i) {
+                const int q = kn - 1 - i;
+                tc::mbar_wait_bounded(k_full + q % FX_KSTAGES, (q / FX_KSTAGES) & 1, ATC_WAIT);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // --------------------------------------------------------------- MMA
+        if (lane == 0) {
+            constexpr uint32_t ID = tc::make_idesc(1, 1, 128, 256);
+            const uint32_t qa = tc::smem_u32(smem + L::OFF_Q);
+            bool ok = true;
+            int qn = 0, kn = 0;
+            for (int it = blockIdx.x; it < cp.n_items && ok; it += gridDim.x) {
+                int b, qb, kt0;
+                const int nt = fx_item(cp, it, b, qb, kt0);
+                if (nt == 0) continue;
+                for (int g = 0; g < p.Hkv && ok; ++g) {
+                    if (!atc::wait(q_full, qn & 1, abort_flag)) { ok = false; break; }
+                    ++qn;
+                    for (int i = 0; i < nt; ++i) {
+                        const int ks = kn % FX_KSTAGES, sb = kn & 1;
+                        if (!atc::wait(k_full + ks, (kn / FX_KSTAGES) & 1, abort_flag)) { ok = false; break; }
+                        // buffer sb was last read by the score warps for tile kn - 2
+                        if (kn >= 2 && !atc::wait(s_empty + sb, ((kn >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+                        tc::fence_after_sync();
+                        const uint32_t ka = tc::smem_u32(smem + L::OFF_K + ks * L::K_BYTES);
+#pragma unroll
+                        for (int kq = 0; kq < 8; ++kq) {
+                            const int h = kq / 4, kk = kq % 4;
+                            const uint64_t ad = atc::desc_sw128(ka + h * (FX_KT * 128) + kk * 32, 16, 1024);
+                            const uint64_t bd = atc::desc_sw128(qa + h * (FX_QB * 16 * 128) + kk * 32, 16, 1024);
+                            tc::mma_bf16(tmem + sb * 256, ad, bd, ID, kq > 0 ? 1u : 0u);
+                        }
+                        tc::mma_commit(k_empty + ks);
+                        tc::mma_commit(s_full + sb);
+                        ++kn;
+                    }
+                    if (!ok) break;
+                    tc::mma_commit(q_empty);
+                }
+            }
+            if (!ok) fail();
+            tc::mma_commit(drain);
+            tc::mbar_wait_bounded(drain, 0, ATC_WAIT);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------ score warps
+        // Thread = one key of the tile (TMEM lane); the two warps of a lane
+        // quadrant take the block's queries 0-7 / 8-15 (columns 0-127 / 128-255).
+        const int quad = warp & 3, half = (warp - 2) >> 2;
+        const int kr = quad * 32 + lane;
+        const uint32_t lrow = (uint32_t)(quad * 32) << 16;
+        const float4 *ls = reinterpret_cast<const float4 *>(smem + L::OFF_LSE) + half * 8 * 4;
+        bool ok = true;
+        int qn = 0, kn = 0;
+        for (int it = blockIdx.x; it < cp.n_items && ok; it += gridDim.x) {
+            int b, qb, kt0;
+            const int nt = fx_item(cp, it, b, qb, kt0);
+            if (nt == 0) continue;
+            // this thread's eight queries: chunk rows trb .. trb + 7 and their candidate counts
+            const int trb = qb * FX_QB + half * 8;
+            int nw[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                nw[u] = trb + u < p.Rt ? (int)fs_candidates((long long)p.t0 + trb + u, p.window) : 0;
+            int32_t *drow = p.dense + ((long long)b * p.Rt + min(trb, p.Rt - 1)) * p.stride;
+            for (int g = 0; g < p.Hkv && ok; ++g) {
+                // the block's Q and lse (the wait makes the lse copy visible)
+                if (!__all_sync(0xffffffffu, atc::wait(q_full, qn & 1, abort_flag))) { ok = false; break; }
+                ++qn;
+                for (int i = 0; i < nt; ++i) {
+                    const int sb = kn & 1;
+                    if (!__all_sync(0xffffffffu, atc::wait(s_full + sb, (kn >> 1) & 1, abort_flag))) {
+                        ok = false;
+                        break;
+                    }
+                    tc::fence_after_sync();
+                    const int j = (kt0 + i) * FX_KT + kr;
+#pragma unroll
+                    for (int part = 0; part < 2; ++part) {
+                        uint32_t sr[64];
+#pragma unroll
+                        for (int c = 0; c < 4; ++c)
+                            tc::tmem_ld16(tmem + lrow + sb * 256 + half * 128 + part * 64 + c * 16,
+                                          *reinterpret_cast<uint32_t(*)[16]>(sr + c * 16));
+                        tc::tmem_ld_wait();
+                        if (part == 1) {
+                            tc::fence_before_sync();
+                            atc::arrive(s_empty + sb);
+                        }
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            const int u = part * 4 + c;
+                            float acc = 0.f;
+#pragma unroll
+                            for (int h4 = 0; h4 < 4; ++h4) {
+                                const float4 l = ls[u * 4 + h4];
+                                const uint32_t *s4 = sr + c * 16 + h4 * 4;
+                                acc += ex2_fast(fmaf(__uint_as_float(s4[0]), p.scale_log2, -l.x * kLog2e));
+                                acc += ex2_fast(fmaf(__uint_as_float(s4[1]), p.scale_log2, -l.y * kLog2e));
+                                acc += ex2_fast(fmaf(__uint_as_float(s4[2]), p.scale_log2, -l.z * kLog2e));
+                                acc += ex2_fast(fmaf(__uint_as_float(s4[3]), p.scale_log2, -l.w * kLog2e));
+                            }
+                            if (j < nw[u]) {
+                                int32_t *dp = drow + (long long)u * p.stride + j;
+                                *dp = __float_as_int(g > 0 ? acc + __int_as_float(*dp) : acc);
+                            }
+                        }
+                    }
+                    ++kn;
+                }
+                if (!ok) break;
+                atc::arrive(lse_free);
+            }
+        }
+        if (!ok) fail();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 1) tc::tmem_dealloc(tmem, FX_TM_COLS);
 }
 
 // fp32 -> bf16 rows (the full layer's output)

@@ -1728,6 +1728,44 @@ static int launch_full_score(const FullScoreParams &p, cudaStream_t st) {
     return SA_OK;
 }
 
+// The score pass on the tensor cores (head dim 128, 16 query heads per KV
+// head); SA_FULL_SCORE=mma selects the mma.sync kernel.
+static bool full_score_tc_allowed(const FullScoreParams &p, int d) {
+    static int v = -1;
+    if (v < 0) {
+        const char *e = std::getenv("SA_FULL_SCORE");
+        v = (e && std::strcmp(e, "mma") == 0) ? 0 : 1;
+    }
+    return v && d == 128 && p.G == 16 && aligned16(p.lse) && (long long)p.B * p.T * p.Hq + 16 < INT_MAX &&
+           (long long)p.B * p.T + FX_KT < INT_MAX;
+}
+
+static int launch_full_score_tc(const FullScoreParams &fp, unsigned *ew, cudaStream_t st) {
+    FxParams cp{};
+    cp.f = fp;
+    cp.err = ew;
+    cp.nqb = (fp.Rt + FX_QB - 1) / FX_QB;
+    const long long t_last = (long long)fp.t0 + fp.Rt - 1;
+    const long long n_max = std::max(0LL, fp.window > 0 ? t_last - fp.window + 1 : t_last + 1);
+    const long long n_piece = ((n_max + FX_KT - 1) / FX_KT + FX_PIECE - 1) / FX_PIECE;
+    const long long items = n_piece * fp.B * cp.nqb;
+    if (items == 0) return SA_OK;
+    if (items > INT_MAX) return fail(SA_ERR_UNSUPPORTED, "full_score_tc: %lld items", items);
+    cp.n_items = (int)items;
+    CUtensorMap qm, km;
+    int rc = bf16_tensor_map(&qm, fp.q, (long long)fp.B * fp.T * fp.Hq, 128, 16);
+    if (!rc) rc = bf16_tensor_map_3d(&km, fp.k, 128, fp.Hkv, (long long)fp.B * fp.T, FX_KT);
+    if (rc) return rc;
+    constexpr int smem = FxSmem::ALLOC;
+    static_assert(smem <= 227 * 1024, "shared memory");
+    rc = set_smem(full_score_tc_kernel, smem);
+    if (rc) return rc;
+    const int grid = (int)std::min<long long>(items, sm_count());
+    launch_k("full_score_tc_kernel", full_score_tc_kernel, grid, FX_THREADS, smem, st, qm, km, cp);
+    SA_CHECK_LAUNCH("full_score_tc_kernel");
+    return SA_OK;
+}
+
 template <int NT>
 static int launch_select_dense(const IdxParams &p, int words, cudaStream_t st) {
     const int smem = select_smem_staged<64>(words, 0);
@@ -1794,7 +1832,9 @@ int sa_full_attn_topk(const void *q, const void *k, const void *v, int B, int T,
         fp.B = B; fp.T = T; fp.Hq = Hq; fp.Hkv = Hkv; fp.G = G;
         fp.t0 = t0; fp.Rt = Rt; fp.window = window; fp.scale_log2 = scale * kLog2e;
         fp.dense = dense; fp.stride = lay.stride;
-        rc = d == 64 ? launch_full_score<64>(fp, st) : launch_full_score<128>(fp, st);
+        rc = full_score_tc_allowed(fp, d) ? launch_full_score_tc(fp, ew, st)
+             : d == 64                    ? launch_full_score<64>(fp, st)
+                                          : launch_full_score<128>(fp, st);
         if (rc) return rc;
         IdxParams ip{};
         ip.B = B; ip.Tq = T; ip.L = T; ip.q_pos0 = 0; ip.window = window; ip.topk = topk;
