@@ -212,7 +212,8 @@ struct FxSmem {
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_K = OFF_Q + Q_BYTES;
     static constexpr int OFF_LSE = OFF_K + FX_KSTAGES * K_BYTES;   // [16 queries][16 heads] natural lse
-    static constexpr int OFF_BAR = OFF_LSE + FX_QB * 16 * 4;
+    static constexpr int OFF_NL = OFF_LSE + FX_QB * 16 * 4;       // per score warp: -lse * log2(e) of its 8 queries
+    static constexpr int OFF_BAR = OFF_NL + 8 * 8 * 16 * 4;
     // q_full, q_empty, lse_free, k_full[S], k_empty[S], s_full[2], s_empty[2], drain
     static constexpr int N_BAR = 3 + 2 * FX_KSTAGES + 4 + 1;
     static constexpr int OFF_MISC = OFF_BAR + N_BAR * 8;           // tmem slot, abort flag
@@ -379,6 +380,7 @@ __global__ void __launch_bounds__(FX_THREADS, 1)
         const int kr = quad * 32 + lane;
         const uint32_t lrow = (uint32_t)(quad * 32) << 16;
         const float4 *ls = reinterpret_cast<const float4 *>(smem + L::OFF_LSE) + half * 8 * 4;
+        float4 *nl = reinterpret_cast<float4 *>(smem + L::OFF_NL) + (warp - 2) * 8 * 4;
         bool ok = true;
         int qn = 0, kn = 0;
         for (int it = blockIdx.x; it < cp.n_items && ok; it += gridDim.x) {
@@ -396,6 +398,11 @@ __global__ void __launch_bounds__(FX_THREADS, 1)
                 // the block's Q and lse (the wait makes the lse copy visible)
                 if (!__all_sync(0xffffffffu, atc::wait(q_full, qn & 1, abort_flag))) { ok = false; break; }
                 ++qn;
+                {   // this warp's copy of -lse * log2(e) for its 8 queries x 16 heads
+                    const float4 l = ls[lane];
+                    nl[lane] = make_float4(-l.x * kLog2e, -l.y * kLog2e, -l.z * kLog2e, -l.w * kLog2e);
+                    __syncwarp();
+                }
                 for (int i = 0; i < nt; ++i) {
                     const int sb = kn & 1;
                     if (!__all_sync(0xffffffffu, atc::wait(s_full + sb, (kn >> 1) & 1, abort_flag))) {
@@ -422,12 +429,13 @@ __global__ void __launch_bounds__(FX_THREADS, 1)
                             float acc = 0.f;
 #pragma unroll
                             for (int h4 = 0; h4 < 4; ++h4) {
-                                const float4 l = ls[u * 4 + h4];
-                                const uint32_t *s4 = sr + c * 16 + h4 * 4;
-                                acc += ex2_fast(fmaf(__uint_as_float(s4[0]), p.scale_log2, -l.x * kLog2e));
-                                acc += ex2_fast(fmaf(__uint_as_float(s4[1]), p.scale_log2, -l.y * kLog2e));
-                                acc += ex2_fast(fmaf(__uint_as_float(s4[2]), p.scale_log2, -l.z * kLog2e));
-                                acc += ex2_fast(fmaf(__uint_as_float(s4[3]), p.scale_log2, -l.w * kLog2e));
+                                const float4 l = nl[u * 4 + h4];
+                                const float lv[4] = {l.x, l.y, l.z, l.w};
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    const float x = fmaf(__uint_as_float(sr[c * 16 + h4 * 4 + e]), p.scale_log2, lv[e]);
+                                    acc += ex2_fast(x);
+                                }
                             }
                             if (j < nw[u]) {
                                 int32_t *dp = drow + (long long)u * p.stride + j;
