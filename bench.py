@@ -574,6 +574,7 @@ def extra_measurements(args, dev, torch, api, lib, inputs, flush, world, peaks, 
         res[f"hysparse2_full_indexer{T // 1024}k"] = {
             "ms_per_step": round(ms, 3), "tflops": round(world * ffl / (ms / 1e3) / 1e12, 2),
             "algorithmic_flops": ffl,
+            "tensor_frac": round(ffl / (ms / 1e3) / 1e12 / peaks["bf16_tflops"], 4),
             "note": "full causal attention layer (out, lse) + exact head-summed probability scores + "
                     f"window 128 / top-1024 selection; 1 x {T} tokens, 16 q heads / 1 kv head, d=128"}
         del gf, gfd, fout, flse, fidx, fws
