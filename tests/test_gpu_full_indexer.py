@@ -70,6 +70,7 @@ def _check_sets(idx, ref_idx, sc, topk, window, T, rows):
     (1, 2065, 16, 1, 128, 1024, 128),   # the HySparse2 selection, ragged, several score chunks of keys
     (1, 700, 32, 2, 128, 100, 32),      # two KV groups of 16 heads on the tcgen05 score pass
     (2, 333, 16, 1, 128, 50, 0),        # two sequences, no window, ragged query blocks
+    (2, 450, 64, 4, 128, 60, 8),        # four KV groups of 16 heads, two sequences
 ])
 def test_full_attn_indexer_parity(cuda_ok, B, T, Hq, Hkv, d, topk, window):
     g = inputs.gen_dsa(B, T, Hq, Hkv, d, 1, 32, seed=T + d)
