@@ -29,7 +29,14 @@
 // into one of two 256-column TMEM buffers.  A score thread owns one key (one
 // TMEM lane) and eight queries, so the sum over the heads is a sum of the 16
 // columns of a query in its own registers: no shuffles; a warp stores 128
-// bytes of a dense row per query.
+// bytes of a dense row per query.  Warp roles (320 threads, one persistent
+// CTA per SM): warp 0 loads the block's Q (TMA) and lse (bulk copies) and a
+// 4-stage ring of K tiles; warp 1 issues the MMAs and owns the TMEM; warps
+// 2-9 are the score warps (two per TMEM lane quadrant, queries 0-7 / 8-15).
+// Work items are (batch element, 16-query block, piece of <= 32 key tiles),
+// pieces the slowest index.  Every wait is bounded; on a timeout the kernel
+// records ERR_TIMEOUT, stops issuing work, lets its own copies and MMAs
+// finish (bounded) and frees its TMEM.
 #pragma once
 
 #include "attn_tc.cuh"
