@@ -46,3 +46,39 @@ def test_stalled_wait_reports_timeout_then_recovers(cuda_ok):
     assert len(keep) >= 333 - 3
     assert_out_close(out.reshape(-1, 32, 128)[keep], ref["out"][keep], "nsa out after timeout")
     assert_lse_close(lse3.reshape(-1, 32, 3)[keep], ref["lse_branch"][keep], "nsa lse after timeout")
+
+
+def test_stalled_exact_indexer_reports_timeout_then_recovers(cuda_ok):
+    """The exact indexer's tensor-core kernels (the full layer and the score
+    pass) under the stall hook: nothing is loaded or multiplied, their waits
+    run out and the call reports SA_ERR_TIMEOUT.  The workspace and the LSE
+    are zero-filled first, so the select that follows reads valid (zero)
+    scores.  The next call matches the oracle."""
+    import torch
+    from test_gpu_full_indexer import _check_out, _check_sets
+    B, T, Hq, Hkv, d, topk, window = 1, 300, 16, 1, 128, 64, 16
+    g = inputs.gen_dsa(B, T, Hq, Hkv, d, 1, 32, seed=T + d)
+    q, k, v = (g[n].cuda() for n in ("q", "k", "v"))
+    lib = _lib.load()
+    ws = torch.zeros(lib.sa_full_attn_topk_workspace_size(B, T, Hq, Hkv, d, topk, window),
+                     dtype=torch.uint8, device="cuda")
+    out = torch.zeros((B, T, Hq, d), dtype=torch.bfloat16, device="cuda")
+    lse = torch.zeros((B, T, Hq), dtype=torch.float32, device="cuda")
+    idx = torch.empty((B, T, topk + window), dtype=torch.int32, device="cuda")
+    api.check_device_status()
+    try:
+        api.debug_set_spin_limit(20_000_000)
+        api.debug_inject_stall(True)
+        api.full_attn_topk(q, k, v, topk, window, out=out, lse=lse, out_idx=idx, workspace=ws)
+        with pytest.raises(SAError) as ei:
+            api.check_device_status()
+        assert ei.value.status == _lib.SA_ERR_TIMEOUT, str(ei.value)
+    finally:
+        api.debug_inject_stall(False)
+        api.debug_set_spin_limit(0)
+    out, lse, idx = api.full_attn_topk(q, k, v, topk, window)
+    api.check_device_status()
+    ref_out, ref_lse, ref_idx, sc = oracle.full_attn_topk(g["q"], g["k"], g["v"], topk, window,
+                                                          want_scores=True)
+    _check_out(out, lse, ref_out, ref_lse)
+    _check_sets(idx, ref_idx, sc, topk, window, T, None)
